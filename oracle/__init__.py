@@ -1,0 +1,292 @@
+"""Plain fp64 CPU oracle for the CSA / HCA hot path -- TEST INFRASTRUCTURE.
+
+Only the tests, the smoke check in ``__graft_entry__`` and the CPU-baseline
+leg of ``bench.py`` may import this package.  The product path (the CUDA
+library and its Python binding) never imports, links or executes anything
+here, and this package imports nothing from the product.
+
+The arithmetic lives in ``csa_oracle.c`` (plain C, fp64, OpenMP over query
+rows); this module only compiles it with gcc and marshals numpy arrays.
+Every function states which passage of the pages it follows:
+
+* [P1] "DeepSeek V4 CSA + CP 迁移到 HP：困难点深度分析" (gitcode issue)
+* [P3] "DS-V4 分析&学习"
+* [P5] "百万上下文从「奢侈品」变「日用品」：DeepSeek V4 CSA/HCA 混合注意力架构深度解析"
+
+Parity of the indexer's head combination (sum over heads of ReLU(q_h . k))
+against the method as DeepSeek runs it is unpinned: the pages print no
+formula for it; the oracle pins it only to its own stated reading.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "csa_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``csa_oracle.c`` into ``liboracle.so`` (gcc, -O2, OpenMP, no fast-math)."""
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", "-fno-fast-math",
+           "-ffp-contract=off", _SRC, "-o", tmp, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.c_void_p
+        i32, i64 = ctypes.c_int, ctypes.c_long
+        lib.oracle_num_threads.restype = i32
+        lib.oracle_e4m3_decode.argtypes = [ctypes.c_uint8]
+        lib.oracle_e4m3_decode.restype = ctypes.c_double
+        lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
+        lib.oracle_e4m3_encode.restype = ctypes.c_uint8
+        lib.oracle_quantize_rows_e4m3.argtypes = [P, i64, i32, P, P]
+        lib.oracle_num_entries.argtypes = [i64, i64]
+        lib.oracle_num_entries.restype = i64
+        lib.oracle_visible_entries.argtypes = [i64, i32, i64]
+        lib.oracle_visible_entries.restype = i64
+        lib.oracle_compress.argtypes = [P, i32, i32, i32, P, i32, i32, i32, P]
+        lib.oracle_indexer_scores.argtypes = [P, P, i32, i32, i32, i32, i32, P, P, i32, P, i64, P]
+        lib.oracle_indexer_topk.argtypes = [P, P, i32, i32, i32, i32, i32, P, P, i32, i32, P, i64,
+                                            P, P, P]
+        lib.oracle_sparse_attn.argtypes = [P, i32, i32, i32, i32, P, i32, P, i32, P, i32, P, P,
+                                           i32, P, ctypes.c_double, P, i64, P, P]
+        lib.oracle_hca_attn.argtypes = [P, i32, i32, i32, i32, P, i32, P, i32, P, i32, P, P, i32,
+                                        P, ctypes.c_double, P, i64, P, P]
+        _lib = lib
+        return lib
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _i32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.int32))
+
+
+def _ptr(a: np.ndarray):
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle uses (``OMP_NUM_THREADS`` or all host cores)."""
+    return int(_load().oracle_num_threads())
+
+
+# --------------------------------------------------------------------------
+# FP8 E4M3 (OCP 8-bit floating point specification, E4M3 encoding)
+# --------------------------------------------------------------------------
+def e4m3_decode(codes) -> np.ndarray:
+    """Value of each E4M3 code (uint8), as fp64 (NaN for the NaN codes)."""
+    lib = _load()
+    c = np.asarray(codes, dtype=np.uint8)
+    return np.array([lib.oracle_e4m3_decode(int(v)) for v in c.ravel()]).reshape(c.shape)
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """Round fp32 values to E4M3 codes: nearest, ties to even, saturate at 448."""
+    lib = _load()
+    a = np.asarray(x, dtype=np.float32)
+    return np.array([lib.oracle_e4m3_encode(float(v)) for v in a.ravel()],
+                    dtype=np.uint8).reshape(a.shape)
+
+
+def quantize_rows_e4m3(x) -> tuple[np.ndarray, np.ndarray]:
+    """Per-row E4M3 quantisation in fp32: scale = amax/448 (1 for a zero row),
+    code = E4M3(x / scale).  Returns (codes uint8 [..., d], scales fp32 [...])."""
+    a = np.ascontiguousarray(np.asarray(x, dtype=np.float32))
+    d = a.shape[-1]
+    rows = a.size // d if d else 0
+    codes = np.empty(a.shape, dtype=np.uint8)
+    scales = np.empty(a.shape[:-1], dtype=np.float32)
+    _load().oracle_quantize_rows_e4m3(_ptr(a), rows, d, _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def dequantize_rows_e4m3(codes, scales) -> np.ndarray:
+    """codes * scale per row, exactly, in fp64."""
+    table = e4m3_decode(np.arange(256, dtype=np.uint8))
+    return table[np.asarray(codes, dtype=np.uint8)] * np.asarray(scales, np.float64)[..., None]
+
+
+# --------------------------------------------------------------------------
+# Stage 1: compression ([P5] §3.2; [P3] §1.3; [P1] §3.2)
+# --------------------------------------------------------------------------
+def num_entries(n: int, m: int) -> int:
+    """floor(n/m): a trailing partial block yields no entry ([P5] §3.2)."""
+    return int(_load().oracle_num_entries(n, m))
+
+
+def visible_entries(t: int, m: int, n_entries: int) -> int:
+    """Entries visible to the query at position t: min(floor((t+1)/m), n_entries)."""
+    return int(_load().oracle_visible_entries(t, m, n_entries))
+
+
+def compress(x, W, m: int, overlap: bool) -> np.ndarray:
+    """out[b,i] = mean(x[b, win(i)]) @ W for i < floor(n/m) (fp64).
+    x: [B, n, d_in]; W: [d_in, d_out]."""
+    x = _f64(x)
+    W = _f64(W)
+    B, n, d_in = x.shape
+    d_out = W.shape[1]
+    assert W.shape[0] == d_in
+    N_c = num_entries(n, m)
+    out = np.zeros((B, N_c, d_out), dtype=np.float64)
+    if N_c:
+        _load().oracle_compress(_ptr(x), B, n, d_in, _ptr(W), d_out, m, int(bool(overlap)),
+                                _ptr(out))
+    return out
+
+
+# --------------------------------------------------------------------------
+# Stage 2: indexer scores and top-k ([P5] §3.2; [P3] §1.2, §4)
+# --------------------------------------------------------------------------
+def _rows_arg(rows, total):
+    if rows is None:
+        return np.arange(total, dtype=np.int64)
+    return np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+
+
+def _defaults(B, n_q, N_cap, n_entries, q_pos):
+    if n_entries is None:
+        n_entries = np.full(B, N_cap, dtype=np.int32)
+    if q_pos is None:
+        q_pos = np.broadcast_to(np.arange(n_q, dtype=np.int32), (B, n_q))
+    return _i32(n_entries), _i32(q_pos)
+
+
+def indexer_scores(qI, kI, m: int, n_entries=None, q_pos=None, rows=None) -> np.ndarray:
+    """Scores sum_h ReLU(qI[t,h].kI[s]) of the listed query rows (flattened
+    b*n_q+q; all rows by default) against every entry; NaN where invisible.
+    qI: [B, n_q, H_I, d_I]; kI: [B, N_cap, d_I] (dequantised values)."""
+    qI = _f64(qI)
+    kI = _f64(kI)
+    B, n_q, H_I, d_I = qI.shape
+    N_cap = kI.shape[1]
+    n_entries, q_pos = _defaults(B, n_q, N_cap, n_entries, q_pos)
+    rows = _rows_arg(rows, B * n_q)
+    out = np.empty((rows.size, N_cap), dtype=np.float64)
+    _load().oracle_indexer_scores(_ptr(qI), _ptr(kI), B, n_q, H_I, d_I, N_cap, _ptr(n_entries),
+                                  _ptr(q_pos), m, _ptr(rows), rows.size, _ptr(out))
+    return out
+
+
+def indexer_topk(qI, kI, m: int, topk: int, n_entries=None, q_pos=None, rows=None):
+    """Per query row: the topk largest visible scores (ties -> lower index,
+    -1 padding).  Returns (idx [n_rows, topk] int32 in (score desc, index
+    asc) order, kth [n_rows, 2] = k-th and (k+1)-th largest scores (NaN if
+    absent), smax [n_rows] = largest |score|)."""
+    qI = _f64(qI)
+    kI = _f64(kI)
+    B, n_q, H_I, d_I = qI.shape
+    N_cap = kI.shape[1]
+    n_entries, q_pos = _defaults(B, n_q, N_cap, n_entries, q_pos)
+    rows = _rows_arg(rows, B * n_q)
+    idx = np.empty((rows.size, topk), dtype=np.int32)
+    kth = np.empty((rows.size, 2), dtype=np.float64)
+    smax = np.empty(rows.size, dtype=np.float64)
+    _load().oracle_indexer_topk(_ptr(qI), _ptr(kI), B, n_q, H_I, d_I, N_cap, _ptr(n_entries),
+                                _ptr(q_pos), m, topk, _ptr(rows), rows.size, _ptr(idx),
+                                _ptr(kth), _ptr(smax))
+    return idx, kth, smax
+
+
+# --------------------------------------------------------------------------
+# Stage 3: joint-softmax attention ([P3] §1.2, §1.4, §1.5; [P5] §4.3, §5.2)
+# --------------------------------------------------------------------------
+def _raw_defaults(B, L_raw, raw_pos0, raw_len):
+    if raw_pos0 is None:
+        raw_pos0 = np.zeros(B, dtype=np.int32)
+    if raw_len is None:
+        raw_len = np.full(B, L_raw, dtype=np.int32)
+    return _i32(raw_pos0), _i32(raw_len)
+
+
+def sparse_attn(q, kv_c, idx, kv_raw, window: int, q_pos=None, raw_pos0=None, raw_len=None,
+                scale: float | None = None, rows=None):
+    """Joint softmax over {kv_c[idx[r, j]] : idx >= 0} ∪ window raw rows.
+    q: [B, n_q, H, D]; kv_c: [B, N_cap, D]; idx: [B, n_q, topk];
+    kv_raw: [B, L_raw, D].  Returns (o [n_rows, H, D], lse [n_rows, H])."""
+    q = _f64(q)
+    kv_c = _f64(kv_c)
+    kv_raw = _f64(kv_raw)
+    idx = _i32(idx)
+    B, n_q, H, D = q.shape
+    N_cap = kv_c.shape[1]
+    L_raw = kv_raw.shape[1]
+    topk = idx.shape[-1]
+    _, q_pos = _defaults(B, n_q, N_cap, None, q_pos)
+    raw_pos0, raw_len = _raw_defaults(B, L_raw, raw_pos0, raw_len)
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    rows = _rows_arg(rows, B * n_q)
+    out = np.empty((rows.size, H, D), dtype=np.float64)
+    lse = np.empty((rows.size, H), dtype=np.float64)
+    _load().oracle_sparse_attn(_ptr(q), B, n_q, H, D, _ptr(kv_c), N_cap, _ptr(idx), topk,
+                               _ptr(kv_raw), L_raw, _ptr(raw_pos0), _ptr(raw_len), window,
+                               _ptr(q_pos), float(scale), _ptr(rows), rows.size, _ptr(out),
+                               _ptr(lse))
+    return out, lse
+
+
+def hca_attn(q, kv_c, m: int, kv_raw, window: int, n_entries=None, q_pos=None, raw_pos0=None,
+             raw_len=None, scale: float | None = None, rows=None):
+    """Dense attention over every visible entry s < min(floor((t+1)/m),
+    n_entries) plus the window, under one softmax.  Shapes as sparse_attn."""
+    q = _f64(q)
+    kv_c = _f64(kv_c)
+    kv_raw = _f64(kv_raw)
+    B, n_q, H, D = q.shape
+    N_cap = kv_c.shape[1]
+    L_raw = kv_raw.shape[1]
+    n_entries, q_pos = _defaults(B, n_q, N_cap, n_entries, q_pos)
+    raw_pos0, raw_len = _raw_defaults(B, L_raw, raw_pos0, raw_len)
+    if scale is None:
+        scale = 1.0 / np.sqrt(D)
+    rows = _rows_arg(rows, B * n_q)
+    out = np.empty((rows.size, H, D), dtype=np.float64)
+    lse = np.empty((rows.size, H), dtype=np.float64)
+    _load().oracle_hca_attn(_ptr(q), B, n_q, H, D, _ptr(kv_c), N_cap, _ptr(n_entries), m,
+                            _ptr(kv_raw), L_raw, _ptr(raw_pos0), _ptr(raw_len), window,
+                            _ptr(q_pos), float(scale), _ptr(rows), rows.size, _ptr(out),
+                            _ptr(lse))
+    return out, lse
+
+
+# --------------------------------------------------------------------------
+# End to end: stage 1 -> 2 -> 3 (a composition of the functions above)
+# --------------------------------------------------------------------------
+def csa_forward(q, kv, qI, kI_raw, W_c, W_Ic, m: int, topk: int, window: int, rows=None):
+    """Whole CSA prefill for one batch of sequences (positions 0..n-1):
+    compress kv and the indexer keys with overlap, score + top-k, attend.
+    Returns (o [n_rows, H, D], lse, idx [n_rows, topk])."""
+    kv_c = compress(kv, W_c, m, True)
+    kI_c = compress(kI_raw, W_Ic, m, True)
+    B, n_q = np.asarray(q).shape[:2]
+    idx, _, _ = indexer_topk(qI, kI_c, m, topk, rows=rows)
+    full_idx = np.full((B, n_q, topk), -1, dtype=np.int32)
+    r = _rows_arg(rows, B * n_q)
+    full_idx.reshape(B * n_q, topk)[r] = idx
+    o, lse = sparse_attn(q, kv_c, full_idx, kv, window, rows=rows)
+    return o, lse, idx
