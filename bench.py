@@ -1,0 +1,493 @@
+#!/usr/bin/env python
+"""Benchmark of the CSA hot path on B200.
+
+Headline: CSA prefill queries/s at n = 65536 (batch 1, 64x128 heads MQA, m = 4
+overlapping, fp8 e4m3 indexer 4x64 with per-row scales, top-512, window 512,
+1% 4x-norm outlier keys).  One step = the whole path over one batch:
+compress(kv) -> compress(indexer keys, fp8) -> indexer + top-k -> sparse
+attention.  Also reported: CSA decode tok/s at 128K context (batch 64,
+32768-entry compressed cache, 512-row SWA cache, top-512; one step =
+indexer + top-k -> sparse attention).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torch.distributed.run) every rank runs its own
+batch with no collective on the data path (weak scaling); the time is the
+max over ranks.  Rank 0 prints one JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from long_context_compressed_03_b200 import api, synth  # noqa: E402
+
+PREFILL = "csa_prefill_n64k_fp8idx"
+DECODE = "csa_decode_b64_ctx128k"
+METRIC = "CSA prefill queries/s at n=64K & decode tok/s at 128K ctx; % HBM/TC roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
+# keyed by kernel family; valid only while the kernel source hashes the same.
+NCU_TRAFFIC = {}
+
+
+# ---------------------------------------------------------------------- helpers
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def src_hash(name: str) -> str:
+    p = os.path.join(ROOT, "long_context_compressed_03_b200", "csrc", name)
+    with open(p, "rb") as f:
+        return hashlib.sha1(f.read()).hexdigest()[:12]
+
+
+def visible(t, m, ne):
+    return np.minimum((t + 1) // m, ne)
+
+
+def prefill_work(w):
+    """Algorithmic flops / bytes per stage for one prefill step (see DESIGN)."""
+    B, n, H, D, m, k, W = w.B, w.n, w.H, w.D, w.m, w.topk, w.window
+    HI, dI = w.H_I, w.d_I
+    N_c = n // m
+    t = np.arange(n, dtype=np.int64)
+    V = visible(t, m, N_c)
+    e = 2  # bf16
+    comp_kv_bytes = B * n * D * e + B * N_c * D * e + D * D * e
+    comp_kI_bytes = B * n * dI * e + B * N_c * (dI * 1 + 4) + dI * dI * e
+    sel = V > k
+    idx_flops = 2.0 * B * HI * dI * float(V[sel].sum())
+    idx_bytes = B * n * HI * dI * e + B * N_c * (dI + 4) + B * n * k * 4
+    keys = np.minimum(k, V) + np.minimum(W, t + 1)
+    attn_flops = 4.0 * B * H * D * float(keys.sum())
+    attn_bytes = 2 * B * n * H * D * e + B * N_c * D * e + B * n * D * e + B * n * k * 4
+    return {
+        "compress_kv": dict(bytes=comp_kv_bytes, flops=2.0 * B * N_c * D * D),
+        "compress_kI": dict(bytes=comp_kI_bytes, flops=2.0 * B * N_c * dI * dI),
+        "indexer_topk": dict(bytes=idx_bytes, flops=idx_flops),
+        "sparse_attn": dict(bytes=attn_bytes, flops=attn_flops),
+    }
+
+
+def decode_work(w, inp):
+    B, H, D, k, W, HI, dI = w.B, w.H, w.D, w.topk, w.window, w.H_I, w.d_I
+    ne = inp["n_entries"].numpy().astype(np.int64)
+    idx_bytes = int((ne * (dI + 4)).sum()) + B * HI * dI * 2 + B * k * 4
+    idx_flops = 2.0 * HI * dI * float(ne.sum())
+    keys = np.minimum(k, ne) + W
+    attn_bytes = int(B * k * D * 2 + B * W * D * 2 + 2 * B * H * D * 2 + B * k * 4)
+    attn_flops = 4.0 * H * D * float(keys.sum())
+    return {"indexer_topk": dict(bytes=idx_bytes, flops=idx_flops),
+            "sparse_attn": dict(bytes=attn_bytes, flops=attn_flops)}
+
+
+class ClockSampler:
+    """Samples SM clock / power / throttle reasons with nvidia-smi while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, local_rank: int):
+        cvd = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        ids = [s.strip() for s in cvd.split(",") if s.strip()]
+        self.gpu = ids[local_rank] if local_rank < len(ids) else str(local_rank)
+        self.proc = None
+        self.lines = []
+        self.error = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", self.gpu], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+            time.sleep(0.3)
+        except Exception as e:  # no nvidia-smi
+            self.error = str(e)
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.25)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        if self.error or not self.lines:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [],
+                    "note": self.error or "no samples"}
+        sm, smax, power, reasons = [], None, [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "note": "unparsed"}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": smax, "reasons": sorted(reasons),
+                "samples": len(sm), "power_w_max": max(power) if power else None}
+
+
+# ---------------------------------------------------------------------- our arm
+class PrefillPath:
+    """Device buffers + the four ABI calls of one prefill step."""
+
+    def __init__(self, w, inp, dev):
+        self.w = w
+        self.d = {k: v.to(dev) for k, v in inp.items()}
+        B, n = w.B, w.n
+        N_c = n // w.m
+        self.kv_c = torch.empty(B, N_c, w.D, dtype=torch.bfloat16, device=dev)
+        self.kI_c = torch.empty(B, N_c, w.d_I, dtype=torch.uint8, device=dev)
+        self.kI_s = torch.empty(B, N_c, dtype=torch.float32, device=dev)
+        self.idx = torch.empty(B, n, w.topk, dtype=torch.int32, device=dev)
+        self.out = torch.empty_like(self.d["q"])
+        self.names = ["compress_kv", "compress_kI", "indexer_topk", "sparse_attn"]
+        self.ev = None
+
+    def step(self, record=False):
+        d, w = self.d, self.w
+        calls = [
+            lambda: api.csa_compress(d["kv"], d["W_c"], w.m, True, self.kv_c),
+            lambda: api.csa_compress(d["kI_raw"], d["W_Ic"], w.m, True, self.kI_c, self.kI_s),
+            lambda: api.csa_indexer_topk(d["qI"], self.kI_c, w.m, w.topk, self.idx,
+                                         kI_scale=self.kI_s),
+            lambda: api.csa_sparse_attn(d["q"], self.kv_c, self.idx, d["kv"], w.window,
+                                        self.out),
+        ]
+        if not record:
+            for c in calls:
+                c()
+            return None
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+        evs[0].record()
+        for i, c in enumerate(calls):
+            c()
+            evs[i + 1].record()
+        return evs
+
+
+def run_prefill(w, dev, steps, warmup, dist_ctx, rank):
+    inp = synth.csa_prefill_inputs(w, seed=rank)
+    path = PrefillPath(w, inp, dev)
+    for _ in range(warmup):
+        path.step()
+    torch.cuda.synchronize()
+    launches0 = api.csa_kernel_launches()
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", 0)))
+    per_step = []
+    with clocks:
+        dist_ctx.barrier()
+        torch.cuda.synchronize()
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        start.record()
+        for _ in range(steps):
+            per_step.append(path.step(record=True))
+        end.record()
+        torch.cuda.synchronize()
+        dist_ctx.barrier()
+    launches = api.csa_kernel_launches() - launches0
+    total_ms = start.elapsed_time(end)
+    kern_ms = {nm: 0.0 for nm in path.names}
+    for evs in per_step:
+        for i, nm in enumerate(path.names):
+            kern_ms[nm] += evs[i].elapsed_time(evs[i + 1])
+    kern_ms = {k: v / steps for k, v in kern_ms.items()}
+    return dict(total_ms=total_ms, kern_ms=kern_ms, launches=launches, clocks=clocks.summary(),
+                path=path, inp=inp)
+
+
+def run_e2e(w, inp, dev, steps):
+    """Same step through the public API with pinned host inputs: h2d copies of
+    the step's inputs and a d2h read of its result are inside the timed region."""
+    host = {k: v.pin_memory() for k, v in inp.items()}
+    path = PrefillPath(w, inp, dev)
+    out_host = torch.empty(path.out.shape, dtype=path.out.dtype).pin_memory()
+    idx_host = torch.empty(path.idx.shape, dtype=path.idx.dtype).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = out_host.numel() * out_host.element_size() + idx_host.numel() * idx_host.element_size()
+
+    def one():
+        for k, v in host.items():
+            path.d[k].copy_(v, non_blocking=True)
+        path.step()
+        out_host.copy_(path.out, non_blocking=True)
+        idx_host.copy_(path.idx, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(steps):
+        one()
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / steps
+    return dict(ms=ms, h2d=h2d, d2h=d2h)
+
+
+def run_decode(dev, steps, warmup, rank):
+    w = synth.WORKLOADS[DECODE]
+    inp = synth.csa_decode_inputs(w, seed=rank)
+    d = {k: v.to(dev) for k, v in inp.items()}
+    idx = torch.empty(w.B, 1, w.topk, dtype=torch.int32, device=dev)
+    out = torch.empty_like(d["q"])
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)   # > L2 (126 MB)
+
+    def step(record):
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(3)] if record else None
+        if record:
+            evs[0].record()
+        api.csa_indexer_topk(d["qI"], d["kI_c"], w.m, w.topk, idx, kI_scale=d["kI_scale"],
+                             n_entries=d["n_entries"], q_pos=d["q_pos"])
+        if record:
+            evs[1].record()
+        api.csa_sparse_attn(d["q"], d["kv_c"], idx, d["swa"], w.window, out,
+                            raw_pos0=d["raw_pos0"], raw_len=d["raw_len"], q_pos=d["q_pos"])
+        if record:
+            evs[2].record()
+        return evs
+
+    for _ in range(warmup):
+        step(False)
+    torch.cuda.synchronize()
+    recs = []
+    for _ in range(steps):
+        flush.fill_(1)                     # evict the caches from L2 between steps
+        recs.append(step(True))
+    torch.cuda.synchronize()
+    t_idx = [r[0].elapsed_time(r[1]) for r in recs]
+    t_att = [r[1].elapsed_time(r[2]) for r in recs]
+    tot = [a + b for a, b in zip(t_idx, t_att)]
+    return dict(w=w, inp=inp, ms=float(np.mean(tot)), ms_median=float(np.median(tot)),
+                kern_ms={"indexer_topk": float(np.mean(t_idx)), "sparse_attn": float(np.mean(t_att))})
+
+
+# ---------------------------------------------------------------------- oracle arm
+def oracle_prefill_sample(w, inp, n_sample, seed=5):
+    """The fp64 oracle on a bounded sample of the prefill workload: both
+    compressors over the whole sequence, then indexer + top-k and attention
+    for n_sample sampled queries.  Returns (seconds per query, detail)."""
+    import oracle
+    f64 = lambda t: t.detach().to("cpu", torch.float64).numpy()
+    n = w.n
+    t0 = time.perf_counter()
+    kv_c = oracle.compress(f64(inp["kv"]), f64(inp["W_c"]), w.m, True)
+    kI_c = oracle.compress(f64(inp["kI_raw"]), f64(inp["W_Ic"]), w.m, True)
+    t_comp = time.perf_counter() - t0
+    codes, scales = oracle.quantize_rows_e4m3(kI_c.astype(np.float32))
+    rows = synth.query_sample(n, w.m, w.window, n_sample, seed=seed).numpy()[:n_sample]
+    rb = np.zeros(rows.size, np.int32)
+    rt = rows.astype(np.int32)
+    qrows = oracle.quantized_query_rows(inp["qI"][0, rows].float().numpy())
+    t1 = time.perf_counter()
+    idx, _, _ = oracle.indexer_topk_rows(qrows, rb, rt, codes, w.m, w.topk,
+                                         np.array([n // w.m], np.int32), scales)
+    oracle.sparse_attn_rows(f64(inp["q"][0, rows]), rb, rt, kv_c, idx, f64(inp["kv"]), w.window)
+    t_rows = time.perf_counter() - t1
+    per_query = t_comp / n + t_rows / rows.size
+    return per_query, dict(compress_s=t_comp, rows=int(rows.size), rows_s=t_rows)
+
+
+def cpu_baseline(w, inp, n_sample):
+    import oracle
+    per_q, det = oracle_prefill_sample(w, inp, n_sample)
+    return {"value": 1.0 / per_q, "unit": "queries/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": (f"fp64 oracle: both compressors over all {w.n} tokens "
+                       f"({det['compress_s']:.2f} s) + indexer/top-k and attention for "
+                       f"{det['rows']} of {w.n} queries ({det['rows_s']:.2f} s); "
+                       f"queries/s = 1 / (compress_s/n + rows_s/rows)")}
+
+
+# ---------------------------------------------------------------------- distributed
+class DistCtx:
+    def __init__(self, gpus):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.on = self.world > 1
+        if self.on:
+            import datetime
+            import torch.distributed as dist
+            torch.cuda.set_device(self.local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", self.local))
+            self.dist = dist
+
+    def barrier(self):
+        if self.on:
+            self.dist.barrier()
+
+    def max(self, v: float) -> float:
+        if not self.on:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        self.dist.all_reduce(t, op=self.dist.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.on:
+            self.dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--cpu-sample", type=int, default=4096,
+                    help="queries the oracle baseline scores (bounded CPU sample)")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    w = synth.WORKLOADS[PREFILL]
+    config = {"workload": PREFILL, "B": w.B, "n": w.n, "H": w.H, "D": w.D, "m": w.m,
+              "overlap": True, "topk": w.topk, "window": w.window, "indexer": "e4m3 per-row scale",
+              "H_I": w.H_I, "d_I": w.d_I, "outliers": "1% tokens x4", "seed": "rank",
+              "l2": "inputs larger than L2 (q alone is 1 GiB); decode flushes L2 between steps",
+              "parallelism": f"replicas x{args.gpus}"}
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        if rank != 0:
+            return 0
+        import oracle
+        inp = synth.csa_prefill_inputs(w, seed=0)
+        sample = max(16, args.cpu_sample // 4)
+        times = []
+        for _ in range(args.warmup):
+            oracle_prefill_sample(w, inp, 16)
+        for i in range(args.steps):
+            per_q, det = oracle_prefill_sample(w, inp, sample, seed=10 + i)
+            times.append(per_q)
+        per_q = float(np.mean(times))
+        v = 1.0 / per_q
+        line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "queries/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": per_q * w.n * 1e3, "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1))",
+                "config": config,
+                "cpu_baseline": {"value": v, "unit": "queries/s", "cores": oracle.num_threads(),
+                                 "kind": "oracle",
+                                 "sample": f"{sample} sampled queries per step + full compress, "
+                                           f"extrapolated to n={w.n}"},
+                "e2e": {"value": v, "unit": "queries/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return 0
+
+    dist_ctx = DistCtx(args.gpus)
+    rank = dist_ctx.rank
+    dev = torch.device("cuda", dist_ctx.local)
+    torch.cuda.set_device(dev)
+    api.load()
+    peaks, peak_src = load_peaks()
+
+    pre = run_prefill(w, dev, args.steps, args.warmup, dist_ctx, rank)
+    t_max = dist_ctx.max(pre["total_ms"])
+    ms_step = t_max / args.steps
+    queries = w.B * w.n * dist_ctx.world
+    value = queries / (ms_step / 1e3)
+
+    work = prefill_work(w)
+    dom = max(pre["kern_ms"], key=pre["kern_ms"].get)
+    dom_work = work[dom]
+    tensor_kernels = {"sparse_attn", "indexer_topk"}
+    if dom in tensor_kernels:
+        achieved = dom_work["flops"] / (pre["kern_ms"][dom] / 1e3) / 1e12
+        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak}
+    else:
+        achieved = dom_work["bytes"] / (pre["kern_ms"][dom] / 1e3) / 1e9
+        peak = peaks["hbm_gbs"]
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak}
+    tr = NCU_TRAFFIC.get(dom)
+    roof["traffic"] = tr["bytes"] if tr and tr["src"] == src_hash(tr["file"]) else None
+    roof["kernel"] = dom
+    roof["peak_source"] = f"{peak_src} ({'sustained bf16' if roof['unit'] == 'TFLOP/s' else 'hbm copy'})"
+    stages = {}
+    for nm, ms in pre["kern_ms"].items():
+        wk = work[nm]
+        stages[nm] = {"ms": ms, "share": ms / max(1e-9, sum(pre["kern_ms"].values())),
+                      "TFLOP/s": wk["flops"] / (ms / 1e3) / 1e12,
+                      "GB/s": wk["bytes"] / (ms / 1e3) / 1e9}
+
+    line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": dist_ctx.world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded N(0,1), 1% 4x outlier keys)", "config": config,
+            "roofline": roof, "stages": stages, "gpu_launches": pre["launches"],
+            "clocks": pre["clocks"]}
+
+    if not args.no_decode:
+        dec = run_decode(dev, args.steps, args.warmup, rank)
+        dms = dist_ctx.max(dec["ms"])
+        dw = decode_work(dec["w"], dec["inp"])
+        dstages = {nm: {"ms": ms, "GB/s": dw[nm]["bytes"] / (ms / 1e3) / 1e9,
+                        "frac_hbm": dw[nm]["bytes"] / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+                   for nm, ms in dec["kern_ms"].items()}
+        line["decode"] = {"workload": DECODE, "value": dec["w"].B * dist_ctx.world / (dms / 1e3),
+                          "unit": "tok/s", "ms_per_step": dms, "ms_median": dec["ms_median"],
+                          "l2": "flushed (512 MiB write) between steps", "stages": dstages}
+    if not args.no_e2e:
+        e2e = run_e2e(w, pre["inp"], dev, max(3, args.steps // 2))
+        ems = dist_ctx.max(e2e["ms"])
+        line["e2e"] = {"value": queries / (ems / 1e3), "unit": "queries/s",
+                       "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                       "ms_per_step": ems}
+    if rank == 0 and dist_ctx.world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, pre["inp"], args.cpu_sample)
+    if rank == 0:
+        print(json.dumps(line))
+    dist_ctx.close()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,181 @@
+/*
+ * csa_b200.h -- C ABI of the B200 (sm_100a) Compressed Sparse Attention
+ * (CSA) / Heavily Compressed Attention (HCA) library, libcsa_b200.so.
+ *
+ * The method, from the pages this library follows:
+ *   "DS-V4 分析&学习" §1.2: CSA compresses every m tokens into one KV entry,
+ *     a Lightning Indexer scores the entries, each query keeps its top-k and
+ *     attends to those k compressed entries plus a sliding window of raw KV;
+ *     §1.3: an entry sees 2m adjacent positions (neighbouring blocks
+ *     overlap); §1.4: HCA compresses 128:1 and attends densely; §4: the
+ *     indexer QK path runs in low precision.
+ *   "百万上下文从「奢侈品」变「日用品」…" §3.2: compression is a mean pool over
+ *     the block followed by a projection, floor(n/m) entries, the indexer is
+ *     a dot product followed by a per-query top-k; §5.2: the window of query
+ *     i is [max(0, i-W+1), i] and scores are scaled by 1/sqrt(head_dim).
+ *   "DeepSeek V4 CSA + CP 迁移到 HP：困难点深度分析" §3.2: ratio 4 compresses
+ *     with overlap, ratio 128 without; §7.2: the indexer has a compressor of
+ *     its own, sharing the main compressor's entry index space.
+ *
+ * Conventions shared by every entry point
+ *   - Tensor arguments are DEVICE pointers to caller-owned memory; the
+ *     library never allocates, frees or keeps them.  Layouts are batch-first,
+ *     contiguous, last dimension innermost.  Every tensor base pointer must
+ *     be 16-byte aligned (else CSA_ERR_MISALIGNED).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
+ *     default stream).  Arguments are validated on the host first; on any
+ *     error nothing is launched.  A launch failure returns CSA_ERR_CUDA.
+ *     No call aborts, exits or throws; the text of the last error of the
+ *     calling thread is returned by csa_last_error_detail().
+ *   - Device index arrays that the host cannot read (n_entries, q_pos,
+ *     raw_pos0, raw_len, idx) are clamped by the kernels to the buffers'
+ *     extents, so a bad value never reads out of bounds.
+ *   - Results are deterministic: the same inputs give bit-identical outputs.
+ *   - Positions: a query row carries the absolute position t of its token
+ *     (q_pos; NULL means t = the row's index q, i.e. a prefill from 0).
+ *     Compressed entry i covers positions up to m(i+1)-1 and is visible to t
+ *     iff i < min(floor((t+1)/m), n_entries[b]).  Raw row j of batch element
+ *     b holds position raw_pos0[b]+j for 0 <= j < raw_len[b]; positions < 0
+ *     are never attended (a partly filled sliding-window cache).
+ */
+#ifndef CSA_B200_H
+#define CSA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    CSA_OK = 0,
+    CSA_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad combination */
+    CSA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (dtype, head count, size) */
+    CSA_ERR_MISALIGNED = 3,   /* a tensor base pointer is not 16-byte aligned */
+    CSA_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
+    CSA_ERR_TIMEOUT = 5       /* reserved: a bounded device-side wait expired */
+} csa_status_t;
+
+typedef enum {
+    CSA_DT_F32 = 0,   /* IEEE binary32 */
+    CSA_DT_BF16 = 1,  /* bfloat16 */
+    CSA_DT_E4M3 = 2   /* OCP FP8 E4M3 with one fp32 scale per row */
+} csa_dtype_t;
+
+/* Static text of a status code ("CSA_OK", ...). */
+const char* csa_status_string(int status);
+
+/* Thread-local detail of the last non-OK return on the calling thread ("" if none). */
+const char* csa_last_error_detail(void);
+
+/* ABI version: 100 * major + minor. */
+int csa_version(void);
+
+/* Number of kernels this library has launched in the process so far
+ * (diagnostics: lets a caller count the device work behind its calls). */
+unsigned long long csa_kernel_launches(void);
+
+/*
+ * csa_compress -- stage 1: overlapping (or plain) mean-pool compression
+ * followed by a projection, optionally quantised to fp8.
+ * Follows "百万上下文从「奢侈品」变「日用品」…" §3.2 (C[i] = W . mean of the
+ * block's rows, floor(n/m) entries) and "DS-V4 分析&学习" §1.3 (2m-position
+ * overlapping windows); ratio 128 without overlap per "DeepSeek V4 CSA + CP
+ * 迁移到 HP…" §3.2.
+ *
+ *   out[b, i, :] = (mean_{p in win(i)} x[b, p, :]) @ W,   0 <= i < floor(n/m)
+ *     overlap = 1: win(i) = [m(i-1), m(i+1)) ∩ [0, n)  (own block + previous)
+ *     overlap = 0: win(i) = [m i, m(i+1))
+ *
+ *   x     [B, n, d_in]     x_dt = CSA_DT_F32 or CSA_DT_BF16
+ *   W     [d_in, d_out]    same dtype as x, applied as row-vector @ W
+ *   out   [B, floor(n/m), d_out]  out_dt:
+ *           CSA_DT_F32  (x_dt F32 only), CSA_DT_BF16 (round to nearest even),
+ *           CSA_DT_E4M3 (uint8 codes; out_row_scale [B, floor(n/m)] fp32 gets
+ *           amax/448 of the row, 1 for a zero row; code = E4M3(v/scale),
+ *           nearest-even, saturating)
+ *   out_row_scale  required iff out_dt == CSA_DT_E4M3, else must be NULL.
+ *   Limits: 16 <= d_in, d_out <= 256 and multiples of 16; m >= 1.
+ *   Pooling and the projection accumulate in fp32.
+ */
+csa_status_t csa_compress(const void* x, int x_dt, int B, int n, int d_in, const void* W,
+                          int d_out, int m, int overlap, void* out, int out_dt,
+                          float* out_row_scale, void* stream);
+
+/*
+ * csa_indexer_topk -- stage 2: Lightning-Indexer score + causal per-query
+ * top-k, fused: the score matrix never reaches global memory.
+ * Follows "百万上下文从「奢侈品」变「日用品」…" §3.2 (query . compressed-key
+ * score, torch.topk per query) and §8.2 (scores must not be materialised),
+ * "DS-V4 分析&学习" §1.2 and §4 (low-precision indexer QK).
+ *
+ *   score[t, s] = sum_h ReLU(qI[t, h, :] . kI[s, :])  for visible s
+ *   idx_out[b, q, :] = the topk entries of largest score; equal scores are
+ *     taken lowest index first; with V < topk visible entries the row holds
+ *     those V entries followed by -1.  The order inside a row is not part of
+ *     the contract (it is deterministic).
+ *
+ *   qI [B, n_q, H_I, d_I]: qI_dt F32, BF16, or E4M3 with qI_scale [B, n_q, H_I].
+ *      With kI_dt == CSA_DT_E4M3 and qI_dt == CSA_DT_BF16 (qI_scale NULL), each
+ *      (query, head) row is quantised in the kernel exactly as csa_compress
+ *      quantises a row (fp32: scale = amax/448, code = E4M3(x/scale)).
+ *   kI [B, N_cap, d_I]: kI_dt F32, BF16, or E4M3 with kI_scale [B, N_cap].
+ *      Supported pairs: (F32,F32), (BF16,BF16), (BF16,E4M3), (E4M3,E4M3).
+ *      With fp8 the score is sk_s * sum_h sq_h * ReLU(q8_h . k8_s).
+ *   n_entries [B] valid entries per element (NULL: N_cap); q_pos [B, n_q] (NULL: q).
+ *   m: compression ratio (visibility rule above).  1 <= topk <= 2048.
+ *   Limits: 1 <= H_I <= 16, d_I multiple of 16 and <= 256, N_cap <= 40960.
+ *   idx_out [B, n_q, topk] int32.
+ */
+csa_status_t csa_indexer_topk(const void* qI, int qI_dt, const float* qI_scale, const void* kI,
+                              int kI_dt, const float* kI_scale, int B, int n_q, int H_I, int d_I,
+                              int N_cap, const int* n_entries, const int* q_pos, int m, int topk,
+                              int* idx_out, void* stream);
+
+/*
+ * csa_sparse_attn -- stage 3: joint-softmax MQA over the selected compressed
+ * entries plus the sliding window of raw KV (shared KV: one vector is both
+ * key and value, one KV head for all query heads).
+ * Follows "DS-V4 分析&学习" §1.2, §1.5 and "百万上下文从「奢侈品」变「日用品」…"
+ * §5.2 (window [max(0,t-W+1), t], scale 1/sqrt(D)).
+ *
+ *   For query row (b, q) at position t and head h:
+ *     keys = { kv_c[b, s] : s = idx[b, q, j], 0 <= s < N_cap }      (compressed)
+ *          ∪ { kv_raw[b, j] : position raw_pos0[b]+j in [max(0,t-W+1), t] } (window)
+ *     as a multiset (nothing de-duplicated), z = softmax_scale * q . key,
+ *     out = sum softmax(z) key, lse_out = log(sum exp z) (natural log).
+ *     An empty key set gives out = 0 and lse = -inf.
+ *   q [B, n_q, H, D] and kv_c [B, N_cap, D], kv_raw [B, L_raw, D], out [B, n_q, H, D]
+ *     share dt (CSA_DT_F32 or CSA_DT_BF16); accumulation is fp32.
+ *   idx [B, n_q, topk] int32; negative entries are padding, entries >= N_cap
+ *     are ignored.  topk may be 0 (window only; idx may then be NULL).
+ *   raw_pos0 / raw_len [B] (NULL: 0 / L_raw); q_pos [B, n_q] (NULL: q).
+ *   softmax_scale <= 0 selects 1/sqrt(D).  lse_out [B, n_q, H] fp32 or NULL.
+ *   Limits: D multiple of 16, 16 <= D <= 256; H in {1,2,4,...,128}; window >= 0.
+ */
+csa_status_t csa_sparse_attn(const void* q, int dt, int B, int n_q, int H, int D,
+                             const void* kv_c, int N_cap, const int* idx, int topk,
+                             const void* kv_raw, int L_raw, const int* raw_pos0,
+                             const int* raw_len, int window, const int* q_pos,
+                             float softmax_scale, void* out, float* lse_out, void* stream);
+
+/*
+ * hca_dense_attn -- HCA: dense attention over every visible compressed entry
+ * (no top-k) plus the sliding window, under one softmax.
+ * Follows "DS-V4 分析&学习" §1.4 and "百万上下文从「奢侈品」变「日用品」…" §4.3.
+ *
+ *   keys = { kv_c[b, s] : s < min(floor((t+1)/m), n_entries[b], N_cap) } ∪ window,
+ *   otherwise exactly as csa_sparse_attn.  n_entries [B] (NULL: N_cap).
+ */
+csa_status_t hca_dense_attn(const void* q, int dt, int B, int n_q, int H, int D,
+                            const void* kv_c, int N_cap, const int* n_entries, int m,
+                            const void* kv_raw, int L_raw, const int* raw_pos0,
+                            const int* raw_len, int window, const int* q_pos,
+                            float softmax_scale, void* out, float* lse_out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* CSA_B200_H */

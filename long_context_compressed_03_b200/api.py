@@ -1,0 +1,233 @@
+"""Thin Python binding of libcsa_b200.so (see include/csa_b200.h).
+
+Argument marshalling only: each function of the C ABI has a Python function
+of the same name that takes torch CUDA tensors, derives sizes and dtype
+codes from them, passes raw device pointers and the current CUDA stream, and
+raises ``CsaError`` on a non-OK status.  Every step of the computation runs
+in the library's kernels; there is no fallback of any kind -- if the library
+is missing or fails to load, the first call raises.
+
+Convenience wrappers (``compress``, ``indexer_topk``, ``sparse_attn``,
+``hca_attn``, ``csa_prefill``) allocate their outputs with ``torch.empty``
+and call the ABI functions.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libcsa_b200.so")
+
+CSA_OK, CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_MISALIGNED, CSA_ERR_CUDA, \
+    CSA_ERR_TIMEOUT = range(6)
+DT_F32, DT_BF16, DT_E4M3 = 0, 1, 2
+
+# symbol -> (restype, argtypes); mirrors include/csa_b200.h
+P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+SIGNATURES = {
+    "csa_status_string": (ctypes.c_char_p, [I]),
+    "csa_last_error_detail": (ctypes.c_char_p, []),
+    "csa_version": (I, []),
+    "csa_kernel_launches": (ctypes.c_ulonglong, []),
+    "csa_compress": (I, [P, I, I, I, I, P, I, I, I, P, I, P, P]),
+    "csa_indexer_topk": (I, [P, I, P, P, I, P, I, I, I, I, I, P, P, I, I, P, P]),
+    "csa_sparse_attn": (I, [P, I, I, I, I, I, P, I, P, I, P, I, P, P, I, P, F, P, P, P]),
+    "hca_dense_attn": (I, [P, I, I, I, I, I, P, I, P, I, P, I, P, P, I, P, F, P, P, P]),
+}
+
+
+class CsaError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        super().__init__(f"{_status_name(status)}: {detail}")
+        self.status = status
+        self.detail = detail
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load(path: str | None = None) -> ctypes.CDLL:
+    """Load the library (once).  Raises if it is missing: there is no fallback."""
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        p = path or LIB_PATH
+        if not os.path.exists(p):
+            raise RuntimeError(f"libcsa_b200.so not found at {p}; build it with "
+                               "`python -m long_context_compressed_03_b200.build`")
+        lib = ctypes.CDLL(p)
+        for name, (res, args) in SIGNATURES.items():
+            fn = getattr(lib, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = lib
+        return lib
+
+
+def _status_name(status: int) -> str:
+    try:
+        return load().csa_status_string(status).decode()
+    except Exception:  # pragma: no cover - only when the library cannot load
+        return f"status {status}"
+
+
+def _check(status: int) -> None:
+    if status != CSA_OK:
+        raise CsaError(status, load().csa_last_error_detail().decode())
+
+
+def _ptr(t: torch.Tensor | None):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor arguments must be CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("tensor arguments must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return DT_F32
+    if t.dtype == torch.bfloat16:
+        return DT_BF16
+    if t.dtype in (torch.uint8, torch.float8_e4m3fn):
+        return DT_E4M3
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        stream = stream.cuda_stream
+    return ctypes.c_void_p(int(stream))
+
+
+def _i32(t: torch.Tensor | None, name: str):
+    if t is not None and t.dtype != torch.int32:
+        raise ValueError(f"{name} must be int32")
+    return _ptr(t)
+
+
+# ---------------------------------------------------------------- the ABI, by name
+def csa_version() -> int:
+    return int(load().csa_version())
+
+
+def csa_kernel_launches() -> int:
+    """Kernels the library has launched in this process so far."""
+    return int(load().csa_kernel_launches())
+
+
+def csa_compress(x: torch.Tensor, W: torch.Tensor, m: int, overlap: bool, out: torch.Tensor,
+                 out_row_scale: torch.Tensor | None = None, stream=None) -> None:
+    """x [B, n, d_in], W [d_in, d_out] -> out [B, n//m, d_out] (+ scales for fp8)."""
+    B, n, d_in = x.shape
+    d_out = W.shape[1]
+    _check(load().csa_compress(_ptr(x), _dt(x), B, n, d_in, _ptr(W), d_out, m, int(bool(overlap)),
+                               _ptr(out), _dt(out), _ptr(out_row_scale), _stream(stream)))
+
+
+def csa_indexer_topk(qI: torch.Tensor, kI: torch.Tensor, m: int, topk: int, idx_out: torch.Tensor,
+                     qI_scale: torch.Tensor | None = None, kI_scale: torch.Tensor | None = None,
+                     n_entries: torch.Tensor | None = None, q_pos: torch.Tensor | None = None,
+                     stream=None) -> None:
+    """qI [B, n_q, H_I, d_I], kI [B, N_cap, d_I] -> idx_out [B, n_q, topk] int32."""
+    B, n_q, H_I, d_I = qI.shape
+    N_cap = kI.shape[1]
+    _check(load().csa_indexer_topk(_ptr(qI), _dt(qI), _ptr(qI_scale), _ptr(kI), _dt(kI),
+                                   _ptr(kI_scale), B, n_q, H_I, d_I, N_cap,
+                                   _i32(n_entries, "n_entries"), _i32(q_pos, "q_pos"), m, topk,
+                                   _i32(idx_out, "idx_out"), _stream(stream)))
+
+
+def csa_sparse_attn(q: torch.Tensor, kv_c: torch.Tensor, idx: torch.Tensor | None,
+                    kv_raw: torch.Tensor, window: int, out: torch.Tensor,
+                    lse_out: torch.Tensor | None = None, raw_pos0: torch.Tensor | None = None,
+                    raw_len: torch.Tensor | None = None, q_pos: torch.Tensor | None = None,
+                    softmax_scale: float = 0.0, stream=None) -> None:
+    """q [B, n_q, H, D], kv_c [B, N_cap, D], idx [B, n_q, topk], kv_raw [B, L_raw, D]."""
+    B, n_q, H, D = q.shape
+    topk = 0 if idx is None else idx.shape[-1]
+    _check(load().csa_sparse_attn(_ptr(q), _dt(q), B, n_q, H, D, _ptr(kv_c), kv_c.shape[1],
+                                  _i32(idx, "idx"), topk, _ptr(kv_raw), kv_raw.shape[1],
+                                  _i32(raw_pos0, "raw_pos0"), _i32(raw_len, "raw_len"), window,
+                                  _i32(q_pos, "q_pos"), float(softmax_scale), _ptr(out),
+                                  _ptr(lse_out), _stream(stream)))
+
+
+def hca_dense_attn(q: torch.Tensor, kv_c: torch.Tensor, m: int, kv_raw: torch.Tensor, window: int,
+                   out: torch.Tensor, lse_out: torch.Tensor | None = None,
+                   n_entries: torch.Tensor | None = None, raw_pos0: torch.Tensor | None = None,
+                   raw_len: torch.Tensor | None = None, q_pos: torch.Tensor | None = None,
+                   softmax_scale: float = 0.0, stream=None) -> None:
+    """Dense attention over every visible entry of kv_c plus the window."""
+    B, n_q, H, D = q.shape
+    _check(load().hca_dense_attn(_ptr(q), _dt(q), B, n_q, H, D, _ptr(kv_c), kv_c.shape[1],
+                                 _i32(n_entries, "n_entries"), m, _ptr(kv_raw), kv_raw.shape[1],
+                                 _i32(raw_pos0, "raw_pos0"), _i32(raw_len, "raw_len"), window,
+                                 _i32(q_pos, "q_pos"), float(softmax_scale), _ptr(out),
+                                 _ptr(lse_out), _stream(stream)))
+
+
+# ---------------------------------------------------------------- allocating wrappers
+def compress(x: torch.Tensor, W: torch.Tensor, m: int, overlap: bool, out_dtype=None,
+             stream=None):
+    """Returns out (and the per-row scales when out_dtype is fp8: (codes, scales))."""
+    B, n, _ = x.shape
+    N_c = n // m
+    out_dtype = x.dtype if out_dtype is None else out_dtype
+    if out_dtype in (torch.uint8, torch.float8_e4m3fn):
+        out = torch.empty(B, N_c, W.shape[1], dtype=torch.uint8, device=x.device)
+        scale = torch.empty(B, N_c, dtype=torch.float32, device=x.device)
+        csa_compress(x, W, m, overlap, out, scale, stream=stream)
+        return out, scale
+    out = torch.empty(B, N_c, W.shape[1], dtype=out_dtype, device=x.device)
+    csa_compress(x, W, m, overlap, out, stream=stream)
+    return out
+
+
+def indexer_topk(qI, kI, m: int, topk: int, qI_scale=None, kI_scale=None, n_entries=None,
+                 q_pos=None, stream=None) -> torch.Tensor:
+    B, n_q = qI.shape[:2]
+    idx = torch.empty(B, n_q, topk, dtype=torch.int32, device=qI.device)
+    csa_indexer_topk(qI, kI, m, topk, idx, qI_scale=qI_scale, kI_scale=kI_scale,
+                     n_entries=n_entries, q_pos=q_pos, stream=stream)
+    return idx
+
+
+def sparse_attn(q, kv_c, idx, kv_raw, window: int, with_lse: bool = False, **kw):
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if with_lse else None
+    csa_sparse_attn(q, kv_c, idx, kv_raw, window, out, lse_out=lse, **kw)
+    return (out, lse) if with_lse else out
+
+
+def hca_attn(q, kv_c, m: int, kv_raw, window: int, with_lse: bool = False, **kw):
+    out = torch.empty_like(q)
+    lse = torch.empty(q.shape[:3], dtype=torch.float32, device=q.device) if with_lse else None
+    hca_dense_attn(q, kv_c, m, kv_raw, window, out, lse_out=lse, **kw)
+    return (out, lse) if with_lse else out
+
+
+def csa_prefill(q, kv, qI, kI_raw, W_c, W_Ic, m: int, topk: int, window: int,
+                indexer_fp8: bool, stream=None):
+    """The whole CSA prefill hot path (positions 0..n-1 of each sequence):
+    compress kv, compress the indexer keys (fp8 + row scales when
+    ``indexer_fp8``), indexer + top-k, joint sparse attention.
+    Returns dict(out, idx, kv_c, kI_c, kI_scale)."""
+    kv_c = compress(kv, W_c, m, True, stream=stream)
+    if indexer_fp8:
+        kI_c, kI_scale = compress(kI_raw, W_Ic, m, True, out_dtype=torch.uint8, stream=stream)
+    else:
+        kI_c, kI_scale = compress(kI_raw, W_Ic, m, True, stream=stream), None
+    idx = indexer_topk(qI, kI_c, m, topk, kI_scale=kI_scale, stream=stream)
+    out = sparse_attn(q, kv_c, idx, kv, window, stream=stream)
+    return dict(out=out, idx=idx, kv_c=kv_c, kI_c=kI_c, kI_scale=kI_scale)

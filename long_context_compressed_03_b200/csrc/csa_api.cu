@@ -1,0 +1,184 @@
+// csa_api.cu -- the extern "C" boundary of libcsa_b200.so (see csa_b200.h).
+//
+// Every entry point validates its arguments on the host, maps them onto the
+// internal launch structs and launches on the caller's stream.  Nothing is
+// allocated, nothing is synchronised, no exception or abort crosses the ABI.
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+
+#include "csa_b200.h"
+#include "kernels.h"
+
+namespace csa {
+static std::atomic<unsigned long long> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+}  // namespace csa
+
+namespace {
+
+thread_local char g_detail[512] = "";
+
+csa_status_t fail(csa_status_t st, const char* fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_detail, sizeof g_detail, fmt, ap);
+    va_end(ap);
+    return st;
+}
+
+csa_status_t ok() {
+    g_detail[0] = '\0';
+    return CSA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+csa_status_t from_cuda(cudaError_t e, const char* what, const char* why) {
+    if (e == cudaSuccess) return ok();
+    if (e == cudaErrorNotSupported && why) return fail(CSA_ERR_UNSUPPORTED, "%s", why);
+    return fail(CSA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+#define REQUIRE(cond, ...) \
+    do {                   \
+        if (!(cond)) return fail(CSA_ERR_INVALID_ARG, __VA_ARGS__); \
+    } while (0)
+#define REQUIRE_ALIGNED(p, name) \
+    do {                         \
+        if ((p) && !aligned16(p)) return fail(CSA_ERR_MISALIGNED, "%s is not 16-byte aligned", name); \
+    } while (0)
+
+bool is_dt(int d) { return d == CSA_DT_F32 || d == CSA_DT_BF16 || d == CSA_DT_E4M3; }
+
+}  // namespace
+
+extern "C" {
+
+const char* csa_status_string(int status) {
+    switch (status) {
+        case CSA_OK: return "CSA_OK";
+        case CSA_ERR_INVALID_ARG: return "CSA_ERR_INVALID_ARG";
+        case CSA_ERR_UNSUPPORTED: return "CSA_ERR_UNSUPPORTED";
+        case CSA_ERR_MISALIGNED: return "CSA_ERR_MISALIGNED";
+        case CSA_ERR_CUDA: return "CSA_ERR_CUDA";
+        case CSA_ERR_TIMEOUT: return "CSA_ERR_TIMEOUT";
+    }
+    return "CSA_ERR_UNKNOWN";
+}
+
+const char* csa_last_error_detail(void) { return g_detail; }
+
+int csa_version(void) { return 100; }
+
+unsigned long long csa_kernel_launches(void) { return csa::g_launches.load(); }
+
+csa_status_t csa_compress(const void* x, int x_dt, int B, int n, int d_in, const void* W,
+                          int d_out, int m, int overlap, void* out, int out_dt,
+                          float* out_row_scale, void* stream) {
+    REQUIRE(B >= 0 && n >= 0, "csa_compress: negative B or n");
+    REQUIRE(m >= 1, "csa_compress: m must be >= 1");
+    REQUIRE(overlap == 0 || overlap == 1, "csa_compress: overlap must be 0 or 1");
+    REQUIRE(is_dt(x_dt) && is_dt(out_dt), "csa_compress: unknown dtype");
+    REQUIRE(d_in > 0 && d_out > 0, "csa_compress: d_in and d_out must be positive");
+    if (d_in % 16 || d_out % 16 || d_in > 256 || d_out > 256)
+        return fail(CSA_ERR_UNSUPPORTED, "csa_compress: d_in, d_out must be multiples of 16 in [16, 256]");
+    if (x_dt == CSA_DT_E4M3) return fail(CSA_ERR_UNSUPPORTED, "csa_compress: fp8 input is not supported");
+    if (out_dt == CSA_DT_F32 && x_dt != CSA_DT_F32)
+        return fail(CSA_ERR_UNSUPPORTED, "csa_compress: F32 output needs F32 input");
+    REQUIRE((out_dt == CSA_DT_E4M3) == (out_row_scale != nullptr),
+            "csa_compress: out_row_scale is required for E4M3 output and must be NULL otherwise");
+    const int N_c = n / m;
+    if ((long)B * N_c == 0) return ok();
+    REQUIRE(x && W && out, "csa_compress: null tensor pointer");
+    REQUIRE_ALIGNED(x, "x");
+    REQUIRE_ALIGNED(W, "W");
+    REQUIRE_ALIGNED(out, "out");
+    REQUIRE_ALIGNED(out_row_scale, "out_row_scale");
+    csa::CompressArgs a{x, x_dt, B, n, d_in, W, d_out, m, overlap, out, out_dt, out_row_scale, N_c};
+    const char* why = nullptr;
+    return from_cuda(csa::launch_compress(a, static_cast<cudaStream_t>(stream), &why), "csa_compress", why);
+}
+
+csa_status_t csa_indexer_topk(const void* qI, int qI_dt, const float* qI_scale, const void* kI,
+                              int kI_dt, const float* kI_scale, int B, int n_q, int H_I, int d_I,
+                              int N_cap, const int* n_entries, const int* q_pos, int m, int topk,
+                              int* idx_out, void* stream) {
+    REQUIRE(B >= 0 && n_q >= 0 && N_cap >= 0, "csa_indexer_topk: negative size");
+    REQUIRE(H_I >= 1 && d_I >= 1, "csa_indexer_topk: H_I and d_I must be positive");
+    REQUIRE(m >= 1, "csa_indexer_topk: m must be >= 1");
+    REQUIRE(topk >= 1 && topk <= 2048, "csa_indexer_topk: topk must be in [1, 2048]");
+    REQUIRE(is_dt(qI_dt) && is_dt(kI_dt), "csa_indexer_topk: unknown dtype");
+    if (d_I % 16) return fail(CSA_ERR_UNSUPPORTED, "csa_indexer_topk: d_I must be a multiple of 16");
+    REQUIRE((qI_dt == CSA_DT_E4M3) == (qI_scale != nullptr),
+            "csa_indexer_topk: qI_scale is required iff qI is E4M3");
+    REQUIRE((kI_dt == CSA_DT_E4M3) == (kI_scale != nullptr),
+            "csa_indexer_topk: kI_scale is required iff kI is E4M3");
+    if ((long)B * n_q == 0) return ok();
+    REQUIRE(qI && idx_out, "csa_indexer_topk: null tensor pointer");
+    REQUIRE(kI || N_cap == 0, "csa_indexer_topk: null kI");
+    REQUIRE_ALIGNED(qI, "qI");
+    REQUIRE_ALIGNED(kI, "kI");
+    REQUIRE_ALIGNED(idx_out, "idx_out");
+    REQUIRE_ALIGNED(qI_scale, "qI_scale");
+    REQUIRE_ALIGNED(kI_scale, "kI_scale");
+    REQUIRE_ALIGNED(n_entries, "n_entries");
+    REQUIRE_ALIGNED(q_pos, "q_pos");
+    csa::IndexerArgs a{qI, qI_dt, qI_scale, kI, kI_dt, kI_scale, B, n_q, H_I, d_I, N_cap,
+                       n_entries, q_pos, m, topk, idx_out};
+    const char* why = nullptr;
+    return from_cuda(csa::launch_indexer_topk(a, static_cast<cudaStream_t>(stream), &why),
+                     "csa_indexer_topk", why);
+}
+
+static csa_status_t attention_common(const char* name, csa::AttnArgs& a, void* stream) {
+    REQUIRE(a.B >= 0 && a.n_q >= 0 && a.N_cap >= 0 && a.L_raw >= 0, "%s: negative size", name);
+    REQUIRE(a.H >= 1 && a.D >= 1, "%s: H and D must be positive", name);
+    REQUIRE(a.window >= 0, "%s: window must be >= 0", name);
+    REQUIRE(a.dt == CSA_DT_F32 || a.dt == CSA_DT_BF16 || a.dt == CSA_DT_E4M3, "%s: unknown dtype", name);
+    if (a.dt == CSA_DT_E4M3) return fail(CSA_ERR_UNSUPPORTED, "%s: dt must be F32 or BF16", name);
+    if (a.D % 16 || a.D > 256) return fail(CSA_ERR_UNSUPPORTED, "%s: D must be a multiple of 16 <= 256", name);
+    if ((long)a.B * a.n_q == 0) return ok();
+    REQUIRE(a.q && a.out, "%s: null q or out", name);
+    REQUIRE(a.kv_c || a.N_cap == 0, "%s: null kv_c", name);
+    REQUIRE(a.kv_raw || a.L_raw == 0, "%s: null kv_raw", name);
+    REQUIRE_ALIGNED(a.q, "q");
+    REQUIRE_ALIGNED(a.kv_c, "kv_c");
+    REQUIRE_ALIGNED(a.kv_raw, "kv_raw");
+    REQUIRE_ALIGNED(a.out, "out");
+    REQUIRE_ALIGNED(a.lse_out, "lse_out");
+    REQUIRE_ALIGNED(a.idx, "idx");
+    REQUIRE_ALIGNED(a.raw_pos0, "raw_pos0");
+    REQUIRE_ALIGNED(a.raw_len, "raw_len");
+    REQUIRE_ALIGNED(a.q_pos, "q_pos");
+    REQUIRE_ALIGNED(a.n_entries, "n_entries");
+    if (!(a.scale > 0.0f)) a.scale = 1.0f / sqrtf((float)a.D);
+    const char* why = nullptr;
+    return from_cuda(csa::launch_attention(a, static_cast<cudaStream_t>(stream), &why), name, why);
+}
+
+csa_status_t csa_sparse_attn(const void* q, int dt, int B, int n_q, int H, int D,
+                             const void* kv_c, int N_cap, const int* idx, int topk,
+                             const void* kv_raw, int L_raw, const int* raw_pos0,
+                             const int* raw_len, int window, const int* q_pos,
+                             float softmax_scale, void* out, float* lse_out, void* stream) {
+    REQUIRE(topk >= 0 && topk <= 2048, "csa_sparse_attn: topk must be in [0, 2048]");
+    REQUIRE(idx || topk == 0 || (long)B * n_q == 0, "csa_sparse_attn: null idx");
+    csa::AttnArgs a{q, dt, B, n_q, H, D, kv_c, N_cap, idx, topk, nullptr, 1, 0, kv_raw, L_raw,
+                    raw_pos0, raw_len, window, q_pos, softmax_scale, out, lse_out};
+    return attention_common("csa_sparse_attn", a, stream);
+}
+
+csa_status_t hca_dense_attn(const void* q, int dt, int B, int n_q, int H, int D,
+                            const void* kv_c, int N_cap, const int* n_entries, int m,
+                            const void* kv_raw, int L_raw, const int* raw_pos0,
+                            const int* raw_len, int window, const int* q_pos,
+                            float softmax_scale, void* out, float* lse_out, void* stream) {
+    REQUIRE(m >= 1, "hca_dense_attn: m must be >= 1");
+    csa::AttnArgs a{q, dt, B, n_q, H, D, kv_c, N_cap, nullptr, 0, n_entries, m, 1, kv_raw, L_raw,
+                    raw_pos0, raw_len, window, q_pos, softmax_scale, out, lse_out};
+    return attention_common("hca_dense_attn", a, stream);
+}
+
+}  // extern "C"

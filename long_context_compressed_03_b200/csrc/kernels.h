@@ -1,0 +1,52 @@
+// kernels.h -- internal launch interface between the C ABI and the kernels.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace csa {
+
+struct CompressArgs {
+    const void* x; int x_dt;
+    int B, n, d_in;
+    const void* W; int d_out;
+    int m, overlap;
+    void* out; int out_dt;
+    float* out_row_scale;
+    int N_c;
+};
+
+struct IndexerArgs {
+    const void* qI; int qI_dt; const float* qI_scale;
+    const void* kI; int kI_dt; const float* kI_scale;
+    int B, n_q, H_I, d_I, N_cap;
+    const int* n_entries; const int* q_pos;
+    int m, topk;
+    int* idx_out;
+};
+
+struct AttnArgs {
+    const void* q; int dt;
+    int B, n_q, H, D;
+    const void* kv_c; int N_cap;
+    const int* idx; int topk;         // sparse mode
+    const int* n_entries; int m;      // dense (HCA) mode
+    int dense;
+    const void* kv_raw; int L_raw;
+    const int* raw_pos0; const int* raw_len;
+    int window;
+    const int* q_pos;
+    float scale;
+    void* out; float* lse_out;
+};
+
+// Counts one kernel launch (read back through csa_kernel_launches()).
+void count_launch();
+
+// Each returns cudaSuccess or the launch error; `why` receives a static
+// reason string when the configuration is unsupported (returned as
+// cudaErrorNotSupported).
+cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s, const char** why);
+cudaError_t launch_indexer_topk(const IndexerArgs& a, cudaStream_t s, const char** why);
+cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s, const char** why);
+
+}  // namespace csa

@@ -66,13 +66,14 @@ def _load():
         lib.oracle_visible_entries.argtypes = [i64, i32, i64]
         lib.oracle_visible_entries.restype = i64
         lib.oracle_compress.argtypes = [P, i32, i32, i32, P, i32, i32, i32, P]
-        lib.oracle_indexer_scores.argtypes = [P, P, i32, i32, i32, i32, i32, P, P, i32, P, i64, P]
-        lib.oracle_indexer_topk.argtypes = [P, P, i32, i32, i32, i32, i32, P, P, i32, i32, P, i64,
-                                            P, P, P]
-        lib.oracle_sparse_attn.argtypes = [P, i32, i32, i32, i32, P, i32, P, i32, P, i32, P, P,
-                                           i32, P, ctypes.c_double, P, i64, P, P]
-        lib.oracle_hca_attn.argtypes = [P, i32, i32, i32, i32, P, i32, P, i32, P, i32, P, P, i32,
-                                        P, ctypes.c_double, P, i64, P, P]
+        dbl = ctypes.c_double
+        lib.oracle_indexer_scores.argtypes = [P, P, P, i64, i32, i32, P, P, P, i32, P, i32, P]
+        lib.oracle_indexer_topk.argtypes = [P, P, P, i64, i32, i32, P, P, P, i32, P, i32, i32, P,
+                                            P, P]
+        lib.oracle_sparse_attn.argtypes = [P, P, P, i64, i32, i32, P, i32, P, i32, P, i32, P, P,
+                                           i32, dbl, P, P]
+        lib.oracle_hca_attn.argtypes = [P, P, P, i64, i32, i32, P, i32, P, i32, P, i32, P, P, i32,
+                                        dbl, P, P]
         _lib = lib
         return lib
 
@@ -176,40 +177,86 @@ def _defaults(B, n_q, N_cap, n_entries, q_pos):
     return _i32(n_entries), _i32(q_pos)
 
 
-def indexer_scores(qI, kI, m: int, n_entries=None, q_pos=None, rows=None) -> np.ndarray:
-    """Scores sum_h ReLU(qI[t,h].kI[s]) of the listed query rows (flattened
-    b*n_q+q; all rows by default) against every entry; NaN where invisible.
-    qI: [B, n_q, H_I, d_I]; kI: [B, N_cap, d_I] (dequantised values)."""
-    qI = _f64(qI)
-    kI = _f64(kI)
-    B, n_q, H_I, d_I = qI.shape
-    N_cap = kI.shape[1]
-    n_entries, q_pos = _defaults(B, n_q, N_cap, n_entries, q_pos)
-    rows = _rows_arg(rows, B * n_q)
-    out = np.empty((rows.size, N_cap), dtype=np.float64)
-    _load().oracle_indexer_scores(_ptr(qI), _ptr(kI), B, n_q, H_I, d_I, N_cap, _ptr(n_entries),
-                                  _ptr(q_pos), m, _ptr(rows), rows.size, _ptr(out))
+def _keys_arg(kI, kI_scale):
+    """(fp64 values, codes, scales) pointers for fp64 keys or E4M3 codes + scales."""
+    if kI_scale is None:
+        k = _f64(kI)
+        return k, None, None, (_ptr(k), None, None)
+    c = np.ascontiguousarray(np.asarray(kI, dtype=np.uint8))
+    sc = np.ascontiguousarray(np.asarray(kI_scale, dtype=np.float32))
+    return None, c, sc, (None, _ptr(c), _ptr(sc))
+
+
+def quantized_query_rows(qI_rows) -> np.ndarray:
+    """fp64 values of query rows after the per-(row, head) E4M3 quantisation
+    the indexer applies to bf16 queries against fp8 keys (fp32 procedure)."""
+    q = np.asarray(qI_rows, dtype=np.float32)
+    codes, scales = quantize_rows_e4m3(q)
+    return dequantize_rows_e4m3(codes, scales)
+
+
+def indexer_scores_rows(qI_rows, row_b, row_t, kI, m: int, n_entries, kI_scale=None):
+    """Scores sum_h ReLU(qI . kI[s]) of listed query rows against every entry.
+    qI_rows [R, H_I, d_I] fp64 (dequantised); row_b/row_t [R] batch element
+    and absolute position; kI [B, N_cap, d_I] fp64 values, or E4M3 codes
+    with kI_scale [B, N_cap]; n_entries [B].  Returns [R, N_cap], NaN where
+    the entry is not visible."""
+    q = _f64(qI_rows)
+    R, H_I, d_I = q.shape
+    keep = _keys_arg(kI, kI_scale)
+    N_cap = np.asarray(kI).shape[1]
+    rb, rt, ne = _i32(row_b), _i32(row_t), _i32(n_entries)
+    out = np.empty((R, N_cap), dtype=np.float64)
+    _load().oracle_indexer_scores(_ptr(q), _ptr(rb), _ptr(rt), R, H_I, d_I, *keep[3], N_cap,
+                                  _ptr(ne), m, _ptr(out))
     return out
 
 
-def indexer_topk(qI, kI, m: int, topk: int, n_entries=None, q_pos=None, rows=None):
-    """Per query row: the topk largest visible scores (ties -> lower index,
-    -1 padding).  Returns (idx [n_rows, topk] int32 in (score desc, index
-    asc) order, kth [n_rows, 2] = k-th and (k+1)-th largest scores (NaN if
-    absent), smax [n_rows] = largest |score|)."""
-    qI = _f64(qI)
-    kI = _f64(kI)
-    B, n_q, H_I, d_I = qI.shape
-    N_cap = kI.shape[1]
-    n_entries, q_pos = _defaults(B, n_q, N_cap, n_entries, q_pos)
-    rows = _rows_arg(rows, B * n_q)
-    idx = np.empty((rows.size, topk), dtype=np.int32)
-    kth = np.empty((rows.size, 2), dtype=np.float64)
-    smax = np.empty(rows.size, dtype=np.float64)
-    _load().oracle_indexer_topk(_ptr(qI), _ptr(kI), B, n_q, H_I, d_I, N_cap, _ptr(n_entries),
-                                _ptr(q_pos), m, topk, _ptr(rows), rows.size, _ptr(idx),
-                                _ptr(kth), _ptr(smax))
+def indexer_topk_rows(qI_rows, row_b, row_t, kI, m: int, topk: int, n_entries, kI_scale=None):
+    """Per listed query row: the topk largest visible scores (ties -> lower
+    index, -1 padding).  Returns (idx [R, topk] int32 in (score desc, index
+    asc) order, kth [R, 2] = k-th and (k+1)-th largest scores (NaN if
+    absent), smax [R] = largest |score|)."""
+    q = _f64(qI_rows)
+    R, H_I, d_I = q.shape
+    keep = _keys_arg(kI, kI_scale)
+    N_cap = np.asarray(kI).shape[1]
+    rb, rt, ne = _i32(row_b), _i32(row_t), _i32(n_entries)
+    idx = np.empty((R, topk), dtype=np.int32)
+    kth = np.empty((R, 2), dtype=np.float64)
+    smax = np.empty(R, dtype=np.float64)
+    _load().oracle_indexer_topk(_ptr(q), _ptr(rb), _ptr(rt), R, H_I, d_I, *keep[3], N_cap,
+                                _ptr(ne), m, topk, _ptr(idx), _ptr(kth), _ptr(smax))
     return idx, kth, smax
+
+
+def _full_rows(B, n_q, q_pos, rows):
+    r = _rows_arg(rows, B * n_q)
+    qp = np.asarray(q_pos).reshape(-1)
+    return r, (r // n_q).astype(np.int32), qp[r].astype(np.int32)
+
+
+def indexer_scores(qI, kI, m: int, n_entries=None, q_pos=None, rows=None, kI_scale=None):
+    """indexer_scores_rows over full tensors qI [B, n_q, H_I, d_I]; rows are
+    flattened b*n_q+q (all by default)."""
+    qI = _f64(qI)
+    B, n_q, H_I, d_I = qI.shape
+    N_cap = np.asarray(kI).shape[1]
+    n_entries, q_pos = _defaults(B, n_q, N_cap, n_entries, q_pos)
+    r, rb, rt = _full_rows(B, n_q, q_pos, rows)
+    return indexer_scores_rows(qI.reshape(B * n_q, H_I, d_I)[r], rb, rt, kI, m, n_entries,
+                               kI_scale)
+
+
+def indexer_topk(qI, kI, m: int, topk: int, n_entries=None, q_pos=None, rows=None, kI_scale=None):
+    """indexer_topk_rows over full tensors (see indexer_scores)."""
+    qI = _f64(qI)
+    B, n_q, H_I, d_I = qI.shape
+    N_cap = np.asarray(kI).shape[1]
+    n_entries, q_pos = _defaults(B, n_q, N_cap, n_entries, q_pos)
+    r, rb, rt = _full_rows(B, n_q, q_pos, rows)
+    return indexer_topk_rows(qI.reshape(B * n_q, H_I, d_I)[r], rb, rt, kI, m, topk, n_entries,
+                             kI_scale)
 
 
 # --------------------------------------------------------------------------
@@ -223,70 +270,90 @@ def _raw_defaults(B, L_raw, raw_pos0, raw_len):
     return _i32(raw_pos0), _i32(raw_len)
 
 
-def sparse_attn(q, kv_c, idx, kv_raw, window: int, q_pos=None, raw_pos0=None, raw_len=None,
-                scale: float | None = None, rows=None):
-    """Joint softmax over {kv_c[idx[r, j]] : idx >= 0} ∪ window raw rows.
-    q: [B, n_q, H, D]; kv_c: [B, N_cap, D]; idx: [B, n_q, topk];
-    kv_raw: [B, L_raw, D].  Returns (o [n_rows, H, D], lse [n_rows, H])."""
-    q = _f64(q)
+def sparse_attn_rows(q_rows, row_b, row_t, kv_c, idx_rows, kv_raw, window: int, raw_pos0=None,
+                     raw_len=None, scale: float | None = None):
+    """Joint softmax over {kv_c[b, idx] : 0 <= idx < N_cap} ∪ window raw rows
+    for listed query rows.  q_rows [R, H, D]; row_b/row_t [R]; kv_c
+    [B, N_cap, D]; idx_rows [R, topk]; kv_raw [B, L_raw, D].
+    Returns (o [R, H, D], lse [R, H])."""
+    q = _f64(q_rows)
+    R, H, D = q.shape
     kv_c = _f64(kv_c)
     kv_raw = _f64(kv_raw)
-    idx = _i32(idx)
-    B, n_q, H, D = q.shape
-    N_cap = kv_c.shape[1]
+    idx = _i32(idx_rows).reshape(R, -1) if R else _i32(np.zeros((0, 0)))
+    topk = idx.shape[1] if R else 0
+    B, N_cap = kv_c.shape[0], kv_c.shape[1]
     L_raw = kv_raw.shape[1]
-    topk = idx.shape[-1]
-    _, q_pos = _defaults(B, n_q, N_cap, None, q_pos)
     raw_pos0, raw_len = _raw_defaults(B, L_raw, raw_pos0, raw_len)
-    if scale is None:
-        scale = 1.0 / np.sqrt(D)
-    rows = _rows_arg(rows, B * n_q)
-    out = np.empty((rows.size, H, D), dtype=np.float64)
-    lse = np.empty((rows.size, H), dtype=np.float64)
-    _load().oracle_sparse_attn(_ptr(q), B, n_q, H, D, _ptr(kv_c), N_cap, _ptr(idx), topk,
-                               _ptr(kv_raw), L_raw, _ptr(raw_pos0), _ptr(raw_len), window,
-                               _ptr(q_pos), float(scale), _ptr(rows), rows.size, _ptr(out),
-                               _ptr(lse))
+    scale = 1.0 / np.sqrt(D) if scale is None else scale
+    rb, rt = _i32(row_b), _i32(row_t)
+    out = np.empty((R, H, D), dtype=np.float64)
+    lse = np.empty((R, H), dtype=np.float64)
+    _load().oracle_sparse_attn(_ptr(q), _ptr(rb), _ptr(rt), R, H, D, _ptr(kv_c), N_cap,
+                               _ptr(idx), topk, _ptr(kv_raw), L_raw, _ptr(raw_pos0),
+                               _ptr(raw_len), window, float(scale), _ptr(out), _ptr(lse))
     return out, lse
+
+
+def hca_attn_rows(q_rows, row_b, row_t, kv_c, m: int, kv_raw, window: int, n_entries=None,
+                  raw_pos0=None, raw_len=None, scale: float | None = None):
+    """Dense attention over every visible entry s < min(floor((t+1)/m),
+    n_entries) plus the window, one softmax, for listed query rows."""
+    q = _f64(q_rows)
+    R, H, D = q.shape
+    kv_c = _f64(kv_c)
+    kv_raw = _f64(kv_raw)
+    B, N_cap = kv_c.shape[0], kv_c.shape[1]
+    L_raw = kv_raw.shape[1]
+    if n_entries is None:
+        n_entries = np.full(B, N_cap, dtype=np.int32)
+    ne = _i32(n_entries)
+    raw_pos0, raw_len = _raw_defaults(B, L_raw, raw_pos0, raw_len)
+    scale = 1.0 / np.sqrt(D) if scale is None else scale
+    rb, rt = _i32(row_b), _i32(row_t)
+    out = np.empty((R, H, D), dtype=np.float64)
+    lse = np.empty((R, H), dtype=np.float64)
+    _load().oracle_hca_attn(_ptr(q), _ptr(rb), _ptr(rt), R, H, D, _ptr(kv_c), N_cap, _ptr(ne), m,
+                            _ptr(kv_raw), L_raw, _ptr(raw_pos0), _ptr(raw_len), window,
+                            float(scale), _ptr(out), _ptr(lse))
+    return out, lse
+
+
+def sparse_attn(q, kv_c, idx, kv_raw, window: int, q_pos=None, raw_pos0=None, raw_len=None,
+                scale: float | None = None, rows=None):
+    """sparse_attn_rows over full tensors q [B, n_q, H, D], idx [B, n_q, topk]."""
+    q = _f64(q)
+    B, n_q, H, D = q.shape
+    _, q_pos = _defaults(B, n_q, 0, None, q_pos)
+    r, rb, rt = _full_rows(B, n_q, q_pos, rows)
+    idx = _i32(idx).reshape(B * n_q, -1)
+    return sparse_attn_rows(q.reshape(B * n_q, H, D)[r], rb, rt, kv_c, idx[r], kv_raw, window,
+                            raw_pos0, raw_len, scale)
 
 
 def hca_attn(q, kv_c, m: int, kv_raw, window: int, n_entries=None, q_pos=None, raw_pos0=None,
              raw_len=None, scale: float | None = None, rows=None):
-    """Dense attention over every visible entry s < min(floor((t+1)/m),
-    n_entries) plus the window, under one softmax.  Shapes as sparse_attn."""
+    """hca_attn_rows over full tensors q [B, n_q, H, D]."""
     q = _f64(q)
-    kv_c = _f64(kv_c)
-    kv_raw = _f64(kv_raw)
     B, n_q, H, D = q.shape
-    N_cap = kv_c.shape[1]
-    L_raw = kv_raw.shape[1]
-    n_entries, q_pos = _defaults(B, n_q, N_cap, n_entries, q_pos)
-    raw_pos0, raw_len = _raw_defaults(B, L_raw, raw_pos0, raw_len)
-    if scale is None:
-        scale = 1.0 / np.sqrt(D)
-    rows = _rows_arg(rows, B * n_q)
-    out = np.empty((rows.size, H, D), dtype=np.float64)
-    lse = np.empty((rows.size, H), dtype=np.float64)
-    _load().oracle_hca_attn(_ptr(q), B, n_q, H, D, _ptr(kv_c), N_cap, _ptr(n_entries), m,
-                            _ptr(kv_raw), L_raw, _ptr(raw_pos0), _ptr(raw_len), window,
-                            _ptr(q_pos), float(scale), _ptr(rows), rows.size, _ptr(out),
-                            _ptr(lse))
-    return out, lse
+    _, q_pos = _defaults(B, n_q, 0, None, q_pos)
+    r, rb, rt = _full_rows(B, n_q, q_pos, rows)
+    return hca_attn_rows(q.reshape(B * n_q, H, D)[r], rb, rt, kv_c, m, kv_raw, window, n_entries,
+                         raw_pos0, raw_len, scale)
 
 
 # --------------------------------------------------------------------------
 # End to end: stage 1 -> 2 -> 3 (a composition of the functions above)
 # --------------------------------------------------------------------------
 def csa_forward(q, kv, qI, kI_raw, W_c, W_Ic, m: int, topk: int, window: int, rows=None):
-    """Whole CSA prefill for one batch of sequences (positions 0..n-1):
-    compress kv and the indexer keys with overlap, score + top-k, attend.
-    Returns (o [n_rows, H, D], lse, idx [n_rows, topk])."""
+    """Whole CSA prefill for a batch of sequences (positions 0..n-1): compress
+    kv and the indexer keys with overlap, score + top-k, attend.
+    Returns (o [R, H, D], lse [R, H], idx [R, topk]) for the listed rows."""
     kv_c = compress(kv, W_c, m, True)
     kI_c = compress(kI_raw, W_Ic, m, True)
-    B, n_q = np.asarray(q).shape[:2]
     idx, _, _ = indexer_topk(qI, kI_c, m, topk, rows=rows)
-    full_idx = np.full((B, n_q, topk), -1, dtype=np.int32)
-    r = _rows_arg(rows, B * n_q)
-    full_idx.reshape(B * n_q, topk)[r] = idx
-    o, lse = sparse_attn(q, kv_c, full_idx, kv, window, rows=rows)
+    B, n_q = np.asarray(q).shape[:2]
+    q = _f64(q)
+    r, rb, rt = _full_rows(B, n_q, np.broadcast_to(np.arange(n_q), (B, n_q)), rows)
+    o, lse = sparse_attn_rows(q.reshape(B * n_q, *q.shape[2:])[r], rb, rt, kv_c, idx, kv, window)
     return o, lse, idx

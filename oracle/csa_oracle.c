@@ -175,11 +175,24 @@ long oracle_visible_entries(long t, int m, long n_entries) {
  * One shared indexer key row per entry (MQA-like); each indexer head passes
  * its dot product through a ReLU before the heads are summed.
  *
- * rows: list of flattened query rows r = b*n_q + q to score; scores gets
- * n_rows x N_cap values, NaN where the entry is not visible.
- * qI: [B, n_q, H_I, d_I] (already dequantised), kI: [B, N_cap, d_I].
- * q_pos: [B, n_q] absolute positions; n_entries: [B].
+ * Query rows are given as a list: row rr has batch element row_b[rr],
+ * absolute position row_t[rr] and query values qI_rows[rr, H_I, d_I] (fp64,
+ * already dequantised).  Keys kI [B, N_cap, d_I] are given either as fp64
+ * values (kI_f64) or as E4M3 codes with one fp32 scale per entry (kI_codes +
+ * kI_scale), dequantised here in fp64.
+ * scores receives n_rows x N_cap values, NaN where the entry is not visible.
  * --------------------------------------------------------------------- */
+static void key_row(const double* kI_f64, const uint8_t* kI_codes, const float* kI_scale, int b,
+                    long s, int N_cap, int d_I, double* out) {
+    long base = ((long)b * N_cap + s) * d_I;
+    if (kI_f64) {
+        for (int c = 0; c < d_I; ++c) out[c] = kI_f64[base + c];
+    } else {
+        double sc = (double)kI_scale[(long)b * N_cap + s];
+        for (int c = 0; c < d_I; ++c) out[c] = oracle_e4m3_decode(kI_codes[base + c]) * sc;
+    }
+}
+
 static double score_one(const double* qrow, int H_I, int d_I, const double* krow) {
     double s = 0.0;
     for (int h = 0; h < H_I; ++h) {
@@ -190,23 +203,26 @@ static double score_one(const double* qrow, int H_I, int d_I, const double* krow
     return s;
 }
 
-void oracle_indexer_scores(const double* qI, const double* kI, int B, int n_q, int H_I, int d_I,
-                           int N_cap, const int* n_entries, const int* q_pos, int m,
-                           const long* rows, long n_rows, double* scores) {
-    (void)B;
+void oracle_indexer_scores(const double* qI_rows, const int* row_b, const int* row_t, long n_rows,
+                           int H_I, int d_I, const double* kI_f64, const uint8_t* kI_codes,
+                           const float* kI_scale, int N_cap, const int* n_entries, int m,
+                           double* scores) {
     #pragma omp parallel for schedule(dynamic, 4)
     for (long rr = 0; rr < n_rows; ++rr) {
-        long r = rows[rr];
-        int b = (int)(r / n_q);
-        const double* qrow = qI + r * (long)H_I * d_I;
-        long V = oracle_visible_entries(q_pos[r], m, n_entries[b]);
+        int b = row_b[rr];
+        const double* qrow = qI_rows + rr * (long)H_I * d_I;
+        long V = oracle_visible_entries(row_t[rr], m, n_entries[b]);
         double* out = scores + rr * (long)N_cap;
+        double* krow = (double*)malloc(sizeof(double) * (size_t)d_I);
         for (long s = 0; s < N_cap; ++s) {
-            if (s < V)
-                out[s] = score_one(qrow, H_I, d_I, kI + ((long)b * N_cap + s) * d_I);
-            else
+            if (s < V) {
+                key_row(kI_f64, kI_codes, kI_scale, b, s, N_cap, d_I, krow);
+                out[s] = score_one(qrow, H_I, d_I, krow);
+            } else {
                 out[s] = NAN;
+            }
         }
+        free(krow);
     }
 }
 
@@ -228,20 +244,21 @@ static int cmp_scored(const void* a, const void* b) {
     return (x->i < y->i) ? -1 : (x->i > y->i);
 }
 
-void oracle_indexer_topk(const double* qI, const double* kI, int B, int n_q, int H_I, int d_I,
-                         int N_cap, const int* n_entries, const int* q_pos, int m, int topk,
-                         const long* rows, long n_rows, int* idx_out, double* kth, double* smax) {
-    (void)B;
+void oracle_indexer_topk(const double* qI_rows, const int* row_b, const int* row_t, long n_rows,
+                         int H_I, int d_I, const double* kI_f64, const uint8_t* kI_codes,
+                         const float* kI_scale, int N_cap, const int* n_entries, int m, int topk,
+                         int* idx_out, double* kth, double* smax) {
     #pragma omp parallel for schedule(dynamic, 4)
     for (long rr = 0; rr < n_rows; ++rr) {
-        long r = rows[rr];
-        int b = (int)(r / n_q);
-        const double* qrow = qI + r * (long)H_I * d_I;
-        long V = oracle_visible_entries(q_pos[r], m, n_entries[b]);
+        int b = row_b[rr];
+        const double* qrow = qI_rows + rr * (long)H_I * d_I;
+        long V = oracle_visible_entries(row_t[rr], m, n_entries[b]);
         scored_t* all = (scored_t*)malloc(sizeof(scored_t) * (size_t)(V > 0 ? V : 1));
+        double* krow = (double*)malloc(sizeof(double) * (size_t)d_I);
         double amax = 0.0;
         for (long s = 0; s < V; ++s) {
-            all[s].s = score_one(qrow, H_I, d_I, kI + ((long)b * N_cap + s) * d_I);
+            key_row(kI_f64, kI_codes, kI_scale, b, s, N_cap, d_I, krow);
+            all[s].s = score_one(qrow, H_I, d_I, krow);
             all[s].i = s;
             if (fabs(all[s].s) > amax) amax = fabs(all[s].s);
         }
@@ -253,6 +270,7 @@ void oracle_indexer_topk(const double* qI, const double* kI, int B, int n_q, int
             kth[2 * rr + 1] = (topk < V) ? all[topk].s : NAN;
         }
         if (smax) smax[rr] = amax;
+        free(krow);
         free(all);
     }
 }
@@ -262,7 +280,8 @@ void oracle_indexer_topk(const double* qI, const double* kI, int B, int n_q, int
  * plus the sliding window of raw KV ([P3] §1.2, §1.5; [P5] §5.2).
  *
  * Keys and values are the same vectors (shared-KV MQA: one KV head serves
- * every query head).  For query row r at absolute position t and head h:
+ * every query head).  For query row rr (batch element row_b[rr], absolute
+ * position t = row_t[rr], query q_rows[rr, H, D]) and head h:
  *   S_c(t) = the compressed entries listed for the row,
  *   S_w(t) = raw positions p with max(0, t-W+1) <= p <= t that the raw
  *            buffer holds (raw row j holds position raw_pos0[b] + j, rows
@@ -313,29 +332,27 @@ static long window_keys(const double* kv_raw, int b, int L_raw, int D, const int
     return nk;
 }
 
-/* Sparse attention: S_c(t) = the non-negative entries of idx[r, :] below
- * N_cap (negative entries are padding; entries >= N_cap are ignored). */
-void oracle_sparse_attn(const double* q, int B, int n_q, int H, int D, const double* kv_c,
-                        int N_cap, const int* idx, int topk, const double* kv_raw, int L_raw,
-                        const int* raw_pos0, const int* raw_len, int window, const int* q_pos,
-                        double scale, const long* rows, long n_rows, double* out, double* lse) {
-    (void)B;
+/* Sparse attention: S_c(t) = the non-negative entries of idx_rows[rr, :]
+ * below N_cap (negative entries are padding; entries >= N_cap are ignored). */
+void oracle_sparse_attn(const double* q_rows, const int* row_b, const int* row_t, long n_rows, int H,
+                        int D, const double* kv_c, int N_cap, const int* idx_rows, int topk,
+                        const double* kv_raw, int L_raw, const int* raw_pos0, const int* raw_len,
+                        int window, double scale, double* out, double* lse) {
     #pragma omp parallel for schedule(dynamic, 4)
     for (long rr = 0; rr < n_rows; ++rr) {
-        long r = rows[rr];
-        int b = (int)(r / n_q);
-        long t = q_pos[r];
+        int b = row_b[rr];
+        long t = row_t[rr];
         long cap = (long)topk + (window > 0 ? window : 0);
         const double** keys = (const double**)malloc(sizeof(double*) * (size_t)(cap + 1));
         double* z = (double*)malloc(sizeof(double) * (size_t)(cap + 1));
         long nk = 0;
         for (int j = 0; j < topk; ++j) {
-            int s = idx[r * (long)topk + j];
+            int s = idx_rows[rr * (long)topk + j];
             if (s < 0 || s >= N_cap) continue;
             keys[nk++] = kv_c + ((long)b * N_cap + s) * D;
         }
         nk = window_keys(kv_raw, b, L_raw, D, raw_pos0, raw_len, window, t, keys, nk);
-        attend_row(q + r * (long)H * D, H, D, scale, keys, nk, out + rr * (long)H * D,
+        attend_row(q_rows + rr * (long)H * D, H, D, scale, keys, nk, out + rr * (long)H * D,
                    lse ? lse + rr * (long)H : NULL, z);
         free(keys);
         free(z);
@@ -344,16 +361,14 @@ void oracle_sparse_attn(const double* q, int B, int n_q, int H, int D, const dou
 
 /* HCA dense attention ([P3] §1.4; [P5] §4.3): S_c(t) = every entry
  * s < min(floor((t+1)/m), n_entries[b]) -- no top-k -- plus the window. */
-void oracle_hca_attn(const double* q, int B, int n_q, int H, int D, const double* kv_c, int N_cap,
-                     const int* n_entries, int m, const double* kv_raw, int L_raw,
-                     const int* raw_pos0, const int* raw_len, int window, const int* q_pos,
-                     double scale, const long* rows, long n_rows, double* out, double* lse) {
-    (void)B;
+void oracle_hca_attn(const double* q_rows, const int* row_b, const int* row_t, long n_rows, int H,
+                     int D, const double* kv_c, int N_cap, const int* n_entries, int m,
+                     const double* kv_raw, int L_raw, const int* raw_pos0, const int* raw_len,
+                     int window, double scale, double* out, double* lse) {
     #pragma omp parallel for schedule(dynamic, 4)
     for (long rr = 0; rr < n_rows; ++rr) {
-        long r = rows[rr];
-        int b = (int)(r / n_q);
-        long t = q_pos[r];
+        int b = row_b[rr];
+        long t = row_t[rr];
         long V = oracle_visible_entries(t, m, n_entries[b]);
         if (V > N_cap) V = N_cap;
         long cap = V + (window > 0 ? window : 0);
@@ -362,7 +377,7 @@ void oracle_hca_attn(const double* q, int B, int n_q, int H, int D, const double
         long nk = 0;
         for (long s = 0; s < V; ++s) keys[nk++] = kv_c + ((long)b * N_cap + s) * D;
         nk = window_keys(kv_raw, b, L_raw, D, raw_pos0, raw_len, window, t, keys, nk);
-        attend_row(q + r * (long)H * D, H, D, scale, keys, nk, out + rr * (long)H * D,
+        attend_row(q_rows + rr * (long)H * D, H, D, scale, keys, nk, out + rr * (long)H * D,
                    lse ? lse + rr * (long)H : NULL, z);
         free(keys);
         free(z);

@@ -1,0 +1,137 @@
+"""Host-side checks of the C ABI: the library loads, exports every symbol the
+header declares, the binding's signature table matches the header, and
+argument validation rejects bad calls before anything reaches the GPU.
+CPU only: every call here fails validation (or is a no-op), so no kernel
+is launched and no device memory is touched."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from long_context_compressed_03_b200 import api, build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "csa_b200.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build_mod.build()
+    return api.load()
+
+
+def _declared():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    protos = {}
+    for m in re.finditer(r"(?:csa_status_t|const char\s*\*|unsigned long long|int)\s+(\w+)\s*\(([^)]*)\)\s*;",
+                         text):
+        name, params = m.group(1), m.group(2).strip()
+        n = 0 if params in ("", "void") else len(params.split(","))
+        protos[name] = n
+    return protos
+
+
+def test_header_declares_the_four_stage_entry_points():
+    d = _declared()
+    for name in ("csa_compress", "csa_indexer_topk", "csa_sparse_attn", "hca_dense_attn",
+                 "csa_status_string", "csa_last_error_detail", "csa_version"):
+        assert name in d
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_binding_signatures_match_header_arity():
+    d = _declared()
+    for name, n in d.items():
+        assert name in api.SIGNATURES, name
+        assert len(api.SIGNATURES[name][1]) == n, name
+
+
+def test_status_strings(lib):
+    assert api.csa_version() == 100
+    assert lib.csa_status_string(0) == b"CSA_OK"
+    assert lib.csa_status_string(3) == b"CSA_ERR_MISALIGNED"
+    assert lib.csa_status_string(99) == b"CSA_ERR_UNKNOWN"
+
+
+FAKE = ctypes.c_void_p(0x10000)     # never dereferenced: validation fails first
+ODD = ctypes.c_void_p(0x10001)
+
+
+def _detail(lib):
+    return lib.csa_last_error_detail().decode()
+
+
+def test_compress_validation(lib):
+    f = lib.csa_compress
+    assert f(FAKE, 1, 1, 64, 128, FAKE, 128, 0, 1, FAKE, 1, None, None) == api.CSA_ERR_INVALID_ARG
+    assert "m must be" in _detail(lib)
+    assert f(FAKE, 1, 1, 64, 128, FAKE, 128, 4, 2, FAKE, 1, None, None) == api.CSA_ERR_INVALID_ARG
+    assert f(FAKE, 1, 1, 64, 120, FAKE, 128, 4, 1, FAKE, 1, None, None) == api.CSA_ERR_UNSUPPORTED
+    assert f(FAKE, 1, 1, 64, 128, FAKE, 128, 4, 1, FAKE, 0, None, None) == api.CSA_ERR_UNSUPPORTED
+    # fp8 output without a scale buffer, and a scale buffer without fp8
+    assert f(FAKE, 1, 1, 64, 128, FAKE, 128, 4, 1, FAKE, 2, None, None) == api.CSA_ERR_INVALID_ARG
+    assert f(FAKE, 1, 1, 64, 128, FAKE, 128, 4, 1, FAKE, 1, FAKE, None) == api.CSA_ERR_INVALID_ARG
+    assert f(ODD, 1, 1, 64, 128, FAKE, 128, 4, 1, FAKE, 1, None, None) == api.CSA_ERR_MISALIGNED
+    assert f(None, 1, 1, 64, 128, FAKE, 128, 4, 1, FAKE, 1, None, None) == api.CSA_ERR_INVALID_ARG
+    # no entries (n < m, or B = 0): nothing to do, nothing launched
+    assert f(None, 1, 1, 3, 128, None, 128, 4, 1, None, 1, None, None) == api.CSA_OK
+    assert f(None, 1, 0, 64, 128, None, 128, 4, 1, None, 1, None, None) == api.CSA_OK
+
+
+def test_indexer_validation(lib):
+    f = lib.csa_indexer_topk
+    args = [FAKE, 1, None, FAKE, 1, None, 1, 8, 4, 64, 16, None, None, 4, 8, FAKE, None]
+    bad = list(args); bad[14] = 0                      # topk = 0
+    assert f(*bad) == api.CSA_ERR_INVALID_ARG
+    bad = list(args); bad[14] = 4096                   # topk > 2048
+    assert f(*bad) == api.CSA_ERR_INVALID_ARG
+    bad = list(args); bad[4] = 2                       # fp8 keys without scales
+    assert f(*bad) == api.CSA_ERR_INVALID_ARG
+    bad = list(args); bad[9] = 60                      # d_I not a multiple of 16
+    assert f(*bad) == api.CSA_ERR_UNSUPPORTED
+    bad = list(args); bad[0] = ODD
+    assert f(*bad) == api.CSA_ERR_MISALIGNED
+    bad = list(args); bad[13] = 0                      # m = 0
+    assert f(*bad) == api.CSA_ERR_INVALID_ARG
+    ok = list(args); ok[7] = 0                         # n_q = 0: no-op
+    assert f(*ok) == api.CSA_OK
+
+
+def test_attention_validation(lib):
+    f = lib.csa_sparse_attn
+    args = [FAKE, 1, 1, 8, 64, 128, FAKE, 16, FAKE, 4, FAKE, 8, None, None, 4, None,
+            ctypes.c_float(0.0), FAKE, None, None]
+    bad = list(args); bad[14] = -1
+    assert f(*bad) == api.CSA_ERR_INVALID_ARG
+    bad = list(args); bad[5] = 100
+    assert f(*bad) == api.CSA_ERR_UNSUPPORTED
+    bad = list(args); bad[1] = 2
+    assert f(*bad) == api.CSA_ERR_UNSUPPORTED
+    bad = list(args); bad[8] = None                    # idx NULL with topk > 0
+    assert f(*bad) == api.CSA_ERR_INVALID_ARG
+    bad = list(args); bad[17] = ODD
+    assert f(*bad) == api.CSA_ERR_MISALIGNED
+    ok = list(args); ok[2] = 0
+    assert f(*ok) == api.CSA_OK
+    g = lib.hca_dense_attn
+    hargs = [FAKE, 1, 1, 8, 64, 128, FAKE, 16, None, 0, FAKE, 8, None, None, 4, None,
+             ctypes.c_float(0.0), FAKE, None, None]
+    assert g(*hargs) == api.CSA_ERR_INVALID_ARG          # m = 0
+    assert "m must be" in _detail(lib)
+
+
+def test_binding_raises_loudly_without_library(tmp_path):
+    import importlib
+    mod = importlib.reload(api)
+    try:
+        with pytest.raises(RuntimeError, match="not found"):
+            mod._lib = None
+            mod.load(str(tmp_path / "missing.so"))
+    finally:
+        importlib.reload(api)
