@@ -76,6 +76,13 @@ int csa_version(void);
  * (diagnostics: lets a caller count the device work behind its calls). */
 unsigned long long csa_kernel_launches(void);
 
+/* Kernels that wait on on-chip barriers bound every wait (1 s); when one
+ * expires the kernel records it in a per-device error word, stops and exits
+ * cleanly.  This call synchronises `stream`, reads the word and returns
+ * CSA_ERR_TIMEOUT if it is set (clearing it when `clear` is non-zero),
+ * CSA_OK otherwise. */
+csa_status_t csa_check_device_error(void* stream, int clear);
+
 /*
  * csa_compress -- stage 1: overlapping (or plain) mean-pool compression
  * followed by a projection, optionally quantised to fp8.

@@ -33,6 +33,7 @@ SIGNATURES = {
     "csa_last_error_detail": (ctypes.c_char_p, []),
     "csa_version": (I, []),
     "csa_kernel_launches": (ctypes.c_ulonglong, []),
+    "csa_check_device_error": (I, [P, I]),
     "csa_compress": (I, [P, I, I, I, I, P, I, I, I, P, I, P, P]),
     "csa_indexer_topk": (I, [P, I, P, P, I, P, I, I, I, I, I, P, P, I, I, P, P]),
     "csa_sparse_attn": (I, [P, I, I, I, I, I, P, I, P, I, P, I, P, P, I, P, F, P, P, P]),
@@ -124,6 +125,12 @@ def csa_version() -> int:
 def csa_kernel_launches() -> int:
     """Kernels the library has launched in this process so far."""
     return int(load().csa_kernel_launches())
+
+
+def csa_check_device_error(clear: bool = True, stream=None) -> None:
+    """Synchronise the stream and raise CsaError(CSA_ERR_TIMEOUT) if a kernel's
+    bounded on-chip wait expired since the last check."""
+    _check(load().csa_check_device_error(_stream(stream), int(bool(clear))))
 
 
 def csa_compress(x: torch.Tensor, W: torch.Tensor, m: int, overlap: bool, out: torch.Tensor,

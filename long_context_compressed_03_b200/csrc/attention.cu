@@ -194,6 +194,11 @@ cudaError_t launch_dims(const AttnArgs& a, cudaStream_t s, const char** why) {
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s, const char** why) {
     if (a.B <= 0 || a.n_q <= 0) return cudaSuccess;
+    if (attention_tc_supported(a)) {
+        uint32_t* err = device_error_word();
+        if (!err) return cudaErrorUnknown;
+        return launch_attention_tc(a, err, s);
+    }
     if (a.dt == DT_F32) return launch_dims<float>(a, s, why);
     if (a.dt == DT_BF16) return launch_dims<__nv_bfloat16>(a, s, why);
     *why = "attention: dt must be F32 or BF16";

@@ -1,0 +1,608 @@
+// attention_tc.cu -- tensor-core (tcgen05) prefill attention for the CSA /
+// HCA joint softmax with 64 query heads of dimension 128 sharing one KV head.
+//
+// For query token t and head h (one softmax over the multiset union):
+//   keys = compressed set(t) ∪ raw window [max(0, t-W+1), t]
+//   o = sum softmax(scale * q.key) key          (key = value: shared-KV MQA)
+// ("DS-V4 分析&学习" §1.2, §1.4, §1.5; "百万上下文从「奢侈品」变「日用品」…"
+//  §4.3, §5.2.)  Compressed set: the token's top-k entries (sparse mode) or
+// every entry s < floor((t+1)/m) (dense / HCA mode).
+//
+// Work unit: one CTA owns 4 consecutive tokens of one sequence as two M=128
+// tiles (2 tokens x 64 heads each).  Every head of a token attends to the
+// same keys, so a key tile of 128 rows x 128 dims serves a whole M tile.
+//   - window tiles (and dense-mode prefix tiles) are shared by both M tiles
+//     and loaded once per CTA by 2D TMA;
+//   - sparse-mode compressed tiles belong to one token: they are fetched
+//     with TMA row gathers (4 rows per instruction) straight into the
+//     128-byte-swizzled layout the tensor core reads, and the rows of the
+//     other token in the M tile are masked.
+// Roles (12 warps): warp 0 issues TMA, warp 1 allocates TMEM and one lane
+// issues every MMA, warps 4-7 / 8-11 run the softmax of M tile 0 / 1.
+// TMEM: S0 [cols 0,128), S1 [128,256), O0 [256,384), O1 [384,512).
+// S = Q K^T (M=128, N<=128, K=128 in 8 steps), P = exp2(S*scale*log2e - m)
+// in bf16 written to swizzled shared memory, O += P V with V the same
+// shared tile read as an MN-major operand.  The running max is only raised
+// (and O rescaled in TMEM) when it grows by more than 2^8, so most tiles need
+// no rescale; the final division by the running sum is exact.
+#include <cudaTypedefs.h>
+
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_common.cuh"
+
+namespace csa {
+namespace {
+
+using namespace tc;
+
+constexpr int kH = 64;
+constexpr int kD = 128;
+constexpr int kRows = 128;          // rows of an M tile
+constexpr int kTokens = 4;          // tokens per CTA
+constexpr int kBN = 128;            // keys per tile
+constexpr int kStages = 3;
+constexpr int kThreads = 384;
+constexpr int kHalf = 16384;        // one 64-column half of a 128-row tile
+constexpr int kTileBytes = 32768;   // 128 rows x 128 bf16
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRescaleLog2 = 8.0f;
+
+struct __align__(8) Ctrl {
+    uint64_t bar_q;
+    uint64_t full[kStages];
+    uint64_t freeb[kStages];
+    uint64_t s_full[2];
+    uint64_t pv_done[2];
+    uint64_t p_ready[2];
+    uint64_t fin;
+    uint32_t mask[kStages][4];      // gathered tiles: valid rows of the stage
+    uint32_t tmem_base;
+    int abort;
+};
+
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + 2 * kTileBytes /*Q*/ + 2 * kTileBytes /*P*/ +
+                              kStages * kTileBytes + sizeof(Ctrl);
+
+struct TcParams {
+    const int* idx;            // sparse: [B, n, topk]
+    int topk;
+    const int* n_entries;      // dense
+    int m;
+    int dense;
+    int B, n, N_cap, L_raw, window;
+    float scale_log2;          // softmax scale * log2(e)
+    __nv_bfloat16* out;
+    float* lse;
+    uint32_t* err;
+};
+
+struct Geometry {
+    int Tc;        // compressed tiles per M tile
+    int Tw;        // window tiles
+    int T;         // tiles per M tile
+    int bn_c_last; // N of the last compressed tile
+    int bn_w_last;
+    int p_lo;      // first window position
+    int Lw;
+    int Vmax;      // dense: entries needed by the CTA's last token
+};
+
+__device__ __forceinline__ int round16(int v) { return (v + 15) & ~15; }
+
+// 2^x with the MUFU instruction (ex2.approx of -inf is +0).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ Geometry geometry(const TcParams& p, int b, int t0) {
+    Geometry g;
+    const int t_last = min(t0 + kTokens - 1, p.n - 1);
+    if (p.dense) {
+        const int ne = clampi(p.n_entries ? p.n_entries[b] : p.N_cap, 0, p.N_cap);
+        g.Vmax = min((t_last + 1) / p.m, ne);
+        g.Tc = (g.Vmax + kBN - 1) / kBN;
+        g.bn_c_last = g.Tc ? round16(g.Vmax - (g.Tc - 1) * kBN) : 0;
+    } else {
+        g.Vmax = 0;
+        const int cc = (p.topk + kBN - 1) / kBN;
+        g.Tc = 2 * cc;
+        g.bn_c_last = p.topk ? round16(p.topk - (cc - 1) * kBN) : 0;
+    }
+    if (p.window > 0) {
+        g.p_lo = max(0, t0 - p.window + 1);
+        const int p_hi = min(t_last, p.L_raw - 1);
+        g.Lw = max(0, p_hi - g.p_lo + 1);
+    } else {
+        g.p_lo = 0;
+        g.Lw = 0;
+    }
+    g.Tw = (g.Lw + kBN - 1) / kBN;
+    g.bn_w_last = g.Tw ? round16(g.Lw - (g.Tw - 1) * kBN) : 0;
+    g.T = g.Tc + g.Tw;
+    return g;
+}
+
+// Tile j of M tile mt: which load carries it, and its N size.
+struct TileRef {
+    int load;
+    int bn;
+    int kind;   // 0 gathered (sparse compressed), 1 dense prefix, 2 window
+    int token;  // gathered: token (0/1) of the M tile the rows belong to
+    int chunk;  // gathered: chunk of the token's index row; contiguous: tile index in segment
+    bool last_consumer;
+};
+
+__device__ __forceinline__ TileRef tile_ref(const TcParams& p, const Geometry& g, int mt, int j) {
+    TileRef r;
+    if (j < g.Tc) {
+        if (p.dense) {
+            r.load = j;
+            r.kind = 1;
+            r.chunk = j;
+            r.token = 0;
+            r.bn = (j == g.Tc - 1) ? g.bn_c_last : kBN;
+            r.last_consumer = (mt == 1);
+        } else {
+            const int cc = g.Tc / 2;
+            r.load = 2 * j + mt;
+            r.kind = 0;
+            r.token = j / cc;
+            r.chunk = j % cc;
+            r.bn = (r.chunk == cc - 1) ? g.bn_c_last : kBN;
+            r.last_consumer = true;
+        }
+    } else {
+        const int jw = j - g.Tc;
+        r.load = (p.dense ? g.Tc : 2 * g.Tc) + jw;
+        r.kind = 2;
+        r.token = 0;
+        r.chunk = jw;
+        r.bn = (jw == g.Tw - 1) ? g.bn_w_last : kBN;
+        r.last_consumer = (mt == 1);
+    }
+    return r;
+}
+
+__device__ __forceinline__ int total_loads(const TcParams& p, const Geometry& g) {
+    return (p.dense ? g.Tc : 2 * g.Tc) + g.Tw;
+}
+
+__global__ void __launch_bounds__(kThreads, 1)
+attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_c,
+               const __grid_constant__ CUtensorMap tm_w, TcParams p) {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sQ = base;                                  // [2][32 KB]
+    uint8_t* sP = sQ + 2 * kTileBytes;                   // [2][32 KB]
+    uint8_t* sK = sP + 2 * kTileBytes;                   // [kStages][32 KB]
+    Ctrl* ctl = reinterpret_cast<Ctrl*>(sK + kStages * kTileBytes);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tiles_per_seq = (p.n + kTokens - 1) / kTokens;
+    const int b = blockIdx.x / tiles_per_seq;
+    const int t0 = (blockIdx.x - b * tiles_per_seq) * kTokens;
+    const Geometry g = geometry(p, b, t0);
+    volatile int* abort = &ctl->abort;
+
+    if (threadIdx.x == 0) {
+        mbar_init(&ctl->bar_q, 1);
+        for (int s = 0; s < kStages; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->freeb[s], 1);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&ctl->s_full[i], 1);
+            mbar_init(&ctl->pv_done[i], 1);
+            mbar_init(&ctl->p_ready[i], kRows);
+        }
+        mbar_init(&ctl->fin, 1);
+        // a CTA started after another one timed out does no work
+        ctl->abort = (*reinterpret_cast<volatile uint32_t*>(p.err) != 0u) ? 1 : 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&ctl->tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+
+    if (warp == 0) {
+        // ------------------------------------------------------------ producer
+        if (lane == 0) {
+            prefetch_tmap(&tm_q);
+            prefetch_tmap(&tm_c);
+            prefetch_tmap(&tm_w);
+            mbar_arrive_expect_tx(&ctl->bar_q, 2 * kTileBytes);
+            const int qrow = (b * p.n + t0) * kH;
+            for (int mt = 0; mt < 2; ++mt)
+                for (int h = 0; h < 2; ++h)
+                    tma_load_2d(sQ + mt * kTileBytes + h * kHalf, &tm_q, h * 64, qrow + mt * kRows,
+                                &ctl->bar_q);
+        }
+        const int NL = total_loads(p, g);
+        int L = 0;
+        for (; L < NL; ++L) {
+            const int slot = L % kStages, use = L / kStages;
+            int okw = 1;
+            if (lane == 0 && use > 0) okw = mbar_wait(&ctl->freeb[slot], (use - 1) & 1, abort, p.err);
+            if (!__shfl_sync(0xffffffffu, okw, 0)) break;
+            uint8_t* dst = sK + slot * kTileBytes;
+            // which tile is load L?
+            int kind, token = 0, chunk;
+            const int nc = p.dense ? g.Tc : 2 * g.Tc;
+            if (L < nc) {
+                if (p.dense) { kind = 1; chunk = L; }
+                else {
+                    const int j = L >> 1, mt = L & 1, cc = g.Tc / 2;
+                    kind = 0;
+                    token = 2 * mt + j / cc;      // token within the CTA
+                    chunk = j % cc;
+                }
+            } else {
+                kind = 2;
+                chunk = L - nc;
+            }
+            if (kind == 0) {
+                const int t = t0 + token;
+                const int tq = min(t, p.n - 1);
+                const int* irow = p.idx + ((size_t)b * p.n + tq) * p.topk;
+                int rows[4];
+                uint32_t valid = 0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const int c = chunk * kBN + lane * 4 + i;
+                    int s = (c < p.topk) ? irow[c] : -1;
+                    const bool ok = (t < p.n) && s >= 0 && s < p.N_cap;
+                    rows[i] = b * p.N_cap + (ok ? s : 0);
+                    valid |= (ok ? 1u : 0u) << i;
+                }
+                // valid bit of row c = lane*4+i goes to mask word c/32, bit c%32
+                uint32_t w[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t mine = (lane >> 3) == q ? (valid << ((lane & 7) * 4)) : 0u;
+                    uint32_t acc = mine;
+                    for (int off = 16; off; off >>= 1) acc |= __shfl_xor_sync(0xffffffffu, acc, off);
+                    w[q] = acc;
+                }
+                if (lane == 0) {
+                    for (int q = 0; q < 4; ++q) ctl->mask[slot][q] = w[q];
+                    mbar_arrive_expect_tx(&ctl->full[slot], kTileBytes);
+                }
+                for (int l = 0; l < 32; ++l) {
+                    const int y0 = __shfl_sync(0xffffffffu, rows[0], l);
+                    const int y1 = __shfl_sync(0xffffffffu, rows[1], l);
+                    const int y2 = __shfl_sync(0xffffffffu, rows[2], l);
+                    const int y3 = __shfl_sync(0xffffffffu, rows[3], l);
+                    if (lane == 0)
+                        for (int h = 0; h < 2; ++h)
+                            tma_gather4(dst + h * kHalf + l * 4 * 128, &tm_c, h * 64, y0, y1, y2, y3,
+                                        &ctl->full[slot]);
+                }
+            } else if (lane == 0) {
+                const CUtensorMap* tm = (kind == 1) ? &tm_c : &tm_w;
+                const int row = (kind == 1) ? b * p.N_cap + chunk * kBN
+                                            : b * p.L_raw + g.p_lo + chunk * kBN;
+                mbar_arrive_expect_tx(&ctl->full[slot], kTileBytes);
+                for (int h = 0; h < 2; ++h)
+                    tma_load_2d(dst + h * kHalf, tm, h * 64, row, &ctl->full[slot]);
+            }
+            __syncwarp();
+        }
+        // drain: loads still in flight must land before the CTA exits
+        if (lane == 0)
+            for (int Lp = max(0, L - kStages); Lp < L; ++Lp) {
+                volatile int never = 0;
+                mbar_wait(&ctl->full[Lp % kStages], (Lp / kStages) & 1, &never, p.err);
+            }
+    } else if (warp == 1) {
+        // ------------------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            const uint32_t id_qk_full = idesc_bf16(kRows, kBN, false, false);
+            const uint32_t id_pv = idesc_bf16(kRows, kD, false, true);
+            bool ok = mbar_wait(&ctl->bar_q, 0, abort, p.err);
+            tc_fence_after();
+            auto issue_qk = [&](int mt, int j) -> bool {
+                const TileRef r = tile_ref(p, g, mt, j);
+                const int slot = r.load % kStages;
+                if (!mbar_wait(&ctl->full[slot], (r.load / kStages) & 1, abort, p.err)) return false;
+                tc_fence_after();
+                const uint32_t qa = smem_u32(sQ + mt * kTileBytes);
+                const uint32_t ka = smem_u32(sK + slot * kTileBytes);
+                const uint32_t idesc = (r.bn == kBN) ? id_qk_full : idesc_bf16(kRows, r.bn, false, false);
+#pragma unroll
+                for (int k = 0; k < kD / 16; ++k) {
+                    const uint32_t off = (k >> 2) * kHalf + (k & 3) * 32;
+                    mma_bf16_ss(tmem + mt * 128, sw128_desc(qa + off, 16, 1024),
+                                sw128_desc(ka + off, 16, 1024), idesc, k > 0);
+                }
+                mma_commit(&ctl->s_full[mt]);
+                return true;
+            };
+            if (ok && g.T > 0) ok = issue_qk(0, 0) && issue_qk(1, 0);
+            for (int j = 0; ok && j < g.T; ++j) {
+                for (int mt = 0; mt < 2 && ok; ++mt) {
+                    if (!mbar_wait(&ctl->p_ready[mt], j & 1, abort, p.err)) { ok = false; break; }
+                    tc_fence_after();
+                    const TileRef r = tile_ref(p, g, mt, j);
+                    const int slot = r.load % kStages;
+                    const uint32_t pa = smem_u32(sP + mt * kTileBytes);
+                    const uint32_t va = smem_u32(sK + slot * kTileBytes);
+                    for (int kk = 0; kk < r.bn / 16; ++kk) {
+                        const uint32_t aoff = (kk >> 2) * kHalf + (kk & 3) * 32;
+                        mma_bf16_ss(tmem + 256 + mt * 128, sw128_desc(pa + aoff, 16, 1024),
+                                    sw128_desc(va + kk * 2048, kHalf, 1024), id_pv,
+                                    (j > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&ctl->pv_done[mt]);
+                    if (r.last_consumer) mma_commit(&ctl->freeb[slot]);
+                    if (j + 1 < g.T) ok = issue_qk(mt, j + 1);
+                }
+            }
+            // every MMA issued must finish before TMEM is released
+            mma_commit(&ctl->fin);
+            volatile int never = 0;
+            mbar_wait(&ctl->fin, 0, &never, p.err);
+        }
+        __syncwarp();
+    } else if (warp >= 4) {
+        // ------------------------------------------------------------ softmax
+        const int mt = (warp - 4) >> 2;
+        const int r = threadIdx.x - 128 - mt * 128;          // row of the M tile
+        const int quarter = warp & 3;
+        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+        const int u = r >> 6;                                // token of the M tile
+        const int t = t0 + 2 * mt + u;                       // absolute position
+        const bool row_ok = t < p.n;
+        int Vt = 0;
+        if (p.dense && row_ok) {
+            const int ne = clampi(p.n_entries ? p.n_entries[b] : p.N_cap, 0, p.N_cap);
+            Vt = min((t + 1) / p.m, ne);
+        }
+        const int w_lo = t - p.window + 1;                   // window [w_lo, t]
+        float m_used = -INFINITY, l_run = 0.0f;
+        uint8_t* prow = sP + mt * kTileBytes + r * 128;
+        const uint32_t s_addr = tmem + lane_addr + mt * 128;
+        const uint32_t o_addr = tmem + lane_addr + 256 + mt * 128;
+        bool ok = true;
+        for (int j = 0; j < g.T && ok; ++j) {
+            const TileRef tr = tile_ref(p, g, mt, j);
+            // every wait is warp-collective: the TMEM loads below are .sync.aligned
+            if (!__all_sync(0xffffffffu, mbar_wait(&ctl->s_full[mt], j & 1, abort, p.err))) { ok = false; break; }
+            tc_fence_after();
+            // which columns are keys of this row?
+            int c_lo = 0, c_hi = -1;                         // contiguous tiles
+            uint32_t mw[4] = {0u, 0u, 0u, 0u};               // gathered tiles
+            bool gathered = false;
+            if (row_ok) {
+                if (tr.kind == 0) {
+                    if (tr.token == u) {
+                        const int slot = tr.load % kStages;
+                        // the producer wrote the mask before arming this stage
+                        if (!__all_sync(0xffffffffu, mbar_wait(&ctl->full[slot], (tr.load / kStages) & 1, abort, p.err))) { ok = false; break; }
+                        gathered = true;
+#pragma unroll
+                        for (int q = 0; q < 4; ++q) mw[q] = ctl->mask[slot][q];
+                        c_hi = tr.bn - 1;
+                    }
+                } else if (tr.kind == 1) {
+                    c_hi = min(tr.bn, Vt - tr.chunk * kBN) - 1;
+                } else {
+                    const int p0 = g.p_lo + tr.chunk * kBN;
+                    c_lo = max(0, w_lo - p0);
+                    c_hi = min(tr.bn, t - p0 + 1) - 1;
+                }
+            }
+            const bool any = __any_sync(0xffffffffu, c_hi >= c_lo);
+            // pass 1: row max of the valid (scaled) scores
+            float mx = -INFINITY;
+            if (any) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float sv[32];
+                    tmem_ld32(s_addr + q * 32, sv);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int c = q * 32 + i;
+                        bool v = c >= c_lo && c <= c_hi;
+                        if (gathered) v = v && ((mw[q] >> i) & 1u);
+                        if (v) mx = fmaxf(mx, sv[i] * p.scale_log2);
+                    }
+                }
+            }
+            float alpha = 1.0f;
+            bool rescale = false;
+            if (mx != -INFINITY) {
+                if (m_used == -INFINITY) {
+                    m_used = mx;
+                } else if (mx > m_used + kRescaleLog2) {
+                    alpha = ex2(m_used - mx);
+                    m_used = mx;
+                    rescale = true;
+                }
+            }
+            // P buffer free and O stable once the previous P.V has finished
+            if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(&ctl->pv_done[mt], (j - 1) & 1, abort, p.err))) { ok = false; break; }
+            if (__any_sync(0xffffffffu, rescale)) {
+                tc_fence_after();
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float ov[32];
+                    tmem_ld32(o_addr + q * 32, ov);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+                    tmem_st32(o_addr + q * 32, ov);
+                }
+                tmem_st_wait();
+            }
+            // pass 2: P = exp2(s*scale - m) in bf16 into the swizzled P tile
+            float psum = 0.0f;
+            const bool warp_keys = __any_sync(0xffffffffu, mx != -INFINITY);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t pk[16];
+                if (warp_keys) {
+                    float sv[32];
+                    tmem_ld32(s_addr + q * 32, sv);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        const int c = q * 32 + i;
+                        bool v0 = c >= c_lo && c <= c_hi, v1 = c + 1 >= c_lo && c + 1 <= c_hi;
+                        if (gathered) {
+                            v0 = v0 && ((mw[q] >> i) & 1u);
+                            v1 = v1 && ((mw[q] >> (i + 1)) & 1u);
+                        }
+                        v0 = v0 && mx != -INFINITY;
+                        v1 = v1 && mx != -INFINITY;
+                        const float p0 = v0 ? ex2(fmaf(sv[i], p.scale_log2, -m_used)) : 0.0f;
+                        const float p1 = v1 ? ex2(fmaf(sv[i + 1], p.scale_log2, -m_used)) : 0.0f;
+                        psum += p0 + p1;
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                        pk[i >> 1] = *reinterpret_cast<uint32_t*>(&h2);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) pk[i] = 0u;
+                }
+#pragma unroll
+                for (int c4 = 0; c4 < 4; ++c4) {
+                    const int ch = q * 4 + c4;                 // 16-byte chunk of the row
+                    const int half = ch >> 3, cidx = ch & 7;
+                    uint4 v = make_uint4(pk[c4 * 4 + 0], pk[c4 * 4 + 1], pk[c4 * 4 + 2], pk[c4 * 4 + 3]);
+                    *reinterpret_cast<uint4*>(prow + half * kHalf + ((cidx ^ (r & 7)) << 4)) = v;
+                }
+            }
+            l_run = l_run * alpha + psum;
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&ctl->p_ready[mt]);
+        }
+        // epilogue: O / l
+        bool fin_ok = ok && g.T > 0;
+        if (fin_ok) fin_ok = mbar_wait(&ctl->pv_done[mt], (g.T - 1) & 1, abort, p.err);
+        fin_ok = __all_sync(0xffffffffu, fin_ok);
+        if (fin_ok) {
+            tc_fence_after();
+            const float inv = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+            __nv_bfloat16* orow = p.out + ((size_t)(b * p.n + t) * kH + (r & 63)) * kD;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float ov[32];
+                tmem_ld32(o_addr + q * 32, ov);
+                tmem_ld_wait();
+                if (row_ok) {
+#pragma unroll
+                    for (int i = 0; i < 32; i += 8) {
+                        uint4 v;
+                        __nv_bfloat162 h0 = __floats2bfloat162_rn(ov[i] * inv, ov[i + 1] * inv);
+                        __nv_bfloat162 h1 = __floats2bfloat162_rn(ov[i + 2] * inv, ov[i + 3] * inv);
+                        __nv_bfloat162 h2 = __floats2bfloat162_rn(ov[i + 4] * inv, ov[i + 5] * inv);
+                        __nv_bfloat162 h3 = __floats2bfloat162_rn(ov[i + 6] * inv, ov[i + 7] * inv);
+                        v.x = *reinterpret_cast<uint32_t*>(&h0);
+                        v.y = *reinterpret_cast<uint32_t*>(&h1);
+                        v.z = *reinterpret_cast<uint32_t*>(&h2);
+                        v.w = *reinterpret_cast<uint32_t*>(&h3);
+                        *reinterpret_cast<uint4*>(orow + q * 32 + i) = v;
+                    }
+                }
+            }
+            if (row_ok && p.lse)
+                p.lse[(size_t)(b * p.n + t) * kH + (r & 63)] =
+                    l_run > 0.0f ? (m_used + log2f(l_run)) / kLog2e : -INFINITY;
+        } else if (row_ok && g.T == 0) {
+            // no key at all: o = 0, lse = -inf
+            __nv_bfloat16* orow = p.out + ((size_t)(b * p.n + t) * kH + (r & 63)) * kD;
+            for (int i = 0; i < kD; i += 8) *reinterpret_cast<uint4*>(orow + i) = make_uint4(0, 0, 0, 0);
+            if (p.lse) p.lse[(size_t)(b * p.n + t) * kH + (r & 63)] = -INFINITY;
+        }
+    }
+
+    // (the MMA issuer waited above for its final commit: no MMA is in flight)
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+// ---------------------------------------------------------------------- host
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* f = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+    return fn;
+}
+
+// 2D bf16 tensor [rows, 128] with a 128-byte-swizzled box of {64, box_rows}.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)kD, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)kD * 2};
+    cuuint32_t box[2] = {64, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+bool attention_tc_supported(const AttnArgs& a) {
+    return a.dt == DT_BF16 && a.H == kH && a.D == kD && a.q_pos == nullptr &&
+           a.raw_pos0 == nullptr && a.raw_len == nullptr && a.L_raw >= a.n_q && a.n_q > 0 &&
+           a.topk <= 2048;
+}
+
+cudaError_t launch_attention_tc(const AttnArgs& a, uint32_t* err, cudaStream_t s) {
+    CUtensorMap tm_q, tm_c, tm_w;
+    const uint64_t q_rows = (uint64_t)a.B * a.n_q * kH;
+    const uint64_t c_rows = (uint64_t)a.B * (a.N_cap > 0 ? a.N_cap : 1);
+    const uint64_t w_rows = (uint64_t)a.B * a.L_raw;
+    const void* kvc = a.kv_c ? a.kv_c : a.kv_raw;   // any valid address if there are no entries
+    if (!make_map(&tm_q, a.q, q_rows, 128) ||
+        !make_map(&tm_c, kvc, a.N_cap > 0 ? c_rows : w_rows, a.dense ? 128 : 1) ||
+        !make_map(&tm_w, a.kv_raw, w_rows, 128))
+        return cudaErrorInvalidValue;
+    TcParams p;
+    p.idx = a.idx;
+    p.topk = a.dense ? 0 : a.topk;
+    p.n_entries = a.n_entries;
+    p.m = a.m;
+    p.dense = a.dense;
+    p.B = a.B;
+    p.n = a.n_q;
+    p.N_cap = a.N_cap;
+    p.L_raw = a.L_raw;
+    p.window = a.window;
+    p.scale_log2 = a.scale * kLog2e;
+    p.out = static_cast<__nv_bfloat16*>(a.out);
+    p.lse = a.lse_out;
+    p.err = err;
+    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kSmemBytes);
+    if (e != cudaSuccess) return e;
+    const int tiles = (a.n_q + kTokens - 1) / kTokens;
+    attn_tc_kernel<<<(unsigned)(a.B * tiles), kThreads, kSmemBytes, s>>>(tm_q, tm_c, tm_w, p);
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace csa

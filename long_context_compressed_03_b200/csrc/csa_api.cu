@@ -14,6 +14,21 @@
 namespace csa {
 static std::atomic<unsigned long long> g_launches{0};
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+// One error word per device for kernels whose bounded waits expired.
+static __device__ uint32_t g_device_error;
+static uint32_t* g_error_ptr[64];
+
+uint32_t* device_error_word() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (!g_error_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+        g_error_ptr[dev] = static_cast<uint32_t*>(p);
+    }
+    return g_error_ptr[dev];
+}
 }  // namespace csa
 
 namespace {
@@ -73,6 +88,24 @@ const char* csa_last_error_detail(void) { return g_detail; }
 int csa_version(void) { return 100; }
 
 unsigned long long csa_kernel_launches(void) { return csa::g_launches.load(); }
+
+csa_status_t csa_check_device_error(void* stream, int clear) {
+    uint32_t* p = csa::device_error_word();
+    if (!p) return fail(CSA_ERR_CUDA, "csa_check_device_error: no device error word");
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    uint32_t v = 0;
+    cudaError_t e = cudaMemcpyAsync(&v, p, sizeof v, cudaMemcpyDeviceToHost, s);
+    if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+    if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_check_device_error: %s", cudaGetErrorString(e));
+    if (clear && v) {
+        const uint32_t zero = 0;
+        e = cudaMemcpyAsync(p, &zero, sizeof zero, cudaMemcpyHostToDevice, s);
+        if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+        if (e != cudaSuccess) return fail(CSA_ERR_CUDA, "csa_check_device_error: %s", cudaGetErrorString(e));
+    }
+    if (v) return fail(CSA_ERR_TIMEOUT, "a device-side wait exceeded its time limit (code %u)", v);
+    return ok();
+}
 
 csa_status_t csa_compress(const void* x, int x_dt, int B, int n, int d_in, const void* W,
                           int d_out, int m, int overlap, void* out, int out_dt,

@@ -39,6 +39,14 @@ struct AttnArgs {
     void* out; float* lse_out;
 };
 
+// Device address of this library's error word on the current device (set by
+// kernels whose bounded waits expired; read back by csa_check_device_error).
+uint32_t* device_error_word();
+
+// tcgen05 prefill attention (64 heads x 128, bf16, positions 0..n-1).
+bool attention_tc_supported(const AttnArgs& a);
+cudaError_t launch_attention_tc(const AttnArgs& a, uint32_t* err, cudaStream_t s);
+
 // Counts one kernel launch (read back through csa_kernel_launches()).
 void count_launch();
 
