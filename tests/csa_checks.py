@@ -2,7 +2,10 @@
 
 Tolerances (stated once, used by every parity test):
   * attention / compression outputs, max-abs against the fp64 oracle:
-    2e-2 for bf16 paths, 1e-4 for fp32 paths;
+    2e-2 for bf16 paths, 1e-4 for fp32 paths; a bf16-stored output may in
+    addition carry its own storage rounding, at most 2^-8 |ref| (half an
+    ulp, rounded up): above |ref| ~ 8 no bf16 value lies within 2e-2 of the
+    exact result, so the 2e-2 budget is applied on top of that rounding;
   * bf16-stored compression outputs additionally within one bf16 ulp:
     |gpu - ref| <= 2^-8 |ref| + 1e-5;
   * top-k index sets: identical except where the oracle's k-th and (k+1)-th
@@ -76,6 +79,24 @@ def check_topk(gpu_idx: np.ndarray, scores: np.ndarray, k: int) -> dict:
             assert np.all(np.isin(must, chosen)), f"row {r}: near-tie row misses a clear winner"
             assert np.all(s[chosen] >= sk1 - delta), f"row {r}: near-tie row chose a clear loser"
     return dict(rows=R, exact=exact, near_ties=near)
+
+
+def excess_bf16(got: np.ndarray, ref: np.ndarray) -> float:
+    """max over elements of |got - ref| - 2^-8 |ref| (storage rounding of a
+    bf16 output removed); compare with ATOL_BF16."""
+    if got.size == 0:
+        return 0.0
+    return float(np.max(np.abs(got - ref) - np.abs(ref) * 2.0 ** -8))
+
+
+def check_out(got: np.ndarray, ref: np.ndarray, dtype) -> None:
+    """Output tolerance for a kernel result stored in `dtype`."""
+    if dtype == torch.float32:
+        err = max_abs(got, ref)
+        assert err <= ATOL_F32, f"max abs error {err} > {ATOL_F32}"
+    else:
+        err = excess_bf16(got, ref)
+        assert err <= ATOL_BF16, f"error beyond bf16 storage rounding {err} > {ATOL_BF16}"
 
 
 def max_abs(a: np.ndarray, b: np.ndarray) -> float:

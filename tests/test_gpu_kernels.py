@@ -8,7 +8,7 @@ import pytest
 import torch
 
 import oracle
-from csa_checks import ATOL_BF16, ATOL_F32, atol_for, check_topk, max_abs, np64
+from csa_checks import ATOL_BF16, ATOL_F32, check_out, check_topk, max_abs, np64
 from long_context_compressed_03_b200 import api
 
 pytestmark = pytest.mark.gpu
@@ -215,7 +215,7 @@ def test_sparse_attention_matches_oracle(dt, H, D):
     out, lse = api.sparse_attn(q.to(DEV), kv_c.to(DEV), torch.from_numpy(idx).to(DEV),
                                kv.to(DEV), W, with_lse=True)
     ro, rl = oracle.sparse_attn(np64(q), np64(kv_c), idx, np64(kv), W)
-    assert max_abs(np64(out).reshape(ro.shape), ro) <= atol_for(dt)
+    check_out(np64(out).reshape(ro.shape), ro, dt)
     np.testing.assert_allclose(lse.cpu().numpy().reshape(rl.shape), rl, atol=1e-3)
 
 
@@ -231,7 +231,7 @@ def test_hca_attention_matches_oracle(m, W, n):
     empty = np.isneginf(rl)
     assert np.all(got_o[empty.all(axis=1)] == 0.0)
     assert np.array_equal(np.isneginf(got_l), empty)
-    assert max_abs(got_o, ro) <= ATOL_BF16
+    check_out(got_o, ro, torch.bfloat16)
     np.testing.assert_allclose(got_l[~empty], rl[~empty], atol=1e-3)
 
 
@@ -252,7 +252,7 @@ def test_decode_caches_with_partial_swa_and_entry_counts():
                                raw_pos0=T(raw_pos0), raw_len=T(raw_len), q_pos=T(q_pos))
     ro, rl = oracle.sparse_attn(np64(q), np64(kv_c), idx, np64(swa), W, q_pos=q_pos,
                                 raw_pos0=raw_pos0, raw_len=raw_len)
-    assert max_abs(np64(out).reshape(ro.shape), ro) <= ATOL_BF16
+    check_out(np64(out).reshape(ro.shape), ro, torch.bfloat16)
     np.testing.assert_allclose(lse.cpu().numpy().reshape(rl.shape), rl, atol=1e-3)
     # HCA over the same caches
     out2, lse2 = api.hca_attn(q.to(DEV), kv_c.to(DEV), 4, swa.to(DEV), W, with_lse=True,
@@ -260,7 +260,7 @@ def test_decode_caches_with_partial_swa_and_entry_counts():
                               q_pos=T(q_pos))
     ro2, rl2 = oracle.hca_attn(np64(q), np64(kv_c), 4, np64(swa), W, n_entries=ne, q_pos=q_pos,
                                raw_pos0=raw_pos0, raw_len=raw_len)
-    assert max_abs(np64(out2).reshape(ro2.shape), ro2) <= ATOL_BF16
+    check_out(np64(out2).reshape(ro2.shape), ro2, torch.bfloat16)
 
 
 def test_window_only_and_explicit_scale():
@@ -269,7 +269,7 @@ def test_window_only_and_explicit_scale():
     out = api.sparse_attn(q.to(DEV), kv_c.to(DEV), None, kv.to(DEV), W, softmax_scale=0.3)
     ro, _ = oracle.sparse_attn(np64(q), np64(kv_c), np.zeros((B, n, 0), np.int32), np64(kv), W,
                                scale=0.3)
-    assert max_abs(np64(out).reshape(ro.shape), ro) <= ATOL_F32
+    check_out(np64(out).reshape(ro.shape), ro, torch.float32)
 
 
 def test_attention_is_deterministic():
