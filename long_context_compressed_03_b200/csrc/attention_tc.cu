@@ -22,9 +22,11 @@
 // TMEM: S0 [cols 0,128), S1 [128,256), O0 [256,384), O1 [384,512).
 // S = Q K^T (M=128, N<=128, K=128 in 8 steps), P = exp2(S*scale*log2e - m)
 // in bf16 written to swizzled shared memory, O += P V with V the same
-// shared tile read as an MN-major operand.  The running max is only raised
-// (and O rescaled in TMEM) when it grows by more than 2^8, so most tiles need
-// no rescale; the final division by the running sum is exact.
+// shared tile read as an MN-major operand.  The running sum adds the
+// bf16-rounded weights the MMA actually multiplies, so the result is an
+// exact convex combination of the keys under those weights.  The running max
+// is only raised (and O rescaled in TMEM) when it grows by more than 2^8, so
+// most tiles need no rescale; the final division by the running sum is exact.
 #include <cudaTypedefs.h>
 
 #include <math.h>
@@ -467,9 +469,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         v1 = v1 && mx != -INFINITY;
                         const float p0 = v0 ? ex2(fmaf(sv[i], p.scale_log2, -m_used)) : 0.0f;
                         const float p1 = v1 ? ex2(fmaf(sv[i + 1], p.scale_log2, -m_used)) : 0.0f;
-                        psum += p0 + p1;
                         __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
                         pk[i >> 1] = *reinterpret_cast<uint32_t*>(&h2);
+                        // the sum uses the rounded weights the MMA multiplies
+                        const float2 pr = __bfloat1622float2(h2);
+                        psum += pr.x + pr.y;
                     }
                 } else {
 #pragma unroll
