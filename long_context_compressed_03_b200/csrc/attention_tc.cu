@@ -52,6 +52,7 @@ constexpr int kTileBytes = 32768;   // 128 rows x 128 bf16
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
 
+
 struct __align__(8) Ctrl {
     uint64_t bar_q;
     uint64_t full[kStages];
@@ -82,6 +83,7 @@ struct TcParams {
 };
 
 struct Geometry {
+    int cc;        // sparse: chunks of 128 in a token's index row
     int Tc;        // compressed tiles per M tile
     int Tw;        // window tiles
     int T;         // tiles per M tile
@@ -107,11 +109,13 @@ __device__ __forceinline__ Geometry geometry(const TcParams& p, int b, int t0) {
     if (p.dense) {
         const int ne = clampi(p.n_entries ? p.n_entries[b] : p.N_cap, 0, p.N_cap);
         g.Vmax = min((t_last + 1) / p.m, ne);
+        g.cc = 0;
         g.Tc = (g.Vmax + kBN - 1) / kBN;
         g.bn_c_last = g.Tc ? round16(g.Vmax - (g.Tc - 1) * kBN) : 0;
     } else {
         g.Vmax = 0;
         const int cc = (p.topk + kBN - 1) / kBN;
+        g.cc = cc;
         g.Tc = 2 * cc;
         g.bn_c_last = p.topk ? round16(p.topk - (cc - 1) * kBN) : 0;
     }
@@ -150,7 +154,7 @@ __device__ __forceinline__ TileRef tile_ref(const TcParams& p, const Geometry& g
             r.bn = (j == g.Tc - 1) ? g.bn_c_last : kBN;
             r.last_consumer = (mt == 1);
         } else {
-            const int cc = g.Tc / 2;
+            const int cc = g.cc;
             r.load = 2 * j + mt;
             r.kind = 0;
             r.token = j / cc;
@@ -172,6 +176,97 @@ __device__ __forceinline__ TileRef tile_ref(const TcParams& p, const Geometry& g
 
 __device__ __forceinline__ int total_loads(const TcParams& p, const Geometry& g) {
     return (p.dense ? g.Tc : 2 * g.Tc) + g.Tw;
+}
+
+// Valid-column bits of a 128-key tile for one row: columns [c_lo, c_hi]
+// intersected with the gathered-row mask gm.
+__device__ __forceinline__ void valid_bits(int c_lo, int c_hi, const uint32_t gm[4], uint32_t vm[4]) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int lo = max(c_lo - 32 * q, 0), hi = min(c_hi - 32 * q, 31);
+        vm[q] = (lo > hi) ? 0u : ((0xffffffffu >> (31 - hi)) & (0xffffffffu << lo)) & gm[q];
+    }
+}
+
+// Row max (base-2 scaled) of the valid columns of this thread's S row.
+__device__ __forceinline__ float tile_max(uint32_t s_addr, const uint32_t vm[4], float sl2) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        float sv[32];
+        tmem_ld32(s_addr + q * 32, sv);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const float z = ((vm[q] >> i) & 1u) ? sv[i] * sl2 : -INFINITY;
+            mx = fmaxf(mx, z);
+        }
+    }
+    return mx;
+}
+
+// P row = exp2(z - m) for the valid columns (0 elsewhere), written as bf16
+// into the swizzled P tile; accumulates the exact and the rounded sums and
+// returns the max of the valid z.  m = +inf writes an all-zero row.
+__device__ __forceinline__ float tile_exp(uint32_t s_addr, uint8_t* prow, int r, const uint32_t vm[4],
+                                          float sl2, float m, float& se, float& sr) {
+    float mx = -INFINITY;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        float sv[32];
+        tmem_ld32(s_addr + q * 32, sv);
+#pragma unroll
+        for (int i = 0; i < 32; i += 8) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) {
+                const float z0 = ((vm[q] >> (i + e)) & 1u) ? sv[i + e] * sl2 : -INFINITY;
+                const float z1 = ((vm[q] >> (i + e + 1)) & 1u) ? sv[i + e + 1] * sl2 : -INFINITY;
+                mx = fmaxf(mx, fmaxf(z0, z1));
+                const float p0 = ex2(z0 - m), p1 = ex2(z1 - m);
+                __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                pk[e >> 1] = *reinterpret_cast<uint32_t*>(&h2);
+                const float2 pr = __bfloat1622float2(h2);
+                se += p0 + p1;
+                sr += pr.x + pr.y;
+            }
+            const int ch = (q * 32 + i) >> 3;                    // 16-byte chunk of the row
+            *reinterpret_cast<uint4*>(prow + (ch >> 3) * kHalf + (((ch & 7) ^ (r & 7)) << 4)) =
+                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        }
+    }
+    return mx;
+}
+
+// Rare path: a score exceeded the running max by more than 2^8.  Raise the
+// max, rescale the sums and O, and redo the tile's P row.
+__device__ __noinline__ void raise_and_redo(uint32_t s_addr, uint32_t o_addr, uint8_t* prow, int r,
+                                            uint32_t v0, uint32_t v1, uint32_t v2, uint32_t v3,
+                                            float sl2, float mx, bool raise, bool rescale_o,
+                                            float* m_used, float* l_r, float* l_e, float* se,
+                                            float* sr) {
+    float alpha = 1.0f;
+    if (raise) {
+        alpha = (*m_used == -INFINITY) ? 0.0f : ex2(*m_used - mx);
+        *m_used = mx;
+        *l_r *= alpha;
+        *l_e *= alpha;
+    }
+    if (rescale_o) {
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+            float ov[32];
+            tmem_ld32(o_addr + q * 32, ov);
+#pragma unroll
+            for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+            tmem_st32(o_addr + q * 32, ov);
+        }
+        tmem_st_wait();
+    }
+    const uint32_t vm[4] = {v0, v1, v2, v3};
+    float e = 0.0f, rr = 0.0f;
+    tile_exp(s_addr, prow, r, vm, sl2, (*m_used == -INFINITY) ? INFINITY : *m_used, e, rr);
+    *se = e;
+    *sr = rr;
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -230,51 +325,57 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                                 &ctl->bar_q);
         }
         const int NL = total_loads(p, g);
+        const int nc = p.dense ? g.Tc : 2 * g.Tc;
         int L = 0;
         for (; L < NL; ++L) {
             const int slot = L % kStages, use = L / kStages;
-            int okw = 1;
-            if (lane == 0 && use > 0) okw = mbar_wait(&ctl->freeb[slot], (use - 1) & 1, abort, p.err);
-            if (!__shfl_sync(0xffffffffu, okw, 0)) break;
             uint8_t* dst = sK + slot * kTileBytes;
             // which tile is load L?
             int kind, token = 0, chunk;
-            const int nc = p.dense ? g.Tc : 2 * g.Tc;
             if (L < nc) {
                 if (p.dense) { kind = 1; chunk = L; }
                 else {
-                    const int j = L >> 1, mt = L & 1, cc = g.Tc / 2;
+                    const int j = L >> 1, mt = L & 1;
                     kind = 0;
-                    token = 2 * mt + j / cc;      // token within the CTA
-                    chunk = j % cc;
+                    token = 2 * mt + j / g.cc;    // token within the CTA
+                    chunk = j - (j / g.cc) * g.cc;
                 }
             } else {
                 kind = 2;
                 chunk = L - nc;
             }
+            // gathered tiles: read the index row before waiting for the slot
+            int rows[4] = {0, 0, 0, 0};
+            uint32_t w[4] = {0u, 0u, 0u, 0u};
             if (kind == 0) {
                 const int t = t0 + token;
                 const int tq = min(t, p.n - 1);
                 const int* irow = p.idx + ((size_t)b * p.n + tq) * p.topk;
-                int rows[4];
-                uint32_t valid = 0;
+                int sv[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) {
                     const int c = chunk * kBN + lane * 4 + i;
-                    int s = (c < p.topk) ? irow[c] : -1;
-                    const bool ok = (t < p.n) && s >= 0 && s < p.N_cap;
-                    rows[i] = b * p.N_cap + (ok ? s : 0);
+                    sv[i] = (c < p.topk) ? __ldg(irow + c) : -1;
+                }
+                uint32_t valid = 0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const bool ok = (t < p.n) && sv[i] >= 0 && sv[i] < p.N_cap;
+                    rows[i] = b * p.N_cap + (ok ? sv[i] : 0);
                     valid |= (ok ? 1u : 0u) << i;
                 }
                 // valid bit of row c = lane*4+i goes to mask word c/32, bit c%32
-                uint32_t w[4];
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
-                    const uint32_t mine = (lane >> 3) == q ? (valid << ((lane & 7) * 4)) : 0u;
-                    uint32_t acc = mine;
+                    uint32_t acc = (lane >> 3) == q ? (valid << ((lane & 7) * 4)) : 0u;
                     for (int off = 16; off; off >>= 1) acc |= __shfl_xor_sync(0xffffffffu, acc, off);
                     w[q] = acc;
                 }
+            }
+            int okw = 1;
+            if (lane == 0 && use > 0) okw = mbar_wait(&ctl->freeb[slot], (use - 1) & 1, abort, p.err);
+            if (!__shfl_sync(0xffffffffu, okw, 0)) break;
+            if (kind == 0) {
                 if (lane == 0) {
                     for (int q = 0; q < 4; ++q) ctl->mask[slot][q] = w[q];
                     mbar_arrive_expect_tx(&ctl->full[slot], kTileBytes);
@@ -370,27 +471,27 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             Vt = min((t + 1) / p.m, ne);
         }
         const int w_lo = t - p.window + 1;                   // window [w_lo, t]
-        float m_used = -INFINITY, l_run = 0.0f;
+        // m_used: running max (base 2); l_r: sum of the bf16-rounded weights
+        // (normalises O); l_e: sum of the unrounded weights (the lse output)
+        float m_used = -INFINITY, l_r = 0.0f, l_e = 0.0f;
         uint8_t* prow = sP + mt * kTileBytes + r * 128;
         const uint32_t s_addr = tmem + lane_addr + mt * 128;
         const uint32_t o_addr = tmem + lane_addr + 256 + mt * 128;
         bool ok = true;
         for (int j = 0; j < g.T && ok; ++j) {
             const TileRef tr = tile_ref(p, g, mt, j);
-            // every wait is warp-collective: the TMEM loads below are .sync.aligned
+            // every wait is warp-collective: the TMEM accesses below are .sync.aligned
             if (!__all_sync(0xffffffffu, mbar_wait(&ctl->s_full[mt], j & 1, abort, p.err))) { ok = false; break; }
             tc_fence_after();
             // which columns are keys of this row?
-            int c_lo = 0, c_hi = -1;                         // contiguous tiles
-            uint32_t mw[4] = {0u, 0u, 0u, 0u};               // gathered tiles
-            bool gathered = false;
+            int c_lo = 0, c_hi = -1;                         // contiguous range
+            uint32_t mw[4] = {~0u, ~0u, ~0u, ~0u};           // gathered tiles: valid rows
             if (row_ok) {
                 if (tr.kind == 0) {
                     if (tr.token == u) {
                         const int slot = tr.load % kStages;
                         // the producer wrote the mask before arming this stage
                         if (!__all_sync(0xffffffffu, mbar_wait(&ctl->full[slot], (tr.load / kStages) & 1, abort, p.err))) { ok = false; break; }
-                        gathered = true;
 #pragma unroll
                         for (int q = 0; q < 4; ++q) mw[q] = ctl->mask[slot][q];
                         c_hi = tr.bn - 1;
@@ -403,91 +504,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     c_hi = min(tr.bn, t - p0 + 1) - 1;
                 }
             }
-            const bool any = __any_sync(0xffffffffu, c_hi >= c_lo);
-            // pass 1: row max of the valid (scaled) scores
-            float mx = -INFINITY;
-            if (any) {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float sv[32];
-                    tmem_ld32(s_addr + q * 32, sv);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int c = q * 32 + i;
-                        bool v = c >= c_lo && c <= c_hi;
-                        if (gathered) v = v && ((mw[q] >> i) & 1u);
-                        if (v) mx = fmaxf(mx, sv[i] * p.scale_log2);
-                    }
-                }
-            }
-            float alpha = 1.0f;
-            bool rescale = false;
-            if (mx != -INFINITY) {
-                if (m_used == -INFINITY) {
-                    m_used = mx;
-                } else if (mx > m_used + kRescaleLog2) {
-                    alpha = ex2(m_used - mx);
-                    m_used = mx;
-                    rescale = true;
-                }
-            }
             // P buffer free and O stable once the previous P.V has finished
             if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(&ctl->pv_done[mt], (j - 1) & 1, abort, p.err))) { ok = false; break; }
-            if (__any_sync(0xffffffffu, rescale)) {
-                tc_fence_after();
+            uint32_t vm[4];
+            valid_bits(c_lo, c_hi, mw, vm);
+            const bool has = (vm[0] | vm[1] | vm[2] | vm[3]) != 0u;
+            if (!__any_sync(0xffffffffu, has)) {
+                // no key of this tile is visible to any row of the warp: P = 0
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float ov[32];
-                    tmem_ld32(o_addr + q * 32, ov);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-                    tmem_st32(o_addr + q * 32, ov);
+                for (int ch = 0; ch < 16; ++ch)
+                    *reinterpret_cast<uint4*>(prow + (ch >> 3) * kHalf + (((ch & 7) ^ (r & 7)) << 4)) =
+                        make_uint4(0u, 0u, 0u, 0u);
+            } else {
+                // a row's first keys set its running max
+                if (__any_sync(0xffffffffu, has && m_used == -INFINITY)) {
+                    const float mx0 = tile_max(s_addr, vm, p.scale_log2);
+                    if (m_used == -INFINITY) m_used = mx0;
                 }
-                tmem_st_wait();
+                // P = exp2(z - m_used); m_used = -inf only for rows without keys
+                float se = 0.0f, sr = 0.0f;
+                const float m_eff = (m_used == -INFINITY) ? INFINITY : m_used;
+                const float mx = tile_exp(s_addr, prow, r, vm, p.scale_log2, m_eff, se, sr);
+                const bool raise = mx > m_used + kRescaleLog2;
+                if (__any_sync(0xffffffffu, raise))
+                    raise_and_redo(s_addr, o_addr, prow, r, vm[0], vm[1], vm[2], vm[3], p.scale_log2,
+                                   mx, raise, j > 0, &m_used, &l_r, &l_e, &se, &sr);
+                l_r += sr;
+                l_e += se;
             }
-            // pass 2: P = exp2(s*scale - m) in bf16 into the swizzled P tile
-            float psum = 0.0f;
-            const bool warp_keys = __any_sync(0xffffffffu, mx != -INFINITY);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t pk[16];
-                if (warp_keys) {
-                    float sv[32];
-                    tmem_ld32(s_addr + q * 32, sv);
-                    tmem_ld_wait();
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        const int c = q * 32 + i;
-                        bool v0 = c >= c_lo && c <= c_hi, v1 = c + 1 >= c_lo && c + 1 <= c_hi;
-                        if (gathered) {
-                            v0 = v0 && ((mw[q] >> i) & 1u);
-                            v1 = v1 && ((mw[q] >> (i + 1)) & 1u);
-                        }
-                        v0 = v0 && mx != -INFINITY;
-                        v1 = v1 && mx != -INFINITY;
-                        const float p0 = v0 ? ex2(fmaf(sv[i], p.scale_log2, -m_used)) : 0.0f;
-                        const float p1 = v1 ? ex2(fmaf(sv[i + 1], p.scale_log2, -m_used)) : 0.0f;
-                        __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                        pk[i >> 1] = *reinterpret_cast<uint32_t*>(&h2);
-                        // the sum uses the rounded weights the MMA multiplies
-                        const float2 pr = __bfloat1622float2(h2);
-                        psum += pr.x + pr.y;
-                    }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) pk[i] = 0u;
-                }
-#pragma unroll
-                for (int c4 = 0; c4 < 4; ++c4) {
-                    const int ch = q * 4 + c4;                 // 16-byte chunk of the row
-                    const int half = ch >> 3, cidx = ch & 7;
-                    uint4 v = make_uint4(pk[c4 * 4 + 0], pk[c4 * 4 + 1], pk[c4 * 4 + 2], pk[c4 * 4 + 3]);
-                    *reinterpret_cast<uint4*>(prow + half * kHalf + ((cidx ^ (r & 7)) << 4)) = v;
-                }
-            }
-            l_run = l_run * alpha + psum;
             fence_proxy_async_smem();
             tc_fence_before();
             mbar_arrive(&ctl->p_ready[mt]);
@@ -498,13 +542,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         fin_ok = __all_sync(0xffffffffu, fin_ok);
         if (fin_ok) {
             tc_fence_after();
-            const float inv = l_run > 0.0f ? 1.0f / l_run : 0.0f;
+            const float inv = l_r > 0.0f ? 1.0f / l_r : 0.0f;
             __nv_bfloat16* orow = p.out + ((size_t)(b * p.n + t) * kH + (r & 63)) * kD;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 float ov[32];
                 tmem_ld32(o_addr + q * 32, ov);
-                tmem_ld_wait();
                 if (row_ok) {
 #pragma unroll
                     for (int i = 0; i < 32; i += 8) {
@@ -523,7 +566,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             if (row_ok && p.lse)
                 p.lse[(size_t)(b * p.n + t) * kH + (r & 63)] =
-                    l_run > 0.0f ? (m_used + log2f(l_run)) / kLog2e : -INFINITY;
+                    l_e > 0.0f ? (m_used + log2f(l_e)) / kLog2e : -INFINITY;
         } else if (row_ok && g.T == 0) {
             // no key at all: o = 0, lse = -inf
             __nv_bfloat16* orow = p.out + ((size_t)(b * p.n + t) * kH + (r & 63)) * kD;
