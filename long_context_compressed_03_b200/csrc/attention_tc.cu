@@ -17,12 +17,13 @@
 //     with TMA row gathers (4 rows per instruction) straight into the
 //     128-byte-swizzled layout the tensor core reads, and the rows of the
 //     other token in the M tile are masked.
-// Roles (12 warps): warp 0 issues TMA, warp 1 allocates TMEM and one lane
-// issues every MMA, warps 4-7 / 8-11 run the softmax of M tile 0 / 1.
+// Roles (10 warps): warp 0 issues TMA, warp 1 allocates TMEM and one lane
+// issues every MMA, warps 2-5 / 6-9 run the softmax of M tile 0 / 1 (a warp
+// reaches TMEM lanes 32*(warp%4) .. +31, so each group covers all 128 rows).
 // TMEM: S0 [cols 0,128), S1 [128,256), O0 [256,384), O1 [384,512).
 // S = Q K^T (M=128, N<=128, K=128 in 8 steps), P = exp2(S*scale*log2e - m)
-// in bf16 written to swizzled shared memory, O += P V with V the same
-// shared tile read as an MN-major operand.  The running sum adds the
+// in bf16 written back into the first 64 columns of S, O += P V with P read
+// from tensor memory and V the same shared tile read as an MN-major operand.  The running sum adds the
 // bf16-rounded weights the MMA actually multiplies, so the result is an
 // exact convex combination of the keys under those weights.  The running max
 // is only raised (and O rescaled in TMEM) when it grows by more than 2^8, so
@@ -45,8 +46,8 @@ constexpr int kD = 128;
 constexpr int kRows = 128;          // rows of an M tile
 constexpr int kTokens = 4;          // tokens per CTA
 constexpr int kBN = 128;            // keys per tile
-constexpr int kStages = 3;
-constexpr int kThreads = 384;
+constexpr int kStages = 5;
+constexpr int kThreads = 320;
 constexpr int kHalf = 16384;        // one 64-column half of a 128-row tile
 constexpr int kTileBytes = 32768;   // 128 rows x 128 bf16
 constexpr float kLog2e = 1.4426950408889634f;
@@ -66,7 +67,7 @@ struct __align__(8) Ctrl {
     int abort;
 };
 
-constexpr size_t kSmemBytes = 1024 /*align slack*/ + 2 * kTileBytes /*Q*/ + 2 * kTileBytes /*P*/ +
+constexpr size_t kSmemBytes = 1024 /*align slack*/ + 2 * kTileBytes /*Q*/ +
                               kStages * kTileBytes + sizeof(Ctrl);
 
 struct TcParams {
@@ -191,82 +192,62 @@ __device__ __forceinline__ void valid_bits(int c_lo, int c_hi, const uint32_t gm
 // Row max (base-2 scaled) of the valid columns of this thread's S row.
 __device__ __forceinline__ float tile_max(uint32_t s_addr, const uint32_t vm[4], float sl2) {
     float mx = -INFINITY;
-#pragma unroll
+#pragma unroll 1
     for (int q = 0; q < 4; ++q) {
+        const uint32_t mq = q == 0 ? vm[0] : (q == 1 ? vm[1] : (q == 2 ? vm[2] : vm[3]));
         float sv[32];
         tmem_ld32(s_addr + q * 32, sv);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
-            const float z = ((vm[q] >> i) & 1u) ? sv[i] * sl2 : -INFINITY;
+            const float z = ((mq >> i) & 1u) ? sv[i] * sl2 : -INFINITY;
             mx = fmaxf(mx, z);
         }
     }
     return mx;
 }
 
-// P row = exp2(z - m) for the valid columns (0 elsewhere), written as bf16
-// into the swizzled P tile; accumulates the exact and the rounded sums and
-// returns the max of the valid z.  m = +inf writes an all-zero row.
-__device__ __forceinline__ float tile_exp(uint32_t s_addr, uint8_t* prow, int r, const uint32_t vm[4],
-                                          float sl2, float m, float& se, float& sr) {
-    float mx = -INFINITY;
-#pragma unroll
+// P row = exp2(z - m) for the valid columns (0 elsewhere) as bf16 pairs,
+// written over the first 64 columns of S as it goes: chunk q reads S
+// columns [32q, 32q+32) and writes P columns [16q, 16q+16), which have
+// already been read.  Accumulates the exact and the rounded sums.
+// m = +inf writes an all-zero row.
+__device__ __forceinline__ void tile_exp(uint32_t s_addr, const uint32_t vm[4], float sl2, float m,
+                                         float& se, float& sr) {
+    // kept rolled: unrolling lets the compiler interleave chunks past the
+    // register budget
+#pragma unroll 1
     for (int q = 0; q < 4; ++q) {
+        const uint32_t mq = q == 0 ? vm[0] : (q == 1 ? vm[1] : (q == 2 ? vm[2] : vm[3]));
         float sv[32];
         tmem_ld32(s_addr + q * 32, sv);
+        uint32_t pk[16];
 #pragma unroll
-        for (int i = 0; i < 32; i += 8) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int e = 0; e < 8; e += 2) {
-                const float z0 = ((vm[q] >> (i + e)) & 1u) ? sv[i + e] * sl2 : -INFINITY;
-                const float z1 = ((vm[q] >> (i + e + 1)) & 1u) ? sv[i + e + 1] * sl2 : -INFINITY;
-                mx = fmaxf(mx, fmaxf(z0, z1));
-                const float p0 = ex2(z0 - m), p1 = ex2(z1 - m);
-                __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-                pk[e >> 1] = *reinterpret_cast<uint32_t*>(&h2);
-                const float2 pr = __bfloat1622float2(h2);
-                se += p0 + p1;
-                sr += pr.x + pr.y;
-            }
-            const int ch = (q * 32 + i) >> 3;                    // 16-byte chunk of the row
-            *reinterpret_cast<uint4*>(prow + (ch >> 3) * kHalf + (((ch & 7) ^ (r & 7)) << 4)) =
-                make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        for (int e = 0; e < 32; e += 2) {
+            const float z0 = ((mq >> e) & 1u) ? sv[e] * sl2 : -INFINITY;
+            const float z1 = ((mq >> (e + 1)) & 1u) ? sv[e + 1] * sl2 : -INFINITY;
+            const float p0 = ex2(z0 - m), p1 = ex2(z1 - m);
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+            pk[e >> 1] = *reinterpret_cast<uint32_t*>(&h2);
+            const float2 pr = __bfloat1622float2(h2);
+            se += p0 + p1;
+            sr += pr.x + pr.y;
         }
+        tmem_st16(s_addr + q * 16, pk);
     }
-    return mx;
 }
 
-// Rare path: a score exceeded the running max by more than 2^8.  Raise the
-// max, rescale the sums and O, and redo the tile's P row.
-__device__ __noinline__ void raise_and_redo(uint32_t s_addr, uint32_t o_addr, uint8_t* prow, int r,
-                                            uint32_t v0, uint32_t v1, uint32_t v2, uint32_t v3,
-                                            float sl2, float mx, bool raise, bool rescale_o,
-                                            float* m_used, float* l_r, float* l_e, float* se,
-                                            float* sr) {
-    float alpha = 1.0f;
-    if (raise) {
-        alpha = (*m_used == -INFINITY) ? 0.0f : ex2(*m_used - mx);
-        *m_used = mx;
-        *l_r *= alpha;
-        *l_e *= alpha;
-    }
-    if (rescale_o) {
+// The row max rose by more than 2^8 (or a row sees its first keys): rescale
+// the sums and O.  alpha = 0 for a row without earlier keys.
+__device__ __noinline__ void rescale_o(uint32_t o_addr, float alpha) {
 #pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-            float ov[32];
-            tmem_ld32(o_addr + q * 32, ov);
+    for (int q = 0; q < 4; ++q) {
+        float ov[32];
+        tmem_ld32(o_addr + q * 32, ov);
 #pragma unroll
-            for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-            tmem_st32(o_addr + q * 32, ov);
-        }
-        tmem_st_wait();
+        for (int i = 0; i < 32; ++i) ov[i] *= alpha;
+        tmem_st32(o_addr + q * 32, ov);
     }
-    const uint32_t vm[4] = {v0, v1, v2, v3};
-    float e = 0.0f, rr = 0.0f;
-    tile_exp(s_addr, prow, r, vm, sl2, (*m_used == -INFINITY) ? INFINITY : *m_used, e, rr);
-    *se = e;
-    *sr = rr;
+    tmem_st_wait();
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -275,8 +256,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = base;                                  // [2][32 KB]
-    uint8_t* sP = sQ + 2 * kTileBytes;                   // [2][32 KB]
-    uint8_t* sK = sP + 2 * kTileBytes;                   // [kStages][32 KB]
+    uint8_t* sK = sQ + 2 * kTileBytes;                   // [kStages][32 KB]
     Ctrl* ctl = reinterpret_cast<Ctrl*>(sK + kStages * kTileBytes);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -374,22 +354,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             }
             int okw = 1;
             if (lane == 0 && use > 0) okw = mbar_wait(&ctl->freeb[slot], (use - 1) & 1, abort, p.err);
+            // lane 0 acquired the free slot; __syncwarp orders the other lanes after it
+            __syncwarp();
             if (!__shfl_sync(0xffffffffu, okw, 0)) break;
             if (kind == 0) {
                 if (lane == 0) {
                     for (int q = 0; q < 4; ++q) ctl->mask[slot][q] = w[q];
                     mbar_arrive_expect_tx(&ctl->full[slot], kTileBytes);
                 }
-                for (int l = 0; l < 32; ++l) {
-                    const int y0 = __shfl_sync(0xffffffffu, rows[0], l);
-                    const int y1 = __shfl_sync(0xffffffffu, rows[1], l);
-                    const int y2 = __shfl_sync(0xffffffffu, rows[2], l);
-                    const int y3 = __shfl_sync(0xffffffffu, rows[3], l);
-                    if (lane == 0)
-                        for (int h = 0; h < 2; ++h)
-                            tma_gather4(dst + h * kHalf + l * 4 * 128, &tm_c, h * 64, y0, y1, y2, y3,
-                                        &ctl->full[slot]);
-                }
+                __syncwarp();
+                // every lane fetches its own four rows, both 64-column halves
+                for (int h = 0; h < 2; ++h)
+                    tma_gather4(dst + h * kHalf + lane * 4 * 128, &tm_c, h * 64, rows[0], rows[1],
+                                rows[2], rows[3], &ctl->full[slot]);
             } else if (lane == 0) {
                 const CUtensorMap* tm = (kind == 1) ? &tm_c : &tm_w;
                 const int row = (kind == 1) ? b * p.N_cap + chunk * kBN
@@ -437,14 +414,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     tc_fence_after();
                     const TileRef r = tile_ref(p, g, mt, j);
                     const int slot = r.load % kStages;
-                    const uint32_t pa = smem_u32(sP + mt * kTileBytes);
                     const uint32_t va = smem_u32(sK + slot * kTileBytes);
-                    for (int kk = 0; kk < r.bn / 16; ++kk) {
-                        const uint32_t aoff = (kk >> 2) * kHalf + (kk & 3) * 32;
-                        mma_bf16_ss(tmem + 256 + mt * 128, sw128_desc(pa + aoff, 16, 1024),
+                    // P (bf16, two per column) sits in the first 64 columns of S
+                    for (int kk = 0; kk < r.bn / 16; ++kk)
+                        mma_bf16_ts(tmem + 256 + mt * 128, tmem + mt * 128 + kk * 8,
                                     sw128_desc(va + kk * 2048, kHalf, 1024), id_pv,
                                     (j > 0 || kk > 0) ? 1u : 0u);
-                    }
                     mma_commit(&ctl->pv_done[mt]);
                     if (r.last_consumer) mma_commit(&ctl->freeb[slot]);
                     if (j + 1 < g.T) ok = issue_qk(mt, j + 1);
@@ -456,11 +431,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_wait(&ctl->fin, 0, &never, p.err);
         }
         __syncwarp();
-    } else if (warp >= 4) {
+    } else {
         // ------------------------------------------------------------ softmax
-        const int mt = (warp - 4) >> 2;
-        const int r = threadIdx.x - 128 - mt * 128;          // row of the M tile
+        const int mt = (warp - 2) >> 2;
         const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;                   // row of the M tile
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         const int u = r >> 6;                                // token of the M tile
         const int t = t0 + 2 * mt + u;                       // absolute position
@@ -474,7 +449,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // m_used: running max (base 2); l_r: sum of the bf16-rounded weights
         // (normalises O); l_e: sum of the unrounded weights (the lse output)
         float m_used = -INFINITY, l_r = 0.0f, l_e = 0.0f;
-        uint8_t* prow = sP + mt * kTileBytes + r * 128;
         const uint32_t s_addr = tmem + lane_addr + mt * 128;
         const uint32_t o_addr = tmem + lane_addr + 256 + mt * 128;
         bool ok = true;
@@ -509,30 +483,33 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             uint32_t vm[4];
             valid_bits(c_lo, c_hi, mw, vm);
             const bool has = (vm[0] | vm[1] | vm[2] | vm[3]) != 0u;
+            float se = 0.0f, sr = 0.0f;
             if (!__any_sync(0xffffffffu, has)) {
                 // no key of this tile is visible to any row of the warp: P = 0
+                uint32_t zero[16];
 #pragma unroll
-                for (int ch = 0; ch < 16; ++ch)
-                    *reinterpret_cast<uint4*>(prow + (ch >> 3) * kHalf + (((ch & 7) ^ (r & 7)) << 4)) =
-                        make_uint4(0u, 0u, 0u, 0u);
+                for (int i = 0; i < 16; ++i) zero[i] = 0u;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) tmem_st16(s_addr + q * 16, zero);
             } else {
-                // a row's first keys set its running max
-                if (__any_sync(0xffffffffu, has && m_used == -INFINITY)) {
-                    const float mx0 = tile_max(s_addr, vm, p.scale_log2);
-                    if (m_used == -INFINITY) m_used = mx0;
+                // pass 1: the tile's row max; raise the running max (and
+                // rescale O) when it grows by more than 2^8
+                const float mx = tile_max(s_addr, vm, p.scale_log2);
+                const bool raise = mx > m_used + kRescaleLog2;   // true for a row's first keys
+                float alpha = 1.0f;
+                if (raise) {
+                    alpha = (m_used == -INFINITY) ? 0.0f : ex2(m_used - mx);
+                    m_used = mx;
+                    l_r *= alpha;
+                    l_e *= alpha;
                 }
-                // P = exp2(z - m_used); m_used = -inf only for rows without keys
-                float se = 0.0f, sr = 0.0f;
-                const float m_eff = (m_used == -INFINITY) ? INFINITY : m_used;
-                const float mx = tile_exp(s_addr, prow, r, vm, p.scale_log2, m_eff, se, sr);
-                const bool raise = mx > m_used + kRescaleLog2;
-                if (__any_sync(0xffffffffu, raise))
-                    raise_and_redo(s_addr, o_addr, prow, r, vm[0], vm[1], vm[2], vm[3], p.scale_log2,
-                                   mx, raise, j > 0, &m_used, &l_r, &l_e, &se, &sr);
+                if (j > 0 && __any_sync(0xffffffffu, raise)) rescale_o(o_addr, alpha);
+                // pass 2: P = exp2(z - m_used) over S
+                tile_exp(s_addr, vm, p.scale_log2, (m_used == -INFINITY) ? INFINITY : m_used, se, sr);
                 l_r += sr;
                 l_e += se;
             }
-            fence_proxy_async_smem();
+            tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&ctl->p_ready[mt]);
         }
