@@ -1,0 +1,512 @@
+// indexer_tc.cu -- tensor-core Lightning-Indexer scores fused with an exact
+// per-query top-k (prefill: 128 consecutive queries of one sequence per CTA).
+//
+// score[t, s] = ks_s * sum_h qs_{t,h} * ReLU(q_{t,h} . k_s)   for s < V(t)
+// idx[t, :]   = the topk largest scores, equal scores lowest index first
+// ("百万上下文从「奢侈品」变「日用品」…" §3.2 indexer + top-k, §8.2 streaming
+//  selection without materialising the scores; "DS-V4 分析&学习" §4 low-
+//  precision indexer QK.)  fp8: q and k are E4M3 codes with per-row scales
+// qs, ks (the bf16 queries are quantised here, in fp32, exactly as the
+// compressor quantises a row); bf16: qs = ks = 1.
+//
+// Scores: for every chunk of 64 entries the MMA warp issues one tcgen05 MMA
+// per indexer head (M = 128 queries, N = 64 entries, K = 64) into TMEM;
+// two epilogue warpgroups take alternate chunks (TMEM: 2 buffers x 4 heads
+// x 64 columns).  Each epilogue thread owns one query row.
+//
+// Selection: every (row, entry) gets the unique 48-bit key
+//   K = (bits of the non-negative fp32 score) << 16 | (65535 - s),
+// which orders like (score desc, index asc) -- the top-k tie rule.  An
+// MSB-first radix select over 8-bit digits finds, per row, the digit prefix
+// that holds the k-th largest key: each pass recomputes the scores (the
+// tensor cores make that cheap) and histograms the next digit of the keys
+// that match the row's current prefix into per-row u16 bins in shared
+// memory ([bin][row] layout: conflict-free).  Once a row's boundary bin has
+// at most kCap keys, a final pass writes every key above the boundary to the
+// output and collects the boundary bin, which is then sorted exactly.  The
+// score matrix never leaves the SM.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc_common.cuh"
+
+namespace csa {
+namespace {
+
+using namespace tc;
+
+constexpr int kRows = 128;      // queries per CTA = MMA M
+constexpr int kN = 64;          // entries per chunk = MMA N
+constexpr int kHeads = 4;       // indexer heads held in TMEM
+constexpr int kDim = 64;        // indexer head dim = MMA K
+constexpr int kThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2-5 / 6-9 epilogue groups
+constexpr int kCap = 64;        // boundary-bin capacity per row
+constexpr int kLevels = 6;      // 48-bit key, 8-bit digits
+
+template <bool FP8>
+struct Cfg {
+    static constexpr int kElem = FP8 ? 1 : 2;
+    static constexpr int kRowBytes = kDim * kElem;                  // 64 / 128
+    static constexpr int kATile = kRows * kRowBytes;                // per head
+    static constexpr int kBTile = kN * kRowBytes;                   // per chunk
+    static constexpr int kStages = FP8 ? 4 : 3;
+    static constexpr int kKSteps = FP8 ? 2 : 4;                     // K=32 (fp8) / 16 (bf16)
+    static constexpr int kHist = 2 * 256 * kRows * 2;               // two groups, u16 bins
+    static constexpr size_t kSmem = 1024 + kHeads * kATile + kStages * kBTile + kHist + 8192;
+};
+
+struct IdxParams {
+    const void* qI;            // [B, n, H_I, 64] bf16 or e4m3 codes
+    const float* qI_scale;     // e4m3 queries given as codes: [B, n, H_I]
+    const float* kI_scale;     // e4m3 keys: [B, N_cap]
+    int q_mode;                // 0 bf16 (bf16 keys), 1 bf16 quantised here, 2 e4m3 codes
+    int B, n, H_I, N_cap, m, topk;
+    const int* n_entries;
+    int* idx_out;
+    uint32_t* err;
+};
+
+struct __align__(8) Ctrl {
+    uint64_t full[4];
+    uint64_t freeb[4];
+    uint64_t acc_full[2];
+    uint64_t acc_free[2];
+    uint64_t fin;
+    uint32_t tmem_base;
+    int abort;
+    int next_emit;             // 1: the next pass emits
+};
+
+// Per-row selection state (shared by both epilogue groups).
+struct RowState {
+    uint64_t prefix[kRows];    // key prefix above the current digit
+    int level[kRows];          // digit being histogrammed (or, when ready, the last one)
+    int rank[kRows];           // keys still needed from the prefix's bin
+    int ready[kRows];          // boundary bin small enough (or keys unique)
+    int V[kRows];              // visible entries (0 for rows beyond n)
+    int emitted[2][kRows];     // output slots used by each epilogue group
+    int listed[kRows];         // boundary keys collected
+    float qs[kRows][kHeads];   // per-head query scales
+};
+
+__device__ __forceinline__ int shift_of(int level) { return 40 - 8 * level; }
+
+// No-swizzle K-major layout for a [128 x kRowBytes] operand written by threads:
+// 8-row x 16-byte core matrices, LBO = 128 B between core matrices along K,
+// SBO = (kRowBytes/16) * 128 B between 8-row groups.
+template <int kRowBytes>
+__device__ __forceinline__ uint32_t a_offset(int r, int chunk16) {
+    return (uint32_t)((r >> 3) * (kRowBytes / 16) * 128 + chunk16 * 128 + (r & 7) * 16);
+}
+__device__ __forceinline__ uint64_t desc_noswizzle(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;
+    return d;   // layout type 0: no swizzle
+}
+__device__ __forceinline__ uint64_t desc_sw(uint32_t saddr, uint32_t sbo, uint32_t layout) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)1u << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+    d |= (uint64_t)1u << 46;
+    d |= (uint64_t)layout << 61;
+    return d;
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
+    uint32_t* r = reinterpret_cast<uint32_t*>(v);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr)
+        : "memory");
+}
+
+template <bool FP8>
+__global__ void __launch_bounds__(kThreads, 1)
+indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
+    using C = Cfg<FP8>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* sA = base;                                       // [kHeads][kATile]
+    uint8_t* sB = sA + kHeads * C::kATile;                    // [kStages][kBTile]
+    uint16_t* hist = reinterpret_cast<uint16_t*>(sB + C::kStages * C::kBTile);   // [2][256][128]
+    uint64_t* list = reinterpret_cast<uint64_t*>(hist);      // [128][kCap] (aliases hist)
+    RowState* rs = reinterpret_cast<RowState*>(reinterpret_cast<uint8_t*>(hist) + C::kHist);
+    Ctrl* ctl = reinterpret_cast<Ctrl*>(reinterpret_cast<uint8_t*>(rs) + sizeof(RowState));
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int tiles_per_seq = (p.n + kRows - 1) / kRows;
+    // heavy tiles (late queries see more entries) first
+    const int tile = gridDim.x - 1 - blockIdx.x;
+    const int b = tile / tiles_per_seq;
+    const int t0 = (tile - b * tiles_per_seq) * kRows;
+    const int ne = clampi(p.n_entries ? p.n_entries[b] : p.N_cap, 0, p.N_cap);
+    const int t_last = min(t0 + kRows - 1, p.n - 1);
+    const int Vmax = min((t_last + 1) / p.m, ne);
+    const int nchunks = (Vmax + kN - 1) / kN;
+    volatile int* abort = &ctl->abort;
+
+    // ---------------------------------------------------------------- setup
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < C::kStages; ++s) {
+            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->freeb[s], 1);
+        }
+        for (int g = 0; g < 2; ++g) {
+            mbar_init(&ctl->acc_full[g], 1);
+            mbar_init(&ctl->acc_free[g], kRows);
+        }
+        mbar_init(&ctl->fin, 1);
+        ctl->abort = (*reinterpret_cast<volatile uint32_t*>(p.err) != 0u) ? 1 : 0;
+        ctl->next_emit = 0;
+        fence_barrier_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&ctl->tmem_base, 512);
+        tmem_relinquish();
+    }
+    // rows: visibility and the query operand (one warp per (row, head) pair)
+    for (int r = threadIdx.x; r < kRows; r += kThreads) {
+        const int t = t0 + r;
+        const int V = (t < p.n) ? min((t + 1) / p.m, ne) : 0;
+        rs->V[r] = V;
+        rs->level[r] = 0;
+        rs->prefix[r] = 0;
+        rs->rank[r] = p.topk;
+        rs->ready[r] = (V <= p.topk) ? 1 : 0;   // rows with V <= k take every visible entry
+        rs->emitted[0][r] = 0;
+        rs->emitted[1][r] = 0;
+        rs->listed[r] = 0;
+    }
+    for (int pair = warp; pair < kRows * kHeads; pair += kThreads / 32) {
+        const int r = pair >> 2, h = pair & 3;
+        const int t = min(t0 + r, p.n - 1);
+        const size_t qrow = ((size_t)b * p.n + t) * p.H_I + h;
+        float v0 = 0.0f, v1 = 0.0f;   // elements 2*lane, 2*lane+1
+        float qs = 1.0f;
+        uint32_t packed;              // two output elements (fp8: 2 bytes; bf16: 4 bytes)
+        if (h < p.H_I) {
+            if (p.q_mode == 2) {
+                const uint8_t* src = static_cast<const uint8_t*>(p.qI) + qrow * kDim;
+                packed = (uint32_t)src[2 * lane] | ((uint32_t)src[2 * lane + 1] << 8);
+                qs = p.qI_scale[qrow];
+            } else {
+                const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(p.qI) + qrow * kDim;
+                v0 = __bfloat162float(src[2 * lane]);
+                v1 = __bfloat162float(src[2 * lane + 1]);
+                if (p.q_mode == 1) {
+                    float amax = fmaxf(fabsf(v0), fabsf(v1));
+                    for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+                    qs = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+                    packed = (uint32_t)e4m3_code(__fdiv_rn(v0, qs)) | ((uint32_t)e4m3_code(__fdiv_rn(v1, qs)) << 8);
+                } else {
+                    __nv_bfloat162 h2 = __floats2bfloat162_rn(v0, v1);
+                    packed = *reinterpret_cast<uint32_t*>(&h2);
+                }
+            }
+        } else {
+            packed = 0u;              // absent head: zero queries score zero
+        }
+        uint8_t* at = sA + h * C::kATile;
+        const int byte = 2 * lane * C::kElem;                    // byte offset of element 2*lane
+        const uint32_t off = a_offset<C::kRowBytes>(r, byte >> 4) + (byte & 15);
+        if (FP8)
+            *reinterpret_cast<uint16_t*>(at + off) = (uint16_t)packed;
+        else
+            *reinterpret_cast<uint32_t*>(at + off) = packed;
+        if (lane == 0) rs->qs[r][h] = (h < p.H_I) ? qs : 0.0f;
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = ctl->tmem_base;
+
+    // any row that needs selection at all?
+    int need = 0;
+    for (int r = 0; r < kRows; ++r) need |= (rs->ready[r] == 0);
+
+    // role counters that persist across passes
+    int L = 0;                 // producer / MMA: chunk loads issued
+    int use_buf[2] = {0, 0};   // MMA: issues into each TMEM buffer
+    int cons = 0;              // epilogue: chunks consumed by this group
+    const bool is_epi = warp >= 2;
+    const int grp = is_epi ? ((warp - 2) >> 2) : 0;
+    const int r = (warp & 3) * 32 + lane;                    // epilogue row
+    const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
+
+    for (int pass = 0; need && pass <= kLevels; ++pass) {
+        const bool emit = ctl->next_emit != 0;
+        if (!emit) {
+            for (int i = threadIdx.x; i < 2 * 256 * kRows / 2; i += kThreads)
+                reinterpret_cast<uint32_t*>(hist)[i] = 0u;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            // ------------------------------------------------------------ TMA producer
+            if (lane == 0) {
+                for (int c = 0; c < nchunks; ++c, ++L) {
+                    const int slot = L % C::kStages, u = L / C::kStages;
+                    if (u > 0 && !mbar_wait(&ctl->freeb[slot], (u - 1) & 1, abort, p.err)) break;
+                    mbar_arrive_expect_tx(&ctl->full[slot], C::kBTile);
+                    tma_load_2d(sB + slot * C::kBTile, &tm_k, 0, b * p.N_cap + c * kN, &ctl->full[slot]);
+                }
+            }
+            __syncwarp();
+            L = __shfl_sync(0xffffffffu, L, 0);
+        } else if (warp == 1) {
+            // ------------------------------------------------------------ MMA issuer
+            if (lane == 0) {
+                const uint32_t idesc = FP8 ? idesc_e4m3(kRows, kN) : idesc_bf16(kRows, kN, false, false);
+                for (int c = 0; c < nchunks; ++c, ++L) {
+                    const int slot = L % C::kStages;
+                    const int g = c & 1;
+                    if (!mbar_wait(&ctl->full[slot], (L / C::kStages) & 1, abort, p.err)) break;
+                    if (use_buf[g] > 0 && !mbar_wait(&ctl->acc_free[g], (use_buf[g] - 1) & 1, abort, p.err)) break;
+                    tc_fence_after();
+                    const uint32_t bsa = smem_u32(sB + slot * C::kBTile);
+                    for (int h = 0; h < kHeads; ++h) {
+                        const uint32_t asa = smem_u32(sA + h * C::kATile);
+                        for (int k = 0; k < C::kKSteps; ++k) {
+                            // each K step covers 32 bytes of a row
+                            const uint64_t ad = desc_noswizzle(asa + k * 256, 128, (C::kRowBytes / 16) * 128);
+                            const uint64_t bd = FP8 ? desc_sw(bsa + k * 32, 512, 4 /*SW64*/)
+                                                    : desc_sw(bsa + k * 32, 1024, 2 /*SW128*/);
+                            if (FP8)
+                                mma_f8_ss(tmem + g * 256 + h * kN, ad, bd, idesc, k > 0);
+                            else
+                                mma_bf16_ss(tmem + g * 256 + h * kN, ad, bd, idesc, k > 0);
+                        }
+                    }
+                    mma_commit(&ctl->acc_full[g]);
+                    mma_commit(&ctl->freeb[slot]);
+                    ++use_buf[g];
+                }
+            }
+            __syncwarp();
+            L = __shfl_sync(0xffffffffu, L, 0);
+            use_buf[0] = __shfl_sync(0xffffffffu, use_buf[0], 0);
+            use_buf[1] = __shfl_sync(0xffffffffu, use_buf[1], 0);
+        } else {
+            // ------------------------------------------------------------ epilogue
+            const int V = rs->V[r];
+            const bool active = rs->ready[r] == 0 || emit;   // rows still selecting, or emitting
+            const int level = rs->level[r];
+            const uint64_t prefix = rs->prefix[r];
+            const int sh = shift_of(level);
+            const bool rdy = rs->ready[r] != 0;
+            const bool all_rows = V <= p.topk;                // take-everything rows emit at the end
+            float qs[kHeads];
+#pragma unroll
+            for (int h = 0; h < kHeads; ++h) qs[h] = rs->qs[r][h];
+            uint16_t* hrow = hist + grp * 256 * kRows + r;
+            const float* ksc = p.kI_scale ? p.kI_scale + (size_t)b * p.N_cap : nullptr;
+            int* orow = p.idx_out + ((size_t)b * p.n + min(t0 + r, p.n - 1)) * p.topk;
+            const bool row_ok = t0 + r < p.n;
+            // group 0 fills a row from the front, group 1 from the back: each
+            // group's sequence is deterministic, so the row order is too
+            int nem = 0;
+            bool okg = true;
+            for (int c = grp; c < nchunks; c += 2) {
+                okg = __all_sync(0xffffffffu, mbar_wait(&ctl->acc_full[grp], cons & 1, abort, p.err));
+                if (!okg) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int part = 0; part < kN / 16; ++part) {
+                    float acc[kHeads][16];
+#pragma unroll
+                    for (int h = 0; h < kHeads; ++h)
+                        tmem_ld16(tmem + lane_addr + grp * 256 + h * kN + part * 16, acc[h]);
+                    if (!(active && row_ok && !all_rows)) continue;
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int s = c * kN + part * 16 + e;
+                        if (s >= V) continue;
+                        float sc = 0.0f;
+#pragma unroll
+                        for (int h = 0; h < kHeads; ++h) sc = fmaf(qs[h], relu0(acc[h][e]), sc);
+                        if (FP8) sc *= __ldg(ksc + s);
+                        const uint64_t key = ((uint64_t)__float_as_uint(relu0(sc)) << 16) | (uint64_t)(65535 - s);
+                        if (!emit) {
+                            if (level == 0 || (key >> (sh + 8)) == prefix) {
+                                uint16_t* cell = hrow + ((key >> sh) & 255u) * kRows;
+                                *cell = (uint16_t)(*cell + 1);
+                            }
+                        } else {
+                            const uint64_t kp = key >> sh;
+                            if (kp > prefix) {
+                                const int pos = grp == 0 ? nem : p.topk - 1 - nem;
+                                if (nem < p.topk) orow[pos] = s;
+                                ++nem;
+                            } else if (kp == prefix) {
+                                const int pos = atomicAdd(&rs->listed[r], 1);
+                                if (pos < kCap) list[r * kCap + pos] = key;
+                            }
+                        }
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&ctl->acc_free[grp]);
+                ++cons;
+            }
+            if (emit) rs->emitted[grp][r] = nem;
+            (void)rdy;
+        }
+        __syncthreads();
+        if (*abort) break;
+        // ---------------------------------------------------------------- per-row bookkeeping
+        if (warp >= 2 && grp == 0) {
+            const int V = rs->V[r];
+            if (!emit) {
+                if (!rs->ready[r] && V > p.topk) {
+                    // merge the two groups' bins; find the digit holding rank
+                    int rank = rs->rank[r];
+                    int run = 0, digit = 0, inbin = 0;
+                    for (int d = 255; d >= 0; --d) {
+                        const int cnt = hist[d * kRows + r] + hist[256 * kRows + d * kRows + r];
+                        if (run + cnt >= rank) { digit = d; inbin = cnt; break; }
+                        run += cnt;
+                    }
+                    const int level = rs->level[r];
+                    rs->prefix[r] = (rs->prefix[r] << 8) | (uint64_t)digit;
+                    rs->rank[r] = rank - run;
+                    if (inbin <= kCap || level == kLevels - 1) {
+                        rs->ready[r] = 1;          // emit with this prefix at this level's shift
+                    } else {
+                        rs->level[r] = level + 1;
+                    }
+                }
+            } else if (t0 + r < p.n) {
+                int* orow = p.idx_out + ((size_t)b * p.n + t0 + r) * p.topk;
+                if (V <= p.topk) {
+                    for (int j = 0; j < p.topk; ++j) orow[j] = j < V ? j : -1;
+                } else {
+                    // boundary keys: the rank largest, by insertion into a sorted prefix
+                    const int nl = min(rs->listed[r], kCap);
+                    uint64_t* lr = list + r * kCap;
+                    for (int i = 1; i < nl; ++i) {
+                        const uint64_t v = lr[i];
+                        int j = i - 1;
+                        while (j >= 0 && lr[j] < v) { lr[j + 1] = lr[j]; --j; }
+                        lr[j + 1] = v;
+                    }
+                    int pos = rs->emitted[0][r];
+                    const int end = p.topk - rs->emitted[1][r];
+                    const int want = min(rs->rank[r], nl);
+                    for (int i = 0; i < want && pos < end; ++i, ++pos)
+                        orow[pos] = 65535 - (int)(lr[i] & 0xFFFFu);
+                    for (; pos < end; ++pos) orow[pos] = -1;   // unreachable when counts agree
+                }
+            }
+        }
+        __syncthreads();
+        if (emit) break;
+        // the next pass emits once every selecting row is ready
+        if (threadIdx.x == 0) {
+            int all_ready = 1;
+            for (int i = 0; i < kRows; ++i) all_ready &= rs->ready[i];
+            ctl->next_emit = all_ready;
+        }
+        __syncthreads();
+    }
+    if (!need) {
+        // every row takes all its visible entries
+        for (int i = threadIdx.x; i < kRows; i += kThreads) {
+            if (t0 + i >= p.n) continue;
+            int* orow = p.idx_out + ((size_t)b * p.n + t0 + i) * p.topk;
+            const int V = rs->V[i];
+            for (int j = 0; j < p.topk; ++j) orow[j] = j < V ? j : -1;
+        }
+    }
+    // no MMA may be in flight when TMEM is released
+    if (warp == 1) {
+        if (lane == 0) {
+            mma_commit(&ctl->fin);
+            volatile int never = 0;
+            mbar_wait(&ctl->fin, 0, &never, p.err);
+        }
+        __syncwarp();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 1) tmem_dealloc(tmem, 512);
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        cudaDriverEntryPointQueryResult q;
+        void* f = nullptr;
+        if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &f, 12000, cudaEnableDefault,
+                                             &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    }
+    return fn;
+}
+
+}  // namespace
+
+bool indexer_tc_supported(const IndexerArgs& a) {
+    const bool fp8 = a.kI_dt == DT_E4M3 && (a.qI_dt == DT_BF16 || a.qI_dt == DT_E4M3);
+    const bool bf16 = a.kI_dt == DT_BF16 && a.qI_dt == DT_BF16;
+    return (fp8 || bf16) && a.d_I == kDim && a.H_I <= kHeads && a.q_pos == nullptr &&
+           a.N_cap <= 65536 && a.n_q >= 1;
+}
+
+cudaError_t launch_indexer_tc(const IndexerArgs& a, uint32_t* err, cudaStream_t s) {
+    const bool fp8 = a.kI_dt == DT_E4M3;
+    auto fn = encode_fn();
+    if (!fn) return cudaErrorInvalidValue;
+    CUtensorMap tm;
+    const int row_bytes = fp8 ? kDim : kDim * 2;
+    cuuint64_t dims[2] = {(cuuint64_t)(fp8 ? kDim : kDim), (cuuint64_t)a.B * (a.N_cap > 0 ? a.N_cap : 1)};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {(cuuint32_t)kDim, (cuuint32_t)kN};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(&tm, fp8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                    const_cast<void*>(a.kI), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    fp8 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+    IdxParams p;
+    p.qI = a.qI;
+    p.qI_scale = a.qI_scale;
+    p.kI_scale = a.kI_scale;
+    p.q_mode = fp8 ? (a.qI_dt == DT_E4M3 ? 2 : 1) : 0;
+    p.B = a.B;
+    p.n = a.n_q;
+    p.H_I = a.H_I;
+    p.N_cap = a.N_cap;
+    p.m = a.m;
+    p.topk = a.topk;
+    p.n_entries = a.n_entries;
+    p.idx_out = a.idx_out;
+    p.err = err;
+    const int tiles = (a.n_q + kRows - 1) / kRows;
+    if (fp8) {
+        auto k = indexer_tc_kernel<true>;
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg<true>::kSmem);
+        if (e != cudaSuccess) return e;
+        k<<<(unsigned)(a.B * tiles), kThreads, Cfg<true>::kSmem, s>>>(tm, p);
+    } else {
+        auto k = indexer_tc_kernel<false>;
+        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg<false>::kSmem);
+        if (e != cudaSuccess) return e;
+        k<<<(unsigned)(a.B * tiles), kThreads, Cfg<false>::kSmem, s>>>(tm, p);
+    }
+    count_launch();
+    return cudaGetLastError();
+}
+
+}  // namespace csa

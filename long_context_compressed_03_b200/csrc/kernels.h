@@ -47,6 +47,10 @@ uint32_t* device_error_word();
 bool attention_tc_supported(const AttnArgs& a);
 cudaError_t launch_attention_tc(const AttnArgs& a, uint32_t* err, cudaStream_t s);
 
+// tcgen05 indexer + fused exact top-k for prefill (d_I = 64, H_I <= 4).
+bool indexer_tc_supported(const IndexerArgs& a);
+cudaError_t launch_indexer_tc(const IndexerArgs& a, uint32_t* err, cudaStream_t s);
+
 // Counts one kernel launch (read back through csa_kernel_launches()).
 void count_launch();
 
