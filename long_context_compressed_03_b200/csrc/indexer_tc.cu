@@ -21,7 +21,8 @@
 // that holds the k-th largest key: each pass recomputes the scores (the
 // tensor cores make that cheap) and histograms the next digit of the keys
 // that match the row's current prefix into per-row u16 bins in shared
-// memory ([bin][row] layout: conflict-free).  Once a row's boundary bin has
+// memory ([bin][row] layout: conflict-free; both epilogue groups add with
+// fire-and-forget shared atomics).  Once a row's boundary bin has
 // at most kCap keys, a final pass writes every key above the boundary to the
 // output and collects the boundary bin, which is then sorted exactly.  The
 // score matrix never leaves the SM.
@@ -52,7 +53,7 @@ struct Cfg {
     static constexpr int kBTile = kN * kRowBytes;                   // per chunk
     static constexpr int kStages = FP8 ? 4 : 3;
     static constexpr int kKSteps = FP8 ? 2 : 4;                     // K=32 (fp8) / 16 (bf16)
-    static constexpr int kHist = 2 * 256 * kRows * 2;               // two groups, u16 bins
+    static constexpr int kHist = 256 * kRows * 4;                   // u32 bins, both groups
     static constexpr size_t kSmem = 1024 + kHeads * kATile + kStages * kBTile + kHist + 8192;
 };
 
@@ -130,6 +131,20 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
         : "memory");
 }
 
+// Four heads x 16 columns (head h at column offset h*stride) with one wait.
+__device__ __forceinline__ void tmem_ld16x4(uint32_t taddr, int stride, float (*v)[16]) {
+    uint32_t* r = reinterpret_cast<uint32_t*>(&v[0][0]);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%64];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%65];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47}, [%66];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%67];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr), "r"(taddr + stride), "r"(taddr + 2 * stride), "r"(taddr + 3 * stride)
+        : "memory");
+}
+
 template <bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
@@ -138,7 +153,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sA = base;                                       // [kHeads][kATile]
     uint8_t* sB = sA + kHeads * C::kATile;                    // [kStages][kBTile]
-    uint16_t* hist = reinterpret_cast<uint16_t*>(sB + C::kStages * C::kBTile);   // [2][256][128]
+    uint32_t* hist = reinterpret_cast<uint32_t*>(sB + C::kStages * C::kBTile);   // [256][128]
     uint64_t* list = reinterpret_cast<uint64_t*>(hist);      // [128][kCap] (aliases hist)
     RowState* rs = reinterpret_cast<RowState*>(reinterpret_cast<uint8_t*>(hist) + C::kHist);
     Ctrl* ctl = reinterpret_cast<Ctrl*>(reinterpret_cast<uint8_t*>(rs) + sizeof(RowState));
@@ -247,8 +262,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
     for (int pass = 0; need && pass <= kLevels; ++pass) {
         const bool emit = ctl->next_emit != 0;
         if (!emit) {
-            for (int i = threadIdx.x; i < 2 * 256 * kRows / 2; i += kThreads)
-                reinterpret_cast<uint32_t*>(hist)[i] = 0u;
+            for (int i = threadIdx.x; i < 256 * kRows; i += kThreads) hist[i] = 0u;
         }
         __syncthreads();
         if (warp == 0) {
@@ -308,7 +322,9 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
             float qs[kHeads];
 #pragma unroll
             for (int h = 0; h < kHeads; ++h) qs[h] = rs->qs[r][h];
-            uint16_t* hrow = hist + grp * 256 * kRows + r;
+            uint32_t* hrow = hist + r;
+            const uint32_t prefix32 = (uint32_t)prefix;      // levels 0-3: score bits only
+            const int sh32 = 24 - 8 * level;
             const float* ksc = p.kI_scale ? p.kI_scale + (size_t)b * p.N_cap : nullptr;
             int* orow = p.idx_out + ((size_t)b * p.n + min(t0 + r, p.n - 1)) * p.topk;
             const bool row_ok = t0 + r < p.n;
@@ -323,9 +339,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
 #pragma unroll 1
                 for (int part = 0; part < kN / 16; ++part) {
                     float acc[kHeads][16];
-#pragma unroll
-                    for (int h = 0; h < kHeads; ++h)
-                        tmem_ld16(tmem + lane_addr + grp * 256 + h * kN + part * 16, acc[h]);
+                    tmem_ld16x4(tmem + lane_addr + grp * 256 + part * 16, kN, acc);
                     if (!(active && row_ok && !all_rows)) continue;
 #pragma unroll
                     for (int e = 0; e < 16; ++e) {
@@ -335,12 +349,17 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
 #pragma unroll
                         for (int h = 0; h < kHeads; ++h) sc = fmaf(qs[h], relu0(acc[h][e]), sc);
                         if (FP8) sc *= __ldg(ksc + s);
-                        const uint64_t key = ((uint64_t)__float_as_uint(relu0(sc)) << 16) | (uint64_t)(65535 - s);
+                        const uint32_t sbits = __float_as_uint(relu0(sc));
+                        if (!emit && level < 4) {
+                            // digits of the score bits: 32-bit arithmetic
+                            if (level == 0 || (sbits >> (sh32 + 8)) == prefix32)
+                                atomicAdd(hrow + ((sbits >> sh32) & 255u) * kRows, 1u);
+                            continue;
+                        }
+                        const uint64_t key = ((uint64_t)sbits << 16) | (uint64_t)(65535 - s);
                         if (!emit) {
-                            if (level == 0 || (key >> (sh + 8)) == prefix) {
-                                uint16_t* cell = hrow + ((key >> sh) & 255u) * kRows;
-                                *cell = (uint16_t)(*cell + 1);
-                            }
+                            if ((key >> (sh + 8)) == prefix)
+                                atomicAdd(hrow + ((key >> sh) & 255u) * kRows, 1u);
                         } else {
                             const uint64_t kp = key >> sh;
                             if (kp > prefix) {
@@ -372,7 +391,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
                     int rank = rs->rank[r];
                     int run = 0, digit = 0, inbin = 0;
                     for (int d = 255; d >= 0; --d) {
-                        const int cnt = hist[d * kRows + r] + hist[256 * kRows + d * kRows + r];
+                        const int cnt = (int)hist[d * kRows + r];
                         if (run + cnt >= rank) { digit = d; inbin = cnt; break; }
                         run += cnt;
                     }
