@@ -9,10 +9,10 @@
 // qs, ks (the bf16 queries are quantised here, in fp32, exactly as the
 // compressor quantises a row); bf16: qs = ks = 1.
 //
-// Scores: for every chunk of 64 entries the MMA warp issues one tcgen05 MMA
-// per indexer head (M = 128 queries, N = 64 entries, K = 64) into TMEM;
-// two epilogue warpgroups take alternate chunks (TMEM: 2 buffers x 4 heads
-// x 64 columns).  Each epilogue thread owns one query row.
+// Scores: for every chunk of 32 entries the MMA warp issues one tcgen05 MMA
+// per indexer head (M = 128 queries, N = 32 entries, K = 64) into TMEM;
+// four epilogue warpgroups take chunks in turn (TMEM: 4 buffers x 4 heads
+// x 32 columns).  Each epilogue thread owns one query row.
 //
 // Selection: every (row, entry) gets the unique 48-bit key
 //   K = (bits of the non-negative fp32 score) << 16 | (65535 - s),
@@ -24,9 +24,12 @@
 // memory ([bin][row] layout: conflict-free; both epilogue groups add with
 // fire-and-forget shared atomics).  Once a row's boundary bin has
 // at most kCap keys, a final pass writes every key above the boundary to the
-// output and collects the boundary bin, which is then sorted exactly.  The
-// score matrix never leaves the SM.
+// output and collects the boundary bin, which is then sorted exactly; each
+// selected row is finally sorted by entry index (a deterministic order).
+// The score matrix never leaves the SM.
 #include <cudaTypedefs.h>
+
+#include <climits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -38,10 +41,11 @@ namespace {
 using namespace tc;
 
 constexpr int kRows = 128;      // queries per CTA = MMA M
-constexpr int kN = 64;          // entries per chunk = MMA N
+constexpr int kN = 32;          // entries per chunk = MMA N
+constexpr int kGroups = 4;      // epilogue warpgroups (one TMEM buffer each)
 constexpr int kHeads = 4;       // indexer heads held in TMEM
 constexpr int kDim = 64;        // indexer head dim = MMA K
-constexpr int kThreads = 320;   // warp 0 TMA, warp 1 MMA, warps 2-5 / 6-9 epilogue groups
+constexpr int kThreads = 576;   // warp 0 TMA, warp 1 MMA, warps 2-17: four epilogue groups
 constexpr int kCap = 64;        // boundary-bin capacity per row
 constexpr int kLevels = 6;      // 48-bit key, 8-bit digits
 
@@ -71,8 +75,8 @@ struct IdxParams {
 struct __align__(8) Ctrl {
     uint64_t full[4];
     uint64_t freeb[4];
-    uint64_t acc_full[2];
-    uint64_t acc_free[2];
+    uint64_t acc_full[kGroups];
+    uint64_t acc_free[kGroups];
     uint64_t fin;
     uint32_t tmem_base;
     int abort;
@@ -86,7 +90,7 @@ struct RowState {
     int rank[kRows];           // keys still needed from the prefix's bin
     int ready[kRows];          // boundary bin small enough (or keys unique)
     int V[kRows];              // visible entries (0 for rows beyond n)
-    int emitted[2][kRows];     // output slots used by each epilogue group
+    int emitted[kRows];        // output slots used
     int listed[kRows];         // boundary keys collected
     float qs[kRows][kHeads];   // per-head query scales
 };
@@ -145,6 +149,98 @@ __device__ __forceinline__ void tmem_ld16x4(uint32_t taddr, int stride, float (*
         : "memory");
 }
 
+enum PassKind { kHist0 = 0, kHist32 = 1, kHist64 = 2, kEmit = 3 };
+
+struct RowCtx {
+    int V;
+    uint64_t prefix;
+    int sh;
+    uint32_t* hrow;
+    int* orow;
+    uint64_t* list;
+    int* emitted;
+    int* listed;
+    int topk;
+    float qs[kHeads];
+};
+
+// Four heads x 8 columns (head h at column offset h*kN) with one wait.
+__device__ __forceinline__ void tmem_ld8x4(uint32_t taddr, float (*v)[8]) {
+    uint32_t* r = reinterpret_cast<uint32_t*>(&v[0][0]);
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%32];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%8, %9, %10, %11, %12, %13, %14, %15}, [%33];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%16, %17, %18, %19, %20, %21, %22, %23}, [%34];\n\t"
+        "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%24, %25, %26, %27, %28, %29, %30, %31}, [%35];\n\t"
+        "tcgen05.wait::ld.sync.aligned;"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+          "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+          "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+          "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr), "r"(taddr + kN), "r"(taddr + 2 * kN), "r"(taddr + 3 * kN)
+        : "memory");
+}
+
+// One chunk of 32 entries for this thread's row, in the pass's mode.  The
+// TMEM loads are warp-collective, so every thread runs them; rows that are
+// not selecting skip the arithmetic.
+template <bool FP8, int KIND>
+__device__ __forceinline__ void chunk_pass(uint32_t taddr, const float* ksc, int c, bool active,
+                                           const RowCtx& rc) {
+#pragma unroll 1
+    for (int part = 0; part < kN / 8; ++part) {
+        float acc[kHeads][8];
+        tmem_ld8x4(taddr + part * 8, acc);
+        if (!active) continue;
+        const int s0 = c * kN + part * 8;
+        if (s0 >= rc.V) continue;
+        const int ne = min(8, rc.V - s0);
+        float ks[8];
+        if (FP8) {
+            // s0 is a multiple of 8 below V <= N_cap (a multiple of 4): the
+            // first four scales are in bounds, the next four when ne > 4
+            const float4 k0 = __ldg(reinterpret_cast<const float4*>(ksc + s0));
+            const float4 k1 = ne > 4 ? __ldg(reinterpret_cast<const float4*>(ksc + s0 + 4))
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+            ks[0] = k0.x; ks[1] = k0.y; ks[2] = k0.z; ks[3] = k0.w;
+            ks[4] = k1.x; ks[5] = k1.y; ks[6] = k1.z; ks[7] = k1.w;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+            if (e >= ne) break;
+            float sc = rc.qs[0] * fmaxf(acc[0][e], 0.0f);
+#pragma unroll
+            for (int h = 1; h < kHeads; ++h) sc = fmaf(rc.qs[h], fmaxf(acc[h][e], 0.0f), sc);
+            if (FP8) sc *= ks[e];
+            const uint32_t sbits = __float_as_uint(sc) & 0x7FFFFFFFu;   // sc >= 0; drop a -0 sign
+            if (KIND == kHist0) {
+                atomicAdd(rc.hrow + (sbits >> 24) * kRows, 1u);
+            } else if (KIND == kHist32) {
+                const int sh32 = rc.sh - 16;
+                if ((sbits >> (sh32 + 8)) == (uint32_t)rc.prefix)
+                    atomicAdd(rc.hrow + ((sbits >> sh32) & 255u) * kRows, 1u);
+            } else {
+                const int s = s0 + e;
+                const uint64_t key = ((uint64_t)sbits << 16) | (uint64_t)(65535 - s);
+                if (KIND == kHist64) {
+                    if ((key >> (rc.sh + 8)) == rc.prefix)
+                        atomicAdd(rc.hrow + ((key >> rc.sh) & 255u) * kRows, 1u);
+                } else {
+                    const uint64_t kp = key >> rc.sh;
+                    if (kp > rc.prefix) {
+                        const int pos = atomicAdd(rc.emitted, 1);
+                        if (pos < rc.topk) rc.orow[pos] = s;
+                    } else if (kp == rc.prefix) {
+                        const int pos = atomicAdd(rc.listed, 1);
+                        if (pos < kCap) rc.list[pos] = key;
+                    }
+                }
+            }
+        }
+    }
+}
+
 template <bool FP8>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
@@ -176,7 +272,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
             mbar_init(&ctl->full[s], 1);
             mbar_init(&ctl->freeb[s], 1);
         }
-        for (int g = 0; g < 2; ++g) {
+        for (int g = 0; g < kGroups; ++g) {
             mbar_init(&ctl->acc_full[g], 1);
             mbar_init(&ctl->acc_free[g], kRows);
         }
@@ -198,8 +294,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
         rs->prefix[r] = 0;
         rs->rank[r] = p.topk;
         rs->ready[r] = (V <= p.topk) ? 1 : 0;   // rows with V <= k take every visible entry
-        rs->emitted[0][r] = 0;
-        rs->emitted[1][r] = 0;
+        rs->emitted[r] = 0;
         rs->listed[r] = 0;
     }
     for (int pair = warp; pair < kRows * kHeads; pair += kThreads / 32) {
@@ -252,10 +347,10 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
 
     // role counters that persist across passes
     int L = 0;                 // producer / MMA: chunk loads issued
-    int use_buf[2] = {0, 0};   // MMA: issues into each TMEM buffer
+    int use_buf[kGroups] = {0, 0, 0, 0};   // MMA: issues into each TMEM buffer
     int cons = 0;              // epilogue: chunks consumed by this group
     const bool is_epi = warp >= 2;
-    const int grp = is_epi ? ((warp - 2) >> 2) : 0;
+    const int grp = is_epi ? ((warp - 2) >> 2) : 0;      // warps 2-5, 6-9, 10-13, 14-17
     const int r = (warp & 3) * 32 + lane;                    // epilogue row
     const uint32_t lane_addr = (uint32_t)((warp & 3) * 32) << 16;
 
@@ -283,7 +378,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
                 const uint32_t idesc = FP8 ? idesc_e4m3(kRows, kN) : idesc_bf16(kRows, kN, false, false);
                 for (int c = 0; c < nchunks; ++c, ++L) {
                     const int slot = L % C::kStages;
-                    const int g = c & 1;
+                    const int g = c % kGroups;
                     if (!mbar_wait(&ctl->full[slot], (L / C::kStages) & 1, abort, p.err)) break;
                     if (use_buf[g] > 0 && !mbar_wait(&ctl->acc_free[g], (use_buf[g] - 1) & 1, abort, p.err)) break;
                     tc_fence_after();
@@ -296,9 +391,9 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
                             const uint64_t bd = FP8 ? desc_sw(bsa + k * 32, 512, 4 /*SW64*/)
                                                     : desc_sw(bsa + k * 32, 1024, 2 /*SW128*/);
                             if (FP8)
-                                mma_f8_ss(tmem + g * 256 + h * kN, ad, bd, idesc, k > 0);
+                                mma_f8_ss(tmem + g * 128 + h * kN, ad, bd, idesc, k > 0);
                             else
-                                mma_bf16_ss(tmem + g * 256 + h * kN, ad, bd, idesc, k > 0);
+                                mma_bf16_ss(tmem + g * 128 + h * kN, ad, bd, idesc, k > 0);
                         }
                     }
                     mma_commit(&ctl->acc_full[g]);
@@ -308,82 +403,46 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
             }
             __syncwarp();
             L = __shfl_sync(0xffffffffu, L, 0);
-            use_buf[0] = __shfl_sync(0xffffffffu, use_buf[0], 0);
-            use_buf[1] = __shfl_sync(0xffffffffu, use_buf[1], 0);
+            for (int g = 0; g < kGroups; ++g) use_buf[g] = __shfl_sync(0xffffffffu, use_buf[g], 0);
         } else {
             // ------------------------------------------------------------ epilogue
             const int V = rs->V[r];
-            const bool active = rs->ready[r] == 0 || emit;   // rows still selecting, or emitting
-            const int level = rs->level[r];
-            const uint64_t prefix = rs->prefix[r];
-            const int sh = shift_of(level);
-            const bool rdy = rs->ready[r] != 0;
-            const bool all_rows = V <= p.topk;                // take-everything rows emit at the end
-            float qs[kHeads];
-#pragma unroll
-            for (int h = 0; h < kHeads; ++h) qs[h] = rs->qs[r][h];
-            uint32_t* hrow = hist + r;
-            const uint32_t prefix32 = (uint32_t)prefix;      // levels 0-3: score bits only
-            const int sh32 = 24 - 8 * level;
-            const float* ksc = p.kI_scale ? p.kI_scale + (size_t)b * p.N_cap : nullptr;
-            int* orow = p.idx_out + ((size_t)b * p.n + min(t0 + r, p.n - 1)) * p.topk;
             const bool row_ok = t0 + r < p.n;
-            // group 0 fills a row from the front, group 1 from the back: each
-            // group's sequence is deterministic, so the row order is too
-            int nem = 0;
-            bool okg = true;
-            for (int c = grp; c < nchunks; c += 2) {
-                okg = __all_sync(0xffffffffu, mbar_wait(&ctl->acc_full[grp], cons & 1, abort, p.err));
-                if (!okg) break;
+            const bool active = row_ok && V > p.topk && (rs->ready[r] == 0 || emit);
+            const int level = rs->level[r];
+            const int kind = emit ? kEmit : (level == 0 ? kHist0 : (level < 4 ? kHist32 : kHist64));
+            RowCtx rc;
+            rc.V = V;
+            rc.prefix = rs->prefix[r];
+            rc.sh = shift_of(level);
+            rc.hrow = hist + r;
+            rc.orow = p.idx_out + ((size_t)b * p.n + min(t0 + r, p.n - 1)) * p.topk;
+            rc.list = list + r * kCap;
+            rc.emitted = &rs->emitted[r];
+            rc.listed = &rs->listed[r];
+            rc.topk = p.topk;
+#pragma unroll
+            for (int h = 0; h < kHeads; ++h) rc.qs[h] = rs->qs[r][h];
+            const float* ksc = FP8 ? p.kI_scale + (size_t)b * p.N_cap : nullptr;
+            for (int c = grp; c < nchunks; c += kGroups) {
+                if (!__all_sync(0xffffffffu, mbar_wait(&ctl->acc_full[grp], cons & 1, abort, p.err))) break;
                 tc_fence_after();
-#pragma unroll 1
-                for (int part = 0; part < kN / 16; ++part) {
-                    float acc[kHeads][16];
-                    tmem_ld16x4(tmem + lane_addr + grp * 256 + part * 16, kN, acc);
-                    if (!(active && row_ok && !all_rows)) continue;
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int s = c * kN + part * 16 + e;
-                        if (s >= V) continue;
-                        float sc = 0.0f;
-#pragma unroll
-                        for (int h = 0; h < kHeads; ++h) sc = fmaf(qs[h], relu0(acc[h][e]), sc);
-                        if (FP8) sc *= __ldg(ksc + s);
-                        const uint32_t sbits = __float_as_uint(relu0(sc));
-                        if (!emit && level < 4) {
-                            // digits of the score bits: 32-bit arithmetic
-                            if (level == 0 || (sbits >> (sh32 + 8)) == prefix32)
-                                atomicAdd(hrow + ((sbits >> sh32) & 255u) * kRows, 1u);
-                            continue;
-                        }
-                        const uint64_t key = ((uint64_t)sbits << 16) | (uint64_t)(65535 - s);
-                        if (!emit) {
-                            if ((key >> (sh + 8)) == prefix)
-                                atomicAdd(hrow + ((key >> sh) & 255u) * kRows, 1u);
-                        } else {
-                            const uint64_t kp = key >> sh;
-                            if (kp > prefix) {
-                                const int pos = grp == 0 ? nem : p.topk - 1 - nem;
-                                if (nem < p.topk) orow[pos] = s;
-                                ++nem;
-                            } else if (kp == prefix) {
-                                const int pos = atomicAdd(&rs->listed[r], 1);
-                                if (pos < kCap) list[r * kCap + pos] = key;
-                            }
-                        }
-                    }
+                const uint32_t taddr = tmem + lane_addr + grp * 128;
+                switch (kind) {
+                    case kHist0: chunk_pass<FP8, kHist0>(taddr, ksc, c, active, rc); break;
+                    case kHist32: chunk_pass<FP8, kHist32>(taddr, ksc, c, active, rc); break;
+                    case kHist64: chunk_pass<FP8, kHist64>(taddr, ksc, c, active, rc); break;
+                    default: chunk_pass<FP8, kEmit>(taddr, ksc, c, active, rc); break;
                 }
                 tc_fence_before();
                 mbar_arrive(&ctl->acc_free[grp]);
                 ++cons;
             }
-            if (emit) rs->emitted[grp][r] = nem;
-            (void)rdy;
         }
         __syncthreads();
         if (*abort) break;
         // ---------------------------------------------------------------- per-row bookkeeping
-        if (warp >= 2 && grp == 0) {
+        if (is_epi && grp == 0) {
             const int V = rs->V[r];
             if (!emit) {
                 if (!rs->ready[r] && V > p.topk) {
@@ -418,17 +477,51 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
                         while (j >= 0 && lr[j] < v) { lr[j + 1] = lr[j]; --j; }
                         lr[j + 1] = v;
                     }
-                    int pos = rs->emitted[0][r];
-                    const int end = p.topk - rs->emitted[1][r];
+                    int pos = min(rs->emitted[r], p.topk);
                     const int want = min(rs->rank[r], nl);
-                    for (int i = 0; i < want && pos < end; ++i, ++pos)
+                    for (int i = 0; i < want && pos < p.topk; ++i, ++pos)
                         orow[pos] = 65535 - (int)(lr[i] & 0xFFFFu);
-                    for (; pos < end; ++pos) orow[pos] = -1;   // unreachable when counts agree
+                    for (; pos < p.topk; ++pos) orow[pos] = -1;   // unreachable when counts agree
                 }
             }
         }
         __syncthreads();
-        if (emit) break;
+        if (emit) {
+            // the emitted set is exact; its order depends on which group got
+            // there first.  Sort each selected row ascending: a deterministic
+            // (and gather-friendly) order.  One warp per row, bitonic in smem.
+            if (is_epi) {
+                const int ew = warp - 2;
+                int* buf = reinterpret_cast<int*>(hist) + ew * 2048;   // 8 KB per warp
+                const int kk = p.topk;
+                int np2 = 1;
+                while (np2 < kk) np2 <<= 1;
+                for (int rr = ew; rr < kRows; rr += kGroups * 4) {
+                    if (t0 + rr >= p.n || rs->V[rr] <= kk) continue;
+                    int* orow = p.idx_out + ((size_t)b * p.n + t0 + rr) * kk;
+                    for (int i = lane; i < np2; i += 32) buf[i] = i < kk ? orow[i] : INT_MAX;
+                    __syncwarp();
+                    for (int size = 2; size <= np2; size <<= 1) {
+                        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                            for (int i = lane; i < np2 / 2; i += 32) {
+                                const int lo = 2 * i - (i & (stride - 1));
+                                const int hi = lo + stride;
+                                const bool up = (lo & size) == 0;
+                                const int a0 = buf[lo], a1 = buf[hi];
+                                if ((a0 > a1) == up) {
+                                    buf[lo] = a1;
+                                    buf[hi] = a0;
+                                }
+                            }
+                            __syncwarp();
+                        }
+                    }
+                    for (int i = lane; i < kk; i += 32) orow[i] = buf[i];
+                    __syncwarp();
+                }
+            }
+            break;
+        }
         // the next pass emits once every selecting row is ready
         if (threadIdx.x == 0) {
             int all_ready = 1;
@@ -480,7 +573,7 @@ bool indexer_tc_supported(const IndexerArgs& a) {
     const bool fp8 = a.kI_dt == DT_E4M3 && (a.qI_dt == DT_BF16 || a.qI_dt == DT_E4M3);
     const bool bf16 = a.kI_dt == DT_BF16 && a.qI_dt == DT_BF16;
     return (fp8 || bf16) && a.d_I == kDim && a.H_I <= kHeads && a.q_pos == nullptr &&
-           a.N_cap <= 65536 && a.n_q >= 1;
+           a.N_cap <= 65536 && (a.N_cap % 4) == 0 && a.n_q >= 1;
 }
 
 cudaError_t launch_indexer_tc(const IndexerArgs& a, uint32_t* err, cudaStream_t s) {
