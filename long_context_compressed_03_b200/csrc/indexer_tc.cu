@@ -161,6 +161,7 @@ struct RowCtx {
     int* emitted;
     int* listed;
     int topk;
+    bool ks_vec;               // per-entry scales readable as float4
     float qs[kHeads];
 };
 
@@ -182,12 +183,14 @@ __device__ __forceinline__ void tmem_ld8x4(uint32_t taddr, float (*v)[8]) {
         : "memory");
 }
 
-// One chunk of 32 entries for this thread's row, in the pass's mode.  The
-// TMEM loads are warp-collective, so every thread runs them; rows that are
-// not selecting skip the arithmetic.
-template <bool FP8, int KIND>
+// One chunk of 32 entries for this thread's row, in the row's mode (rows of
+// one warp can be at different radix levels).  The TMEM loads are .sync.aligned
+// warp-collective instructions: every lane of the warp runs them at the same
+// point, before any per-row branching; rows that are not selecting skip the
+// arithmetic.
+template <bool FP8>
 __device__ __forceinline__ void chunk_pass(uint32_t taddr, const float* ksc, int c, bool active,
-                                           const RowCtx& rc) {
+                                           int KIND, const RowCtx& rc) {
 #pragma unroll 1
     for (int part = 0; part < kN / 8; ++part) {
         float acc[kHeads][8];
@@ -198,13 +201,19 @@ __device__ __forceinline__ void chunk_pass(uint32_t taddr, const float* ksc, int
         const int ne = min(8, rc.V - s0);
         float ks[8];
         if (FP8) {
-            // s0 is a multiple of 8 below V <= N_cap (a multiple of 4): the
-            // first four scales are in bounds, the next four when ne > 4
-            const float4 k0 = __ldg(reinterpret_cast<const float4*>(ksc + s0));
-            const float4 k1 = ne > 4 ? __ldg(reinterpret_cast<const float4*>(ksc + s0 + 4))
-                                     : make_float4(0.f, 0.f, 0.f, 0.f);
-            ks[0] = k0.x; ks[1] = k0.y; ks[2] = k0.z; ks[3] = k0.w;
-            ks[4] = k1.x; ks[5] = k1.y; ks[6] = k1.z; ks[7] = k1.w;
+            if (rc.ks_vec) {
+                // 16-byte aligned rows: s0 is a multiple of 8 below V <= N_cap
+                // (a multiple of 4), so the first four scales are in bounds,
+                // the next four when ne > 4
+                const float4 k0 = __ldg(reinterpret_cast<const float4*>(ksc + s0));
+                const float4 k1 = ne > 4 ? __ldg(reinterpret_cast<const float4*>(ksc + s0 + 4))
+                                         : make_float4(0.f, 0.f, 0.f, 0.f);
+                ks[0] = k0.x; ks[1] = k0.y; ks[2] = k0.z; ks[3] = k0.w;
+                ks[4] = k1.x; ks[5] = k1.y; ks[6] = k1.z; ks[7] = k1.w;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) ks[e] = e < ne ? __ldg(ksc + s0 + e) : 0.0f;
+            }
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -421,6 +430,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
             rc.emitted = &rs->emitted[r];
             rc.listed = &rs->listed[r];
             rc.topk = p.topk;
+            rc.ks_vec = (p.N_cap & 3) == 0;
 #pragma unroll
             for (int h = 0; h < kHeads; ++h) rc.qs[h] = rs->qs[r][h];
             const float* ksc = FP8 ? p.kI_scale + (size_t)b * p.N_cap : nullptr;
@@ -428,12 +438,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
                 if (!__all_sync(0xffffffffu, mbar_wait(&ctl->acc_full[grp], cons & 1, abort, p.err))) break;
                 tc_fence_after();
                 const uint32_t taddr = tmem + lane_addr + grp * 128;
-                switch (kind) {
-                    case kHist0: chunk_pass<FP8, kHist0>(taddr, ksc, c, active, rc); break;
-                    case kHist32: chunk_pass<FP8, kHist32>(taddr, ksc, c, active, rc); break;
-                    case kHist64: chunk_pass<FP8, kHist64>(taddr, ksc, c, active, rc); break;
-                    default: chunk_pass<FP8, kEmit>(taddr, ksc, c, active, rc); break;
-                }
+                chunk_pass<FP8>(taddr, ksc, c, active, kind, rc);
                 tc_fence_before();
                 mbar_arrive(&ctl->acc_free[grp]);
                 ++cons;
@@ -573,7 +578,7 @@ bool indexer_tc_supported(const IndexerArgs& a) {
     const bool fp8 = a.kI_dt == DT_E4M3 && (a.qI_dt == DT_BF16 || a.qI_dt == DT_E4M3);
     const bool bf16 = a.kI_dt == DT_BF16 && a.qI_dt == DT_BF16;
     return (fp8 || bf16) && a.d_I == kDim && a.H_I <= kHeads && a.q_pos == nullptr &&
-           a.N_cap <= 65536 && (a.N_cap % 4) == 0 && a.n_q >= 1;
+           a.N_cap <= 65536 && a.n_q >= 1;
 }
 
 cudaError_t launch_indexer_tc(const IndexerArgs& a, uint32_t* err, cudaStream_t s) {

@@ -52,15 +52,15 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits for the phase with the given parity to complete.  Spins on try_wait
-// (which suspends the thread in hardware while the phase is pending) and
-// only every 1024 tries looks at the clock and the abort flag.  Gives up
+// (which may suspend the thread in hardware for a while when the phase is
+// pending) and every 64 tries looks at the clock and the abort flag.  Gives up
 // after kWaitLimitNs or once *abort is set; on its own timeout it records
 // ERR_TIMEOUT in *err and sets *abort.  Returns false when it gave up.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint32_t* err) {
     uint64_t t0 = 0;
     while (true) {
-        for (int i = 0; i < 1024; ++i)
+        for (int i = 0; i < 64; ++i)
             if (mbar_try_wait(bar, parity)) return true;
         if (*abort) return false;
         const uint64_t now = globaltimer();

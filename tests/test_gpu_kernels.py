@@ -124,11 +124,13 @@ def _index_case(seed, B, n, H_I, d_I, kind, k, n_entries=None, q_pos=None, ties=
 
 INDEXER_CASES = [
     # (B, n, H_I, d_I, kind, k)
-    (1, 512, 1, 32, "f32", 8),
-    (2, 700, 4, 64, "bf16", 32),
+    (1, 512, 1, 32, "f32", 8),            # fp32: generic kernel
+    (2, 700, 4, 64, "bf16", 32),          # tensor-core path, ragged last tile
     (2, 901, 4, 64, "e4m3", 64),          # bf16 queries quantised in the kernel
+    (2, 912, 4, 64, "e4m3", 64),          # entry count a multiple of 4 (vector scales)
     (1, 1200, 4, 64, "e4m3_given", 100),
-    (1, 333, 16, 32, "bf16", 7),
+    (1, 4100, 2, 64, "e4m3", 300),        # two indexer heads, several CTAs
+    (1, 333, 16, 32, "bf16", 7),          # 16 heads: generic kernel
 ]
 
 
