@@ -378,6 +378,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--cpu-sample", type=int, default=4096,
                     help="queries the oracle baseline scores (bounded CPU sample)")
+    ap.add_argument("--n", type=int, default=0,
+                    help="override the prefill length (smaller cases for profiler captures; "
+                         "the line is then marked as not the headline workload)")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -385,7 +388,11 @@ def main():
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     w = synth.WORKLOADS[PREFILL]
-    config = {"workload": PREFILL, "B": w.B, "n": w.n, "H": w.H, "D": w.D, "m": w.m,
+    if args.n:
+        import dataclasses
+        w = dataclasses.replace(w, n=args.n)
+    config = {"workload": PREFILL if not args.n else f"{PREFILL} (n overridden to {args.n}: "
+                                                       "profiling case, not the headline)", "B": w.B, "n": w.n, "H": w.H, "D": w.D, "m": w.m,
               "overlap": True, "topk": w.topk, "window": w.window, "indexer": "e4m3 per-row scale",
               "H_I": w.H_I, "d_I": w.d_I, "outliers": "1% tokens x4", "seed": "rank",
               "l2": "inputs larger than L2 (q alone is 1 GiB); decode flushes L2 between steps",
