@@ -42,7 +42,12 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
 # keyed by kernel family; valid only while the kernel source hashes the same.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # profiles/attn_tc_csa_prefill_n8192.md: 153.8 MB read + 88.3 MB written at
+    # n=8192, scaled by 8 (units = queries) to one n=65536 launch
+    "sparse_attn": {"bytes": (153.758720e6 + 88.312320e6) * 8, "file": "attention_tc.cu",
+                    "src": "4a33929d631e"},
+}
 
 
 # ---------------------------------------------------------------------- helpers
