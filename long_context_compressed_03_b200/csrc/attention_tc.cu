@@ -13,13 +13,16 @@
 // same keys, so a key tile of 128 rows x 128 dims serves a whole M tile.
 //   - window tiles (and dense-mode prefix tiles) are shared by both M tiles
 //     and loaded once per CTA by 2D TMA;
-//   - sparse-mode compressed tiles belong to one token: they are fetched
-//     with TMA row gathers (4 rows per instruction) straight into the
-//     128-byte-swizzled layout the tensor core reads, and the rows of the
-//     other token in the M tile are masked.
-// Roles (10 warps): warp 0 issues TMA, warp 1 allocates TMEM and one lane
-// issues every MMA, warps 2-5 / 6-9 run the softmax of M tile 0 / 1 (a warp
-// reaches TMEM lanes 32*(warp%4) .. +31, so each group covers all 128 rows).
+//   - sparse-mode compressed tiles belong to one token: their rows are
+//     gathered with 16-byte cp.async copies by 128 loader threads straight
+//     into the 128-byte-swizzled layout the tensor core reads (many
+//     independent requests in flight), and the rows of the other token in
+//     the M tile are masked.
+// Roles (13 warps): warps 0-3 load (Q and contiguous tiles by TMA; the
+// sparse rows by cp.async, 16 lanes per 256-byte row, from index rows staged
+// in shared memory), warp 4 allocates TMEM and one lane issues every MMA,
+// warps 5-8 / 9-12 run the softmax of M tile 0 / 1 (a warp reaches TMEM
+// lanes 32*(warp%4) .. +31, so each group covers all 128 rows).
 // TMEM: S0 [cols 0,128), S1 [128,256), O0 [256,384), O1 [384,512).
 // S = Q K^T (M=128, N<=128, K=128 in 8 steps), P = exp2(S*scale*log2e - m)
 // in bf16 written back into the first 64 columns of S, O += P V with P read
@@ -46,8 +49,11 @@ constexpr int kD = 128;
 constexpr int kRows = 128;          // rows of an M tile
 constexpr int kTokens = 4;          // tokens per CTA
 constexpr int kBN = 128;            // keys per tile
-constexpr int kStages = 5;
-constexpr int kThreads = 320;
+constexpr int kStages = 4;
+constexpr int kLoadThreads = 128;  // warps 0-3: loaders (TMA + cp.async row gathers)
+constexpr int kMmaWarp = 4;        // warp 4: TMEM allocation + MMA issue
+constexpr int kSoftWarp0 = 5;      // warps 5-8 / 9-12: softmax of M tile 0 / 1
+constexpr int kThreads = 13 * 32;
 constexpr int kHalf = 16384;        // one 64-column half of a 128-row tile
 constexpr int kTileBytes = 32768;   // 128 rows x 128 bf16
 constexpr float kLog2e = 1.4426950408889634f;
@@ -65,12 +71,15 @@ struct __align__(8) Ctrl {
     uint32_t mask[kStages][4];      // gathered tiles: valid rows of the stage
     uint32_t tmem_base;
     int abort;
+    int load_go;               // loaders: continue with the next load
 };
 
-constexpr size_t kSmemBytes = 1024 /*align slack*/ + 2 * kTileBytes /*Q*/ +
+constexpr size_t kSmemFixed = 1024 /*align slack*/ + 2 * kTileBytes /*Q*/ +
                               kStages * kTileBytes + sizeof(Ctrl);
+// + the CTA's index rows (sparse mode): kTokens * topk int32
 
 struct TcParams {
+    const void* kv_c;          // sparse: [B, N_cap, 128] bf16 (rows gathered by cp.async)
     const int* idx;            // sparse: [B, n, topk]
     int topk;
     const int* n_entries;      // dense
@@ -258,6 +267,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint8_t* sQ = base;                                  // [2][32 KB]
     uint8_t* sK = sQ + 2 * kTileBytes;                   // [kStages][32 KB]
     Ctrl* ctl = reinterpret_cast<Ctrl*>(sK + kStages * kTileBytes);
+    int* sIdx = reinterpret_cast<int*>(ctl + 1);         // [kTokens][topk]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int tiles_per_seq = (p.n + kTokens - 1) / kTokens;
@@ -269,7 +279,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     if (threadIdx.x == 0) {
         mbar_init(&ctl->bar_q, 1);
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&ctl->full[s], 1);
+            mbar_init(&ctl->full[s], kLoadThreads + 1);
             mbar_init(&ctl->freeb[s], 1);
         }
         for (int i = 0; i < 2; ++i) {
@@ -282,7 +292,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         ctl->abort = (*reinterpret_cast<volatile uint32_t*>(p.err) != 0u) ? 1 : 0;
         fence_barrier_init();
     }
-    if (warp == 1) {
+    if (warp == kMmaWarp) {
         tmem_alloc(&ctl->tmem_base, 512);
         tmem_relinquish();
     }
@@ -291,9 +301,10 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
-        if (lane == 0) {
+    if (warp < kLoadThreads / 32) {
+        // ------------------------------------------------------------ loaders
+        const int lt = threadIdx.x;                          // 0 .. kLoadThreads-1
+        if (lt == 0) {
             prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_c);
             prefetch_tmap(&tm_w);
@@ -304,8 +315,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     tma_load_2d(sQ + mt * kTileBytes + h * kHalf, &tm_q, h * 64, qrow + mt * kRows,
                                 &ctl->bar_q);
         }
+        // the CTA's index rows, once (out-of-range tokens read as padding)
+        if (!p.dense) {
+            for (int i = lt; i < kTokens * p.topk; i += kLoadThreads) {
+                const int tok = i / p.topk, c = i - tok * p.topk;
+                const int t = t0 + tok;
+                sIdx[i] = (t < p.n) ? __ldg(p.idx + ((size_t)b * p.n + t) * p.topk + c) : -1;
+            }
+        }
+        named_sync(1, kLoadThreads);
         const int NL = total_loads(p, g);
         const int nc = p.dense ? g.Tc : 2 * g.Tc;
+        const uint8_t* kvc_rows = static_cast<const uint8_t*>(p.kv_c) + (size_t)b * p.N_cap * (kD * 2);
         int L = 0;
         for (; L < NL; ++L) {
             const int slot = L % kStages, use = L / kStages;
@@ -324,66 +345,59 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 kind = 2;
                 chunk = L - nc;
             }
-            // gathered tiles: read the index row before waiting for the slot
-            int rows[4] = {0, 0, 0, 0};
-            uint32_t w[4] = {0u, 0u, 0u, 0u};
-            if (kind == 0) {
-                const int t = t0 + token;
-                const int tq = min(t, p.n - 1);
-                const int* irow = p.idx + ((size_t)b * p.n + tq) * p.topk;
-                int sv[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const int c = chunk * kBN + lane * 4 + i;
-                    sv[i] = (c < p.topk) ? __ldg(irow + c) : -1;
-                }
-                uint32_t valid = 0;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const bool ok = (t < p.n) && sv[i] >= 0 && sv[i] < p.N_cap;
-                    rows[i] = b * p.N_cap + (ok ? sv[i] : 0);
-                    valid |= (ok ? 1u : 0u) << i;
-                }
-                // valid bit of row c = lane*4+i goes to mask word c/32, bit c%32
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t acc = (lane >> 3) == q ? (valid << ((lane & 7) * 4)) : 0u;
-                    for (int off = 16; off; off >>= 1) acc |= __shfl_xor_sync(0xffffffffu, acc, off);
-                    w[q] = acc;
-                }
+            // one thread acquires the free slot and decides for all loaders;
+            // the named barrier orders the others after it
+            if (lt == 0) {
+                const bool okw = use == 0 || mbar_wait(&ctl->freeb[slot], (use - 1) & 1, abort, p.err);
+                ctl->load_go = (okw && !*abort) ? 1 : 0;
             }
-            int okw = 1;
-            if (lane == 0 && use > 0) okw = mbar_wait(&ctl->freeb[slot], (use - 1) & 1, abort, p.err);
-            // lane 0 acquired the free slot; __syncwarp orders the other lanes after it
-            __syncwarp();
-            if (!__shfl_sync(0xffffffffu, okw, 0)) break;
+            named_sync(1, kLoadThreads);
+            if (!ctl->load_go) break;
             if (kind == 0) {
-                if (lane == 0) {
-                    for (int q = 0; q < 4; ++q) ctl->mask[slot][q] = w[q];
+                const int* ir = sIdx + token * p.topk + chunk * kBN;
+                const int tpos = t0 + token;
+                // valid-row mask: thread lt checks row lt
+                {
+                    const int c = chunk * kBN + lt;
+                    const int sv = (c < p.topk) ? ir[lt] : -1;
+                    const bool ok = tpos < p.n && sv >= 0 && sv < p.N_cap;
+                    const uint32_t bits = __ballot_sync(0xffffffffu, ok);
+                    if (lane == 0) ctl->mask[slot][warp] = bits;
+                }
+                // rows: 16 lanes per 256-byte row, 8 rows per round, 16 rounds
+                const int c16 = lt & 15, half = c16 >> 3, cc = c16 & 7;
+#pragma unroll 4
+                for (int it = 0; it < kBN / 8; ++it) {
+                    const int row = it * 8 + (lt >> 4);
+                    const int c = chunk * kBN + row;
+                    int sv = (c < p.topk) ? ir[row] : -1;
+                    if (tpos >= p.n || sv < 0 || sv >= p.N_cap) sv = 0;   // masked; any valid row
+                    const uint8_t* src = kvc_rows + (size_t)sv * (kD * 2) + c16 * 16;
+                    cp_async16(dst + half * kHalf + row * 128 + ((cc ^ (row & 7)) << 4), src);
+                }
+                cp_async_arrive_noinc(&ctl->full[slot]);
+                named_sync(1, kLoadThreads);                 // every mask word is written
+                if (lt == 0) mbar_arrive(&ctl->full[slot]);  // releases the mask
+            } else {
+                if (lt == 0) {
+                    const CUtensorMap* tm = (kind == 1) ? &tm_c : &tm_w;
+                    const int row = (kind == 1) ? b * p.N_cap + chunk * kBN
+                                                : b * p.L_raw + g.p_lo + chunk * kBN;
                     mbar_arrive_expect_tx(&ctl->full[slot], kTileBytes);
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_2d(dst + h * kHalf, tm, h * 64, row, &ctl->full[slot]);
                 }
-                __syncwarp();
-                // every lane fetches its own four rows, both 64-column halves
-                for (int h = 0; h < 2; ++h)
-                    tma_gather4(dst + h * kHalf + lane * 4 * 128, &tm_c, h * 64, rows[0], rows[1],
-                                rows[2], rows[3], &ctl->full[slot]);
-            } else if (lane == 0) {
-                const CUtensorMap* tm = (kind == 1) ? &tm_c : &tm_w;
-                const int row = (kind == 1) ? b * p.N_cap + chunk * kBN
-                                            : b * p.L_raw + g.p_lo + chunk * kBN;
-                mbar_arrive_expect_tx(&ctl->full[slot], kTileBytes);
-                for (int h = 0; h < 2; ++h)
-                    tma_load_2d(dst + h * kHalf, tm, h * 64, row, &ctl->full[slot]);
+                mbar_arrive(&ctl->full[slot]);
             }
-            __syncwarp();
         }
-        // drain: loads still in flight must land before the CTA exits
-        if (lane == 0)
+        // drain: copies still in flight must land before the CTA exits
+        cp_async_wait_all();
+        if (lt == 0)
             for (int Lp = max(0, L - kStages); Lp < L; ++Lp) {
                 volatile int never = 0;
                 mbar_wait(&ctl->full[Lp % kStages], (Lp / kStages) & 1, &never, p.err);
             }
-    } else if (warp == 1) {
+    } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer
         if (lane == 0) {
             const uint32_t id_qk_full = idesc_bf16(kRows, kBN, false, false);
@@ -433,7 +447,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         __syncwarp();
     } else {
         // ------------------------------------------------------------ softmax
-        const int mt = (warp - 2) >> 2;
+        const int mt = (warp - kSoftWarp0) >> 2;
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;                   // row of the M tile
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
@@ -556,7 +570,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 1) tmem_dealloc(tmem, 512);
+    if (warp == kMmaWarp) tmem_dealloc(tmem, 512);
 }
 
 // ---------------------------------------------------------------------- host
@@ -592,7 +606,7 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows)
 bool attention_tc_supported(const AttnArgs& a) {
     return a.dt == DT_BF16 && a.H == kH && a.D == kD && a.q_pos == nullptr &&
            a.raw_pos0 == nullptr && a.raw_len == nullptr && a.L_raw >= a.n_q && a.n_q > 0 &&
-           a.topk <= 2048;
+           a.topk <= 1024;   // the CTA's index rows are staged in shared memory
 }
 
 cudaError_t launch_attention_tc(const AttnArgs& a, uint32_t* err, cudaStream_t s) {
@@ -606,6 +620,7 @@ cudaError_t launch_attention_tc(const AttnArgs& a, uint32_t* err, cudaStream_t s
         !make_map(&tm_w, a.kv_raw, w_rows, 128))
         return cudaErrorInvalidValue;
     TcParams p;
+    p.kv_c = kvc;
     p.idx = a.idx;
     p.topk = a.dense ? 0 : a.topk;
     p.n_entries = a.n_entries;
@@ -620,11 +635,12 @@ cudaError_t launch_attention_tc(const AttnArgs& a, uint32_t* err, cudaStream_t s
     p.out = static_cast<__nv_bfloat16*>(a.out);
     p.lse = a.lse_out;
     p.err = err;
+    const size_t smem = kSmemFixed + (a.dense ? 0 : (size_t)kTokens * a.topk * sizeof(int));
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)kSmemBytes);
+                                         (int)smem);
     if (e != cudaSuccess) return e;
     const int tiles = (a.n_q + kTokens - 1) / kTokens;
-    attn_tc_kernel<<<(unsigned)(a.B * tiles), kThreads, kSmemBytes, s>>>(tm_q, tm_c, tm_w, p);
+    attn_tc_kernel<<<(unsigned)(a.B * tiles), kThreads, smem, s>>>(tm_q, tm_c, tm_w, p);
     count_launch();
     return cudaGetLastError();
 }
