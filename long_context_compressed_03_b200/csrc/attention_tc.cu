@@ -50,10 +50,15 @@ constexpr int kRows = 128;          // rows of an M tile
 constexpr int kTokens = 4;          // tokens per CTA
 constexpr int kBN = 128;            // keys per tile
 constexpr int kStages = 4;
-constexpr int kLoadThreads = 128;  // warps 0-3: loaders (TMA + cp.async row gathers)
-constexpr int kMmaWarp = 4;        // warp 4: TMEM allocation + MMA issue
-constexpr int kSoftWarp0 = 5;      // warps 5-8 / 9-12: softmax of M tile 0 / 1
-constexpr int kThreads = 13 * 32;
+#ifndef CSA_ATTN_LOAD_WARPS
+#define CSA_ATTN_LOAD_WARPS 4
+#endif
+constexpr int kLoadWarps = CSA_ATTN_LOAD_WARPS;   // loaders (TMA + cp.async row gathers)
+constexpr int kLoadThreads = kLoadWarps * 32;
+constexpr int kMmaWarp = kLoadWarps;               // TMEM allocation + MMA issue
+constexpr int kSoftWarp0 = kLoadWarps + 1;         // 4 + 4 softmax warps for M tiles 0 / 1
+constexpr int kThreads = (kLoadWarps + 9) * 32;
+static_assert(kLoadThreads >= 128 && kLoadThreads % 128 == 0, "loaders cover the 128 rows of a tile");
 constexpr int kHalf = 16384;        // one 64-column half of a 128-row tile
 constexpr int kTileBytes = 32768;   // 128 rows x 128 bf16
 constexpr float kLog2e = 1.4426950408889634f;
@@ -356,19 +361,20 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (kind == 0) {
                 const int* ir = sIdx + token * p.topk + chunk * kBN;
                 const int tpos = t0 + token;
-                // valid-row mask: thread lt checks row lt
-                {
+                // valid-row mask: loader thread lt < 128 checks row lt
+                if (lt < kBN) {
                     const int c = chunk * kBN + lt;
                     const int sv = (c < p.topk) ? ir[lt] : -1;
                     const bool ok = tpos < p.n && sv >= 0 && sv < p.N_cap;
                     const uint32_t bits = __ballot_sync(0xffffffffu, ok);
                     if (lane == 0) ctl->mask[slot][warp] = bits;
                 }
-                // rows: 16 lanes per 256-byte row, 8 rows per round, 16 rounds
+                // rows: 16 lanes per 256-byte row, kLoadThreads/16 rows per round
+                constexpr int kRowsPerRound = kLoadThreads / 16;
                 const int c16 = lt & 15, half = c16 >> 3, cc = c16 & 7;
 #pragma unroll 4
-                for (int it = 0; it < kBN / 8; ++it) {
-                    const int row = it * 8 + (lt >> 4);
+                for (int it = 0; it < kBN / kRowsPerRound; ++it) {
+                    const int row = it * kRowsPerRound + (lt >> 4);
                     const int c = chunk * kBN + row;
                     int sv = (c < p.topk) ? ir[row] : -1;
                     if (tpos >= p.n || sv < 0 || sv >= p.N_cap) sv = 0;   // masked; any valid row
