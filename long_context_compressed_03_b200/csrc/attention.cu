@@ -15,6 +15,7 @@
 // "virtual" keys so both share a single softmax.
 #include <math.h>
 
+#include "attn_rows.cuh"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -24,36 +25,6 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kBK = 32;
 constexpr float kLog2e = 1.4426950408889634f;
-
-struct RowKeys {
-    int n_comp;      // compressed virtual keys (idx slots or visible entries)
-    int win_lo;      // first raw row of the window
-    int n_win;       // raw rows in the window
-};
-
-__device__ __forceinline__ RowKeys row_keys(const AttnArgs& a, int row, int b, int t) {
-    RowKeys k;
-    if (a.dense) {
-        const int ne = clampi(a.n_entries ? a.n_entries[b] : a.N_cap, 0, a.N_cap);
-        k.n_comp = t < 0 ? 0 : min((t + 1) / a.m, ne);
-    } else {
-        k.n_comp = a.topk;
-    }
-    const int p0 = a.raw_pos0 ? a.raw_pos0[b] : 0;
-    const int len = clampi(a.raw_len ? a.raw_len[b] : a.L_raw, 0, a.L_raw);
-    // positions [max(0, t-W+1), t] ∩ [max(p0, 0), p0 + len - 1], as raw rows
-    long lo = max((long)t - a.window + 1, 0L);
-    lo = max(lo, (long)max(p0, 0));
-    long hi = min((long)t, (long)p0 + len - 1);
-    if (a.window <= 0 || hi < lo) {
-        k.win_lo = 0;
-        k.n_win = 0;
-    } else {
-        k.win_lo = (int)(lo - p0);
-        k.n_win = (int)(hi - lo + 1);
-    }
-    return k;
-}
 
 template <typename T, int H, int D>
 __global__ void __launch_bounds__(kThreads) attn_generic_kernel(AttnArgs a) {
@@ -71,7 +42,7 @@ __global__ void __launch_bounds__(kThreads) attn_generic_kernel(AttnArgs a) {
     const int row = blockIdx.x;
     const int b = row / a.n_q;
     const int t = a.q_pos ? a.q_pos[row] : row - b * a.n_q;
-    const RowKeys rk = row_keys(a, row, b, t);
+    const RowKeys rk = row_keys(a, b, t);
     const int total = rk.n_comp + rk.n_win;
 
     const T* q = static_cast<const T*>(a.q) + (size_t)row * H * D;
@@ -199,6 +170,7 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s, const char** why
         if (!err) return cudaErrorUnknown;
         return launch_attention_tc(a, err, s);
     }
+    if (attention_split_supported(a)) return launch_attention_split(a, s);
     if (a.dt == DT_F32) return launch_dims<float>(a, s, why);
     if (a.dt == DT_BF16) return launch_dims<__nv_bfloat16>(a, s, why);
     *why = "attention: dt must be F32 or BF16";

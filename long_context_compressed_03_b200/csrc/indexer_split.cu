@@ -1,0 +1,374 @@
+// indexer_split.cu -- stage 2 for few query rows (decode): indexer scores and
+// the exact causal top-k, with one row's visible entries split over the CTAs
+// of a thread-block cluster.
+//
+// score[t, s] = sum_h ReLU(qI[t, h] . kI[s]),  s < V(t) = min(floor((t+1)/m), n_entries)
+// idx[t, :]   = the topk largest scores, equal scores lowest index first, -1 padded
+// ("百万上下文从「奢侈品」变「日用品」…" §3.2 indexer score and top-k, §8.2
+//  selection without materialising the score matrix; "DS-V4 分析&学习" §1.2,
+//  §4 fp8 indexer keys with per-row scales.)
+//
+// A decode row scores up to N_cap fp8 keys (about 68 bytes each with the
+// scale) and keeps only topk, so the step streams the key cache once.  Row r
+// is served by a C-CTA cluster; CTA c owns the contiguous entry range
+// [c ch, (c+1) ch) and
+//   * scores it with e4m3 mma.sync (m16n8k32, fp32 accumulate): the key rows
+//     are the A operand loaded straight from global memory, 16 bytes per
+//     thread and row, and the query codes of up to 8 heads are the B
+//     operand; both sides use the same permutation of the d_I axis, which a
+//     dot product does not see.  Each score is kept in shared memory as the
+//     bit pattern of a non-negative fp32 value, which orders like the value;
+//   * runs a four-digit MSB-first radix select together with its peers: each
+//     CTA histograms its own keys, the 256-bin histograms are summed over
+//     DSMEM after a cluster barrier, and every CTA derives the same digit, so
+//     all agree on the exact k-th largest key K and on how many keys equal
+//     to K are taken;
+//   * writes its keys > K and its share of the lowest-index keys == K at
+//     offsets given by the counts of the lower-ranked CTAs (ties therefore
+//     resolve to the lowest indices across the whole row, and the output is
+//     identical from call to call).
+// The query row is quantised per head in fp32 exactly as the oracle does
+// (scale = amax / 448, codes rounded to nearest even, saturating) unless
+// codes and scales are given.
+#include <cooperative_groups.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace cg = cooperative_groups;
+
+namespace csa {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+constexpr int kMaxHeads = 8;       // one n8 block of the MMA
+constexpr int kGroup = 32;         // entries per warp step (two m16 tiles)
+constexpr int kMaxChunk = 48 * 1024;   // scores per CTA held in shared memory
+static_assert(kWarps == kMaxHeads, "one warp quantises one query head");
+
+struct SplitShared {
+    unsigned hist[2][256];
+    unsigned tot[256];
+    unsigned warp_tot[2][kWarps];
+    unsigned cnt[2];               // this CTA's keys > K and == K (read by the peers)
+    unsigned digit, rank, off_gt, off_eq;
+    float qs[kMaxHeads];
+    alignas(16) uint8_t qc[kMaxHeads * 128];   // query codes [head][d_I]
+};
+
+// D(16x8, f32) += A(16x32, e4m3, row) * B(32x8, e4m3, col)
+__device__ __forceinline__ void mma_e4m3(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Sum over the four lanes of a quad (lanes 4g .. 4g+3).
+__device__ __forceinline__ float quad_sum(float v) {
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    v += __shfl_xor_sync(0xffffffffu, v, 2);
+    return v;
+}
+
+template <int NU>
+struct Rows {              // one warp step: rows g, g+8, g+16, g+24 of a 32-entry group
+    uint4 u[4][NU];
+    float sc;              // scale of the entry this thread finalises
+};
+
+template <int NU>
+__device__ __forceinline__ void load_rows(Rows<NU>& r, const uint8_t* kb, const float* ksc, int base, int hi,
+                                          int g, int tq, int wsel) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int e = base + g + 8 * q;
+#pragma unroll
+        for (int nu = 0; nu < NU; ++nu)
+            r.u[q][nu] = e < hi ? __ldcs(reinterpret_cast<const uint4*>(kb + (size_t)e * (64 * NU) + 64 * nu + 16 * tq))
+                                : make_uint4(0u, 0u, 0u, 0u);
+    }
+    const int ew = base + wsel;
+    r.sc = ew < hi ? __ldcs(ksc + ew) : 0.0f;
+}
+
+template <int QD, int NU>
+__global__ void __launch_bounds__(kThreads) indexer_split_kernel(IndexerArgs a) {
+    extern __shared__ unsigned keys[];      // [ch] score keys of this CTA's entries
+    __shared__ SplitShared sh;
+    cg::cluster_group cluster = cg::this_cluster();
+    const int C = (int)cluster.num_blocks();
+    const int rank = (int)cluster.block_rank();
+    constexpr int d = 64 * NU;
+
+    const int row = blockIdx.y;
+    const int b = row / a.n_q;
+    const int H = a.H_I, topk = a.topk;
+    int* out = a.idx_out + (size_t)row * topk;
+    const int t = a.q_pos ? a.q_pos[row] : row - b * a.n_q;
+    const int ne = clampi(a.n_entries ? a.n_entries[b] : a.N_cap, 0, a.N_cap);
+    const int V = t < 0 ? 0 : min((t + 1) / a.m, ne);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    if (V <= topk) {        // every CTA of the cluster takes this branch together
+        for (int j = rank * kThreads + tid; j < topk; j += C * kThreads) out[j] = j < V ? j : -1;
+        return;
+    }
+    const int ch = ((V + C - 1) / C + kGroup - 1) / kGroup * kGroup;
+    const int lo = min(V, rank * ch), hi = min(V, lo + ch);
+    const int nloc = hi - lo;
+
+    // ---- query codes and per-head scales (heads >= H_I are zero)
+    if constexpr (QD == DT_E4M3) {
+        const uint8_t* src = static_cast<const uint8_t*>(a.qI) + (size_t)row * H * d;
+        for (int p = tid; p < kMaxHeads * d; p += kThreads) sh.qc[p] = p < H * d ? src[p] : 0;
+        if (tid < kMaxHeads) sh.qs[tid] = tid < H ? a.qI_scale[(size_t)row * H + tid] : 0.0f;
+    } else {
+        const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(a.qI) + (size_t)row * H * d;
+        const int h = warp;   // kWarps == kMaxHeads
+        if (h < H) {
+            float amax = 0.0f;
+            for (int c = lane; c < d; c += 32) amax = fmaxf(amax, fabsf(__bfloat162float(src[h * d + c])));
+            for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+            const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+            for (int c = lane; c < d; c += 32)
+                sh.qc[h * d + c] = e4m3_code(__fdiv_rn(__bfloat162float(src[h * d + c]), scale));
+            if (lane == 0) sh.qs[h] = scale;
+        } else {
+            for (int c = lane; c < d; c += 32) sh.qc[h * d + c] = 0;
+            if (lane == 0) sh.qs[h] = 0.0f;
+        }
+    }
+    __syncthreads();
+
+    // ---- scores of [lo, hi)
+    {
+        const int g = lane >> 2, tq = lane & 3;
+        // B fragments: head g, the 16 query bytes at [64 nu + 16 tq, +16)
+        uint32_t bq[NU][4];
+#pragma unroll
+        for (int nu = 0; nu < NU; ++nu) {
+            const uint4 v = *reinterpret_cast<const uint4*>(sh.qc + g * d + 64 * nu + 16 * tq);
+            bq[nu][0] = v.x; bq[nu][1] = v.y; bq[nu][2] = v.z; bq[nu][3] = v.w;
+        }
+        const float qs0 = sh.qs[2 * tq], qs1 = sh.qs[2 * tq + 1];
+        const uint8_t* kb = static_cast<const uint8_t*>(a.kI) + (size_t)b * a.N_cap * d;
+        const float* ksc = a.kI_scale + (size_t)b * a.N_cap;
+        const int wsel = (tq >> 1) * 16 + (tq & 1) * 8 + g;   // the entry this thread finalises
+        const int step = kWarps * kGroup;
+        Rows<NU> cur, nxt;
+        int base = lo + warp * kGroup;
+        if (base < hi) load_rows<NU>(cur, kb, ksc, base, hi, g, tq, wsel);
+        for (; base < hi; base += step) {
+            if (base + step < hi) load_rows<NU>(nxt, kb, ksc, base + step, hi, g, tq, wsel);
+            float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int nu = 0; nu < NU; ++nu) {
+                // A rows g / g+8 (tile 0) and g+16 / g+24 (tile 1); k slots 4tq.. <- bytes 16tq..
+                mma_e4m3(c0, cur.u[0][nu].x, cur.u[1][nu].x, cur.u[0][nu].y, cur.u[1][nu].y, bq[nu][0], bq[nu][1]);
+                mma_e4m3(c0, cur.u[0][nu].z, cur.u[1][nu].z, cur.u[0][nu].w, cur.u[1][nu].w, bq[nu][2], bq[nu][3]);
+                mma_e4m3(c1, cur.u[2][nu].x, cur.u[3][nu].x, cur.u[2][nu].y, cur.u[3][nu].y, bq[nu][0], bq[nu][1]);
+                mma_e4m3(c1, cur.u[2][nu].z, cur.u[3][nu].z, cur.u[2][nu].w, cur.u[3][nu].w, bq[nu][2], bq[nu][3]);
+            }
+            // heads 2tq, 2tq+1 of entries g, g+8, g+16, g+24
+            const float p0 = quad_sum(fmaf(qs0, relu0(c0[0]), qs1 * relu0(c0[1])));
+            const float p1 = quad_sum(fmaf(qs0, relu0(c0[2]), qs1 * relu0(c0[3])));
+            const float p2 = quad_sum(fmaf(qs0, relu0(c1[0]), qs1 * relu0(c1[1])));
+            const float p3 = quad_sum(fmaf(qs0, relu0(c1[2]), qs1 * relu0(c1[3])));
+            const float mine = tq == 0 ? p0 : (tq == 1 ? p1 : (tq == 2 ? p2 : p3));
+            const int e = base + wsel;
+            if (e < hi) keys[e - lo] = __float_as_uint(relu0(mine * cur.sc));
+            cur = nxt;
+        }
+    }
+    __syncthreads();
+
+    // ---- cluster-wide radix select: exact k-th largest key K, and how many == K to take
+    unsigned prefix = 0, pmask = 0, need = (unsigned)topk;
+    for (int rd = 0; rd < 4; ++rd) {
+        const int shift = 24 - 8 * rd;
+        unsigned* hist = sh.hist[rd & 1];   // the other buffer may still be read by peers
+        hist[tid] = 0;
+        __syncthreads();
+        for (int i = tid; i < nloc; i += kThreads) {
+            const unsigned k = keys[i];
+            if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+        }
+        cluster.sync();
+        unsigned tot = 0;
+        for (int c = 0; c < C; ++c) tot += cluster.map_shared_rank(hist, c)[tid];
+        sh.tot[tid] = tot;
+        __syncthreads();
+        if (warp == 0) {
+            // lane l owns digits 255-8l .. 248-8l (descending)
+            unsigned cnt[8], sum = 0;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) { cnt[i] = sh.tot[255 - 8 * lane - i]; sum += cnt[i]; }
+            unsigned incl = sum;
+            for (int off = 1; off < 32; off <<= 1) {
+                const unsigned v = __shfl_up_sync(0xffffffffu, incl, off);
+                if (lane >= off) incl += v;
+            }
+            const unsigned excl = incl - sum;
+            if (excl < need && need <= incl) {
+                unsigned run = excl;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    if (run < need && need <= run + cnt[i]) {
+                        sh.digit = 255u - 8u * lane - i;
+                        sh.rank = need - run;
+                    }
+                    run += cnt[i];
+                }
+            }
+        }
+        __syncthreads();
+        prefix |= sh.digit << shift;
+        pmask |= 255u << shift;
+        need = sh.rank;
+    }
+    const unsigned K = prefix;
+    const unsigned need_eq = need;                 // >= 1 keys equal to K are taken
+    const unsigned n_gt = (unsigned)topk - need_eq;
+
+    // ---- offsets of this CTA's keys among the row's keys > K and == K
+    {
+        unsigned gt = 0, eq = 0;
+        for (int i = tid; i < nloc; i += kThreads) {
+            const unsigned k = keys[i];
+            gt += k > K;
+            eq += k == K;
+        }
+        for (int off = 16; off; off >>= 1) {
+            gt += __shfl_xor_sync(0xffffffffu, gt, off);
+            eq += __shfl_xor_sync(0xffffffffu, eq, off);
+        }
+        if (lane == 0) { sh.warp_tot[0][warp] = gt; sh.warp_tot[1][warp] = eq; }
+        __syncthreads();
+        if (tid == 0) {
+            unsigned sg = 0, se = 0;
+            for (int w = 0; w < kWarps; ++w) { sg += sh.warp_tot[0][w]; se += sh.warp_tot[1][w]; }
+            sh.cnt[0] = sg;
+            sh.cnt[1] = se;
+        }
+        cluster.sync();
+        if (tid == 0) {
+            unsigned og = 0, oe = 0;
+            for (int c = 0; c < rank; ++c) {
+                const unsigned* pc = cluster.map_shared_rank(sh.cnt, c);
+                og += pc[0];
+                oe += pc[1];
+            }
+            sh.off_gt = og;
+            sh.off_eq = oe;
+        }
+        __syncthreads();
+    }
+
+    // ---- ordered emission: keys > K at [0, n_gt), the first need_eq keys == K after them
+    unsigned run_gt = sh.off_gt, run_eq = sh.off_eq;
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int base = 0; base < nloc; base += kThreads) {
+        const int i = base + tid;
+        const unsigned k = i < nloc ? keys[i] : 0u;
+        const bool gt = i < nloc && k > K;
+        const bool eq = i < nloc && k == K;
+        const unsigned bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
+        __syncthreads();     // the previous pass is done with warp_tot
+        if (lane == 0) { sh.warp_tot[0][warp] = __popc(bg); sh.warp_tot[1][warp] = __popc(be); }
+        __syncthreads();
+        unsigned off_g = 0, off_e = 0, tot_g = 0, tot_e = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+            if (w < warp) { off_g += sh.warp_tot[0][w]; off_e += sh.warp_tot[1][w]; }
+            tot_g += sh.warp_tot[0][w];
+            tot_e += sh.warp_tot[1][w];
+        }
+        if (gt) {
+            const unsigned r = run_gt + off_g + __popc(bg & lt_mask);
+            if (r < n_gt) out[r] = lo + i;
+        }
+        if (eq) {
+            const unsigned r = run_eq + off_e + __popc(be & lt_mask);
+            if (r < need_eq) out[n_gt + r] = lo + i;
+        }
+        run_gt += tot_g;
+        run_eq += tot_e;
+    }
+    cluster.sync();     // keep this CTA's shared memory alive until every peer has read it
+}
+
+int num_sms() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+// Cluster size: the largest power of two <= 16 with rows x C CTAs within four
+// per SM (enough loads in flight to keep HBM busy) and at least 256 entries
+// per CTA; larger if a row's share would not fit shared memory.
+int choose_cluster(const IndexerArgs& a) {
+    const long rows = (long)a.B * a.n_q;
+    int C = 1;
+    while (2 * C <= 16 && rows * 2 * C <= 4L * num_sms() && a.N_cap / (2 * C) >= 256) C *= 2;
+    while (C < 16 && ((long)a.N_cap + C - 1) / C > kMaxChunk) C *= 2;
+    return C;
+}
+
+long chunk_cap(const IndexerArgs& a, int C) {
+    return std::max<long>(((long)a.N_cap + C - 1) / C + kGroup - 1, kGroup) / kGroup * kGroup;
+}
+
+template <int QD, int NU>
+cudaError_t launch_t(const IndexerArgs& a, cudaStream_t s) {
+    const int C = choose_cluster(a);
+    const size_t smem = sizeof(unsigned) * (size_t)chunk_cap(a, C);
+    auto kern = indexer_split_kernel<QD, NU>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (C > 8) {
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)C, (unsigned)(a.B * a.n_q), 1);
+    cfg.blockDim = dim3(kThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)C;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, kern, a);
+    count_launch();
+    return e != cudaSuccess ? e : cudaGetLastError();
+}
+
+}  // namespace
+
+bool indexer_split_supported(const IndexerArgs& a) {
+    if (a.kI_dt != DT_E4M3 || a.kI_scale == nullptr) return false;
+    if (!(a.qI_dt == DT_BF16 || (a.qI_dt == DT_E4M3 && a.qI_scale != nullptr))) return false;
+    if ((a.d_I != 64 && a.d_I != 128) || a.H_I < 1 || a.H_I > kMaxHeads) return false;
+    if ((long)a.B * a.n_q > 65535) return false;
+    return chunk_cap(a, choose_cluster(a)) <= kMaxChunk;
+}
+
+cudaError_t launch_indexer_split(const IndexerArgs& a, cudaStream_t s) {
+    if (a.qI_dt == DT_E4M3) return a.d_I == 64 ? launch_t<DT_E4M3, 1>(a, s) : launch_t<DT_E4M3, 2>(a, s);
+    return a.d_I == 64 ? launch_t<DT_BF16, 1>(a, s) : launch_t<DT_BF16, 2>(a, s);
+}
+
+}  // namespace csa

@@ -231,14 +231,15 @@ cudaError_t launch_indexer_topk(const IndexerArgs& a, cudaStream_t s, const char
         *why = "csa_indexer_topk: H_I > 16 or d_I > 256";
         return cudaErrorNotSupported;
     }
-    if (a.N_cap > 40960) {
-        *why = "csa_indexer_topk: N_cap > 40960";
-        return cudaErrorNotSupported;
-    }
     if (indexer_tc_supported(a)) {
         uint32_t* err = device_error_word();
         if (!err) return cudaErrorUnknown;
         return launch_indexer_tc(a, err, s);
+    }
+    if (indexer_split_supported(a)) return launch_indexer_split(a, s);
+    if (a.N_cap > 40960) {
+        *why = "csa_indexer_topk: N_cap > 40960 needs fp8 keys with scales, d_I in {64, 128}, H_I <= 8";
+        return cudaErrorNotSupported;
     }
     if (a.qI_dt == DT_F32 && a.kI_dt == DT_F32) return launch_t<DT_F32, DT_F32>(a, s);
     if (a.qI_dt == DT_BF16 && a.kI_dt == DT_BF16) return launch_t<DT_BF16, DT_BF16>(a, s);

@@ -51,6 +51,16 @@ cudaError_t launch_attention_tc(const AttnArgs& a, uint32_t* err, cudaStream_t s
 bool indexer_tc_supported(const IndexerArgs& a);
 cudaError_t launch_indexer_tc(const IndexerArgs& a, uint32_t* err, cudaStream_t s);
 
+// Cluster split-KV attention for few query rows (decode): bf16, D in {64, 128},
+// H in {16, 32, 64, 128}.
+bool attention_split_supported(const AttnArgs& a);
+cudaError_t launch_attention_split(const AttnArgs& a, cudaStream_t s);
+
+// Cluster split indexer + exact top-k for few query rows (decode): fp8 keys
+// with per-row scales, d_I in {64, 128}, H_I <= 8.
+bool indexer_split_supported(const IndexerArgs& a);
+cudaError_t launch_indexer_split(const IndexerArgs& a, cudaStream_t s);
+
 // Counts one kernel launch (read back through csa_kernel_launches()).
 void count_launch();
 
