@@ -224,18 +224,22 @@ __global__ void __launch_bounds__(H * 2, min_blocks<H>()) attn_split_kernel(Attn
                 }
             }
         }
-        // ---- mask, online softmax (rows g and g + 8 of the warp's heads)
+        // ---- mask (only tiles with invalid slots), online softmax (rows g, g + 8)
         const uint32_t v_lo = sValid[j * 2], v_hi = sValid[j * 2 + 1];
+        if ((v_lo & v_hi) != 0xffffffffu) {
+#pragma unroll
+            for (int nb = 0; nb < 8; ++nb) {
+                const uint32_t word = nb < 4 ? v_lo : v_hi;
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int bit = (nb & 3) * 8 + 2 * tq + (e & 1);
+                    if (!((word >> bit) & 1u)) s[nb][e] = -INFINITY;
+                }
+            }
+        }
         float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
         for (int nb = 0; nb < 8; ++nb) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int key = nb * 8 + 2 * tq + (e & 1);
-                const uint32_t word = key < 32 ? v_lo : v_hi;
-                const bool ok = (word >> (key & 31)) & 1u;
-                s[nb][e] = ok ? s[nb][e] * sl2 : -INFINITY;
-            }
             mx0 = fmaxf(mx0, fmaxf(s[nb][0], s[nb][1]));
             mx1 = fmaxf(mx1, fmaxf(s[nb][2], s[nb][3]));
         }
@@ -243,18 +247,19 @@ __global__ void __launch_bounds__(H * 2, min_blocks<H>()) attn_split_kernel(Attn
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+        // running maxima are kept in the scaled base-2 domain (sl2 > 0 keeps the order)
+        const float n0 = fmaxf(m0, mx0 * sl2), n1 = fmaxf(m1, mx1 * sl2);
         const float al0 = n0 == -INFINITY ? 1.0f : exp2f(m0 - n0);
         const float al1 = n1 == -INFINITY ? 1.0f : exp2f(m1 - n1);
         m0 = n0;
         m1 = n1;
+        const float z0 = n0 == -INFINITY ? 0.0f : n0, z1 = n1 == -INFINITY ? 0.0f : n1;
         float r0 = 0.f, r1 = 0.f, e0 = 0.f, e1 = 0.f;
 #pragma unroll
         for (int nb = 0; nb < 8; ++nb) {
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-                const float mm = e < 2 ? n0 : n1;
-                const float p = s[nb][e] == -INFINITY ? 0.0f : exp2f(s[nb][e] - mm);
+                const float p = exp2f(fmaf(s[nb][e], sl2, -(e < 2 ? z0 : z1)));   // masked: exp2(-inf) = 0
                 const float pr = __bfloat162float(__float2bfloat16_rn(p));
                 s[nb][e] = pr;                       // the weight the PV product uses
                 if (e < 2) { r0 += pr; e0 += p; } else { r1 += pr; e1 += p; }
@@ -264,10 +269,12 @@ __global__ void __launch_bounds__(H * 2, min_blocks<H>()) attn_split_kernel(Attn
         lr1 = lr1 * al1 + r1;
         le0 = le0 * al0 + e0;
         le1 = le1 * al1 + e1;
+        if (!__all_sync(0xffffffffu, al0 == 1.0f && al1 == 1.0f)) {
 #pragma unroll
-        for (int i = 0; i < kND; ++i) {
-            o[i][0] *= al0; o[i][1] *= al0;
-            o[i][2] *= al1; o[i][3] *= al1;
+            for (int i = 0; i < kND; ++i) {
+                o[i][0] *= al0; o[i][1] *= al0;
+                o[i][2] *= al1; o[i][3] *= al1;
+            }
         }
         // ---- O += P V (V = the same key rows)
         {
@@ -318,23 +325,33 @@ __global__ void __launch_bounds__(H * 2, min_blocks<H>()) attn_split_kernel(Attn
     for (int it = tid; it < hpc * (D / 4); it += kThreads) {
         const int hl = it / (D / 4), d4 = it - hl * (D / 4);
         const int h = rank * hpc + hl;
+        // every peer's state and slice is requested before any is combined
+        RowState st[16];
+        float4 v[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            if (c < C) {
+                st[c] = cluster.map_shared_rank(sSt, c)[h];
+                v[c] = *reinterpret_cast<const float4*>(cluster.map_shared_rank(sO, c) + h * kOS + d4 * 4);
+            } else {
+                st[c] = RowState{-INFINITY, 0.f, 0.f};
+                v[c] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+        }
         float M = -INFINITY;
-        for (int c = 0; c < C; ++c) M = fmaxf(M, cluster.map_shared_rank(sSt, c)[h].m);
+#pragma unroll
+        for (int c = 0; c < 16; ++c) M = fmaxf(M, st[c].m);
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         float lr = 0.f, le = 0.f;
-        if (M != -INFINITY) {
-            for (int c = 0; c < C; ++c) {
-                const RowState st = cluster.map_shared_rank(sSt, c)[h];
-                if (st.m == -INFINITY) continue;
-                const float w = exp2f(st.m - M);
-                const float4 v = *reinterpret_cast<const float4*>(cluster.map_shared_rank(sO, c) + h * kOS + d4 * 4);
-                acc.x = fmaf(w, v.x, acc.x);
-                acc.y = fmaf(w, v.y, acc.y);
-                acc.z = fmaf(w, v.z, acc.z);
-                acc.w = fmaf(w, v.w, acc.w);
-                lr = fmaf(w, st.lr, lr);
-                le = fmaf(w, st.le, le);
-            }
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+            const float w = st[c].m == -INFINITY ? 0.0f : exp2f(st[c].m - M);
+            acc.x = fmaf(w, v[c].x, acc.x);
+            acc.y = fmaf(w, v[c].y, acc.y);
+            acc.z = fmaf(w, v[c].z, acc.z);
+            acc.w = fmaf(w, v[c].w, acc.w);
+            lr = fmaf(w, st[c].lr, lr);
+            le = fmaf(w, st[c].le, le);
         }
         const float inv = lr > 0.f ? 1.0f / lr : 0.0f;
         T16* out = static_cast<T16*>(a.out) + ((size_t)row * H + h) * D + d4 * 4;

@@ -250,6 +250,70 @@ __device__ __forceinline__ void tile_exp(uint32_t s_addr, const uint32_t vm[4], 
     }
 }
 
+__device__ __forceinline__ float max3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    return (uint64_t)__float_as_uint(lo) | ((uint64_t)__float_as_uint(hi) << 32);
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+
+// tile_max for a row whose 128 columns are all keys: the max of S, scaled
+// once (the scale is positive, so the maximum element is the same).
+__device__ __forceinline__ float tile_max_full(uint32_t s_addr, float sl2) {
+    float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+        float sv[32];
+        tmem_ld32(s_addr + q * 32, sv);
+#pragma unroll
+        for (int i = 0; i < 32; i += 4) {
+            mx0 = max3(mx0, sv[i], sv[i + 1]);
+            mx1 = max3(mx1, sv[i + 2], sv[i + 3]);
+        }
+    }
+    return fmaxf(mx0, mx1) * sl2;
+}
+
+// tile_exp for a row whose 128 columns are all keys, on packed f32x2 math:
+// z = S * scale - m in one rounding, P = 2^z, the rounded weights summed in
+// pairs; the exact sum only when the log-sum-exp is wanted.
+__device__ __forceinline__ void tile_exp_full(uint32_t s_addr, float sl2, float m, bool want_se,
+                                              float& se, float& sr) {
+    const uint64_t sl2x2 = f2_pack(sl2, sl2), negm = f2_pack(-m, -m);
+    uint64_t accr = 0, acce = 0;      // (+0, +0)
+#pragma unroll 1
+    for (int q = 0; q < 4; ++q) {
+        float sv[32];
+        tmem_ld32(s_addr + q * 32, sv);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+            const uint64_t z = f2_fma(f2_pack(sv[e], sv[e + 1]), sl2x2, negm);
+            const float p0 = ex2(__uint_as_float((uint32_t)z)), p1 = ex2(__uint_as_float((uint32_t)(z >> 32)));
+            __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+            const uint32_t hb = *reinterpret_cast<uint32_t*>(&h2);
+            pk[e >> 1] = hb;
+            accr = f2_add(accr, f2_pack(__uint_as_float(hb << 16), __uint_as_float(hb & 0xffff0000u)));
+            if (want_se) acce = f2_add(acce, f2_pack(p0, p1));
+        }
+        tmem_st16(s_addr + q * 16, pk);
+    }
+    sr += __uint_as_float((uint32_t)accr) + __uint_as_float((uint32_t)(accr >> 32));
+    se += __uint_as_float((uint32_t)acce) + __uint_as_float((uint32_t)(acce >> 32));
+}
+
 // The row max rose by more than 2^8 (or a row sees its first keys): rescale
 // the sums and O.  alpha = 0 for a row without earlier keys.
 __device__ __noinline__ void rescale_o(uint32_t o_addr, float alpha) {
@@ -514,7 +578,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             } else {
                 // pass 1: the tile's row max; raise the running max (and
                 // rescale O) when it grows by more than 2^8
-                const float mx = tile_max(s_addr, vm, p.scale_log2);
+                const bool full = (vm[0] & vm[1] & vm[2] & vm[3]) == 0xffffffffu;   // uniform per warp
+                const float mx = full ? tile_max_full(s_addr, p.scale_log2) : tile_max(s_addr, vm, p.scale_log2);
                 const bool raise = mx > m_used + kRescaleLog2;   // true for a row's first keys
                 float alpha = 1.0f;
                 if (raise) {
@@ -525,7 +590,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 }
                 if (j > 0 && __any_sync(0xffffffffu, raise)) rescale_o(o_addr, alpha);
                 // pass 2: P = exp2(z - m_used) over S
-                tile_exp(s_addr, vm, p.scale_log2, (m_used == -INFINITY) ? INFINITY : m_used, se, sr);
+                const float mm = (m_used == -INFINITY) ? INFINITY : m_used;
+                if (full)
+                    tile_exp_full(s_addr, p.scale_log2, mm, p.lse != nullptr, se, sr);
+                else
+                    tile_exp(s_addr, vm, p.scale_log2, mm, se, sr);
                 l_r += sr;
                 l_e += se;
             }

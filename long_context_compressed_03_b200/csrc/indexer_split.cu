@@ -18,11 +18,11 @@
 //     operand; both sides use the same permutation of the d_I axis, which a
 //     dot product does not see.  Each score is kept in shared memory as the
 //     bit pattern of a non-negative fp32 value, which orders like the value;
-//   * runs a four-digit MSB-first radix select together with its peers: each
-//     CTA histograms its own keys, the 256-bin histograms are summed over
-//     DSMEM after a cluster barrier, and every CTA derives the same digit, so
-//     all agree on the exact k-th largest key K and on how many keys equal
-//     to K are taken;
+//   * runs a four-digit MSB-first radix select (8-bit digits of the 31-bit
+//     non-negative keys) together with its peers: each CTA histograms
+//     its own keys, the histograms are summed over DSMEM after a cluster
+//     barrier, and every CTA derives the same digit, so all agree on the
+//     exact k-th largest key K and on how many keys equal to K are taken;
 //   * writes its keys > K and its share of the lowest-index keys == K at
 //     offsets given by the counts of the lower-ranked CTAs (ties therefore
 //     resolve to the lowest indices across the whole row, and the output is
@@ -48,12 +48,16 @@ constexpr int kMaxHeads = 8;       // one n8 block of the MMA
 constexpr int kGroup = 32;         // entries per warp step (two m16 tiles)
 constexpr int kMaxChunk = 48 * 1024;   // scores per CTA held in shared memory
 static_assert(kWarps == kMaxHeads, "one warp quantises one query head");
+// Radix digits of the 31-bit keys: bits 30-23, 22-15, 14-7 and 7-0 (the last
+// digit repeats bit 7, which the third round fixed).  Four 256-bin rounds
+// measured faster than three rounds of 2048 / 1024 bins.
+constexpr int kRounds = 4;
+__device__ __forceinline__ int round_shift(int rd) { return rd == 0 ? 23 : (rd == 1 ? 15 : (rd == 2 ? 7 : 0)); }
+__device__ __forceinline__ int round_bits(int) { return 8; }
 
 struct SplitShared {
-    unsigned hist[2][256];
-    unsigned tot[256];
     unsigned warp_tot[2][kWarps];
-    unsigned cnt[2];               // this CTA's keys > K and == K (read by the peers)
+    alignas(8) unsigned cnt[2];    // this CTA's keys > K and == K (read by the peers)
     unsigned digit, rank, off_gt, off_eq;
     float qs[kMaxHeads];
     alignas(16) uint8_t qc[kMaxHeads * 128];   // query codes [head][d_I]
@@ -95,9 +99,15 @@ __device__ __forceinline__ void load_rows(Rows<NU>& r, const uint8_t* kb, const 
     r.sc = ew < hi ? __ldcs(ksc + ew) : 0.0f;
 }
 
+// Resident CTAs per SM the register budget is sized for (d_I = 64: four).
+template <int NU>
+constexpr int min_blocks() { return NU == 1 ? 4 : 2; }
+
 template <int QD, int NU>
-__global__ void __launch_bounds__(kThreads) indexer_split_kernel(IndexerArgs a) {
-    extern __shared__ unsigned keys[];      // [ch] score keys of this CTA's entries
+__global__ void __launch_bounds__(kThreads, min_blocks<NU>()) indexer_split_kernel(IndexerArgs a) {
+    extern __shared__ __align__(16) unsigned dyn[];   // [2][256] histograms, then [ch] keys
+    unsigned* hist_buf = dyn;
+    unsigned* keys = dyn + 2 * 256;                   // score keys of this CTA's entries
     __shared__ SplitShared sh;
     cg::cluster_group cluster = cg::this_cluster();
     const int C = (int)cluster.num_blocks();
@@ -186,58 +196,90 @@ __global__ void __launch_bounds__(kThreads) indexer_split_kernel(IndexerArgs a) 
     }
     __syncthreads();
 
-    // ---- cluster-wide radix select: exact k-th largest key K, and how many == K to take
+    // ---- cluster-wide radix select: exact k-th largest key K, and how many == K to take.
+    // Keys are non-negative fp32 bit patterns (bit 31 clear); the digits of
+    // kShift / kBits settle all 31 bits (a digit may repeat bits an earlier
+    // round fixed: they match the prefix).
     unsigned prefix = 0, pmask = 0, need = (unsigned)topk;
-    for (int rd = 0; rd < 4; ++rd) {
-        const int shift = 24 - 8 * rd;
-        unsigned* hist = sh.hist[rd & 1];   // the other buffer may still be read by peers
-        hist[tid] = 0;
+#pragma unroll 1
+    for (int rd = 0; rd < kRounds; ++rd) {
+        const int shift = round_shift(rd);
+        const int nbins = 1 << round_bits(rd);
+        const unsigned dmask = (unsigned)nbins - 1u;
+        unsigned* hist = hist_buf + (rd & 1) * 256;    // the other buffer may still be read by peers
+        for (int i = tid; i < nbins; i += kThreads) hist[i] = 0;
         __syncthreads();
         for (int i = tid; i < nloc; i += kThreads) {
             const unsigned k = keys[i];
-            if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+            if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & dmask], 1u);
         }
         cluster.sync();
-        unsigned tot = 0;
-        for (int c = 0; c < C; ++c) tot += cluster.map_shared_rank(hist, c)[tid];
-        sh.tot[tid] = tot;
-        __syncthreads();
-        if (warp == 0) {
-            // lane l owns digits 255-8l .. 248-8l (descending)
-            unsigned cnt[8], sum = 0;
+        // thread t owns the bpt bins just below nbins - bpt t (highest digits first)
+        const int bpt = nbins / kThreads;            // 1, 4 or 8
+        const int b0 = nbins - bpt * (tid + 1);
+        unsigned cnt[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) { cnt[i] = sh.tot[255 - 8 * lane - i]; sum += cnt[i]; }
-            unsigned incl = sum;
-            for (int off = 1; off < 32; off <<= 1) {
-                const unsigned v = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += v;
-            }
-            const unsigned excl = incl - sum;
-            if (excl < need && need <= incl) {
-                unsigned run = excl;
+        for (int i = 0; i < 8; ++i) cnt[i] = 0;
 #pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    if (run < need && need <= run + cnt[i]) {
-                        sh.digit = 255u - 8u * lane - i;
-                        sh.rank = need - run;
+        for (int c = 0; c < 16; ++c) {               // every peer's bins requested before use
+            if (c < C) {
+                const unsigned* ph = cluster.map_shared_rank(hist, c) + b0;
+                if (bpt == 1) {
+                    cnt[0] += *ph;
+                } else {
+                    const uint4 lo4 = *reinterpret_cast<const uint4*>(ph);
+                    cnt[0] += lo4.x; cnt[1] += lo4.y; cnt[2] += lo4.z; cnt[3] += lo4.w;
+                    if (bpt == 8) {
+                        const uint4 hi4 = *reinterpret_cast<const uint4*>(ph + 4);
+                        cnt[4] += hi4.x; cnt[5] += hi4.y; cnt[6] += hi4.z; cnt[7] += hi4.w;
                     }
-                    run += cnt[i];
                 }
+            }
+        }
+        unsigned sum = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sum += cnt[i];
+        // block-wide inclusive scan of the per-thread sums, in thread order
+        unsigned incl = sum;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const unsigned v = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += v;
+        }
+        if (lane == 31) sh.warp_tot[0][warp] = incl;
+        __syncthreads();
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w)
+            if (w < warp) incl += sh.warp_tot[0][w];
+        const unsigned excl = incl - sum;
+        if (excl < need && need <= incl) {
+            unsigned run = excl;
+            // this thread's bins in descending digit order: b0 + bpt - 1 down to b0
+#pragma unroll
+            for (int i = 7; i >= 0; --i) {
+                if (i < bpt && run < need && need <= run + cnt[i]) {
+                    sh.digit = (unsigned)(b0 + i);
+                    sh.rank = need - run;
+                }
+                if (i < bpt) run += cnt[i];
             }
         }
         __syncthreads();
         prefix |= sh.digit << shift;
-        pmask |= 255u << shift;
+        pmask |= dmask << shift;
         need = sh.rank;
+        __syncthreads();     // warp_tot and digit are rewritten next round
     }
     const unsigned K = prefix;
     const unsigned need_eq = need;                 // >= 1 keys equal to K are taken
     const unsigned n_gt = (unsigned)topk - need_eq;
 
-    // ---- offsets of this CTA's keys among the row's keys > K and == K
+    // ---- each warp owns a contiguous block of this CTA's keys; count, then emit in order
+    const int per = ((nloc + kWarps - 1) / kWarps + 31) & ~31;
+    const int w_lo = min(nloc, warp * per), w_hi = min(nloc, w_lo + per);
     {
         unsigned gt = 0, eq = 0;
-        for (int i = tid; i < nloc; i += kThreads) {
+        for (int i = w_lo + lane; i < w_hi; i += 32) {
             const unsigned k = keys[i];
             gt += k > K;
             eq += k == K;
@@ -255,48 +297,40 @@ __global__ void __launch_bounds__(kThreads) indexer_split_kernel(IndexerArgs a) 
             sh.cnt[1] = se;
         }
         cluster.sync();
-        if (tid == 0) {
-            unsigned og = 0, oe = 0;
-            for (int c = 0; c < rank; ++c) {
-                const unsigned* pc = cluster.map_shared_rank(sh.cnt, c);
-                og += pc[0];
-                oe += pc[1];
+        if (warp == 0) {     // lane c reads the counts of peer c < rank
+            uint2 pc = make_uint2(0u, 0u);
+            if (lane < rank) pc = *reinterpret_cast<const uint2*>(cluster.map_shared_rank(sh.cnt, lane));
+            for (int off = 16; off; off >>= 1) {
+                pc.x += __shfl_xor_sync(0xffffffffu, pc.x, off);
+                pc.y += __shfl_xor_sync(0xffffffffu, pc.y, off);
             }
-            sh.off_gt = og;
-            sh.off_eq = oe;
+            if (lane == 0) { sh.off_gt = pc.x; sh.off_eq = pc.y; }
         }
         __syncthreads();
     }
 
     // ---- ordered emission: keys > K at [0, n_gt), the first need_eq keys == K after them
     unsigned run_gt = sh.off_gt, run_eq = sh.off_eq;
-    const unsigned lt_mask = (1u << lane) - 1u;
-    for (int base = 0; base < nloc; base += kThreads) {
-        const int i = base + tid;
-        const unsigned k = i < nloc ? keys[i] : 0u;
-        const bool gt = i < nloc && k > K;
-        const bool eq = i < nloc && k == K;
-        const unsigned bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
-        __syncthreads();     // the previous pass is done with warp_tot
-        if (lane == 0) { sh.warp_tot[0][warp] = __popc(bg); sh.warp_tot[1][warp] = __popc(be); }
-        __syncthreads();
-        unsigned off_g = 0, off_e = 0, tot_g = 0, tot_e = 0;
 #pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-            if (w < warp) { off_g += sh.warp_tot[0][w]; off_e += sh.warp_tot[1][w]; }
-            tot_g += sh.warp_tot[0][w];
-            tot_e += sh.warp_tot[1][w];
-        }
+    for (int w = 0; w < kWarps; ++w)
+        if (w < warp) { run_gt += sh.warp_tot[0][w]; run_eq += sh.warp_tot[1][w]; }
+    const unsigned lt_mask = (1u << lane) - 1u;
+    for (int base = w_lo; base < w_hi; base += 32) {
+        const int i = base + lane;
+        const unsigned k = i < w_hi ? keys[i] : 0u;
+        const bool gt = i < w_hi && k > K;
+        const bool eq = i < w_hi && k == K;
+        const unsigned bg = __ballot_sync(0xffffffffu, gt), be = __ballot_sync(0xffffffffu, eq);
         if (gt) {
-            const unsigned r = run_gt + off_g + __popc(bg & lt_mask);
+            const unsigned r = run_gt + __popc(bg & lt_mask);
             if (r < n_gt) out[r] = lo + i;
         }
         if (eq) {
-            const unsigned r = run_eq + off_e + __popc(be & lt_mask);
+            const unsigned r = run_eq + __popc(be & lt_mask);
             if (r < need_eq) out[n_gt + r] = lo + i;
         }
-        run_gt += tot_g;
-        run_eq += tot_e;
+        run_gt += __popc(bg);
+        run_eq += __popc(be);
     }
     cluster.sync();     // keep this CTA's shared memory alive until every peer has read it
 }
@@ -313,13 +347,14 @@ int num_sms() {
     return cached[dev];
 }
 
-// Cluster size: the largest power of two <= 16 with rows x C CTAs within four
-// per SM (enough loads in flight to keep HBM busy) and at least 256 entries
-// per CTA; larger if a row's share would not fit shared memory.
+// Cluster size: the largest power of two <= 16 with rows x C CTAs within one
+// wave of resident CTAs and at least 256 entries per CTA; larger if a row's
+// share would not fit shared memory.
 int choose_cluster(const IndexerArgs& a) {
     const long rows = (long)a.B * a.n_q;
+    const long slots = (long)num_sms() * (a.d_I == 64 ? min_blocks<1>() : min_blocks<2>());
     int C = 1;
-    while (2 * C <= 16 && rows * 2 * C <= 4L * num_sms() && a.N_cap / (2 * C) >= 256) C *= 2;
+    while (2 * C <= 16 && rows * 2 * C <= slots && a.N_cap / (2 * C) >= 256) C *= 2;
     while (C < 16 && ((long)a.N_cap + C - 1) / C > kMaxChunk) C *= 2;
     return C;
 }
@@ -331,7 +366,7 @@ long chunk_cap(const IndexerArgs& a, int C) {
 template <int QD, int NU>
 cudaError_t launch_t(const IndexerArgs& a, cudaStream_t s) {
     const int C = choose_cluster(a);
-    const size_t smem = sizeof(unsigned) * (size_t)chunk_cap(a, C);
+    const size_t smem = sizeof(unsigned) * ((size_t)chunk_cap(a, C) + 2 * 256);
     auto kern = indexer_split_kernel<QD, NU>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

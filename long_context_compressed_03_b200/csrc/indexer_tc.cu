@@ -25,11 +25,10 @@
 // fire-and-forget shared atomics).  Once a row's boundary bin has
 // at most kCap keys, a final pass writes every key above the boundary to the
 // output and collects the boundary bin, which is then sorted exactly; each
-// selected row is finally sorted by entry index (a deterministic order).
+// selected row is finally rewritten in ascending entry order through a
+// bitmap (a deterministic order).
 // The score matrix never leaves the SM.
 #include <cudaTypedefs.h>
-
-#include <climits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -122,33 +121,6 @@ __device__ __forceinline__ uint64_t desc_sw(uint32_t saddr, uint32_t sbo, uint32
     return d;
 }
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float* v) {
-    uint32_t* r = reinterpret_cast<uint32_t*>(v);
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-        "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-          "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-          "=r"(r[14]), "=r"(r[15])
-        : "r"(taddr)
-        : "memory");
-}
-
-// Four heads x 16 columns (head h at column offset h*stride) with one wait.
-__device__ __forceinline__ void tmem_ld16x4(uint32_t taddr, int stride, float (*v)[16]) {
-    uint32_t* r = reinterpret_cast<uint32_t*>(&v[0][0]);
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%64];\n\t"
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%65];\n\t"
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47}, [%66];\n\t"
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%67];\n\t"
-        "tcgen05.wait::ld.sync.aligned;"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
-        : "r"(taddr), "r"(taddr + stride), "r"(taddr + 2 * stride), "r"(taddr + 3 * stride)
-        : "memory");
-}
-
 enum PassKind { kHist0 = 0, kHist32 = 1, kHist64 = 2, kEmit = 3 };
 
 struct RowCtx {
@@ -161,7 +133,6 @@ struct RowCtx {
     int* emitted;
     int* listed;
     int topk;
-    bool ks_vec;               // per-entry scales readable as float4
     float qs[kHeads];
 };
 
@@ -189,40 +160,33 @@ __device__ __forceinline__ void tmem_ld8x4(uint32_t taddr, float (*v)[8]) {
 // point, before any per-row branching; rows that are not selecting skip the
 // arithmetic.
 template <bool FP8>
-__device__ __forceinline__ void chunk_pass(uint32_t taddr, const float* ksc, int c, bool active,
+__device__ __forceinline__ void chunk_pass(uint32_t taddr, float ksv, int c, bool active,
                                            int KIND, const RowCtx& rc) {
 #pragma unroll 1
     for (int part = 0; part < kN / 8; ++part) {
         float acc[kHeads][8];
         tmem_ld8x4(taddr + part * 8, acc);
+        // lane e of the warp holds the key scale of entry c*kN + e: broadcast
+        // the part's eight before any per-row branching (warp-collective)
+        float ks[8];
+        if (FP8) {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) ks[e] = __shfl_sync(0xffffffffu, ksv, part * 8 + e);
+        }
         if (!active) continue;
         const int s0 = c * kN + part * 8;
         if (s0 >= rc.V) continue;
         const int ne = min(8, rc.V - s0);
-        float ks[8];
-        if (FP8) {
-            if (rc.ks_vec) {
-                // 16-byte aligned rows: s0 is a multiple of 8 below V <= N_cap
-                // (a multiple of 4), so the first four scales are in bounds,
-                // the next four when ne > 4
-                const float4 k0 = __ldg(reinterpret_cast<const float4*>(ksc + s0));
-                const float4 k1 = ne > 4 ? __ldg(reinterpret_cast<const float4*>(ksc + s0 + 4))
-                                         : make_float4(0.f, 0.f, 0.f, 0.f);
-                ks[0] = k0.x; ks[1] = k0.y; ks[2] = k0.z; ks[3] = k0.w;
-                ks[4] = k1.x; ks[5] = k1.y; ks[6] = k1.z; ks[7] = k1.w;
-            } else {
-#pragma unroll
-                for (int e = 0; e < 8; ++e) ks[e] = e < ne ? __ldg(ksc + s0 + e) : 0.0f;
-            }
-        }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
             if (e >= ne) break;
-            float sc = rc.qs[0] * fmaxf(acc[0][e], 0.0f);
+            // a + |a| = 2 ReLU(a) exactly (+0 for a <= 0), and rc.qs holds qs / 2, so
+            // this is sum_h qs_h ReLU(a_h) on the FMA pipe, always +0 or positive
+            float sc = rc.qs[0] * (acc[0][e] + fabsf(acc[0][e]));
 #pragma unroll
-            for (int h = 1; h < kHeads; ++h) sc = fmaf(rc.qs[h], fmaxf(acc[h][e], 0.0f), sc);
+            for (int h = 1; h < kHeads; ++h) sc = fmaf(rc.qs[h], acc[h][e] + fabsf(acc[h][e]), sc);
             if (FP8) sc *= ks[e];
-            const uint32_t sbits = __float_as_uint(sc) & 0x7FFFFFFFu;   // sc >= 0; drop a -0 sign
+            const uint32_t sbits = __float_as_uint(sc);
             if (KIND == kHist0) {
                 atomicAdd(rc.hrow + (sbits >> 24) * kRows, 1u);
             } else if (KIND == kHist32) {
@@ -430,15 +394,22 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
             rc.emitted = &rs->emitted[r];
             rc.listed = &rs->listed[r];
             rc.topk = p.topk;
-            rc.ks_vec = (p.N_cap & 3) == 0;
 #pragma unroll
-            for (int h = 0; h < kHeads; ++h) rc.qs[h] = rs->qs[r][h];
+            for (int h = 0; h < kHeads; ++h) rc.qs[h] = 0.5f * rs->qs[r][h];   // exact: a power of two
             const float* ksc = FP8 ? p.kI_scale + (size_t)b * p.N_cap : nullptr;
+            // this lane's key scale for entry c*kN + lane, loaded one chunk ahead
+            auto scale_of = [&](int c) -> float {
+                const int e = c * kN + lane;
+                return (FP8 && c < nchunks && e < Vmax) ? __ldg(ksc + e) : 0.0f;
+            };
+            float ksv = scale_of(grp);
             for (int c = grp; c < nchunks; c += kGroups) {
+                const float ksv_next = scale_of(c + kGroups);
                 if (!__all_sync(0xffffffffu, mbar_wait(&ctl->acc_full[grp], cons & 1, abort, p.err))) break;
                 tc_fence_after();
                 const uint32_t taddr = tmem + lane_addr + grp * 128;
-                chunk_pass<FP8>(taddr, ksc, c, active, kind, rc);
+                chunk_pass<FP8>(taddr, ksv, c, active, kind, rc);
+                ksv = ksv_next;
                 tc_fence_before();
                 mbar_arrive(&ctl->acc_free[grp]);
                 ++cons;
@@ -493,35 +464,44 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
         __syncthreads();
         if (emit) {
             // the emitted set is exact; its order depends on which group got
-            // there first.  Sort each selected row ascending: a deterministic
-            // (and gather-friendly) order.  One warp per row, bitonic in smem.
+            // there first.  Rewrite each selected row in ascending entry order
+            // (deterministic and gather-friendly): one warp per row marks the
+            // entries in a bitmap over [0, V) in shared memory, then walks it.
             if (is_epi) {
                 const int ew = warp - 2;
-                int* buf = reinterpret_cast<int*>(hist) + ew * 2048;   // 8 KB per warp
+                uint32_t* bm = hist + ew * 2048;                 // 8 KB per warp: V <= 65536
                 const int kk = p.topk;
-                int np2 = 1;
-                while (np2 < kk) np2 <<= 1;
                 for (int rr = ew; rr < kRows; rr += kGroups * 4) {
-                    if (t0 + rr >= p.n || rs->V[rr] <= kk) continue;
+                    const int V = rs->V[rr];
+                    if (t0 + rr >= p.n || V <= kk) continue;
                     int* orow = p.idx_out + ((size_t)b * p.n + t0 + rr) * kk;
-                    for (int i = lane; i < np2; i += 32) buf[i] = i < kk ? orow[i] : INT_MAX;
+                    const int nw = (V + 31) >> 5;
+                    for (int i = lane; i < nw; i += 32) bm[i] = 0u;
                     __syncwarp();
-                    for (int size = 2; size <= np2; size <<= 1) {
-                        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-                            for (int i = lane; i < np2 / 2; i += 32) {
-                                const int lo = 2 * i - (i & (stride - 1));
-                                const int hi = lo + stride;
-                                const bool up = (lo & size) == 0;
-                                const int a0 = buf[lo], a1 = buf[hi];
-                                if ((a0 > a1) == up) {
-                                    buf[lo] = a1;
-                                    buf[hi] = a0;
-                                }
-                            }
-                            __syncwarp();
-                        }
+                    for (int i = lane; i < kk; i += 32) {
+                        const int sidx = orow[i];
+                        if (sidx >= 0 && sidx < V) atomicOr(&bm[sidx >> 5], 1u << (sidx & 31));
                     }
-                    for (int i = lane; i < kk; i += 32) orow[i] = buf[i];
+                    __syncwarp();
+                    int basepos = 0;
+                    for (int w0 = 0; w0 < nw; w0 += 32) {
+                        uint32_t word = (w0 + lane < nw) ? bm[w0 + lane] : 0u;
+                        const int cnt = __popc(word);
+                        int incl = cnt;
+#pragma unroll
+                        for (int off = 1; off < 32; off <<= 1) {
+                            const int v = __shfl_up_sync(0xffffffffu, incl, off);
+                            if (lane >= off) incl += v;
+                        }
+                        int pos = basepos + incl - cnt;
+                        while (word) {
+                            const int bit = __ffs(word) - 1;
+                            word &= word - 1u;
+                            if (pos < kk) orow[pos] = ((w0 + lane) << 5) + bit;
+                            ++pos;
+                        }
+                        basepos += __shfl_sync(0xffffffffu, incl, 31);
+                    }
                     __syncwarp();
                 }
             }
