@@ -55,9 +55,10 @@ constexpr int kStages = 4;
 #endif
 constexpr int kLoadWarps = CSA_ATTN_LOAD_WARPS;   // loaders (TMA + cp.async row gathers)
 constexpr int kLoadThreads = kLoadWarps * 32;
-constexpr int kMmaWarp = kLoadWarps;               // TMEM allocation + MMA issue
+constexpr int kMmaWarp = kLoadWarps;               // TMEM allocation, MMA issue, Q loads
 constexpr int kSoftWarp0 = kLoadWarps + 1;         // 4 + 4 softmax warps for M tiles 0 / 1
-constexpr int kThreads = (kLoadWarps + 9) * 32;
+constexpr int kEpiWarp0 = kSoftWarp0 + 8;          // 4 + 4 epilogue warps for M tiles 0 / 1
+constexpr int kThreads = (kLoadWarps + 17) * 32;
 static_assert(kLoadThreads >= 128 && kLoadThreads % 128 == 0, "loaders cover the 128 rows of a tile");
 constexpr int kHalf = 16384;        // one 64-column half of a 128-row tile
 constexpr int kTileBytes = 32768;   // 128 rows x 128 bf16
@@ -67,6 +68,10 @@ constexpr float kRescaleLog2 = 8.0f;
 
 struct __align__(8) Ctrl {
     uint64_t bar_q;
+    uint64_t q_free;                // the unit's last QK has read Q
+    uint64_t o_full[2];             // the unit's last P.V has landed in O
+    uint64_t o_free[2];             // the epilogue has read O
+    uint64_t stats_ready[2];        // the softmax has published the unit's row statistics
     uint64_t full[kStages];
     uint64_t freeb[kStages];
     uint64_t s_full[2];
@@ -79,8 +84,12 @@ struct __align__(8) Ctrl {
     int load_go;               // loaders: continue with the next load
 };
 
+struct RowStat {            // per row of an M tile at the end of a unit
+    float m, lr, le;
+};
+constexpr size_t kStatBytes = sizeof(RowStat) * 2 /*unit parity*/ * 2 /*M tiles*/ * kRows;
 constexpr size_t kSmemFixed = 1024 /*align slack*/ + 2 * kTileBytes /*Q*/ +
-                              kStages * kTileBytes + sizeof(Ctrl);
+                              kStages * kTileBytes + sizeof(Ctrl) + kStatBytes;
 // + the CTA's index rows (sparse mode): kTokens * topk int32
 
 struct TcParams {
@@ -328,6 +337,21 @@ __device__ __noinline__ void rescale_o(uint32_t o_addr, float alpha) {
     tmem_st_wait();
 }
 
+// Units of work: unit u covers tokens [t0, t0 + 4) of sequence b, where
+// u = b * units_per_seq + t0 / 4.  The kernel is persistent: CTA c takes units
+// c, c + gridDim.x, ... in that order, and every role walks the same list, so
+// barrier phases run on across units.
+struct Unit {
+    int b, t0;
+};
+__device__ __forceinline__ Unit unit_of(const TcParams& p, int u) {
+    const int per = (p.n + kTokens - 1) / kTokens;
+    Unit r;
+    r.b = u / per;
+    r.t0 = (u - r.b * per) * kTokens;
+    return r;
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_c,
                const __grid_constant__ CUtensorMap tm_w, TcParams p) {
@@ -336,17 +360,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     uint8_t* sQ = base;                                  // [2][32 KB]
     uint8_t* sK = sQ + 2 * kTileBytes;                   // [kStages][32 KB]
     Ctrl* ctl = reinterpret_cast<Ctrl*>(sK + kStages * kTileBytes);
-    int* sIdx = reinterpret_cast<int*>(ctl + 1);         // [kTokens][topk]
+    RowStat* stats = reinterpret_cast<RowStat*>(ctl + 1);        // [2][2][kRows]
+    int* sIdx = reinterpret_cast<int*>(stats + 4 * kRows);       // [kTokens][topk]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tiles_per_seq = (p.n + kTokens - 1) / kTokens;
-    const int b = blockIdx.x / tiles_per_seq;
-    const int t0 = (blockIdx.x - b * tiles_per_seq) * kTokens;
-    const Geometry g = geometry(p, b, t0);
+    const int n_units = p.B * ((p.n + kTokens - 1) / kTokens);
     volatile int* abort = &ctl->abort;
 
     if (threadIdx.x == 0) {
         mbar_init(&ctl->bar_q, 1);
+        mbar_init(&ctl->q_free, 1);
         for (int s = 0; s < kStages; ++s) {
             mbar_init(&ctl->full[s], kLoadThreads + 1);
             mbar_init(&ctl->freeb[s], 1);
@@ -355,6 +378,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_init(&ctl->s_full[i], 1);
             mbar_init(&ctl->pv_done[i], 1);
             mbar_init(&ctl->p_ready[i], kRows);
+            mbar_init(&ctl->o_full[i], 1);
+            mbar_init(&ctl->o_free[i], kRows);
+            mbar_init(&ctl->stats_ready[i], kRows);
         }
         mbar_init(&ctl->fin, 1);
         // a CTA started after another one timed out does no work
@@ -374,140 +400,191 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         // ------------------------------------------------------------ loaders
         const int lt = threadIdx.x;                          // 0 .. kLoadThreads-1
         if (lt == 0) {
-            prefetch_tmap(&tm_q);
             prefetch_tmap(&tm_c);
             prefetch_tmap(&tm_w);
-            mbar_arrive_expect_tx(&ctl->bar_q, 2 * kTileBytes);
-            const int qrow = (b * p.n + t0) * kH;
-            for (int mt = 0; mt < 2; ++mt)
-                for (int h = 0; h < 2; ++h)
-                    tma_load_2d(sQ + mt * kTileBytes + h * kHalf, &tm_q, h * 64, qrow + mt * kRows,
-                                &ctl->bar_q);
         }
-        // the CTA's index rows, once (out-of-range tokens read as padding)
-        if (!p.dense) {
-            for (int i = lt; i < kTokens * p.topk; i += kLoadThreads) {
-                const int tok = i / p.topk, c = i - tok * p.topk;
-                const int t = t0 + tok;
-                sIdx[i] = (t < p.n) ? __ldg(p.idx + ((size_t)b * p.n + t) * p.topk + c) : -1;
-            }
-        }
-        named_sync(1, kLoadThreads);
-        const int NL = total_loads(p, g);
-        const int nc = p.dense ? g.Tc : 2 * g.Tc;
-        const uint8_t* kvc_rows = static_cast<const uint8_t*>(p.kv_c) + (size_t)b * p.N_cap * (kD * 2);
-        int L = 0;
-        for (; L < NL; ++L) {
-            const int slot = L % kStages, use = L / kStages;
-            uint8_t* dst = sK + slot * kTileBytes;
-            // which tile is load L?
-            int kind, token = 0, chunk;
-            if (L < nc) {
-                if (p.dense) { kind = 1; chunk = L; }
-                else {
-                    const int j = L >> 1, mt = L & 1;
-                    kind = 0;
-                    token = 2 * mt + j / g.cc;    // token within the CTA
-                    chunk = j - (j / g.cc) * g.cc;
+        int Lg = 0;                                          // loads issued by this CTA
+        bool go = true;
+        for (int u = blockIdx.x; u < n_units && go; u += gridDim.x) {
+            const Unit un = unit_of(p, u);
+            const int b = un.b, t0 = un.t0;
+            const Geometry g = geometry(p, b, t0);
+            // the unit's index rows (out-of-range tokens read as padding); the
+            // previous unit's gathers have all been issued
+            named_sync(1, kLoadThreads);
+            if (!p.dense) {
+                for (int i = lt; i < kTokens * p.topk; i += kLoadThreads) {
+                    const int tok = i / p.topk, c = i - tok * p.topk;
+                    const int t = t0 + tok;
+                    sIdx[i] = (t < p.n) ? __ldg(p.idx + ((size_t)b * p.n + t) * p.topk + c) : -1;
                 }
-            } else {
-                kind = 2;
-                chunk = L - nc;
-            }
-            // one thread acquires the free slot and decides for all loaders;
-            // the named barrier orders the others after it
-            if (lt == 0) {
-                const bool okw = use == 0 || mbar_wait(&ctl->freeb[slot], (use - 1) & 1, abort, p.err);
-                ctl->load_go = (okw && !*abort) ? 1 : 0;
             }
             named_sync(1, kLoadThreads);
-            if (!ctl->load_go) break;
-            if (kind == 0) {
-                const int* ir = sIdx + token * p.topk + chunk * kBN;
-                const int tpos = t0 + token;
-                // valid-row mask: loader thread lt < 128 checks row lt
-                if (lt < kBN) {
-                    const int c = chunk * kBN + lt;
-                    const int sv = (c < p.topk) ? ir[lt] : -1;
-                    const bool ok = tpos < p.n && sv >= 0 && sv < p.N_cap;
-                    const uint32_t bits = __ballot_sync(0xffffffffu, ok);
-                    if (lane == 0) ctl->mask[slot][warp] = bits;
+            const int NL = total_loads(p, g);
+            const int nc = p.dense ? g.Tc : 2 * g.Tc;
+            const uint8_t* kvc_rows = static_cast<const uint8_t*>(p.kv_c) + (size_t)b * p.N_cap * (kD * 2);
+            for (int L = 0; L < NL; ++L, ++Lg) {
+                const int slot = Lg % kStages, use = Lg / kStages;
+                uint8_t* dst = sK + slot * kTileBytes;
+                // which tile is load L of the unit?
+                int kind, token = 0, chunk;
+                if (L < nc) {
+                    if (p.dense) { kind = 1; chunk = L; }
+                    else {
+                        const int j = L >> 1, mt = L & 1;
+                        kind = 0;
+                        token = 2 * mt + j / g.cc;    // token within the unit
+                        chunk = j - (j / g.cc) * g.cc;
+                    }
+                } else {
+                    kind = 2;
+                    chunk = L - nc;
                 }
-                // rows: 16 lanes per 256-byte row, kLoadThreads/16 rows per round
-                constexpr int kRowsPerRound = kLoadThreads / 16;
-                const int c16 = lt & 15, half = c16 >> 3, cc = c16 & 7;
-#pragma unroll 4
-                for (int it = 0; it < kBN / kRowsPerRound; ++it) {
-                    const int row = it * kRowsPerRound + (lt >> 4);
-                    const int c = chunk * kBN + row;
-                    int sv = (c < p.topk) ? ir[row] : -1;
-                    if (tpos >= p.n || sv < 0 || sv >= p.N_cap) sv = 0;   // masked; any valid row
-                    const uint8_t* src = kvc_rows + (size_t)sv * (kD * 2) + c16 * 16;
-                    cp_async16(dst + half * kHalf + row * 128 + ((cc ^ (row & 7)) << 4), src);
-                }
-                cp_async_arrive_noinc(&ctl->full[slot]);
-                named_sync(1, kLoadThreads);                 // every mask word is written
-                if (lt == 0) mbar_arrive(&ctl->full[slot]);  // releases the mask
-            } else {
+                // one thread acquires the free slot and decides for all loaders;
+                // the named barrier orders the others after it
                 if (lt == 0) {
-                    const CUtensorMap* tm = (kind == 1) ? &tm_c : &tm_w;
-                    const int row = (kind == 1) ? b * p.N_cap + chunk * kBN
-                                                : b * p.L_raw + g.p_lo + chunk * kBN;
-                    mbar_arrive_expect_tx(&ctl->full[slot], kTileBytes);
-                    for (int h = 0; h < 2; ++h)
-                        tma_load_2d(dst + h * kHalf, tm, h * 64, row, &ctl->full[slot]);
+                    const bool okw = use == 0 || mbar_wait(&ctl->freeb[slot], (use - 1) & 1, abort, p.err);
+                    ctl->load_go = (okw && !*abort) ? 1 : 0;
                 }
-                mbar_arrive(&ctl->full[slot]);
+                named_sync(1, kLoadThreads);
+                if (!ctl->load_go) { go = false; break; }
+                if (kind == 0) {
+                    const int* ir = sIdx + token * p.topk + chunk * kBN;
+                    const int tpos = t0 + token;
+                    // valid-row mask: loader thread lt < 128 checks row lt
+                    if (lt < kBN) {
+                        const int c = chunk * kBN + lt;
+                        const int sv = (c < p.topk) ? ir[lt] : -1;
+                        const bool ok = tpos < p.n && sv >= 0 && sv < p.N_cap;
+                        const uint32_t bits = __ballot_sync(0xffffffffu, ok);
+                        if (lane == 0) ctl->mask[slot][warp] = bits;
+                    }
+                    // rows: 16 lanes per 256-byte row, kLoadThreads/16 rows per round
+                    constexpr int kRowsPerRound = kLoadThreads / 16;
+                    const int c16 = lt & 15, half = c16 >> 3, cc = c16 & 7;
+#pragma unroll 4
+                    for (int it = 0; it < kBN / kRowsPerRound; ++it) {
+                        const int row = it * kRowsPerRound + (lt >> 4);
+                        const int c = chunk * kBN + row;
+                        int sv = (c < p.topk) ? ir[row] : -1;
+                        if (tpos >= p.n || sv < 0 || sv >= p.N_cap) sv = 0;   // masked; any valid row
+                        const uint8_t* src = kvc_rows + (size_t)sv * (kD * 2) + c16 * 16;
+                        cp_async16(dst + half * kHalf + row * 128 + ((cc ^ (row & 7)) << 4), src);
+                    }
+                    cp_async_arrive_noinc(&ctl->full[slot]);
+                    named_sync(1, kLoadThreads);                 // every mask word is written
+                    if (lt == 0) mbar_arrive(&ctl->full[slot]);  // releases the mask
+                } else {
+                    if (lt == 0) {
+                        const CUtensorMap* tm = (kind == 1) ? &tm_c : &tm_w;
+                        const int row = (kind == 1) ? b * p.N_cap + chunk * kBN
+                                                    : b * p.L_raw + g.p_lo + chunk * kBN;
+                        mbar_arrive_expect_tx(&ctl->full[slot], kTileBytes);
+                        for (int h = 0; h < 2; ++h)
+                            tma_load_2d(dst + h * kHalf, tm, h * 64, row, &ctl->full[slot]);
+                    }
+                    mbar_arrive(&ctl->full[slot]);
+                }
             }
         }
         // drain: copies still in flight must land before the CTA exits
         cp_async_wait_all();
         if (lt == 0)
-            for (int Lp = max(0, L - kStages); Lp < L; ++Lp) {
+            for (int Lp = max(0, Lg - kStages); Lp < Lg; ++Lp) {
                 volatile int never = 0;
                 mbar_wait(&ctl->full[Lp % kStages], (Lp / kStages) & 1, &never, p.err);
             }
     } else if (warp == kMmaWarp) {
-        // ------------------------------------------------------------ MMA issuer
+        // ------------------------------------------------------------ MMA issuer (+ Q loads)
         if (lane == 0) {
+            prefetch_tmap(&tm_q);
             const uint32_t id_qk_full = idesc_bf16(kRows, kBN, false, false);
             const uint32_t id_pv = idesc_bf16(kRows, kD, false, true);
-            bool ok = mbar_wait(&ctl->bar_q, 0, abort, p.err);
-            tc_fence_after();
-            auto issue_qk = [&](int mt, int j) -> bool {
-                const TileRef r = tile_ref(p, g, mt, j);
-                const int slot = r.load % kStages;
-                if (!mbar_wait(&ctl->full[slot], (r.load / kStages) & 1, abort, p.err)) return false;
-                tc_fence_after();
-                const uint32_t qa = smem_u32(sQ + mt * kTileBytes);
-                const uint32_t ka = smem_u32(sK + slot * kTileBytes);
-                const uint32_t idesc = (r.bn == kBN) ? id_qk_full : idesc_bf16(kRows, r.bn, false, false);
-#pragma unroll
-                for (int k = 0; k < kD / 16; ++k) {
-                    const uint32_t off = (k >> 2) * kHalf + (k & 3) * 32;
-                    mma_bf16_ss(tmem + mt * 128, sw128_desc(qa + off, 16, 1024),
-                                sw128_desc(ka + off, 16, 1024), idesc, k > 0);
-                }
-                mma_commit(&ctl->s_full[mt]);
-                return true;
+            auto load_q = [&](int u) {
+                const Unit un = unit_of(p, u);
+                mbar_arrive_expect_tx(&ctl->bar_q, 2 * kTileBytes);
+                const int qrow = (un.b * p.n + un.t0) * kH;
+                for (int mt = 0; mt < 2; ++mt)
+                    for (int h = 0; h < 2; ++h)
+                        tma_load_2d(sQ + mt * kTileBytes + h * kHalf, &tm_q, h * 64, qrow + mt * kRows,
+                                    &ctl->bar_q);
             };
-            if (ok && g.T > 0) ok = issue_qk(0, 0) && issue_qk(1, 0);
-            for (int j = 0; ok && j < g.T; ++j) {
-                for (int mt = 0; mt < 2 && ok; ++mt) {
-                    if (!mbar_wait(&ctl->p_ready[mt], j & 1, abort, p.err)) { ok = false; break; }
-                    tc_fence_after();
+            int L0 = 0;                       // loads before this unit
+            int J[2] = {0, 0};                // tiles before this unit, per M tile
+            int k = 0;                        // units done
+            bool ok = true;
+            if (blockIdx.x < n_units) load_q(blockIdx.x);
+            for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++k) {
+                const Unit un = unit_of(p, u);
+                const Geometry g = geometry(p, un.b, un.t0);
+                ok = mbar_wait(&ctl->bar_q, k & 1, abort, p.err);
+                tc_fence_after();
+                auto issue_qk = [&](int mt, int j) -> bool {
                     const TileRef r = tile_ref(p, g, mt, j);
-                    const int slot = r.load % kStages;
-                    const uint32_t va = smem_u32(sK + slot * kTileBytes);
-                    // P (bf16, two per column) sits in the first 64 columns of S
-                    for (int kk = 0; kk < r.bn / 16; ++kk)
-                        mma_bf16_ts(tmem + 256 + mt * 128, tmem + mt * 128 + kk * 8,
-                                    sw128_desc(va + kk * 2048, kHalf, 1024), id_pv,
-                                    (j > 0 || kk > 0) ? 1u : 0u);
-                    mma_commit(&ctl->pv_done[mt]);
-                    if (r.last_consumer) mma_commit(&ctl->freeb[slot]);
-                    if (j + 1 < g.T) ok = issue_qk(mt, j + 1);
+                    const int ld = L0 + r.load;
+                    const int slot = ld % kStages;
+                    if (!mbar_wait(&ctl->full[slot], (ld / kStages) & 1, abort, p.err)) return false;
+                    tc_fence_after();
+                    const uint32_t qa = smem_u32(sQ + mt * kTileBytes);
+                    const uint32_t ka = smem_u32(sK + slot * kTileBytes);
+                    const uint32_t idesc = (r.bn == kBN) ? id_qk_full : idesc_bf16(kRows, r.bn, false, false);
+#pragma unroll
+                    for (int kq = 0; kq < kD / 16; ++kq) {
+                        const uint32_t off = (kq >> 2) * kHalf + (kq & 3) * 32;
+                        mma_bf16_ss(tmem + mt * 128, sw128_desc(qa + off, 16, 1024),
+                                    sw128_desc(ka + off, 16, 1024), idesc, kq > 0);
+                    }
+                    mma_commit(&ctl->s_full[mt]);
+                    return true;
+                };
+                const int un_next = u + gridDim.x;
+                // after the unit's last QK: once it has read Q, load the next unit's
+                auto next_q = [&]() -> bool {
+                    mma_commit(&ctl->q_free);
+                    if (un_next >= n_units) return true;
+                    if (!mbar_wait(&ctl->q_free, k & 1, abort, p.err)) return false;
+                    load_q(un_next);
+                    return true;
+                };
+                if (ok && g.T > 0) ok = issue_qk(0, 0) && issue_qk(1, 0);
+                if (ok && g.T <= 1) ok = next_q();
+                // the previous unit's O must have been read before this unit's first P.V
+                bool o_ready[2] = {k == 0, k == 0};
+                for (int j = 0; ok && j < g.T; ++j) {
+                    for (int mt = 0; mt < 2 && ok; ++mt) {
+                        if (!mbar_wait(&ctl->p_ready[mt], (J[mt] + j) & 1, abort, p.err)) { ok = false; break; }
+                        if (!o_ready[mt]) {
+                            if (!mbar_wait(&ctl->o_free[mt], (k - 1) & 1, abort, p.err)) { ok = false; break; }
+                            o_ready[mt] = true;
+                        }
+                        tc_fence_after();
+                        const TileRef r = tile_ref(p, g, mt, j);
+                        const int ld = L0 + r.load;
+                        const int slot = ld % kStages;
+                        const uint32_t va = smem_u32(sK + slot * kTileBytes);
+                        // P (bf16, two per column) sits in the first 64 columns of S
+                        for (int kk = 0; kk < r.bn / 16; ++kk)
+                            mma_bf16_ts(tmem + 256 + mt * 128, tmem + mt * 128 + kk * 8,
+                                        sw128_desc(va + kk * 2048, kHalf, 1024), id_pv,
+                                        (j > 0 || kk > 0) ? 1u : 0u);
+                        mma_commit(&ctl->pv_done[mt]);
+                        if (r.last_consumer) mma_commit(&ctl->freeb[slot]);
+                        if (j + 1 < g.T) {
+                            ok = issue_qk(mt, j + 1);
+                            if (ok && mt == 1 && j + 2 == g.T) ok = next_q();
+                        }
+                    }
                 }
+                // this unit's O is complete (or untouched when it has no tiles)
+                if (ok) {
+                    for (int mt = 0; mt < 2; ++mt) {
+                        if (!o_ready[mt] && !mbar_wait(&ctl->o_free[mt], (k - 1) & 1, abort, p.err)) { ok = false; break; }
+                        mma_commit(&ctl->o_full[mt]);
+                    }
+                }
+                L0 += total_loads(p, g);
+                J[0] += g.T;
+                J[1] += g.T;
             }
             // every MMA issued must finish before TMEM is released
             mma_commit(&ctl->fin);
@@ -515,129 +592,160 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             mbar_wait(&ctl->fin, 0, &never, p.err);
         }
         __syncwarp();
-    } else {
+    } else if (warp < kEpiWarp0) {
         // ------------------------------------------------------------ softmax
         const int mt = (warp - kSoftWarp0) >> 2;
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;                   // row of the M tile
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        const int u = r >> 6;                                // token of the M tile
-        const int t = t0 + 2 * mt + u;                       // absolute position
-        const bool row_ok = t < p.n;
-        int Vt = 0;
-        if (p.dense && row_ok) {
-            const int ne = clampi(p.n_entries ? p.n_entries[b] : p.N_cap, 0, p.N_cap);
-            Vt = min((t + 1) / p.m, ne);
-        }
-        const int w_lo = t - p.window + 1;                   // window [w_lo, t]
-        // m_used: running max (base 2); l_r: sum of the bf16-rounded weights
-        // (normalises O); l_e: sum of the unrounded weights (the lse output)
-        float m_used = -INFINITY, l_r = 0.0f, l_e = 0.0f;
+        const int u_tok = r >> 6;                            // token of the M tile
         const uint32_t s_addr = tmem + lane_addr + mt * 128;
         const uint32_t o_addr = tmem + lane_addr + 256 + mt * 128;
+        int J = 0;                                           // tiles before this unit
+        int L0 = 0;                                          // loads before this unit
+        int k = 0;
         bool ok = true;
-        for (int j = 0; j < g.T && ok; ++j) {
-            const TileRef tr = tile_ref(p, g, mt, j);
-            // every wait is warp-collective: the TMEM accesses below are .sync.aligned
-            if (!__all_sync(0xffffffffu, mbar_wait(&ctl->s_full[mt], j & 1, abort, p.err))) { ok = false; break; }
-            tc_fence_after();
-            // which columns are keys of this row?
-            int c_lo = 0, c_hi = -1;                         // contiguous range
-            uint32_t mw[4] = {~0u, ~0u, ~0u, ~0u};           // gathered tiles: valid rows
-            if (row_ok) {
-                if (tr.kind == 0) {
-                    if (tr.token == u) {
-                        const int slot = tr.load % kStages;
-                        // the producer wrote the mask before arming this stage
-                        if (!__all_sync(0xffffffffu, mbar_wait(&ctl->full[slot], (tr.load / kStages) & 1, abort, p.err))) { ok = false; break; }
-#pragma unroll
-                        for (int q = 0; q < 4; ++q) mw[q] = ctl->mask[slot][q];
-                        c_hi = tr.bn - 1;
-                    }
-                } else if (tr.kind == 1) {
-                    c_hi = min(tr.bn, Vt - tr.chunk * kBN) - 1;
-                } else {
-                    const int p0 = g.p_lo + tr.chunk * kBN;
-                    c_lo = max(0, w_lo - p0);
-                    c_hi = min(tr.bn, t - p0 + 1) - 1;
-                }
+        for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++k) {
+            const Unit un = unit_of(p, u);
+            const int b = un.b, t0 = un.t0;
+            const Geometry g = geometry(p, b, t0);
+            const int t = t0 + 2 * mt + u_tok;               // absolute position
+            const bool row_ok = t < p.n;
+            int Vt = 0;
+            if (p.dense && row_ok) {
+                const int ne = clampi(p.n_entries ? p.n_entries[b] : p.N_cap, 0, p.N_cap);
+                Vt = min((t + 1) / p.m, ne);
             }
-            // P buffer free and O stable once the previous P.V has finished
-            if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(&ctl->pv_done[mt], (j - 1) & 1, abort, p.err))) { ok = false; break; }
-            uint32_t vm[4];
-            valid_bits(c_lo, c_hi, mw, vm);
-            const bool has = (vm[0] | vm[1] | vm[2] | vm[3]) != 0u;
-            float se = 0.0f, sr = 0.0f;
-            if (!__any_sync(0xffffffffu, has)) {
-                // no key of this tile is visible to any row of the warp: P = 0
-                uint32_t zero[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) zero[i] = 0u;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) tmem_st16(s_addr + q * 16, zero);
-            } else {
-                // pass 1: the tile's row max; raise the running max (and
-                // rescale O) when it grows by more than 2^8
-                const bool full = (vm[0] & vm[1] & vm[2] & vm[3]) == 0xffffffffu;   // uniform per warp
-                const float mx = full ? tile_max_full(s_addr, p.scale_log2) : tile_max(s_addr, vm, p.scale_log2);
-                const bool raise = mx > m_used + kRescaleLog2;   // true for a row's first keys
-                float alpha = 1.0f;
-                if (raise) {
-                    alpha = (m_used == -INFINITY) ? 0.0f : ex2(m_used - mx);
-                    m_used = mx;
-                    l_r *= alpha;
-                    l_e *= alpha;
-                }
-                if (j > 0 && __any_sync(0xffffffffu, raise)) rescale_o(o_addr, alpha);
-                // pass 2: P = exp2(z - m_used) over S
-                const float mm = (m_used == -INFINITY) ? INFINITY : m_used;
-                if (full)
-                    tile_exp_full(s_addr, p.scale_log2, mm, p.lse != nullptr, se, sr);
-                else
-                    tile_exp(s_addr, vm, p.scale_log2, mm, se, sr);
-                l_r += sr;
-                l_e += se;
-            }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&ctl->p_ready[mt]);
-        }
-        // epilogue: O / l
-        bool fin_ok = ok && g.T > 0;
-        if (fin_ok) fin_ok = mbar_wait(&ctl->pv_done[mt], (g.T - 1) & 1, abort, p.err);
-        fin_ok = __all_sync(0xffffffffu, fin_ok);
-        if (fin_ok) {
-            tc_fence_after();
-            const float inv = l_r > 0.0f ? 1.0f / l_r : 0.0f;
-            __nv_bfloat16* orow = p.out + ((size_t)(b * p.n + t) * kH + (r & 63)) * kD;
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                float ov[32];
-                tmem_ld32(o_addr + q * 32, ov);
+            const int w_lo = t - p.window + 1;               // window [w_lo, t]
+            // m_used: running max (base 2); l_r: sum of the bf16-rounded weights
+            // (normalises O); l_e: sum of the unrounded weights (the lse output)
+            float m_used = -INFINITY, l_r = 0.0f, l_e = 0.0f;
+            for (int j = 0; j < g.T && ok; ++j) {
+                const TileRef tr = tile_ref(p, g, mt, j);
+                // every wait is warp-collective: the TMEM accesses below are .sync.aligned
+                if (!__all_sync(0xffffffffu, mbar_wait(&ctl->s_full[mt], (J + j) & 1, abort, p.err))) { ok = false; break; }
+                tc_fence_after();
+                // which columns are keys of this row?
+                int c_lo = 0, c_hi = -1;                     // contiguous range
+                uint32_t mw[4] = {~0u, ~0u, ~0u, ~0u};       // gathered tiles: valid rows
                 if (row_ok) {
+                    if (tr.kind == 0) {
+                        if (tr.token == u_tok) {
+                            const int lg = L0 + tr.load;     // the loaders' index of this tile
+                            const int slot = lg % kStages;
+                            // the producer wrote the mask before arming this stage
+                            if (!__all_sync(0xffffffffu, mbar_wait(&ctl->full[slot], (lg / kStages) & 1, abort, p.err))) { ok = false; break; }
 #pragma unroll
-                    for (int i = 0; i < 32; i += 8) {
-                        uint4 v;
-                        __nv_bfloat162 h0 = __floats2bfloat162_rn(ov[i] * inv, ov[i + 1] * inv);
-                        __nv_bfloat162 h1 = __floats2bfloat162_rn(ov[i + 2] * inv, ov[i + 3] * inv);
-                        __nv_bfloat162 h2 = __floats2bfloat162_rn(ov[i + 4] * inv, ov[i + 5] * inv);
-                        __nv_bfloat162 h3 = __floats2bfloat162_rn(ov[i + 6] * inv, ov[i + 7] * inv);
-                        v.x = *reinterpret_cast<uint32_t*>(&h0);
-                        v.y = *reinterpret_cast<uint32_t*>(&h1);
-                        v.z = *reinterpret_cast<uint32_t*>(&h2);
-                        v.w = *reinterpret_cast<uint32_t*>(&h3);
-                        *reinterpret_cast<uint4*>(orow + q * 32 + i) = v;
+                            for (int q = 0; q < 4; ++q) mw[q] = ctl->mask[slot][q];
+                            c_hi = tr.bn - 1;
+                        }
+                    } else if (tr.kind == 1) {
+                        c_hi = min(tr.bn, Vt - tr.chunk * kBN) - 1;
+                    } else {
+                        const int p0 = g.p_lo + tr.chunk * kBN;
+                        c_lo = max(0, w_lo - p0);
+                        c_hi = min(tr.bn, t - p0 + 1) - 1;
                     }
                 }
+                // P buffer free and O stable once the previous P.V has finished
+                if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(&ctl->pv_done[mt], (J + j - 1) & 1, abort, p.err))) { ok = false; break; }
+                uint32_t vm[4];
+                valid_bits(c_lo, c_hi, mw, vm);
+                const bool has = (vm[0] | vm[1] | vm[2] | vm[3]) != 0u;
+                float se = 0.0f, sr = 0.0f;
+                if (!__any_sync(0xffffffffu, has)) {
+                    // no key of this tile is visible to any row of the warp: P = 0
+                    uint32_t zero[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) zero[i] = 0u;
+#pragma unroll
+                    for (int q = 0; q < 4; ++q) tmem_st16(s_addr + q * 16, zero);
+                } else {
+                    // pass 1: the tile's row max; raise the running max (and
+                    // rescale O) when it grows by more than 2^8
+                    const bool full = (vm[0] & vm[1] & vm[2] & vm[3]) == 0xffffffffu;   // uniform per warp
+                    const float mx = full ? tile_max_full(s_addr, p.scale_log2) : tile_max(s_addr, vm, p.scale_log2);
+                    const bool raise = mx > m_used + kRescaleLog2;   // true for a row's first keys
+                    float alpha = 1.0f;
+                    if (raise) {
+                        alpha = (m_used == -INFINITY) ? 0.0f : ex2(m_used - mx);
+                        m_used = mx;
+                        l_r *= alpha;
+                        l_e *= alpha;
+                    }
+                    if (j > 0 && __any_sync(0xffffffffu, raise)) rescale_o(o_addr, alpha);
+                    // pass 2: P = exp2(z - m_used) over S
+                    const float mm = (m_used == -INFINITY) ? INFINITY : m_used;
+                    if (full)
+                        tile_exp_full(s_addr, p.scale_log2, mm, p.lse != nullptr, se, sr);
+                    else
+                        tile_exp(s_addr, vm, p.scale_log2, mm, se, sr);
+                    l_r += sr;
+                    l_e += se;
+                }
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&ctl->p_ready[mt]);
             }
-            if (row_ok && p.lse)
-                p.lse[(size_t)(b * p.n + t) * kH + (r & 63)] =
-                    l_e > 0.0f ? (m_used + log2f(l_e)) / kLog2e : -INFINITY;
-        } else if (row_ok && g.T == 0) {
-            // no key at all: o = 0, lse = -inf
-            __nv_bfloat16* orow = p.out + ((size_t)(b * p.n + t) * kH + (r & 63)) * kD;
-            for (int i = 0; i < kD; i += 8) *reinterpret_cast<uint4*>(orow + i) = make_uint4(0, 0, 0, 0);
-            if (p.lse) p.lse[(size_t)(b * p.n + t) * kH + (r & 63)] = -INFINITY;
+            if (!ok) break;
+            // publish the row statistics of this unit for the epilogue
+            stats[((k & 1) * 2 + mt) * kRows + r] = RowStat{m_used, l_r, l_e};
+            mbar_arrive(&ctl->stats_ready[mt]);
+            J += g.T;
+            L0 += total_loads(p, g);
+        }
+    } else {
+        // ------------------------------------------------------------ epilogue: O / l
+        const int mt = (warp - kEpiWarp0) >> 2;
+        const int quarter = warp & 3;
+        const int r = quarter * 32 + lane;
+        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
+        const int u_tok = r >> 6;
+        const uint32_t o_addr = tmem + lane_addr + 256 + mt * 128;
+        int k = 0;
+        for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++k) {
+            const Unit un = unit_of(p, u);
+            const Geometry g = geometry(p, un.b, un.t0);
+            const int t = un.t0 + 2 * mt + u_tok;
+            const bool row_ok = t < p.n;
+            bool w_ok = mbar_wait(&ctl->stats_ready[mt], k & 1, abort, p.err);
+            const RowStat st = stats[((k & 1) * 2 + mt) * kRows + r];
+            w_ok = w_ok && mbar_wait(&ctl->o_full[mt], k & 1, abort, p.err);
+            if (!__all_sync(0xffffffffu, w_ok)) break;
+            tc_fence_after();
+            __nv_bfloat16* orow = p.out + ((size_t)(un.b * p.n + t) * kH + (r & 63)) * kD;
+            if (g.T > 0) {
+                const float inv = st.lr > 0.0f ? 1.0f / st.lr : 0.0f;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    float ov[32];
+                    tmem_ld32(o_addr + q * 32, ov);
+                    if (row_ok) {
+#pragma unroll
+                        for (int i = 0; i < 32; i += 8) {
+                            uint4 v;
+                            __nv_bfloat162 h0 = __floats2bfloat162_rn(ov[i] * inv, ov[i + 1] * inv);
+                            __nv_bfloat162 h1 = __floats2bfloat162_rn(ov[i + 2] * inv, ov[i + 3] * inv);
+                            __nv_bfloat162 h2 = __floats2bfloat162_rn(ov[i + 4] * inv, ov[i + 5] * inv);
+                            __nv_bfloat162 h3 = __floats2bfloat162_rn(ov[i + 6] * inv, ov[i + 7] * inv);
+                            v.x = *reinterpret_cast<uint32_t*>(&h0);
+                            v.y = *reinterpret_cast<uint32_t*>(&h1);
+                            v.z = *reinterpret_cast<uint32_t*>(&h2);
+                            v.w = *reinterpret_cast<uint32_t*>(&h3);
+                            *reinterpret_cast<uint4*>(orow + q * 32 + i) = v;
+                        }
+                    }
+                }
+                if (row_ok && p.lse)
+                    p.lse[(size_t)(un.b * p.n + t) * kH + (r & 63)] =
+                        st.le > 0.0f ? (st.m + log2f(st.le)) / kLog2e : -INFINITY;
+            } else if (row_ok) {
+                // no key at all: o = 0, lse = -inf
+                for (int i = 0; i < kD; i += 8) *reinterpret_cast<uint4*>(orow + i) = make_uint4(0, 0, 0, 0);
+                if (p.lse) p.lse[(size_t)(un.b * p.n + t) * kH + (r & 63)] = -INFINITY;
+            }
+            tc_fence_before();
+            mbar_arrive(&ctl->o_free[mt]);
         }
     }
 
@@ -714,8 +822,11 @@ cudaError_t launch_attention_tc(const AttnArgs& a, uint32_t* err, cudaStream_t s
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    const int tiles = (a.n_q + kTokens - 1) / kTokens;
-    attn_tc_kernel<<<(unsigned)(a.B * tiles), kThreads, smem, s>>>(tm_q, tm_c, tm_w, p);
+    const int units = a.B * ((a.n_q + kTokens - 1) / kTokens);
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = units < sms ? units : sms;     // persistent: one CTA per SM
+    attn_tc_kernel<<<(unsigned)grid, kThreads, smem, s>>>(tm_q, tm_c, tm_w, p);
     count_launch();
     return cudaGetLastError();
 }
