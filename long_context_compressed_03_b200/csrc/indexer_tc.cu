@@ -154,14 +154,52 @@ __device__ __forceinline__ void tmem_ld8x4(uint32_t taddr, float (*v)[8]) {
         : "memory");
 }
 
-// One chunk of 32 entries for this thread's row, in the row's mode (rows of
-// one warp can be at different radix levels).  The TMEM loads are .sync.aligned
-// warp-collective instructions: every lane of the warp runs them at the same
-// point, before any per-row branching; rows that are not selecting skip the
-// arithmetic.
-template <bool FP8>
+// One score of this thread's row: fold the four heads, then histogram or
+// emit its key according to the row's pass kind.  KIND_T < 0 takes the kind
+// at run time (rows of one warp at different radix levels).
+template <bool FP8, int KIND_T>
+__device__ __forceinline__ void score_one(const float (&acc)[kHeads][8], int e, float ks, int s,
+                                          int kind_rt, const RowCtx& rc) {
+    const int KIND = KIND_T >= 0 ? KIND_T : kind_rt;
+    // a + |a| = 2 ReLU(a) exactly (+0 for a <= 0), and rc.qs holds qs / 2, so
+    // this is sum_h qs_h ReLU(a_h) on the FMA pipe, always +0 or positive
+    float sc = rc.qs[0] * (acc[0][e] + fabsf(acc[0][e]));
+#pragma unroll
+    for (int h = 1; h < kHeads; ++h) sc = fmaf(rc.qs[h], acc[h][e] + fabsf(acc[h][e]), sc);
+    if (FP8) sc *= ks;
+    const uint32_t sbits = __float_as_uint(sc);
+    if (KIND == kHist0) {
+        atomicAdd(rc.hrow + (sbits >> 24) * kRows, 1u);
+    } else if (KIND == kHist32) {
+        const int sh32 = rc.sh - 16;
+        if ((sbits >> (sh32 + 8)) == (uint32_t)rc.prefix)
+            atomicAdd(rc.hrow + ((sbits >> sh32) & 255u) * kRows, 1u);
+    } else {
+        const uint64_t key = ((uint64_t)sbits << 16) | (uint64_t)(65535 - s);
+        if (KIND == kHist64) {
+            if ((key >> (rc.sh + 8)) == rc.prefix)
+                atomicAdd(rc.hrow + ((key >> rc.sh) & 255u) * kRows, 1u);
+        } else {
+            const uint64_t kp = key >> rc.sh;
+            if (kp > rc.prefix) {
+                const int pos = atomicAdd(rc.emitted, 1);
+                if (pos < rc.topk) rc.orow[pos] = s;
+            } else if (kp == rc.prefix) {
+                const int pos = atomicAdd(rc.listed, 1);
+                if (pos < kCap) rc.list[pos] = key;
+            }
+        }
+    }
+}
+
+// One chunk of 32 entries for this thread's row.  The TMEM loads and the
+// scale broadcasts are .sync.aligned / warp-collective: every lane of the
+// warp runs them at the same point, before any per-row branching; rows that
+// are not selecting skip the arithmetic.  KIND_T >= 0 when every selecting
+// row of the warp is in the same pass kind (the usual case).
+template <bool FP8, int KIND_T>
 __device__ __forceinline__ void chunk_pass(uint32_t taddr, float ksv, int c, bool active,
-                                           int KIND, const RowCtx& rc) {
+                                           int kind_rt, const RowCtx& rc) {
 #pragma unroll 1
     for (int part = 0; part < kN / 8; ++part) {
         float acc[kHeads][8];
@@ -169,47 +207,17 @@ __device__ __forceinline__ void chunk_pass(uint32_t taddr, float ksv, int c, boo
         // lane e of the warp holds the key scale of entry c*kN + e: broadcast
         // the part's eight before any per-row branching (warp-collective)
         float ks[8];
-        if (FP8) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) ks[e] = __shfl_sync(0xffffffffu, ksv, part * 8 + e);
-        }
+        for (int e = 0; e < 8; ++e) ks[e] = FP8 ? __shfl_sync(0xffffffffu, ksv, part * 8 + e) : 1.0f;
         if (!active) continue;
         const int s0 = c * kN + part * 8;
-        if (s0 >= rc.V) continue;
-        const int ne = min(8, rc.V - s0);
+        if (s0 + 8 <= rc.V) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-            if (e >= ne) break;
-            // a + |a| = 2 ReLU(a) exactly (+0 for a <= 0), and rc.qs holds qs / 2, so
-            // this is sum_h qs_h ReLU(a_h) on the FMA pipe, always +0 or positive
-            float sc = rc.qs[0] * (acc[0][e] + fabsf(acc[0][e]));
+            for (int e = 0; e < 8; ++e) score_one<FP8, KIND_T>(acc, e, ks[e], s0 + e, kind_rt, rc);
+        } else {
 #pragma unroll
-            for (int h = 1; h < kHeads; ++h) sc = fmaf(rc.qs[h], acc[h][e] + fabsf(acc[h][e]), sc);
-            if (FP8) sc *= ks[e];
-            const uint32_t sbits = __float_as_uint(sc);
-            if (KIND == kHist0) {
-                atomicAdd(rc.hrow + (sbits >> 24) * kRows, 1u);
-            } else if (KIND == kHist32) {
-                const int sh32 = rc.sh - 16;
-                if ((sbits >> (sh32 + 8)) == (uint32_t)rc.prefix)
-                    atomicAdd(rc.hrow + ((sbits >> sh32) & 255u) * kRows, 1u);
-            } else {
-                const int s = s0 + e;
-                const uint64_t key = ((uint64_t)sbits << 16) | (uint64_t)(65535 - s);
-                if (KIND == kHist64) {
-                    if ((key >> (rc.sh + 8)) == rc.prefix)
-                        atomicAdd(rc.hrow + ((key >> rc.sh) & 255u) * kRows, 1u);
-                } else {
-                    const uint64_t kp = key >> rc.sh;
-                    if (kp > rc.prefix) {
-                        const int pos = atomicAdd(rc.emitted, 1);
-                        if (pos < rc.topk) rc.orow[pos] = s;
-                    } else if (kp == rc.prefix) {
-                        const int pos = atomicAdd(rc.listed, 1);
-                        if (pos < kCap) rc.list[pos] = key;
-                    }
-                }
-            }
+            for (int e = 0; e < 8; ++e)
+                if (s0 + e < rc.V) score_one<FP8, KIND_T>(acc, e, ks[e], s0 + e, kind_rt, rc);
         }
     }
 }
@@ -403,12 +411,22 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
                 return (FP8 && c < nchunks && e < Vmax) ? __ldg(ksc + e) : 0.0f;
             };
             float ksv = scale_of(grp);
+            // the pass kind shared by every selecting row of the warp, or -1
+            const uint32_t act = __ballot_sync(0xffffffffu, active);
+            const int k0 = __shfl_sync(0xffffffffu, kind, act ? __ffs(act) - 1 : 0);
+            const int wkind = __all_sync(0xffffffffu, !active || kind == k0) ? k0 : -1;
             for (int c = grp; c < nchunks; c += kGroups) {
                 const float ksv_next = scale_of(c + kGroups);
                 if (!__all_sync(0xffffffffu, mbar_wait(&ctl->acc_full[grp], cons & 1, abort, p.err))) break;
                 tc_fence_after();
                 const uint32_t taddr = tmem + lane_addr + grp * 128;
-                chunk_pass<FP8>(taddr, ksv, c, active, kind, rc);
+                switch (wkind) {
+                    case kHist0: chunk_pass<FP8, kHist0>(taddr, ksv, c, active, kind, rc); break;
+                    case kHist32: chunk_pass<FP8, kHist32>(taddr, ksv, c, active, kind, rc); break;
+                    case kHist64: chunk_pass<FP8, kHist64>(taddr, ksv, c, active, kind, rc); break;
+                    case kEmit: chunk_pass<FP8, kEmit>(taddr, ksv, c, active, kind, rc); break;
+                    default: chunk_pass<FP8, -1>(taddr, ksv, c, active, kind, rc); break;
+                }
                 ksv = ksv_next;
                 tc_fence_before();
                 mbar_arrive(&ctl->acc_free[grp]);
