@@ -37,6 +37,7 @@ from long_context_compressed_03_b200 import api, synth  # noqa: E402
 
 PREFILL = "csa_prefill_n64k_fp8idx"
 DECODE = "csa_decode_b64_ctx128k"
+HCA_DECODE = "hca_decode_b16_ctx1m"
 METRIC = "CSA prefill queries/s at n=64K & decode tok/s at 128K ctx; % HBM/TC roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -307,6 +308,38 @@ def run_decode(dev, steps, warmup, rank):
                 kern_ms={"indexer_topk": float(np.mean(t_idx)), "sparse_attn": float(np.mean(t_att))})
 
 
+def run_hca_decode(dev, steps, warmup, rank):
+    """HCA decode at a 2^20-token context (batch 16, 8192 entries + 512-token
+    window per element): one dense attention launch per step, L2 flushed."""
+    w = synth.WORKLOADS[HCA_DECODE]
+    inp = synth.hca_decode_inputs(w, seed=rank)
+    d = {k: v.to(dev) for k, v in inp.items()}
+    out = torch.empty_like(d["q"])
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+
+    def step():
+        api.hca_dense_attn(d["q"], d["kv_c"], w.m, d["swa"], w.window, out,
+                           n_entries=d["n_entries"], raw_pos0=d["raw_pos0"], raw_len=d["raw_len"],
+                           q_pos=d["q_pos"])
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(steps):
+        flush.fill_(1)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        step()
+        b.record()
+        ts.append((a, b))
+    torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in ts]
+    nbytes = w.B * (w.N_cap + w.window) * w.D * 2 + 2 * w.B * w.H * w.D * 2
+    flops = 4.0 * w.B * w.H * w.D * (w.N_cap + w.window)
+    return dict(w=w, ms=float(np.mean(ms)), ms_median=float(np.median(ms)), bytes=nbytes, flops=flops)
+
+
 # ---------------------------------------------------------------------- oracle arm
 def oracle_prefill_sample(w, inp, n_sample, seed=5):
     """The fp64 oracle on a bounded sample of the prefill workload: both
@@ -487,6 +520,14 @@ def main():
         line["decode"] = {"workload": DECODE, "value": dec["w"].B * dist_ctx.world / (dms / 1e3),
                           "unit": "tok/s", "ms_per_step": dms, "ms_median": dec["ms_median"],
                           "l2": "flushed (512 MiB write) between steps", "stages": dstages}
+        hd = run_hca_decode(dev, args.steps, args.warmup, rank)
+        hms = dist_ctx.max(hd["ms"])
+        line["hca_decode"] = {"workload": HCA_DECODE, "value": hd["w"].B * dist_ctx.world / (hms / 1e3),
+                              "unit": "tok/s", "ms_per_step": hms, "ms_median": hd["ms_median"],
+                              "l2": "flushed (512 MiB write) between steps",
+                              "GB/s": hd["bytes"] / (hms / 1e3) / 1e9,
+                              "frac_hbm": hd["bytes"] / (hms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                              "TFLOP/s": hd["flops"] / (hms / 1e3) / 1e12}
     if not args.no_e2e:
         e2e = run_e2e(w, pre["inp"], dev, max(3, args.steps // 2))
         ems = dist_ctx.max(e2e["ms"])

@@ -75,7 +75,6 @@ struct __align__(8) Ctrl {
     uint64_t full[kStages];
     uint64_t freeb[kStages];
     uint64_t s_full[2];
-    uint64_t pv_done[2];
     uint64_t p_ready[2];
     uint64_t fin;
     uint32_t mask[kStages][4];      // gathered tiles: valid rows of the stage
@@ -376,7 +375,6 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&ctl->s_full[i], 1);
-            mbar_init(&ctl->pv_done[i], 1);
             mbar_init(&ctl->p_ready[i], kRows);
             mbar_init(&ctl->o_full[i], 1);
             mbar_init(&ctl->o_free[i], kRows);
@@ -525,14 +523,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     const int slot = ld % kStages;
                     if (!mbar_wait(&ctl->full[slot], (ld / kStages) & 1, abort, p.err)) return false;
                     tc_fence_after();
-                    const uint32_t qa = smem_u32(sQ + mt * kTileBytes);
-                    const uint32_t ka = smem_u32(sK + slot * kTileBytes);
+                    // descriptors of the k-step 0 operands; a k step adds its byte
+                    // offset / 16 to the start-address field (no carry: smem < 256 KB)
+                    const uint64_t qd = sw128_desc(smem_u32(sQ + mt * kTileBytes), 16, 1024);
+                    const uint64_t kd = sw128_desc(smem_u32(sK + slot * kTileBytes), 16, 1024);
                     const uint32_t idesc = (r.bn == kBN) ? id_qk_full : idesc_bf16(kRows, r.bn, false, false);
 #pragma unroll
                     for (int kq = 0; kq < kD / 16; ++kq) {
-                        const uint32_t off = (kq >> 2) * kHalf + (kq & 3) * 32;
-                        mma_bf16_ss(tmem + mt * 128, sw128_desc(qa + off, 16, 1024),
-                                    sw128_desc(ka + off, 16, 1024), idesc, kq > 0);
+                        const uint32_t off16 = ((kq >> 2) * kHalf + (kq & 3) * 32) >> 4;
+                        mma_bf16_ss(tmem + mt * 128, qd + off16, kd + off16, idesc, kq > 0);
                     }
                     mma_commit(&ctl->s_full[mt]);
                     return true;
@@ -561,13 +560,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         const TileRef r = tile_ref(p, g, mt, j);
                         const int ld = L0 + r.load;
                         const int slot = ld % kStages;
-                        const uint32_t va = smem_u32(sK + slot * kTileBytes);
+                        const uint64_t vd = sw128_desc(smem_u32(sK + slot * kTileBytes), kHalf, 1024);
                         // P (bf16, two per column) sits in the first 64 columns of S
                         for (int kk = 0; kk < r.bn / 16; ++kk)
                             mma_bf16_ts(tmem + 256 + mt * 128, tmem + mt * 128 + kk * 8,
-                                        sw128_desc(va + kk * 2048, kHalf, 1024), id_pv,
+                                        vd + (uint64_t)(kk * (2048 >> 4)), id_pv,
                                         (j > 0 || kk > 0) ? 1u : 0u);
-                        mma_commit(&ctl->pv_done[mt]);
                         if (r.last_consumer) mma_commit(&ctl->freeb[slot]);
                         if (j + 1 < g.T) {
                             ok = issue_qk(mt, j + 1);
@@ -647,8 +645,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         c_hi = min(tr.bn, t - p0 + 1) - 1;
                     }
                 }
-                // P buffer free and O stable once the previous P.V has finished
-                if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(&ctl->pv_done[mt], (J + j - 1) & 1, abort, p.err))) { ok = false; break; }
+                // (s_full of tile j is committed after the P.V of tile j-1 was issued
+                // by the same thread, so that P.V has completed: O is stable and the
+                // P columns are free)
                 uint32_t vm[4];
                 valid_bits(c_lo, c_hi, mw, vm);
                 const bool has = (vm[0] | vm[1] | vm[2] | vm[3]) != 0u;
