@@ -44,10 +44,10 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
 # keyed by kernel family; valid only while the kernel source hashes the same.
 NCU_TRAFFIC = {
-    # profiles/attn_tc_csa_prefill_n8192.md: 153.8 MB read + 88.3 MB written at
-    # n=8192, scaled by 8 (units = queries) to one n=65536 launch
-    "sparse_attn": {"bytes": (153.758720e6 + 88.312320e6) * 8, "file": "attention_tc.cu",
-                    "src": "4a33929d631e"},
+    # profiles/attn_tc_csa_prefill_n16384.md: 307.4 MB read + 220.7 MB written at
+    # n=16384, scaled by 4 (units = queries) to one n=65536 launch
+    "sparse_attn": {"bytes": (307.398912e6 + 220.704000e6) * 4, "file": "attention_tc.cu",
+                    "src": "b7b1aa0562f9"},
 }
 
 
@@ -420,6 +420,8 @@ def main():
                     help="override the prefill length (smaller cases for profiler captures; "
                          "the line is then marked as not the headline workload)")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--decode-only", action="store_true",
+                    help="run only the decode steps (profiler captures of the decode kernels)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args()
@@ -471,6 +473,20 @@ def main():
     torch.cuda.set_device(dev)
     api.load()
     peaks, peak_src = load_peaks()
+    if args.decode_only:
+        dec = run_decode(dev, args.steps, args.warmup, rank)
+        hd = run_hca_decode(dev, args.steps, args.warmup, rank)
+        line = {"metric": "CSA decode tok/s at 128K ctx (decode only: profiling case, not the headline)",
+                "value": dec["w"].B * dist_ctx.world / (dist_ctx.max(dec["ms"]) / 1e3), "unit": "tok/s",
+                "n_gpus": dist_ctx.world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": dist_ctx.max(dec["ms"]), "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+                "config": {"workload": DECODE, "hca_workload": HCA_DECODE},
+                "stages_ms": dec["kern_ms"], "hca_decode_ms": dist_ctx.max(hd["ms"])}
+        if rank == 0:
+            print(json.dumps(line))
+        dist_ctx.close()
+        return 0
 
     pre = run_prefill(w, dev, args.steps, args.warmup, dist_ctx, rank)
     t_max = dist_ctx.max(pre["total_ms"])
