@@ -7,12 +7,16 @@
 //  "DS-V4 分析&学习" §1.3 2m-position overlap; "DeepSeek V4 CSA + CP 迁移到 HP…"
 //  §3.2 ratio 4 overlapping, ratio 128 not.)
 //
-// One CTA owns a tile of ET consecutive entries of one batch element.  It
-// streams the tile's blocks once (each block's m rows summed in fp32, rows
-// read coalesced along the feature dimension), forms the pooled rows from
-// one or two block sums, multiplies them by W (fp32 FMA, W read through L2)
-// and writes the tile in the requested format; the fp8 epilogue reduces each
-// row's amax across a warp and quantises it in place.
+// One CTA owns a tile of 64 consecutive entries of one batch element.
+//  * Pooling: each thread owns one feature column for a run of entries and
+//    walks the blocks once with a running block sum (an overlapping entry is
+//    the previous block's sum plus its own), so x is read once, coalesced
+//    along features; pooled rows (fp32) go to shared memory.
+//  * Projection: a register-tiled fp32 product with W staged in shared memory
+//    32 rows at a time; each thread accumulates 8 entries x 4 outputs, the
+//    pooled values of a warp's 8 entries being broadcast reads.
+//  * Epilogue: bf16/fp32 stores, or per-row amax across a warp and E4M3
+//    quantisation (IEEE division, round to nearest even, saturating).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -20,7 +24,8 @@ namespace csa {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kTile = 32;  // entries per CTA
+constexpr int kTile = 64;   // entries per CTA
+constexpr int kKC = 32;     // rows of W staged per step
 
 template <typename Tin, int OUT>
 __global__ void __launch_bounds__(kThreads) compress_kernel(CompressArgs a) {
@@ -29,45 +34,81 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(CompressArgs a) {
     const int b = blockIdx.y;
     const int i0 = blockIdx.x * kTile;
     const int ne = min(kTile, N_c - i0);
-    float* bsum = smem;                           // [kTile + 1][d_in]: blocks i0-1 .. i0+kTile-1
-    float* pooled = bsum + (kTile + 1) * d_in;    // [kTile][d_in]
-    float* outs = pooled + kTile * d_in;          // [kTile][d_out]
+    float* pooled = smem;                          // [kTile][d_in]
+    float* wst = pooled + kTile * d_in;            // [kKC][128]
+    float* outs = wst + kKC * 128;                 // [kTile][d_out]
     const Tin* x = static_cast<const Tin*>(a.x) + (size_t)b * n * d_in;
     const Tin* W = static_cast<const Tin*>(a.W);
+    const int tid = threadIdx.x;
 
-    // block sums of blocks jb = i0-1+jj (jj = 0 .. ne)
-    for (int p = threadIdx.x; p < (ne + 1) * d_in; p += kThreads) {
-        const int jj = p / d_in, c = p - jj * d_in;
-        const int jb = i0 - 1 + jj;
-        float acc = 0.0f;
-        if (jb >= 0 && (a.overlap || jj > 0)) {
-            const Tin* src = x + (size_t)jb * m * d_in + c;
-            for (int r = 0; r < m; ++r) acc += to_f32(src[(size_t)r * d_in]);
+    // ---- pooling: thread -> (column c, run of entries)
+    {
+        const int tpc = kThreads / d_in;                 // threads per column (>= 1)
+        const int per = (kTile + tpc - 1) / tpc;         // entries per thread
+        if (tid < tpc * d_in) {
+            const int c = tid % d_in, part = tid / d_in;
+            const int e0 = part * per;
+            auto block_sum = [&](int jb) -> float {      // sum of block jb's m rows (0 if absent)
+                float acc = 0.0f;
+                if (jb >= 0) {
+                    const Tin* src = x + (size_t)jb * m * d_in + c;
+                    for (int r = 0; r < m; ++r) acc += to_f32(src[(size_t)r * d_in]);
+                }
+                return acc;
+            };
+            float prev = (a.overlap && e0 < ne) ? block_sum(i0 + e0 - 1) : 0.0f;
+            for (int e = e0; e < e0 + per && e < ne; ++e) {
+                const int i = i0 + e;
+                const float cur = block_sum(i);
+                const int lo = a.overlap ? max(0, m * (i - 1)) : m * i;
+                const float cnt = (float)(m * (i + 1) - lo);
+                pooled[e * d_in + c] = (a.overlap ? prev + cur : cur) / cnt;
+                prev = cur;
+            }
         }
-        bsum[p] = acc;
     }
-    __syncthreads();
-    for (int p = threadIdx.x; p < ne * d_in; p += kThreads) {
-        const int e = p / d_in, c = p - e * d_in;
-        const int i = i0 + e;
-        const int lo = a.overlap ? max(0, m * (i - 1)) : m * i;
-        const float cnt = (float)(m * (i + 1) - lo);
-        const float s = bsum[(e + 1) * d_in + c] + (a.overlap ? bsum[e * d_in + c] : 0.0f);
-        pooled[p] = s / cnt;
-    }
-    __syncthreads();
-    for (int p = threadIdx.x; p < ne * d_out; p += kThreads) {
-        const int e = p / d_out, o = p - e * d_out;
-        const float* pr = pooled + e * d_in;
-        float acc = 0.0f;
-        for (int c = 0; c < d_in; ++c) acc = fmaf(pr[c], to_f32(W[(size_t)c * d_out + o]), acc);
-        outs[p] = acc;
+    // ---- projection: outs[e][o] = sum_k pooled[e][k] W[k][o]
+    const int ty = tid >> 5, tx = tid & 31;            // entries 8 ty .. +7, outputs ob + 4 tx .. +3
+    for (int ob = 0; ob < d_out; ob += 128) {
+        const int ow = min(128, d_out - ob);
+        float acc[8][4];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) acc[r][0] = acc[r][1] = acc[r][2] = acc[r][3] = 0.0f;
+        for (int k0 = 0; k0 < d_in; k0 += kKC) {
+            const int kc = min(kKC, d_in - k0);        // 16 or 32 (d_in is a multiple of 16)
+            __syncthreads();                           // pooled ready / previous W chunk consumed
+            for (int q = tid; q < kc * ow; q += kThreads) {
+                const int kr = q / ow, oc = q - kr * ow;
+                wst[kr * 128 + oc] = to_f32(W[(size_t)(k0 + kr) * d_out + ob + oc]);
+            }
+            __syncthreads();
+            if (4 * tx < ow) {
+#pragma unroll 4
+                for (int kk = 0; kk < kc; ++kk) {
+                    const float4 w4 = *reinterpret_cast<const float4*>(wst + kk * 128 + 4 * tx);
+#pragma unroll
+                    for (int r = 0; r < 8; ++r) {
+                        const float pv = pooled[(8 * ty + r) * d_in + k0 + kk];
+                        acc[r][0] = fmaf(pv, w4.x, acc[r][0]);
+                        acc[r][1] = fmaf(pv, w4.y, acc[r][1]);
+                        acc[r][2] = fmaf(pv, w4.z, acc[r][2]);
+                        acc[r][3] = fmaf(pv, w4.w, acc[r][3]);
+                    }
+                }
+            }
+        }
+        if (4 * tx < ow) {
+#pragma unroll
+            for (int r = 0; r < 8; ++r)
+                *reinterpret_cast<float4*>(outs + (8 * ty + r) * d_out + ob + 4 * tx) =
+                    make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
+        }
     }
     __syncthreads();
 
     const size_t row0 = (size_t)b * N_c + i0;
     if constexpr (OUT == DT_E4M3) {
-        const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+        const int warp = tid >> 5, lane = tid & 31;
         uint8_t* out = static_cast<uint8_t*>(a.out);
         for (int e = warp; e < ne; e += kThreads / 32) {
             float amax = 0.0f;
@@ -81,14 +122,14 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(CompressArgs a) {
     } else {
         using Tout = typename std::conditional<OUT == DT_F32, float, __nv_bfloat16>::type;
         Tout* out = static_cast<Tout*>(a.out);
-        for (int p = threadIdx.x; p < ne * d_out; p += kThreads)
+        for (int p = tid; p < ne * d_out; p += kThreads)
             store_out<Tout>(out + row0 * d_out + p, outs[p]);
     }
 }
 
 template <typename Tin, int OUT>
 cudaError_t launch_t(const CompressArgs& a, cudaStream_t s) {
-    const size_t smem = sizeof(float) * ((size_t)(2 * kTile + 1) * a.d_in + (size_t)kTile * a.d_out);
+    const size_t smem = sizeof(float) * ((size_t)kTile * a.d_in + (size_t)kKC * 128 + (size_t)kTile * a.d_out);
     auto kern = compress_kernel<Tin, OUT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
