@@ -66,6 +66,7 @@ def _load():
         lib.oracle_visible_entries.argtypes = [i64, i32, i64]
         lib.oracle_visible_entries.restype = i64
         lib.oracle_compress.argtypes = [P, i32, i32, i32, P, i32, i32, i32, P]
+        lib.oracle_compress_append.argtypes = [P, P, i32, i32, P, i32, i32, i32, P, P, i32, P]
         dbl = ctypes.c_double
         lib.oracle_indexer_scores.argtypes = [P, P, P, i64, i32, i32, P, P, P, i32, P, i32, P]
         lib.oracle_indexer_topk.argtypes = [P, P, P, i64, i32, i32, P, P, P, i32, P, i32, i32, P,
@@ -157,6 +158,39 @@ def compress(x, W, m: int, overlap: bool) -> np.ndarray:
     if N_c:
         _load().oracle_compress(_ptr(x), B, n, d_in, _ptr(W), d_out, m, int(bool(overlap)),
                                 _ptr(out))
+    return out
+
+
+def compress_append(state, x_new, W, m: int, overlap: bool, pos, out, N_cap: int) -> np.ndarray:
+    """One decode step of the compressor state ("DS-V4 分析&学习" opening summary
+    and §1.3): adds each element's new token to its running block sum and, when
+    the token completes block j = pos // m, writes entry j (mean over its window,
+    then @ W) into ``out[b, j]``.  ``state`` [B, 2, d_in] fp64 and ``out``
+    [B, N_cap, d_out] fp64 are updated in place; returns done [B] (the entry
+    written, or -1)."""
+    x_new = _f64(x_new)
+    W = _f64(W)
+    B, d_in = x_new.shape
+    d_out = W.shape[1]
+    assert state.dtype == np.float64 and state.flags.c_contiguous and state.shape == (B, 2, d_in)
+    assert out.dtype == np.float64 and out.flags.c_contiguous and out.shape == (B, N_cap, d_out)
+    pos = _i32(pos)
+    done = np.empty(B, np.int32)
+    _load().oracle_compress_append(_ptr(state), _ptr(x_new), B, d_in, _ptr(W), d_out, m,
+                                   int(bool(overlap)), _ptr(pos), _ptr(out), N_cap, _ptr(done))
+    return done
+
+
+def compress_stream(x, W, m: int, overlap: bool) -> np.ndarray:
+    """Feeds x [B, n, d_in] to ``compress_append`` one position at a time and
+    returns the entries it wrote, [B, floor(n/m), d_out]."""
+    x = _f64(x)
+    B, n, d_in = x.shape
+    N_c = num_entries(n, m)
+    state = np.zeros((B, 2, d_in), np.float64)
+    out = np.zeros((B, N_c, _f64(W).shape[1]), np.float64)
+    for p in range(n):
+        compress_append(state, x[:, p], W, m, overlap, np.full(B, p, np.int32), out, N_c)
     return out
 
 

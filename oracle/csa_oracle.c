@@ -158,6 +158,55 @@ void oracle_compress(const double* x, int B, int n, int d_in, const double* W, i
 }
 
 /* ------------------------------------------------------------------------
+ * Decode-time compression state ("DS-V4 分析&学习", opening summary: the KV
+ * cache is the compressed cache plus a state cache and a tail state; §1.3:
+ * an overlapping entry spans the previous and the current block, which makes
+ * the decode-time state the part to maintain).
+ *
+ * state[b] holds two rows of d_in values: row 0 the sum of the last complete
+ * block's m rows, row 1 the running sum of the current block.  The token at
+ * absolute position pos[b] (negative: element b has no token this step) is
+ * added to row 1.  When it completes block j = pos/m, entry j is the mean
+ * over its window -- blocks j-1 and j (2m rows) when overlap and j > 0, block
+ * j alone otherwise -- times W; it is written to out[b, j] when j < N_cap, and
+ * done[b] = j.  Then row 0 takes row 1 and row 1 restarts at zero.  done[b]
+ * is -1 when no entry completed.  Tokens must arrive in position order.
+ * --------------------------------------------------------------------- */
+void oracle_compress_append(double* state, const double* x_new, int B, int d_in, const double* W,
+                            int d_out, int m, int overlap, const int* pos, double* out, int N_cap,
+                            int* done) {
+    for (int b = 0; b < B; ++b) {
+        done[b] = -1;
+        const long p = pos[b];
+        if (p < 0) continue;
+        double* prev = state + (long)b * 2 * d_in;
+        double* cur = prev + d_in;
+        const double* xr = x_new + (long)b * d_in;
+        for (int c = 0; c < d_in; ++c) cur[c] += xr[c];
+        if ((p + 1) % m != 0) continue;
+        const long j = p / m;
+        const int both = overlap && j > 0;
+        const double cnt = both ? 2.0 * m : (double)m;
+        if (j < N_cap) {
+            double* o = out + ((long)b * N_cap + j) * d_out;
+            for (int k = 0; k < d_out; ++k) {
+                double acc = 0.0;
+                for (int c = 0; c < d_in; ++c) {
+                    const double pooled = ((both ? prev[c] : 0.0) + cur[c]) / cnt;
+                    acc += pooled * W[(long)c * d_out + k];
+                }
+                o[k] = acc;
+            }
+        }
+        done[b] = (int)j;
+        for (int c = 0; c < d_in; ++c) {
+            prev[c] = cur[c];
+            cur[c] = 0.0;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------
  * Causal visibility of compressed entries.  Entry i covers positions up to
  * m(i+1)-1 and becomes visible to the query at absolute position t once its
  * block is complete: i < floor((t+1)/m), further clamped to the number of

@@ -438,3 +438,52 @@ def test_end_to_end_is_causal():
     assert np.array_equal(o1[:t + 1], o2[:t + 1])
     assert np.array_equal(i1[:t + 1], i2[:t + 1])
     assert not np.allclose(o1[t + 1:], o2[t + 1:])
+
+
+# ---------------------------------------------------------------- decode-time compression state
+def test_append_stream_equals_batch_compression():
+    # feeding a sequence one token at a time must rebuild exactly the entries
+    # the (separately pinned) batch compressor computes, ragged tails included
+    rng = np.random.default_rng(31)
+    for B, n, d_in, d_out, m, overlap in [(2, 37, 16, 24, 4, True), (3, 300, 32, 16, 128, False),
+                                          (1, 9, 8, 8, 1, False), (2, 64, 16, 16, 4, False),
+                                          (1, 4, 8, 8, 4, True)]:
+        x = rng.standard_normal((B, n, d_in))
+        W = rng.standard_normal((d_in, d_out))
+        np.testing.assert_allclose(oracle.compress_stream(x, W, m, overlap),
+                                   oracle.compress(x, W, m, overlap), rtol=0, atol=1e-12)
+
+
+def test_append_writes_only_on_block_completion_and_skips_absent_tokens():
+    rng = np.random.default_rng(32)
+    B, d, m = 3, 8, 4
+    W = rng.standard_normal((d, d))
+    state = np.zeros((B, 2, d))
+    out = np.full((B, 5, d), 7.0)
+    # element 0 at positions 0..3 (completes entry 0 at p=3), element 1 has no token, element 2
+    # starts at position 4 (its first block is absent: only block 1 completes, alone)
+    for p in range(4):
+        x = rng.standard_normal((B, d))
+        done = oracle.compress_append(state, x, W, m, True, np.array([p, -1, 4 + p], np.int32), out, 5)
+        want = [0 if p == 3 else -1, -1, 1 if p == 3 else -1]
+        assert list(done) == want
+    assert np.all(out[1] == 7.0) and np.all(state[1] == 0.0)      # untouched element
+    assert np.all(out[0, 1:] == 7.0) and np.all(out[2, [0, 2, 3, 4]] == 7.0)
+    assert np.all(state[:, 1][[0, 2]] == 0.0)                      # running sums restarted
+
+
+def test_append_constant_input_and_cache_bound():
+    # constant rows c: every entry is c * (column sums of W), overlap or not;
+    # an entry past N_cap is not written but the state still advances
+    d, m, c = 8, 4, 0.75
+    W = np.random.default_rng(33).standard_normal((d, 5))
+    for overlap in (True, False):
+        state = np.zeros((1, 2, d))
+        out = np.zeros((1, 2, 5))
+        for p in range(4 * m):
+            done = oracle.compress_append(state, np.full((1, d), c), W, m, overlap,
+                                          np.array([p], np.int32), out, 2)
+            if (p + 1) % m == 0:
+                assert done[0] == p // m
+        np.testing.assert_allclose(out[0], np.tile(c * W.sum(axis=0), (2, 1)), rtol=0, atol=1e-12)
+        assert np.allclose(state[0, 0], m * c)                   # last complete block's sum
