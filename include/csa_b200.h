@@ -111,6 +111,43 @@ csa_status_t csa_compress(const void* x, int x_dt, int B, int n, int d_in, const
                           float* out_row_scale, void* stream);
 
 /*
+ * csa_compress_append -- decode-time stage 1: one new token per batch element
+ * updates the compressor state and, when it completes a block, writes that
+ * block's compressed entry into the cache.
+ * Follows "DS-V4 分析&学习", opening summary (the KV cache is the compressed
+ * cache plus a state cache and a tail state) and §1.3 (an overlapping entry
+ * spans the previous and the current block, so decode keeps both sums).
+ *
+ *   state[b, 0, :]  sum of the last complete block's m rows        (fp32)
+ *   state[b, 1, :]  running sum of the current block                (fp32)
+ *   For the token at absolute position p = pos[b] (p < 0: element b has no
+ *   token this step and nothing of it changes):
+ *     state[b, 1, :] += x_new[b, :]
+ *     if (p + 1) % m == 0, block j = p / m is complete:
+ *       cache[b, j, :] = (mean of blocks j-1 and j if overlap and j > 0,
+ *                         else of block j alone) @ W       (if j < N_cap)
+ *       n_entries[b] = j + 1                   (if j < N_cap and n_entries != NULL)
+ *       state[b, 0, :] = state[b, 1, :];  state[b, 1, :] = 0
+ *   Feeding positions 0 .. n-1 in order reproduces csa_compress on the whole
+ *   sequence (up to fp32 rounding of the sums).
+ *
+ *   x_new  [B, d_in]        x_dt = CSA_DT_F32 or CSA_DT_BF16
+ *   W      [d_in, d_out]    same dtype as x_new
+ *   pos    device int32 [B]
+ *   state  device fp32 [B, 2, d_in], caller-owned, zero before the first token
+ *   cache  [B, N_cap, d_out]  out_dt as in csa_compress (E4M3: cache_scale
+ *          [B, N_cap] fp32 gets the row's amax/448); cache_scale required iff
+ *          out_dt == CSA_DT_E4M3, else NULL.
+ *   n_entries  device int32 [B] or NULL.
+ *   Limits as csa_compress.  Calls on one state must be ordered (same stream
+ *   or synchronised): each call reads and writes it.
+ */
+csa_status_t csa_compress_append(const void* x_new, int x_dt, int B, int d_in, const void* W,
+                                 int d_out, int m, int overlap, const int* pos, float* state,
+                                 void* cache, int out_dt, float* cache_scale, int N_cap,
+                                 int* n_entries, void* stream);
+
+/*
  * csa_indexer_topk -- stage 2: Lightning-Indexer score + causal per-query
  * top-k, fused: the score matrix never reaches global memory.
  * Follows "百万上下文从「奢侈品」变「日用品」…" §3.2 (query . compressed-key

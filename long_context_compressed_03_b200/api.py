@@ -35,6 +35,7 @@ SIGNATURES = {
     "csa_kernel_launches": (ctypes.c_ulonglong, []),
     "csa_check_device_error": (I, [P, I]),
     "csa_compress": (I, [P, I, I, I, I, P, I, I, I, P, I, P, P]),
+    "csa_compress_append": (I, [P, I, I, I, P, I, I, I, P, P, P, I, P, I, P, P]),
     "csa_indexer_topk": (I, [P, I, P, P, I, P, I, I, I, I, I, P, P, I, I, P, P]),
     "csa_sparse_attn": (I, [P, I, I, I, I, I, P, I, P, I, P, I, P, P, I, P, F, P, P, P]),
     "hca_dense_attn": (I, [P, I, I, I, I, I, P, I, P, I, P, I, P, P, I, P, F, P, P, P]),
@@ -140,6 +141,22 @@ def csa_compress(x: torch.Tensor, W: torch.Tensor, m: int, overlap: bool, out: t
     d_out = W.shape[1]
     _check(load().csa_compress(_ptr(x), _dt(x), B, n, d_in, _ptr(W), d_out, m, int(bool(overlap)),
                                _ptr(out), _dt(out), _ptr(out_row_scale), _stream(stream)))
+
+
+def csa_compress_append(x_new: torch.Tensor, W: torch.Tensor, m: int, overlap: bool,
+                        pos: torch.Tensor, state: torch.Tensor, cache: torch.Tensor,
+                        cache_scale: torch.Tensor | None = None,
+                        n_entries: torch.Tensor | None = None, stream=None) -> None:
+    """x_new [B, d_in], pos [B] int32, state [B, 2, d_in] fp32 (zero before the first
+    token), cache [B, N_cap, d_out] (+ cache_scale [B, N_cap] for fp8)."""
+    B, d_in = x_new.shape
+    d_out = W.shape[1]
+    if state.dtype != torch.float32:
+        raise ValueError("state must be float32")
+    _check(load().csa_compress_append(_ptr(x_new), _dt(x_new), B, d_in, _ptr(W), d_out, m,
+                                      int(bool(overlap)), _i32(pos, "pos"), _ptr(state),
+                                      _ptr(cache), _dt(cache), _ptr(cache_scale), cache.shape[1],
+                                      _i32(n_entries, "n_entries"), _stream(stream)))
 
 
 def csa_indexer_topk(qI: torch.Tensor, kI: torch.Tensor, m: int, topk: int, idx_out: torch.Tensor,

@@ -134,6 +134,37 @@ csa_status_t csa_compress(const void* x, int x_dt, int B, int n, int d_in, const
     return from_cuda(csa::launch_compress(a, static_cast<cudaStream_t>(stream), &why), "csa_compress", why);
 }
 
+csa_status_t csa_compress_append(const void* x_new, int x_dt, int B, int d_in, const void* W,
+                                 int d_out, int m, int overlap, const int* pos, float* state,
+                                 void* cache, int out_dt, float* cache_scale, int N_cap,
+                                 int* n_entries, void* stream) {
+    REQUIRE(B >= 0 && N_cap >= 0, "csa_compress_append: negative B or N_cap");
+    REQUIRE(m >= 1, "csa_compress_append: m must be >= 1");
+    REQUIRE(overlap == 0 || overlap == 1, "csa_compress_append: overlap must be 0 or 1");
+    REQUIRE(is_dt(x_dt) && is_dt(out_dt), "csa_compress_append: unknown dtype");
+    REQUIRE(d_in > 0 && d_out > 0, "csa_compress_append: d_in and d_out must be positive");
+    if (d_in % 16 || d_out % 16 || d_in > 256 || d_out > 256)
+        return fail(CSA_ERR_UNSUPPORTED, "csa_compress_append: d_in, d_out must be multiples of 16 in [16, 256]");
+    if (x_dt == CSA_DT_E4M3) return fail(CSA_ERR_UNSUPPORTED, "csa_compress_append: fp8 input is not supported");
+    if (out_dt == CSA_DT_F32 && x_dt != CSA_DT_F32)
+        return fail(CSA_ERR_UNSUPPORTED, "csa_compress_append: F32 output needs F32 input");
+    REQUIRE((out_dt == CSA_DT_E4M3) == (cache_scale != nullptr),
+            "csa_compress_append: cache_scale is required for E4M3 output and must be NULL otherwise");
+    if (B == 0) return ok();
+    REQUIRE(x_new && W && pos && state, "csa_compress_append: null pointer");
+    REQUIRE(cache || N_cap == 0, "csa_compress_append: null cache");
+    REQUIRE_ALIGNED(x_new, "x_new");
+    REQUIRE_ALIGNED(W, "W");
+    REQUIRE_ALIGNED(state, "state");
+    REQUIRE_ALIGNED(cache, "cache");
+    REQUIRE_ALIGNED(cache_scale, "cache_scale");
+    csa::AppendArgs a{x_new, x_dt, B, d_in, W, d_out, m, overlap, pos, state, cache, out_dt,
+                      cache_scale, N_cap, n_entries};
+    const char* why = nullptr;
+    return from_cuda(csa::launch_compress_append(a, static_cast<cudaStream_t>(stream), &why),
+                     "csa_compress_append", why);
+}
+
 csa_status_t csa_indexer_topk(const void* qI, int qI_dt, const float* qI_scale, const void* kI,
                               int kI_dt, const float* kI_scale, int B, int n_q, int H_I, int d_I,
                               int N_cap, const int* n_entries, const int* q_pos, int m, int topk,

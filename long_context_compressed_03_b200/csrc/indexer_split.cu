@@ -209,9 +209,15 @@ __global__ void __launch_bounds__(kThreads, min_blocks<NU>()) indexer_split_kern
         unsigned* hist = hist_buf + (rd & 1) * 256;    // the other buffer may still be read by peers
         for (int i = tid; i < nbins; i += kThreads) hist[i] = 0;
         __syncthreads();
-        for (int i = tid; i < nloc; i += kThreads) {
-            const unsigned k = keys[i];
-            if ((k & pmask) == prefix) atomicAdd(&hist[(k >> shift) & dmask], 1u);
+        // warp-aggregated: lanes with the same digit add once (the leading
+        // digits of similar scores collide heavily)
+        for (int i0 = 0; i0 < nloc; i0 += kThreads) {
+            const int i = i0 + tid;
+            const unsigned k = i < nloc ? keys[i] : 0u;
+            const bool take = i < nloc && (k & pmask) == prefix;
+            const unsigned d = take ? (k >> shift) & dmask : 0xffffffffu;
+            const unsigned peers = __match_any_sync(0xffffffffu, d);
+            if (take && lane == __ffs(peers) - 1) atomicAdd(&hist[d], (unsigned)__popc(peers));
         }
         cluster.sync();
         // thread t owns the bpt bins just below nbins - bpt t (highest digits first)

@@ -15,6 +15,19 @@ struct CompressArgs {
     int N_c;
 };
 
+struct AppendArgs {
+    const void* x; int x_dt;
+    int B, d_in;
+    const void* W; int d_out;
+    int m, overlap;
+    const int* pos;
+    float* state;
+    void* cache; int out_dt;
+    float* cache_scale;
+    int N_cap;
+    int* n_entries;
+};
+
 struct IndexerArgs {
     const void* qI; int qI_dt; const float* qI_scale;
     const void* kI; int kI_dt; const float* kI_scale;
@@ -68,6 +81,7 @@ void count_launch();
 // reason string when the configuration is unsupported (returned as
 // cudaErrorNotSupported).
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s, const char** why);
+cudaError_t launch_compress_append(const AppendArgs& a, cudaStream_t s, const char** why);
 cudaError_t launch_indexer_topk(const IndexerArgs& a, cudaStream_t s, const char** why);
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s, const char** why);
 

@@ -35,8 +35,8 @@ def _declared():
 
 def test_header_declares_the_four_stage_entry_points():
     d = _declared()
-    for name in ("csa_compress", "csa_indexer_topk", "csa_sparse_attn", "hca_dense_attn",
-                 "csa_status_string", "csa_last_error_detail", "csa_version"):
+    for name in ("csa_compress", "csa_compress_append", "csa_indexer_topk", "csa_sparse_attn",
+                 "hca_dense_attn", "csa_status_string", "csa_last_error_detail", "csa_version"):
         assert name in d
 
 
@@ -82,6 +82,24 @@ def test_compress_validation(lib):
     # no entries (n < m, or B = 0): nothing to do, nothing launched
     assert f(None, 1, 1, 3, 128, None, 128, 4, 1, None, 1, None, None) == api.CSA_OK
     assert f(None, 1, 0, 64, 128, None, 128, 4, 1, None, 1, None, None) == api.CSA_OK
+
+
+def test_compress_append_validation(lib):
+    f = lib.csa_compress_append
+    #       x_new dt B  d_in W    d_out m  ov pos   state cache dt scale N_cap n_ent stream
+    args = [FAKE, 1, 2, 64, FAKE, 64, 4, 1, FAKE, FAKE, FAKE, 1, None, 16, None, None]
+    bad = list(args); bad[6] = 0                       # m = 0
+    assert f(*bad) == api.CSA_ERR_INVALID_ARG
+    bad = list(args); bad[3] = 40                      # d_in not a multiple of 16
+    assert f(*bad) == api.CSA_ERR_UNSUPPORTED
+    bad = list(args); bad[11] = 2                      # fp8 cache without scales
+    assert f(*bad) == api.CSA_ERR_INVALID_ARG
+    bad = list(args); bad[8] = None                    # no positions
+    assert f(*bad) == api.CSA_ERR_INVALID_ARG
+    bad = list(args); bad[9] = ODD                     # misaligned state
+    assert f(*bad) == api.CSA_ERR_MISALIGNED
+    ok = list(args); ok[2] = 0                         # B = 0: no-op
+    assert f(*ok) == api.CSA_OK
 
 
 def test_indexer_validation(lib):

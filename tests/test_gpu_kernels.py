@@ -286,3 +286,51 @@ def test_binding_rejects_host_tensors():
     x = torch.zeros(1, 8, 16)
     with pytest.raises(ValueError):
         api.csa_compress(x, torch.zeros(16, 16), 4, True, torch.zeros(1, 2, 16))
+
+
+# ---------------------------------------------------------------- decode-time compression
+@pytest.mark.parametrize("case", [
+    # (B, n, d_in, d_out, m, overlap, x dtype, cache kind, N_cap)
+    (3, 37, 128, 128, 4, True, torch.bfloat16, "bf16", 16),     # CSA main compressor, ragged
+    (2, 41, 64, 64, 4, True, torch.bfloat16, "e4m3", 12),       # fp8 indexer-key cache
+    (2, 300, 128, 128, 128, False, torch.bfloat16, "bf16", 3),  # HCA ratio
+    (1, 24, 32, 48, 4, False, torch.float32, "f32", 4),         # cache shorter than the stream
+])
+def test_compress_append_stream_matches_oracle(case):
+    """Tokens fed one at a time through csa_compress_append rebuild the entries
+    of the oracle's batch compression (positions staggered per element)."""
+    B, n, d_in, d_out, m, overlap, dt, kind, N_cap = case
+    g = _gen(200 + n)
+    x = _randn(g, B, n, d_in, dtype=dt)
+    W = _randn(g, d_in, d_out, dtype=dt, std=1 / math.sqrt(d_in))
+    start = np.arange(B) * 3                     # element b starts its sequence at step 3b
+    steps = n + int(start.max())
+    state = torch.zeros(B, 2, d_in, dtype=torch.float32, device=DEV)
+    if kind == "e4m3":
+        cache = torch.zeros(B, N_cap, d_out, dtype=torch.uint8, device=DEV)
+        scale = torch.zeros(B, N_cap, dtype=torch.float32, device=DEV)
+    else:
+        cache = torch.zeros(B, N_cap, d_out, dtype=torch.float32 if kind == "f32" else torch.bfloat16,
+                            device=DEV)
+        scale = None
+    n_ent = torch.zeros(B, dtype=torch.int32, device=DEV)
+    xd, Wd = x.to(DEV), W.to(DEV)
+    rows = torch.arange(B, device=DEV)
+    for s in range(steps):
+        p = s - start
+        pos = torch.from_numpy(np.where((p >= 0) & (p < n), p, -1).astype(np.int32)).to(DEV)
+        tok = xd[rows, torch.from_numpy(np.clip(p, 0, n - 1)).to(DEV)].contiguous()
+        api.csa_compress_append(tok, Wd, m, overlap, pos, state, cache, cache_scale=scale,
+                                n_entries=n_ent)
+    torch.cuda.synchronize()
+    ref = oracle.compress(np64(x), np64(W), m, overlap)
+    N_w = min(N_cap, ref.shape[1])
+    assert np.array_equal(n_ent.cpu().numpy(), np.full(B, min(n // m, N_cap), np.int32))
+    if kind == "e4m3":
+        deq = oracle.dequantize_rows_e4m3(cache.cpu().numpy()[:, :N_w], scale.cpu().numpy()[:, :N_w])
+        r = ref[:, :N_w]
+        sc = scale.cpu().numpy()[:, :N_w]
+        np.testing.assert_allclose(sc, np.abs(r).max(axis=-1) / 448.0, rtol=1e-5)
+        assert np.all(np.abs(deq - r) <= np.abs(r) * 2.0 ** -3 + sc[..., None] * 2.0 ** -9)
+    else:
+        check_out(np64(cache)[:, :N_w], ref[:, :N_w], torch.float32 if kind == "f32" else torch.bfloat16)
