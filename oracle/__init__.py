@@ -61,6 +61,7 @@ def _load():
         lib.oracle_e4m3_encode.argtypes = [ctypes.c_float]
         lib.oracle_e4m3_encode.restype = ctypes.c_uint8
         lib.oracle_quantize_rows_e4m3.argtypes = [P, i64, i32, P, P]
+        lib.oracle_hadamard_rows_f32.argtypes = [P, i64, i32]
         lib.oracle_num_entries.argtypes = [i64, i64]
         lib.oracle_num_entries.restype = i64
         lib.oracle_visible_entries.argtypes = [i64, i32, i64]
@@ -124,6 +125,16 @@ def quantize_rows_e4m3(x) -> tuple[np.ndarray, np.ndarray]:
     scales = np.empty(a.shape[:-1], dtype=np.float32)
     _load().oracle_quantize_rows_e4m3(_ptr(a), rows, d, _ptr(codes), _ptr(scales))
     return codes, scales
+
+
+def hadamard_rows_f32(x) -> np.ndarray:
+    """Rows rotated by the normalised Walsh-Hadamard matrix, in fp32, in the
+    fixed butterfly order the kernels use (see csa_oracle.c)."""
+    a = np.array(x, dtype=np.float32, copy=True, order="C")
+    d = a.shape[-1]
+    assert d > 0 and d & (d - 1) == 0, "d must be a power of two"
+    _load().oracle_hadamard_rows_f32(_ptr(a), a.size // d, d)
+    return a
 
 
 def dequantize_rows_e4m3(codes, scales) -> np.ndarray:
@@ -221,10 +232,14 @@ def _keys_arg(kI, kI_scale):
     return None, c, sc, (None, _ptr(c), _ptr(sc))
 
 
-def quantized_query_rows(qI_rows) -> np.ndarray:
+def quantized_query_rows(qI_rows, rotate: bool = False) -> np.ndarray:
     """fp64 values of query rows after the per-(row, head) E4M3 quantisation
-    the indexer applies to bf16 queries against fp8 keys (fp32 procedure)."""
+    the indexer applies to bf16 queries against fp8 keys (fp32 procedure);
+    with ``rotate`` the rows are Hadamard-rotated (fp32) first, as against
+    rotated keys."""
     q = np.asarray(qI_rows, dtype=np.float32)
+    if rotate:
+        q = hadamard_rows_f32(q)
     codes, scales = quantize_rows_e4m3(q)
     return dequantize_rows_e4m3(codes, scales)
 

@@ -116,6 +116,32 @@ void oracle_quantize_rows_e4m3(const float* x, long rows, int d, uint8_t* codes,
 }
 
 /* ------------------------------------------------------------------------
+ * Hadamard rotation of indexer rows before fp8 (the survey's NEXT-2 reading
+ * of the DSA-lineage indexer that "DS-V4 分析&学习" §1.2 and the gitcode
+ * analysis name: a rotation spreads outlier channels before E4M3, and dot
+ * products are unchanged because the normalised Walsh-Hadamard matrix H_d is
+ * orthonormal and symmetric).  In place, in fp32, in a fixed order that the
+ * kernels reproduce exactly: for stride s = 1, 2, 4, ..., d/2 every pair
+ * (i, i + s) with i & s == 0 becomes (x_i + x_{i+s}, x_i - x_{i+s}); then every
+ * value is multiplied by fp32(1/sqrt(d)).  d is a power of two.
+ * --------------------------------------------------------------------- */
+void oracle_hadamard_rows_f32(float* x, long rows, int d) {
+    const float norm = (float)(1.0 / sqrt((double)d));
+    for (long r = 0; r < rows; ++r) {
+        float* row = x + r * (long)d;
+        for (int s = 1; s < d; s <<= 1) {
+            for (int i = 0; i < d; ++i) {
+                if (i & s) continue;
+                const float a = row[i], b = row[i + s];
+                row[i] = a + b;
+                row[i + s] = a - b;
+            }
+        }
+        for (int i = 0; i < d; ++i) row[i] = row[i] * norm;
+    }
+}
+
+/* ------------------------------------------------------------------------
  * Stage 1: KV compression ([P5] §3.2 formula; [P3] §1.3; [P1] §3.2).
  *
  * out[b, i, :] = (mean over p in win(i) of x[b, p, :]) @ W,   i < floor(n/m)

@@ -487,3 +487,43 @@ def test_append_constant_input_and_cache_bound():
                 assert done[0] == p // m
         np.testing.assert_allclose(out[0], np.tile(c * W.sum(axis=0), (2, 1)), rtol=0, atol=1e-12)
         assert np.allclose(state[0, 0], m * c)                   # last complete block's sum
+
+
+# ---------------------------------------------------------------- Hadamard rotation (indexer rows)
+def _sylvester(d):
+    H = np.array([[1.0]])
+    while H.shape[0] < d:
+        H = np.block([[H, H], [H, -H]])
+    return H / np.sqrt(d)
+
+
+def test_hadamard_rows_match_the_sylvester_matrix():
+    rng = np.random.default_rng(41)
+    for d in (16, 64, 128):
+        x = rng.standard_normal((5, d)).astype(np.float32)
+        got = oracle.hadamard_rows_f32(x).astype(np.float64)
+        want = x.astype(np.float64) @ _sylvester(d).T
+        np.testing.assert_allclose(got, want, rtol=0, atol=1e-5 * np.abs(want).max())
+
+
+def test_hadamard_is_an_involution_and_keeps_dot_products():
+    rng = np.random.default_rng(42)
+    q = rng.standard_normal((64, 64)).astype(np.float32)
+    k = rng.standard_normal((64, 64)).astype(np.float32)
+    hq, hk = oracle.hadamard_rows_f32(q), oracle.hadamard_rows_f32(k)
+    np.testing.assert_allclose(oracle.hadamard_rows_f32(hq), q, rtol=0, atol=1e-5)
+    dots = (q.astype(np.float64) * k).sum(-1)
+    hdots = (hq.astype(np.float64) * hk).sum(-1)
+    np.testing.assert_allclose(hdots, dots, rtol=0, atol=1e-4)
+    # an outlier channel is spread over every coordinate: the row amax drops
+    x = np.zeros((1, 64), np.float32)
+    x[0, 5] = 100.0
+    assert np.allclose(np.abs(oracle.hadamard_rows_f32(x)), 12.5)
+
+
+def test_rotated_query_quantisation_is_rotate_then_quantise():
+    rng = np.random.default_rng(43)
+    q = rng.standard_normal((7, 4, 64)).astype(np.float32)
+    codes, scales = oracle.quantize_rows_e4m3(oracle.hadamard_rows_f32(q))
+    np.testing.assert_array_equal(oracle.quantized_query_rows(q, rotate=True),
+                                  oracle.dequantize_rows_e4m3(codes, scales))
