@@ -60,7 +60,9 @@ typedef enum {
 typedef enum {
     CSA_DT_F32 = 0,   /* IEEE binary32 */
     CSA_DT_BF16 = 1,  /* bfloat16 */
-    CSA_DT_E4M3 = 2   /* OCP FP8 E4M3 with one fp32 scale per row */
+    CSA_DT_E4M3 = 2,  /* OCP FP8 E4M3 with one fp32 scale per row */
+    CSA_DT_E4M3_HADAMARD = 3  /* as CSA_DT_E4M3, of rows rotated first by the normalised
+                                 Walsh-Hadamard matrix (indexer keys; see csa_compress) */
 } csa_dtype_t;
 
 /* Static text of a status code ("CSA_OK", ...). */
@@ -102,7 +104,16 @@ csa_status_t csa_check_device_error(void* stream, int clear);
  *           CSA_DT_E4M3 (uint8 codes; out_row_scale [B, floor(n/m)] fp32 gets
  *           amax/448 of the row, 1 for a zero row; code = E4M3(v/scale),
  *           nearest-even, saturating)
- *   out_row_scale  required iff out_dt == CSA_DT_E4M3, else must be NULL.
+ *           CSA_DT_E4M3_HADAMARD: as CSA_DT_E4M3, of the row rotated first by
+ *           the normalised Walsh-Hadamard matrix H (d_out a power of two): in
+ *           fp32, for stride s = 1, 2, ..., d_out/2 each pair (i, i+s) with
+ *           i & s == 0 becomes (x_i + x_{i+s}, x_i - x_{i+s}), then every value
+ *           is multiplied by fp32(1/sqrt(d_out)).  H is orthonormal, so
+ *           indexer scores against rotated queries are unchanged up to the fp8
+ *           rounding, which the rotation spreads over all channels (a reading
+ *           of the DSA-lineage fp8 indexer that "DS-V4 分析&学习" §1.2 builds
+ *           on; no formula for it is printed there).
+ *   out_row_scale  required iff out_dt is an E4M3 type, else must be NULL.
  *   Limits: 16 <= d_in, d_out <= 256 and multiples of 16; m >= 1.
  *   Pooling and the projection accumulate in fp32.
  */
@@ -135,9 +146,10 @@ csa_status_t csa_compress(const void* x, int x_dt, int B, int n, int d_in, const
  *   W      [d_in, d_out]    same dtype as x_new
  *   pos    device int32 [B]
  *   state  device fp32 [B, 2, d_in], caller-owned, zero before the first token
- *   cache  [B, N_cap, d_out]  out_dt as in csa_compress (E4M3: cache_scale
- *          [B, N_cap] fp32 gets the row's amax/448); cache_scale required iff
- *          out_dt == CSA_DT_E4M3, else NULL.
+ *   cache  [B, N_cap, d_out]  out_dt as in csa_compress (E4M3 types:
+ *          cache_scale [B, N_cap] fp32 gets the row's amax/448; the Hadamard
+ *          type rotates the row first); cache_scale required iff out_dt is an
+ *          E4M3 type, else NULL.
  *   n_entries  device int32 [B] or NULL.
  *   Limits as csa_compress.  Calls on one state must be ordered (same stream
  *   or synchronised): each call reads and writes it.
@@ -164,6 +176,11 @@ csa_status_t csa_compress_append(const void* x_new, int x_dt, int B, int d_in, c
  *      With kI_dt == CSA_DT_E4M3 and qI_dt == CSA_DT_BF16 (qI_scale NULL), each
  *      (query, head) row is quantised in the kernel exactly as csa_compress
  *      quantises a row (fp32: scale = amax/448, code = E4M3(x/scale)).
+ *      With kI_dt == CSA_DT_E4M3_HADAMARD (keys from csa_compress with that
+ *      type), a bf16 query row is rotated the same way before it is
+ *      quantised; E4M3 query codes (qI_dt == CSA_DT_E4M3) are taken as given
+ *      (already rotated).  Needs d_I a power of two; served by the fp8
+ *      tensor-core and cluster kernels (d_I 64, or 128 for few rows).
  *   kI [B, N_cap, d_I]: kI_dt F32, BF16, or E4M3 with kI_scale [B, N_cap].
  *      Supported pairs: (F32,F32), (BF16,BF16), (BF16,E4M3), (E4M3,E4M3).
  *      With fp8 the score is sk_s * sum_h sq_h * ReLU(q8_h . k8_s).

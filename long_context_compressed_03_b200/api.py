@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(_PKG, "libcsa_b200.so")
 
 CSA_OK, CSA_ERR_INVALID_ARG, CSA_ERR_UNSUPPORTED, CSA_ERR_MISALIGNED, CSA_ERR_CUDA, \
     CSA_ERR_TIMEOUT = range(6)
-DT_F32, DT_BF16, DT_E4M3 = 0, 1, 2
+DT_F32, DT_BF16, DT_E4M3, DT_E4M3_HADAMARD = 0, 1, 2, 3
 
 # symbol -> (restype, argtypes); mirrors include/csa_b200.h
 P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
@@ -104,6 +104,16 @@ def _dt(t: torch.Tensor) -> int:
     raise ValueError(f"unsupported dtype {t.dtype}")
 
 
+def _dt_rot(t: torch.Tensor, rotated: bool) -> int:
+    """dtype code of an fp8 tensor whose rows are (or are to be) Hadamard-rotated."""
+    d = _dt(t)
+    if rotated:
+        if d != DT_E4M3:
+            raise ValueError("Hadamard rotation applies to fp8 (uint8 / float8_e4m3fn) rows only")
+        return DT_E4M3_HADAMARD
+    return d
+
+
 def _stream(stream) -> ctypes.c_void_p:
     if stream is None:
         stream = torch.cuda.current_stream()
@@ -135,38 +145,47 @@ def csa_check_device_error(clear: bool = True, stream=None) -> None:
 
 
 def csa_compress(x: torch.Tensor, W: torch.Tensor, m: int, overlap: bool, out: torch.Tensor,
-                 out_row_scale: torch.Tensor | None = None, stream=None) -> None:
-    """x [B, n, d_in], W [d_in, d_out] -> out [B, n//m, d_out] (+ scales for fp8)."""
+                 out_row_scale: torch.Tensor | None = None, hadamard: bool = False,
+                 stream=None) -> None:
+    """x [B, n, d_in], W [d_in, d_out] -> out [B, n//m, d_out] (+ scales for fp8;
+    ``hadamard``: fp8 rows rotated by the normalised Walsh-Hadamard matrix first)."""
     B, n, d_in = x.shape
     d_out = W.shape[1]
     _check(load().csa_compress(_ptr(x), _dt(x), B, n, d_in, _ptr(W), d_out, m, int(bool(overlap)),
-                               _ptr(out), _dt(out), _ptr(out_row_scale), _stream(stream)))
+                               _ptr(out), _dt_rot(out, hadamard), _ptr(out_row_scale),
+                               _stream(stream)))
 
 
 def csa_compress_append(x_new: torch.Tensor, W: torch.Tensor, m: int, overlap: bool,
                         pos: torch.Tensor, state: torch.Tensor, cache: torch.Tensor,
                         cache_scale: torch.Tensor | None = None,
-                        n_entries: torch.Tensor | None = None, stream=None) -> None:
+                        n_entries: torch.Tensor | None = None, hadamard: bool = False,
+                        stream=None) -> None:
     """x_new [B, d_in], pos [B] int32, state [B, 2, d_in] fp32 (zero before the first
-    token), cache [B, N_cap, d_out] (+ cache_scale [B, N_cap] for fp8)."""
+    token), cache [B, N_cap, d_out] (+ cache_scale [B, N_cap] for fp8; ``hadamard`` as
+    in csa_compress)."""
     B, d_in = x_new.shape
     d_out = W.shape[1]
     if state.dtype != torch.float32:
         raise ValueError("state must be float32")
     _check(load().csa_compress_append(_ptr(x_new), _dt(x_new), B, d_in, _ptr(W), d_out, m,
                                       int(bool(overlap)), _i32(pos, "pos"), _ptr(state),
-                                      _ptr(cache), _dt(cache), _ptr(cache_scale), cache.shape[1],
+                                      _ptr(cache), _dt_rot(cache, hadamard), _ptr(cache_scale),
+                                      cache.shape[1],
                                       _i32(n_entries, "n_entries"), _stream(stream)))
 
 
 def csa_indexer_topk(qI: torch.Tensor, kI: torch.Tensor, m: int, topk: int, idx_out: torch.Tensor,
                      qI_scale: torch.Tensor | None = None, kI_scale: torch.Tensor | None = None,
                      n_entries: torch.Tensor | None = None, q_pos: torch.Tensor | None = None,
-                     stream=None) -> None:
-    """qI [B, n_q, H_I, d_I], kI [B, N_cap, d_I] -> idx_out [B, n_q, topk] int32."""
+                     kI_rotated: bool = False, stream=None) -> None:
+    """qI [B, n_q, H_I, d_I], kI [B, N_cap, d_I] -> idx_out [B, n_q, topk] int32.
+    ``kI_rotated``: fp8 keys written with the Hadamard rotation (bf16 queries are
+    rotated in the kernel; fp8 query codes are taken as already rotated)."""
     B, n_q, H_I, d_I = qI.shape
     N_cap = kI.shape[1]
-    _check(load().csa_indexer_topk(_ptr(qI), _dt(qI), _ptr(qI_scale), _ptr(kI), _dt(kI),
+    _check(load().csa_indexer_topk(_ptr(qI), _dt(qI), _ptr(qI_scale), _ptr(kI),
+                                   _dt_rot(kI, kI_rotated),
                                    _ptr(kI_scale), B, n_q, H_I, d_I, N_cap,
                                    _i32(n_entries, "n_entries"), _i32(q_pos, "q_pos"), m, topk,
                                    _i32(idx_out, "idx_out"), _stream(stream)))
@@ -203,7 +222,7 @@ def hca_dense_attn(q: torch.Tensor, kv_c: torch.Tensor, m: int, kv_raw: torch.Te
 
 # ---------------------------------------------------------------- allocating wrappers
 def compress(x: torch.Tensor, W: torch.Tensor, m: int, overlap: bool, out_dtype=None,
-             stream=None):
+             hadamard: bool = False, stream=None):
     """Returns out (and the per-row scales when out_dtype is fp8: (codes, scales))."""
     B, n, _ = x.shape
     N_c = n // m
@@ -211,7 +230,7 @@ def compress(x: torch.Tensor, W: torch.Tensor, m: int, overlap: bool, out_dtype=
     if out_dtype in (torch.uint8, torch.float8_e4m3fn):
         out = torch.empty(B, N_c, W.shape[1], dtype=torch.uint8, device=x.device)
         scale = torch.empty(B, N_c, dtype=torch.float32, device=x.device)
-        csa_compress(x, W, m, overlap, out, scale, stream=stream)
+        csa_compress(x, W, m, overlap, out, scale, hadamard=hadamard, stream=stream)
         return out, scale
     out = torch.empty(B, N_c, W.shape[1], dtype=out_dtype, device=x.device)
     csa_compress(x, W, m, overlap, out, stream=stream)
@@ -219,11 +238,11 @@ def compress(x: torch.Tensor, W: torch.Tensor, m: int, overlap: bool, out_dtype=
 
 
 def indexer_topk(qI, kI, m: int, topk: int, qI_scale=None, kI_scale=None, n_entries=None,
-                 q_pos=None, stream=None) -> torch.Tensor:
+                 q_pos=None, kI_rotated: bool = False, stream=None) -> torch.Tensor:
     B, n_q = qI.shape[:2]
     idx = torch.empty(B, n_q, topk, dtype=torch.int32, device=qI.device)
     csa_indexer_topk(qI, kI, m, topk, idx, qI_scale=qI_scale, kI_scale=kI_scale,
-                     n_entries=n_entries, q_pos=q_pos, stream=stream)
+                     n_entries=n_entries, q_pos=q_pos, kI_rotated=kI_rotated, stream=stream)
     return idx
 
 
@@ -242,16 +261,19 @@ def hca_attn(q, kv_c, m: int, kv_raw, window: int, with_lse: bool = False, **kw)
 
 
 def csa_prefill(q, kv, qI, kI_raw, W_c, W_Ic, m: int, topk: int, window: int,
-                indexer_fp8: bool, stream=None):
+                indexer_fp8: bool, indexer_hadamard: bool = False, stream=None):
     """The whole CSA prefill hot path (positions 0..n-1 of each sequence):
     compress kv, compress the indexer keys (fp8 + row scales when
-    ``indexer_fp8``), indexer + top-k, joint sparse attention.
+    ``indexer_fp8``, Hadamard-rotated first when ``indexer_hadamard``),
+    indexer + top-k, joint sparse attention.
     Returns dict(out, idx, kv_c, kI_c, kI_scale)."""
     kv_c = compress(kv, W_c, m, True, stream=stream)
+    rot = bool(indexer_fp8 and indexer_hadamard)
     if indexer_fp8:
-        kI_c, kI_scale = compress(kI_raw, W_Ic, m, True, out_dtype=torch.uint8, stream=stream)
+        kI_c, kI_scale = compress(kI_raw, W_Ic, m, True, out_dtype=torch.uint8, hadamard=rot,
+                                  stream=stream)
     else:
         kI_c, kI_scale = compress(kI_raw, W_Ic, m, True, stream=stream), None
-    idx = indexer_topk(qI, kI_c, m, topk, kI_scale=kI_scale, stream=stream)
+    idx = indexer_topk(qI, kI_c, m, topk, kI_scale=kI_scale, kI_rotated=rot, stream=stream)
     out = sparse_attn(q, kv_c, idx, kv, window, stream=stream)
     return dict(out=out, idx=idx, kv_c=kv_c, kI_c=kI_c, kI_scale=kI_scale)

@@ -7,7 +7,27 @@
 
 namespace csa {
 
-enum Dtype : int { DT_F32 = 0, DT_BF16 = 1, DT_E4M3 = 2 };
+enum Dtype : int { DT_F32 = 0, DT_BF16 = 1, DT_E4M3 = 2, DT_E4M3H = 3 };
+
+// Normalised Walsh-Hadamard rotation of a row of d fp32 values (d a power of
+// two) in shared memory, by one warp, in the order the fp8 Hadamard type
+// defines: for stride s = 1, 2, ..., d/2 every pair (i, i+s) with i & s == 0
+// becomes (x_i + x_{i+s}, x_i - x_{i+s}); then each value is multiplied by
+// norm = fp32(1/sqrt(d)) (computed on the host, passed in).
+__device__ __forceinline__ void hadamard_row_warp(float* row, int d, float norm) {
+    const int lane = threadIdx.x & 31;
+    for (int s = 1; s < d; s <<= 1) {
+        for (int p = lane; p < d / 2; p += 32) {
+            const int i = (p / s) * 2 * s + (p % s);
+            const float a = row[i], b = row[i + s];
+            row[i] = a + b;
+            row[i + s] = a - b;
+        }
+        __syncwarp();
+    }
+    for (int i = lane; i < d; i += 32) row[i] = row[i] * norm;
+    __syncwarp();
+}
 
 __device__ __forceinline__ float to_f32(float v) { return v; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 v) { return __bfloat162float(v); }

@@ -16,7 +16,8 @@
 //    32 rows at a time; each thread accumulates 8 entries x 4 outputs, the
 //    pooled values of a warp's 8 entries being broadcast reads.
 //  * Epilogue: bf16/fp32 stores, or per-row amax across a warp and E4M3
-//    quantisation (IEEE division, round to nearest even, saturating).
+//    quantisation (IEEE division, round to nearest even, saturating), for the
+//    Hadamard type after the warp rotates the row in shared memory.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -107,10 +108,11 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(CompressArgs a) {
     __syncthreads();
 
     const size_t row0 = (size_t)b * N_c + i0;
-    if constexpr (OUT == DT_E4M3) {
+    if constexpr (OUT == DT_E4M3 || OUT == DT_E4M3H) {
         const int warp = tid >> 5, lane = tid & 31;
         uint8_t* out = static_cast<uint8_t*>(a.out);
         for (int e = warp; e < ne; e += kThreads / 32) {
+            if constexpr (OUT == DT_E4M3H) hadamard_row_warp(outs + e * d_out, d_out, a.hnorm);
             float amax = 0.0f;
             for (int o = lane; o < d_out; o += 32) amax = fmaxf(amax, fabsf(outs[e * d_out + o]));
             for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
@@ -147,9 +149,11 @@ cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s, const char** 
         if (a.out_dt == DT_F32) return launch_t<float, DT_F32>(a, s);
         if (a.out_dt == DT_BF16) return launch_t<float, DT_BF16>(a, s);
         if (a.out_dt == DT_E4M3) return launch_t<float, DT_E4M3>(a, s);
+        if (a.out_dt == DT_E4M3H) return launch_t<float, DT_E4M3H>(a, s);
     } else if (a.x_dt == DT_BF16) {
         if (a.out_dt == DT_BF16) return launch_t<__nv_bfloat16, DT_BF16>(a, s);
         if (a.out_dt == DT_E4M3) return launch_t<__nv_bfloat16, DT_E4M3>(a, s);
+        if (a.out_dt == DT_E4M3H) return launch_t<__nv_bfloat16, DT_E4M3H>(a, s);
     }
     *why = "csa_compress: unsupported (x_dt, out_dt) pair";
     return cudaErrorNotSupported;

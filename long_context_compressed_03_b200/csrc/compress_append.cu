@@ -10,7 +10,8 @@
 // One CTA per batch element: the state update is a d_in-wide vector add, the
 // completed entry a d_in x d_out product with W read through L2 (fp32 FMA,
 // pooled row staged in shared memory), and the E4M3 epilogue reduces the
-// row's amax across the CTA.  The work per step is a few KB: the launch is
+// row's amax across the CTA (after one warp rotates the row, for the
+// Hadamard type).  The work per step is a few KB: the launch is
 // bound by latency, not bandwidth.
 #include "common.cuh"
 #include "kernels.h"
@@ -56,7 +57,11 @@ __global__ void __launch_bounds__(kThreads) compress_append_kernel(AppendArgs a)
     }
     __syncthreads();
     const size_t row = (size_t)b * a.N_cap + j;
-    if constexpr (OUT == DT_E4M3) {
+    if constexpr (OUT == DT_E4M3 || OUT == DT_E4M3H) {
+        if constexpr (OUT == DT_E4M3H) {
+            if (tid < 32) hadamard_row_warp(outs, d_out, a.hnorm);
+            __syncthreads();
+        }
         float amax = 0.0f;
         for (int o = tid; o < d_out; o += kThreads) amax = fmaxf(amax, fabsf(outs[o]));
         for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
@@ -92,9 +97,11 @@ cudaError_t launch_compress_append(const AppendArgs& a, cudaStream_t s, const ch
         if (a.out_dt == DT_F32) return launch_t<float, DT_F32>(a, s);
         if (a.out_dt == DT_BF16) return launch_t<float, DT_BF16>(a, s);
         if (a.out_dt == DT_E4M3) return launch_t<float, DT_E4M3>(a, s);
+        if (a.out_dt == DT_E4M3H) return launch_t<float, DT_E4M3H>(a, s);
     } else if (a.x_dt == DT_BF16) {
         if (a.out_dt == DT_BF16) return launch_t<__nv_bfloat16, DT_BF16>(a, s);
         if (a.out_dt == DT_E4M3) return launch_t<__nv_bfloat16, DT_E4M3>(a, s);
+        if (a.out_dt == DT_E4M3H) return launch_t<__nv_bfloat16, DT_E4M3H>(a, s);
     }
     *why = "csa_compress_append: unsupported (x_dt, out_dt) pair";
     return cudaErrorNotSupported;

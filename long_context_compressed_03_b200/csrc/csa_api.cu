@@ -8,6 +8,8 @@
 #include <cstdio>
 #include <cstring>
 
+#include <cmath>
+
 #include "csa_b200.h"
 #include "kernels.h"
 
@@ -65,7 +67,13 @@ csa_status_t from_cuda(cudaError_t e, const char* what, const char* why) {
         if ((p) && !aligned16(p)) return fail(CSA_ERR_MISALIGNED, "%s is not 16-byte aligned", name); \
     } while (0)
 
-bool is_dt(int d) { return d == CSA_DT_F32 || d == CSA_DT_BF16 || d == CSA_DT_E4M3; }
+bool is_dt(int d) {
+    return d == CSA_DT_F32 || d == CSA_DT_BF16 || d == CSA_DT_E4M3 || d == CSA_DT_E4M3_HADAMARD;
+}
+bool is_fp8(int d) { return d == CSA_DT_E4M3 || d == CSA_DT_E4M3_HADAMARD; }
+bool pow2(int v) { return v > 0 && (v & (v - 1)) == 0; }
+// fp32(1/sqrt(d)), rounded as the oracle rounds it
+float hadamard_norm(int d) { return (float)(1.0 / std::sqrt((double)d)); }
 
 }  // namespace
 
@@ -117,10 +125,12 @@ csa_status_t csa_compress(const void* x, int x_dt, int B, int n, int d_in, const
     REQUIRE(d_in > 0 && d_out > 0, "csa_compress: d_in and d_out must be positive");
     if (d_in % 16 || d_out % 16 || d_in > 256 || d_out > 256)
         return fail(CSA_ERR_UNSUPPORTED, "csa_compress: d_in, d_out must be multiples of 16 in [16, 256]");
-    if (x_dt == CSA_DT_E4M3) return fail(CSA_ERR_UNSUPPORTED, "csa_compress: fp8 input is not supported");
+    if (is_fp8(x_dt)) return fail(CSA_ERR_UNSUPPORTED, "csa_compress: fp8 input is not supported");
+    if (out_dt == CSA_DT_E4M3_HADAMARD && !pow2(d_out))
+        return fail(CSA_ERR_UNSUPPORTED, "csa_compress: the Hadamard fp8 type needs d_out a power of two");
     if (out_dt == CSA_DT_F32 && x_dt != CSA_DT_F32)
         return fail(CSA_ERR_UNSUPPORTED, "csa_compress: F32 output needs F32 input");
-    REQUIRE((out_dt == CSA_DT_E4M3) == (out_row_scale != nullptr),
+    REQUIRE(is_fp8(out_dt) == (out_row_scale != nullptr),
             "csa_compress: out_row_scale is required for E4M3 output and must be NULL otherwise");
     const int N_c = n / m;
     if ((long)B * N_c == 0) return ok();
@@ -129,7 +139,8 @@ csa_status_t csa_compress(const void* x, int x_dt, int B, int n, int d_in, const
     REQUIRE_ALIGNED(W, "W");
     REQUIRE_ALIGNED(out, "out");
     REQUIRE_ALIGNED(out_row_scale, "out_row_scale");
-    csa::CompressArgs a{x, x_dt, B, n, d_in, W, d_out, m, overlap, out, out_dt, out_row_scale, N_c};
+    csa::CompressArgs a{x, x_dt, B, n, d_in, W, d_out, m, overlap, out, out_dt, out_row_scale, N_c,
+                        hadamard_norm(d_out)};
     const char* why = nullptr;
     return from_cuda(csa::launch_compress(a, static_cast<cudaStream_t>(stream), &why), "csa_compress", why);
 }
@@ -145,10 +156,12 @@ csa_status_t csa_compress_append(const void* x_new, int x_dt, int B, int d_in, c
     REQUIRE(d_in > 0 && d_out > 0, "csa_compress_append: d_in and d_out must be positive");
     if (d_in % 16 || d_out % 16 || d_in > 256 || d_out > 256)
         return fail(CSA_ERR_UNSUPPORTED, "csa_compress_append: d_in, d_out must be multiples of 16 in [16, 256]");
-    if (x_dt == CSA_DT_E4M3) return fail(CSA_ERR_UNSUPPORTED, "csa_compress_append: fp8 input is not supported");
+    if (is_fp8(x_dt)) return fail(CSA_ERR_UNSUPPORTED, "csa_compress_append: fp8 input is not supported");
+    if (out_dt == CSA_DT_E4M3_HADAMARD && !pow2(d_out))
+        return fail(CSA_ERR_UNSUPPORTED, "csa_compress_append: the Hadamard fp8 type needs d_out a power of two");
     if (out_dt == CSA_DT_F32 && x_dt != CSA_DT_F32)
         return fail(CSA_ERR_UNSUPPORTED, "csa_compress_append: F32 output needs F32 input");
-    REQUIRE((out_dt == CSA_DT_E4M3) == (cache_scale != nullptr),
+    REQUIRE(is_fp8(out_dt) == (cache_scale != nullptr),
             "csa_compress_append: cache_scale is required for E4M3 output and must be NULL otherwise");
     if (B == 0) return ok();
     REQUIRE(x_new && W && pos && state, "csa_compress_append: null pointer");
@@ -159,7 +172,7 @@ csa_status_t csa_compress_append(const void* x_new, int x_dt, int B, int d_in, c
     REQUIRE_ALIGNED(cache, "cache");
     REQUIRE_ALIGNED(cache_scale, "cache_scale");
     csa::AppendArgs a{x_new, x_dt, B, d_in, W, d_out, m, overlap, pos, state, cache, out_dt,
-                      cache_scale, N_cap, n_entries};
+                      cache_scale, N_cap, n_entries, hadamard_norm(d_out)};
     const char* why = nullptr;
     return from_cuda(csa::launch_compress_append(a, static_cast<cudaStream_t>(stream), &why),
                      "csa_compress_append", why);
@@ -175,10 +188,14 @@ csa_status_t csa_indexer_topk(const void* qI, int qI_dt, const float* qI_scale, 
     REQUIRE(topk >= 1 && topk <= 2048, "csa_indexer_topk: topk must be in [1, 2048]");
     REQUIRE(is_dt(qI_dt) && is_dt(kI_dt), "csa_indexer_topk: unknown dtype");
     if (d_I % 16) return fail(CSA_ERR_UNSUPPORTED, "csa_indexer_topk: d_I must be a multiple of 16");
+    if (qI_dt == CSA_DT_E4M3_HADAMARD)
+        return fail(CSA_ERR_UNSUPPORTED, "csa_indexer_topk: give rotated query codes as CSA_DT_E4M3");
     REQUIRE((qI_dt == CSA_DT_E4M3) == (qI_scale != nullptr),
             "csa_indexer_topk: qI_scale is required iff qI is E4M3");
-    REQUIRE((kI_dt == CSA_DT_E4M3) == (kI_scale != nullptr),
+    REQUIRE(is_fp8(kI_dt) == (kI_scale != nullptr),
             "csa_indexer_topk: kI_scale is required iff kI is E4M3");
+    if (kI_dt == CSA_DT_E4M3_HADAMARD && !pow2(d_I))
+        return fail(CSA_ERR_UNSUPPORTED, "csa_indexer_topk: Hadamard keys need d_I a power of two");
     if ((long)B * n_q == 0) return ok();
     REQUIRE(qI && idx_out, "csa_indexer_topk: null tensor pointer");
     REQUIRE(kI || N_cap == 0, "csa_indexer_topk: null kI");
@@ -190,7 +207,7 @@ csa_status_t csa_indexer_topk(const void* qI, int qI_dt, const float* qI_scale, 
     REQUIRE_ALIGNED(n_entries, "n_entries");
     REQUIRE_ALIGNED(q_pos, "q_pos");
     csa::IndexerArgs a{qI, qI_dt, qI_scale, kI, kI_dt, kI_scale, B, n_q, H_I, d_I, N_cap,
-                       n_entries, q_pos, m, topk, idx_out};
+                       n_entries, q_pos, m, topk, idx_out, hadamard_norm(d_I)};
     const char* why = nullptr;
     return from_cuda(csa::launch_indexer_topk(a, static_cast<cudaStream_t>(stream), &why),
                      "csa_indexer_topk", why);
@@ -200,8 +217,8 @@ static csa_status_t attention_common(const char* name, csa::AttnArgs& a, void* s
     REQUIRE(a.B >= 0 && a.n_q >= 0 && a.N_cap >= 0 && a.L_raw >= 0, "%s: negative size", name);
     REQUIRE(a.H >= 1 && a.D >= 1, "%s: H and D must be positive", name);
     REQUIRE(a.window >= 0, "%s: window must be >= 0", name);
-    REQUIRE(a.dt == CSA_DT_F32 || a.dt == CSA_DT_BF16 || a.dt == CSA_DT_E4M3, "%s: unknown dtype", name);
-    if (a.dt == CSA_DT_E4M3) return fail(CSA_ERR_UNSUPPORTED, "%s: dt must be F32 or BF16", name);
+    REQUIRE(is_dt(a.dt), "%s: unknown dtype", name);
+    if (is_fp8(a.dt)) return fail(CSA_ERR_UNSUPPORTED, "%s: dt must be F32 or BF16", name);
     if (a.D % 16 || a.D > 256) return fail(CSA_ERR_UNSUPPORTED, "%s: D must be a multiple of 16 <= 256", name);
     if ((long)a.B * a.n_q == 0) return ok();
     REQUIRE(a.q && a.out, "%s: null q or out", name);

@@ -28,8 +28,9 @@
 //     resolve to the lowest indices across the whole row, and the output is
 //     identical from call to call).
 // The query row is quantised per head in fp32 exactly as the oracle does
-// (scale = amax / 448, codes rounded to nearest even, saturating) unless
-// codes and scales are given.
+// (scale = amax / 448, codes rounded to nearest even, saturating), after a
+// fixed-order Walsh-Hadamard rotation when the keys are of the rotated fp8
+// type, unless codes and scales are given.
 #include <cooperative_groups.h>
 
 #include <algorithm>
@@ -140,12 +141,43 @@ __global__ void __launch_bounds__(kThreads, min_blocks<NU>()) indexer_split_kern
         const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(a.qI) + (size_t)row * H * d;
         const int h = warp;   // kWarps == kMaxHeads
         if (h < H) {
+            constexpr int J = d / 32;          // this lane holds elements lane + 32 j
+            float v[J];
+#pragma unroll
+            for (int j = 0; j < J; ++j) v[j] = __bfloat162float(src[h * d + lane + 32 * j]);
+            if (a.kI_dt == DT_E4M3H) {
+                // Walsh-Hadamard butterflies in stride order: strides 1..16
+                // pair lane with lane ^ s (the lower lane holds the left
+                // operand), strides 32, 64 pair this lane's own elements.
+#pragma unroll
+                for (int sl = 1; sl < 32; sl <<= 1) {
+                    const bool hi = (lane & sl) != 0;
+#pragma unroll
+                    for (int j = 0; j < J; ++j) {
+                        const float pv = __shfl_xor_sync(0xffffffffu, v[j], sl);
+                        v[j] = hi ? pv - v[j] : v[j] + pv;
+                    }
+                }
+#pragma unroll
+                for (int sj = 1; sj < J; sj <<= 1) {
+#pragma unroll
+                    for (int j = 0; j < J; ++j) {
+                        if (j & sj) continue;
+                        const float x0 = v[j], x1 = v[j + sj];
+                        v[j] = x0 + x1;
+                        v[j + sj] = x0 - x1;
+                    }
+                }
+#pragma unroll
+                for (int j = 0; j < J; ++j) v[j] = v[j] * a.hnorm;
+            }
             float amax = 0.0f;
-            for (int c = lane; c < d; c += 32) amax = fmaxf(amax, fabsf(__bfloat162float(src[h * d + c])));
+#pragma unroll
+            for (int j = 0; j < J; ++j) amax = fmaxf(amax, fabsf(v[j]));
             for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
             const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-            for (int c = lane; c < d; c += 32)
-                sh.qc[h * d + c] = e4m3_code(__fdiv_rn(__bfloat162float(src[h * d + c]), scale));
+#pragma unroll
+            for (int j = 0; j < J; ++j) sh.qc[h * d + lane + 32 * j] = e4m3_code(__fdiv_rn(v[j], scale));
             if (lane == 0) sh.qs[h] = scale;
         } else {
             for (int c = lane; c < d; c += 32) sh.qc[h * d + c] = 0;
@@ -400,7 +432,7 @@ cudaError_t launch_t(const IndexerArgs& a, cudaStream_t s) {
 }  // namespace
 
 bool indexer_split_supported(const IndexerArgs& a) {
-    if (a.kI_dt != DT_E4M3 || a.kI_scale == nullptr) return false;
+    if ((a.kI_dt != DT_E4M3 && a.kI_dt != DT_E4M3H) || a.kI_scale == nullptr) return false;
     if (!(a.qI_dt == DT_BF16 || (a.qI_dt == DT_E4M3 && a.qI_scale != nullptr))) return false;
     if ((a.d_I != 64 && a.d_I != 128) || a.H_I < 1 || a.H_I > kMaxHeads) return false;
     if ((long)a.B * a.n_q > 65535) return false;

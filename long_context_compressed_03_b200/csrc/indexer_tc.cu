@@ -64,7 +64,9 @@ struct IdxParams {
     const void* qI;            // [B, n, H_I, 64] bf16 or e4m3 codes
     const float* qI_scale;     // e4m3 queries given as codes: [B, n, H_I]
     const float* kI_scale;     // e4m3 keys: [B, N_cap]
-    int q_mode;                // 0 bf16 (bf16 keys), 1 bf16 quantised here, 2 e4m3 codes
+    int q_mode;                // 0 bf16 (bf16 keys), 1 bf16 quantised here, 2 e4m3 codes,
+                               // 3 bf16 Hadamard-rotated, then quantised here
+    float hnorm;               // q_mode 3: fp32(1/sqrt(64))
     int B, n, H_I, N_cap, m, topk;
     const int* n_entries;
     int* idx_out;
@@ -294,7 +296,25 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
                 const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(p.qI) + qrow * kDim;
                 v0 = __bfloat162float(src[2 * lane]);
                 v1 = __bfloat162float(src[2 * lane + 1]);
-                if (p.q_mode == 1) {
+                if (p.q_mode == 3) {
+                    // Walsh-Hadamard butterflies in stride order 1, 2, ..., 32:
+                    // stride 1 pairs this lane's two elements, stride 2s pairs
+                    // lane with lane ^ s (the lower lane holds the left operand).
+                    const float a0 = v0;
+                    v0 = a0 + v1;
+                    v1 = a0 - v1;
+#pragma unroll
+                    for (int sl = 1; sl < 32; sl <<= 1) {
+                        const float p0 = __shfl_xor_sync(0xffffffffu, v0, sl);
+                        const float p1 = __shfl_xor_sync(0xffffffffu, v1, sl);
+                        const bool hi = (lane & sl) != 0;
+                        v0 = hi ? p0 - v0 : v0 + p0;
+                        v1 = hi ? p1 - v1 : v1 + p1;
+                    }
+                    v0 = v0 * p.hnorm;
+                    v1 = v1 * p.hnorm;
+                }
+                if (p.q_mode == 1 || p.q_mode == 3) {
                     float amax = fmaxf(fabsf(v0), fabsf(v1));
                     for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
                     qs = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
@@ -573,14 +593,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }  // namespace
 
 bool indexer_tc_supported(const IndexerArgs& a) {
-    const bool fp8 = a.kI_dt == DT_E4M3 && (a.qI_dt == DT_BF16 || a.qI_dt == DT_E4M3);
+    const bool fp8 = (a.kI_dt == DT_E4M3 || a.kI_dt == DT_E4M3H) &&
+                     (a.qI_dt == DT_BF16 || a.qI_dt == DT_E4M3);
     const bool bf16 = a.kI_dt == DT_BF16 && a.qI_dt == DT_BF16;
     return (fp8 || bf16) && a.d_I == kDim && a.H_I <= kHeads && a.q_pos == nullptr &&
            a.N_cap <= 65536 && a.n_q >= 1;
 }
 
 cudaError_t launch_indexer_tc(const IndexerArgs& a, uint32_t* err, cudaStream_t s) {
-    const bool fp8 = a.kI_dt == DT_E4M3;
+    const bool fp8 = a.kI_dt == DT_E4M3 || a.kI_dt == DT_E4M3H;
     auto fn = encode_fn();
     if (!fn) return cudaErrorInvalidValue;
     CUtensorMap tm;
@@ -598,7 +619,8 @@ cudaError_t launch_indexer_tc(const IndexerArgs& a, uint32_t* err, cudaStream_t 
     p.qI = a.qI;
     p.qI_scale = a.qI_scale;
     p.kI_scale = a.kI_scale;
-    p.q_mode = fp8 ? (a.qI_dt == DT_E4M3 ? 2 : 1) : 0;
+    p.q_mode = fp8 ? (a.qI_dt == DT_E4M3 ? 2 : (a.kI_dt == DT_E4M3H ? 3 : 1)) : 0;
+    p.hnorm = a.hnorm;
     p.B = a.B;
     p.n = a.n_q;
     p.H_I = a.H_I;

@@ -245,6 +245,12 @@ cudaError_t launch_indexer_topk(const IndexerArgs& a, cudaStream_t s, const char
     if (a.qI_dt == DT_BF16 && a.kI_dt == DT_BF16) return launch_t<DT_BF16, DT_BF16>(a, s);
     if (a.qI_dt == DT_BF16 && a.kI_dt == DT_E4M3) return launch_t<DT_BF16, DT_E4M3>(a, s);
     if (a.qI_dt == DT_E4M3 && a.kI_dt == DT_E4M3) return launch_t<DT_E4M3, DT_E4M3>(a, s);
+    // rotated keys against query codes that the caller rotated: plain fp8 scoring
+    if (a.qI_dt == DT_E4M3 && a.kI_dt == DT_E4M3H) return launch_t<DT_E4M3, DT_E4M3>(a, s);
+    if (a.kI_dt == DT_E4M3H) {
+        *why = "csa_indexer_topk: Hadamard keys with bf16 queries need d_I 64 (or 128 with few rows)";
+        return cudaErrorNotSupported;
+    }
     *why = "csa_indexer_topk: unsupported (qI_dt, kI_dt) pair";
     return cudaErrorNotSupported;
 }

@@ -13,6 +13,7 @@ struct CompressArgs {
     void* out; int out_dt;
     float* out_row_scale;
     int N_c;
+    float hnorm;               // fp32(1/sqrt(d_out)) for the Hadamard fp8 type
 };
 
 struct AppendArgs {
@@ -26,6 +27,7 @@ struct AppendArgs {
     float* cache_scale;
     int N_cap;
     int* n_entries;
+    float hnorm;               // fp32(1/sqrt(d_out)) for the Hadamard fp8 type
 };
 
 struct IndexerArgs {
@@ -35,6 +37,7 @@ struct IndexerArgs {
     const int* n_entries; const int* q_pos;
     int m, topk;
     int* idx_out;
+    float hnorm;               // fp32(1/sqrt(d_I)): keys of the Hadamard fp8 type
 };
 
 struct AttnArgs {

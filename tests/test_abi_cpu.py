@@ -121,6 +121,41 @@ def test_indexer_validation(lib):
     assert f(*ok) == api.CSA_OK
 
 
+def test_hadamard_type_validation(lib):
+    # the rotated fp8 type: d_out / d_I must be powers of two, scales are
+    # required, queries are never given as that type, attention rejects it
+    H = api.DT_E4M3_HADAMARD
+    f = lib.csa_compress
+    #       x   dt B  n   d_in W    d_out m  ov out  dt scale stream
+    args = [FAKE, 1, 1, 64, 64, FAKE, 64, 4, 1, FAKE, H, FAKE, None]
+    bad = list(args); bad[6] = 48                      # d_out not a power of two
+    assert f(*bad) == api.CSA_ERR_UNSUPPORTED
+    assert "power of two" in _detail(lib)
+    bad = list(args); bad[11] = None                   # no scales
+    assert f(*bad) == api.CSA_ERR_INVALID_ARG
+    ok = list(args); ok[2] = 0                         # B = 0: no-op
+    assert f(*ok) == api.CSA_OK
+    g = lib.csa_compress_append
+    args = [FAKE, 1, 2, 64, FAKE, 96, 4, 1, FAKE, FAKE, FAKE, H, FAKE, 16, None, None]
+    assert g(*args) == api.CSA_ERR_UNSUPPORTED        # d_out = 96
+    ok = list(args); ok[5] = 128; ok[2] = 0
+    assert g(*ok) == api.CSA_OK
+    h = lib.csa_indexer_topk
+    args = [FAKE, 1, None, FAKE, H, FAKE, 1, 8, 4, 64, 16, None, None, 4, 8, FAKE, None]
+    bad = list(args); bad[9] = 48                      # d_I not a power of two
+    assert h(*bad) == api.CSA_ERR_UNSUPPORTED
+    bad = list(args); bad[5] = None                    # rotated keys without scales
+    assert h(*bad) == api.CSA_ERR_INVALID_ARG
+    bad = list(args); bad[1] = H; bad[2] = FAKE        # queries as the rotated type
+    assert h(*bad) == api.CSA_ERR_UNSUPPORTED
+    ok = list(args); ok[7] = 0
+    assert h(*ok) == api.CSA_OK
+    a = lib.csa_sparse_attn
+    args = [FAKE, H, 1, 8, 64, 128, FAKE, 16, FAKE, 4, FAKE, 8, None, None, 4, None,
+            ctypes.c_float(0.0), FAKE, None, None]
+    assert a(*args) == api.CSA_ERR_UNSUPPORTED
+
+
 def test_attention_validation(lib):
     f = lib.csa_sparse_attn
     args = [FAKE, 1, 1, 8, 64, 128, FAKE, 16, FAKE, 4, FAKE, 8, None, None, 4, None,

@@ -37,12 +37,23 @@ def _fp8_rows(x: torch.Tensor):
     return codes, sc
 
 
+def _sylvester(d):
+    """Normalised Sylvester-Hadamard matrix (fp64), independent of the kernels."""
+    h = np.ones((1, 1))
+    while h.shape[0] < d:
+        h = np.block([[h, h], [h, -h]])
+    return h / math.sqrt(d)
+
+
 def _decode_indexer(seed, B, n_q, N_cap, H_I, d_I, k, ctx, q_kind="bf16", m=4, tie_rows=False):
     g = _gen(seed)
     qI = torch.randn(B, n_q, H_I, d_I, generator=g).to(torch.bfloat16)
     kI = torch.randn(B, N_cap, d_I, generator=g)
     if tie_rows:
         kI[:] = kI[:, :1]                        # every entry identical: all scores tie
+    rot = q_kind == "bf16_rot"
+    if rot:                                      # keys stored Hadamard-rotated
+        kI = torch.from_numpy(kI.double().numpy() @ _sylvester(d_I)).float()
     codes, sc = _fp8_rows(kI)
     ne = np.minimum(np.asarray(ctx) // m, N_cap).astype(np.int32)
     q_pos = np.stack([np.asarray(ctx) - 1 - j for j in range(n_q)], axis=1).astype(np.int32)
@@ -52,8 +63,8 @@ def _decode_indexer(seed, B, n_q, N_cap, H_I, d_I, k, ctx, q_kind="bf16", m=4, t
         idx = api.indexer_topk(T(qc), T(codes), m, k, qI_scale=T(qs), **kw)
         q_rows = oracle.dequantize_rows_e4m3(qc.numpy(), qs.numpy())
     else:
-        idx = api.indexer_topk(T(qI), T(codes), m, k, **kw)
-        q_rows = oracle.quantized_query_rows(qI.float().numpy())
+        idx = api.indexer_topk(T(qI), T(codes), m, k, kI_rotated=rot, **kw)
+        q_rows = oracle.quantized_query_rows(qI.float().numpy(), rotate=rot)
     q_rows = q_rows.reshape(B * n_q, H_I, d_I)
     rb = np.repeat(np.arange(B, dtype=np.int32), n_q)
     scores = oracle.indexer_scores_rows(q_rows, rb, q_pos.reshape(-1), codes.numpy(), m, ne, sc.numpy())
@@ -66,6 +77,8 @@ def _decode_indexer(seed, B, n_q, N_cap, H_I, d_I, k, ctx, q_kind="bf16", m=4, t
     (2, 2, 50000, 8, 128, 512, "e4m3"),     # 16-CTA clusters, more entries than one CTA holds
     (64, 4, 2100, 4, 64, 100, "bf16"),      # many rows: small clusters
     (3, 1, 9000, 1, 64, 2048, "bf16"),      # one head, the largest k
+    (4, 1, 6000, 4, 64, 256, "bf16_rot"),   # Hadamard-rotated keys, query rotated in the kernel
+    (2, 2, 30000, 8, 128, 512, "bf16_rot"), # d_I = 128: butterflies across a lane's own elements
 ])
 def test_decode_indexer_matches_oracle(case):
     B, n_q, N_cap, H_I, d_I, k, qk = case

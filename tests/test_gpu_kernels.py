@@ -67,6 +67,42 @@ def test_compress_matches_oracle(case):
         assert max_abs(got, ref) <= ATOL_BF16
 
 
+def _hadamard64(d):
+    """Normalised Sylvester-Hadamard matrix in fp64 (symmetric, orthonormal),
+    built independently of the kernels' butterfly order."""
+    h = np.ones((1, 1))
+    while h.shape[0] < d:
+        h = np.block([[h, h], [h, -h]])
+    return h / math.sqrt(d)
+
+
+@pytest.mark.parametrize("case", [
+    # (B, n, d_in, d_out, m, overlap, x dtype)
+    (2, 1003, 64, 64, 4, True, torch.bfloat16),     # fp8 indexer keys, ragged tail
+    (1, 700, 128, 128, 4, True, torch.float32),
+    (1, 300, 256, 256, 4, True, torch.bfloat16),
+    (1, 200, 32, 16, 1, False, torch.bfloat16),
+])
+def test_compress_hadamard_fp8_matches_rotated_oracle(case):
+    """Rows rotated by the normalised Walsh-Hadamard matrix before the fp8
+    cast: the codes dequantise to H @ (oracle row) within one E4M3 step."""
+    B, n, d_in, d_out, m, overlap, dt = case
+    g = _gen(500 + n)
+    x = _randn(g, B, n, d_in, dtype=dt)
+    W = _randn(g, d_in, d_out, dtype=dt, std=1.0 / math.sqrt(d_in))
+    ref = oracle.compress(np64(x), np64(W), m, overlap) @ _hadamard64(d_out)
+    codes, scale = api.compress(x.to(DEV), W.to(DEV), m, overlap, out_dtype=torch.uint8,
+                                hadamard=True)
+    codes, scale = codes.cpu().numpy(), scale.cpu().numpy()
+    deq = oracle.dequantize_rows_e4m3(codes, scale)
+    np.testing.assert_allclose(scale, np.abs(ref).max(axis=-1) / 448.0, rtol=1e-5)
+    assert np.all(np.abs(deq - ref) <= np.abs(ref) * 2.0 ** -3 + scale[..., None] * 2.0 ** -9)
+    # rotating back recovers the row to within the fp8 error spread by H
+    back = deq @ _hadamard64(d_out)
+    unrot = oracle.compress(np64(x), np64(W), m, overlap)
+    assert max_abs(back, unrot) <= 0.1 * np.abs(unrot).max()
+
+
 def test_compress_no_entries_is_a_noop():
     x = torch.zeros(1, 3, 16, device=DEV, dtype=torch.bfloat16)
     W = torch.zeros(16, 16, device=DEV, dtype=torch.bfloat16)
@@ -103,7 +139,16 @@ def _index_case(seed, B, n, H_I, d_I, kind, k, n_entries=None, q_pos=None, ties=
         codes = (kI.float() / sc[..., None]).to(torch.float8_e4m3fn).view(torch.uint8)
         dev["kI"], dev["kI_scale"] = codes.to(DEV), sc.to(DEV)
         orc["kI"], orc["kI_scale"] = codes.numpy(), sc.numpy()
-        if kind == "e4m3_given":
+        if kind == "e4m3_rot":
+            # keys rotated in fp64 by an independent Sylvester matrix, cast by torch
+            kr = torch.from_numpy(np64(kI) @ _hadamard64(d_I)).float()
+            amax = kr.abs().amax(-1)
+            sc = torch.where(amax > 0, amax / 448.0, torch.ones_like(amax))
+            codes = (kr / sc[..., None]).to(torch.float8_e4m3fn).view(torch.uint8)
+            dev["kI"], dev["kI_scale"] = codes.to(DEV), sc.to(DEV)
+            orc["kI"], orc["kI_scale"] = codes.numpy(), sc.numpy()
+            orc["q_rows"] = oracle.quantized_query_rows(qrows.astype(np.float32), rotate=True)
+        elif kind == "e4m3_given":
             qa = qI.float().abs().amax(-1)
             qs = torch.where(qa > 0, qa / 448.0, torch.ones_like(qa))
             qc = (qI.float() / qs[..., None]).to(torch.float8_e4m3fn).view(torch.uint8)
@@ -131,6 +176,8 @@ INDEXER_CASES = [
     (1, 1200, 4, 64, "e4m3_given", 100),
     (1, 4100, 2, 64, "e4m3", 300),        # two indexer heads, several CTAs
     (1, 333, 16, 32, "bf16", 7),          # 16 heads: generic kernel
+    (2, 901, 4, 64, "e4m3_rot", 64),      # Hadamard-rotated keys, queries rotated in the kernel
+    (1, 4100, 2, 64, "e4m3_rot", 300),
 ]
 
 
@@ -139,7 +186,7 @@ def test_indexer_topk_matches_oracle(case):
     B, n, H_I, d_I, kind, k = case
     dev, orc, ne, rb, rt, m = _index_case(7 + n, B, n, H_I, d_I, kind, k)
     idx = api.indexer_topk(dev["qI"], dev["kI"], m, k, qI_scale=dev.get("qI_scale"),
-                           kI_scale=dev.get("kI_scale"))
+                           kI_scale=dev.get("kI_scale"), kI_rotated=kind == "e4m3_rot")
     got = idx.cpu().numpy().reshape(B * n, k)
     scores = oracle.indexer_scores_rows(orc["q_rows"], rb, rt, orc["kI"], m, ne, orc["kI_scale"])
     stats = check_topk(got, scores, k)
@@ -293,6 +340,7 @@ def test_binding_rejects_host_tensors():
     # (B, n, d_in, d_out, m, overlap, x dtype, cache kind, N_cap)
     (3, 37, 128, 128, 4, True, torch.bfloat16, "bf16", 16),     # CSA main compressor, ragged
     (2, 41, 64, 64, 4, True, torch.bfloat16, "e4m3", 12),       # fp8 indexer-key cache
+    (2, 57, 64, 64, 4, True, torch.bfloat16, "e4m3_rot", 16),   # Hadamard-rotated fp8 keys
     (2, 300, 128, 128, 128, False, torch.bfloat16, "bf16", 3),  # HCA ratio
     (1, 24, 32, 48, 4, False, torch.float32, "f32", 4),         # cache shorter than the stream
 ])
@@ -306,7 +354,7 @@ def test_compress_append_stream_matches_oracle(case):
     start = np.arange(B) * 3                     # element b starts its sequence at step 3b
     steps = n + int(start.max())
     state = torch.zeros(B, 2, d_in, dtype=torch.float32, device=DEV)
-    if kind == "e4m3":
+    if kind in ("e4m3", "e4m3_rot"):
         cache = torch.zeros(B, N_cap, d_out, dtype=torch.uint8, device=DEV)
         scale = torch.zeros(B, N_cap, dtype=torch.float32, device=DEV)
     else:
@@ -321,12 +369,14 @@ def test_compress_append_stream_matches_oracle(case):
         pos = torch.from_numpy(np.where((p >= 0) & (p < n), p, -1).astype(np.int32)).to(DEV)
         tok = xd[rows, torch.from_numpy(np.clip(p, 0, n - 1)).to(DEV)].contiguous()
         api.csa_compress_append(tok, Wd, m, overlap, pos, state, cache, cache_scale=scale,
-                                n_entries=n_ent)
+                                n_entries=n_ent, hadamard=kind == "e4m3_rot")
     torch.cuda.synchronize()
     ref = oracle.compress(np64(x), np64(W), m, overlap)
+    if kind == "e4m3_rot":
+        ref = ref @ _hadamard64(d_out)
     N_w = min(N_cap, ref.shape[1])
     assert np.array_equal(n_ent.cpu().numpy(), np.full(B, min(n // m, N_cap), np.int32))
-    if kind == "e4m3":
+    if kind in ("e4m3", "e4m3_rot"):
         deq = oracle.dequantize_rows_e4m3(cache.cpu().numpy()[:, :N_w], scale.cpu().numpy()[:, :N_w])
         r = ref[:, :N_w]
         sc = scale.cpu().numpy()[:, :N_w]
