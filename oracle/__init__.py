@@ -69,8 +69,8 @@ def _load():
         lib.oracle_compress.argtypes = [P, i32, i32, i32, P, i32, i32, i32, P]
         lib.oracle_compress_append.argtypes = [P, P, i32, i32, P, i32, i32, i32, P, P, i32, P]
         dbl = ctypes.c_double
-        lib.oracle_indexer_scores.argtypes = [P, P, P, i64, i32, i32, P, P, P, i32, P, i32, P]
-        lib.oracle_indexer_topk.argtypes = [P, P, P, i64, i32, i32, P, P, P, i32, P, i32, i32, P,
+        lib.oracle_indexer_scores.argtypes = [P, P, P, P, i64, i32, i32, P, P, P, i32, P, i32, P]
+        lib.oracle_indexer_topk.argtypes = [P, P, P, P, i64, i32, i32, P, P, P, i32, P, i32, i32, P,
                                             P, P]
         lib.oracle_sparse_attn.argtypes = [P, P, P, i64, i32, i32, P, i32, P, i32, P, i32, P, P,
                                            i32, dbl, P, P]
@@ -244,37 +244,49 @@ def quantized_query_rows(qI_rows, rotate: bool = False) -> np.ndarray:
     return dequantize_rows_e4m3(codes, scales)
 
 
-def indexer_scores_rows(qI_rows, row_b, row_t, kI, m: int, n_entries, kI_scale=None):
-    """Scores sum_h ReLU(qI . kI[s]) of listed query rows against every entry.
-    qI_rows [R, H_I, d_I] fp64 (dequantised); row_b/row_t [R] batch element
-    and absolute position; kI [B, N_cap, d_I] fp64 values, or E4M3 codes
-    with kI_scale [B, N_cap]; n_entries [B].  Returns [R, N_cap], NaN where
-    the entry is not visible."""
+def _weights_arg(weights, R, H_I):
+    if weights is None:
+        return None, None
+    w = np.ascontiguousarray(np.asarray(weights, dtype=np.float64).reshape(R, H_I))
+    return w, _ptr(w)
+
+
+def indexer_scores_rows(qI_rows, row_b, row_t, kI, m: int, n_entries, kI_scale=None,
+                        weights=None):
+    """Scores sum_h w_h ReLU(qI_h . kI[s]) of listed query rows against every
+    entry.  qI_rows [R, H_I, d_I] fp64 (dequantised); weights [R, H_I] per-head
+    gate weights (None: all 1); row_b/row_t [R] batch element and absolute
+    position; kI [B, N_cap, d_I] fp64 values, or E4M3 codes with kI_scale
+    [B, N_cap]; n_entries [B].  Returns [R, N_cap], NaN where the entry is not
+    visible."""
     q = _f64(qI_rows)
     R, H_I, d_I = q.shape
+    w, wp = _weights_arg(weights, R, H_I)
     keep = _keys_arg(kI, kI_scale)
     N_cap = np.asarray(kI).shape[1]
     rb, rt, ne = _i32(row_b), _i32(row_t), _i32(n_entries)
     out = np.empty((R, N_cap), dtype=np.float64)
-    _load().oracle_indexer_scores(_ptr(q), _ptr(rb), _ptr(rt), R, H_I, d_I, *keep[3], N_cap,
+    _load().oracle_indexer_scores(_ptr(q), wp, _ptr(rb), _ptr(rt), R, H_I, d_I, *keep[3], N_cap,
                                   _ptr(ne), m, _ptr(out))
     return out
 
 
-def indexer_topk_rows(qI_rows, row_b, row_t, kI, m: int, topk: int, n_entries, kI_scale=None):
+def indexer_topk_rows(qI_rows, row_b, row_t, kI, m: int, topk: int, n_entries, kI_scale=None,
+                      weights=None):
     """Per listed query row: the topk largest visible scores (ties -> lower
     index, -1 padding).  Returns (idx [R, topk] int32 in (score desc, index
     asc) order, kth [R, 2] = k-th and (k+1)-th largest scores (NaN if
     absent), smax [R] = largest |score|)."""
     q = _f64(qI_rows)
     R, H_I, d_I = q.shape
+    w, wp = _weights_arg(weights, R, H_I)
     keep = _keys_arg(kI, kI_scale)
     N_cap = np.asarray(kI).shape[1]
     rb, rt, ne = _i32(row_b), _i32(row_t), _i32(n_entries)
     idx = np.empty((R, topk), dtype=np.int32)
     kth = np.empty((R, 2), dtype=np.float64)
     smax = np.empty(R, dtype=np.float64)
-    _load().oracle_indexer_topk(_ptr(q), _ptr(rb), _ptr(rt), R, H_I, d_I, *keep[3], N_cap,
+    _load().oracle_indexer_topk(_ptr(q), wp, _ptr(rb), _ptr(rt), R, H_I, d_I, *keep[3], N_cap,
                                 _ptr(ne), m, topk, _ptr(idx), _ptr(kth), _ptr(smax))
     return idx, kth, smax
 
@@ -285,27 +297,31 @@ def _full_rows(B, n_q, q_pos, rows):
     return r, (r // n_q).astype(np.int32), qp[r].astype(np.int32)
 
 
-def indexer_scores(qI, kI, m: int, n_entries=None, q_pos=None, rows=None, kI_scale=None):
-    """indexer_scores_rows over full tensors qI [B, n_q, H_I, d_I]; rows are
-    flattened b*n_q+q (all by default)."""
+def indexer_scores(qI, kI, m: int, n_entries=None, q_pos=None, rows=None, kI_scale=None,
+                   weights=None):
+    """indexer_scores_rows over full tensors qI [B, n_q, H_I, d_I] (weights
+    [B, n_q, H_I] or None); rows are flattened b*n_q+q (all by default)."""
     qI = _f64(qI)
     B, n_q, H_I, d_I = qI.shape
     N_cap = np.asarray(kI).shape[1]
     n_entries, q_pos = _defaults(B, n_q, N_cap, n_entries, q_pos)
     r, rb, rt = _full_rows(B, n_q, q_pos, rows)
+    w = None if weights is None else _f64(weights).reshape(B * n_q, H_I)[r]
     return indexer_scores_rows(qI.reshape(B * n_q, H_I, d_I)[r], rb, rt, kI, m, n_entries,
-                               kI_scale)
+                               kI_scale, w)
 
 
-def indexer_topk(qI, kI, m: int, topk: int, n_entries=None, q_pos=None, rows=None, kI_scale=None):
+def indexer_topk(qI, kI, m: int, topk: int, n_entries=None, q_pos=None, rows=None, kI_scale=None,
+                 weights=None):
     """indexer_topk_rows over full tensors (see indexer_scores)."""
     qI = _f64(qI)
     B, n_q, H_I, d_I = qI.shape
     N_cap = np.asarray(kI).shape[1]
     n_entries, q_pos = _defaults(B, n_q, N_cap, n_entries, q_pos)
     r, rb, rt = _full_rows(B, n_q, q_pos, rows)
+    w = None if weights is None else _f64(weights).reshape(B * n_q, H_I)[r]
     return indexer_topk_rows(qI.reshape(B * n_q, H_I, d_I)[r], rb, rt, kI, m, topk, n_entries,
-                             kI_scale)
+                             kI_scale, w)
 
 
 # --------------------------------------------------------------------------

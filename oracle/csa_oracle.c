@@ -116,9 +116,9 @@ void oracle_quantize_rows_e4m3(const float* x, long rows, int d, uint8_t* codes,
 }
 
 /* ------------------------------------------------------------------------
- * Hadamard rotation of indexer rows before fp8 (the survey's NEXT-2 reading
- * of the DSA-lineage indexer that "DS-V4 分析&学习" §1.2 and the gitcode
- * analysis name: a rotation spreads outlier channels before E4M3, and dot
+ * Hadamard rotation of indexer rows before fp8 (a reading of the DSA-lineage
+ * indexer that "DS-V4 分析&学习" §1.2 and the gitcode analysis name, which
+ * print no formula for it: a rotation spreads outlier channels before E4M3, and dot
  * products are unchanged because the normalised Walsh-Hadamard matrix H_d is
  * orthonormal and symmetric).  In place, in fp32, in a fixed order that the
  * kernels reproduce exactly: for stride s = 1, 2, 4, ..., d/2 every pair
@@ -246,13 +246,16 @@ long oracle_visible_entries(long t, int m, long n_entries) {
 
 /* ------------------------------------------------------------------------
  * Stage 2: Lightning-Indexer score ([P5] §3.2 stage two; [P3] §1.2, §4).
- * score[t, s] = sum_h ReLU( qI[t, h, :] . kI[s, :] ),  s < V(t).
+ * score[t, s] = sum_h w[t, h] * ReLU( qI[t, h, :] . kI[s, :] ),  s < V(t).
  * One shared indexer key row per entry (MQA-like); each indexer head passes
- * its dot product through a ReLU before the heads are summed.
+ * its dot product through a ReLU before the heads are summed.  The per-query,
+ * per-head gate weights w (any sign) are the gated form of the DSA-lineage
+ * indexer the pages name ([P3] §1.2; [P1] head) without printing it; w_rows
+ * NULL means w = 1 (the plain sum).
  *
  * Query rows are given as a list: row rr has batch element row_b[rr],
  * absolute position row_t[rr] and query values qI_rows[rr, H_I, d_I] (fp64,
- * already dequantised).  Keys kI [B, N_cap, d_I] are given either as fp64
+ * already dequantised), optional weights w_rows[rr, H_I].  Keys kI [B, N_cap, d_I] are given either as fp64
  * values (kI_f64) or as E4M3 codes with one fp32 scale per entry (kI_codes +
  * kI_scale), dequantised here in fp64.
  * scores receives n_rows x N_cap values, NaN where the entry is not visible.
@@ -268,17 +271,19 @@ static void key_row(const double* kI_f64, const uint8_t* kI_codes, const float* 
     }
 }
 
-static double score_one(const double* qrow, int H_I, int d_I, const double* krow) {
+static double score_one(const double* qrow, const double* wrow, int H_I, int d_I,
+                        const double* krow) {
     double s = 0.0;
     for (int h = 0; h < H_I; ++h) {
         double dot = 0.0;
         for (int c = 0; c < d_I; ++c) dot += qrow[(long)h * d_I + c] * krow[c];
-        if (dot > 0.0) s += dot;
+        if (dot > 0.0) s += (wrow ? wrow[h] : 1.0) * dot;
     }
     return s;
 }
 
-void oracle_indexer_scores(const double* qI_rows, const int* row_b, const int* row_t, long n_rows,
+void oracle_indexer_scores(const double* qI_rows, const double* w_rows, const int* row_b,
+                           const int* row_t, long n_rows,
                            int H_I, int d_I, const double* kI_f64, const uint8_t* kI_codes,
                            const float* kI_scale, int N_cap, const int* n_entries, int m,
                            double* scores) {
@@ -286,13 +291,14 @@ void oracle_indexer_scores(const double* qI_rows, const int* row_b, const int* r
     for (long rr = 0; rr < n_rows; ++rr) {
         int b = row_b[rr];
         const double* qrow = qI_rows + rr * (long)H_I * d_I;
+        const double* wrow = w_rows ? w_rows + rr * (long)H_I : NULL;
         long V = oracle_visible_entries(row_t[rr], m, n_entries[b]);
         double* out = scores + rr * (long)N_cap;
         double* krow = (double*)malloc(sizeof(double) * (size_t)d_I);
         for (long s = 0; s < N_cap; ++s) {
             if (s < V) {
                 key_row(kI_f64, kI_codes, kI_scale, b, s, N_cap, d_I, krow);
-                out[s] = score_one(qrow, H_I, d_I, krow);
+                out[s] = score_one(qrow, wrow, H_I, d_I, krow);
             } else {
                 out[s] = NAN;
             }
@@ -319,7 +325,8 @@ static int cmp_scored(const void* a, const void* b) {
     return (x->i < y->i) ? -1 : (x->i > y->i);
 }
 
-void oracle_indexer_topk(const double* qI_rows, const int* row_b, const int* row_t, long n_rows,
+void oracle_indexer_topk(const double* qI_rows, const double* w_rows, const int* row_b,
+                         const int* row_t, long n_rows,
                          int H_I, int d_I, const double* kI_f64, const uint8_t* kI_codes,
                          const float* kI_scale, int N_cap, const int* n_entries, int m, int topk,
                          int* idx_out, double* kth, double* smax) {
@@ -327,13 +334,14 @@ void oracle_indexer_topk(const double* qI_rows, const int* row_b, const int* row
     for (long rr = 0; rr < n_rows; ++rr) {
         int b = row_b[rr];
         const double* qrow = qI_rows + rr * (long)H_I * d_I;
+        const double* wrow = w_rows ? w_rows + rr * (long)H_I : NULL;
         long V = oracle_visible_entries(row_t[rr], m, n_entries[b]);
         scored_t* all = (scored_t*)malloc(sizeof(scored_t) * (size_t)(V > 0 ? V : 1));
         double* krow = (double*)malloc(sizeof(double) * (size_t)d_I);
         double amax = 0.0;
         for (long s = 0; s < V; ++s) {
             key_row(kI_f64, kI_codes, kI_scale, b, s, N_cap, d_I, krow);
-            all[s].s = score_one(qrow, H_I, d_I, krow);
+            all[s].s = score_one(qrow, wrow, H_I, d_I, krow);
             all[s].i = s;
             if (fabs(all[s].s) > amax) amax = fabs(all[s].s);
         }

@@ -283,6 +283,80 @@ def test_kth_scores_match_numpy_sort():
             assert smax[t] == np.abs(row).max()
 
 
+# ---------------------------------------------------------------- gated indexer
+def test_gated_scores_hand_worked_example():
+    # two heads, d = 2, weights (2, -3); worked by hand:
+    #   key (1,0):  dots ( 1, -1) -> 2*1 + -3*0 =  2
+    #   key (0,1):  dots ( 2,  1) -> 2*2 + -3*1 =  1
+    #   key (1,1):  dots ( 3,  0) -> 2*3 + -3*0 =  6
+    #   key (-1,-1): dots (-3, 0) -> 0
+    #   key (-1,0): dots (-1,  1) -> 0 + -3*1  = -3
+    q = np.array([[[[1.0, 2.0], [-1.0, 1.0]]]])                     # [1, 1, 2, 2]
+    k = np.array([[[1, 0], [0, 1], [1, 1], [-1, -1], [-1, 0]]], dtype=np.float64)
+    w = np.array([[[2.0, -3.0]]])
+    pos = np.array([[19]], np.int32)                                 # all 5 entries visible
+    s = oracle.indexer_scores(q, k, 4, q_pos=pos, weights=w)
+    assert s[0].tolist() == [2.0, 1.0, 6.0, 0.0, -3.0]
+    idx, kth, smax = oracle.indexer_topk(q, k, 4, 5, q_pos=pos, weights=w)
+    assert idx[0].tolist() == [2, 0, 1, 3, 4]                        # negatives rank below zero
+    idx3, kth3, _ = oracle.indexer_topk(q, k, 4, 3, q_pos=pos, weights=w)
+    assert idx3[0].tolist() == [2, 0, 1] and kth3[0].tolist() == [1.0, 0.0]
+    assert smax[0] == 6.0
+
+
+def test_unit_weights_and_one_hot_weights_reduce_to_known_scores():
+    rng = np.random.default_rng(21)
+    qI = rng.standard_normal((2, 30, 4, 8))
+    kI = rng.standard_normal((2, 9, 8))
+    plain = oracle.indexer_scores(qI, kI, 4)
+    ones = oracle.indexer_scores(qI, kI, 4, weights=np.ones((2, 30, 4)))
+    assert np.array_equal(np.isnan(plain), np.isnan(ones))
+    assert np.array_equal(plain[~np.isnan(plain)], ones[~np.isnan(ones)])
+    for j in range(4):
+        onehot = np.zeros((2, 30, 4))
+        onehot[..., j] = 1.0
+        got = oracle.indexer_scores(qI, kI, 4, weights=onehot)
+        single = oracle.indexer_scores(qI[:, :, j:j + 1], kI, 4)
+        ok = ~np.isnan(single)
+        assert np.array_equal(got[ok], single[ok])
+
+
+def test_gated_scores_are_linear_and_odd_in_the_weights():
+    rng = np.random.default_rng(22)
+    qI = rng.standard_normal((1, 40, 3, 8))
+    kI = rng.standard_normal((1, 10, 8))
+    w1 = rng.standard_normal((1, 40, 3))
+    w2 = rng.standard_normal((1, 40, 3))
+    s1 = oracle.indexer_scores(qI, kI, 4, weights=w1)
+    s2 = oracle.indexer_scores(qI, kI, 4, weights=w2)
+    s12 = oracle.indexer_scores(qI, kI, 4, weights=2.5 * w1 + w2)
+    ok = ~np.isnan(s1)
+    np.testing.assert_allclose(s12[ok], 2.5 * s1[ok] + s2[ok], rtol=1e-12, atol=1e-12)
+    neg = oracle.indexer_scores(qI, kI, 4, weights=-w1)
+    assert np.array_equal(neg[ok], -s1[ok])                         # each term negates exactly
+
+
+def test_gated_topk_matches_brute_force_on_tiny_inputs():
+    # per-head ReLU dots and the weighted sum written out with Python loops
+    rng = np.random.default_rng(23)
+    H, d, N, n, k = 3, 4, 11, 48, 5
+    qI = rng.standard_normal((1, n, H, d))
+    kI = rng.standard_normal((1, N, d))
+    w = rng.standard_normal((1, n, H))
+    idx, _, _ = oracle.indexer_topk(qI, kI, 4, k, weights=w)
+    for t in range(n):
+        V = min((t + 1) // 4, N)
+        scores = []
+        for s_ in range(V):
+            tot = 0.0
+            for h in range(H):
+                dot = sum(float(qI[0, t, h, c]) * float(kI[0, s_, c]) for c in range(d))
+                tot += float(w[0, t, h]) * max(dot, 0.0)
+            scores.append(tot)
+        want = sorted(range(V), key=lambda i: (-scores[i], i))[:k]
+        assert idx[t][:min(k, V)].tolist() == want
+
+
 # ---------------------------------------------------------------- attention
 def _sdpa_mqa(q, kv, mask=None, causal=False):
     """torch scaled_dot_product_attention in fp64 with one shared KV head."""
