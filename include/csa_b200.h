@@ -166,7 +166,7 @@ csa_status_t csa_compress_append(const void* x_new, int x_dt, int B, int d_in, c
  * score, torch.topk per query) and §8.2 (scores must not be materialised),
  * "DS-V4 分析&学习" §1.2 and §4 (low-precision indexer QK).
  *
- *   score[t, s] = sum_h ReLU(qI[t, h, :] . kI[s, :])  for visible s
+ *   score[t, s] = sum_h w[t, h] * ReLU(qI[t, h, :] . kI[s, :])  for visible s
  *   idx_out[b, q, :] = the topk entries of largest score; equal scores are
  *     taken lowest index first; with V < topk visible entries the row holds
  *     those V entries followed by -1.  The order inside a row is not part of
@@ -181,6 +181,12 @@ csa_status_t csa_compress_append(const void* x_new, int x_dt, int B, int d_in, c
  *      quantised; E4M3 query codes (qI_dt == CSA_DT_E4M3) are taken as given
  *      (already rotated).  Needs d_I a power of two; served by the fp8
  *      tensor-core and cluster kernels (d_I 64, or 128 for few rows).
+ *   qI_weight [B, n_q, H_I] fp32: per-query, per-head gate weights w of any
+ *      sign (the gated form of the DSA-lineage indexer that "DS-V4 分析&学习"
+ *      §1.2 names; no formula is printed there), or NULL for w = 1.  Scores
+ *      may then be negative; they still order as real numbers (-0 equals +0),
+ *      below every zero score.  The weight multiplies the head's ReLU output,
+ *      folded into the per-head query scale in fp32 by the kernels.
  *   kI [B, N_cap, d_I]: kI_dt F32, BF16, or E4M3 with kI_scale [B, N_cap].
  *      Supported pairs: (F32,F32), (BF16,BF16), (BF16,E4M3), (E4M3,E4M3).
  *      With fp8 the score is sk_s * sum_h sq_h * ReLU(q8_h . k8_s).
@@ -189,7 +195,8 @@ csa_status_t csa_compress_append(const void* x_new, int x_dt, int B, int d_in, c
  *   Limits: 1 <= H_I <= 16, d_I multiple of 16 and <= 256, N_cap <= 40960.
  *   idx_out [B, n_q, topk] int32.
  */
-csa_status_t csa_indexer_topk(const void* qI, int qI_dt, const float* qI_scale, const void* kI,
+csa_status_t csa_indexer_topk(const void* qI, int qI_dt, const float* qI_scale,
+                              const float* qI_weight, const void* kI,
                               int kI_dt, const float* kI_scale, int B, int n_q, int H_I, int d_I,
                               int N_cap, const int* n_entries, const int* q_pos, int m, int topk,
                               int* idx_out, void* stream);

@@ -36,7 +36,7 @@ SIGNATURES = {
     "csa_check_device_error": (I, [P, I]),
     "csa_compress": (I, [P, I, I, I, I, P, I, I, I, P, I, P, P]),
     "csa_compress_append": (I, [P, I, I, I, P, I, I, I, P, P, P, I, P, I, P, P]),
-    "csa_indexer_topk": (I, [P, I, P, P, I, P, I, I, I, I, I, P, P, I, I, P, P]),
+    "csa_indexer_topk": (I, [P, I, P, P, P, I, P, I, I, I, I, I, P, P, I, I, P, P]),
     "csa_sparse_attn": (I, [P, I, I, I, I, I, P, I, P, I, P, I, P, P, I, P, F, P, P, P]),
     "hca_dense_attn": (I, [P, I, I, I, I, I, P, I, P, I, P, I, P, P, I, P, F, P, P, P]),
 }
@@ -178,13 +178,19 @@ def csa_compress_append(x_new: torch.Tensor, W: torch.Tensor, m: int, overlap: b
 def csa_indexer_topk(qI: torch.Tensor, kI: torch.Tensor, m: int, topk: int, idx_out: torch.Tensor,
                      qI_scale: torch.Tensor | None = None, kI_scale: torch.Tensor | None = None,
                      n_entries: torch.Tensor | None = None, q_pos: torch.Tensor | None = None,
-                     kI_rotated: bool = False, stream=None) -> None:
+                     kI_rotated: bool = False, qI_weight: torch.Tensor | None = None,
+                     stream=None) -> None:
     """qI [B, n_q, H_I, d_I], kI [B, N_cap, d_I] -> idx_out [B, n_q, topk] int32.
     ``kI_rotated``: fp8 keys written with the Hadamard rotation (bf16 queries are
-    rotated in the kernel; fp8 query codes are taken as already rotated)."""
+    rotated in the kernel; fp8 query codes are taken as already rotated).
+    ``qI_weight`` [B, n_q, H_I] fp32: per-head gate weights, any sign
+    (score = sum_h w_h ReLU(q_h . k))."""
     B, n_q, H_I, d_I = qI.shape
     N_cap = kI.shape[1]
-    _check(load().csa_indexer_topk(_ptr(qI), _dt(qI), _ptr(qI_scale), _ptr(kI),
+    if qI_weight is not None and (qI_weight.dtype != torch.float32 or
+                                  tuple(qI_weight.shape) != (B, n_q, H_I)):
+        raise ValueError("qI_weight must be float32 [B, n_q, H_I]")
+    _check(load().csa_indexer_topk(_ptr(qI), _dt(qI), _ptr(qI_scale), _ptr(qI_weight), _ptr(kI),
                                    _dt_rot(kI, kI_rotated),
                                    _ptr(kI_scale), B, n_q, H_I, d_I, N_cap,
                                    _i32(n_entries, "n_entries"), _i32(q_pos, "q_pos"), m, topk,
@@ -238,11 +244,13 @@ def compress(x: torch.Tensor, W: torch.Tensor, m: int, overlap: bool, out_dtype=
 
 
 def indexer_topk(qI, kI, m: int, topk: int, qI_scale=None, kI_scale=None, n_entries=None,
-                 q_pos=None, kI_rotated: bool = False, stream=None) -> torch.Tensor:
+                 q_pos=None, kI_rotated: bool = False, qI_weight=None,
+                 stream=None) -> torch.Tensor:
     B, n_q = qI.shape[:2]
     idx = torch.empty(B, n_q, topk, dtype=torch.int32, device=qI.device)
     csa_indexer_topk(qI, kI, m, topk, idx, qI_scale=qI_scale, kI_scale=kI_scale,
-                     n_entries=n_entries, q_pos=q_pos, kI_rotated=kI_rotated, stream=stream)
+                     n_entries=n_entries, q_pos=q_pos, kI_rotated=kI_rotated,
+                     qI_weight=qI_weight, stream=stream)
     return idx
 
 
@@ -261,11 +269,12 @@ def hca_attn(q, kv_c, m: int, kv_raw, window: int, with_lse: bool = False, **kw)
 
 
 def csa_prefill(q, kv, qI, kI_raw, W_c, W_Ic, m: int, topk: int, window: int,
-                indexer_fp8: bool, indexer_hadamard: bool = False, stream=None):
+                indexer_fp8: bool, indexer_hadamard: bool = False, qI_weight=None, stream=None):
     """The whole CSA prefill hot path (positions 0..n-1 of each sequence):
     compress kv, compress the indexer keys (fp8 + row scales when
     ``indexer_fp8``, Hadamard-rotated first when ``indexer_hadamard``),
-    indexer + top-k, joint sparse attention.
+    indexer + top-k (gated by ``qI_weight`` [B, n, H_I] when given), joint
+    sparse attention.
     Returns dict(out, idx, kv_c, kI_c, kI_scale)."""
     kv_c = compress(kv, W_c, m, True, stream=stream)
     rot = bool(indexer_fp8 and indexer_hadamard)
@@ -274,6 +283,7 @@ def csa_prefill(q, kv, qI, kI_raw, W_c, W_Ic, m: int, topk: int, window: int,
                                   stream=stream)
     else:
         kI_c, kI_scale = compress(kI_raw, W_Ic, m, True, stream=stream), None
-    idx = indexer_topk(qI, kI_c, m, topk, kI_scale=kI_scale, kI_rotated=rot, stream=stream)
+    idx = indexer_topk(qI, kI_c, m, topk, kI_scale=kI_scale, kI_rotated=rot, qI_weight=qI_weight,
+                       stream=stream)
     out = sparse_attn(q, kv_c, idx, kv, window, stream=stream)
     return dict(out=out, idx=idx, kv_c=kv_c, kI_c=kI_c, kI_scale=kI_scale)

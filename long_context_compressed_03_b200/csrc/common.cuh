@@ -9,6 +9,14 @@ namespace csa {
 
 enum Dtype : int { DT_F32 = 0, DT_BF16 = 1, DT_E4M3 = 2, DT_E4M3H = 3 };
 
+// Order-preserving map of an fp32 score to an unsigned radix key: a larger
+// score gives a larger key, negative scores sort below every zero, and -0
+// and +0 share one key (they are equal scores).
+__device__ __forceinline__ uint32_t score_key(float x) {
+    const uint32_t u = __float_as_uint(x);
+    return x == 0.0f ? 0x80000000u : (u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u));
+}
+
 // Normalised Walsh-Hadamard rotation of a row of d fp32 values (d a power of
 // two) in shared memory, by one warp, in the order the fp8 Hadamard type
 // defines: for stride s = 1, 2, ..., d/2 every pair (i, i+s) with i & s == 0

@@ -178,8 +178,8 @@ csa_status_t csa_compress_append(const void* x_new, int x_dt, int B, int d_in, c
                      "csa_compress_append", why);
 }
 
-csa_status_t csa_indexer_topk(const void* qI, int qI_dt, const float* qI_scale, const void* kI,
-                              int kI_dt, const float* kI_scale, int B, int n_q, int H_I, int d_I,
+csa_status_t csa_indexer_topk(const void* qI, int qI_dt, const float* qI_scale,
+                              const float* qI_weight, const void* kI, int kI_dt, const float* kI_scale, int B, int n_q, int H_I, int d_I,
                               int N_cap, const int* n_entries, const int* q_pos, int m, int topk,
                               int* idx_out, void* stream) {
     REQUIRE(B >= 0 && n_q >= 0 && N_cap >= 0, "csa_indexer_topk: negative size");
@@ -203,11 +203,12 @@ csa_status_t csa_indexer_topk(const void* qI, int qI_dt, const float* qI_scale, 
     REQUIRE_ALIGNED(kI, "kI");
     REQUIRE_ALIGNED(idx_out, "idx_out");
     REQUIRE_ALIGNED(qI_scale, "qI_scale");
+    REQUIRE_ALIGNED(qI_weight, "qI_weight");
     REQUIRE_ALIGNED(kI_scale, "kI_scale");
     REQUIRE_ALIGNED(n_entries, "n_entries");
     REQUIRE_ALIGNED(q_pos, "q_pos");
     csa::IndexerArgs a{qI, qI_dt, qI_scale, kI, kI_dt, kI_scale, B, n_q, H_I, d_I, N_cap,
-                       n_entries, q_pos, m, topk, idx_out, hadamard_norm(d_I)};
+                       n_entries, q_pos, m, topk, idx_out, hadamard_norm(d_I), qI_weight};
     const char* why = nullptr;
     return from_cuda(csa::launch_indexer_topk(a, static_cast<cudaStream_t>(stream), &why),
                      "csa_indexer_topk", why);

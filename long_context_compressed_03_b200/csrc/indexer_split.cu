@@ -2,7 +2,8 @@
 // the exact causal top-k, with one row's visible entries split over the CTAs
 // of a thread-block cluster.
 //
-// score[t, s] = sum_h ReLU(qI[t, h] . kI[s]),  s < V(t) = min(floor((t+1)/m), n_entries)
+// score[t, s] = sum_h w[t, h] ReLU(qI[t, h] . kI[s]),  s < V(t) = min(floor((t+1)/m), n_entries)
+//               (w: gate weights of any sign, 1 when none are given)
 // idx[t, :]   = the topk largest scores, equal scores lowest index first, -1 padded
 // ("百万上下文从「奢侈品」变「日用品」…" §3.2 indexer score and top-k, §8.2
 //  selection without materialising the score matrix; "DS-V4 分析&学习" §1.2,
@@ -49,11 +50,11 @@ constexpr int kMaxHeads = 8;       // one n8 block of the MMA
 constexpr int kGroup = 32;         // entries per warp step (two m16 tiles)
 constexpr int kMaxChunk = 48 * 1024;   // scores per CTA held in shared memory
 static_assert(kWarps == kMaxHeads, "one warp quantises one query head");
-// Radix digits of the 31-bit keys: bits 30-23, 22-15, 14-7 and 7-0 (the last
-// digit repeats bit 7, which the third round fixed).  Four 256-bin rounds
-// measured faster than three rounds of 2048 / 1024 bins.
+// Radix digits of the 32-bit keys (score_key: signed scores with gate
+// weights): bits 31-24, 23-16, 15-8 and 7-0.  Four 256-bin rounds measured
+// faster than three rounds of 2048 / 1024 bins.
 constexpr int kRounds = 4;
-__device__ __forceinline__ int round_shift(int rd) { return rd == 0 ? 23 : (rd == 1 ? 15 : (rd == 2 ? 7 : 0)); }
+__device__ __forceinline__ int round_shift(int rd) { return 24 - 8 * rd; }
 __device__ __forceinline__ int round_bits(int) { return 8; }
 
 struct SplitShared {
@@ -136,7 +137,10 @@ __global__ void __launch_bounds__(kThreads, min_blocks<NU>()) indexer_split_kern
     if constexpr (QD == DT_E4M3) {
         const uint8_t* src = static_cast<const uint8_t*>(a.qI) + (size_t)row * H * d;
         for (int p = tid; p < kMaxHeads * d; p += kThreads) sh.qc[p] = p < H * d ? src[p] : 0;
-        if (tid < kMaxHeads) sh.qs[tid] = tid < H ? a.qI_scale[(size_t)row * H + tid] : 0.0f;
+        if (tid < kMaxHeads)
+            sh.qs[tid] = tid < H ? a.qI_scale[(size_t)row * H + tid] *
+                                       (a.qI_weight ? a.qI_weight[(size_t)row * H + tid] : 1.0f)
+                                 : 0.0f;
     } else {
         const __nv_bfloat16* src = static_cast<const __nv_bfloat16*>(a.qI) + (size_t)row * H * d;
         const int h = warp;   // kWarps == kMaxHeads
@@ -178,7 +182,7 @@ __global__ void __launch_bounds__(kThreads, min_blocks<NU>()) indexer_split_kern
             const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
 #pragma unroll
             for (int j = 0; j < J; ++j) sh.qc[h * d + lane + 32 * j] = e4m3_code(__fdiv_rn(v[j], scale));
-            if (lane == 0) sh.qs[h] = scale;
+            if (lane == 0) sh.qs[h] = a.qI_weight ? scale * a.qI_weight[(size_t)row * H + h] : scale;
         } else {
             for (int c = lane; c < d; c += 32) sh.qc[h * d + c] = 0;
             if (lane == 0) sh.qs[h] = 0.0f;
@@ -222,16 +226,15 @@ __global__ void __launch_bounds__(kThreads, min_blocks<NU>()) indexer_split_kern
             const float p3 = quad_sum(fmaf(qs0, relu0(c1[2]), qs1 * relu0(c1[3])));
             const float mine = tq == 0 ? p0 : (tq == 1 ? p1 : (tq == 2 ? p2 : p3));
             const int e = base + wsel;
-            if (e < hi) keys[e - lo] = __float_as_uint(relu0(mine * cur.sc));
+            if (e < hi) keys[e - lo] = score_key(mine * cur.sc);
             cur = nxt;
         }
     }
     __syncthreads();
 
     // ---- cluster-wide radix select: exact k-th largest key K, and how many == K to take.
-    // Keys are non-negative fp32 bit patterns (bit 31 clear); the digits of
-    // kShift / kBits settle all 31 bits (a digit may repeat bits an earlier
-    // round fixed: they match the prefix).
+    // Keys are score_key() images of the fp32 scores; four 8-bit digits
+    // settle all 32 bits.
     unsigned prefix = 0, pmask = 0, need = (unsigned)topk;
 #pragma unroll 1
     for (int rd = 0; rd < kRounds; ++rd) {

@@ -1,7 +1,8 @@
 // indexer_tc.cu -- tensor-core Lightning-Indexer scores fused with an exact
 // per-query top-k (prefill: 128 consecutive queries of one sequence per CTA).
 //
-// score[t, s] = ks_s * sum_h qs_{t,h} * ReLU(q_{t,h} . k_s)   for s < V(t)
+// score[t, s] = ks_s * sum_h w_{t,h} qs_{t,h} * ReLU(q_{t,h} . k_s)   for s < V(t)
+// (w: gate weights of any sign, 1 when none are given)
 // idx[t, :]   = the topk largest scores, equal scores lowest index first
 // ("百万上下文从「奢侈品」变「日用品」…" §3.2 indexer + top-k, §8.2 streaming
 //  selection without materialising the scores; "DS-V4 分析&学习" §4 low-
@@ -16,6 +17,8 @@
 //
 // Selection: every (row, entry) gets the unique 48-bit key
 //   K = (bits of the non-negative fp32 score) << 16 | (65535 - s),
+// (with gate weights the scores are signed and score_key() supplies the
+// order-preserving 32 bits instead of the raw bit pattern)
 // which orders like (score desc, index asc) -- the top-k tie rule.  An
 // MSB-first radix select over 8-bit digits finds, per row, the digit prefix
 // that holds the k-th largest key: each pass recomputes the scores (the
@@ -64,6 +67,7 @@ struct IdxParams {
     const void* qI;            // [B, n, H_I, 64] bf16 or e4m3 codes
     const float* qI_scale;     // e4m3 queries given as codes: [B, n, H_I]
     const float* kI_scale;     // e4m3 keys: [B, N_cap]
+    const float* qw;           // gate weights [B, n, H_I] (GATED kernels only)
     int q_mode;                // 0 bf16 (bf16 keys), 1 bf16 quantised here, 2 e4m3 codes,
                                // 3 bf16 Hadamard-rotated, then quantised here
     float hnorm;               // q_mode 3: fp32(1/sqrt(64))
@@ -159,17 +163,18 @@ __device__ __forceinline__ void tmem_ld8x4(uint32_t taddr, float (*v)[8]) {
 // One score of this thread's row: fold the four heads, then histogram or
 // emit its key according to the row's pass kind.  KIND_T < 0 takes the kind
 // at run time (rows of one warp at different radix levels).
-template <bool FP8, int KIND_T>
+template <bool FP8, bool GATED, int KIND_T>
 __device__ __forceinline__ void score_one(const float (&acc)[kHeads][8], int e, float ks, int s,
                                           int kind_rt, const RowCtx& rc) {
     const int KIND = KIND_T >= 0 ? KIND_T : kind_rt;
-    // a + |a| = 2 ReLU(a) exactly (+0 for a <= 0), and rc.qs holds qs / 2, so
-    // this is sum_h qs_h ReLU(a_h) on the FMA pipe, always +0 or positive
+    // a + |a| = 2 ReLU(a) exactly (+0 for a <= 0), and rc.qs holds qs / 2
+    // (times the gate weight), so this is sum_h qs_h ReLU(a_h) on the FMA
+    // pipe: +0 or positive without weights, of any sign with them
     float sc = rc.qs[0] * (acc[0][e] + fabsf(acc[0][e]));
 #pragma unroll
     for (int h = 1; h < kHeads; ++h) sc = fmaf(rc.qs[h], acc[h][e] + fabsf(acc[h][e]), sc);
     if (FP8) sc *= ks;
-    const uint32_t sbits = __float_as_uint(sc);
+    const uint32_t sbits = GATED ? score_key(sc) : __float_as_uint(sc);
     if (KIND == kHist0) {
         atomicAdd(rc.hrow + (sbits >> 24) * kRows, 1u);
     } else if (KIND == kHist32) {
@@ -199,7 +204,7 @@ __device__ __forceinline__ void score_one(const float (&acc)[kHeads][8], int e, 
 // warp runs them at the same point, before any per-row branching; rows that
 // are not selecting skip the arithmetic.  KIND_T >= 0 when every selecting
 // row of the warp is in the same pass kind (the usual case).
-template <bool FP8, int KIND_T>
+template <bool FP8, bool GATED, int KIND_T>
 __device__ __forceinline__ void chunk_pass(uint32_t taddr, float ksv, int c, bool active,
                                            int kind_rt, const RowCtx& rc) {
 #pragma unroll 1
@@ -215,16 +220,16 @@ __device__ __forceinline__ void chunk_pass(uint32_t taddr, float ksv, int c, boo
         const int s0 = c * kN + part * 8;
         if (s0 + 8 <= rc.V) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) score_one<FP8, KIND_T>(acc, e, ks[e], s0 + e, kind_rt, rc);
+            for (int e = 0; e < 8; ++e) score_one<FP8, GATED, KIND_T>(acc, e, ks[e], s0 + e, kind_rt, rc);
         } else {
 #pragma unroll
             for (int e = 0; e < 8; ++e)
-                if (s0 + e < rc.V) score_one<FP8, KIND_T>(acc, e, ks[e], s0 + e, kind_rt, rc);
+                if (s0 + e < rc.V) score_one<FP8, GATED, KIND_T>(acc, e, ks[e], s0 + e, kind_rt, rc);
         }
     }
 }
 
-template <bool FP8>
+template <bool FP8, bool GATED>
 __global__ void __launch_bounds__(kThreads, 1)
 indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
     using C = Cfg<FP8>;
@@ -334,6 +339,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
             *reinterpret_cast<uint16_t*>(at + off) = (uint16_t)packed;
         else
             *reinterpret_cast<uint32_t*>(at + off) = packed;
+        if (GATED && h < p.H_I) qs *= p.qw[qrow];
         if (lane == 0) rs->qs[r][h] = (h < p.H_I) ? qs : 0.0f;
     }
     fence_proxy_async_smem();
@@ -441,11 +447,11 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
                 tc_fence_after();
                 const uint32_t taddr = tmem + lane_addr + grp * 128;
                 switch (wkind) {
-                    case kHist0: chunk_pass<FP8, kHist0>(taddr, ksv, c, active, kind, rc); break;
-                    case kHist32: chunk_pass<FP8, kHist32>(taddr, ksv, c, active, kind, rc); break;
-                    case kHist64: chunk_pass<FP8, kHist64>(taddr, ksv, c, active, kind, rc); break;
-                    case kEmit: chunk_pass<FP8, kEmit>(taddr, ksv, c, active, kind, rc); break;
-                    default: chunk_pass<FP8, -1>(taddr, ksv, c, active, kind, rc); break;
+                    case kHist0: chunk_pass<FP8, GATED, kHist0>(taddr, ksv, c, active, kind, rc); break;
+                    case kHist32: chunk_pass<FP8, GATED, kHist32>(taddr, ksv, c, active, kind, rc); break;
+                    case kHist64: chunk_pass<FP8, GATED, kHist64>(taddr, ksv, c, active, kind, rc); break;
+                    case kEmit: chunk_pass<FP8, GATED, kEmit>(taddr, ksv, c, active, kind, rc); break;
+                    default: chunk_pass<FP8, GATED, -1>(taddr, ksv, c, active, kind, rc); break;
                 }
                 ksv = ksv_next;
                 tc_fence_before();
@@ -590,6 +596,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
     return fn;
 }
 
+template <bool FP8, bool GATED>
+cudaError_t launch_k(dim3 grid, const CUtensorMap& tm, const IdxParams& p, cudaStream_t s) {
+    auto k = indexer_tc_kernel<FP8, GATED>;
+    cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg<FP8>::kSmem);
+    if (e != cudaSuccess) return e;
+    k<<<grid, kThreads, Cfg<FP8>::kSmem, s>>>(tm, p);
+    return cudaSuccess;
+}
+
 }  // namespace
 
 bool indexer_tc_supported(const IndexerArgs& a) {
@@ -630,18 +645,15 @@ cudaError_t launch_indexer_tc(const IndexerArgs& a, uint32_t* err, cudaStream_t 
     p.n_entries = a.n_entries;
     p.idx_out = a.idx_out;
     p.err = err;
+    p.qw = a.qI_weight;
     const int tiles = (a.n_q + kRows - 1) / kRows;
-    if (fp8) {
-        auto k = indexer_tc_kernel<true>;
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg<true>::kSmem);
-        if (e != cudaSuccess) return e;
-        k<<<(unsigned)(a.B * tiles), kThreads, Cfg<true>::kSmem, s>>>(tm, p);
-    } else {
-        auto k = indexer_tc_kernel<false>;
-        cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)Cfg<false>::kSmem);
-        if (e != cudaSuccess) return e;
-        k<<<(unsigned)(a.B * tiles), kThreads, Cfg<false>::kSmem, s>>>(tm, p);
-    }
+    const dim3 grid((unsigned)(a.B * tiles));
+    cudaError_t e;
+    if (fp8)
+        e = a.qI_weight ? launch_k<true, true>(grid, tm, p, s) : launch_k<true, false>(grid, tm, p, s);
+    else
+        e = a.qI_weight ? launch_k<false, true>(grid, tm, p, s) : launch_k<false, false>(grid, tm, p, s);
+    if (e != cudaSuccess) return e;
     count_launch();
     return cudaGetLastError();
 }

@@ -1,13 +1,14 @@
 // indexer_topk.cu -- stage 2: Lightning-Indexer score + fused causal top-k.
 //
-// score[t, s] = sum_h ReLU(qI[t, h] . kI[s]),  s < V(t) = min(floor((t+1)/m), n_entries)
+// score[t, s] = sum_h w[t, h] ReLU(qI[t, h] . kI[s]),  s < V(t) = min(floor((t+1)/m), n_entries)
+//               (w: gate weights of any sign, 1 when none are given)
 // idx[t, :]   = the topk largest scores, equal scores lowest index first, -1 padded
 // ("百万上下文从「奢侈品」变「日用品」…" §3.2 indexer score + torch.topk, §8.2
 //  streaming selection; "DS-V4 分析&学习" §1.2, §4 low-precision indexer QK.)
 //
 // One CTA owns one query row.  It scores the row's visible entries into
-// shared memory (never global memory) as the bit patterns of non-negative
-// fp32 scores, which order like the values; a four-digit MSB-first radix
+// shared memory (never global memory) as order-preserving 32-bit images of
+// the fp32 scores (score_key); a four-digit MSB-first radix
 // select finds the exact k-th largest key K and how many keys equal to K
 // are needed; a block-wide ordered scan then writes every entry with key > K
 // and the lowest-index entries with key == K.  Rows with V <= topk skip the
@@ -61,7 +62,8 @@ template <int KD>
 __device__ __forceinline__ size_t elem_bytes() { return KD == DT_F32 ? 4 : (KD == DT_BF16 ? 2 : 1); }
 
 // Q modes: the query row as held in shared memory is always fp32 values `qv`
-// with one positive multiplier per head `qs` (1 unless fp8).
+// with one multiplier per head `qs`: the fp8 scale (1 unless fp8) times the
+// head's gate weight (1 without weights).
 template <int QD, int KD>
 __global__ void __launch_bounds__(kThreads) indexer_topk_kernel(IndexerArgs a) {
     extern __shared__ unsigned keys[];   // [N_cap] score keys of this row
@@ -106,6 +108,10 @@ __global__ void __launch_bounds__(kThreads) indexer_topk_kernel(IndexerArgs a) {
         for (int h = threadIdx.x; h < H; h += kThreads) qs[h] = 1.0f;
     }
     __syncthreads();
+    if (a.qI_weight) {
+        for (int h = threadIdx.x; h < H; h += kThreads) qs[h] *= a.qI_weight[(size_t)row * H + h];
+        __syncthreads();
+    }
 
     // ---- scores of the visible entries, as order-preserving keys
     const uint8_t* kbase = static_cast<const uint8_t*>(a.kI) + (size_t)b * a.N_cap * d * elem_bytes<KD>();
@@ -131,7 +137,7 @@ __global__ void __launch_bounds__(kThreads) indexer_topk_kernel(IndexerArgs a) {
         for (int h = 0; h < kMaxHeads; ++h)
             if (h < H) sc = fmaf(qs[h], relu0(dots[h]), sc);
         if constexpr (KD == DT_E4M3) sc *= a.kI_scale[(size_t)b * a.N_cap + s];
-        keys[s] = __float_as_uint(relu0(sc));
+        keys[s] = score_key(sc);
     }
     __syncthreads();
 

@@ -38,6 +38,7 @@ struct IndexerArgs {
     int m, topk;
     int* idx_out;
     float hnorm;               // fp32(1/sqrt(d_I)): keys of the Hadamard fp8 type
+    const float* qI_weight;    // [B, n_q, H_I] gate weights or NULL (all 1)
 };
 
 struct AttnArgs {

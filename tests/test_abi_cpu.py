@@ -104,20 +104,23 @@ def test_compress_append_validation(lib):
 
 def test_indexer_validation(lib):
     f = lib.csa_indexer_topk
-    args = [FAKE, 1, None, FAKE, 1, None, 1, 8, 4, 64, 16, None, None, 4, 8, FAKE, None]
-    bad = list(args); bad[14] = 0                      # topk = 0
+    #       qI  dt scale wt  kI   dt scale B  n_q H  d   N   ne    pos   m  k  idx   stream
+    args = [FAKE, 1, None, None, FAKE, 1, None, 1, 8, 4, 64, 16, None, None, 4, 8, FAKE, None]
+    bad = list(args); bad[15] = 0                      # topk = 0
     assert f(*bad) == api.CSA_ERR_INVALID_ARG
-    bad = list(args); bad[14] = 4096                   # topk > 2048
+    bad = list(args); bad[15] = 4096                   # topk > 2048
     assert f(*bad) == api.CSA_ERR_INVALID_ARG
-    bad = list(args); bad[4] = 2                       # fp8 keys without scales
+    bad = list(args); bad[5] = 2                       # fp8 keys without scales
     assert f(*bad) == api.CSA_ERR_INVALID_ARG
-    bad = list(args); bad[9] = 60                      # d_I not a multiple of 16
+    bad = list(args); bad[10] = 60                     # d_I not a multiple of 16
     assert f(*bad) == api.CSA_ERR_UNSUPPORTED
     bad = list(args); bad[0] = ODD
     assert f(*bad) == api.CSA_ERR_MISALIGNED
-    bad = list(args); bad[13] = 0                      # m = 0
+    bad = list(args); bad[3] = ODD                     # misaligned gate weights
+    assert f(*bad) == api.CSA_ERR_MISALIGNED
+    bad = list(args); bad[14] = 0                      # m = 0
     assert f(*bad) == api.CSA_ERR_INVALID_ARG
-    ok = list(args); ok[7] = 0                         # n_q = 0: no-op
+    ok = list(args); ok[8] = 0                         # n_q = 0: no-op
     assert f(*ok) == api.CSA_OK
 
 
@@ -141,14 +144,14 @@ def test_hadamard_type_validation(lib):
     ok = list(args); ok[5] = 128; ok[2] = 0
     assert g(*ok) == api.CSA_OK
     h = lib.csa_indexer_topk
-    args = [FAKE, 1, None, FAKE, H, FAKE, 1, 8, 4, 64, 16, None, None, 4, 8, FAKE, None]
-    bad = list(args); bad[9] = 48                      # d_I not a power of two
+    args = [FAKE, 1, None, None, FAKE, H, FAKE, 1, 8, 4, 64, 16, None, None, 4, 8, FAKE, None]
+    bad = list(args); bad[10] = 48                     # d_I not a power of two
     assert h(*bad) == api.CSA_ERR_UNSUPPORTED
-    bad = list(args); bad[5] = None                    # rotated keys without scales
+    bad = list(args); bad[6] = None                    # rotated keys without scales
     assert h(*bad) == api.CSA_ERR_INVALID_ARG
     bad = list(args); bad[1] = H; bad[2] = FAKE        # queries as the rotated type
     assert h(*bad) == api.CSA_ERR_UNSUPPORTED
-    ok = list(args); ok[7] = 0
+    ok = list(args); ok[8] = 0
     assert h(*ok) == api.CSA_OK
     a = lib.csa_sparse_attn
     args = [FAKE, H, 1, 8, 64, 128, FAKE, 16, FAKE, 4, FAKE, 8, None, None, 4, None,

@@ -45,7 +45,8 @@ def _sylvester(d):
     return h / math.sqrt(d)
 
 
-def _decode_indexer(seed, B, n_q, N_cap, H_I, d_I, k, ctx, q_kind="bf16", m=4, tie_rows=False):
+def _decode_indexer(seed, B, n_q, N_cap, H_I, d_I, k, ctx, q_kind="bf16", m=4, tie_rows=False,
+                    gated=False):
     g = _gen(seed)
     qI = torch.randn(B, n_q, H_I, d_I, generator=g).to(torch.bfloat16)
     kI = torch.randn(B, N_cap, d_I, generator=g)
@@ -58,6 +59,9 @@ def _decode_indexer(seed, B, n_q, N_cap, H_I, d_I, k, ctx, q_kind="bf16", m=4, t
     ne = np.minimum(np.asarray(ctx) // m, N_cap).astype(np.int32)
     q_pos = np.stack([np.asarray(ctx) - 1 - j for j in range(n_q)], axis=1).astype(np.int32)
     kw = dict(kI_scale=T(sc), n_entries=T(ne), q_pos=T(q_pos))
+    w = torch.randn(B, n_q, H_I, generator=g) if gated else None
+    if gated:
+        kw["qI_weight"] = T(w)
     if q_kind == "e4m3":
         qc, qs = _fp8_rows(qI)
         idx = api.indexer_topk(T(qc), T(codes), m, k, qI_scale=T(qs), **kw)
@@ -67,7 +71,9 @@ def _decode_indexer(seed, B, n_q, N_cap, H_I, d_I, k, ctx, q_kind="bf16", m=4, t
         q_rows = oracle.quantized_query_rows(qI.float().numpy(), rotate=rot)
     q_rows = q_rows.reshape(B * n_q, H_I, d_I)
     rb = np.repeat(np.arange(B, dtype=np.int32), n_q)
-    scores = oracle.indexer_scores_rows(q_rows, rb, q_pos.reshape(-1), codes.numpy(), m, ne, sc.numpy())
+    wr = None if w is None else w.double().numpy().reshape(B * n_q, H_I)
+    scores = oracle.indexer_scores_rows(q_rows, rb, q_pos.reshape(-1), codes.numpy(), m, ne, sc.numpy(),
+                                        weights=wr)
     return idx.cpu().numpy().reshape(B * n_q, k), scores, ne, q_pos
 
 
@@ -90,6 +96,23 @@ def test_decode_indexer_matches_oracle(case):
     if B > 2:
         ctx[2] = 4 * (k // 2)               # fewer visible than k: -1 padding
     got, scores, _, _ = _decode_indexer(17 + B, B, n_q, N_cap, H_I, d_I, k, ctx, qk)
+    stats = check_topk(got, scores, k)
+    assert stats["exact"] + stats["near_ties"] == stats["rows"]
+
+
+@pytest.mark.parametrize("case", [
+    # (B, n_q, N_cap, H_I, d_I, k, q kind)
+    (5, 1, 3000, 4, 64, 64, "bf16"),
+    (2, 2, 50000, 8, 128, 512, "e4m3"),     # 16-CTA clusters, signed keys across ranks
+    (4, 1, 6000, 4, 64, 256, "bf16_rot"),
+])
+def test_decode_indexer_gated_matches_oracle(case):
+    B, n_q, N_cap, H_I, d_I, k, qk = case
+    rng = np.random.default_rng(N_cap + 1)
+    ctx = rng.integers(4 * k, 4 * N_cap + 40, size=B)
+    ctx[0] = 4 * N_cap + 3
+    got, scores, _, _ = _decode_indexer(57 + B, B, n_q, N_cap, H_I, d_I, k, ctx, qk, gated=True)
+    assert np.nanmin(scores) < 0.0                  # the weights made negative scores
     stats = check_topk(got, scores, k)
     assert stats["exact"] + stats["near_ties"] == stats["rows"]
 

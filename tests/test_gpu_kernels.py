@@ -193,6 +193,42 @@ def test_indexer_topk_matches_oracle(case):
     assert stats["exact"] + stats["near_ties"] == stats["rows"]
 
 
+@pytest.mark.parametrize("case", [
+    # (B, n, H_I, d_I, kind, k, weight sign)
+    (2, 700, 4, 64, "bf16", 32, "mixed"),        # tensor-core kernel, bf16
+    (2, 901, 4, 64, "e4m3", 64, "mixed"),        # tensor-core kernel, fp8
+    (1, 4100, 2, 64, "e4m3", 300, "mixed"),
+    (1, 1200, 4, 64, "e4m3_rot", 100, "mixed"),  # with rotated keys
+    (2, 901, 4, 64, "e4m3", 64, "negative"),     # every score <= 0: zeros first, lowest index
+    (1, 512, 3, 32, "f32", 8, "mixed"),          # SIMT kernel
+    (1, 333, 16, 32, "bf16", 7, "mixed"),
+])
+def test_indexer_gated_matches_oracle(case):
+    """score = sum_h w_h ReLU(q_h . k) with per-(query, head) weights of any sign."""
+    B, n, H_I, d_I, kind, k, sign = case
+    dev, orc, ne, rb, rt, m = _index_case(31 + n, B, n, H_I, d_I, kind, k)
+    w = torch.randn(B, n, H_I, generator=_gen(77 + n))
+    if sign == "negative":
+        w = -w.abs()
+    idx = api.indexer_topk(dev["qI"], dev["kI"], m, k, qI_scale=dev.get("qI_scale"),
+                           kI_scale=dev.get("kI_scale"), kI_rotated=kind == "e4m3_rot",
+                           qI_weight=w.to(DEV))
+    got = idx.cpu().numpy().reshape(B * n, k)
+    scores = oracle.indexer_scores_rows(orc["q_rows"], rb, rt, orc["kI"], m, ne, orc["kI_scale"],
+                                        weights=w.double().numpy().reshape(B * n, H_I))
+    stats = check_topk(got, scores, k)
+    assert stats["exact"] + stats["near_ties"] == stats["rows"]
+    if sign == "negative":
+        # rows with at least k zero scores take exactly the k lowest-index zeros
+        for r in range(B * n):
+            V = int(np.sum(~np.isnan(scores[r])))
+            zeros = np.flatnonzero(scores[r][:V] == 0.0)
+            if V > k and zeros.size >= k + 8:
+                near = np.flatnonzero(np.abs(scores[r][:V]) < 1e-3)
+                if near.size == zeros.size:          # no fp32-vs-fp64 sign doubt near zero
+                    assert np.array_equal(np.sort(got[r]), zeros[:k])
+
+
 def test_indexer_decode_positions_and_entry_counts():
     B, n_q, k = 3, 5, 16
     n = 400
