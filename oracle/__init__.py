@@ -67,6 +67,7 @@ def _load():
         lib.oracle_visible_entries.argtypes = [i64, i32, i64]
         lib.oracle_visible_entries.restype = i64
         lib.oracle_compress.argtypes = [P, i32, i32, i32, P, i32, i32, i32, P]
+        lib.oracle_compress_gated.argtypes = [P, i32, i32, i32, P, P, P, i32, i32, i32, P]
         lib.oracle_compress_append.argtypes = [P, P, i32, i32, P, i32, i32, i32, P, P, i32, P]
         dbl = ctypes.c_double
         lib.oracle_indexer_scores.argtypes = [P, P, P, P, i64, i32, i32, P, P, P, i32, P, i32, P]
@@ -169,6 +170,27 @@ def compress(x, W, m: int, overlap: bool) -> np.ndarray:
     if N_c:
         _load().oracle_compress(_ptr(x), B, n, d_in, _ptr(W), d_out, m, int(bool(overlap)),
                                 _ptr(out))
+    return out
+
+
+def compress_gated(x, W_kv, W_gate, ape, m: int, overlap: bool) -> np.ndarray:
+    """The gated-softmax compressor (reading in csa_oracle.c): per channel, a
+    softmax over the window's positions of (x @ W_gate + ape[p mod m]) weights
+    x @ W_kv; overlapping windows take the first half of the projected
+    channels from the previous block and the second half from the current one.
+    x [B, n, d_in]; W_kv, W_gate [d_in, c*d_out]; ape [m, c*d_out], c = 2 if
+    overlap else 1.  Returns [B, floor(n/m), d_out] (fp64)."""
+    x, W_kv, W_gate, ape = _f64(x), _f64(W_kv), _f64(W_gate), _f64(ape)
+    B, n, d_in = x.shape
+    c = 2 if overlap else 1
+    assert W_kv.shape == W_gate.shape and W_kv.shape[0] == d_in and W_kv.shape[1] % c == 0
+    d_out = W_kv.shape[1] // c
+    assert ape.shape == (m, c * d_out)
+    N_c = num_entries(n, m)
+    out = np.zeros((B, N_c, d_out), dtype=np.float64)
+    if N_c:
+        _load().oracle_compress_gated(_ptr(x), B, n, d_in, _ptr(W_kv), _ptr(W_gate), _ptr(ape),
+                                      d_out, m, int(bool(overlap)), _ptr(out))
     return out
 
 

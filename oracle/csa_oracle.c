@@ -184,6 +184,68 @@ void oracle_compress(const double* x, int B, int n, int d_in, const double* W, i
 }
 
 /* ------------------------------------------------------------------------
+ * Stage 1, learned variant: the gated-softmax compressor.  [P1] §3.2 lists
+ * the production compressor's parts -- a KV projection (linear_wkv), a gate
+ * projection (linear_wgate), softmax / split / reshape, and an APE parameter;
+ * ratio 4 overlapping, ratio 128 not -- but prints no formula.  Reading:
+ *
+ *   c = 2 when overlapping, else 1; each position p projects to
+ *     v_p = x_p @ W_kv                     (c * d_out values)
+ *     z_p = x_p @ W_gate + ape[p mod m]    (c * d_out logits; ape is [m, c*d_out])
+ *   Entry i < floor(n/m), channel e < d_out, is a softmax-weighted pool over
+ *   the positions of its window, taken per channel:
+ *     overlapping: block i-1 contributes (z_p[e], v_p[e]) -- the first half of
+ *       the projected channels -- and block i contributes (z_p[d_out+e],
+ *       v_p[d_out+e]) -- the second half ("split"); entry 0 has block 0 only;
+ *     otherwise: block i contributes (z_p[e], v_p[e]).
+ *   out[i, e] = sum_p exp(z - zmax) v / sum_p exp(z - zmax)  over those terms.
+ * --------------------------------------------------------------------- */
+void oracle_compress_gated(const double* x, int B, int n, int d_in, const double* W_kv,
+                           const double* W_gate, const double* ape, int d_out, int m, int overlap,
+                           double* out) {
+    int N_c = (int)oracle_num_entries(n, m);
+    int cw = overlap ? 2 * d_out : d_out;          /* projected width */
+    #pragma omp parallel for collapse(2) schedule(static)
+    for (int b = 0; b < B; ++b) {
+        for (int i = 0; i < N_c; ++i) {
+            /* the window's terms: (position, channel offset of its half) */
+            long first = (overlap && i > 0) ? (long)m * (i - 1) : (long)m * i;
+            long last = (long)m * (i + 1);          /* exclusive */
+            long nt = last - first;
+            double* z = (double*)malloc(sizeof(double) * (size_t)nt);
+            double* v = (double*)malloc(sizeof(double) * (size_t)nt);
+            double* o = out + ((long)b * N_c + i) * d_out;
+            for (int e = 0; e < d_out; ++e) {
+                for (long t = 0; t < nt; ++t) {
+                    long p = first + t;
+                    int half = (overlap && p >= (long)m * i) ? d_out : 0;
+                    int ch = half + e;
+                    const double* row = x + ((long)b * n + p) * d_in;
+                    double zv = 0.0, vv = 0.0;
+                    for (int k = 0; k < d_in; ++k) {
+                        zv += row[k] * W_gate[(long)k * cw + ch];
+                        vv += row[k] * W_kv[(long)k * cw + ch];
+                    }
+                    z[t] = zv + ape[(long)(p % m) * cw + ch];
+                    v[t] = vv;
+                }
+                double zmax = -INFINITY;
+                for (long t = 0; t < nt; ++t) if (z[t] > zmax) zmax = z[t];
+                double num = 0.0, den = 0.0;
+                for (long t = 0; t < nt; ++t) {
+                    double w = exp(z[t] - zmax);
+                    num += w * v[t];
+                    den += w;
+                }
+                o[e] = num / den;
+            }
+            free(z);
+            free(v);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------
  * Decode-time compression state ("DS-V4 分析&学习", opening summary: the KV
  * cache is the compressed cache plus a state cache and a tail state; §1.3:
  * an overlapping entry spans the previous and the current block, which makes

@@ -283,6 +283,78 @@ def test_kth_scores_match_numpy_sort():
             assert smax[t] == np.abs(row).max()
 
 
+# ---------------------------------------------------------------- gated compressor
+def test_gated_compress_hand_worked_example():
+    # m = 2, no overlap, d_in = d_out = 1, W_kv = 1, W_gate = ln 2, ape = 0:
+    # weights are 2^x, so block (1, 2) pools to (2*1 + 4*2)/6 = 5/3 and block
+    # (3, 4) to (8*3 + 16*4)/24 = 11/3; the trailing position 5 makes no entry
+    x = np.array([[[1.0], [2.0], [3.0], [4.0], [5.0]]])
+    out = oracle.compress_gated(x, np.ones((1, 1)), np.full((1, 1), math.log(2.0)),
+                                np.zeros((2, 1)), 2, False)
+    np.testing.assert_allclose(out[0, :, 0], [5.0 / 3.0, 11.0 / 3.0], rtol=1e-15)
+
+
+def test_gated_compress_overlap_routes_channel_halves_by_block():
+    # d_out = 1, overlap: the previous block is read through projected channel
+    # 0 and the current block through channel 1.  W_kv = (1, 10) and equal
+    # logits: entry 0 = mean of 10 x over block 0; entry i > 0 = mean of
+    # (x over block i-1, 10 x over block i)
+    x = np.arange(1.0, 9.0).reshape(1, 8, 1)
+    out = oracle.compress_gated(x, np.array([[1.0, 10.0]]), np.zeros((1, 2)), np.zeros((2, 2)),
+                                2, True)
+    assert out.shape == (1, 4, 1)
+    np.testing.assert_allclose(out[0, 0, 0], 10 * (1 + 2) / 2)
+    for i in range(1, 4):
+        prev = x[0, 2 * i - 2:2 * i, 0]
+        cur = 10 * x[0, 2 * i:2 * i + 2, 0]
+        np.testing.assert_allclose(out[0, i, 0], (prev.sum() + cur.sum()) / 4, rtol=1e-15)
+
+
+@pytest.mark.parametrize("overlap", [True, False])
+def test_gated_compress_with_flat_gates_is_the_mean_pool(overlap):
+    # zero gate weights and a constant APE give a uniform softmax; with both
+    # channel halves of W_kv equal to W this is mean-then-project (linear)
+    rng = np.random.default_rng(31)
+    B, n, d_in, d_out, m = 2, 37, 6, 5, 4
+    x = rng.standard_normal((B, n, d_in))
+    W = rng.standard_normal((d_in, d_out))
+    c = 2 if overlap else 1
+    W_kv = np.concatenate([W] * c, axis=1)
+    ape = np.full((m, c * d_out), 0.7)
+    got = oracle.compress_gated(x, W_kv, np.zeros((d_in, c * d_out)), ape, m, overlap)
+    np.testing.assert_allclose(got, oracle.compress(x, W, m, overlap), rtol=1e-12, atol=1e-12)
+
+
+def test_gated_compress_dominant_gate_selects_one_position():
+    # a logit 60 above the rest puts weight 1 - O(e^-60) on one position
+    rng = np.random.default_rng(32)
+    B, n, d_in, d_out, m = 1, 16, 3, 2, 4
+    x = rng.standard_normal((B, n, d_in))
+    W_kv = rng.standard_normal((d_in, 2 * d_out))
+    ape = np.zeros((m, 2 * d_out))
+    ape[1, d_out:] = 60.0          # current block, its position 1, every channel
+    out = oracle.compress_gated(x, W_kv, np.zeros((d_in, 2 * d_out)), ape, m, True)
+    for i in range(n // m):
+        v = x[0, m * i + 1] @ W_kv[:, d_out:]
+        np.testing.assert_allclose(out[0, i], v, rtol=1e-12, atol=1e-12)
+
+
+def test_gated_compress_is_causal_and_shift_invariant_in_the_logits():
+    rng = np.random.default_rng(33)
+    B, n, d_in, d_out, m = 1, 24, 4, 3, 4
+    x = rng.standard_normal((B, n, d_in))
+    W_kv = rng.standard_normal((d_in, 2 * d_out))
+    W_g = rng.standard_normal((d_in, 2 * d_out))
+    ape = rng.standard_normal((m, 2 * d_out))
+    a = oracle.compress_gated(x, W_kv, W_g, ape, m, True)
+    y = x.copy()
+    y[0, 13:] += 5.0               # entries 0..2 end before position 12
+    b = oracle.compress_gated(y, W_kv, W_g, ape, m, True)
+    assert np.array_equal(a[0, :3], b[0, :3]) and not np.allclose(a[0, 3:], b[0, 3:])
+    c = oracle.compress_gated(x, W_kv, W_g, ape + 3.25, m, True)
+    np.testing.assert_allclose(c, a, rtol=1e-12, atol=1e-12)
+
+
 # ---------------------------------------------------------------- gated indexer
 def test_gated_scores_hand_worked_example():
     # two heads, d = 2, weights (2, -3); worked by hand:
