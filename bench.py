@@ -242,6 +242,58 @@ def run_prefill(w, dev, steps, warmup, dist_ctx, rank):
                 path=path, inp=inp)
 
 
+def run_variants(w, path, dev, steps, rank):
+    """The NEXT-row variants of the prefill workload, each timed alone with
+    CUDA events and L2 flushed between iterations (their inputs are smaller
+    than L2): the gated-softmax compressor on kv, the Hadamard-rotated fp8
+    compression of the indexer keys, and the indexer + top-k with gate
+    weights against the rotated keys."""
+    d, B, n, m = path.d, w.B, w.n, w.m
+    N_c = n // m
+    gw = {k: v.to(dev) for k, v in synth.gated_compressor_weights(w.D, w.D, m, True, seed=rank).items()}
+    qw = synth.indexer_variant_inputs(B, n, w.H_I, seed=rank)["qI_weight"].to(dev)
+    kv_g = torch.empty(B, N_c, w.D, dtype=torch.bfloat16, device=dev)
+    kI_r = torch.empty(B, N_c, w.d_I, dtype=torch.uint8, device=dev)
+    kI_rs = torch.empty(B, N_c, dtype=torch.float32, device=dev)
+    idx = torch.empty(B, n, w.topk, dtype=torch.int32, device=dev)
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=dev)
+    calls = {
+        "compress_gated_kv": lambda: api.csa_compress_gated(d["kv"], gw["W_kv"], gw["W_gate"],
+                                                            gw["ape"], m, True, kv_g),
+        "compress_kI_hadamard": lambda: api.csa_compress(d["kI_raw"], d["W_Ic"], m, True, kI_r,
+                                                         kI_rs, hadamard=True),
+        "indexer_topk_gated_hadamard": lambda: api.csa_indexer_topk(
+            d["qI"], kI_r, m, w.topk, idx, kI_scale=kI_rs, kI_rotated=True, qI_weight=qw),
+    }
+    e = 2
+    c = 2
+    work = {
+        "compress_gated_kv": dict(flops=2.0 * B * n * w.D * 2 * c * w.D,
+                                  bytes=B * n * w.D * e + 2 * w.D * c * w.D * e + m * c * w.D * 4
+                                  + B * N_c * w.D * e),
+        "compress_kI_hadamard": prefill_work(w)["compress_kI"],
+        "indexer_topk_gated_hadamard": prefill_work(w)["indexer_topk"],
+    }
+    out = {}
+    for name, fn in calls.items():
+        for _ in range(2):
+            fn()
+        ts = []
+        for _ in range(steps):
+            flush.fill_(1)
+            a_, b_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a_.record()
+            fn()
+            b_.record()
+            ts.append((a_, b_))
+        torch.cuda.synchronize()
+        ms = float(np.mean([a_.elapsed_time(b_) for a_, b_ in ts]))
+        out[name] = {"ms": ms, "TFLOP/s": work[name]["flops"] / (ms / 1e3) / 1e12,
+                     "GB/s": work[name]["bytes"] / (ms / 1e3) / 1e9}
+    del flush
+    return out
+
+
 def run_e2e(w, inp, dev, steps):
     """Same step through the public API with pinned host inputs: h2d copies of
     the step's inputs and a d2h read of its result are inside the timed region."""
@@ -453,6 +505,8 @@ def main():
     ap.add_argument("--n", type=int, default=0,
                     help="override the prefill length (smaller cases for profiler captures; "
                          "the line is then marked as not the headline workload)")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the timing of the NEXT-row variants")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--decode-only", action="store_true",
                     help="run only the decode steps (profiler captures of the decode kernels)")
@@ -558,6 +612,13 @@ def main():
             "roofline": roof, "stages": stages, "gpu_launches": pre["launches"],
             "clocks": pre["clocks"]}
 
+    if not args.no_variants:
+        line["variants"] = {
+            "workload": PREFILL, "l2": "flushed (512 MiB write) between iterations",
+            "note": "NEXT rows, each timed alone: gated-softmax compressor (kv, d 128, m 4 "
+                    "overlapping), Hadamard-rotated fp8 indexer keys, gated indexer + top-k "
+                    "against rotated keys",
+            **run_variants(w, pre["path"], dev, max(3, args.steps), rank)}
     if not args.no_decode:
         dec = run_decode(dev, args.steps, args.warmup, rank)
         dval, dms = dist_ctx.job_rate(dec["w"].B, dec["ms"])

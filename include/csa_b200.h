@@ -122,6 +122,33 @@ csa_status_t csa_compress(const void* x, int x_dt, int B, int n, int d_in, const
                           float* out_row_scale, void* stream);
 
 /*
+ * csa_compress_gated -- stage 1, learned variant: the gated-softmax
+ * compressor.  "DeepSeek V4 CSA + CP 迁移到 HP：困难点深度分析" §3.2 lists the
+ * production compressor's parts (a KV projection linear_wkv, a gate
+ * projection linear_wgate, softmax / split / reshape, an APE parameter;
+ * ratio 4 overlapping, ratio 128 not) without a formula; this is the reading:
+ *
+ *   c = 2 if overlap else 1;  for every position p:
+ *     v_p = x[b, p] @ W_kv,   z_p = x[b, p] @ W_gate + ape[p mod m]   (c*d_out each)
+ *   entry i < floor(n/m), channel e < d_out:
+ *     overlap: terms (z_p[e], v_p[e]) for p in block i-1 (absent for i = 0)
+ *              and (z_p[d_out+e], v_p[d_out+e]) for p in block i;
+ *     plain:   terms (z_p[e], v_p[e]) for p in block i;
+ *     out[b, i, e] = sum_terms softmax(z) v.
+ *
+ *   x      [B, n, d_in]       x_dt CSA_DT_F32 or CSA_DT_BF16
+ *   W_kv, W_gate [d_in, c*d_out]  same dtype as x
+ *   ape    [m, c*d_out]       fp32
+ *   out, out_dt, out_row_scale: as csa_compress (fp32 / bf16 / E4M3 / rotated E4M3).
+ *   Limits: 16 <= d_in, d_out <= 256, multiples of 16; m >= 1.  Projections,
+ *   softmax and pooling run in fp32 (expf).  Pointers 16-byte aligned.
+ *   Errors as csa_compress; nothing is launched on a validation error.
+ */
+csa_status_t csa_compress_gated(const void* x, int x_dt, int B, int n, int d_in, const void* W_kv,
+                                const void* W_gate, const float* ape, int d_out, int m, int overlap,
+                                void* out, int out_dt, float* out_row_scale, void* stream);
+
+/*
  * csa_compress_append -- decode-time stage 1: one new token per batch element
  * updates the compressor state and, when it completes a block, writes that
  * block's compressed entry into the cache.

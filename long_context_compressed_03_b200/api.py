@@ -35,6 +35,7 @@ SIGNATURES = {
     "csa_kernel_launches": (ctypes.c_ulonglong, []),
     "csa_check_device_error": (I, [P, I]),
     "csa_compress": (I, [P, I, I, I, I, P, I, I, I, P, I, P, P]),
+    "csa_compress_gated": (I, [P, I, I, I, I, P, P, P, I, I, I, P, I, P, P]),
     "csa_compress_append": (I, [P, I, I, I, P, I, I, I, P, P, P, I, P, I, P, P]),
     "csa_indexer_topk": (I, [P, I, P, P, P, I, P, I, I, I, I, I, P, P, I, I, P, P]),
     "csa_sparse_attn": (I, [P, I, I, I, I, I, P, I, P, I, P, I, P, P, I, P, F, P, P, P]),
@@ -156,6 +157,25 @@ def csa_compress(x: torch.Tensor, W: torch.Tensor, m: int, overlap: bool, out: t
                                _stream(stream)))
 
 
+def csa_compress_gated(x: torch.Tensor, W_kv: torch.Tensor, W_gate: torch.Tensor,
+                       ape: torch.Tensor, m: int, overlap: bool, out: torch.Tensor,
+                       out_row_scale: torch.Tensor | None = None, hadamard: bool = False,
+                       stream=None) -> None:
+    """x [B, n, d_in]; W_kv, W_gate [d_in, c*d_out]; ape [m, c*d_out] fp32
+    (c = 2 if overlap else 1) -> out [B, n//m, d_out] (+ scales for fp8)."""
+    B, n, d_in = x.shape
+    c = 2 if overlap else 1
+    d_out = W_kv.shape[1] // c
+    if ape.dtype != torch.float32:
+        raise ValueError("ape must be float32")
+    if tuple(W_gate.shape) != tuple(W_kv.shape) or tuple(ape.shape) != (m, c * d_out):
+        raise ValueError("W_kv, W_gate must be [d_in, c*d_out] and ape [m, c*d_out]")
+    _check(load().csa_compress_gated(_ptr(x), _dt(x), B, n, d_in, _ptr(W_kv), _ptr(W_gate),
+                                     _ptr(ape), d_out, m, int(bool(overlap)), _ptr(out),
+                                     _dt_rot(out, hadamard), _ptr(out_row_scale),
+                                     _stream(stream)))
+
+
 def csa_compress_append(x_new: torch.Tensor, W: torch.Tensor, m: int, overlap: bool,
                         pos: torch.Tensor, state: torch.Tensor, cache: torch.Tensor,
                         cache_scale: torch.Tensor | None = None,
@@ -240,6 +260,24 @@ def compress(x: torch.Tensor, W: torch.Tensor, m: int, overlap: bool, out_dtype=
         return out, scale
     out = torch.empty(B, N_c, W.shape[1], dtype=out_dtype, device=x.device)
     csa_compress(x, W, m, overlap, out, stream=stream)
+    return out
+
+
+def compress_gated(x, W_kv, W_gate, ape, m: int, overlap: bool, out_dtype=None,
+                   hadamard: bool = False, stream=None):
+    """Allocating form of csa_compress_gated: out (or (codes, scales) for fp8)."""
+    B, n, _ = x.shape
+    N_c = n // m
+    d_out = W_kv.shape[1] // (2 if overlap else 1)
+    out_dtype = x.dtype if out_dtype is None else out_dtype
+    if out_dtype in (torch.uint8, torch.float8_e4m3fn):
+        out = torch.empty(B, N_c, d_out, dtype=torch.uint8, device=x.device)
+        scale = torch.empty(B, N_c, dtype=torch.float32, device=x.device)
+        csa_compress_gated(x, W_kv, W_gate, ape, m, overlap, out, scale, hadamard=hadamard,
+                           stream=stream)
+        return out, scale
+    out = torch.empty(B, N_c, d_out, dtype=out_dtype, device=x.device)
+    csa_compress_gated(x, W_kv, W_gate, ape, m, overlap, out, stream=stream)
     return out
 
 

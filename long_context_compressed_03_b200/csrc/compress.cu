@@ -19,6 +19,7 @@
 //    quantisation (IEEE division, round to nearest even, saturating), for the
 //    Hadamard type after the warp rotates the row in shared memory.
 #include "common.cuh"
+#include "entry_epilogue.cuh"
 #include "kernels.h"
 
 namespace csa {
@@ -107,26 +108,8 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(CompressArgs a) {
     }
     __syncthreads();
 
-    const size_t row0 = (size_t)b * N_c + i0;
-    if constexpr (OUT == DT_E4M3 || OUT == DT_E4M3H) {
-        const int warp = tid >> 5, lane = tid & 31;
-        uint8_t* out = static_cast<uint8_t*>(a.out);
-        for (int e = warp; e < ne; e += kThreads / 32) {
-            if constexpr (OUT == DT_E4M3H) hadamard_row_warp(outs + e * d_out, d_out, a.hnorm);
-            float amax = 0.0f;
-            for (int o = lane; o < d_out; o += 32) amax = fmaxf(amax, fabsf(outs[e * d_out + o]));
-            for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
-            const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-            for (int o = lane; o < d_out; o += 32)
-                out[(row0 + e) * d_out + o] = e4m3_code(__fdiv_rn(outs[e * d_out + o], scale));
-            if (lane == 0) a.out_row_scale[row0 + e] = scale;
-        }
-    } else {
-        using Tout = typename std::conditional<OUT == DT_F32, float, __nv_bfloat16>::type;
-        Tout* out = static_cast<Tout*>(a.out);
-        for (int p = tid; p < ne * d_out; p += kThreads)
-            store_out<Tout>(out + row0 * d_out + p, outs[p]);
-    }
+    store_entry_rows<OUT, kThreads>(outs, ne, d_out, a.out, a.out_row_scale, (size_t)b * N_c + i0,
+                                    a.hnorm);
 }
 
 template <typename Tin, int OUT>

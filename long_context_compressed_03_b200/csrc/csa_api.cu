@@ -145,6 +145,39 @@ csa_status_t csa_compress(const void* x, int x_dt, int B, int n, int d_in, const
     return from_cuda(csa::launch_compress(a, static_cast<cudaStream_t>(stream), &why), "csa_compress", why);
 }
 
+csa_status_t csa_compress_gated(const void* x, int x_dt, int B, int n, int d_in, const void* W_kv,
+                                const void* W_gate, const float* ape, int d_out, int m, int overlap,
+                                void* out, int out_dt, float* out_row_scale, void* stream) {
+    REQUIRE(B >= 0 && n >= 0, "csa_compress_gated: negative B or n");
+    REQUIRE(m >= 1, "csa_compress_gated: m must be >= 1");
+    REQUIRE(overlap == 0 || overlap == 1, "csa_compress_gated: overlap must be 0 or 1");
+    REQUIRE(is_dt(x_dt) && is_dt(out_dt), "csa_compress_gated: unknown dtype");
+    REQUIRE(d_in > 0 && d_out > 0, "csa_compress_gated: d_in and d_out must be positive");
+    if (d_in % 16 || d_out % 16 || d_in > 256 || d_out > 256)
+        return fail(CSA_ERR_UNSUPPORTED, "csa_compress_gated: d_in, d_out must be multiples of 16 in [16, 256]");
+    if (is_fp8(x_dt)) return fail(CSA_ERR_UNSUPPORTED, "csa_compress_gated: fp8 input is not supported");
+    if (out_dt == CSA_DT_E4M3_HADAMARD && !pow2(d_out))
+        return fail(CSA_ERR_UNSUPPORTED, "csa_compress_gated: the Hadamard fp8 type needs d_out a power of two");
+    if (out_dt == CSA_DT_F32 && x_dt != CSA_DT_F32)
+        return fail(CSA_ERR_UNSUPPORTED, "csa_compress_gated: F32 output needs F32 input");
+    REQUIRE(is_fp8(out_dt) == (out_row_scale != nullptr),
+            "csa_compress_gated: out_row_scale is required for E4M3 output and must be NULL otherwise");
+    const int N_c = n / m;
+    if ((long)B * N_c == 0) return ok();
+    REQUIRE(x && W_kv && W_gate && ape && out, "csa_compress_gated: null tensor pointer");
+    REQUIRE_ALIGNED(x, "x");
+    REQUIRE_ALIGNED(W_kv, "W_kv");
+    REQUIRE_ALIGNED(W_gate, "W_gate");
+    REQUIRE_ALIGNED(ape, "ape");
+    REQUIRE_ALIGNED(out, "out");
+    REQUIRE_ALIGNED(out_row_scale, "out_row_scale");
+    csa::GatedArgs a{x, x_dt, B, n, d_in, W_kv, W_gate, ape, d_out, m, overlap, out, out_dt,
+                     out_row_scale, N_c, hadamard_norm(d_out)};
+    const char* why = nullptr;
+    return from_cuda(csa::launch_compress_gated(a, static_cast<cudaStream_t>(stream), &why),
+                     "csa_compress_gated", why);
+}
+
 csa_status_t csa_compress_append(const void* x_new, int x_dt, int B, int d_in, const void* W,
                                  int d_out, int m, int overlap, const int* pos, float* state,
                                  void* cache, int out_dt, float* cache_scale, int N_cap,

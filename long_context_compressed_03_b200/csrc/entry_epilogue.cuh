@@ -1,0 +1,41 @@
+// entry_epilogue.cuh -- the store of compressed entries (stage 1), shared by
+// the mean-pool and the gated compressors.
+//
+// rows[e][0 .. d_out) (fp32, shared memory) are written as entry row0 + e of
+// the output: fp32 / bf16 stores, or one E4M3 row with scale = amax/448
+// (1 for a zero row), code = E4M3(v / scale) by IEEE division, nearest even,
+// saturating -- after a Walsh-Hadamard rotation of the row for the rotated
+// type.  Every thread of the CTA calls it; warps take rows in turn.
+#pragma once
+
+#include <type_traits>
+
+#include "common.cuh"
+
+namespace csa {
+
+template <int OUT, int kThreads>
+__device__ __forceinline__ void store_entry_rows(float* rows, int ne, int d_out, void* out_v,
+                                                 float* row_scale, size_t row0, float hnorm) {
+    const int tid = threadIdx.x;
+    if constexpr (OUT == DT_E4M3 || OUT == DT_E4M3H) {
+        const int warp = tid >> 5, lane = tid & 31;
+        uint8_t* out = static_cast<uint8_t*>(out_v);
+        for (int e = warp; e < ne; e += kThreads / 32) {
+            if constexpr (OUT == DT_E4M3H) hadamard_row_warp(rows + e * d_out, d_out, hnorm);
+            float amax = 0.0f;
+            for (int o = lane; o < d_out; o += 32) amax = fmaxf(amax, fabsf(rows[e * d_out + o]));
+            for (int off = 16; off; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+            const float scale = amax > 0.0f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+            for (int o = lane; o < d_out; o += 32)
+                out[(row0 + e) * d_out + o] = e4m3_code(__fdiv_rn(rows[e * d_out + o], scale));
+            if (lane == 0) row_scale[row0 + e] = scale;
+        }
+    } else {
+        using Tout = typename std::conditional<OUT == DT_F32, float, __nv_bfloat16>::type;
+        Tout* out = static_cast<Tout*>(out_v);
+        for (int p = tid; p < ne * d_out; p += kThreads) store_out<Tout>(out + row0 * d_out + p, rows[p]);
+    }
+}
+
+}  // namespace csa

@@ -16,6 +16,19 @@ struct CompressArgs {
     float hnorm;               // fp32(1/sqrt(d_out)) for the Hadamard fp8 type
 };
 
+struct GatedArgs {
+    const void* x; int x_dt;
+    int B, n, d_in;
+    const void* W_kv;          // [d_in, c*d_out], x_dt
+    const void* W_gate;        // [d_in, c*d_out], x_dt
+    const float* ape;          // [m, c*d_out]
+    int d_out, m, overlap;     // c = 2 if overlap else 1
+    void* out; int out_dt;
+    float* out_row_scale;
+    int N_c;
+    float hnorm;
+};
+
 struct AppendArgs {
     const void* x; int x_dt;
     int B, d_in;
@@ -85,6 +98,7 @@ void count_launch();
 // reason string when the configuration is unsupported (returned as
 // cudaErrorNotSupported).
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s, const char** why);
+cudaError_t launch_compress_gated(const GatedArgs& a, cudaStream_t s, const char** why);
 cudaError_t launch_compress_append(const AppendArgs& a, cudaStream_t s, const char** why);
 cudaError_t launch_indexer_topk(const IndexerArgs& a, cudaStream_t s, const char** why);
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s, const char** why);

@@ -224,6 +224,27 @@ def hca_prefill_inputs(w: Workload, seed: int = 0, n: int | None = None, B: int 
     return dict(q=q.to(dt), kv=kv.to(dt), W_c=W_c.to(dt))
 
 
+def indexer_variant_inputs(B: int, n: int, H_I: int, seed: int = 0):
+    """Gate weights for the gated indexer: w [B, n, H_I] ~ N(0, 1) (any sign;
+    the pages give no distribution)."""
+    g = torch.Generator().manual_seed(seed)
+    return dict(qI_weight=_randn(g, (B, n, H_I)))
+
+
+def gated_compressor_weights(d_in: int, d_out: int, m: int, overlap: bool, dtype="bf16",
+                             seed: int = 0):
+    """Weights of the gated-softmax compressor.  Draw order: W_kv, W_gate
+    [d_in, c*d_out] ~ N(0, 1/d_in), ape [m, c*d_out] ~ N(0, 1) (fp32);
+    c = 2 if overlap else 1."""
+    c = 2 if overlap else 1
+    g = torch.Generator().manual_seed(seed)
+    W_kv = _randn(g, (d_in, c * d_out), 1.0 / math.sqrt(d_in))
+    W_gate = _randn(g, (d_in, c * d_out), 1.0 / math.sqrt(d_in))
+    ape = _randn(g, (m, c * d_out))
+    dt = torch_dtype(dtype)
+    return dict(W_kv=W_kv.to(dt), W_gate=W_gate.to(dt), ape=ape)
+
+
 def query_sample(n: int, m: int, window: int, count: int, seed: int = 1) -> torch.Tensor:
     """A fixed, seeded subset of query positions for sampled checks at full
     size: positions 0..m, the block boundaries around the first few entries,

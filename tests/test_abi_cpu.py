@@ -84,6 +84,28 @@ def test_compress_validation(lib):
     assert f(None, 1, 0, 64, 128, None, 128, 4, 1, None, 1, None, None) == api.CSA_OK
 
 
+def test_compress_gated_validation(lib):
+    f = lib.csa_compress_gated
+    #       x   dt B  n   d_in Wkv  Wg   ape  d_out m  ov out  dt scale stream
+    args = [FAKE, 1, 1, 64, 64, FAKE, FAKE, FAKE, 64, 4, 1, FAKE, 1, None, None]
+    bad = list(args); bad[9] = 0                       # m = 0
+    assert f(*bad) == api.CSA_ERR_INVALID_ARG
+    bad = list(args); bad[8] = 40                      # d_out not a multiple of 16
+    assert f(*bad) == api.CSA_ERR_UNSUPPORTED
+    bad = list(args); bad[7] = None                    # no APE
+    assert f(*bad) == api.CSA_ERR_INVALID_ARG
+    bad = list(args); bad[12] = 2                      # fp8 output without scales
+    assert f(*bad) == api.CSA_ERR_INVALID_ARG
+    bad = list(args); bad[1] = 2                       # fp8 input
+    assert f(*bad) == api.CSA_ERR_UNSUPPORTED
+    bad = list(args); bad[6] = ODD                     # misaligned gate weights
+    assert f(*bad) == api.CSA_ERR_MISALIGNED
+    bad = list(args); bad[12] = 0                      # F32 output from BF16 input
+    assert f(*bad) == api.CSA_ERR_UNSUPPORTED
+    ok = list(args); ok[3] = 3                         # n < m: no entries, no-op
+    assert f(*ok) == api.CSA_OK
+
+
 def test_compress_append_validation(lib):
     f = lib.csa_compress_append
     #       x_new dt B  d_in W    d_out m  ov pos   state cache dt scale N_cap n_ent stream

@@ -103,6 +103,64 @@ def test_compress_hadamard_fp8_matches_rotated_oracle(case):
     assert max_abs(back, unrot) <= 0.1 * np.abs(unrot).max()
 
 
+GATED_CASES = [
+    # (B, n, d_in, d_out, m, overlap, x dtype, out kind)
+    (2, 1003, 64, 64, 4, True, torch.bfloat16, "bf16"),         # ratio 4, overlapping, ragged tail
+    (1, 700, 128, 128, 4, True, torch.float32, "f32"),
+    (1, 128 * 5 + 77, 128, 128, 128, False, torch.bfloat16, "bf16"),   # ratio 128: windows span steps
+    (2, 300, 32, 48, 4, True, torch.bfloat16, "e4m3"),          # a half slice (48 = 32 + 16), fp8 out
+    (1, 260, 64, 64, 4, True, torch.bfloat16, "e4m3_rot"),
+    (1, 130, 16, 16, 1, True, torch.float32, "f32"),            # m = 1: 63 entries per CTA
+    (1, 500, 16, 32, 64, True, torch.bfloat16, "bf16"),         # m = 64 overlapping: 128 positions
+    (3, 37, 16, 16, 4, False, torch.float32, "f32"),
+]
+
+
+@pytest.mark.parametrize("case", GATED_CASES)
+def test_compress_gated_matches_oracle(case):
+    B, n, d_in, d_out, m, overlap, dt, kind = case
+    c = 2 if overlap else 1
+    g = _gen(300 + n + m)
+    x = _randn(g, B, n, d_in, dtype=dt)
+    W_kv = _randn(g, d_in, c * d_out, dtype=dt, std=1 / math.sqrt(d_in))
+    W_g = _randn(g, d_in, c * d_out, dtype=dt, std=2 / math.sqrt(d_in))
+    ape = _randn(g, m, c * d_out)
+    ref = oracle.compress_gated(np64(x), np64(W_kv), np64(W_g), np64(ape), m, overlap)
+    args = (x.to(DEV), W_kv.to(DEV), W_g.to(DEV), ape.to(DEV), m, overlap)
+    if kind in ("e4m3", "e4m3_rot"):
+        rot = kind == "e4m3_rot"
+        if rot:
+            ref = ref @ _hadamard64(d_out)
+        codes, scale = api.compress_gated(*args, out_dtype=torch.uint8, hadamard=rot)
+        codes, scale = codes.cpu().numpy(), scale.cpu().numpy()
+        deq = oracle.dequantize_rows_e4m3(codes, scale)
+        np.testing.assert_allclose(scale, np.abs(ref).max(axis=-1) / 448.0, rtol=1e-5)
+        assert np.all(np.abs(deq - ref) <= np.abs(ref) * 2.0 ** -3 + scale[..., None] * 2.0 ** -9)
+        return
+    out_dt = torch.float32 if kind == "f32" else torch.bfloat16
+    out = api.compress_gated(*args, out_dtype=out_dt)
+    torch.cuda.synchronize()
+    got = np64(out)
+    assert got.shape == ref.shape
+    if kind == "f32":
+        assert max_abs(got, ref) <= ATOL_F32
+    else:
+        assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-5)
+
+
+def test_compress_gated_flat_gates_equal_the_mean_pool_kernel():
+    """Zero gate weights, constant APE and W_kv = [W | W]: the two compressors
+    of this library agree (uniform softmax = mean, and the projection is linear)."""
+    g = _gen(9)
+    B, n, d, m = 2, 515, 64, 4
+    x = _randn(g, B, n, d).to(DEV)
+    W = _randn(g, d, d, std=1 / math.sqrt(d)).to(DEV)
+    gated = api.compress_gated(x, torch.cat([W, W], 1), torch.zeros(d, 2 * d, device=DEV),
+                               torch.full((m, 2 * d), 0.3, device=DEV), m, True)
+    mean = api.compress(x, W, m, True)
+    assert torch.allclose(gated, mean, atol=2e-5, rtol=1e-5)
+
+
 def test_compress_no_entries_is_a_noop():
     x = torch.zeros(1, 3, 16, device=DEV, dtype=torch.bfloat16)
     W = torch.zeros(16, 16, device=DEV, dtype=torch.bfloat16)
