@@ -269,6 +269,52 @@ csa_status_t hca_dense_attn(const void* q, int dt, int B, int n_q, int H, int D,
                             const int* raw_len, int window, const int* q_pos,
                             float softmax_scale, void* out, float* lse_out, void* stream);
 
+/*
+ * Paged caches (serving layout).  The _paged entry points below take the
+ * compressed caches as a pool of fixed-size pages instead of one [B, N_cap, *]
+ * block per element:
+ *   pool          [num_pages, page_size, row]   (kv_c rows, or indexer-key rows,
+ *                 with the per-row fp32 scales as a pool [num_pages, page_size])
+ *   block_table   device int32 [B, max_pages]: logical entry s of element b
+ *                 lives at row s mod page_size of page block_table[b][s / page_size].
+ *   page_size     a power of two in [1, 2^20]; the logical capacity is
+ *                 N_cap = max_pages * page_size (at most 2^30).
+ * A page id outside [0, num_pages) marks a page that is not there: its entries
+ * are never read or written (attention skips them like padding, the indexer
+ * scores them as zero rows, append drops the write).  Every other argument,
+ * the arithmetic and the results are those of the unpaged entry point of the
+ * same name; paged calls are served by the decode kernels (cluster-split and
+ * SIMT), not the prefill tensor-core kernels.  These calls are this library's
+ * serving layout, not a step the pages describe (they name paged KV pools for
+ * serving, "百万上下文从「奢侈品」变「日用品」…" §8.3).
+ */
+csa_status_t csa_compress_append_paged(const void* x_new, int x_dt, int B, int d_in, const void* W,
+                                       int d_out, int m, int overlap, const int* pos, float* state,
+                                       void* cache_pages, int out_dt, float* cache_scale_pages,
+                                       const int* block_table, int max_pages, int page_size,
+                                       int num_pages, int* n_entries, void* stream);
+
+csa_status_t csa_indexer_topk_paged(const void* qI, int qI_dt, const float* qI_scale,
+                                    const float* qI_weight, const void* kI_pages, int kI_dt,
+                                    const float* kI_scale_pages, const int* block_table,
+                                    int max_pages, int page_size, int num_pages, int B, int n_q,
+                                    int H_I, int d_I, const int* n_entries, const int* q_pos,
+                                    int m, int topk, int* idx_out, void* stream);
+
+csa_status_t csa_sparse_attn_paged(const void* q, int dt, int B, int n_q, int H, int D,
+                                   const void* kv_c_pages, const int* block_table, int max_pages,
+                                   int page_size, int num_pages, const int* idx, int topk,
+                                   const void* kv_raw, int L_raw, const int* raw_pos0,
+                                   const int* raw_len, int window, const int* q_pos,
+                                   float softmax_scale, void* out, float* lse_out, void* stream);
+
+csa_status_t hca_dense_attn_paged(const void* q, int dt, int B, int n_q, int H, int D,
+                                  const void* kv_c_pages, const int* block_table, int max_pages,
+                                  int page_size, int num_pages, const int* n_entries, int m,
+                                  const void* kv_raw, int L_raw, const int* raw_pos0,
+                                  const int* raw_len, int window, const int* q_pos,
+                                  float softmax_scale, void* out, float* lse_out, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -40,6 +40,12 @@ SIGNATURES = {
     "csa_indexer_topk": (I, [P, I, P, P, P, I, P, I, I, I, I, I, P, P, I, I, P, P]),
     "csa_sparse_attn": (I, [P, I, I, I, I, I, P, I, P, I, P, I, P, P, I, P, F, P, P, P]),
     "hca_dense_attn": (I, [P, I, I, I, I, I, P, I, P, I, P, I, P, P, I, P, F, P, P, P]),
+    "csa_compress_append_paged": (I, [P, I, I, I, P, I, I, I, P, P, P, I, P, P, I, I, I, P, P]),
+    "csa_indexer_topk_paged": (I, [P, I, P, P, P, I, P, P, I, I, I, I, I, I, I, P, P, I, I, P, P]),
+    "csa_sparse_attn_paged": (I, [P, I, I, I, I, I, P, P, I, I, I, P, I, P, I, P, P, I, P, F, P, P,
+                                  P]),
+    "hca_dense_attn_paged": (I, [P, I, I, I, I, I, P, P, I, I, I, P, I, P, I, P, P, I, P, F, P, P,
+                                 P]),
 }
 
 
@@ -244,6 +250,83 @@ def hca_dense_attn(q: torch.Tensor, kv_c: torch.Tensor, m: int, kv_raw: torch.Te
                                  _i32(raw_pos0, "raw_pos0"), _i32(raw_len, "raw_len"), window,
                                  _i32(q_pos, "q_pos"), float(softmax_scale), _ptr(out),
                                  _ptr(lse_out), _stream(stream)))
+
+
+# ---------------------------------------------------------------- paged caches
+class PagedCache:
+    """A page pool and its block table: ``pool`` [num_pages, page_size, row...]
+    (and ``scale`` [num_pages, page_size] for fp8 rows), ``block_table``
+    [B, max_pages] int32 (ids outside [0, num_pages) mark absent pages)."""
+
+    def __init__(self, pool: torch.Tensor, block_table: torch.Tensor,
+                 scale: torch.Tensor | None = None):
+        if pool.dim() < 3:
+            raise ValueError("pool must be [num_pages, page_size, row...]")
+        self.pool, self.block_table, self.scale = pool, block_table, scale
+        self.num_pages, self.page_size = pool.shape[0], pool.shape[1]
+        self.max_pages = block_table.shape[1]
+
+    @property
+    def args(self):
+        return (_i32(self.block_table, "block_table"), self.max_pages, self.page_size,
+                self.num_pages)
+
+
+def csa_compress_append_paged(x_new: torch.Tensor, W: torch.Tensor, m: int, overlap: bool,
+                              pos: torch.Tensor, state: torch.Tensor, cache: PagedCache,
+                              n_entries: torch.Tensor | None = None, hadamard: bool = False,
+                              stream=None) -> None:
+    """csa_compress_append into a paged cache (entry j of element b goes to its page)."""
+    B, d_in = x_new.shape
+    d_out = W.shape[1]
+    if state.dtype != torch.float32:
+        raise ValueError("state must be float32")
+    _check(load().csa_compress_append_paged(
+        _ptr(x_new), _dt(x_new), B, d_in, _ptr(W), d_out, m, int(bool(overlap)),
+        _i32(pos, "pos"), _ptr(state), _ptr(cache.pool), _dt_rot(cache.pool, hadamard),
+        _ptr(cache.scale), *cache.args, _i32(n_entries, "n_entries"), _stream(stream)))
+
+
+def csa_indexer_topk_paged(qI: torch.Tensor, kI: PagedCache, m: int, topk: int,
+                           idx_out: torch.Tensor, qI_scale: torch.Tensor | None = None,
+                           n_entries: torch.Tensor | None = None, q_pos: torch.Tensor | None = None,
+                           kI_rotated: bool = False, qI_weight: torch.Tensor | None = None,
+                           stream=None) -> None:
+    """csa_indexer_topk over a paged indexer-key cache (kI.scale: fp8 row scales)."""
+    B, n_q, H_I, d_I = qI.shape
+    _check(load().csa_indexer_topk_paged(
+        _ptr(qI), _dt(qI), _ptr(qI_scale), _ptr(qI_weight), _ptr(kI.pool),
+        _dt_rot(kI.pool, kI_rotated), _ptr(kI.scale), *kI.args, B, n_q, H_I, d_I,
+        _i32(n_entries, "n_entries"), _i32(q_pos, "q_pos"), m, topk, _i32(idx_out, "idx_out"),
+        _stream(stream)))
+
+
+def csa_sparse_attn_paged(q: torch.Tensor, kv_c: PagedCache, idx: torch.Tensor | None,
+                          kv_raw: torch.Tensor, window: int, out: torch.Tensor,
+                          lse_out: torch.Tensor | None = None, raw_pos0: torch.Tensor | None = None,
+                          raw_len: torch.Tensor | None = None, q_pos: torch.Tensor | None = None,
+                          softmax_scale: float = 0.0, stream=None) -> None:
+    B, n_q, H, D = q.shape
+    topk = 0 if idx is None else idx.shape[-1]
+    _check(load().csa_sparse_attn_paged(
+        _ptr(q), _dt(q), B, n_q, H, D, _ptr(kv_c.pool), *kv_c.args, _i32(idx, "idx"), topk,
+        _ptr(kv_raw), kv_raw.shape[1], _i32(raw_pos0, "raw_pos0"), _i32(raw_len, "raw_len"),
+        window, _i32(q_pos, "q_pos"), float(softmax_scale), _ptr(out), _ptr(lse_out),
+        _stream(stream)))
+
+
+def hca_dense_attn_paged(q: torch.Tensor, kv_c: PagedCache, m: int, kv_raw: torch.Tensor,
+                         window: int, out: torch.Tensor, lse_out: torch.Tensor | None = None,
+                         n_entries: torch.Tensor | None = None,
+                         raw_pos0: torch.Tensor | None = None, raw_len: torch.Tensor | None = None,
+                         q_pos: torch.Tensor | None = None, softmax_scale: float = 0.0,
+                         stream=None) -> None:
+    B, n_q, H, D = q.shape
+    _check(load().hca_dense_attn_paged(
+        _ptr(q), _dt(q), B, n_q, H, D, _ptr(kv_c.pool), *kv_c.args, _i32(n_entries, "n_entries"),
+        m, _ptr(kv_raw), kv_raw.shape[1], _i32(raw_pos0, "raw_pos0"), _i32(raw_len, "raw_len"),
+        window, _i32(q_pos, "q_pos"), float(softmax_scale), _ptr(out), _ptr(lse_out),
+        _stream(stream)))
 
 
 # ---------------------------------------------------------------- allocating wrappers

@@ -46,7 +46,7 @@ __global__ void __launch_bounds__(kThreads) attn_generic_kernel(AttnArgs a) {
     const int total = rk.n_comp + rk.n_win;
 
     const T* q = static_cast<const T*>(a.q) + (size_t)row * H * D;
-    const T* kvc = static_cast<const T*>(a.kv_c) + (size_t)b * a.N_cap * D;
+    const T* kvc = static_cast<const T*>(a.kv_c);          // rows from cache_row()
     const T* kvr = static_cast<const T*>(a.kv_raw) + (size_t)b * a.L_raw * D;
     const float qscale = a.scale * kLog2e;
     for (int p = threadIdx.x; p < H * D; p += kThreads) {
@@ -67,7 +67,10 @@ __global__ void __launch_bounds__(kThreads) attn_generic_kernel(AttnArgs a) {
             const T* ptr = nullptr;
             if (kk < rk.n_comp) {
                 const int s = a.dense ? kk : a.idx[(size_t)row * a.topk + kk];
-                if (s >= 0 && s < a.N_cap) ptr = kvc + (size_t)s * D;
+                if (s >= 0 && s < a.N_cap) {
+                    const long r = cache_row(a.pages, a.N_cap, b, s);
+                    if (r >= 0) ptr = kvc + (size_t)r * D;
+                }
             } else if (kk < total) {
                 ptr = kvr + (size_t)(rk.win_lo + kk - rk.n_comp) * D;
             }
@@ -165,7 +168,7 @@ cudaError_t launch_dims(const AttnArgs& a, cudaStream_t s, const char** why) {
 
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s, const char** why) {
     if (a.B <= 0 || a.n_q <= 0) return cudaSuccess;
-    if (attention_tc_supported(a)) {
+    if (a.pages.bt == nullptr && attention_tc_supported(a)) {   // paged caches: decode kernels
         uint32_t* err = device_error_word();
         if (!err) return cudaErrorUnknown;
         return launch_attention_tc(a, err, s);

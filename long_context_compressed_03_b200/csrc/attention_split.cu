@@ -130,10 +130,11 @@ __global__ void __launch_bounds__(H * 2, min_blocks<H>()) attn_split_kernel(Attn
     const int g = lane >> 2, tq = lane & 3;
 
     using T16 = __nv_bfloat16;
-    const T16* kvc = static_cast<const T16*>(a.kv_c) + (size_t)b * a.N_cap * D;
+    const T16* kvc = static_cast<const T16*>(a.kv_c);         // rows from cache_row()
     const T16* kvr = static_cast<const T16*>(a.kv_raw) + (size_t)b * a.L_raw * D;
 
-    // ---- row codes: >= 0 compressed entry, <= -2 raw row -(code + 2), -1 none
+    // ---- row codes: >= 0 physical row of a compressed entry, <= -2 raw row
+    //      -(code + 2), -1 none
     for (int i0 = 0; i0 < ntile * kBN; i0 += kThreads) {
         const int i = i0 + tid;
         const int kk = lo + i;
@@ -141,7 +142,7 @@ __global__ void __launch_bounds__(H * 2, min_blocks<H>()) attn_split_kernel(Attn
         if (i < ntile * kBN && kk < hi) {
             if (kk < rk.n_comp) {
                 const int s = a.dense ? kk : a.idx[(size_t)row * a.topk + kk];
-                code = (s >= 0 && s < a.N_cap) ? s : -1;
+                code = (s >= 0 && s < a.N_cap) ? (int)cache_row(a.pages, a.N_cap, b, s) : -1;
             } else {
                 code = -(rk.win_lo + kk - rk.n_comp) - 2;
             }

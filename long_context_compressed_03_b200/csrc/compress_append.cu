@@ -48,6 +48,8 @@ __global__ void __launch_bounds__(kThreads) compress_append_kernel(AppendArgs a)
         }
     }
     if (!complete || j >= a.N_cap) return;              // uniform across the CTA
+    const long crow = cache_row(a.pages, a.N_cap, b, j);
+    if (crow < 0) return;                               // page outside the pool: not written
     __syncthreads();
     const Tin* W = static_cast<const Tin*>(a.W);
     for (int o = tid; o < d_out; o += kThreads) {
@@ -56,7 +58,7 @@ __global__ void __launch_bounds__(kThreads) compress_append_kernel(AppendArgs a)
         outs[o] = acc;
     }
     __syncthreads();
-    const size_t row = (size_t)b * a.N_cap + j;
+    const size_t row = (size_t)crow;
     if constexpr (OUT == DT_E4M3 || OUT == DT_E4M3H) {
         if constexpr (OUT == DT_E4M3H) {
             if (tid < 32) hadamard_row_warp(outs, d_out, a.hnorm);

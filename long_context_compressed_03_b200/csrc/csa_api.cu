@@ -178,10 +178,10 @@ csa_status_t csa_compress_gated(const void* x, int x_dt, int B, int n, int d_in,
                      "csa_compress_gated", why);
 }
 
-csa_status_t csa_compress_append(const void* x_new, int x_dt, int B, int d_in, const void* W,
-                                 int d_out, int m, int overlap, const int* pos, float* state,
-                                 void* cache, int out_dt, float* cache_scale, int N_cap,
-                                 int* n_entries, void* stream) {
+static csa_status_t compress_append_impl(const void* x_new, int x_dt, int B, int d_in, const void* W,
+                                         int d_out, int m, int overlap, const int* pos, float* state,
+                                         void* cache, int out_dt, float* cache_scale, int N_cap,
+                                         int* n_entries, const csa::PageMap& pm, void* stream) {
     REQUIRE(B >= 0 && N_cap >= 0, "csa_compress_append: negative B or N_cap");
     REQUIRE(m >= 1, "csa_compress_append: m must be >= 1");
     REQUIRE(overlap == 0 || overlap == 1, "csa_compress_append: overlap must be 0 or 1");
@@ -205,16 +205,17 @@ csa_status_t csa_compress_append(const void* x_new, int x_dt, int B, int d_in, c
     REQUIRE_ALIGNED(cache, "cache");
     REQUIRE_ALIGNED(cache_scale, "cache_scale");
     csa::AppendArgs a{x_new, x_dt, B, d_in, W, d_out, m, overlap, pos, state, cache, out_dt,
-                      cache_scale, N_cap, n_entries, hadamard_norm(d_out)};
+                      cache_scale, N_cap, n_entries, hadamard_norm(d_out), pm};
     const char* why = nullptr;
     return from_cuda(csa::launch_compress_append(a, static_cast<cudaStream_t>(stream), &why),
                      "csa_compress_append", why);
 }
 
-csa_status_t csa_indexer_topk(const void* qI, int qI_dt, const float* qI_scale,
-                              const float* qI_weight, const void* kI, int kI_dt, const float* kI_scale, int B, int n_q, int H_I, int d_I,
-                              int N_cap, const int* n_entries, const int* q_pos, int m, int topk,
-                              int* idx_out, void* stream) {
+static csa_status_t indexer_impl(const void* qI, int qI_dt, const float* qI_scale,
+                                 const float* qI_weight, const void* kI, int kI_dt,
+                                 const float* kI_scale, int B, int n_q, int H_I, int d_I, int N_cap,
+                                 const int* n_entries, const int* q_pos, int m, int topk,
+                                 int* idx_out, const csa::PageMap& pm, void* stream) {
     REQUIRE(B >= 0 && n_q >= 0 && N_cap >= 0, "csa_indexer_topk: negative size");
     REQUIRE(H_I >= 1 && d_I >= 1, "csa_indexer_topk: H_I and d_I must be positive");
     REQUIRE(m >= 1, "csa_indexer_topk: m must be >= 1");
@@ -241,10 +242,77 @@ csa_status_t csa_indexer_topk(const void* qI, int qI_dt, const float* qI_scale,
     REQUIRE_ALIGNED(n_entries, "n_entries");
     REQUIRE_ALIGNED(q_pos, "q_pos");
     csa::IndexerArgs a{qI, qI_dt, qI_scale, kI, kI_dt, kI_scale, B, n_q, H_I, d_I, N_cap,
-                       n_entries, q_pos, m, topk, idx_out, hadamard_norm(d_I), qI_weight};
+                       n_entries, q_pos, m, topk, idx_out, hadamard_norm(d_I), qI_weight, pm};
     const char* why = nullptr;
     return from_cuda(csa::launch_indexer_topk(a, static_cast<cudaStream_t>(stream), &why),
                      "csa_indexer_topk", why);
+}
+
+// The page map of a paged entry point (validated), or an error status.
+static csa_status_t page_map(const char* name, int B, const int* block_table, int max_pages,
+                             int page_size, int num_pages, csa::PageMap* pm, int* N_cap) {
+    REQUIRE(max_pages >= 0 && num_pages >= 0, "%s: negative max_pages or num_pages", name);
+    REQUIRE(page_size >= 1 && page_size <= (1 << 20) && pow2(page_size),
+            "%s: page_size must be a power of two in [1, 2^20]", name);
+    REQUIRE((long)max_pages * page_size <= (1L << 30), "%s: max_pages * page_size above 2^30", name);
+    REQUIRE((long)num_pages * page_size <= (1L << 31) - 1, "%s: page pool above 2^31 - 1 rows", name);
+    REQUIRE(block_table || B == 0 || max_pages == 0, "%s: null block_table", name);
+    REQUIRE_ALIGNED(block_table, "block_table");
+    int shift = 0;
+    while ((1 << shift) < page_size) ++shift;
+    pm->bt = block_table;
+    pm->max_pages = max_pages;
+    pm->page_shift = shift;
+    pm->num_pages = num_pages;
+    *N_cap = max_pages * page_size;
+    return ok();
+}
+
+csa_status_t csa_compress_append(const void* x_new, int x_dt, int B, int d_in, const void* W,
+                                 int d_out, int m, int overlap, const int* pos, float* state,
+                                 void* cache, int out_dt, float* cache_scale, int N_cap,
+                                 int* n_entries, void* stream) {
+    return compress_append_impl(x_new, x_dt, B, d_in, W, d_out, m, overlap, pos, state, cache,
+                                out_dt, cache_scale, N_cap, n_entries, csa::PageMap{}, stream);
+}
+
+csa_status_t csa_compress_append_paged(const void* x_new, int x_dt, int B, int d_in, const void* W,
+                                       int d_out, int m, int overlap, const int* pos, float* state,
+                                       void* cache_pages, int out_dt, float* cache_scale_pages,
+                                       const int* block_table, int max_pages, int page_size,
+                                       int num_pages, int* n_entries, void* stream) {
+    csa::PageMap pm;
+    int N_cap = 0;
+    const csa_status_t st = page_map("csa_compress_append_paged", B, block_table, max_pages,
+                                     page_size, num_pages, &pm, &N_cap);
+    if (st != CSA_OK) return st;
+    return compress_append_impl(x_new, x_dt, B, d_in, W, d_out, m, overlap, pos, state,
+                                cache_pages, out_dt, cache_scale_pages, N_cap, n_entries, pm,
+                                stream);
+}
+
+csa_status_t csa_indexer_topk(const void* qI, int qI_dt, const float* qI_scale,
+                              const float* qI_weight, const void* kI, int kI_dt,
+                              const float* kI_scale, int B, int n_q, int H_I, int d_I, int N_cap,
+                              const int* n_entries, const int* q_pos, int m, int topk,
+                              int* idx_out, void* stream) {
+    return indexer_impl(qI, qI_dt, qI_scale, qI_weight, kI, kI_dt, kI_scale, B, n_q, H_I, d_I,
+                        N_cap, n_entries, q_pos, m, topk, idx_out, csa::PageMap{}, stream);
+}
+
+csa_status_t csa_indexer_topk_paged(const void* qI, int qI_dt, const float* qI_scale,
+                                    const float* qI_weight, const void* kI_pages, int kI_dt,
+                                    const float* kI_scale_pages, const int* block_table,
+                                    int max_pages, int page_size, int num_pages, int B, int n_q,
+                                    int H_I, int d_I, const int* n_entries, const int* q_pos,
+                                    int m, int topk, int* idx_out, void* stream) {
+    csa::PageMap pm;
+    int N_cap = 0;
+    const csa_status_t st = page_map("csa_indexer_topk_paged", B, block_table, max_pages,
+                                     page_size, num_pages, &pm, &N_cap);
+    if (st != CSA_OK) return st;
+    return indexer_impl(qI, qI_dt, qI_scale, qI_weight, kI_pages, kI_dt, kI_scale_pages, B, n_q,
+                        H_I, d_I, N_cap, n_entries, q_pos, m, topk, idx_out, pm, stream);
 }
 
 static csa_status_t attention_common(const char* name, csa::AttnArgs& a, void* stream) {
@@ -285,6 +353,24 @@ csa_status_t csa_sparse_attn(const void* q, int dt, int B, int n_q, int H, int D
     return attention_common("csa_sparse_attn", a, stream);
 }
 
+csa_status_t csa_sparse_attn_paged(const void* q, int dt, int B, int n_q, int H, int D,
+                                   const void* kv_c_pages, const int* block_table, int max_pages,
+                                   int page_size, int num_pages, const int* idx, int topk,
+                                   const void* kv_raw, int L_raw, const int* raw_pos0,
+                                   const int* raw_len, int window, const int* q_pos,
+                                   float softmax_scale, void* out, float* lse_out, void* stream) {
+    REQUIRE(topk >= 0 && topk <= 2048, "csa_sparse_attn_paged: topk must be in [0, 2048]");
+    REQUIRE(idx || topk == 0 || (long)B * n_q == 0, "csa_sparse_attn_paged: null idx");
+    csa::PageMap pm;
+    int N_cap = 0;
+    const csa_status_t st = page_map("csa_sparse_attn_paged", B, block_table, max_pages, page_size,
+                                     num_pages, &pm, &N_cap);
+    if (st != CSA_OK) return st;
+    csa::AttnArgs a{q, dt, B, n_q, H, D, kv_c_pages, N_cap, idx, topk, nullptr, 1, 0, kv_raw,
+                    L_raw, raw_pos0, raw_len, window, q_pos, softmax_scale, out, lse_out, pm};
+    return attention_common("csa_sparse_attn_paged", a, stream);
+}
+
 csa_status_t hca_dense_attn(const void* q, int dt, int B, int n_q, int H, int D,
                             const void* kv_c, int N_cap, const int* n_entries, int m,
                             const void* kv_raw, int L_raw, const int* raw_pos0,
@@ -294,6 +380,23 @@ csa_status_t hca_dense_attn(const void* q, int dt, int B, int n_q, int H, int D,
     csa::AttnArgs a{q, dt, B, n_q, H, D, kv_c, N_cap, nullptr, 0, n_entries, m, 1, kv_raw, L_raw,
                     raw_pos0, raw_len, window, q_pos, softmax_scale, out, lse_out};
     return attention_common("hca_dense_attn", a, stream);
+}
+
+csa_status_t hca_dense_attn_paged(const void* q, int dt, int B, int n_q, int H, int D,
+                                  const void* kv_c_pages, const int* block_table, int max_pages,
+                                  int page_size, int num_pages, const int* n_entries, int m,
+                                  const void* kv_raw, int L_raw, const int* raw_pos0,
+                                  const int* raw_len, int window, const int* q_pos,
+                                  float softmax_scale, void* out, float* lse_out, void* stream) {
+    REQUIRE(m >= 1, "hca_dense_attn_paged: m must be >= 1");
+    csa::PageMap pm;
+    int N_cap = 0;
+    const csa_status_t st = page_map("hca_dense_attn_paged", B, block_table, max_pages, page_size,
+                                     num_pages, &pm, &N_cap);
+    if (st != CSA_OK) return st;
+    csa::AttnArgs a{q, dt, B, n_q, H, D, kv_c_pages, N_cap, nullptr, 0, n_entries, m, 1, kv_raw,
+                    L_raw, raw_pos0, raw_len, window, q_pos, softmax_scale, out, lse_out, pm};
+    return attention_common("hca_dense_attn_paged", a, stream);
 }
 
 }  // extern "C"

@@ -86,28 +86,59 @@ struct Rows {              // one warp step: rows g, g+8, g+16, g+24 of a 32-ent
     float sc;              // scale of the entry this thread finalises
 };
 
-template <int NU>
-__device__ __forceinline__ void load_rows(Rows<NU>& r, const uint8_t* kb, const float* ksc, int base, int hi,
-                                          int g, int tq, int wsel) {
+// Where this CTA's key rows live.  Plain layout: row b * N_cap + e.  Paged:
+// the page of entry e comes from the block-table slice staged in shared
+// memory (spg, pages p_lo ..), else straight from the block table.
+struct RowSrc {
+    const uint8_t* kb;     // plain: this element's first key row; paged: the pool
+    const float* ksc;      // plain: this element's first scale; paged: the scale pool
+    const int* spg;        // paged: staged page ids (or nullptr)
+    const int* btrow;      // paged: this element's block-table row
+    int p_lo, shift, num_pages;
+};
+
+template <bool PAGED>
+__device__ __forceinline__ long key_row(const RowSrc& rs, int e) {
+    if constexpr (!PAGED) {
+        return e;
+    } else {
+        const int j = e >> rs.shift;
+        const int pg = rs.spg ? rs.spg[j - rs.p_lo] : __ldg(rs.btrow + j);
+        if (pg < 0 || pg >= rs.num_pages) return -1;
+        return ((long)pg << rs.shift) + (e & ((1 << rs.shift) - 1));
+    }
+}
+
+template <int NU, bool PAGED>
+__device__ __forceinline__ void load_rows(Rows<NU>& r, const RowSrc& rs, int base, int hi, int g,
+                                          int tq, int wsel) {
+    // base is a multiple of 32: with pages of >= 32 entries the whole group
+    // lies in one page and one lookup serves it
+    const bool one_page = PAGED && rs.shift >= 5;
+    const long rbase = one_page ? key_row<PAGED>(rs, base) : 0;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
         const int e = base + g + 8 * q;
+        const long row = e >= hi ? -1 : (one_page ? (rbase < 0 ? -1 : rbase + (e - base)) : key_row<PAGED>(rs, e));
 #pragma unroll
         for (int nu = 0; nu < NU; ++nu)
-            r.u[q][nu] = e < hi ? __ldcs(reinterpret_cast<const uint4*>(kb + (size_t)e * (64 * NU) + 64 * nu + 16 * tq))
-                                : make_uint4(0u, 0u, 0u, 0u);
+            r.u[q][nu] = row >= 0 ? __ldcs(reinterpret_cast<const uint4*>(rs.kb + (size_t)row * (64 * NU) + 64 * nu + 16 * tq))
+                                  : make_uint4(0u, 0u, 0u, 0u);
     }
     const int ew = base + wsel;
-    r.sc = ew < hi ? __ldcs(ksc + ew) : 0.0f;
+    const long rw = ew >= hi ? -1 : (one_page ? (rbase < 0 ? -1 : rbase + wsel) : key_row<PAGED>(rs, ew));
+    r.sc = rw >= 0 ? __ldcs(rs.ksc + rw) : 0.0f;
 }
+
+constexpr int kPageSlots = 1024;   // block-table entries a paged CTA stages in shared memory
 
 // Resident CTAs per SM the register budget is sized for (d_I = 64: four).
 template <int NU>
 constexpr int min_blocks() { return NU == 1 ? 4 : 2; }
 
-template <int QD, int NU>
+template <int QD, int NU, bool PAGED>
 __global__ void __launch_bounds__(kThreads, min_blocks<NU>()) indexer_split_kernel(IndexerArgs a) {
-    extern __shared__ __align__(16) unsigned dyn[];   // [2][256] histograms, then [ch] keys
+    extern __shared__ __align__(16) unsigned dyn[];   // [2][256] histograms, [ch] keys, (paged) page ids
     unsigned* hist_buf = dyn;
     unsigned* keys = dyn + 2 * 256;                   // score keys of this CTA's entries
     __shared__ SplitShared sh;
@@ -188,6 +219,19 @@ __global__ void __launch_bounds__(kThreads, min_blocks<NU>()) indexer_split_kern
             if (lane == 0) sh.qs[h] = 0.0f;
         }
     }
+    // ---- paged caches: this CTA's slice of the block table into shared memory
+    bool pages_staged = false;
+    const int ch_alloc = max((a.N_cap + C - 1) / C + kGroup - 1, kGroup) / kGroup * kGroup;
+    if constexpr (PAGED) {
+        const int p_lo = lo >> a.pages.page_shift;
+        const int np = hi > lo ? ((hi - 1) >> a.pages.page_shift) - p_lo + 1 : 0;
+        pages_staged = np <= kPageSlots;
+        if (pages_staged) {
+            int* spg = reinterpret_cast<int*>(keys + ch_alloc);
+            const int* btrow = a.pages.bt + (size_t)b * a.pages.max_pages;
+            for (int i = tid; i < np; i += kThreads) spg[i] = btrow[p_lo + i];
+        }
+    }
     __syncthreads();
 
     // ---- scores of [lo, hi)
@@ -201,15 +245,26 @@ __global__ void __launch_bounds__(kThreads, min_blocks<NU>()) indexer_split_kern
             bq[nu][0] = v.x; bq[nu][1] = v.y; bq[nu][2] = v.z; bq[nu][3] = v.w;
         }
         const float qs0 = sh.qs[2 * tq], qs1 = sh.qs[2 * tq + 1];
-        const uint8_t* kb = static_cast<const uint8_t*>(a.kI) + (size_t)b * a.N_cap * d;
-        const float* ksc = a.kI_scale + (size_t)b * a.N_cap;
+        RowSrc src;
+        src.kb = static_cast<const uint8_t*>(a.kI);
+        src.ksc = a.kI_scale;
+        if constexpr (!PAGED) {
+            src.kb += (size_t)b * a.N_cap * d;
+            src.ksc += (size_t)b * a.N_cap;
+        } else {
+            src.btrow = a.pages.bt + (size_t)b * a.pages.max_pages;
+            src.shift = a.pages.page_shift;
+            src.num_pages = a.pages.num_pages;
+            src.p_lo = lo >> src.shift;
+            src.spg = pages_staged ? reinterpret_cast<const int*>(keys + ch_alloc) : nullptr;
+        }
         const int wsel = (tq >> 1) * 16 + (tq & 1) * 8 + g;   // the entry this thread finalises
         const int step = kWarps * kGroup;
         Rows<NU> cur, nxt;
         int base = lo + warp * kGroup;
-        if (base < hi) load_rows<NU>(cur, kb, ksc, base, hi, g, tq, wsel);
+        if (base < hi) load_rows<NU, PAGED>(cur, src, base, hi, g, tq, wsel);
         for (; base < hi; base += step) {
-            if (base + step < hi) load_rows<NU>(nxt, kb, ksc, base + step, hi, g, tq, wsel);
+            if (base + step < hi) load_rows<NU, PAGED>(nxt, src, base + step, hi, g, tq, wsel);
             float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int nu = 0; nu < NU; ++nu) {
@@ -404,11 +459,11 @@ long chunk_cap(const IndexerArgs& a, int C) {
     return std::max<long>(((long)a.N_cap + C - 1) / C + kGroup - 1, kGroup) / kGroup * kGroup;
 }
 
-template <int QD, int NU>
+template <int QD, int NU, bool PAGED>
 cudaError_t launch_t(const IndexerArgs& a, cudaStream_t s) {
     const int C = choose_cluster(a);
-    const size_t smem = sizeof(unsigned) * ((size_t)chunk_cap(a, C) + 2 * 256);
-    auto kern = indexer_split_kernel<QD, NU>;
+    const size_t smem = sizeof(unsigned) * ((size_t)chunk_cap(a, C) + 2 * 256 + (PAGED ? kPageSlots : 0));
+    auto kern = indexer_split_kernel<QD, NU, PAGED>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (C > 8) {
@@ -442,9 +497,15 @@ bool indexer_split_supported(const IndexerArgs& a) {
     return chunk_cap(a, choose_cluster(a)) <= kMaxChunk;
 }
 
+template <bool PAGED>
+cudaError_t launch_paging(const IndexerArgs& a, cudaStream_t s) {
+    if (a.qI_dt == DT_E4M3)
+        return a.d_I == 64 ? launch_t<DT_E4M3, 1, PAGED>(a, s) : launch_t<DT_E4M3, 2, PAGED>(a, s);
+    return a.d_I == 64 ? launch_t<DT_BF16, 1, PAGED>(a, s) : launch_t<DT_BF16, 2, PAGED>(a, s);
+}
+
 cudaError_t launch_indexer_split(const IndexerArgs& a, cudaStream_t s) {
-    if (a.qI_dt == DT_E4M3) return a.d_I == 64 ? launch_t<DT_E4M3, 1>(a, s) : launch_t<DT_E4M3, 2>(a, s);
-    return a.d_I == 64 ? launch_t<DT_BF16, 1>(a, s) : launch_t<DT_BF16, 2>(a, s);
+    return a.pages.bt ? launch_paging<true>(a, s) : launch_paging<false>(a, s);
 }
 
 }  // namespace csa

@@ -114,9 +114,14 @@ __global__ void __launch_bounds__(kThreads) indexer_topk_kernel(IndexerArgs a) {
     }
 
     // ---- scores of the visible entries, as order-preserving keys
-    const uint8_t* kbase = static_cast<const uint8_t*>(a.kI) + (size_t)b * a.N_cap * d * elem_bytes<KD>();
+    const uint8_t* kbase = static_cast<const uint8_t*>(a.kI);   // rows from cache_row()
     for (int s = threadIdx.x; s < V; s += kThreads) {
-        const void* krow = kbase + (size_t)s * d * elem_bytes<KD>();
+        const long crow = cache_row(a.pages, a.N_cap, b, s);
+        if (crow < 0) {                      // page outside the pool: an absent (zero) row
+            keys[s] = score_key(0.0f);
+            continue;
+        }
+        const void* krow = kbase + (size_t)crow * d * elem_bytes<KD>();
         float dots[kMaxHeads];
 #pragma unroll
         for (int h = 0; h < kMaxHeads; ++h) dots[h] = 0.0f;
@@ -136,7 +141,7 @@ __global__ void __launch_bounds__(kThreads) indexer_topk_kernel(IndexerArgs a) {
 #pragma unroll
         for (int h = 0; h < kMaxHeads; ++h)
             if (h < H) sc = fmaf(qs[h], relu0(dots[h]), sc);
-        if constexpr (KD == DT_E4M3) sc *= a.kI_scale[(size_t)b * a.N_cap + s];
+        if constexpr (KD == DT_E4M3) sc *= a.kI_scale[crow];
         keys[s] = score_key(sc);
     }
     __syncthreads();
@@ -237,13 +242,13 @@ cudaError_t launch_indexer_topk(const IndexerArgs& a, cudaStream_t s, const char
         *why = "csa_indexer_topk: H_I > 16 or d_I > 256";
         return cudaErrorNotSupported;
     }
-    if (indexer_tc_supported(a)) {
+    if (a.pages.bt == nullptr && indexer_tc_supported(a)) {     // paged caches: decode kernels
         uint32_t* err = device_error_word();
         if (!err) return cudaErrorUnknown;
         return launch_indexer_tc(a, err, s);
     }
     if (indexer_split_supported(a)) return launch_indexer_split(a, s);
-    if (a.N_cap > 40960) {
+    if (a.N_cap > 40960) {      // one row's score keys must fit the CTA's shared memory
         *why = "csa_indexer_topk: N_cap > 40960 needs fp8 keys with scales, d_I in {64, 128}, H_I <= 8";
         return cudaErrorNotSupported;
     }

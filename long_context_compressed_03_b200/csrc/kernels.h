@@ -5,6 +5,26 @@
 
 namespace csa {
 
+// A paged cache.  Logical entry s (0 <= s < N_cap = max_pages * page size) of
+// batch element b is physical row
+//   bt[b * max_pages + (s >> page_shift)] * page size + (s & (page size - 1))
+// of the page pool; bt == nullptr means the plain layout, row b * N_cap + s.
+struct PageMap {
+    const int* bt = nullptr;
+    int max_pages = 0;
+    int page_shift = 0;
+    int num_pages = 0;         // pool size in pages: page ids outside [0, num_pages) are absent
+};
+
+// Physical row of logical entry s of element b, or -1 when its page id lies
+// outside the pool (the entry is then treated as absent: never read or written).
+__host__ __device__ __forceinline__ long cache_row(const PageMap& pm, int N_cap, int b, int s) {
+    if (!pm.bt) return (long)b * N_cap + s;
+    const int pg = pm.bt[(size_t)b * pm.max_pages + (s >> pm.page_shift)];
+    if (pg < 0 || pg >= pm.num_pages) return -1;
+    return ((long)pg << pm.page_shift) + (s & ((1 << pm.page_shift) - 1));
+}
+
 struct CompressArgs {
     const void* x; int x_dt;
     int B, n, d_in;
@@ -41,6 +61,7 @@ struct AppendArgs {
     int N_cap;
     int* n_entries;
     float hnorm;               // fp32(1/sqrt(d_out)) for the Hadamard fp8 type
+    PageMap pages;             // cache (and cache_scale) layout
 };
 
 struct IndexerArgs {
@@ -52,6 +73,7 @@ struct IndexerArgs {
     int* idx_out;
     float hnorm;               // fp32(1/sqrt(d_I)): keys of the Hadamard fp8 type
     const float* qI_weight;    // [B, n_q, H_I] gate weights or NULL (all 1)
+    PageMap pages;             // kI (and kI_scale) layout
 };
 
 struct AttnArgs {
@@ -67,6 +89,7 @@ struct AttnArgs {
     const int* q_pos;
     float scale;
     void* out; float* lse_out;
+    PageMap pages;             // kv_c layout
 };
 
 // Device address of this library's error word on the current device (set by

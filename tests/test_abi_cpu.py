@@ -181,6 +181,38 @@ def test_hadamard_type_validation(lib):
     assert a(*args) == api.CSA_ERR_UNSUPPORTED
 
 
+def test_paged_entry_point_validation(lib):
+    # the page map is checked before anything is launched
+    f = lib.csa_sparse_attn_paged
+    #       q   dt B  nq H   D    pool  bt   maxp P   np   idx  k  raw  L  p0    len   W  qpos
+    args = [FAKE, 1, 1, 8, 64, 128, FAKE, FAKE, 16, 64, 40, FAKE, 4, FAKE, 8, None, None, 4, None,
+            ctypes.c_float(0.0), FAKE, None, None]
+    bad = list(args); bad[9] = 48                      # page size not a power of two
+    assert f(*bad) == api.CSA_ERR_INVALID_ARG
+    bad = list(args); bad[7] = None                    # no block table
+    assert f(*bad) == api.CSA_ERR_INVALID_ARG
+    bad = list(args); bad[7] = ODD
+    assert f(*bad) == api.CSA_ERR_MISALIGNED
+    bad = list(args); bad[8] = 1 << 20; bad[9] = 1 << 12   # capacity above 2^30 entries
+    assert f(*bad) == api.CSA_ERR_INVALID_ARG
+    ok = list(args); ok[2] = 0                         # B = 0: no-op
+    assert f(*ok) == api.CSA_OK
+    g = lib.csa_indexer_topk_paged
+    #       qI  dt sc   wt   pool dt  scale bt   maxp P  np  B  nq H  d   ne    pos   m  k  idx  stream
+    args = [FAKE, 1, None, None, FAKE, 2, None, FAKE, 16, 64, 40, 1, 1, 4, 64, None, FAKE, 4, 8, FAKE, None]
+    assert g(*args) == api.CSA_ERR_INVALID_ARG        # fp8 keys without their scale pool
+    bad = list(args); bad[6] = FAKE; bad[9] = 0        # page size 0
+    assert g(*bad) == api.CSA_ERR_INVALID_ARG
+    h = lib.csa_compress_append_paged
+    #       x   dt B  d_in W    d_out m  ov pos   state cache dt scale bt  maxp P  np  n_ent stream
+    args = [FAKE, 1, 2, 64, FAKE, 64, 4, 1, FAKE, FAKE, FAKE, 1, None, FAKE, 4, 3, 8, None, None]
+    assert h(*args) == api.CSA_ERR_INVALID_ARG        # page size 3
+    k = lib.hca_dense_attn_paged
+    args = [FAKE, 2, 1, 1, 64, 128, FAKE, FAKE, 16, 64, 40, None, 4, FAKE, 8, None, None, 4, None,
+            ctypes.c_float(0.0), FAKE, None, None]
+    assert k(*args) == api.CSA_ERR_UNSUPPORTED        # fp8 attention operands
+
+
 def test_attention_validation(lib):
     f = lib.csa_sparse_attn
     args = [FAKE, 1, 1, 8, 64, 128, FAKE, 16, FAKE, 4, FAKE, 8, None, None, 4, None,
