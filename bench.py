@@ -294,6 +294,48 @@ def run_variants(w, path, dev, steps, rank):
     return out
 
 
+def run_prefill_varlen(w, path, dev, steps, warmup, S=8):
+    """The prefill step over S packed sequences of mixed lengths (the c3
+    tokens re-cut into S documents; csa_*_varlen entry points), timed like
+    the headline step (inputs larger than L2)."""
+    d = path.d
+    lens = synth.varlen_lengths(w.B * w.n, S, multiple=4, seed=3)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    e = api.varlen_entry_offsets(cu, w.m)
+    T, E = int(cu[-1]), int(e[-1])
+    q, kv = d["q"].reshape(T, w.H, w.D), d["kv"].reshape(T, w.D)
+    qI, kI_raw = d["qI"].reshape(T, w.H_I, w.d_I), d["kI_raw"].reshape(T, w.d_I)
+    kv_c = torch.empty(E, w.D, dtype=torch.bfloat16, device=dev)
+    kI_c = torch.empty(E, w.d_I, dtype=torch.uint8, device=dev)
+    kI_s = torch.empty(E, dtype=torch.float32, device=dev)
+    idx = torch.empty(T, w.topk, dtype=torch.int32, device=dev)
+    out = torch.empty_like(q)
+    names = ["compress_kv", "compress_kI", "indexer_topk", "sparse_attn"]
+
+    def step():
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(5)]
+        evs[0].record()
+        api.csa_compress_varlen(kv, cu, d["W_c"], w.m, True, kv_c)
+        evs[1].record()
+        api.csa_compress_varlen(kI_raw, cu, d["W_Ic"], w.m, True, kI_c, kI_s)
+        evs[2].record()
+        api.csa_indexer_topk_varlen(qI, kI_c, cu, w.m, w.topk, idx, kI_scale=kI_s)
+        evs[3].record()
+        api.csa_sparse_attn_varlen(q, cu, kv_c, w.m, idx, kv, w.window, out)
+        evs[4].record()
+        return evs
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    recs = [step() for _ in range(steps)]
+    torch.cuda.synchronize()
+    ms = float(np.mean([r[0].elapsed_time(r[4]) for r in recs]))
+    stages = {nm: float(np.mean([r[i].elapsed_time(r[i + 1]) for r in recs]))
+              for i, nm in enumerate(names)}
+    return dict(lens=lens, T=T, ms=ms, stages=stages)
+
+
 def run_e2e(w, inp, dev, steps):
     """Same step through the public API with pinned host inputs: h2d copies of
     the step's inputs and a d2h read of its result are inside the timed region."""
@@ -670,6 +712,14 @@ def main():
                     "overlapping), Hadamard-rotated fp8 indexer keys, gated indexer + top-k "
                     "against rotated keys",
             **run_variants(w, pre["path"], dev, max(3, args.steps), rank)}
+    if not args.no_variants:
+        pv = run_prefill_varlen(w, pre["path"], dev, max(3, args.steps), args.warmup)
+        vval, vms = dist_ctx.job_rate(pv["T"], pv["ms"])
+        line["prefill_varlen"] = {
+            "workload": "csa_prefill_packed8_n64k_fp8idx", "value": vval, "unit": "queries/s",
+            "ms_per_step": vms, "lengths": pv["lens"], "stages_ms": pv["stages"],
+            "note": "the c3 tokens re-cut into 8 packed sequences (csa_*_varlen entry points); "
+                    "less causal work than one 64K sequence, so not comparable to the headline"}
     if not args.no_decode:
         dec = run_decode(dev, args.steps, args.warmup, rank)
         dval, dms = dist_ctx.job_rate(dec["w"].B, dec["ms"])

@@ -20,8 +20,11 @@
  * Conventions shared by every entry point
  *   - Tensor arguments are DEVICE pointers to caller-owned memory; the
  *     library never allocates, frees or keeps them.  Layouts are batch-first,
- *     contiguous, last dimension innermost.  Every tensor base pointer must
- *     be 16-byte aligned (else CSA_ERR_MISALIGNED).
+ *     contiguous, last dimension innermost.  Data tensors (activations,
+ *     weights, caches, outputs) must start on a 16-byte boundary;
+ *     per-element arrays (scales, gate weights, APE, compressor state,
+ *     indices, positions, counts, LSE, block tables) on a 4-byte one (else
+ *     CSA_ERR_MISALIGNED).
  *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL is the legacy
  *     default stream).  Arguments are validated on the host first; on any
  *     error nothing is launched.  A launch failure returns CSA_ERR_CUDA.
@@ -52,7 +55,7 @@ typedef enum {
     CSA_OK = 0,
     CSA_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad combination */
     CSA_ERR_UNSUPPORTED = 2,  /* valid but not implemented (dtype, head count, size) */
-    CSA_ERR_MISALIGNED = 3,   /* a tensor base pointer is not 16-byte aligned */
+    CSA_ERR_MISALIGNED = 3,   /* a pointer breaks the alignment rule below */
     CSA_ERR_CUDA = 4,         /* a CUDA runtime call or kernel launch failed */
     CSA_ERR_TIMEOUT = 5       /* reserved: a bounded device-side wait expired */
 } csa_status_t;
@@ -141,7 +144,7 @@ csa_status_t csa_compress(const void* x, int x_dt, int B, int n, int d_in, const
  *   ape    [m, c*d_out]       fp32
  *   out, out_dt, out_row_scale: as csa_compress (fp32 / bf16 / E4M3 / rotated E4M3).
  *   Limits: 16 <= d_in, d_out <= 256, multiples of 16; m >= 1.  Projections,
- *   softmax and pooling run in fp32 (expf).  Pointers 16-byte aligned.
+ *   softmax and pooling run in fp32 (expf).
  *   Errors as csa_compress; nothing is launched on a validation error.
  */
 csa_status_t csa_compress_gated(const void* x, int x_dt, int B, int n, int d_in, const void* W_kv,
@@ -314,6 +317,49 @@ csa_status_t hca_dense_attn_paged(const void* q, int dt, int B, int n_q, int H, 
                                   const void* kv_raw, int L_raw, const int* raw_pos0,
                                   const int* raw_len, int window, const int* q_pos,
                                   float softmax_scale, void* out, float* lse_out, void* stream);
+
+/*
+ * Packed (varlen) prefill.  S sequences are packed along the token dimension:
+ * sequence s owns tokens [cu_seqlens[s], cu_seqlens[s+1]) (cu_seqlens: HOST
+ * int32 [S+1], cu_seqlens[0] = 0, non-decreasing) and, in the packed
+ * compressed dimension, entries [e(s), e(s+1)) with
+ * e(s) = sum_{s' < s} floor(len(s') / m) (csa_varlen_entry_offsets).  Each
+ * sequence is computed exactly as the unpacked call with B = 1, n = len(s)
+ * would compute it: positions, the visibility rule, the window and the top-k
+ * are local to the sequence, and indices in idx are entries of the sequence
+ * (0 .. floor(len/m) - 1, -1 padding).  "DeepSeek V4 CSA + CP 迁移到 HP：
+ * 困难点深度分析" names this layout: actual_seq_len in the attention's
+ * construct signature (§4.2) and compressed cu_seqlens with packed-sequence
+ * support in its migration plan (Phase 3).  The alignment rule applies to
+ * every sequence's slice (it holds whenever the base pointers follow it,
+ * since rows are multiples of 16 bytes).  All sequences are validated
+ * before the first launch; the calls
+ * launch one kernel per non-empty sequence (capturable in a CUDA graph).
+ *   tensors: packed forms of the unpacked calls' arguments, e.g. for
+ *   csa_sparse_attn_varlen q / out [T, H, D], kv_c [E, D], idx [T, topk],
+ *   kv_raw [T, D], lse_out [T, H]; T = cu_seqlens[S], E = e(S).
+ */
+int csa_varlen_entry_offsets(const int* cu_seqlens, int S, int m, int* entry_offsets);
+/*   writes e(0..S) into entry_offsets [S+1] (host) and returns e(S), or -1 on
+ *   an invalid argument. */
+
+csa_status_t csa_compress_varlen(const void* x, int x_dt, int S, const int* cu_seqlens, int d_in,
+                                 const void* W, int d_out, int m, int overlap, void* out,
+                                 int out_dt, float* out_row_scale, void* stream);
+
+csa_status_t csa_indexer_topk_varlen(const void* qI, int qI_dt, const float* qI_scale,
+                                     const float* qI_weight, const void* kI, int kI_dt,
+                                     const float* kI_scale, int S, const int* cu_seqlens, int H_I,
+                                     int d_I, int m, int topk, int* idx_out, void* stream);
+
+csa_status_t csa_sparse_attn_varlen(const void* q, int dt, int S, const int* cu_seqlens, int H,
+                                    int D, const void* kv_c, int m, const int* idx, int topk,
+                                    const void* kv_raw, int window, float softmax_scale, void* out,
+                                    float* lse_out, void* stream);
+
+csa_status_t hca_dense_attn_varlen(const void* q, int dt, int S, const int* cu_seqlens, int H,
+                                   int D, const void* kv_c, int m, const void* kv_raw, int window,
+                                   float softmax_scale, void* out, float* lse_out, void* stream);
 
 #ifdef __cplusplus
 }

@@ -17,6 +17,7 @@ import ctypes
 import os
 import threading
 
+import numpy as np
 import torch
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
@@ -40,6 +41,11 @@ SIGNATURES = {
     "csa_indexer_topk": (I, [P, I, P, P, P, I, P, I, I, I, I, I, P, P, I, I, P, P]),
     "csa_sparse_attn": (I, [P, I, I, I, I, I, P, I, P, I, P, I, P, P, I, P, F, P, P, P]),
     "hca_dense_attn": (I, [P, I, I, I, I, I, P, I, P, I, P, I, P, P, I, P, F, P, P, P]),
+    "csa_varlen_entry_offsets": (I, [P, I, I, P]),
+    "csa_compress_varlen": (I, [P, I, I, P, I, P, I, I, I, P, I, P, P]),
+    "csa_indexer_topk_varlen": (I, [P, I, P, P, P, I, P, I, P, I, I, I, I, P, P]),
+    "csa_sparse_attn_varlen": (I, [P, I, I, P, I, I, P, I, P, I, P, I, F, P, P, P]),
+    "hca_dense_attn_varlen": (I, [P, I, I, P, I, I, P, I, P, I, F, P, P, P]),
     "csa_compress_append_paged": (I, [P, I, I, I, P, I, I, I, P, P, P, I, P, P, I, I, I, P, P]),
     "csa_indexer_topk_paged": (I, [P, I, P, P, P, I, P, P, I, I, I, I, I, I, I, P, P, I, I, P, P]),
     "csa_sparse_attn_paged": (I, [P, I, I, I, I, I, P, P, I, I, I, P, I, P, I, P, P, I, P, F, P, P,
@@ -250,6 +256,70 @@ def hca_dense_attn(q: torch.Tensor, kv_c: torch.Tensor, m: int, kv_raw: torch.Te
                                  _i32(raw_pos0, "raw_pos0"), _i32(raw_len, "raw_len"), window,
                                  _i32(q_pos, "q_pos"), float(softmax_scale), _ptr(out),
                                  _ptr(lse_out), _stream(stream)))
+
+
+# ---------------------------------------------------------------- packed (varlen) prefill
+def _host_cu(cu_seqlens) -> tuple:
+    """cu_seqlens as a host int32 array (kept alive by the caller's frame) + S."""
+    cu = np.ascontiguousarray(np.asarray(cu_seqlens.cpu() if isinstance(cu_seqlens, torch.Tensor)
+                                         else cu_seqlens, dtype=np.int32))
+    return cu, cu.size - 1, cu.ctypes.data_as(ctypes.c_void_p)
+
+
+def varlen_entry_offsets(cu_seqlens, m: int) -> np.ndarray:
+    """e(0..S): where each sequence's compressed entries start in the packed cache."""
+    cu, S, p = _host_cu(cu_seqlens)
+    out = np.zeros(S + 1, np.int32)
+    if load().csa_varlen_entry_offsets(p, S, m, out.ctypes.data_as(ctypes.c_void_p)) < 0:
+        raise ValueError("invalid cu_seqlens or m")
+    return out
+
+
+def csa_compress_varlen(x: torch.Tensor, cu_seqlens, W: torch.Tensor, m: int, overlap: bool,
+                        out: torch.Tensor, out_row_scale: torch.Tensor | None = None,
+                        hadamard: bool = False, stream=None) -> None:
+    """x [T, d_in] packed -> out [E, d_out] packed (E = varlen_entry_offsets(...)[-1])."""
+    cu, S, cup = _host_cu(cu_seqlens)
+    _check(load().csa_compress_varlen(_ptr(x), _dt(x), S, cup, x.shape[-1], _ptr(W), W.shape[1], m,
+                                      int(bool(overlap)), _ptr(out), _dt_rot(out, hadamard),
+                                      _ptr(out_row_scale), _stream(stream)))
+
+
+def csa_indexer_topk_varlen(qI: torch.Tensor, kI: torch.Tensor, cu_seqlens, m: int, topk: int,
+                            idx_out: torch.Tensor, qI_scale=None, kI_scale=None,
+                            kI_rotated: bool = False, qI_weight=None, stream=None) -> None:
+    """qI [T, H_I, d_I], kI [E, d_I] packed -> idx_out [T, topk] (sequence-local entries)."""
+    cu, S, cup = _host_cu(cu_seqlens)
+    _, H_I, d_I = qI.shape
+    _check(load().csa_indexer_topk_varlen(_ptr(qI), _dt(qI), _ptr(qI_scale), _ptr(qI_weight),
+                                          _ptr(kI), _dt_rot(kI, kI_rotated), _ptr(kI_scale), S, cup,
+                                          H_I, d_I, m, topk, _i32(idx_out, "idx_out"),
+                                          _stream(stream)))
+
+
+def csa_sparse_attn_varlen(q: torch.Tensor, cu_seqlens, kv_c: torch.Tensor, m: int,
+                           idx: torch.Tensor | None, kv_raw: torch.Tensor, window: int,
+                           out: torch.Tensor, lse_out: torch.Tensor | None = None,
+                           softmax_scale: float = 0.0, stream=None) -> None:
+    """q / out [T, H, D], kv_c [E, D], idx [T, topk], kv_raw [T, D] (packed)."""
+    cu, S, cup = _host_cu(cu_seqlens)
+    _, H, D = q.shape
+    topk = 0 if idx is None else idx.shape[-1]
+    _check(load().csa_sparse_attn_varlen(_ptr(q), _dt(q), S, cup, H, D, _ptr(kv_c), m,
+                                         _i32(idx, "idx"), topk, _ptr(kv_raw), window,
+                                         float(softmax_scale), _ptr(out), _ptr(lse_out),
+                                         _stream(stream)))
+
+
+def hca_dense_attn_varlen(q: torch.Tensor, cu_seqlens, kv_c: torch.Tensor, m: int,
+                          kv_raw: torch.Tensor, window: int, out: torch.Tensor,
+                          lse_out: torch.Tensor | None = None, softmax_scale: float = 0.0,
+                          stream=None) -> None:
+    cu, S, cup = _host_cu(cu_seqlens)
+    _, H, D = q.shape
+    _check(load().hca_dense_attn_varlen(_ptr(q), _dt(q), S, cup, H, D, _ptr(kv_c), m, _ptr(kv_raw),
+                                        window, float(softmax_scale), _ptr(out), _ptr(lse_out),
+                                        _stream(stream)))
 
 
 # ---------------------------------------------------------------- paged caches

@@ -166,6 +166,14 @@ cudaError_t launch_dims(const AttnArgs& a, cudaStream_t s, const char** why) {
 
 }  // namespace
 
+cudaError_t launch_attention_packed(const AttnArgs& a, cudaStream_t s) {
+    if (a.vl == nullptr || a.pages.bt != nullptr || !attention_tc_supported(a))
+        return cudaErrorNotSupported;
+    uint32_t* err = device_error_word();
+    if (!err) return cudaErrorUnknown;
+    return launch_attention_tc(a, err, s);
+}
+
 cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s, const char** why) {
     if (a.B <= 0 || a.n_q <= 0) return cudaSuccess;
     if (a.pages.bt == nullptr && attention_tc_supported(a)) {   // paged caches: decode kernels

@@ -103,6 +103,7 @@ struct TcParams {
     __nv_bfloat16* out;
     float* lse;
     uint32_t* err;
+    VarlenMap vl;              // packed sequences (vl.S > 0)
 };
 
 struct Geometry {
@@ -126,12 +127,59 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-__device__ __forceinline__ Geometry geometry(const TcParams& p, int b, int t0) {
+// Units of work: unit u covers tokens [t0, t0 + 4) of sequence b, where
+// u = b * units_per_seq + t0 / 4 (packed sequences: u = uoff[b] + t0 / 4).
+// The kernel is persistent: CTA c takes units c, c + gridDim.x, ... in that
+// order, and every role walks the same list, so barrier phases run on across
+// units.  A unit also carries where its sequence's rows start.
+struct Unit {
+    int b, t0;
+    int n;          // the sequence's length
+    int N;          // its compressed entries
+    int L_raw;      // its raw rows
+    int ne_dense;   // dense: entries it may see (n_entries, clamped)
+    size_t tok0;    // row of its token 0 in q / out / lse / idx
+    size_t ent0;    // row of its entry 0 in kv_c
+    size_t raw0;    // row of its raw position 0 in kv_raw
+};
+__device__ __forceinline__ Unit unit_of(const TcParams& p, int u) {
+    Unit r;
+    if (p.vl.S) {
+        int lo = 0, hi = p.vl.S - 1;                  // the last sequence with uoff <= u
+        while (lo < hi) {
+            const int mid = (lo + hi + 1) >> 1;
+            if (p.vl.uoff[mid] <= u) lo = mid; else hi = mid - 1;
+        }
+        r.b = lo;
+        r.t0 = (u - p.vl.uoff[lo]) * kTokens;
+        r.n = p.vl.tok[lo + 1] - p.vl.tok[lo];
+        r.N = r.n / p.m;
+        r.L_raw = r.n;
+        r.ne_dense = r.N;
+        r.tok0 = (size_t)p.vl.tok[lo];
+        r.ent0 = (size_t)p.vl.ent[lo];
+        r.raw0 = r.tok0;
+    } else {
+        const int per = (p.n + kTokens - 1) / kTokens;
+        r.b = u / per;
+        r.t0 = (u - r.b * per) * kTokens;
+        r.n = p.n;
+        r.N = p.N_cap;
+        r.L_raw = p.L_raw;
+        r.ne_dense = p.dense ? clampi(p.n_entries ? p.n_entries[r.b] : p.N_cap, 0, p.N_cap) : 0;
+        r.tok0 = (size_t)r.b * p.n;
+        r.ent0 = (size_t)r.b * p.N_cap;
+        r.raw0 = (size_t)r.b * p.L_raw;
+    }
+    return r;
+}
+
+__device__ __forceinline__ Geometry geometry(const TcParams& p, const Unit& un) {
     Geometry g;
-    const int t_last = min(t0 + kTokens - 1, p.n - 1);
+    const int t0 = un.t0;
+    const int t_last = min(t0 + kTokens - 1, un.n - 1);
     if (p.dense) {
-        const int ne = clampi(p.n_entries ? p.n_entries[b] : p.N_cap, 0, p.N_cap);
-        g.Vmax = min((t_last + 1) / p.m, ne);
+        g.Vmax = min((t_last + 1) / p.m, un.ne_dense);
         g.cc = 0;
         g.Tc = (g.Vmax + kBN - 1) / kBN;
         g.bn_c_last = g.Tc ? round16(g.Vmax - (g.Tc - 1) * kBN) : 0;
@@ -144,7 +192,7 @@ __device__ __forceinline__ Geometry geometry(const TcParams& p, int b, int t0) {
     }
     if (p.window > 0) {
         g.p_lo = max(0, t0 - p.window + 1);
-        const int p_hi = min(t_last, p.L_raw - 1);
+        const int p_hi = min(t_last, un.L_raw - 1);
         g.Lw = max(0, p_hi - g.p_lo + 1);
     } else {
         g.p_lo = 0;
@@ -336,21 +384,6 @@ __device__ __noinline__ void rescale_o(uint32_t o_addr, float alpha) {
     tmem_st_wait();
 }
 
-// Units of work: unit u covers tokens [t0, t0 + 4) of sequence b, where
-// u = b * units_per_seq + t0 / 4.  The kernel is persistent: CTA c takes units
-// c, c + gridDim.x, ... in that order, and every role walks the same list, so
-// barrier phases run on across units.
-struct Unit {
-    int b, t0;
-};
-__device__ __forceinline__ Unit unit_of(const TcParams& p, int u) {
-    const int per = (p.n + kTokens - 1) / kTokens;
-    Unit r;
-    r.b = u / per;
-    r.t0 = (u - r.b * per) * kTokens;
-    return r;
-}
-
 __global__ void __launch_bounds__(kThreads, 1)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_c,
                const __grid_constant__ CUtensorMap tm_w, TcParams p) {
@@ -363,7 +396,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     int* sIdx = reinterpret_cast<int*>(stats + 4 * kRows);       // [kTokens][topk]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_units = p.B * ((p.n + kTokens - 1) / kTokens);
+    const int n_units = p.vl.S ? p.vl.uoff[p.vl.S] : p.B * ((p.n + kTokens - 1) / kTokens);
     volatile int* abort = &ctl->abort;
 
     if (threadIdx.x == 0) {
@@ -405,8 +438,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         bool go = true;
         for (int u = blockIdx.x; u < n_units && go; u += gridDim.x) {
             const Unit un = unit_of(p, u);
-            const int b = un.b, t0 = un.t0;
-            const Geometry g = geometry(p, b, t0);
+            const int t0 = un.t0;
+            const Geometry g = geometry(p, un);
             // the unit's index rows (out-of-range tokens read as padding); the
             // previous unit's gathers have all been issued
             named_sync(1, kLoadThreads);
@@ -414,13 +447,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 for (int i = lt; i < kTokens * p.topk; i += kLoadThreads) {
                     const int tok = i / p.topk, c = i - tok * p.topk;
                     const int t = t0 + tok;
-                    sIdx[i] = (t < p.n) ? __ldg(p.idx + ((size_t)b * p.n + t) * p.topk + c) : -1;
+                    sIdx[i] = (t < un.n) ? __ldg(p.idx + (un.tok0 + t) * p.topk + c) : -1;
                 }
             }
             named_sync(1, kLoadThreads);
             const int NL = total_loads(p, g);
             const int nc = p.dense ? g.Tc : 2 * g.Tc;
-            const uint8_t* kvc_rows = static_cast<const uint8_t*>(p.kv_c) + (size_t)b * p.N_cap * (kD * 2);
+            const uint8_t* kvc_rows = static_cast<const uint8_t*>(p.kv_c) + un.ent0 * (kD * 2);
             for (int L = 0; L < NL; ++L, ++Lg) {
                 const int slot = Lg % kStages, use = Lg / kStages;
                 uint8_t* dst = sK + slot * kTileBytes;
@@ -453,7 +486,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     if (lt < kBN) {
                         const int c = chunk * kBN + lt;
                         const int sv = (c < p.topk) ? ir[lt] : -1;
-                        const bool ok = tpos < p.n && sv >= 0 && sv < p.N_cap;
+                        const bool ok = tpos < un.n && sv >= 0 && sv < un.N;
                         const uint32_t bits = __ballot_sync(0xffffffffu, ok);
                         if (lane == 0) ctl->mask[slot][warp] = bits;
                     }
@@ -465,7 +498,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         const int row = it * kRowsPerRound + (lt >> 4);
                         const int c = chunk * kBN + row;
                         int sv = (c < p.topk) ? ir[row] : -1;
-                        if (tpos >= p.n || sv < 0 || sv >= p.N_cap) sv = 0;   // masked; any valid row
+                        if (tpos >= un.n || sv < 0 || sv >= un.N) sv = 0;   // masked; any valid row
                         const uint8_t* src = kvc_rows + (size_t)sv * (kD * 2) + c16 * 16;
                         cp_async16(dst + half * kHalf + row * 128 + ((cc ^ (row & 7)) << 4), src);
                     }
@@ -475,8 +508,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 } else {
                     if (lt == 0) {
                         const CUtensorMap* tm = (kind == 1) ? &tm_c : &tm_w;
-                        const int row = (kind == 1) ? b * p.N_cap + chunk * kBN
-                                                    : b * p.L_raw + g.p_lo + chunk * kBN;
+                        const int row = (kind == 1) ? (int)un.ent0 + chunk * kBN
+                                                    : (int)un.raw0 + g.p_lo + chunk * kBN;
                         mbar_arrive_expect_tx(&ctl->full[slot], kTileBytes);
                         for (int h = 0; h < 2; ++h)
                             tma_load_2d(dst + h * kHalf, tm, h * 64, row, &ctl->full[slot]);
@@ -501,7 +534,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             auto load_q = [&](int u) {
                 const Unit un = unit_of(p, u);
                 mbar_arrive_expect_tx(&ctl->bar_q, 2 * kTileBytes);
-                const int qrow = (un.b * p.n + un.t0) * kH;
+                const int qrow = (int)(un.tok0 + un.t0) * kH;
                 for (int mt = 0; mt < 2; ++mt)
                     for (int h = 0; h < 2; ++h)
                         tma_load_2d(sQ + mt * kTileBytes + h * kHalf, &tm_q, h * 64, qrow + mt * kRows,
@@ -514,7 +547,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             if (blockIdx.x < n_units) load_q(blockIdx.x);
             for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++k) {
                 const Unit un = unit_of(p, u);
-                const Geometry g = geometry(p, un.b, un.t0);
+                const Geometry g = geometry(p, un);
                 ok = mbar_wait(&ctl->bar_q, k & 1, abort, p.err);
                 tc_fence_after();
                 auto issue_qk = [&](int mt, int j) -> bool {
@@ -605,15 +638,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         bool ok = true;
         for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++k) {
             const Unit un = unit_of(p, u);
-            const int b = un.b, t0 = un.t0;
-            const Geometry g = geometry(p, b, t0);
-            const int t = t0 + 2 * mt + u_tok;               // absolute position
-            const bool row_ok = t < p.n;
+            const int t0 = un.t0;
+            const Geometry g = geometry(p, un);
+            const int t = t0 + 2 * mt + u_tok;               // position in the sequence
+            const bool row_ok = t < un.n;
             int Vt = 0;
-            if (p.dense && row_ok) {
-                const int ne = clampi(p.n_entries ? p.n_entries[b] : p.N_cap, 0, p.N_cap);
-                Vt = min((t + 1) / p.m, ne);
-            }
+            if (p.dense && row_ok) Vt = min((t + 1) / p.m, un.ne_dense);
             const int w_lo = t - p.window + 1;               // window [w_lo, t]
             // m_used: running max (base 2); l_r: sum of the bf16-rounded weights
             // (normalises O); l_e: sum of the unrounded weights (the lse output)
@@ -704,15 +734,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         int k = 0;
         for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++k) {
             const Unit un = unit_of(p, u);
-            const Geometry g = geometry(p, un.b, un.t0);
+            const Geometry g = geometry(p, un);
             const int t = un.t0 + 2 * mt + u_tok;
-            const bool row_ok = t < p.n;
+            const bool row_ok = t < un.n;
             bool w_ok = mbar_wait(&ctl->stats_ready[mt], k & 1, abort, p.err);
             const RowStat st = stats[((k & 1) * 2 + mt) * kRows + r];
             w_ok = w_ok && mbar_wait(&ctl->o_full[mt], k & 1, abort, p.err);
             if (!__all_sync(0xffffffffu, w_ok)) break;
             tc_fence_after();
-            __nv_bfloat16* orow = p.out + ((size_t)(un.b * p.n + t) * kH + (r & 63)) * kD;
+            __nv_bfloat16* orow = p.out + ((un.tok0 + t) * kH + (r & 63)) * kD;
             if (g.T > 0) {
                 const float inv = st.lr > 0.0f ? 1.0f / st.lr : 0.0f;
 #pragma unroll
@@ -736,12 +766,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     }
                 }
                 if (row_ok && p.lse)
-                    p.lse[(size_t)(un.b * p.n + t) * kH + (r & 63)] =
+                    p.lse[(un.tok0 + t) * kH + (r & 63)] =
                         st.le > 0.0f ? (st.m + log2f(st.le)) / kLog2e : -INFINITY;
             } else if (row_ok) {
                 // no key at all: o = 0, lse = -inf
                 for (int i = 0; i < kD; i += 8) *reinterpret_cast<uint4*>(orow + i) = make_uint4(0, 0, 0, 0);
-                if (p.lse) p.lse[(size_t)(un.b * p.n + t) * kH + (r & 63)] = -INFINITY;
+                if (p.lse) p.lse[(un.tok0 + t) * kH + (r & 63)] = -INFINITY;
             }
             tc_fence_before();
             mbar_arrive(&ctl->o_free[mt]);
@@ -817,11 +847,21 @@ cudaError_t launch_attention_tc(const AttnArgs& a, uint32_t* err, cudaStream_t s
     p.out = static_cast<__nv_bfloat16*>(a.out);
     p.lse = a.lse_out;
     p.err = err;
+    int units = a.B * ((a.n_q + kTokens - 1) / kTokens);
+    if (a.vl) {                                     // packed: units per sequence
+        p.vl = *a.vl;
+        p.vl.uoff[0] = 0;
+        for (int q = 0; q < p.vl.S; ++q)
+            p.vl.uoff[q + 1] = p.vl.uoff[q] + (p.vl.tok[q + 1] - p.vl.tok[q] + kTokens - 1) / kTokens;
+        units = p.vl.uoff[p.vl.S];
+        if (units == 0) return cudaSuccess;
+    } else {
+        p.vl.S = 0;
+    }
     const size_t smem = kSmemFixed + (a.dense ? 0 : (size_t)kTokens * a.topk * sizeof(int));
     cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    const int units = a.B * ((a.n_q + kTokens - 1) / kTokens);
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = units < sms ? units : sms;     // persistent: one CTA per SM

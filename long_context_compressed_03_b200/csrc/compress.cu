@@ -25,21 +25,35 @@
 namespace csa {
 namespace {
 
+// The kernel's arguments: the call's, plus the packed-sequence map by value.
+struct CompressKArgs : CompressArgs {
+    VarlenMap map;
+};
+
 constexpr int kThreads = 256;
 constexpr int kTile = 64;   // entries per CTA
 constexpr int kKC = 32;     // rows of W staged per step
 
 template <typename Tin, int OUT>
-__global__ void __launch_bounds__(kThreads) compress_kernel(CompressArgs a) {
+__global__ void __launch_bounds__(kThreads) compress_kernel(CompressKArgs a) {
     extern __shared__ float smem[];
-    const int d_in = a.d_in, d_out = a.d_out, m = a.m, n = a.n, N_c = a.N_c;
+    const int d_in = a.d_in, d_out = a.d_out, m = a.m;
     const int b = blockIdx.y;
+    // element b (or packed sequence b): its tokens start at tok0, its entries at ent0
+    size_t tok0 = (size_t)b * a.n, ent0 = (size_t)b * a.N_c;
+    int N_c = a.N_c;
+    if (a.map.S) {
+        tok0 = (size_t)a.map.tok[b];
+        ent0 = (size_t)a.map.ent[b];
+        N_c = (a.map.tok[b + 1] - a.map.tok[b]) / m;
+    }
     const int i0 = blockIdx.x * kTile;
+    if (i0 >= N_c) return;                         // a shorter packed sequence
     const int ne = min(kTile, N_c - i0);
     float* pooled = smem;                          // [kTile][d_in]
     float* wst = pooled + kTile * d_in;            // [kKC][128]
     float* outs = wst + kKC * 128;                 // [kTile][d_out]
-    const Tin* x = static_cast<const Tin*>(a.x) + (size_t)b * n * d_in;
+    const Tin* x = static_cast<const Tin*>(a.x) + tok0 * d_in;
     const Tin* W = static_cast<const Tin*>(a.W);
     const int tid = threadIdx.x;
 
@@ -108,12 +122,14 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(CompressArgs a) {
     }
     __syncthreads();
 
-    store_entry_rows<OUT, kThreads>(outs, ne, d_out, a.out, a.out_row_scale, (size_t)b * N_c + i0,
-                                    a.hnorm);
+    store_entry_rows<OUT, kThreads>(outs, ne, d_out, a.out, a.out_row_scale, ent0 + i0, a.hnorm);
 }
 
 template <typename Tin, int OUT>
-cudaError_t launch_t(const CompressArgs& a, cudaStream_t s) {
+cudaError_t launch_t(const CompressArgs& args, cudaStream_t s) {
+    CompressKArgs a;
+    static_cast<CompressArgs&>(a) = args;
+    if (args.vl) a.map = *args.vl;
     const size_t smem = sizeof(float) * ((size_t)kTile * a.d_in + (size_t)kKC * 128 + (size_t)kTile * a.d_out);
     auto kern = compress_kernel<Tin, OUT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

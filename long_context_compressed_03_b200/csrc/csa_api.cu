@@ -3,6 +3,7 @@
 // Every entry point validates its arguments on the host, maps them onto the
 // internal launch structs and launches on the caller's stream.  Nothing is
 // allocated, nothing is synchronised, no exception or abort crosses the ABI.
+#include <algorithm>
 #include <atomic>
 #include <cstdarg>
 #include <cstdio>
@@ -65,6 +66,13 @@ csa_status_t from_cuda(cudaError_t e, const char* what, const char* why) {
 #define REQUIRE_ALIGNED(p, name) \
     do {                         \
         if ((p) && !aligned16(p)) return fail(CSA_ERR_MISALIGNED, "%s is not 16-byte aligned", name); \
+    } while (0)
+// Per-element arrays (scales, weights, indices, positions, counts, LSE,
+// block tables) are read and written one element at a time: 4-byte alignment.
+#define REQUIRE_ALIGNED4(p, name) \
+    do {                          \
+        if ((p) && (reinterpret_cast<uintptr_t>(p) & 3u)) \
+            return fail(CSA_ERR_MISALIGNED, "%s is not 4-byte aligned", name); \
     } while (0)
 
 bool is_dt(int d) {
@@ -130,15 +138,15 @@ csa_status_t csa_compress(const void* x, int x_dt, int B, int n, int d_in, const
         return fail(CSA_ERR_UNSUPPORTED, "csa_compress: the Hadamard fp8 type needs d_out a power of two");
     if (out_dt == CSA_DT_F32 && x_dt != CSA_DT_F32)
         return fail(CSA_ERR_UNSUPPORTED, "csa_compress: F32 output needs F32 input");
-    REQUIRE(is_fp8(out_dt) == (out_row_scale != nullptr),
-            "csa_compress: out_row_scale is required for E4M3 output and must be NULL otherwise");
     const int N_c = n / m;
+    REQUIRE((long)B * N_c == 0 || is_fp8(out_dt) == (out_row_scale != nullptr),
+            "csa_compress: out_row_scale is required for E4M3 output and must be NULL otherwise");
     if ((long)B * N_c == 0) return ok();
     REQUIRE(x && W && out, "csa_compress: null tensor pointer");
     REQUIRE_ALIGNED(x, "x");
     REQUIRE_ALIGNED(W, "W");
     REQUIRE_ALIGNED(out, "out");
-    REQUIRE_ALIGNED(out_row_scale, "out_row_scale");
+    REQUIRE_ALIGNED4(out_row_scale, "out_row_scale");
     csa::CompressArgs a{x, x_dt, B, n, d_in, W, d_out, m, overlap, out, out_dt, out_row_scale, N_c,
                         hadamard_norm(d_out)};
     const char* why = nullptr;
@@ -160,17 +168,17 @@ csa_status_t csa_compress_gated(const void* x, int x_dt, int B, int n, int d_in,
         return fail(CSA_ERR_UNSUPPORTED, "csa_compress_gated: the Hadamard fp8 type needs d_out a power of two");
     if (out_dt == CSA_DT_F32 && x_dt != CSA_DT_F32)
         return fail(CSA_ERR_UNSUPPORTED, "csa_compress_gated: F32 output needs F32 input");
-    REQUIRE(is_fp8(out_dt) == (out_row_scale != nullptr),
-            "csa_compress_gated: out_row_scale is required for E4M3 output and must be NULL otherwise");
     const int N_c = n / m;
+    REQUIRE((long)B * N_c == 0 || is_fp8(out_dt) == (out_row_scale != nullptr),
+            "csa_compress_gated: out_row_scale is required for E4M3 output and must be NULL otherwise");
     if ((long)B * N_c == 0) return ok();
     REQUIRE(x && W_kv && W_gate && ape && out, "csa_compress_gated: null tensor pointer");
     REQUIRE_ALIGNED(x, "x");
     REQUIRE_ALIGNED(W_kv, "W_kv");
     REQUIRE_ALIGNED(W_gate, "W_gate");
-    REQUIRE_ALIGNED(ape, "ape");
+    REQUIRE_ALIGNED4(ape, "ape");
     REQUIRE_ALIGNED(out, "out");
-    REQUIRE_ALIGNED(out_row_scale, "out_row_scale");
+    REQUIRE_ALIGNED4(out_row_scale, "out_row_scale");
     csa::GatedArgs a{x, x_dt, B, n, d_in, W_kv, W_gate, ape, d_out, m, overlap, out, out_dt,
                      out_row_scale, N_c, hadamard_norm(d_out)};
     const char* why = nullptr;
@@ -194,16 +202,16 @@ static csa_status_t compress_append_impl(const void* x_new, int x_dt, int B, int
         return fail(CSA_ERR_UNSUPPORTED, "csa_compress_append: the Hadamard fp8 type needs d_out a power of two");
     if (out_dt == CSA_DT_F32 && x_dt != CSA_DT_F32)
         return fail(CSA_ERR_UNSUPPORTED, "csa_compress_append: F32 output needs F32 input");
-    REQUIRE(is_fp8(out_dt) == (cache_scale != nullptr),
+    REQUIRE((long)B * N_cap == 0 || is_fp8(out_dt) == (cache_scale != nullptr),
             "csa_compress_append: cache_scale is required for E4M3 output and must be NULL otherwise");
     if (B == 0) return ok();
     REQUIRE(x_new && W && pos && state, "csa_compress_append: null pointer");
     REQUIRE(cache || N_cap == 0, "csa_compress_append: null cache");
     REQUIRE_ALIGNED(x_new, "x_new");
     REQUIRE_ALIGNED(W, "W");
-    REQUIRE_ALIGNED(state, "state");
+    REQUIRE_ALIGNED4(state, "state");
     REQUIRE_ALIGNED(cache, "cache");
-    REQUIRE_ALIGNED(cache_scale, "cache_scale");
+    REQUIRE_ALIGNED4(cache_scale, "cache_scale");
     csa::AppendArgs a{x_new, x_dt, B, d_in, W, d_out, m, overlap, pos, state, cache, out_dt,
                       cache_scale, N_cap, n_entries, hadamard_norm(d_out), pm};
     const char* why = nullptr;
@@ -224,9 +232,9 @@ static csa_status_t indexer_impl(const void* qI, int qI_dt, const float* qI_scal
     if (d_I % 16) return fail(CSA_ERR_UNSUPPORTED, "csa_indexer_topk: d_I must be a multiple of 16");
     if (qI_dt == CSA_DT_E4M3_HADAMARD)
         return fail(CSA_ERR_UNSUPPORTED, "csa_indexer_topk: give rotated query codes as CSA_DT_E4M3");
-    REQUIRE((qI_dt == CSA_DT_E4M3) == (qI_scale != nullptr),
+    REQUIRE((long)B * n_q == 0 || (qI_dt == CSA_DT_E4M3) == (qI_scale != nullptr),
             "csa_indexer_topk: qI_scale is required iff qI is E4M3");
-    REQUIRE(is_fp8(kI_dt) == (kI_scale != nullptr),
+    REQUIRE((long)B * N_cap == 0 || is_fp8(kI_dt) == (kI_scale != nullptr),
             "csa_indexer_topk: kI_scale is required iff kI is E4M3");
     if (kI_dt == CSA_DT_E4M3_HADAMARD && !pow2(d_I))
         return fail(CSA_ERR_UNSUPPORTED, "csa_indexer_topk: Hadamard keys need d_I a power of two");
@@ -235,12 +243,12 @@ static csa_status_t indexer_impl(const void* qI, int qI_dt, const float* qI_scal
     REQUIRE(kI || N_cap == 0, "csa_indexer_topk: null kI");
     REQUIRE_ALIGNED(qI, "qI");
     REQUIRE_ALIGNED(kI, "kI");
-    REQUIRE_ALIGNED(idx_out, "idx_out");
-    REQUIRE_ALIGNED(qI_scale, "qI_scale");
-    REQUIRE_ALIGNED(qI_weight, "qI_weight");
-    REQUIRE_ALIGNED(kI_scale, "kI_scale");
-    REQUIRE_ALIGNED(n_entries, "n_entries");
-    REQUIRE_ALIGNED(q_pos, "q_pos");
+    REQUIRE_ALIGNED4(idx_out, "idx_out");
+    REQUIRE_ALIGNED4(qI_scale, "qI_scale");
+    REQUIRE_ALIGNED4(qI_weight, "qI_weight");
+    REQUIRE_ALIGNED4(kI_scale, "kI_scale");
+    REQUIRE_ALIGNED4(n_entries, "n_entries");
+    REQUIRE_ALIGNED4(q_pos, "q_pos");
     csa::IndexerArgs a{qI, qI_dt, qI_scale, kI, kI_dt, kI_scale, B, n_q, H_I, d_I, N_cap,
                        n_entries, q_pos, m, topk, idx_out, hadamard_norm(d_I), qI_weight, pm};
     const char* why = nullptr;
@@ -257,7 +265,7 @@ static csa_status_t page_map(const char* name, int B, const int* block_table, in
     REQUIRE((long)max_pages * page_size <= (1L << 30), "%s: max_pages * page_size above 2^30", name);
     REQUIRE((long)num_pages * page_size <= (1L << 31) - 1, "%s: page pool above 2^31 - 1 rows", name);
     REQUIRE(block_table || B == 0 || max_pages == 0, "%s: null block_table", name);
-    REQUIRE_ALIGNED(block_table, "block_table");
+    REQUIRE_ALIGNED4(block_table, "block_table");
     int shift = 0;
     while ((1 << shift) < page_size) ++shift;
     pm->bt = block_table;
@@ -330,12 +338,12 @@ static csa_status_t attention_common(const char* name, csa::AttnArgs& a, void* s
     REQUIRE_ALIGNED(a.kv_c, "kv_c");
     REQUIRE_ALIGNED(a.kv_raw, "kv_raw");
     REQUIRE_ALIGNED(a.out, "out");
-    REQUIRE_ALIGNED(a.lse_out, "lse_out");
-    REQUIRE_ALIGNED(a.idx, "idx");
-    REQUIRE_ALIGNED(a.raw_pos0, "raw_pos0");
-    REQUIRE_ALIGNED(a.raw_len, "raw_len");
-    REQUIRE_ALIGNED(a.q_pos, "q_pos");
-    REQUIRE_ALIGNED(a.n_entries, "n_entries");
+    REQUIRE_ALIGNED4(a.lse_out, "lse_out");
+    REQUIRE_ALIGNED4(a.idx, "idx");
+    REQUIRE_ALIGNED4(a.raw_pos0, "raw_pos0");
+    REQUIRE_ALIGNED4(a.raw_len, "raw_len");
+    REQUIRE_ALIGNED4(a.q_pos, "q_pos");
+    REQUIRE_ALIGNED4(a.n_entries, "n_entries");
     if (!(a.scale > 0.0f)) a.scale = 1.0f / sqrtf((float)a.D);
     const char* why = nullptr;
     return from_cuda(csa::launch_attention(a, static_cast<cudaStream_t>(stream), &why), name, why);
@@ -397,6 +405,250 @@ csa_status_t hca_dense_attn_paged(const void* q, int dt, int B, int n_q, int H, 
     csa::AttnArgs a{q, dt, B, n_q, H, D, kv_c_pages, N_cap, nullptr, 0, n_entries, m, 1, kv_raw,
                     L_raw, raw_pos0, raw_len, window, q_pos, softmax_scale, out, lse_out, pm};
     return attention_common("hca_dense_attn_paged", a, stream);
+}
+
+// ------------------------------------------------------------------ varlen
+// Packed sequences: sequence s owns tokens [cu[s], cu[s+1]) of the packed
+// token dimension and entries [e(s), e(s+1)) of the packed compressed
+// dimension, e(s) = sum over earlier sequences of floor(len/m).  Each call
+// validates every sequence first, then launches the per-sequence kernels on
+// the stream, so nothing is launched on a validation error.
+
+static size_t dt_bytes(int dt) { return dt == CSA_DT_F32 ? 4 : (dt == CSA_DT_BF16 ? 2 : 1); }
+static bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+
+static csa_status_t check_cu(const char* name, int S, const int* cu, int m) {
+    REQUIRE(S >= 0, "%s: negative S", name);
+    REQUIRE(m >= 1, "%s: m must be >= 1", name);
+    REQUIRE(cu || S == 0, "%s: null cu_seqlens", name);
+    if (S == 0) return ok();
+    REQUIRE(cu[0] == 0, "%s: cu_seqlens[0] must be 0", name);
+    for (int s = 0; s < S; ++s)
+        REQUIRE(cu[s + 1] >= cu[s], "%s: cu_seqlens must be non-decreasing (at %d)", name, s);
+    return ok();
+}
+
+int csa_varlen_entry_offsets(const int* cu_seqlens, int S, int m, int* entry_offsets) {
+    if (S < 0 || m < 1 || !entry_offsets || (S > 0 && !cu_seqlens)) return -1;
+    long e = 0;
+    entry_offsets[0] = 0;
+    for (int s = 0; s < S; ++s) {
+        e += (cu_seqlens[s + 1] - cu_seqlens[s]) / m;
+        if (e > 0x7fffffffL) return -1;
+        entry_offsets[s + 1] = (int)e;
+    }
+    return (int)e;
+}
+
+#define PTR_AT(p, elems, bytes) \
+    ((p) ? static_cast<const void*>(static_cast<const uint8_t*>(p) + (size_t)(elems) * (bytes)) : nullptr)
+#define MPTR_AT(p, elems, bytes) \
+    ((p) ? static_cast<void*>(static_cast<uint8_t*>(p) + (size_t)(elems) * (bytes)) : nullptr)
+
+csa_status_t csa_compress_varlen(const void* x, int x_dt, int S, const int* cu_seqlens, int d_in,
+                                 const void* W, int d_out, int m, int overlap, void* out,
+                                 int out_dt, float* out_row_scale, void* stream) {
+    const char* name = "csa_compress_varlen";
+    csa_status_t st = check_cu(name, S, cu_seqlens, m);
+    if (st != CSA_OK) return st;
+    REQUIRE(is_dt(x_dt) && is_dt(out_dt), "%s: unknown dtype", name);
+    const long T = S > 0 ? cu_seqlens[S] : 0;
+    // the shared arguments, once (a call with no batch launches nothing)
+    st = csa_compress(x, x_dt, 0, 0, d_in, W, d_out, m, overlap, out, out_dt, out_row_scale, stream);
+    if (st != CSA_OK) return st;
+    REQUIRE(T == 0 || (x && W && out), "%s: null tensor pointer", name);
+    long E = 0;
+    for (int s = 0; s < S; ++s) E += (cu_seqlens[s + 1] - cu_seqlens[s]) / m;
+    REQUIRE(E == 0 || is_fp8(out_dt) == (out_row_scale != nullptr),
+            "%s: out_row_scale is required for E4M3 output and must be NULL otherwise", name);
+    for (int pass = 0; pass < 2; ++pass) {          // pass 0 validates, pass 1 launches
+        if (pass == 1 && S <= csa::kMaxVarlenSeqs) {   // one launch, offsets by value
+            csa::VarlenMap map;
+            map.S = S;
+            int max_nc = 0;
+            for (int s = 0; s <= S; ++s) {
+                map.tok[s] = cu_seqlens[s];
+                map.ent[s] = s == 0 ? 0 : map.ent[s - 1] + (cu_seqlens[s] - cu_seqlens[s - 1]) / m;
+                if (s > 0) max_nc = std::max(max_nc, (cu_seqlens[s] - cu_seqlens[s - 1]) / m);
+            }
+            if (max_nc == 0) return ok();
+            int max_len = 0;
+            for (int s = 0; s < S; ++s) max_len = std::max(max_len, cu_seqlens[s + 1] - cu_seqlens[s]);
+            csa::CompressArgs a{x, x_dt, S, max_len, d_in, W, d_out, m, overlap, out, out_dt,
+                                out_row_scale, max_nc, hadamard_norm(d_out), &map};
+            const char* why = nullptr;
+            return from_cuda(csa::launch_compress(a, static_cast<cudaStream_t>(stream), &why), name,
+                             why);
+        }
+        long e = 0;
+        for (int s = 0; s < S; ++s) {
+            const int L = cu_seqlens[s + 1] - cu_seqlens[s];
+            const void* xs = PTR_AT(x, (long)cu_seqlens[s] * d_in, dt_bytes(x_dt));
+            void* os = MPTR_AT(out, e * d_out, dt_bytes(out_dt));
+            float* ss = out_row_scale ? out_row_scale + e : nullptr;
+            if (L / m == 0) continue;
+            if (pass == 0) {
+                if (!(aligned16(xs) && aligned16(os) && (!ss || aligned4(ss))))
+                    return fail(CSA_ERR_MISALIGNED, "%s: sequence %d's rows are not 16-byte aligned "
+                                "(token offset %d)", name, s, cu_seqlens[s]);
+            } else {
+                st = csa_compress(xs, x_dt, 1, L, d_in, W, d_out, m, overlap, os, out_dt, ss, stream);
+                if (st != CSA_OK) return st;
+            }
+            e += L / m;
+        }
+    }
+    return ok();
+}
+
+csa_status_t csa_indexer_topk_varlen(const void* qI, int qI_dt, const float* qI_scale,
+                                     const float* qI_weight, const void* kI, int kI_dt,
+                                     const float* kI_scale, int S, const int* cu_seqlens, int H_I,
+                                     int d_I, int m, int topk, int* idx_out, void* stream) {
+    const char* name = "csa_indexer_topk_varlen";
+    csa_status_t st = check_cu(name, S, cu_seqlens, m);
+    if (st != CSA_OK) return st;
+    REQUIRE(is_dt(qI_dt) && is_dt(kI_dt), "%s: unknown dtype", name);
+    st = csa_indexer_topk(qI, qI_dt, qI_scale, qI_weight, kI, kI_dt, kI_scale, 0, 0, H_I, d_I, 0,
+                          nullptr, nullptr, m, topk, idx_out, stream);
+    if (st != CSA_OK) return st;
+    REQUIRE(S == 0 || cu_seqlens[S] == 0 || (qI && idx_out), "%s: null tensor pointer", name);
+    {
+        long E = 0;
+        for (int s = 0; s < S; ++s) E += (cu_seqlens[s + 1] - cu_seqlens[s]) / m;
+        const long T = S > 0 ? cu_seqlens[S] : 0;
+        REQUIRE(E == 0 || kI, "%s: null kI", name);
+        REQUIRE(T == 0 || (qI_dt == CSA_DT_E4M3) == (qI_scale != nullptr),
+                "%s: qI_scale is required iff qI is E4M3", name);
+        REQUIRE(E == 0 || is_fp8(kI_dt) == (kI_scale != nullptr),
+                "%s: kI_scale is required iff kI is E4M3", name);
+    }
+    for (int pass = 0; pass < 2; ++pass) {
+        if (pass == 1 && S <= csa::kMaxVarlenSeqs && kI_dt != CSA_DT_F32) {
+            csa::VarlenMap map;
+            map.S = S;
+            int max_len = 0, max_n = 0;
+            for (int s = 0; s <= S; ++s) {
+                map.tok[s] = cu_seqlens[s];
+                map.ent[s] = s == 0 ? 0 : map.ent[s - 1] + (cu_seqlens[s] - cu_seqlens[s - 1]) / m;
+                if (s > 0) {
+                    max_len = std::max(max_len, cu_seqlens[s] - cu_seqlens[s - 1]);
+                    max_n = std::max(max_n, (cu_seqlens[s] - cu_seqlens[s - 1]) / m);
+                }
+            }
+            if (max_len == 0) return ok();
+            csa::IndexerArgs a{qI, qI_dt, qI_scale, kI, kI_dt, kI_scale, 1, max_len, H_I, d_I,
+                               map.ent[S], nullptr, nullptr, m, topk, idx_out, hadamard_norm(d_I),
+                               qI_weight};
+            a.vl = &map;
+            const cudaError_t ce = csa::launch_indexer_packed(a, max_n, static_cast<cudaStream_t>(stream));
+            if (ce != cudaErrorNotSupported) return from_cuda(ce, name, nullptr);
+            // otherwise: one launch per sequence below
+        }
+        long e = 0;
+        for (int s = 0; s < S; ++s) {
+            const int t0 = cu_seqlens[s], L = cu_seqlens[s + 1] - t0, N = L / m;
+            const void* q = PTR_AT(qI, (long)t0 * H_I * d_I, dt_bytes(qI_dt));
+            const float* qs = qI_scale ? qI_scale + (long)t0 * H_I : nullptr;
+            const float* qw = qI_weight ? qI_weight + (long)t0 * H_I : nullptr;
+            const void* k = PTR_AT(kI, e * d_I, dt_bytes(kI_dt));
+            const float* ks = kI_scale ? kI_scale + e : nullptr;
+            int* idx = idx_out ? idx_out + (long)t0 * topk : nullptr;
+            if (pass == 0 && L > 0) {
+                if (!(aligned16(q) && aligned16(k) && aligned4(idx) && (!qs || aligned4(qs)) &&
+                      (!qw || aligned4(qw)) && (!ks || aligned4(ks))))
+                    return fail(CSA_ERR_MISALIGNED, "%s: sequence %d's rows are not 16-byte aligned "
+                                "(token offset %d, entry offset %ld)", name, s, t0, e);
+            }
+            if (pass == 1 && L > 0) {
+                st = csa_indexer_topk(q, qI_dt, qs, qw, k, kI_dt, ks, 1, L, H_I, d_I, N, nullptr,
+                                      nullptr, m, topk, idx, stream);
+                if (st != CSA_OK) return st;
+            }
+            e += N;
+        }
+    }
+    return ok();
+}
+
+static csa_status_t attn_varlen(const char* name, bool dense, const void* q, int dt, int S,
+                                const int* cu, int H, int D, const void* kv_c, int m,
+                                const int* idx, int topk, const void* kv_raw, int window,
+                                float softmax_scale, void* out, float* lse_out, void* stream) {
+    csa_status_t st = check_cu(name, S, cu, m);
+    if (st != CSA_OK) return st;
+    REQUIRE(is_dt(dt), "%s: unknown dtype", name);
+    st = dense ? hca_dense_attn(q, dt, 0, 0, H, D, kv_c, 0, nullptr, m, kv_raw, 0, nullptr, nullptr,
+                                window, nullptr, softmax_scale, out, lse_out, stream)
+               : csa_sparse_attn(q, dt, 0, 0, H, D, kv_c, 0, idx, topk, kv_raw, 0, nullptr, nullptr,
+                                 window, nullptr, softmax_scale, out, lse_out, stream);
+    if (st != CSA_OK) return st;
+    long E = 0;
+    for (int s = 0; s < S; ++s) E += (cu[s + 1] - cu[s]) / m;
+    REQUIRE(S == 0 || cu[S] == 0 || (q && out && kv_raw && (kv_c || E == 0) && (idx || topk == 0)),
+            "%s: null tensor pointer", name);
+    for (int pass = 0; pass < 2; ++pass) {
+        if (pass == 1 && S <= csa::kMaxVarlenSeqs) {   // one launch, offsets by value
+            csa::VarlenMap map;
+            map.S = S;
+            for (int s = 0; s <= S; ++s) {
+                map.tok[s] = cu[s];
+                map.ent[s] = s == 0 ? 0 : map.ent[s - 1] + (cu[s] - cu[s - 1]) / m;
+            }
+            const int T = cu[S];
+            if (T == 0) return ok();
+            csa::AttnArgs a{q, dt, 1, T, H, D, kv_c, map.ent[S], idx, dense ? 0 : topk,
+                            nullptr, m, dense ? 1 : 0, kv_raw, T, nullptr, nullptr, window, nullptr,
+                            softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf((float)D), out,
+                            lse_out};
+            a.vl = &map;
+            const cudaError_t ce = csa::launch_attention_packed(a, static_cast<cudaStream_t>(stream));
+            if (ce != cudaErrorNotSupported) return from_cuda(ce, name, nullptr);
+            // otherwise: one launch per sequence below
+        }
+        long e = 0;
+        for (int s = 0; s < S; ++s) {
+            const int t0 = cu[s], L = cu[s + 1] - t0, N = L / m;
+            const size_t eb = dt_bytes(dt);
+            const void* qs = PTR_AT(q, (long)t0 * H * D, eb);
+            const void* kc = PTR_AT(kv_c, e * D, eb);
+            const void* kr = PTR_AT(kv_raw, (long)t0 * D, eb);
+            const int* ix = idx ? idx + (long)t0 * topk : nullptr;
+            void* os = MPTR_AT(out, (long)t0 * H * D, eb);
+            float* ls = lse_out ? lse_out + (long)t0 * H : nullptr;
+            if (pass == 0 && L > 0) {
+                if (!(aligned16(qs) && aligned16(kc) && aligned16(kr) && aligned16(os) &&
+                      (!ix || aligned4(ix)) && (!ls || aligned4(ls))))
+                    return fail(CSA_ERR_MISALIGNED, "%s: sequence %d's rows are not 16-byte aligned "
+                                "(token offset %d, entry offset %ld)", name, s, t0, e);
+            }
+            if (pass == 1 && L > 0) {
+                st = dense ? hca_dense_attn(qs, dt, 1, L, H, D, kc, N, nullptr, m, kr, L, nullptr,
+                                            nullptr, window, nullptr, softmax_scale, os, ls, stream)
+                           : csa_sparse_attn(qs, dt, 1, L, H, D, kc, N, ix, topk, kr, L, nullptr,
+                                             nullptr, window, nullptr, softmax_scale, os, ls,
+                                             stream);
+                if (st != CSA_OK) return st;
+            }
+            e += N;
+        }
+    }
+    return ok();
+}
+
+csa_status_t csa_sparse_attn_varlen(const void* q, int dt, int S, const int* cu_seqlens, int H,
+                                    int D, const void* kv_c, int m, const int* idx, int topk,
+                                    const void* kv_raw, int window, float softmax_scale, void* out,
+                                    float* lse_out, void* stream) {
+    return attn_varlen("csa_sparse_attn_varlen", false, q, dt, S, cu_seqlens, H, D, kv_c, m, idx,
+                       topk, kv_raw, window, softmax_scale, out, lse_out, stream);
+}
+
+csa_status_t hca_dense_attn_varlen(const void* q, int dt, int S, const int* cu_seqlens, int H,
+                                   int D, const void* kv_c, int m, const void* kv_raw, int window,
+                                   float softmax_scale, void* out, float* lse_out, void* stream) {
+    return attn_varlen("hca_dense_attn_varlen", true, q, dt, S, cu_seqlens, H, D, kv_c, m, nullptr,
+                       0, kv_raw, window, softmax_scale, out, lse_out, stream);
 }
 
 }  // extern "C"

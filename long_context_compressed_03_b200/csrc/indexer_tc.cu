@@ -75,6 +75,7 @@ struct IdxParams {
     const int* n_entries;
     int* idx_out;
     uint32_t* err;
+    VarlenMap vl;              // packed sequences (vl.S > 0): grid.y = sequence
 };
 
 struct __align__(8) Ctrl {
@@ -243,13 +244,30 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
     Ctrl* ctl = reinterpret_cast<Ctrl*>(reinterpret_cast<uint8_t*>(rs) + sizeof(RowState));
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int tiles_per_seq = (p.n + kRows - 1) / kRows;
-    // heavy tiles (late queries see more entries) first
-    const int tile = gridDim.x - 1 - blockIdx.x;
-    const int b = tile / tiles_per_seq;
-    const int t0 = (tile - b * tiles_per_seq) * kRows;
-    const int ne = clampi(p.n_entries ? p.n_entries[b] : p.N_cap, 0, p.N_cap);
-    const int t_last = min(t0 + kRows - 1, p.n - 1);
+    // this CTA's 128 queries: element (or packed sequence) b, positions
+    // t0 .. of its slen; its rows start at token tok0 and entry ent0.  Heavy
+    // tiles (late queries see more entries) first.
+    int b, t0, slen, ne;
+    size_t tok0, ent0;
+    if (p.vl.S) {
+        b = blockIdx.y;
+        tok0 = (size_t)p.vl.tok[b];
+        ent0 = (size_t)p.vl.ent[b];
+        slen = p.vl.tok[b + 1] - p.vl.tok[b];
+        ne = slen / p.m;
+        t0 = (gridDim.x - 1 - blockIdx.x) * kRows;
+        if (t0 >= slen) return;    // a shorter sequence: nothing set up yet, the whole CTA leaves
+    } else {
+        const int tiles_per_seq = (p.n + kRows - 1) / kRows;
+        const int tile = gridDim.x - 1 - blockIdx.x;
+        b = tile / tiles_per_seq;
+        t0 = (tile - b * tiles_per_seq) * kRows;
+        slen = p.n;
+        tok0 = (size_t)b * p.n;
+        ent0 = (size_t)b * p.N_cap;
+        ne = clampi(p.n_entries ? p.n_entries[b] : p.N_cap, 0, p.N_cap);
+    }
+    const int t_last = min(t0 + kRows - 1, slen - 1);
     const int Vmax = min((t_last + 1) / p.m, ne);
     const int nchunks = (Vmax + kN - 1) / kN;
     volatile int* abort = &ctl->abort;
@@ -276,7 +294,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
     // rows: visibility and the query operand (one warp per (row, head) pair)
     for (int r = threadIdx.x; r < kRows; r += kThreads) {
         const int t = t0 + r;
-        const int V = (t < p.n) ? min((t + 1) / p.m, ne) : 0;
+        const int V = (t < slen) ? min((t + 1) / p.m, ne) : 0;
         rs->V[r] = V;
         rs->level[r] = 0;
         rs->prefix[r] = 0;
@@ -287,8 +305,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
     }
     for (int pair = warp; pair < kRows * kHeads; pair += kThreads / 32) {
         const int r = pair >> 2, h = pair & 3;
-        const int t = min(t0 + r, p.n - 1);
-        const size_t qrow = ((size_t)b * p.n + t) * p.H_I + h;
+        const int t = min(t0 + r, slen - 1);
+        const size_t qrow = (tok0 + t) * p.H_I + h;
         float v0 = 0.0f, v1 = 0.0f;   // elements 2*lane, 2*lane+1
         float qs = 1.0f;
         uint32_t packed;              // two output elements (fp8: 2 bytes; bf16: 4 bytes)
@@ -374,7 +392,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
                     const int slot = L % C::kStages, u = L / C::kStages;
                     if (u > 0 && !mbar_wait(&ctl->freeb[slot], (u - 1) & 1, abort, p.err)) break;
                     mbar_arrive_expect_tx(&ctl->full[slot], C::kBTile);
-                    tma_load_2d(sB + slot * C::kBTile, &tm_k, 0, b * p.N_cap + c * kN, &ctl->full[slot]);
+                    tma_load_2d(sB + slot * C::kBTile, &tm_k, 0, (int)ent0 + c * kN, &ctl->full[slot]);
                 }
             }
             __syncwarp();
@@ -414,7 +432,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
         } else {
             // ------------------------------------------------------------ epilogue
             const int V = rs->V[r];
-            const bool row_ok = t0 + r < p.n;
+            const bool row_ok = t0 + r < slen;
             const bool active = row_ok && V > p.topk && (rs->ready[r] == 0 || emit);
             const int level = rs->level[r];
             const int kind = emit ? kEmit : (level == 0 ? kHist0 : (level < 4 ? kHist32 : kHist64));
@@ -423,14 +441,14 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
             rc.prefix = rs->prefix[r];
             rc.sh = shift_of(level);
             rc.hrow = hist + r;
-            rc.orow = p.idx_out + ((size_t)b * p.n + min(t0 + r, p.n - 1)) * p.topk;
+            rc.orow = p.idx_out + (tok0 + min(t0 + r, slen - 1)) * p.topk;
             rc.list = list + r * kCap;
             rc.emitted = &rs->emitted[r];
             rc.listed = &rs->listed[r];
             rc.topk = p.topk;
 #pragma unroll
             for (int h = 0; h < kHeads; ++h) rc.qs[h] = 0.5f * rs->qs[r][h];   // exact: a power of two
-            const float* ksc = FP8 ? p.kI_scale + (size_t)b * p.N_cap : nullptr;
+            const float* ksc = FP8 ? p.kI_scale + ent0 : nullptr;
             // this lane's key scale for entry c*kN + lane, loaded one chunk ahead
             auto scale_of = [&](int c) -> float {
                 const int e = c * kN + lane;
@@ -483,8 +501,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
                         rs->level[r] = level + 1;
                     }
                 }
-            } else if (t0 + r < p.n) {
-                int* orow = p.idx_out + ((size_t)b * p.n + t0 + r) * p.topk;
+            } else if (t0 + r < slen) {
+                int* orow = p.idx_out + (tok0 + t0 + r) * p.topk;
                 if (V <= p.topk) {
                     for (int j = 0; j < p.topk; ++j) orow[j] = j < V ? j : -1;
                 } else {
@@ -517,8 +535,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
                 const int kk = p.topk;
                 for (int rr = ew; rr < kRows; rr += kGroups * 4) {
                     const int V = rs->V[rr];
-                    if (t0 + rr >= p.n || V <= kk) continue;
-                    int* orow = p.idx_out + ((size_t)b * p.n + t0 + rr) * kk;
+                    if (t0 + rr >= slen || V <= kk) continue;
+                    int* orow = p.idx_out + (tok0 + t0 + rr) * kk;
                     const int nw = (V + 31) >> 5;
                     for (int i = lane; i < nw; i += 32) bm[i] = 0u;
                     __syncwarp();
@@ -562,8 +580,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
     if (!need) {
         // every row takes all its visible entries
         for (int i = threadIdx.x; i < kRows; i += kThreads) {
-            if (t0 + i >= p.n) continue;
-            int* orow = p.idx_out + ((size_t)b * p.n + t0 + i) * p.topk;
+            if (t0 + i >= slen) continue;
+            int* orow = p.idx_out + (tok0 + t0 + i) * p.topk;
             const int V = rs->V[i];
             for (int j = 0; j < p.topk; ++j) orow[j] = j < V ? j : -1;
         }
@@ -647,7 +665,13 @@ cudaError_t launch_indexer_tc(const IndexerArgs& a, uint32_t* err, cudaStream_t 
     p.err = err;
     p.qw = a.qI_weight;
     const int tiles = (a.n_q + kRows - 1) / kRows;
-    const dim3 grid((unsigned)(a.B * tiles));
+    dim3 grid((unsigned)(a.B * tiles));
+    if (a.vl) {                       // packed: one row of tiles per sequence
+        p.vl = *a.vl;
+        grid = dim3((unsigned)tiles, (unsigned)a.vl->S);
+    } else {
+        p.vl.S = 0;
+    }
     cudaError_t e;
     if (fp8)
         e = a.qI_weight ? launch_k<true, true>(grid, tm, p, s) : launch_k<true, false>(grid, tm, p, s);

@@ -236,6 +236,16 @@ cudaError_t launch_t(const IndexerArgs& a, cudaStream_t s) {
 
 }  // namespace
 
+cudaError_t launch_indexer_packed(const IndexerArgs& a, int max_entries, cudaStream_t s) {
+    IndexerArgs shape = a;             // the per-sequence shape decides the kernel
+    shape.N_cap = max_entries;
+    if (a.vl == nullptr || a.pages.bt != nullptr || !indexer_tc_supported(shape))
+        return cudaErrorNotSupported;
+    uint32_t* err = device_error_word();
+    if (!err) return cudaErrorUnknown;
+    return launch_indexer_tc(a, err, s);
+}
+
 cudaError_t launch_indexer_topk(const IndexerArgs& a, cudaStream_t s, const char** why) {
     if (a.B <= 0 || a.n_q <= 0) return cudaSuccess;
     if (a.H_I > kMaxHeads || a.d_I > kMaxDim) {

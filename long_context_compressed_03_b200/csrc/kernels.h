@@ -25,6 +25,17 @@ __host__ __device__ __forceinline__ long cache_row(const PageMap& pm, int N_cap,
     return ((long)pg << pm.page_shift) + (s & ((1 << pm.page_shift) - 1));
 }
 
+// Packed sequences handed to one launch: sequence s owns tokens
+// [tok[s], tok[s+1]) and compressed entries [ent[s], ent[s+1]).  Passed by
+// value in the kernel parameters (no device buffer); S == 0: not packed.
+constexpr int kMaxVarlenSeqs = 128;
+struct VarlenMap {
+    int S = 0;
+    int tok[kMaxVarlenSeqs + 1];
+    int ent[kMaxVarlenSeqs + 1];
+    int uoff[kMaxVarlenSeqs + 1];   // prefill attention: first 4-token unit of each sequence
+};
+
 struct CompressArgs {
     const void* x; int x_dt;
     int B, n, d_in;
@@ -34,6 +45,7 @@ struct CompressArgs {
     float* out_row_scale;
     int N_c;
     float hnorm;               // fp32(1/sqrt(d_out)) for the Hadamard fp8 type
+    const VarlenMap* vl = nullptr;   // packed: B = S, n = longest, N_c = most entries
 };
 
 struct GatedArgs {
@@ -74,6 +86,8 @@ struct IndexerArgs {
     float hnorm;               // fp32(1/sqrt(d_I)): keys of the Hadamard fp8 type
     const float* qI_weight;    // [B, n_q, H_I] gate weights or NULL (all 1)
     PageMap pages;             // kI (and kI_scale) layout
+    const VarlenMap* vl = nullptr;   // packed (tensor-core kernel only): B = S, n_q = longest,
+                                     // N_cap = total entries
 };
 
 struct AttnArgs {
@@ -90,6 +104,8 @@ struct AttnArgs {
     float scale;
     void* out; float* lse_out;
     PageMap pages;             // kv_c layout
+    const VarlenMap* vl = nullptr;   // packed (tensor-core kernel only): B = 1, n_q = L_raw = T
+                                     // tokens, N_cap = total entries
 };
 
 // Device address of this library's error word on the current device (set by
@@ -121,6 +137,13 @@ void count_launch();
 // reason string when the configuration is unsupported (returned as
 // cudaErrorNotSupported).
 cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s, const char** why);
+// One launch over packed sequences (a.vl, a.B = 1, a.N_cap = total entries,
+// a.n_q = longest sequence), or cudaErrorNotSupported when the tensor-core
+// indexer does not serve the per-sequence shape (max_entries entries).
+cudaError_t launch_indexer_packed(const IndexerArgs& a, int max_entries, cudaStream_t s);
+// One launch over packed sequences (a.vl set), or cudaErrorNotSupported when
+// the tensor-core attention does not serve the shape.
+cudaError_t launch_attention_packed(const AttnArgs& a, cudaStream_t s);
 cudaError_t launch_compress_gated(const GatedArgs& a, cudaStream_t s, const char** why);
 cudaError_t launch_compress_append(const AppendArgs& a, cudaStream_t s, const char** why);
 cudaError_t launch_indexer_topk(const IndexerArgs& a, cudaStream_t s, const char** why);

@@ -224,6 +224,17 @@ def hca_prefill_inputs(w: Workload, seed: int = 0, n: int | None = None, B: int 
     return dict(q=q.to(dt), kv=kv.to(dt), W_c=W_c.to(dt))
 
 
+def varlen_lengths(total: int, S: int, multiple: int = 4, seed: int = 0) -> list[int]:
+    """A length mix for packed prefill: S weights ~ U(0.25, 1.75) scaled to
+    total tokens, rounded down to a multiple, the remainder given to the last
+    sequence."""
+    g = torch.Generator().manual_seed(seed)
+    w = 0.25 + 1.5 * torch.rand(S, generator=g, dtype=torch.float64)
+    lens = [int(x) // multiple * multiple for x in (w / w.sum() * total).tolist()]
+    lens[-1] += total - sum(lens)
+    return lens
+
+
 def indexer_variant_inputs(B: int, n: int, H_I: int, seed: int = 0):
     """Gate weights for the gated indexer: w [B, n, H_I] ~ N(0, 1) (any sign;
     the pages give no distribution)."""

@@ -213,6 +213,35 @@ def test_paged_entry_point_validation(lib):
     assert k(*args) == api.CSA_ERR_UNSUPPORTED        # fp8 attention operands
 
 
+def test_varlen_offsets_and_validation(lib):
+    cu = (ctypes.c_int * 4)(0, 5, 5, 13)
+    off = (ctypes.c_int * 4)()
+    assert lib.csa_varlen_entry_offsets(cu, 3, 4, off) == 3
+    assert list(off) == [0, 1, 1, 3]
+    assert lib.csa_varlen_entry_offsets(cu, 3, 0, off) == -1
+    f = lib.csa_indexer_topk_varlen
+    #       qI  dt sc   wt   kI   dt sc   S  cu  H  d   m  k  idx   stream
+    args = [FAKE, 1, None, None, FAKE, 1, None, 3, cu, 4, 64, 4, 8, FAKE, None]
+    bad = list(args); bad[8] = (ctypes.c_int * 4)(0, 5, 4, 13)    # decreasing
+    assert f(*bad) == api.CSA_ERR_INVALID_ARG
+    bad = list(args); bad[8] = (ctypes.c_int * 4)(1, 5, 5, 13)    # must start at 0
+    assert f(*bad) == api.CSA_ERR_INVALID_ARG
+    bad = list(args); bad[0] = ODD             # sequence 0's query rows off the 16-byte grid
+    assert f(*bad) == api.CSA_ERR_MISALIGNED
+    bad = list(args); bad[13] = None
+    assert f(*bad) == api.CSA_ERR_INVALID_ARG
+    ok = list(args); ok[7] = 0                 # no sequences: nothing to do
+    assert f(*ok) == api.CSA_OK
+    g = lib.csa_sparse_attn_varlen
+    #       q   dt S  cu  H   D    kv_c m  idx  k  raw  W  scale             out   lse   stream
+    args = [FAKE, 2, 3, cu, 64, 128, FAKE, 4, FAKE, 8, FAKE, 8, ctypes.c_float(0.0), FAKE, None, None]
+    assert g(*args) == api.CSA_ERR_UNSUPPORTED                    # fp8 attention operands
+    h = lib.csa_compress_varlen
+    #       x   dt S  cu  d_in W    d_out m  ov out  dt scale stream
+    args = [FAKE, 1, 3, cu, 64, FAKE, 64, 4, 1, FAKE, 1, FAKE, None]
+    assert h(*args) == api.CSA_ERR_INVALID_ARG                    # scales with bf16 output
+
+
 def test_attention_validation(lib):
     f = lib.csa_sparse_attn
     args = [FAKE, 1, 1, 8, 64, 128, FAKE, 16, FAKE, 4, FAKE, 8, None, None, 4, None,
