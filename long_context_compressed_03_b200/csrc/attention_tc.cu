@@ -138,9 +138,9 @@ struct Unit {
     int N;          // its compressed entries
     int L_raw;      // its raw rows
     int ne_dense;   // dense: entries it may see (n_entries, clamped)
-    size_t tok0;    // row of its token 0 in q / out / lse / idx
-    size_t ent0;    // row of its entry 0 in kv_c
-    size_t raw0;    // row of its raw position 0 in kv_raw
+    int tok0;       // row of its token 0 in q / out / lse / idx
+    int ent0;       // row of its entry 0 in kv_c
+    int raw0;       // row of its raw position 0 in kv_raw
 };
 __device__ __forceinline__ Unit unit_of(const TcParams& p, int u) {
     Unit r;
@@ -156,8 +156,8 @@ __device__ __forceinline__ Unit unit_of(const TcParams& p, int u) {
         r.N = r.n / p.m;
         r.L_raw = r.n;
         r.ne_dense = r.N;
-        r.tok0 = (size_t)p.vl.tok[lo];
-        r.ent0 = (size_t)p.vl.ent[lo];
+        r.tok0 = p.vl.tok[lo];
+        r.ent0 = p.vl.ent[lo];
         r.raw0 = r.tok0;
     } else {
         const int per = (p.n + kTokens - 1) / kTokens;
@@ -167,9 +167,9 @@ __device__ __forceinline__ Unit unit_of(const TcParams& p, int u) {
         r.N = p.N_cap;
         r.L_raw = p.L_raw;
         r.ne_dense = p.dense ? clampi(p.n_entries ? p.n_entries[r.b] : p.N_cap, 0, p.N_cap) : 0;
-        r.tok0 = (size_t)r.b * p.n;
-        r.ent0 = (size_t)r.b * p.N_cap;
-        r.raw0 = (size_t)r.b * p.L_raw;
+        r.tok0 = r.b * p.n;
+        r.ent0 = r.b * p.N_cap;
+        r.raw0 = r.b * p.L_raw;
     }
     return r;
 }
@@ -447,13 +447,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 for (int i = lt; i < kTokens * p.topk; i += kLoadThreads) {
                     const int tok = i / p.topk, c = i - tok * p.topk;
                     const int t = t0 + tok;
-                    sIdx[i] = (t < un.n) ? __ldg(p.idx + (un.tok0 + t) * p.topk + c) : -1;
+                    sIdx[i] = (t < un.n) ? __ldg(p.idx + (size_t)(un.tok0 + t) * p.topk + c) : -1;
                 }
             }
             named_sync(1, kLoadThreads);
             const int NL = total_loads(p, g);
             const int nc = p.dense ? g.Tc : 2 * g.Tc;
-            const uint8_t* kvc_rows = static_cast<const uint8_t*>(p.kv_c) + un.ent0 * (kD * 2);
+            const uint8_t* kvc_rows = static_cast<const uint8_t*>(p.kv_c) + (size_t)un.ent0 * (kD * 2);
             for (int L = 0; L < NL; ++L, ++Lg) {
                 const int slot = Lg % kStages, use = Lg / kStages;
                 uint8_t* dst = sK + slot * kTileBytes;
@@ -508,8 +508,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 } else {
                     if (lt == 0) {
                         const CUtensorMap* tm = (kind == 1) ? &tm_c : &tm_w;
-                        const int row = (kind == 1) ? (int)un.ent0 + chunk * kBN
-                                                    : (int)un.raw0 + g.p_lo + chunk * kBN;
+                        const int row = (kind == 1) ? un.ent0 + chunk * kBN
+                                                    : un.raw0 + g.p_lo + chunk * kBN;
                         mbar_arrive_expect_tx(&ctl->full[slot], kTileBytes);
                         for (int h = 0; h < 2; ++h)
                             tma_load_2d(dst + h * kHalf, tm, h * 64, row, &ctl->full[slot]);
@@ -534,7 +534,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             auto load_q = [&](int u) {
                 const Unit un = unit_of(p, u);
                 mbar_arrive_expect_tx(&ctl->bar_q, 2 * kTileBytes);
-                const int qrow = (int)(un.tok0 + un.t0) * kH;
+                const int qrow = (un.tok0 + un.t0) * kH;
                 for (int mt = 0; mt < 2; ++mt)
                     for (int h = 0; h < 2; ++h)
                         tma_load_2d(sQ + mt * kTileBytes + h * kHalf, &tm_q, h * 64, qrow + mt * kRows,
@@ -742,7 +742,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             w_ok = w_ok && mbar_wait(&ctl->o_full[mt], k & 1, abort, p.err);
             if (!__all_sync(0xffffffffu, w_ok)) break;
             tc_fence_after();
-            __nv_bfloat16* orow = p.out + ((un.tok0 + t) * kH + (r & 63)) * kD;
+            __nv_bfloat16* orow = p.out + ((size_t)(un.tok0 + t) * kH + (r & 63)) * kD;
             if (g.T > 0) {
                 const float inv = st.lr > 0.0f ? 1.0f / st.lr : 0.0f;
 #pragma unroll
@@ -766,12 +766,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     }
                 }
                 if (row_ok && p.lse)
-                    p.lse[(un.tok0 + t) * kH + (r & 63)] =
+                    p.lse[(size_t)(un.tok0 + t) * kH + (r & 63)] =
                         st.le > 0.0f ? (st.m + log2f(st.le)) / kLog2e : -INFINITY;
             } else if (row_ok) {
                 // no key at all: o = 0, lse = -inf
                 for (int i = 0; i < kD; i += 8) *reinterpret_cast<uint4*>(orow + i) = make_uint4(0, 0, 0, 0);
-                if (p.lse) p.lse[(un.tok0 + t) * kH + (r & 63)] = -INFINITY;
+                if (p.lse) p.lse[(size_t)(un.tok0 + t) * kH + (r & 63)] = -INFINITY;
             }
             tc_fence_before();
             mbar_arrive(&ctl->o_free[mt]);
