@@ -142,9 +142,10 @@ struct Unit {
     int ent0;       // row of its entry 0 in kv_c
     int raw0;       // row of its raw position 0 in kv_raw
 };
+template <bool PACKED>
 __device__ __forceinline__ Unit unit_of(const TcParams& p, int u) {
     Unit r;
-    if (p.vl.S) {
+    if constexpr (PACKED) {
         int lo = 0, hi = p.vl.S - 1;                  // the last sequence with uoff <= u
         while (lo < hi) {
             const int mid = (lo + hi + 1) >> 1;
@@ -160,26 +161,46 @@ __device__ __forceinline__ Unit unit_of(const TcParams& p, int u) {
         r.ent0 = p.vl.ent[lo];
         r.raw0 = r.tok0;
     } else {
+        // the other fields are derived from p and b where they are used
+        // (accessors below), so nothing extra stays live in registers
         const int per = (p.n + kTokens - 1) / kTokens;
         r.b = u / per;
         r.t0 = (u - r.b * per) * kTokens;
-        r.n = p.n;
-        r.N = p.N_cap;
-        r.L_raw = p.L_raw;
-        r.ne_dense = p.dense ? clampi(p.n_entries ? p.n_entries[r.b] : p.N_cap, 0, p.N_cap) : 0;
-        r.tok0 = r.b * p.n;
-        r.ent0 = r.b * p.N_cap;
-        r.raw0 = r.b * p.L_raw;
     }
     return r;
 }
 
+// A unit's fields: stored for packed sequences, derived from the call's
+// uniform shape otherwise.
+template <bool PACKED> __device__ __forceinline__ int u_n(const TcParams& p, const Unit& u) {
+    return PACKED ? u.n : p.n;
+}
+template <bool PACKED> __device__ __forceinline__ int u_N(const TcParams& p, const Unit& u) {
+    return PACKED ? u.N : p.N_cap;
+}
+template <bool PACKED> __device__ __forceinline__ int u_L_raw(const TcParams& p, const Unit& u) {
+    return PACKED ? u.L_raw : p.L_raw;
+}
+template <bool PACKED> __device__ __forceinline__ int u_ne_dense(const TcParams& p, const Unit& u) {
+    return PACKED ? u.ne_dense : clampi(p.n_entries ? p.n_entries[u.b] : p.N_cap, 0, p.N_cap);
+}
+template <bool PACKED> __device__ __forceinline__ int u_tok0(const TcParams& p, const Unit& u) {
+    return PACKED ? u.tok0 : u.b * p.n;
+}
+template <bool PACKED> __device__ __forceinline__ int u_ent0(const TcParams& p, const Unit& u) {
+    return PACKED ? u.ent0 : u.b * p.N_cap;
+}
+template <bool PACKED> __device__ __forceinline__ int u_raw0(const TcParams& p, const Unit& u) {
+    return PACKED ? u.raw0 : u.b * p.L_raw;
+}
+
+template <bool PACKED>
 __device__ __forceinline__ Geometry geometry(const TcParams& p, const Unit& un) {
     Geometry g;
     const int t0 = un.t0;
-    const int t_last = min(t0 + kTokens - 1, un.n - 1);
+    const int t_last = min(t0 + kTokens - 1, u_n<PACKED>(p, un) - 1);
     if (p.dense) {
-        g.Vmax = min((t_last + 1) / p.m, un.ne_dense);
+        g.Vmax = min((t_last + 1) / p.m, u_ne_dense<PACKED>(p, un));
         g.cc = 0;
         g.Tc = (g.Vmax + kBN - 1) / kBN;
         g.bn_c_last = g.Tc ? round16(g.Vmax - (g.Tc - 1) * kBN) : 0;
@@ -192,7 +213,7 @@ __device__ __forceinline__ Geometry geometry(const TcParams& p, const Unit& un) 
     }
     if (p.window > 0) {
         g.p_lo = max(0, t0 - p.window + 1);
-        const int p_hi = min(t_last, un.L_raw - 1);
+        const int p_hi = min(t_last, u_L_raw<PACKED>(p, un) - 1);
         g.Lw = max(0, p_hi - g.p_lo + 1);
     } else {
         g.p_lo = 0;
@@ -384,7 +405,11 @@ __device__ __noinline__ void rescale_o(uint32_t o_addr, float alpha) {
     tmem_st_wait();
 }
 
-__global__ void __launch_bounds__(kThreads, 1)
+// 672 threads x at most 88 registers fit one CTA per SM (59,136 of 65,536);
+// this cap (rather than launch bounds, whose occupancy heuristic spilled)
+// lets the allocator keep every role's state in registers.
+template <bool PACKED>
+__global__ void __maxnreg__(88)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_c,
                const __grid_constant__ CUtensorMap tm_w, TcParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -396,7 +421,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     int* sIdx = reinterpret_cast<int*>(stats + 4 * kRows);       // [kTokens][topk]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int n_units = p.vl.S ? p.vl.uoff[p.vl.S] : p.B * ((p.n + kTokens - 1) / kTokens);
+    const int n_units = PACKED ? p.vl.uoff[p.vl.S] : p.B * ((p.n + kTokens - 1) / kTokens);
     volatile int* abort = &ctl->abort;
 
     if (threadIdx.x == 0) {
@@ -437,9 +462,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         int Lg = 0;                                          // loads issued by this CTA
         bool go = true;
         for (int u = blockIdx.x; u < n_units && go; u += gridDim.x) {
-            const Unit un = unit_of(p, u);
+            const Unit un = unit_of<PACKED>(p, u);
             const int t0 = un.t0;
-            const Geometry g = geometry(p, un);
+            const Geometry g = geometry<PACKED>(p, un);
             // the unit's index rows (out-of-range tokens read as padding); the
             // previous unit's gathers have all been issued
             named_sync(1, kLoadThreads);
@@ -447,13 +472,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 for (int i = lt; i < kTokens * p.topk; i += kLoadThreads) {
                     const int tok = i / p.topk, c = i - tok * p.topk;
                     const int t = t0 + tok;
-                    sIdx[i] = (t < un.n) ? __ldg(p.idx + (size_t)(un.tok0 + t) * p.topk + c) : -1;
+                    sIdx[i] = (t < u_n<PACKED>(p, un)) ? __ldg(p.idx + (size_t)(u_tok0<PACKED>(p, un) + t) * p.topk + c) : -1;
                 }
             }
             named_sync(1, kLoadThreads);
             const int NL = total_loads(p, g);
             const int nc = p.dense ? g.Tc : 2 * g.Tc;
-            const uint8_t* kvc_rows = static_cast<const uint8_t*>(p.kv_c) + (size_t)un.ent0 * (kD * 2);
+            const uint8_t* kvc_rows = static_cast<const uint8_t*>(p.kv_c) + (size_t)u_ent0<PACKED>(p, un) * (kD * 2);
             for (int L = 0; L < NL; ++L, ++Lg) {
                 const int slot = Lg % kStages, use = Lg / kStages;
                 uint8_t* dst = sK + slot * kTileBytes;
@@ -486,7 +511,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     if (lt < kBN) {
                         const int c = chunk * kBN + lt;
                         const int sv = (c < p.topk) ? ir[lt] : -1;
-                        const bool ok = tpos < un.n && sv >= 0 && sv < un.N;
+                        const bool ok = tpos < u_n<PACKED>(p, un) && sv >= 0 && sv < u_N<PACKED>(p, un);
                         const uint32_t bits = __ballot_sync(0xffffffffu, ok);
                         if (lane == 0) ctl->mask[slot][warp] = bits;
                     }
@@ -498,7 +523,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         const int row = it * kRowsPerRound + (lt >> 4);
                         const int c = chunk * kBN + row;
                         int sv = (c < p.topk) ? ir[row] : -1;
-                        if (tpos >= un.n || sv < 0 || sv >= un.N) sv = 0;   // masked; any valid row
+                        if (tpos >= u_n<PACKED>(p, un) || sv < 0 || sv >= u_N<PACKED>(p, un)) sv = 0;   // masked; any valid row
                         const uint8_t* src = kvc_rows + (size_t)sv * (kD * 2) + c16 * 16;
                         cp_async16(dst + half * kHalf + row * 128 + ((cc ^ (row & 7)) << 4), src);
                     }
@@ -508,8 +533,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 } else {
                     if (lt == 0) {
                         const CUtensorMap* tm = (kind == 1) ? &tm_c : &tm_w;
-                        const int row = (kind == 1) ? un.ent0 + chunk * kBN
-                                                    : un.raw0 + g.p_lo + chunk * kBN;
+                        const int row = (kind == 1) ? u_ent0<PACKED>(p, un) + chunk * kBN
+                                                    : u_raw0<PACKED>(p, un) + g.p_lo + chunk * kBN;
                         mbar_arrive_expect_tx(&ctl->full[slot], kTileBytes);
                         for (int h = 0; h < 2; ++h)
                             tma_load_2d(dst + h * kHalf, tm, h * 64, row, &ctl->full[slot]);
@@ -532,9 +557,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             const uint32_t id_qk_full = idesc_bf16(kRows, kBN, false, false);
             const uint32_t id_pv = idesc_bf16(kRows, kD, false, true);
             auto load_q = [&](int u) {
-                const Unit un = unit_of(p, u);
+                const Unit un = unit_of<PACKED>(p, u);
                 mbar_arrive_expect_tx(&ctl->bar_q, 2 * kTileBytes);
-                const int qrow = (un.tok0 + un.t0) * kH;
+                const int qrow = (u_tok0<PACKED>(p, un) + un.t0) * kH;
                 for (int mt = 0; mt < 2; ++mt)
                     for (int h = 0; h < 2; ++h)
                         tma_load_2d(sQ + mt * kTileBytes + h * kHalf, &tm_q, h * 64, qrow + mt * kRows,
@@ -546,8 +571,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             bool ok = true;
             if (blockIdx.x < n_units) load_q(blockIdx.x);
             for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++k) {
-                const Unit un = unit_of(p, u);
-                const Geometry g = geometry(p, un);
+                const Unit un = unit_of<PACKED>(p, u);
+                const Geometry g = geometry<PACKED>(p, un);
                 ok = mbar_wait(&ctl->bar_q, k & 1, abort, p.err);
                 tc_fence_after();
                 auto issue_qk = [&](int mt, int j) -> bool {
@@ -637,13 +662,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         int k = 0;
         bool ok = true;
         for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++k) {
-            const Unit un = unit_of(p, u);
+            const Unit un = unit_of<PACKED>(p, u);
             const int t0 = un.t0;
-            const Geometry g = geometry(p, un);
+            const Geometry g = geometry<PACKED>(p, un);
             const int t = t0 + 2 * mt + u_tok;               // position in the sequence
-            const bool row_ok = t < un.n;
+            const bool row_ok = t < u_n<PACKED>(p, un);
             int Vt = 0;
-            if (p.dense && row_ok) Vt = min((t + 1) / p.m, un.ne_dense);
+            if (p.dense && row_ok) Vt = min((t + 1) / p.m, u_ne_dense<PACKED>(p, un));
             const int w_lo = t - p.window + 1;               // window [w_lo, t]
             // m_used: running max (base 2); l_r: sum of the bf16-rounded weights
             // (normalises O); l_e: sum of the unrounded weights (the lse output)
@@ -733,16 +758,16 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
         const uint32_t o_addr = tmem + lane_addr + 256 + mt * 128;
         int k = 0;
         for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++k) {
-            const Unit un = unit_of(p, u);
-            const Geometry g = geometry(p, un);
+            const Unit un = unit_of<PACKED>(p, u);
+            const Geometry g = geometry<PACKED>(p, un);
             const int t = un.t0 + 2 * mt + u_tok;
-            const bool row_ok = t < un.n;
+            const bool row_ok = t < u_n<PACKED>(p, un);
             bool w_ok = mbar_wait(&ctl->stats_ready[mt], k & 1, abort, p.err);
             const RowStat st = stats[((k & 1) * 2 + mt) * kRows + r];
             w_ok = w_ok && mbar_wait(&ctl->o_full[mt], k & 1, abort, p.err);
             if (!__all_sync(0xffffffffu, w_ok)) break;
             tc_fence_after();
-            __nv_bfloat16* orow = p.out + ((size_t)(un.tok0 + t) * kH + (r & 63)) * kD;
+            __nv_bfloat16* orow = p.out + ((size_t)(u_tok0<PACKED>(p, un) + t) * kH + (r & 63)) * kD;
             if (g.T > 0) {
                 const float inv = st.lr > 0.0f ? 1.0f / st.lr : 0.0f;
 #pragma unroll
@@ -766,12 +791,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     }
                 }
                 if (row_ok && p.lse)
-                    p.lse[(size_t)(un.tok0 + t) * kH + (r & 63)] =
+                    p.lse[(size_t)(u_tok0<PACKED>(p, un) + t) * kH + (r & 63)] =
                         st.le > 0.0f ? (st.m + log2f(st.le)) / kLog2e : -INFINITY;
             } else if (row_ok) {
                 // no key at all: o = 0, lse = -inf
                 for (int i = 0; i < kD; i += 8) *reinterpret_cast<uint4*>(orow + i) = make_uint4(0, 0, 0, 0);
-                if (p.lse) p.lse[(size_t)(un.tok0 + t) * kH + (r & 63)] = -INFINITY;
+                if (p.lse) p.lse[(size_t)(u_tok0<PACKED>(p, un) + t) * kH + (r & 63)] = -INFINITY;
             }
             tc_fence_before();
             mbar_arrive(&ctl->o_free[mt]);
@@ -859,13 +884,14 @@ cudaError_t launch_attention_tc(const AttnArgs& a, uint32_t* err, cudaStream_t s
         p.vl.S = 0;
     }
     const size_t smem = kSmemFixed + (a.dense ? 0 : (size_t)kTokens * a.topk * sizeof(int));
-    cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    auto kern = a.vl ? attn_tc_kernel<true> : attn_tc_kernel<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = units < sms ? units : sms;     // persistent: one CTA per SM
-    attn_tc_kernel<<<(unsigned)grid, kThreads, smem, s>>>(tm_q, tm_c, tm_w, p);
+    kern<<<(unsigned)grid, kThreads, smem, s>>>(tm_q, tm_c, tm_w, p);
     count_launch();
     return cudaGetLastError();
 }

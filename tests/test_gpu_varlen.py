@@ -111,3 +111,42 @@ def test_varlen_hca_equals_per_sequence_calls_and_oracle():
         ro, _ = oracle.hca_attn(np64(inp["q"][None, t0:t1]), np64(kv_c[e0:e1])[None], m,
                                 np64(inp["kv"][None, t0:t1]), W)
         check_out(np64(out[t0:t1])[None], ro, torch.bfloat16)
+
+
+def test_varlen_many_sequences_and_fallback_shapes():
+    """130 short sequences (more than one launch's parameter map holds) and
+    fp32 / 16-head operands (not served by the tensor-core kernels): both go
+    through one launch per sequence and must equal the per-sequence calls."""
+    m, k, W, H, D, H_I, d_I = 4, 8, 16, 16, 64, 2, 32
+    rng = np.random.default_rng(5)
+    lens = rng.integers(0, 40, size=130).tolist()
+    cu = _cu(lens)
+    e = api.varlen_entry_offsets(cu, m)
+    T, E = int(cu[-1]), int(e[-1])
+    g = _gen(9)
+    q = torch.randn(T, H, D, generator=g).to(DEV)
+    kv = torch.randn(T, D, generator=g).to(DEV)
+    qI = torch.randn(T, H_I, d_I, generator=g).to(DEV)
+    kI_raw = torch.randn(T, d_I, generator=g).to(DEV)
+    W_c = (torch.randn(D, D, generator=g) / D ** 0.5).to(DEV)
+    W_Ic = (torch.randn(d_I, d_I, generator=g) / d_I ** 0.5).to(DEV)
+    kv_c = torch.empty(E, D, device=DEV)
+    kI_c = torch.empty(E, d_I, device=DEV)
+    idx = torch.empty(T, k, dtype=torch.int32, device=DEV)
+    out = torch.empty_like(q)
+    api.csa_compress_varlen(kv, cu, W_c, m, True, kv_c)
+    api.csa_compress_varlen(kI_raw, cu, W_Ic, m, True, kI_c)
+    api.csa_indexer_topk_varlen(qI, kI_c, cu, m, k, idx)
+    api.csa_sparse_attn_varlen(q, cu, kv_c, m, idx, kv, W, out)
+    torch.cuda.synchronize()
+    for s, L in enumerate(lens):
+        t0, t1, e0, e1 = cu[s], cu[s + 1], e[s], e[s + 1]
+        if L == 0:
+            continue
+        rk = api.compress(kv[None, t0:t1].contiguous(), W_c, m, True)
+        ri = api.compress(kI_raw[None, t0:t1].contiguous(), W_Ic, m, True)
+        assert torch.equal(kv_c[e0:e1], rk[0]) and torch.equal(kI_c[e0:e1], ri[0])
+        rx = api.indexer_topk(qI[None, t0:t1].contiguous(), ri, m, k)
+        assert torch.equal(idx[t0:t1], rx[0])
+        ro = api.sparse_attn(q[None, t0:t1].contiguous(), rk, rx, kv[None, t0:t1].contiguous(), W)
+        assert torch.equal(out[t0:t1], ro[0])
