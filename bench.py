@@ -18,6 +18,7 @@ max over ranks.  Rank 0 prints one JSON line.
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import hashlib
 import json
 import math
@@ -93,6 +94,35 @@ def prefill_work(w):
         "indexer_topk": dict(bytes=idx_bytes, flops=idx_flops),
         "sparse_attn": dict(bytes=attn_bytes, flops=attn_flops),
     }
+
+
+def varlen_work(w, lens):
+    """prefill_work summed over packed sequences of the given lengths (B = 1 each)."""
+    tot = {}
+    for L in lens:
+        if L <= 0:
+            continue
+        for k_, v in prefill_work(dataclasses.replace(w, B=1, n=int(L))).items():
+            t = tot.setdefault(k_, dict(bytes=0.0, flops=0.0))
+            t["bytes"] += v["bytes"]
+            t["flops"] += v["flops"]
+    return tot
+
+
+def roofline_of(work, ms, peaks, timed_alone):
+    """Where one kernel sits against the roofline its algorithmic intensity
+    picks (ridge = measured bf16 TFLOP/s over measured HBM GB/s): achieved
+    flops or bytes per second over that peak.  Kernels timed alone use the
+    burst bf16 figure, kernels inside a long step the sustained one."""
+    tf = peaks["bf16_tflops"] if timed_alone else peaks.get("bf16_tflops_sustained",
+                                                              peaks["bf16_tflops"])
+    ridge = tf * 1e12 / (peaks["hbm_gbs"] * 1e9)
+    if work["flops"] > ridge * max(work["bytes"], 1.0):
+        a = work["flops"] / (ms / 1e3) / 1e12
+        return {"bound": "tensor", "achieved": a, "peak": tf, "unit": "TFLOP/s", "frac": a / tf}
+    a = work["bytes"] / (ms / 1e3) / 1e9
+    return {"bound": "hbm", "achieved": a, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": a / peaks["hbm_gbs"]}
 
 
 def decode_work(w, inp):
@@ -242,7 +272,7 @@ def run_prefill(w, dev, steps, warmup, dist_ctx, rank):
                 path=path, inp=inp)
 
 
-def run_variants(w, path, dev, steps, rank):
+def run_variants(w, path, dev, steps, rank, peaks):
     """The NEXT-row variants of the prefill workload, each timed alone with
     CUDA events and L2 flushed between iterations (their inputs are smaller
     than L2): the gated-softmax compressor on kv, the Hadamard-rotated fp8
@@ -289,7 +319,8 @@ def run_variants(w, path, dev, steps, rank):
         torch.cuda.synchronize()
         ms = float(np.mean([a_.elapsed_time(b_) for a_, b_ in ts]))
         out[name] = {"ms": ms, "TFLOP/s": work[name]["flops"] / (ms / 1e3) / 1e12,
-                     "GB/s": work[name]["bytes"] / (ms / 1e3) / 1e9}
+                     "GB/s": work[name]["bytes"] / (ms / 1e3) / 1e9,
+                     "roofline": roofline_of(work[name], ms, peaks, timed_alone=True)}
     del flush
     return out
 
@@ -508,7 +539,7 @@ def run_decode_paged(dev, steps, warmup, rank, page_size=64):
     t_idx = [r[0].elapsed_time(r[1]) for r in recs]
     t_att = [r[1].elapsed_time(r[2]) for r in recs]
     tot = [a + b for a, b in zip(t_idx, t_att)]
-    return dict(w=w, ms=float(np.mean(tot)), page_size=page_size,
+    return dict(w=w, ms=float(np.mean(tot)), page_size=page_size, work=decode_work(w, inp),
                 kern_ms={"indexer_topk": float(np.mean(t_idx)), "sparse_attn": float(np.mean(t_att))})
 
 
@@ -649,7 +680,6 @@ def main():
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     w = synth.WORKLOADS[PREFILL]
     if args.n:
-        import dataclasses
         w = dataclasses.replace(w, n=args.n)
     config = {"workload": PREFILL if not args.n else f"{PREFILL} (n overridden to {args.n}: "
                                                        "profiling case, not the headline)", "B": w.B, "n": w.n, "H": w.H, "D": w.D, "m": w.m,
@@ -750,13 +780,15 @@ def main():
             "note": "NEXT rows, each timed alone: gated-softmax compressor (kv, d 128, m 4 "
                     "overlapping), Hadamard-rotated fp8 indexer keys, gated indexer + top-k "
                     "against rotated keys",
-            **run_variants(w, pre["path"], dev, max(3, args.steps), rank)}
+            **run_variants(w, pre["path"], dev, max(3, args.steps), rank, peaks)}
     if not args.no_variants:
         pv = run_prefill_varlen(w, pre["path"], dev, max(3, args.steps), args.warmup)
         vval, vms = dist_ctx.job_rate(pv["T"], pv["ms"])
         line["prefill_varlen"] = {
             "workload": "csa_prefill_packed8_n64k_fp8idx", "value": vval, "unit": "queries/s",
             "ms_per_step": vms, "lengths": pv["lens"], "stages_ms": pv["stages"],
+            "roofline": {nm: roofline_of(wk, pv["stages"][nm], peaks, timed_alone=False)
+                         for nm, wk in varlen_work(w, pv["lens"]).items()},
             "note": "the c3 tokens re-cut into 8 packed sequences (csa_*_varlen entry points); "
                     "less causal work than one 64K sequence, so not comparable to the headline"}
     if not args.no_decode:
@@ -777,6 +809,8 @@ def main():
         line["decode_paged"] = {"workload": DECODE, "value": pval, "unit": "tok/s",
                                 "ms_per_step": pms, "page_size": dp["page_size"],
                                 "stages_ms": dp["kern_ms"],
+                                "roofline": {nm: roofline_of(dp["work"][nm], ms_, peaks, True)
+                                             for nm, ms_ in dp["kern_ms"].items()},
                                 "l2": "flushed (512 MiB write) between steps",
                                 "note": "the decode step over caches scattered into a shuffled "
                                         "page pool (csa_*_paged entry points)"}
