@@ -16,7 +16,7 @@ shard edges.  A CP run must reproduce the single-rank result.  The page
 gathers the halo with an all-gather; here the left neighbour sends it point
 to point, since one neighbour's rows are all a rank needs.
 
-The driver moves data and does the bookkeeping (which rows, which positions).
+This module moves data and does the bookkeeping (which rows, which positions).
 The arithmetic is done by a backend object with three calls:
 
     compress(x [L, d_in], W, m, overlap, fp8) -> entries [L//m, d_out]
@@ -128,7 +128,7 @@ def cp_prefill(shard: Shard, q, kv, qI, kI_raw, W_c, W_Ic, m: int, topk: int, wi
 
 
 class CudaBackend:
-    """The CP driver's arithmetic through this library's entry points."""
+    """The context-parallel arithmetic through this library's entry points."""
 
     def __init__(self, stream=None):
         from . import api

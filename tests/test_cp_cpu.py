@@ -1,8 +1,8 @@
-"""Context-parallel prefill on host cores: two and four gloo ranks run the CP
-driver with the oracle as the arithmetic, and the gathered result must equal,
+"""Context-parallel prefill on host cores: two and four gloo ranks run the context-parallel
+code with the oracle as the arithmetic, and the gathered result must equal,
 bit for bit, the single-rank oracle run over the whole sequence.  This is
 the CP = 1 vs CP > 1 agreement that the migration analysis names as the
-risk of the layout.  Only the driver's exchanges and bookkeeping are under
+risk of the layout.  Only the exchanges and bookkeeping are under
 test; the oracle is plugged in from here."""
 import os
 import socket
@@ -18,7 +18,7 @@ N, H, D, H_I, d_I, M, K, WIN = 256, 4, 16, 2, 16, 4, 12, 24
 
 
 class OracleBackend:
-    """The oracle's stages on fp64 host tensors, shaped as the CP driver calls them."""
+    """The oracle's stages on fp64 host tensors, shaped as cp_prefill calls them."""
 
     def __init__(self):
         import oracle
@@ -61,7 +61,7 @@ def _run(rank, world, inp, fp8, group=None):
     sh = cp.shard_of(N, world, rank, M)
     loc = {k: (v[sh.p0:sh.p1].contiguous() if k in ("q", "kv", "qI", "kI_raw") else v)
            for k, v in inp.items()}
-    if fp8:       # the driver hands fp8 query rows to the backend as values
+    if fp8:       # cp_prefill hands fp8 query rows to the backend as values
         import oracle
         qv = oracle.quantized_query_rows(loc["qI"].numpy().astype(np.float32))
         loc["qI"] = torch.from_numpy(qv)

@@ -1,4 +1,4 @@
-"""The context-parallel driver on one GPU (one rank, no exchange) with this
+"""The context-parallel prefill on one GPU (one rank, no exchange) with this
 library's kernels as the arithmetic: the positioned (decode-shaped) kernels
 serve a shard's queries, and the result must match the oracle."""
 import numpy as np
