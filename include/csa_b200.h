@@ -341,7 +341,8 @@ csa_status_t hca_dense_attn_paged(const void* q, int dt, int B, int n_q, int H, 
  */
 int csa_varlen_entry_offsets(const int* cu_seqlens, int S, int m, int* entry_offsets);
 /*   writes e(0..S) into entry_offsets [S+1] (host) and returns e(S), or -1 on
- *   an invalid argument. */
+ *   an invalid argument (S < 0, m < 1, NULL arrays, cu_seqlens[0] != 0 or a
+ *   decreasing cu_seqlens). */
 
 csa_status_t csa_compress_varlen(const void* x, int x_dt, int S, const int* cu_seqlens, int d_in,
                                  const void* W, int d_out, int m, int overlap, void* out,

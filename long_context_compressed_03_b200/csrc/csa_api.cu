@@ -430,6 +430,9 @@ static csa_status_t check_cu(const char* name, int S, const int* cu, int m) {
 
 int csa_varlen_entry_offsets(const int* cu_seqlens, int S, int m, int* entry_offsets) {
     if (S < 0 || m < 1 || !entry_offsets || (S > 0 && !cu_seqlens)) return -1;
+    if (S > 0 && cu_seqlens[0] != 0) return -1;
+    for (int s = 0; s < S; ++s)
+        if (cu_seqlens[s + 1] < cu_seqlens[s]) return -1;
     long e = 0;
     entry_offsets[0] = 0;
     for (int s = 0; s < S; ++s) {

@@ -274,3 +274,23 @@ def test_binding_raises_loudly_without_library(tmp_path):
             mod.load(str(tmp_path / "missing.so"))
     finally:
         importlib.reload(api)
+
+
+def test_binding_rejects_host_tensors_and_bad_shapes(lib):
+    # the binding marshals CUDA tensors only and checks what it can before the
+    # C call; nothing here reaches a kernel
+    import torch
+    x = torch.zeros(1, 8, 16)
+    W = torch.zeros(16, 16)
+    with pytest.raises(ValueError, match="CUDA"):
+        api.csa_compress(x, W, 4, True, torch.zeros(1, 2, 16))
+    with pytest.raises(ValueError, match="int32"):
+        api._i32(torch.zeros(3, dtype=torch.int64), "q_pos")
+    with pytest.raises(ValueError, match="fp8"):
+        api._dt_rot(torch.zeros(2, 2), True)      # rotation applies to fp8 rows only
+    assert api._dt_rot(torch.zeros(2, 2, dtype=torch.uint8), True) == api.DT_E4M3_HADAMARD
+    with pytest.raises(ValueError, match="pool"):
+        api.PagedCache(torch.zeros(4, 4), torch.zeros(1, 2, dtype=torch.int32))
+    with pytest.raises(ValueError, match="cu_seqlens"):
+        api.varlen_entry_offsets([0, 5, 3], 4)     # decreasing
+    assert api.varlen_entry_offsets([0, 5, 5, 13], 4).tolist() == [0, 1, 1, 3]
