@@ -89,6 +89,15 @@ unsigned long long csa_kernel_launches(void);
 csa_status_t csa_check_device_error(void* stream, int clear);
 
 /*
+ * Test hook for the launch-failure path (it never faults, traps or hangs a
+ * GPU): the next kernel launch of any entry point is skipped, after its
+ * arguments were validated, and the call returns CSA_ERR_CUDA for
+ * `cuda_error` (a cudaError_t value > 0), as a failing launch would.  One
+ * shot; process-wide.
+ */
+csa_status_t csa_debug_inject_launch_error(int cuda_error);
+
+/*
  * csa_compress -- stage 1: overlapping (or plain) mean-pool compression
  * followed by a projection, optionally quantised to fp8.
  * Follows "百万上下文从「奢侈品」变「日用品」…" §3.2 (C[i] = W . mean of the

@@ -35,6 +35,7 @@ SIGNATURES = {
     "csa_version": (I, []),
     "csa_kernel_launches": (ctypes.c_ulonglong, []),
     "csa_check_device_error": (I, [P, I]),
+    "csa_debug_inject_launch_error": (I, [I]),
     "csa_compress": (I, [P, I, I, I, I, P, I, I, I, P, I, P, P]),
     "csa_compress_gated": (I, [P, I, I, I, I, P, P, P, I, I, I, P, I, P, P]),
     "csa_compress_append": (I, [P, I, I, I, P, I, I, I, P, P, P, I, P, I, P, P]),

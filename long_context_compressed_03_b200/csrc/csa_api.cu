@@ -53,6 +53,13 @@ csa_status_t ok() {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Test hook: an error the next launch returns instead of launching (one shot).
+std::atomic<int> g_inject_error{0};
+
+cudaError_t injected_or_launch_marker() {
+    return static_cast<cudaError_t>(g_inject_error.exchange(0));
+}
+
 csa_status_t from_cuda(cudaError_t e, const char* what, const char* why) {
     if (e == cudaSuccess) return ok();
     if (e == cudaErrorNotSupported && why) return fail(CSA_ERR_UNSUPPORTED, "%s", why);
@@ -63,6 +70,11 @@ csa_status_t from_cuda(cudaError_t e, const char* what, const char* why) {
     do {                   \
         if (!(cond)) return fail(CSA_ERR_INVALID_ARG, __VA_ARGS__); \
     } while (0)
+// Every kernel launch of an entry point goes through LAUNCH: with an injected
+// error pending (csa_debug_inject_launch_error) the launch is skipped and the
+// error returned, as a failing launch would.
+#define LAUNCH(expr) (g_inject_error.load() != 0 ? injected_or_launch_marker() : (expr))
+
 #define REQUIRE_ALIGNED(p, name) \
     do {                         \
         if ((p) && !aligned16(p)) return fail(CSA_ERR_MISALIGNED, "%s is not 16-byte aligned", name); \
@@ -150,7 +162,7 @@ csa_status_t csa_compress(const void* x, int x_dt, int B, int n, int d_in, const
     csa::CompressArgs a{x, x_dt, B, n, d_in, W, d_out, m, overlap, out, out_dt, out_row_scale, N_c,
                         hadamard_norm(d_out)};
     const char* why = nullptr;
-    return from_cuda(csa::launch_compress(a, static_cast<cudaStream_t>(stream), &why), "csa_compress", why);
+    return from_cuda(LAUNCH(csa::launch_compress(a, static_cast<cudaStream_t>(stream), &why)), "csa_compress", why);
 }
 
 csa_status_t csa_compress_gated(const void* x, int x_dt, int B, int n, int d_in, const void* W_kv,
@@ -182,7 +194,7 @@ csa_status_t csa_compress_gated(const void* x, int x_dt, int B, int n, int d_in,
     csa::GatedArgs a{x, x_dt, B, n, d_in, W_kv, W_gate, ape, d_out, m, overlap, out, out_dt,
                      out_row_scale, N_c, hadamard_norm(d_out)};
     const char* why = nullptr;
-    return from_cuda(csa::launch_compress_gated(a, static_cast<cudaStream_t>(stream), &why),
+    return from_cuda(LAUNCH(csa::launch_compress_gated(a, static_cast<cudaStream_t>(stream), &why)),
                      "csa_compress_gated", why);
 }
 
@@ -215,7 +227,7 @@ static csa_status_t compress_append_impl(const void* x_new, int x_dt, int B, int
     csa::AppendArgs a{x_new, x_dt, B, d_in, W, d_out, m, overlap, pos, state, cache, out_dt,
                       cache_scale, N_cap, n_entries, hadamard_norm(d_out), pm};
     const char* why = nullptr;
-    return from_cuda(csa::launch_compress_append(a, static_cast<cudaStream_t>(stream), &why),
+    return from_cuda(LAUNCH(csa::launch_compress_append(a, static_cast<cudaStream_t>(stream), &why)),
                      "csa_compress_append", why);
 }
 
@@ -252,7 +264,7 @@ static csa_status_t indexer_impl(const void* qI, int qI_dt, const float* qI_scal
     csa::IndexerArgs a{qI, qI_dt, qI_scale, kI, kI_dt, kI_scale, B, n_q, H_I, d_I, N_cap,
                        n_entries, q_pos, m, topk, idx_out, hadamard_norm(d_I), qI_weight, pm};
     const char* why = nullptr;
-    return from_cuda(csa::launch_indexer_topk(a, static_cast<cudaStream_t>(stream), &why),
+    return from_cuda(LAUNCH(csa::launch_indexer_topk(a, static_cast<cudaStream_t>(stream), &why)),
                      "csa_indexer_topk", why);
 }
 
@@ -346,7 +358,7 @@ static csa_status_t attention_common(const char* name, csa::AttnArgs& a, void* s
     REQUIRE_ALIGNED4(a.n_entries, "n_entries");
     if (!(a.scale > 0.0f)) a.scale = 1.0f / sqrtf((float)a.D);
     const char* why = nullptr;
-    return from_cuda(csa::launch_attention(a, static_cast<cudaStream_t>(stream), &why), name, why);
+    return from_cuda(LAUNCH(csa::launch_attention(a, static_cast<cudaStream_t>(stream), &why)), name, why);
 }
 
 csa_status_t csa_sparse_attn(const void* q, int dt, int B, int n_q, int H, int D,
@@ -405,6 +417,13 @@ csa_status_t hca_dense_attn_paged(const void* q, int dt, int B, int n_q, int H, 
     csa::AttnArgs a{q, dt, B, n_q, H, D, kv_c_pages, N_cap, nullptr, 0, n_entries, m, 1, kv_raw,
                     L_raw, raw_pos0, raw_len, window, q_pos, softmax_scale, out, lse_out, pm};
     return attention_common("hca_dense_attn_paged", a, stream);
+}
+
+// ------------------------------------------------------------------ test hooks
+csa_status_t csa_debug_inject_launch_error(int cuda_error) {
+    REQUIRE(cuda_error > 0, "csa_debug_inject_launch_error: the code must be a CUDA error (> 0)");
+    g_inject_error.store(cuda_error);
+    return ok();
 }
 
 // ------------------------------------------------------------------ varlen
@@ -480,7 +499,7 @@ csa_status_t csa_compress_varlen(const void* x, int x_dt, int S, const int* cu_s
             csa::CompressArgs a{x, x_dt, S, max_len, d_in, W, d_out, m, overlap, out, out_dt,
                                 out_row_scale, max_nc, hadamard_norm(d_out), &map};
             const char* why = nullptr;
-            return from_cuda(csa::launch_compress(a, static_cast<cudaStream_t>(stream), &why), name,
+            return from_cuda(LAUNCH(csa::launch_compress(a, static_cast<cudaStream_t>(stream), &why)), name,
                              why);
         }
         long e = 0;
@@ -544,7 +563,7 @@ csa_status_t csa_indexer_topk_varlen(const void* qI, int qI_dt, const float* qI_
                                map.ent[S], nullptr, nullptr, m, topk, idx_out, hadamard_norm(d_I),
                                qI_weight};
             a.vl = &map;
-            const cudaError_t ce = csa::launch_indexer_packed(a, max_n, static_cast<cudaStream_t>(stream));
+            const cudaError_t ce = LAUNCH(csa::launch_indexer_packed(a, max_n, static_cast<cudaStream_t>(stream)));
             if (ce != cudaErrorNotSupported) return from_cuda(ce, name, nullptr);
             // otherwise: one launch per sequence below
         }
@@ -605,7 +624,7 @@ static csa_status_t attn_varlen(const char* name, bool dense, const void* q, int
                             softmax_scale > 0.0f ? softmax_scale : 1.0f / sqrtf((float)D), out,
                             lse_out};
             a.vl = &map;
-            const cudaError_t ce = csa::launch_attention_packed(a, static_cast<cudaStream_t>(stream));
+            const cudaError_t ce = LAUNCH(csa::launch_attention_packed(a, static_cast<cudaStream_t>(stream)));
             if (ce != cudaErrorNotSupported) return from_cuda(ce, name, nullptr);
             // otherwise: one launch per sequence below
         }

@@ -390,6 +390,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
             if (lane == 0) {
                 for (int c = 0; c < nchunks; ++c, ++L) {
                     const int slot = L % C::kStages, u = L / C::kStages;
+                    if (*abort) break;     // nothing is issued once the CTA aborts
                     if (u > 0 && !mbar_wait(&ctl->freeb[slot], (u - 1) & 1, abort, p.err)) break;
                     mbar_arrive_expect_tx(&ctl->full[slot], C::kBTile);
                     tma_load_2d(sB + slot * C::kBTile, &tm_k, 0, (int)ent0 + c * kN, &ctl->full[slot]);

@@ -294,3 +294,26 @@ def test_binding_rejects_host_tensors_and_bad_shapes(lib):
     with pytest.raises(ValueError, match="cu_seqlens"):
         api.varlen_entry_offsets([0, 5, 3], 4)     # decreasing
     assert api.varlen_entry_offsets([0, 5, 5, 13], 4).tolist() == [0, 1, 1, 3]
+
+
+def test_injected_launch_error_maps_to_cuda_status(lib):
+    # validation runs first, then the injected error stands in for the launch
+    # (one shot).  The arguments are valid device buffers when a GPU is
+    # present, so even a hook that failed to fire would compute on real memory.
+    import torch
+    if torch.cuda.is_available():
+        dev = [torch.zeros(1, 8, 16, device="cuda"), torch.zeros(16, 16, device="cuda"),
+               torch.zeros(1, 2, 16, device="cuda")]
+        x, W, out = (ctypes.c_void_p(t.data_ptr()) for t in dev)
+    else:
+        x = W = out = FAKE
+    assert lib.csa_debug_inject_launch_error(0) == api.CSA_ERR_INVALID_ARG
+    assert lib.csa_debug_inject_launch_error(719) == api.CSA_OK      # cudaErrorLaunchFailure
+    # an invalid call reports its own error and leaves the injection pending
+    assert lib.csa_compress(x, 0, 1, 8, 16, W, 16, 0, 1, out, 0, None, None) == api.CSA_ERR_INVALID_ARG
+    assert lib.csa_compress(x, 0, 1, 8, 16, W, 16, 4, 1, out, 0, None, None) == api.CSA_ERR_CUDA
+    assert "csa_compress" in _detail(lib)
+    if not torch.cuda.is_available():
+        return
+    # consumed: the next call launches normally
+    assert lib.csa_compress(x, 0, 1, 8, 16, W, 16, 4, 1, out, 0, None, None) == api.CSA_OK
