@@ -45,8 +45,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
 # keyed by kernel family; valid only while the kernel source hashes the same.
 NCU_TRAFFIC = {
-    # profiles/attn_tc_csa_prefill_n16384.md: 307.4 MB read + 220.4 MB written at
-    # n=16384, scaled by 4 (units = queries) to one n=65536 launch
+    # the ncu capture of the prefill attention at n=16384: 307.4 MB read + 220.4 MB
+    # written, scaled by 4 (units = queries) to one n=65536 launch
     "sparse_attn": {"bytes": (307.403008e6 + 220.389120e6) * 4, "file": "attention_tc.cu",
                     "src": "ee13d0b93b5e"},
 }

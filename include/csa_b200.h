@@ -93,7 +93,9 @@ csa_status_t csa_check_device_error(void* stream, int clear);
  * GPU): the next kernel launch of any entry point is skipped, after its
  * arguments were validated, and the call returns CSA_ERR_CUDA for
  * `cuda_error` (a cudaError_t value > 0), as a failing launch would.  One
- * shot; process-wide.
+ * shot; process-wide.  cudaErrorNotSupported (801) is rejected with
+ * CSA_ERR_INVALID_ARG: the packed entry points read that code from a launch
+ * as "run one launch per sequence instead", so it would not surface.
  */
 csa_status_t csa_debug_inject_launch_error(int cuda_error);
 

@@ -18,11 +18,12 @@
 //     into the 128-byte-swizzled layout the tensor core reads (many
 //     independent requests in flight), and the rows of the other token in
 //     the M tile are masked.
-// Roles (13 warps): warps 0-3 load (Q and contiguous tiles by TMA; the
-// sparse rows by cp.async, 16 lanes per 256-byte row, from index rows staged
-// in shared memory), warp 4 allocates TMEM and one lane issues every MMA,
-// warps 5-8 / 9-12 run the softmax of M tile 0 / 1 (a warp reaches TMEM
-// lanes 32*(warp%4) .. +31, so each group covers all 128 rows).
+// Roles (21 warps): warps 0-3 load (contiguous tiles by TMA; the sparse
+// rows by cp.async, 16 lanes per 256-byte row, from index rows staged in
+// shared memory), warp 4 allocates TMEM, loads Q by TMA and one lane issues
+// every MMA, warps 5-8 / 9-12 run the softmax of M tile 0 / 1 (a warp
+// reaches TMEM lanes 32*(warp%4) .. +31, so each group covers all 128
+// rows), warps 13-16 / 17-20 write the output of M tile 0 / 1.
 // TMEM: S0 [cols 0,128), S1 [128,256), O0 [256,384), O1 [384,512).
 // S = Q K^T (M=128, N<=128, K=128 in 8 steps), P = exp2(S*scale*log2e - m)
 // in bf16 written back into the first 64 columns of S, O += P V with P read
@@ -556,7 +557,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             prefetch_tmap(&tm_q);
             const uint32_t id_qk_full = idesc_bf16(kRows, kBN, false, false);
             const uint32_t id_pv = idesc_bf16(kRows, kD, false, true);
+            int q_issued = 0, q_done = 0;     // Q loads issued / waited for
             auto load_q = [&](int u) {
+                ++q_issued;
                 const Unit un = unit_of<PACKED>(p, u);
                 mbar_arrive_expect_tx(&ctl->bar_q, 2 * kTileBytes);
                 const int qrow = (u_tok0<PACKED>(p, un) + un.t0) * kH;
@@ -569,11 +572,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             int J[2] = {0, 0};                // tiles before this unit, per M tile
             int k = 0;                        // units done
             bool ok = true;
-            if (blockIdx.x < n_units) load_q(blockIdx.x);
+            // nothing is loaded by a CTA that starts aborted
+            if (blockIdx.x < n_units && !*abort) load_q(blockIdx.x);
             for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++k) {
                 const Unit un = unit_of<PACKED>(p, u);
                 const Geometry g = geometry<PACKED>(p, un);
-                ok = mbar_wait(&ctl->bar_q, k & 1, abort, p.err);
+                ok = q_issued > q_done && mbar_wait(&ctl->bar_q, k & 1, abort, p.err);
+                if (ok) ++q_done;
                 tc_fence_after();
                 auto issue_qk = [&](int mt, int j) -> bool {
                     const TileRef r = tile_ref(p, g, mt, j);
@@ -599,7 +604,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 auto next_q = [&]() -> bool {
                     mma_commit(&ctl->q_free);
                     if (un_next >= n_units) return true;
-                    if (!mbar_wait(&ctl->q_free, k & 1, abort, p.err)) return false;
+                    if (!mbar_wait(&ctl->q_free, k & 1, abort, p.err) || *abort) return false;
                     load_q(un_next);
                     return true;
                 };
@@ -642,10 +647,13 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 J[0] += g.T;
                 J[1] += g.T;
             }
-            // every MMA issued must finish before TMEM is released
+            // every MMA issued must finish before TMEM is released, and a Q
+            // load still in flight (the CTA aborted before waiting for it)
+            // must land before the CTA's shared memory is given up
             mma_commit(&ctl->fin);
             volatile int never = 0;
             mbar_wait(&ctl->fin, 0, &never, p.err);
+            if (q_issued > q_done) mbar_wait(&ctl->bar_q, q_done & 1, &never, p.err);
         }
         __syncwarp();
     } else if (warp < kEpiWarp0) {

@@ -20,17 +20,22 @@ void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 // One error word per device for kernels whose bounded waits expired.
 static __device__ uint32_t g_device_error;
-static uint32_t* g_error_ptr[64];
+// Its device address per device, looked up once.  Host threads may race on
+// the first lookup; they all store the same address, and the atomics make
+// that race well defined.
+static std::atomic<uint32_t*> g_error_ptr[64];
 
 uint32_t* device_error_word() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    if (!g_error_ptr[dev]) {
+    uint32_t* w = g_error_ptr[dev].load(std::memory_order_acquire);
+    if (!w) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
-        g_error_ptr[dev] = static_cast<uint32_t*>(p);
+        w = static_cast<uint32_t*>(p);
+        g_error_ptr[dev].store(w, std::memory_order_release);
     }
-    return g_error_ptr[dev];
+    return w;
 }
 }  // namespace csa
 
@@ -422,6 +427,10 @@ csa_status_t hca_dense_attn_paged(const void* q, int dt, int B, int n_q, int H, 
 // ------------------------------------------------------------------ test hooks
 csa_status_t csa_debug_inject_launch_error(int cuda_error) {
     REQUIRE(cuda_error > 0, "csa_debug_inject_launch_error: the code must be a CUDA error (> 0)");
+    // the packed entry points read cudaErrorNotSupported from a launch as
+    // "take the per-sequence path", which would swallow the injected failure
+    REQUIRE(cuda_error != (int)cudaErrorNotSupported,
+            "csa_debug_inject_launch_error: cudaErrorNotSupported (801) is not a launch failure");
     g_inject_error.store(cuda_error);
     return ok();
 }

@@ -578,6 +578,14 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
         }
         __syncthreads();
     }
+    // key loads still in flight after an abort must land before the CTA's
+    // shared memory is given up: the last load of each stage is the latest
+    // phase of its barrier, so waiting on it covers every earlier one
+    if (warp == 0 && lane == 0) {
+        volatile int never = 0;
+        for (int Lp = max(0, L - C::kStages); Lp < L; ++Lp)
+            mbar_wait(&ctl->full[Lp % C::kStages], (Lp / C::kStages) & 1, &never, p.err);
+    }
     if (!need) {
         // every row takes all its visible entries
         for (int i = threadIdx.x; i < kRows; i += kThreads) {

@@ -1,5 +1,5 @@
 // tc_common.cuh -- sm_100a building blocks written as inline PTX: mbarriers
-// with bounded waits, TMA tensor loads (tiled and row-gather), tcgen05 MMA /
+// with bounded waits, tiled TMA tensor loads, tcgen05 MMA /
 // TMEM allocation / TMEM loads and the shared-memory matrix descriptors.
 #pragma once
 #include <cuda.h>
@@ -88,17 +88,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* m, int
           "r"(smem_u32(bar))
         : "memory");
 }
-// Row gather: four rows y0..y3 (box one row high) starting at inner coordinate x.
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* m, int x, int y0, int y1,
-                                            int y2, int y3, uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-        " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];"
-        ::"r"(smem_u32(dst)), "l"(reinterpret_cast<uint64_t>(m)), "r"(x), "r"(y0), "r"(y1),
-          "r"(y2), "r"(y3), "r"(smem_u32(bar))
-        : "memory");
-}
-
 // 16-byte cp.async global -> shared (L2 only).
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");

@@ -25,3 +25,15 @@ def pytest_collection_modifyitems(config, items):
     for item in items:
         if "gpu" in item.keywords:
             item.add_marker(skip)
+
+
+def pytest_terminal_summary(terminalreporter, exitstatus, config):
+    """Observed errors and margins of every parity check that ran."""
+    try:
+        from csa_checks import LOG
+    except Exception:  # pragma: no cover
+        return
+    if LOG:
+        terminalreporter.section("parity margins")
+        for line in LOG:
+            terminalreporter.write_line(line)

@@ -308,11 +308,17 @@ def test_injected_launch_error_maps_to_cuda_status(lib):
     else:
         x = W = out = FAKE
     assert lib.csa_debug_inject_launch_error(0) == api.CSA_ERR_INVALID_ARG
+    # 801 would be read by the packed entry points as "take the per-sequence path"
+    assert lib.csa_debug_inject_launch_error(801) == api.CSA_ERR_INVALID_ARG
     assert lib.csa_debug_inject_launch_error(719) == api.CSA_OK      # cudaErrorLaunchFailure
     # an invalid call reports its own error and leaves the injection pending
     assert lib.csa_compress(x, 0, 1, 8, 16, W, 16, 0, 1, out, 0, None, None) == api.CSA_ERR_INVALID_ARG
+    before = lib.csa_kernel_launches()
     assert lib.csa_compress(x, 0, 1, 8, 16, W, 16, 4, 1, out, 0, None, None) == api.CSA_ERR_CUDA
-    assert "csa_compress" in _detail(lib)
+    # the injected code's own message (a real launch on fake pointers would
+    # report a different error), and nothing was launched
+    assert "csa_compress" in _detail(lib) and "unspecified launch failure" in _detail(lib)
+    assert lib.csa_kernel_launches() == before
     if not torch.cuda.is_available():
         return
     # consumed: the next call launches normally

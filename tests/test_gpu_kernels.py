@@ -8,7 +8,8 @@ import pytest
 import torch
 
 import oracle
-from csa_checks import ATOL_BF16, ATOL_F32, check_out, check_topk, max_abs, np64
+from csa_checks import (ATOL_BF16, ATOL_F32, check_compress_stored, check_e4m3_rows, check_out,
+                        check_topk, compress_bound, max_abs, np64, rotated_bound)
 from long_context_compressed_03_b200 import api
 
 pytestmark = pytest.mark.gpu
@@ -44,27 +45,18 @@ def test_compress_matches_oracle(case):
     x = _randn(g, B, n, d_in, dtype=dt)
     W = _randn(g, d_in, d_out, dtype=dt, std=1 / math.sqrt(d_in))
     ref = oracle.compress(np64(x), np64(W), m, overlap)
+    bound = compress_bound(np64(x), np64(W), m, overlap)
     xd, Wd = x.to(DEV), W.to(DEV)
     if kind == "e4m3":
         codes, scale = api.compress(xd, Wd, m, overlap, out_dtype=torch.uint8)
-        codes, scale = codes.cpu().numpy(), scale.cpu().numpy()
-        deq = oracle.dequantize_rows_e4m3(codes, scale)
-        amax = np.abs(ref).max(axis=-1)
-        np.testing.assert_allclose(scale, amax / 448.0, rtol=1e-5)
-        # one E4M3 step (3 mantissa bits) of the row's own scale
-        assert np.all(np.abs(deq - ref) <= np.abs(ref) * 2.0 ** -3 + scale[..., None] * 2.0 ** -9)
-        assert max_abs(deq, ref) <= ATOL_BF16 * 4
+        check_e4m3_rows(codes.cpu().numpy(), scale.cpu().numpy(), ref, bound)
         return
     out_dt = torch.float32 if kind == "f32" else torch.bfloat16
     out = api.compress(xd, Wd, m, overlap, out_dtype=out_dt)
     torch.cuda.synchronize()
     got = np64(out)
     assert got.shape == ref.shape
-    if kind == "f32":
-        assert max_abs(got, ref) <= ATOL_F32
-    else:
-        assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-5)
-        assert max_abs(got, ref) <= ATOL_BF16
+    check_compress_stored(got, ref, bound, out_dt)
 
 
 def _hadamard64(d):
@@ -90,16 +82,15 @@ def test_compress_hadamard_fp8_matches_rotated_oracle(case):
     g = _gen(500 + n)
     x = _randn(g, B, n, d_in, dtype=dt)
     W = _randn(g, d_in, d_out, dtype=dt, std=1.0 / math.sqrt(d_in))
-    ref = oracle.compress(np64(x), np64(W), m, overlap) @ _hadamard64(d_out)
+    unrot = oracle.compress(np64(x), np64(W), m, overlap)
+    ref = unrot @ _hadamard64(d_out)
+    bound = rotated_bound(compress_bound(np64(x), np64(W), m, overlap), np64(x), np64(W), m, overlap)
     codes, scale = api.compress(x.to(DEV), W.to(DEV), m, overlap, out_dtype=torch.uint8,
                                 hadamard=True)
     codes, scale = codes.cpu().numpy(), scale.cpu().numpy()
-    deq = oracle.dequantize_rows_e4m3(codes, scale)
-    np.testing.assert_allclose(scale, np.abs(ref).max(axis=-1) / 448.0, rtol=1e-5)
-    assert np.all(np.abs(deq - ref) <= np.abs(ref) * 2.0 ** -3 + scale[..., None] * 2.0 ** -9)
+    check_e4m3_rows(codes, scale, ref, bound)
     # rotating back recovers the row to within the fp8 error spread by H
-    back = deq @ _hadamard64(d_out)
-    unrot = oracle.compress(np64(x), np64(W), m, overlap)
+    back = oracle.dequantize_rows_e4m3(codes, scale) @ _hadamard64(d_out)
     assert max_abs(back, unrot) <= 0.1 * np.abs(unrot).max()
 
 
@@ -142,9 +133,9 @@ def test_compress_gated_matches_oracle(case):
     torch.cuda.synchronize()
     got = np64(out)
     assert got.shape == ref.shape
-    if kind == "f32":
-        assert max_abs(got, ref) <= ATOL_F32
-    else:
+    check_out(got, ref, out_dt)
+    if kind != "f32":
+        # and within one bf16 step of the exact value
         assert np.all(np.abs(got - ref) <= np.abs(ref) * 2.0 ** -8 + 1e-5)
 
 
@@ -466,15 +457,15 @@ def test_compress_append_stream_matches_oracle(case):
                                 n_entries=n_ent, hadamard=kind == "e4m3_rot")
     torch.cuda.synchronize()
     ref = oracle.compress(np64(x), np64(W), m, overlap)
+    bound = compress_bound(np64(x), np64(W), m, overlap)
     if kind == "e4m3_rot":
         ref = ref @ _hadamard64(d_out)
+        bound = rotated_bound(bound, np64(x), np64(W), m, overlap)
     N_w = min(N_cap, ref.shape[1])
     assert np.array_equal(n_ent.cpu().numpy(), np.full(B, min(n // m, N_cap), np.int32))
     if kind in ("e4m3", "e4m3_rot"):
-        deq = oracle.dequantize_rows_e4m3(cache.cpu().numpy()[:, :N_w], scale.cpu().numpy()[:, :N_w])
-        r = ref[:, :N_w]
-        sc = scale.cpu().numpy()[:, :N_w]
-        np.testing.assert_allclose(sc, np.abs(r).max(axis=-1) / 448.0, rtol=1e-5)
-        assert np.all(np.abs(deq - r) <= np.abs(r) * 2.0 ** -3 + sc[..., None] * 2.0 ** -9)
+        check_e4m3_rows(cache.cpu().numpy()[:, :N_w], scale.cpu().numpy()[:, :N_w], ref[:, :N_w],
+                        bound[:, :N_w])
     else:
-        check_out(np64(cache)[:, :N_w], ref[:, :N_w], torch.float32 if kind == "f32" else torch.bfloat16)
+        check_compress_stored(np64(cache)[:, :N_w], ref[:, :N_w], bound[:, :N_w],
+                              torch.float32 if kind == "f32" else torch.bfloat16)
