@@ -26,10 +26,11 @@
 // rows), warps 13-16 / 17-20 write the output of M tile 0 / 1.
 // TMEM: S0 [cols 0,128), S1 [128,256), O0 [256,384), O1 [384,512).
 // S = Q K^T (M=128, N<=128, K=128 in 8 steps), P = exp2(S*scale*log2e - m)
-// in bf16 written back into the first 64 columns of S, O += P V with P read
-// from tensor memory and V the same shared tile read as an MN-major operand.  The running sum adds the
-// bf16-rounded weights the MMA actually multiplies, so the result is an
-// exact convex combination of the keys under those weights.  The running max
+// written back over S as two bf16 halves (hi = bf16(P), lo = bf16(P - hi)),
+// O += P_hi V + P_lo V with P read from tensor memory and V the same shared
+// tile read as an MN-major operand.  The running sum adds the weights the
+// MMA actually multiplies (hi + lo, about 16 significant bits), so the
+// result is an exact convex combination of the keys under those weights.  The running max
 // is only raised (and O rescaled in TMEM) when it grows by more than 2^8, so
 // most tiles need no rescale; the final division by the running sum is exact.
 #include <cudaTypedefs.h>
@@ -298,11 +299,29 @@ __device__ __forceinline__ float tile_max(uint32_t s_addr, const uint32_t vm[4],
     return mx;
 }
 
-// P row = exp2(z - m) for the valid columns (0 elsewhere) as bf16 pairs,
-// written over the first 64 columns of S as it goes: chunk q reads S
-// columns [32q, 32q+32) and writes P columns [16q, 16q+16), which have
-// already been read.  Accumulates the exact and the rounded sums.
-// m = +inf writes an all-zero row.
+// The weight p of a key goes to the P.V product as two bf16 numbers,
+// hi = bf16(p) and lo = bf16(p - hi), whose sum carries about 16 significant
+// bits: a single bf16 weight (8 bits) moves the output by up to 2^-8 of the
+// spread of the values it averages, which for keys of magnitude ~16 is
+// several 1e-2.  hi + lo is exact in fp32.
+__device__ __forceinline__ void split_bf16(float p0, float p1, uint32_t& hi, uint32_t& lo, float& h0,
+                                           float& h1, float& s0, float& s1) {
+    __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
+    hi = *reinterpret_cast<uint32_t*>(&hb);
+    h0 = __uint_as_float(hi << 16);
+    h1 = __uint_as_float(hi & 0xffff0000u);
+    __nv_bfloat162 lb = __floats2bfloat162_rn(p0 - h0, p1 - h1);
+    lo = *reinterpret_cast<uint32_t*>(&lb);
+    s0 = h0 + __uint_as_float(lo << 16);
+    s1 = h1 + __uint_as_float(lo & 0xffff0000u);
+}
+
+// P row = exp2(z - m) for the valid columns (0 elsewhere), written over S as
+// it goes: chunk q reads S columns [32q, 32q+32) and writes the chunk's hi
+// weights (bf16 pairs) to columns [32q, 32q+16) and its lo weights to
+// [32q+16, 32q+32), which it has just read.  Accumulates the exact sum and
+// the sum of the weights the MMA multiplies (hi + lo).  m = +inf writes an
+// all-zero row.
 __device__ __forceinline__ void tile_exp(uint32_t s_addr, const uint32_t vm[4], float sl2, float m,
                                          float& se, float& sr) {
     // kept rolled: unrolling lets the compiler interleave chunks past the
@@ -312,19 +331,22 @@ __device__ __forceinline__ void tile_exp(uint32_t s_addr, const uint32_t vm[4], 
         const uint32_t mq = q == 0 ? vm[0] : (q == 1 ? vm[1] : (q == 2 ? vm[2] : vm[3]));
         float sv[32];
         tmem_ld32(s_addr + q * 32, sv);
-        uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-            const float z0 = ((mq >> e) & 1u) ? sv[e] * sl2 : -INFINITY;
-            const float z1 = ((mq >> (e + 1)) & 1u) ? sv[e + 1] * sl2 : -INFINITY;
-            const float p0 = ex2(z0 - m), p1 = ex2(z1 - m);
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-            pk[e >> 1] = *reinterpret_cast<uint32_t*>(&h2);
-            const float2 pr = __bfloat1622float2(h2);
-            se += p0 + p1;
-            sr += pr.x + pr.y;
+        for (int hh = 0; hh < 2; ++hh) {
+            uint32_t pk[8], pl[8];
+#pragma unroll
+            for (int e = 16 * hh; e < 16 * hh + 16; e += 2) {
+                const float z0 = ((mq >> e) & 1u) ? sv[e] * sl2 : -INFINITY;
+                const float z1 = ((mq >> (e + 1)) & 1u) ? sv[e + 1] * sl2 : -INFINITY;
+                const float p0 = ex2(z0 - m), p1 = ex2(z1 - m);
+                float h0, h1, s0, s1;
+                split_bf16(p0, p1, pk[(e >> 1) & 7], pl[(e >> 1) & 7], h0, h1, s0, s1);
+                se += p0 + p1;
+                sr += s0 + s1;
+            }
+            tmem_st8(s_addr + q * 32 + 8 * hh, pk);
+            tmem_st8(s_addr + q * 32 + 16 + 8 * hh, pl);
         }
-        tmem_st16(s_addr + q * 16, pk);
     }
 }
 
@@ -375,18 +397,21 @@ __device__ __forceinline__ void tile_exp_full(uint32_t s_addr, float sl2, float 
     for (int q = 0; q < 4; ++q) {
         float sv[32];
         tmem_ld32(s_addr + q * 32, sv);
-        uint32_t pk[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-            const uint64_t z = f2_fma(f2_pack(sv[e], sv[e + 1]), sl2x2, negm);
-            const float p0 = ex2(__uint_as_float((uint32_t)z)), p1 = ex2(__uint_as_float((uint32_t)(z >> 32)));
-            __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
-            const uint32_t hb = *reinterpret_cast<uint32_t*>(&h2);
-            pk[e >> 1] = hb;
-            accr = f2_add(accr, f2_pack(__uint_as_float(hb << 16), __uint_as_float(hb & 0xffff0000u)));
-            if (want_se) acce = f2_add(acce, f2_pack(p0, p1));
+        for (int hh = 0; hh < 2; ++hh) {
+            uint32_t pk[8], pl[8];
+#pragma unroll
+            for (int e = 16 * hh; e < 16 * hh + 16; e += 2) {
+                const uint64_t z = f2_fma(f2_pack(sv[e], sv[e + 1]), sl2x2, negm);
+                const float p0 = ex2(__uint_as_float((uint32_t)z)), p1 = ex2(__uint_as_float((uint32_t)(z >> 32)));
+                float h0, h1, s0, s1;
+                split_bf16(p0, p1, pk[(e >> 1) & 7], pl[(e >> 1) & 7], h0, h1, s0, s1);
+                accr = f2_add(accr, f2_pack(s0, s1));
+                if (want_se) acce = f2_add(acce, f2_pack(p0, p1));
+            }
+            tmem_st8(s_addr + q * 32 + 8 * hh, pk);
+            tmem_st8(s_addr + q * 32 + 16 + 8 * hh, pl);
         }
-        tmem_st16(s_addr + q * 16, pk);
     }
     sr += __uint_as_float((uint32_t)accr) + __uint_as_float((uint32_t)(accr >> 32));
     se += __uint_as_float((uint32_t)acce) + __uint_as_float((uint32_t)(acce >> 32));
@@ -406,11 +431,10 @@ __device__ __noinline__ void rescale_o(uint32_t o_addr, float alpha) {
     tmem_st_wait();
 }
 
-// 672 threads x at most 88 registers fit one CTA per SM (59,136 of 65,536);
-// this cap (rather than launch bounds, whose occupancy heuristic spilled)
-// lets the allocator keep every role's state in registers.
+// 21 warps sit on the SM's four 16,384-register partitions as 6 + 5 + 5 + 5,
+// so a thread may hold at most 80 registers (6 x 32 x 80 = 15,360).
 template <bool PACKED>
-__global__ void __maxnreg__(88)
+__global__ void __maxnreg__(80)
 attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_c,
                const __grid_constant__ CUtensorMap tm_w, TcParams p) {
     extern __shared__ uint8_t smem_raw[];
@@ -624,11 +648,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         const int ld = L0 + r.load;
                         const int slot = ld % kStages;
                         const uint64_t vd = sw128_desc(smem_u32(sK + slot * kTileBytes), kHalf, 1024);
-                        // P (bf16, two per column) sits in the first 64 columns of S
-                        for (int kk = 0; kk < r.bn / 16; ++kk)
-                            mma_bf16_ts(tmem + 256 + mt * 128, tmem + mt * 128 + kk * 8,
-                                        vd + (uint64_t)(kk * (2048 >> 4)), id_pv,
-                                        (j > 0 || kk > 0) ? 1u : 0u);
+                        // P sits in S (bf16, two per column): keys [32q, 32q+32)
+                        // as hi weights in columns [32q, 32q+16) and lo weights in
+                        // [32q+16, 32q+32); O += P_hi V + P_lo V per 16-key step
+                        for (int kk = 0; kk < r.bn / 16; ++kk) {
+                            const uint32_t pa = tmem + mt * 128 + (kk >> 1) * 32 + (kk & 1) * 8;
+                            const uint64_t vk = vd + (uint64_t)(kk * (2048 >> 4));
+                            mma_bf16_ts(tmem + 256 + mt * 128, pa, vk, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
+                            mma_bf16_ts(tmem + 256 + mt * 128, pa + 16, vk, id_pv, 1u);
+                        }
                         if (r.last_consumer) mma_commit(&ctl->freeb[slot]);
                         if (j + 1 < g.T) {
                             ok = issue_qk(mt, j + 1);
@@ -721,7 +749,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 #pragma unroll
                     for (int i = 0; i < 16; ++i) zero[i] = 0u;
 #pragma unroll
-                    for (int q = 0; q < 4; ++q) tmem_st16(s_addr + q * 16, zero);
+                    for (int q = 0; q < 8; ++q) tmem_st16(s_addr + q * 16, zero);
                 } else {
                     // pass 1: the tile's row max; raise the running max (and
                     // rescale O) when it grows by more than 2^8
