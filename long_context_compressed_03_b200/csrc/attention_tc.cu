@@ -12,27 +12,36 @@
 // tiles (2 tokens x 64 heads each).  Every head of a token attends to the
 // same keys, so a key tile of 128 rows x 128 dims serves a whole M tile.
 //   - window tiles (and dense-mode prefix tiles) are shared by both M tiles
-//     and loaded once per CTA by 2D TMA;
+//     and loaded once per CTA;
 //   - sparse-mode compressed tiles belong to one token: their rows are
-//     gathered with 16-byte cp.async copies by 128 loader threads straight
-//     into the 128-byte-swizzled layout the tensor core reads (many
-//     independent requests in flight), and the rows of the other token in
-//     the M tile are masked.
-// Roles (21 warps): warps 0-3 load (contiguous tiles by TMA; the sparse
-// rows by cp.async, 16 lanes per 256-byte row, from index rows staged in
-// shared memory), warp 4 allocates TMEM, loads Q by TMA and one lane issues
-// every MMA, warps 5-8 / 9-12 run the softmax of M tile 0 / 1 (a warp
-// reaches TMEM lanes 32*(warp%4) .. +31, so each group covers all 128
-// rows), warps 13-16 / 17-20 write the output of M tile 0 / 1.
+//     gathered by index, and the rows of the other token in the M tile are
+//     masked.
+// Arithmetic is fp16 on the tensor cores with fp32 accumulation: the loader
+// warps read the bf16 key rows with 16-byte loads and write them converted
+// to fp16 into the 128-byte-swizzled layout the tensor core reads; Q is
+// converted in shared memory once per unit.  The conversion is exact for
+// magnitudes in [2^-14, 65504] (smaller values keep an absolute error below
+// 2^-25, larger ones saturate at 65504).  fp16 gives the softmax weights P
+// 11 significant bits: a bf16 P (8 bits) moves the output by up to 2^-8 of
+// the spread of the values it averages, several 1e-2 for keys of magnitude
+// ~16.
+// Roles (21 warps): warps 0-3 load (index rows, key tiles, the Q
+// conversion); warp 4 allocates TMEM, loads each unit's Q by TMA and one
+// lane issues every MMA; warps 5-12 and 13-20 run the softmax of M tile 0
+// / 1: each row of an M tile belongs to two threads, one per 64-column half
+// of the key tile (a warp reaches TMEM lanes 32*(warp%4) .. +31), which
+// exchange their half-row maxima through shared memory once per tile; at
+// the end of a unit the same threads normalise O and write their half of
+// each output row.
 // TMEM: S0 [cols 0,128), S1 [128,256), O0 [256,384), O1 [384,512).
 // S = Q K^T (M=128, N<=128, K=128 in 8 steps), P = exp2(S*scale*log2e - m)
-// written back over S as two bf16 halves (hi = bf16(P), lo = bf16(P - hi)),
-// O += P_hi V + P_lo V with P read from tensor memory and V the same shared
-// tile read as an MN-major operand.  The running sum adds the weights the
-// MMA actually multiplies (hi + lo, about 16 significant bits), so the
-// result is an exact convex combination of the keys under those weights.  The running max
-// is only raised (and O rescaled in TMEM) when it grows by more than 2^8, so
-// most tiles need no rescale; the final division by the running sum is exact.
+// in fp16 written back into S (keys [32q, 32q+32) into columns [32q, 32q+16)),
+// O += P V with P read from tensor memory and V the same shared tile read as
+// an MN-major operand.  The running sum adds the fp16-rounded weights the MMA
+// actually multiplies, so the result is an exact convex combination of the
+// keys under those weights.  The running max is only raised (and O rescaled
+// in TMEM) when it grows by more than 2^8, so most tiles need no rescale;
+// the final division by the running sum is exact.
 #include <cudaTypedefs.h>
 
 #include <math.h>
@@ -52,49 +61,52 @@ constexpr int kRows = 128;          // rows of an M tile
 constexpr int kTokens = 4;          // tokens per CTA
 constexpr int kBN = 128;            // keys per tile
 constexpr int kStages = 4;
-#ifndef CSA_ATTN_LOAD_WARPS
-#define CSA_ATTN_LOAD_WARPS 4
-#endif
-constexpr int kLoadWarps = CSA_ATTN_LOAD_WARPS;   // loaders (TMA + cp.async row gathers)
+constexpr int kLoadWarps = 4;                      // loaders: index rows, key tiles, Q conversion
 constexpr int kLoadThreads = kLoadWarps * 32;
 constexpr int kMmaWarp = kLoadWarps;               // TMEM allocation, MMA issue, Q loads
-constexpr int kSoftWarp0 = kLoadWarps + 1;         // 4 + 4 softmax warps for M tiles 0 / 1
-constexpr int kEpiWarp0 = kSoftWarp0 + 8;          // 4 + 4 epilogue warps for M tiles 0 / 1
-constexpr int kThreads = (kLoadWarps + 17) * 32;
-static_assert(kLoadThreads >= 128 && kLoadThreads % 128 == 0, "loaders cover the 128 rows of a tile");
+constexpr int kSoftLo0 = kLoadWarps + 1;           // 4 + 4 warps: columns 0-63 of M tiles 0 / 1
+constexpr int kSoftHi0 = kSoftLo0 + 8;             // 4 + 4 warps: columns 64-127 of M tiles 0 / 1
+constexpr int kSoftWarps = 16;
+constexpr int kThreads = (kLoadWarps + 1 + kSoftWarps) * 32;
+static_assert(kLoadThreads == 128, "loaders cover the 128 rows of a tile, 16 lanes per row");
 constexpr int kHalf = 16384;        // one 64-column half of a 128-row tile
-constexpr int kTileBytes = 32768;   // 128 rows x 128 bf16
+constexpr int kTileBytes = 32768;   // 128 rows x 128 fp16
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kRescaleLog2 = 8.0f;
 
-
 struct __align__(8) Ctrl {
-    uint64_t bar_q;
+    uint64_t bar_q;                 // the unit's Q (bf16) has landed
+    uint64_t q_conv;                // ... and is converted to fp16
     uint64_t q_free;                // the unit's last QK has read Q
     uint64_t o_full[2];             // the unit's last P.V has landed in O
-    uint64_t o_free[2];             // the epilogue has read O
-    uint64_t stats_ready[2];        // the softmax has published the unit's row statistics
+    uint64_t o_free[2];             // the unit's output has been read out of O
     uint64_t full[kStages];
     uint64_t freeb[kStages];
     uint64_t s_full[2];
     uint64_t p_ready[2];
     uint64_t fin;
+    uint64_t xbar[2][4];            // [M tile][quarter]: the two half-row warps meet
     uint32_t mask[kStages][4];      // gathered tiles: valid rows of the stage
     uint32_t tmem_base;
     int abort;
     int load_go;               // loaders: continue with the next load
 };
 
-struct RowStat {            // per row of an M tile at the end of a unit
-    float m, lr, le;
+// Exchange between the two half-row threads of a row (double-buffered by
+// tile and by unit parity).
+struct Xchg {
+    float mx[2][2][2][kRows];       // [tile parity][M tile][half][row]: half-row maximum of S
+    float l[2][2][2][2][kRows];     // [unit parity][M tile][half][rounded / exact][row]: partial sums
 };
-constexpr size_t kStatBytes = sizeof(RowStat) * 2 /*unit parity*/ * 2 /*M tiles*/ * kRows;
 constexpr size_t kSmemFixed = 1024 /*align slack*/ + 2 * kTileBytes /*Q*/ +
-                              kStages * kTileBytes + sizeof(Ctrl) + kStatBytes;
+                              kStages * kTileBytes + sizeof(Ctrl) + sizeof(Xchg);
 // + the CTA's index rows (sparse mode): kTokens * topk int32
 
 struct TcParams {
-    const void* kv_c;          // sparse: [B, N_cap, 128] bf16 (rows gathered by cp.async)
+    const void* kv_c;          // [rows_c, 128] bf16: compressed entries (gathered or a dense prefix)
+    const void* kv_raw;        // [rows_w, 128] bf16: raw rows (the window)
+    const void* q;             // [B * n * 64, 128] bf16 (Q tiles also come by TMA)
+    long rows_c, rows_w;       // rows present in memory (loads beyond them read zeros)
     const int* idx;            // sparse: [B, n, topk]
     int topk;
     const int* n_entries;      // dense
@@ -108,6 +120,36 @@ struct TcParams {
     VarlenMap vl;              // packed sequences (vl.S > 0)
 };
 
+__device__ __forceinline__ int round16(int v) { return (v + 15) & ~15; }
+
+// 2^x with the MUFU instruction (ex2.approx of -inf is +0).
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// A bf16 pair as an fp16 pair (nearest; saturating at +-65504).
+__device__ __forceinline__ uint32_t bf2_to_h2(uint32_t w) {
+    const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xffff0000u);
+    uint32_t d;
+    asm("cvt.rn.satfinite.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    return d;
+}
+__device__ __forceinline__ uint4 bf8_to_h8(uint4 v) {
+    return make_uint4(bf2_to_h2(v.x), bf2_to_h2(v.y), bf2_to_h2(v.z), bf2_to_h2(v.w));
+}
+// Two fp32 weights as an fp16 pair, and the pair's rounded values.
+__device__ __forceinline__ uint32_t f2_to_h2(float lo, float hi, float& rlo, float& rhi) {
+    uint32_t d;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(d) : "f"(hi), "f"(lo));
+    __half2 h = *reinterpret_cast<__half2*>(&d);
+    const float2 r = __half22float2(h);
+    rlo = r.x;
+    rhi = r.y;
+    return d;
+}
+
 struct Geometry {
     int cc;        // sparse: chunks of 128 in a token's index row
     int Tc;        // compressed tiles per M tile
@@ -120,14 +162,7 @@ struct Geometry {
     int Vmax;      // dense: entries needed by the CTA's last token
 };
 
-__device__ __forceinline__ int round16(int v) { return (v + 15) & ~15; }
 
-// 2^x with the MUFU instruction (ex2.approx of -inf is +0).
-__device__ __forceinline__ float ex2(float x) {
-    float y;
-    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-    return y;
-}
 
 // Units of work: unit u covers tokens [t0, t0 + 4) of sequence b, where
 // u = b * units_per_seq + t0 / 4 (packed sequences: u = uoff[b] + t0 / 4).
@@ -282,74 +317,6 @@ __device__ __forceinline__ void valid_bits(int c_lo, int c_hi, const uint32_t gm
     }
 }
 
-// Row max (base-2 scaled) of the valid columns of this thread's S row.
-__device__ __forceinline__ float tile_max(uint32_t s_addr, const uint32_t vm[4], float sl2) {
-    float mx = -INFINITY;
-#pragma unroll 1
-    for (int q = 0; q < 4; ++q) {
-        const uint32_t mq = q == 0 ? vm[0] : (q == 1 ? vm[1] : (q == 2 ? vm[2] : vm[3]));
-        float sv[32];
-        tmem_ld32(s_addr + q * 32, sv);
-#pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const float z = ((mq >> i) & 1u) ? sv[i] * sl2 : -INFINITY;
-            mx = fmaxf(mx, z);
-        }
-    }
-    return mx;
-}
-
-// The weight p of a key goes to the P.V product as two bf16 numbers,
-// hi = bf16(p) and lo = bf16(p - hi), whose sum carries about 16 significant
-// bits: a single bf16 weight (8 bits) moves the output by up to 2^-8 of the
-// spread of the values it averages, which for keys of magnitude ~16 is
-// several 1e-2.  hi + lo is exact in fp32.
-__device__ __forceinline__ void split_bf16(float p0, float p1, uint32_t& hi, uint32_t& lo, float& h0,
-                                           float& h1, float& s0, float& s1) {
-    __nv_bfloat162 hb = __floats2bfloat162_rn(p0, p1);
-    hi = *reinterpret_cast<uint32_t*>(&hb);
-    h0 = __uint_as_float(hi << 16);
-    h1 = __uint_as_float(hi & 0xffff0000u);
-    __nv_bfloat162 lb = __floats2bfloat162_rn(p0 - h0, p1 - h1);
-    lo = *reinterpret_cast<uint32_t*>(&lb);
-    s0 = h0 + __uint_as_float(lo << 16);
-    s1 = h1 + __uint_as_float(lo & 0xffff0000u);
-}
-
-// P row = exp2(z - m) for the valid columns (0 elsewhere), written over S as
-// it goes: chunk q reads S columns [32q, 32q+32) and writes the chunk's hi
-// weights (bf16 pairs) to columns [32q, 32q+16) and its lo weights to
-// [32q+16, 32q+32), which it has just read.  Accumulates the exact sum and
-// the sum of the weights the MMA multiplies (hi + lo).  m = +inf writes an
-// all-zero row.
-__device__ __forceinline__ void tile_exp(uint32_t s_addr, const uint32_t vm[4], float sl2, float m,
-                                         float& se, float& sr) {
-    // kept rolled: unrolling lets the compiler interleave chunks past the
-    // register budget
-#pragma unroll 1
-    for (int q = 0; q < 4; ++q) {
-        const uint32_t mq = q == 0 ? vm[0] : (q == 1 ? vm[1] : (q == 2 ? vm[2] : vm[3]));
-        float sv[32];
-        tmem_ld32(s_addr + q * 32, sv);
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            uint32_t pk[8], pl[8];
-#pragma unroll
-            for (int e = 16 * hh; e < 16 * hh + 16; e += 2) {
-                const float z0 = ((mq >> e) & 1u) ? sv[e] * sl2 : -INFINITY;
-                const float z1 = ((mq >> (e + 1)) & 1u) ? sv[e + 1] * sl2 : -INFINITY;
-                const float p0 = ex2(z0 - m), p1 = ex2(z1 - m);
-                float h0, h1, s0, s1;
-                split_bf16(p0, p1, pk[(e >> 1) & 7], pl[(e >> 1) & 7], h0, h1, s0, s1);
-                se += p0 + p1;
-                sr += s0 + s1;
-            }
-            tmem_st8(s_addr + q * 32 + 8 * hh, pk);
-            tmem_st8(s_addr + q * 32 + 16 + 8 * hh, pl);
-        }
-    }
-}
-
 __device__ __forceinline__ float max3(float a, float b, float c) {
     float r;
     asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
@@ -369,81 +336,136 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
     return d;
 }
 
-// tile_max for a row whose 128 columns are all keys: the max of S, scaled
-// once (the scale is positive, so the maximum element is the same).
-__device__ __forceinline__ float tile_max_full(uint32_t s_addr, float sl2) {
+
+__device__ __forceinline__ float f2lo(uint64_t v) { return __uint_as_float((uint32_t)v); }
+__device__ __forceinline__ float f2hi(uint64_t v) { return __uint_as_float((uint32_t)(v >> 32)); }
+
+// Row max (of raw S: the scale is positive, so the same element) over the
+// valid columns of this thread's 64-column half (S columns at s_half).
+// full: every column of the half is a key of the row.
+__device__ __forceinline__ float half_max(uint32_t s_half, const uint32_t vm[2], bool full) {
     float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll 1
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 2; ++q) {
+        const uint32_t mq = q == 0 ? vm[0] : vm[1];
+        if (!__any_sync(0xffffffffu, mq != 0u)) continue;    // no key in this chunk for the warp
         float sv[32];
-        tmem_ld32(s_addr + q * 32, sv);
+        tmem_ld32(s_half + q * 32, sv);
+        if (full) {
 #pragma unroll
-        for (int i = 0; i < 32; i += 4) {
-            mx0 = max3(mx0, sv[i], sv[i + 1]);
-            mx1 = max3(mx1, sv[i + 2], sv[i + 3]);
+            for (int i = 0; i < 32; i += 4) {
+                mx0 = max3(mx0, sv[i], sv[i + 1]);
+                mx1 = max3(mx1, sv[i + 2], sv[i + 3]);
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+                if ((mq >> i) & 1u) mx0 = fmaxf(mx0, sv[i]);
         }
     }
-    return fmaxf(mx0, mx1) * sl2;
+    return fmaxf(mx0, mx1);
 }
 
-// tile_exp for a row whose 128 columns are all keys, on packed f32x2 math:
-// z = S * scale - m in one rounding, P = 2^z, the rounded weights summed in
-// pairs; the exact sum only when the log-sum-exp is wanted.
-__device__ __forceinline__ void tile_exp_full(uint32_t s_addr, float sl2, float m, bool want_se,
-                                              float& se, float& sr) {
+// P = exp2(S*sl2 - m) for the valid columns (0 elsewhere) of this thread's
+// half, as fp16 pairs written over S: the 32 keys of chunk q (S columns
+// [32q, 32q+32) of the half) get their weights in the chunk's first 16
+// columns, which it has just read.  Accumulates the sum of the rounded
+// weights (sr, what the MMA multiplies) and, when wanted, of the exact ones
+// (se, for the log-sum-exp).  m = +inf writes zeros.
+__device__ __forceinline__ void half_exp(uint32_t s_half, const uint32_t vm[2], bool full, float sl2,
+                                         float m, bool want_se, float& se, float& sr) {
     const uint64_t sl2x2 = f2_pack(sl2, sl2), negm = f2_pack(-m, -m);
     uint64_t accr = 0, acce = 0;      // (+0, +0)
 #pragma unroll 1
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 2; ++q) {
+        const uint32_t mq = q == 0 ? vm[0] : vm[1];
+        uint32_t pk[16];
+        if (!__any_sync(0xffffffffu, mq != 0u)) {
+            // no key in this chunk for the warp: P = 0 without the exponentials
+#pragma unroll
+            for (int i = 0; i < 16; ++i) pk[i] = 0u;
+            tmem_st16(s_half + q * 32, pk);
+            continue;
+        }
         float sv[32];
-        tmem_ld32(s_addr + q * 32, sv);
+        tmem_ld32(s_half + q * 32, sv);
+        if (full) {
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            uint32_t pk[8], pl[8];
-#pragma unroll
-            for (int e = 16 * hh; e < 16 * hh + 16; e += 2) {
+            for (int e = 0; e < 32; e += 2) {
                 const uint64_t z = f2_fma(f2_pack(sv[e], sv[e + 1]), sl2x2, negm);
-                const float p0 = ex2(__uint_as_float((uint32_t)z)), p1 = ex2(__uint_as_float((uint32_t)(z >> 32)));
-                float h0, h1, s0, s1;
-                split_bf16(p0, p1, pk[(e >> 1) & 7], pl[(e >> 1) & 7], h0, h1, s0, s1);
-                accr = f2_add(accr, f2_pack(s0, s1));
+                const float p0 = ex2(f2lo(z)), p1 = ex2(f2hi(z));
+                float r0, r1;
+                pk[e >> 1] = f2_to_h2(p0, p1, r0, r1);
+                accr = f2_add(accr, f2_pack(r0, r1));
                 if (want_se) acce = f2_add(acce, f2_pack(p0, p1));
             }
-            tmem_st8(s_addr + q * 32 + 8 * hh, pk);
-            tmem_st8(s_addr + q * 32 + 16 + 8 * hh, pl);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 32; e += 2) {
+                const float z0 = ((mq >> e) & 1u) ? fmaf(sv[e], sl2, -m) : -INFINITY;
+                const float z1 = ((mq >> (e + 1)) & 1u) ? fmaf(sv[e + 1], sl2, -m) : -INFINITY;
+                const float p0 = ex2(z0), p1 = ex2(z1);
+                float r0, r1;
+                pk[e >> 1] = f2_to_h2(p0, p1, r0, r1);
+                accr = f2_add(accr, f2_pack(r0, r1));
+                if (want_se) acce = f2_add(acce, f2_pack(p0, p1));
+            }
         }
+        tmem_st16(s_half + q * 32, pk);
     }
-    sr += __uint_as_float((uint32_t)accr) + __uint_as_float((uint32_t)(accr >> 32));
-    se += __uint_as_float((uint32_t)acce) + __uint_as_float((uint32_t)(acce >> 32));
+    sr += f2lo(accr) + f2hi(accr);
+    se += f2lo(acce) + f2hi(acce);
 }
 
-// The row max rose by more than 2^8 (or a row sees its first keys): rescale
-// the sums and O.  alpha = 0 for a row without earlier keys.
-__device__ __noinline__ void rescale_o(uint32_t o_addr, float alpha) {
+// The row max rose by more than 2^8: rescale this thread's half of O.
+__device__ __noinline__ void rescale_o_half(uint32_t o_half, float alpha) {
 #pragma unroll 1
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < 2; ++q) {
         float ov[32];
-        tmem_ld32(o_addr + q * 32, ov);
+        tmem_ld32(o_half + q * 32, ov);
 #pragma unroll
         for (int i = 0; i < 32; ++i) ov[i] *= alpha;
-        tmem_st32(o_addr + q * 32, ov);
+        tmem_st32(o_half + q * 32, ov);
     }
     tmem_st_wait();
+}
+
+// A key tile by the loader threads: 128 rows of 256 bytes, 16 lanes per row
+// (16 bytes each), 8 rows per round, 8 rounds of loads in flight before
+// their converted values are stored into the 128-byte-swizzled fp16 layout.
+// src_of(row) gives the row's global address, or nullptr for a zero row.
+template <typename SrcOf>
+__device__ __forceinline__ void load_tile_h(uint8_t* dst, int lt, SrcOf src_of) {
+    const int c16 = lt & 15, half = c16 >> 3, cc = c16 & 7;
+#pragma unroll 1
+    for (int it0 = 0; it0 < kBN / 8; it0 += 8) {
+        uint4 v[8];
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            const int row = (it0 + b) * 8 + (lt >> 4);
+            const uint8_t* src = src_of(row);
+            v[b] = src ? __ldg(reinterpret_cast<const uint4*>(src) + c16) : make_uint4(0u, 0u, 0u, 0u);
+        }
+#pragma unroll
+        for (int b = 0; b < 8; ++b) {
+            const int row = (it0 + b) * 8 + (lt >> 4);
+            *reinterpret_cast<uint4*>(dst + half * kHalf + row * 128 + ((cc ^ (row & 7)) << 4)) = bf8_to_h8(v[b]);
+        }
+    }
 }
 
 // 21 warps sit on the SM's four 16,384-register partitions as 6 + 5 + 5 + 5,
 // so a thread may hold at most 80 registers (6 x 32 x 80 = 15,360).
 template <bool PACKED>
 __global__ void __maxnreg__(80)
-attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_c,
-               const __grid_constant__ CUtensorMap tm_w, TcParams p) {
+attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcParams p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* sQ = base;                                  // [2][32 KB]
     uint8_t* sK = sQ + 2 * kTileBytes;                   // [kStages][32 KB]
     Ctrl* ctl = reinterpret_cast<Ctrl*>(sK + kStages * kTileBytes);
-    RowStat* stats = reinterpret_cast<RowStat*>(ctl + 1);        // [2][2][kRows]
-    int* sIdx = reinterpret_cast<int*>(stats + 4 * kRows);       // [kTokens][topk]
+    Xchg* xc = reinterpret_cast<Xchg*>(ctl + 1);
+    int* sIdx = reinterpret_cast<int*>(xc + 1);          // [kTokens][topk]
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int n_units = PACKED ? p.vl.uoff[p.vl.S] : p.B * ((p.n + kTokens - 1) / kTokens);
@@ -451,17 +473,18 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
 
     if (threadIdx.x == 0) {
         mbar_init(&ctl->bar_q, 1);
+        mbar_init(&ctl->q_conv, kLoadThreads);
         mbar_init(&ctl->q_free, 1);
         for (int s = 0; s < kStages; ++s) {
-            mbar_init(&ctl->full[s], kLoadThreads + 1);
+            mbar_init(&ctl->full[s], kLoadThreads);
             mbar_init(&ctl->freeb[s], 1);
         }
+        for (int i = 0; i < 8; ++i) mbar_init(&ctl->xbar[i >> 2][i & 3], 2);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&ctl->s_full[i], 1);
-            mbar_init(&ctl->p_ready[i], kRows);
+            mbar_init(&ctl->p_ready[i], 8);          // one arrival per softmax warp of the M tile
             mbar_init(&ctl->o_full[i], 1);
-            mbar_init(&ctl->o_free[i], kRows);
-            mbar_init(&ctl->stats_ready[i], kRows);
+            mbar_init(&ctl->o_free[i], 8);
         }
         mbar_init(&ctl->fin, 1);
         // a CTA started after another one timed out does no work
@@ -477,16 +500,15 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
     tc_fence_after();
     const uint32_t tmem = ctl->tmem_base;
 
-    if (warp < kLoadThreads / 32) {
+    if (warp < kLoadWarps) {
         // ------------------------------------------------------------ loaders
-        const int lt = threadIdx.x;                          // 0 .. kLoadThreads-1
-        if (lt == 0) {
-            prefetch_tmap(&tm_c);
-            prefetch_tmap(&tm_w);
-        }
+        const int lt = threadIdx.x;                          // 0 .. 127
+        const uint8_t* kvc = static_cast<const uint8_t*>(p.kv_c);
+        const uint8_t* kvr = static_cast<const uint8_t*>(p.kv_raw);
         int Lg = 0;                                          // loads issued by this CTA
+        int k = 0;                                           // units done
         bool go = true;
-        for (int u = blockIdx.x; u < n_units && go; u += gridDim.x) {
+        for (int u = blockIdx.x; u < n_units && go; u += gridDim.x, ++k) {
             const Unit un = unit_of<PACKED>(p, u);
             const int t0 = un.t0;
             const Geometry g = geometry<PACKED>(p, un);
@@ -503,8 +525,30 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             named_sync(1, kLoadThreads);
             const int NL = total_loads(p, g);
             const int nc = p.dense ? g.Tc : 2 * g.Tc;
-            const uint8_t* kvc_rows = static_cast<const uint8_t*>(p.kv_c) + (size_t)u_ent0<PACKED>(p, un) * (kD * 2);
-            for (int L = 0; L < NL; ++L, ++Lg) {
+            const long ent0 = u_ent0<PACKED>(p, un);
+            const long raw0 = u_raw0<PACKED>(p, un);
+            const int un_n = u_n<PACKED>(p, un), un_N = u_N<PACKED>(p, un), un_L = u_L_raw<PACKED>(p, un);
+            // Q is converted after the unit's first two loads (which need no Q)
+            const int q_at = min(2, NL);
+            for (int L = 0; L <= NL; ++L) {
+                if (L == q_at) {
+                    // the unit's Q (bf16, by TMA) has landed: convert it in place.
+                    // One thread waits and decides for all loaders.
+                    if (lt == 0) ctl->load_go = mbar_wait(&ctl->bar_q, k & 1, abort, p.err) ? 1 : 0;
+                    named_sync(1, kLoadThreads);
+                    if (!ctl->load_go) { go = false; break; }
+#pragma unroll 1
+                    for (int i0 = lt; i0 < 2 * kTileBytes / 16; i0 += 8 * kLoadThreads) {
+                        uint4 v[8];
+#pragma unroll
+                        for (int b = 0; b < 8; ++b) v[b] = *reinterpret_cast<const uint4*>(sQ + (size_t)(i0 + b * kLoadThreads) * 16);
+#pragma unroll
+                        for (int b = 0; b < 8; ++b) *reinterpret_cast<uint4*>(sQ + (size_t)(i0 + b * kLoadThreads) * 16) = bf8_to_h8(v[b]);
+                    }
+                    fence_proxy_async_smem();
+                    mbar_arrive(&ctl->q_conv);
+                }
+                if (L == NL) break;
                 const int slot = Lg % kStages, use = Lg / kStages;
                 uint8_t* dst = sK + slot * kTileBytes;
                 // which tile is load L of the unit?
@@ -532,56 +576,46 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 if (kind == 0) {
                     const int* ir = sIdx + token * p.topk + chunk * kBN;
                     const int tpos = t0 + token;
-                    // valid-row mask: loader thread lt < 128 checks row lt
-                    if (lt < kBN) {
+                    // valid-row mask: loader thread lt checks row lt
+                    {
                         const int c = chunk * kBN + lt;
                         const int sv = (c < p.topk) ? ir[lt] : -1;
-                        const bool ok = tpos < u_n<PACKED>(p, un) && sv >= 0 && sv < u_N<PACKED>(p, un);
-                        const uint32_t bits = __ballot_sync(0xffffffffu, ok);
+                        const bool okr = tpos < un_n && sv >= 0 && sv < un_N;
+                        const uint32_t bits = __ballot_sync(0xffffffffu, okr);
                         if (lane == 0) ctl->mask[slot][warp] = bits;
                     }
-                    // rows: 16 lanes per 256-byte row, kLoadThreads/16 rows per round
-                    constexpr int kRowsPerRound = kLoadThreads / 16;
-                    const int c16 = lt & 15, half = c16 >> 3, cc = c16 & 7;
-#pragma unroll 4
-                    for (int it = 0; it < kBN / kRowsPerRound; ++it) {
-                        const int row = it * kRowsPerRound + (lt >> 4);
+                    load_tile_h(dst, lt, [&](int row) -> const uint8_t* {
                         const int c = chunk * kBN + row;
-                        int sv = (c < p.topk) ? ir[row] : -1;
-                        if (tpos >= u_n<PACKED>(p, un) || sv < 0 || sv >= u_N<PACKED>(p, un)) sv = 0;   // masked; any valid row
-                        const uint8_t* src = kvc_rows + (size_t)sv * (kD * 2) + c16 * 16;
-                        cp_async16(dst + half * kHalf + row * 128 + ((cc ^ (row & 7)) << 4), src);
-                    }
-                    cp_async_arrive_noinc(&ctl->full[slot]);
-                    named_sync(1, kLoadThreads);                 // every mask word is written
-                    if (lt == 0) mbar_arrive(&ctl->full[slot]);  // releases the mask
+                        const int sv = (c < p.topk) ? ir[row] : -1;
+                        // masked rows are zero rows
+                        return (tpos < un_n && sv >= 0 && sv < un_N) ? kvc + (size_t)(ent0 + sv) * (kD * 2) : nullptr;
+                    });
+                } else if (kind == 1) {
+                    load_tile_h(dst, lt, [&](int row) -> const uint8_t* {
+                        const long gr = ent0 + (long)chunk * kBN + row;
+                        return gr < p.rows_c ? kvc + (size_t)gr * (kD * 2) : nullptr;
+                    });
                 } else {
-                    if (lt == 0) {
-                        const CUtensorMap* tm = (kind == 1) ? &tm_c : &tm_w;
-                        const int row = (kind == 1) ? u_ent0<PACKED>(p, un) + chunk * kBN
-                                                    : u_raw0<PACKED>(p, un) + g.p_lo + chunk * kBN;
-                        mbar_arrive_expect_tx(&ctl->full[slot], kTileBytes);
-                        for (int h = 0; h < 2; ++h)
-                            tma_load_2d(dst + h * kHalf, tm, h * 64, row, &ctl->full[slot]);
-                    }
-                    mbar_arrive(&ctl->full[slot]);
+                    load_tile_h(dst, lt, [&](int row) -> const uint8_t* {
+                        const int pos = g.p_lo + chunk * kBN + row;
+                        const long gr = raw0 + pos;
+                        return (pos < un_L && gr < p.rows_w) ? kvr + (size_t)gr * (kD * 2) : nullptr;
+                    });
                 }
+                // the tile (and, for a gathered one, the mask) is written:
+                // visible to the tensor core once every loader has arrived
+                fence_proxy_async_smem();
+                mbar_arrive(&ctl->full[slot]);
+                ++Lg;
             }
         }
-        // drain: copies still in flight must land before the CTA exits
-        cp_async_wait_all();
-        if (lt == 0)
-            for (int Lp = max(0, Lg - kStages); Lp < Lg; ++Lp) {
-                volatile int never = 0;
-                mbar_wait(&ctl->full[Lp % kStages], (Lp / kStages) & 1, &never, p.err);
-            }
     } else if (warp == kMmaWarp) {
         // ------------------------------------------------------------ MMA issuer (+ Q loads)
         if (lane == 0) {
             prefetch_tmap(&tm_q);
-            const uint32_t id_qk_full = idesc_bf16(kRows, kBN, false, false);
-            const uint32_t id_pv = idesc_bf16(kRows, kD, false, true);
-            int q_issued = 0, q_done = 0;     // Q loads issued / waited for
+            const uint32_t id_qk_full = idesc_f16(kRows, kBN, false, false);
+            const uint32_t id_pv = idesc_f16(kRows, kD, false, true);
+            int q_issued = 0, q_done = 0;     // Q loads issued / converted Q waited for
             auto load_q = [&](int u) {
                 ++q_issued;
                 const Unit un = unit_of<PACKED>(p, u);
@@ -601,7 +635,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++k) {
                 const Unit un = unit_of<PACKED>(p, u);
                 const Geometry g = geometry<PACKED>(p, un);
-                ok = q_issued > q_done && mbar_wait(&ctl->bar_q, k & 1, abort, p.err);
+                ok = q_issued > q_done && mbar_wait(&ctl->q_conv, k & 1, abort, p.err);
                 if (ok) ++q_done;
                 tc_fence_after();
                 auto issue_qk = [&](int mt, int j) -> bool {
@@ -614,7 +648,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                     // offset / 16 to the start-address field (no carry: smem < 256 KB)
                     const uint64_t qd = sw128_desc(smem_u32(sQ + mt * kTileBytes), 16, 1024);
                     const uint64_t kd = sw128_desc(smem_u32(sK + slot * kTileBytes), 16, 1024);
-                    const uint32_t idesc = (r.bn == kBN) ? id_qk_full : idesc_bf16(kRows, r.bn, false, false);
+                    const uint32_t idesc = (r.bn == kBN) ? id_qk_full : idesc_f16(kRows, r.bn, false, false);
 #pragma unroll
                     for (int kq = 0; kq < kD / 16; ++kq) {
                         const uint32_t off16 = ((kq >> 2) * kHalf + (kq & 3) * 32) >> 4;
@@ -648,15 +682,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         const int ld = L0 + r.load;
                         const int slot = ld % kStages;
                         const uint64_t vd = sw128_desc(smem_u32(sK + slot * kTileBytes), kHalf, 1024);
-                        // P sits in S (bf16, two per column): keys [32q, 32q+32)
-                        // as hi weights in columns [32q, 32q+16) and lo weights in
-                        // [32q+16, 32q+32); O += P_hi V + P_lo V per 16-key step
-                        for (int kk = 0; kk < r.bn / 16; ++kk) {
-                            const uint32_t pa = tmem + mt * 128 + (kk >> 1) * 32 + (kk & 1) * 8;
-                            const uint64_t vk = vd + (uint64_t)(kk * (2048 >> 4));
-                            mma_bf16_ts(tmem + 256 + mt * 128, pa, vk, id_pv, (j > 0 || kk > 0) ? 1u : 0u);
-                            mma_bf16_ts(tmem + 256 + mt * 128, pa + 16, vk, id_pv, 1u);
-                        }
+                        // P sits in S (fp16, two per column): keys [32q, 32q+32) in
+                        // columns [32q, 32q+16); one 16-key step per MMA
+                        for (int kk = 0; kk < r.bn / 16; ++kk)
+                            mma_bf16_ts(tmem + 256 + mt * 128, tmem + mt * 128 + (kk >> 1) * 32 + (kk & 1) * 8,
+                                       vd + (uint64_t)(kk * (2048 >> 4)), id_pv, (j > 0 || kk > 0) ? 1u : 0u);
                         if (r.last_consumer) mma_commit(&ctl->freeb[slot]);
                         if (j + 1 < g.T) {
                             ok = issue_qk(mt, j + 1);
@@ -676,23 +706,34 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                 J[1] += g.T;
             }
             // every MMA issued must finish before TMEM is released, and a Q
-            // load still in flight (the CTA aborted before waiting for it)
+            // load still in flight (the CTA aborted before it was converted)
             // must land before the CTA's shared memory is given up
             mma_commit(&ctl->fin);
             volatile int never = 0;
             mbar_wait(&ctl->fin, 0, &never, p.err);
-            if (q_issued > q_done) mbar_wait(&ctl->bar_q, q_done & 1, &never, p.err);
+            if (q_issued > 0) mbar_wait(&ctl->bar_q, (q_issued - 1) & 1, &never, p.err);
         }
         __syncwarp();
-    } else if (warp < kEpiWarp0) {
-        // ------------------------------------------------------------ softmax
-        const int mt = (warp - kSoftWarp0) >> 2;
+    } else {
+        // ------------------------------------------------------------ softmax + output
+        const int h = warp >= kSoftHi0 ? 1 : 0;               // which 64-column half of the tile
+        const int mt = ((h ? warp - kSoftHi0 : warp - kSoftLo0) >> 2);
         const int quarter = warp & 3;
         const int r = quarter * 32 + lane;                   // row of the M tile
         const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
         const int u_tok = r >> 6;                            // token of the M tile
-        const uint32_t s_addr = tmem + lane_addr + mt * 128;
-        const uint32_t o_addr = tmem + lane_addr + 256 + mt * 128;
+        const uint32_t s_half = tmem + lane_addr + mt * 128 + 64 * h;
+        const uint32_t o_half = tmem + lane_addr + 256 + mt * 128 + 64 * h;
+        // the row's two threads (two warps) meet on an mbarrier with bounded waits
+        uint64_t* pair_bar = &ctl->xbar[mt][quarter];
+        int xcount = 0;                                      // exchanges so far
+        auto pair_sync = [&]() -> bool {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(pair_bar);
+            const bool okx = __all_sync(0xffffffffu, mbar_wait(pair_bar, xcount & 1, abort, p.err));
+            ++xcount;
+            return okx;
+        };
         int J = 0;                                           // tiles before this unit
         int L0 = 0;                                          // loads before this unit
         int k = 0;
@@ -706,8 +747,8 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
             int Vt = 0;
             if (p.dense && row_ok) Vt = min((t + 1) / p.m, u_ne_dense<PACKED>(p, un));
             const int w_lo = t - p.window + 1;               // window [w_lo, t]
-            // m_used: running max (base 2); l_r: sum of the bf16-rounded weights
-            // (normalises O); l_e: sum of the unrounded weights (the lse output)
+            // m_used: running max (base 2, shared by the row's two threads);
+            // l_r / l_e: this half's sums of the rounded / exact weights
             float m_used = -INFINITY, l_r = 0.0f, l_e = 0.0f;
             for (int j = 0; j < g.T && ok; ++j) {
                 const TileRef tr = tile_ref(p, g, mt, j);
@@ -722,7 +763,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         if (tr.token == u_tok) {
                             const int lg = L0 + tr.load;     // the loaders' index of this tile
                             const int slot = lg % kStages;
-                            // the producer wrote the mask before arming this stage
+                            // the loaders wrote the mask before arriving on this stage
                             if (!__all_sync(0xffffffffu, mbar_wait(&ctl->full[slot], (lg / kStages) & 1, abort, p.err))) { ok = false; break; }
 #pragma unroll
                             for (int q = 0; q < 4; ++q) mw[q] = ctl->mask[slot][q];
@@ -736,80 +777,75 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         c_hi = min(tr.bn, t - p0 + 1) - 1;
                     }
                 }
-                // (s_full of tile j is committed after the P.V of tile j-1 was issued
-                // by the same thread, so that P.V has completed: O is stable and the
-                // P columns are free)
-                uint32_t vm[4];
-                valid_bits(c_lo, c_hi, mw, vm);
-                const bool has = (vm[0] | vm[1] | vm[2] | vm[3]) != 0u;
-                float se = 0.0f, sr = 0.0f;
-                if (!__any_sync(0xffffffffu, has)) {
-                    // no key of this tile is visible to any row of the warp: P = 0
-                    uint32_t zero[16];
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) zero[i] = 0u;
-#pragma unroll
-                    for (int q = 0; q < 8; ++q) tmem_st16(s_addr + q * 16, zero);
-                } else {
-                    // pass 1: the tile's row max; raise the running max (and
-                    // rescale O) when it grows by more than 2^8
-                    const bool full = (vm[0] & vm[1] & vm[2] & vm[3]) == 0xffffffffu;   // uniform per warp
-                    const float mx = full ? tile_max_full(s_addr, p.scale_log2) : tile_max(s_addr, vm, p.scale_log2);
-                    const bool raise = mx > m_used + kRescaleLog2;   // true for a row's first keys
-                    float alpha = 1.0f;
+                uint32_t vm4[4];
+                valid_bits(c_lo, c_hi, mw, vm4);
+                const uint32_t vm[2] = {h ? vm4[2] : vm4[0], h ? vm4[3] : vm4[1]};
+                const bool has = (vm[0] | vm[1]) != 0u;
+                const bool full = (vm[0] & vm[1]) == 0xffffffffu;
+                const bool warp_has = __any_sync(0xffffffffu, has);
+                // pass 1: this half's max; the row's max from both halves
+                float hm = -INFINITY;
+                if (warp_has) hm = half_max(s_half, vm, full);
+                const int par = (J + j) & 1;
+                xc->mx[par][mt][h][r] = hm;
+                if (!pair_sync()) { ok = false; break; }
+                const float tmx = fmaxf(hm, xc->mx[par][mt][h ^ 1][r]);
+                // raise the running max (and rescale O) when it grows by more
+                // than 2^8; both threads of the row decide alike
+                bool raise = false;
+                float alpha = 1.0f;
+                if (tmx > -INFINITY) {
+                    const float mx = tmx * p.scale_log2;
+                    raise = mx > m_used + kRescaleLog2;      // true for a row's first keys
                     if (raise) {
                         alpha = (m_used == -INFINITY) ? 0.0f : ex2(m_used - mx);
                         m_used = mx;
                         l_r *= alpha;
                         l_e *= alpha;
                     }
-                    if (j > 0 && __any_sync(0xffffffffu, raise)) rescale_o(o_addr, alpha);
-                    // pass 2: P = exp2(z - m_used) over S
+                }
+                if (j > 0 && __any_sync(0xffffffffu, raise)) rescale_o_half(o_half, alpha);
+                // pass 2: P = exp2(z - m_used) over this half of S
+                // (s_full of tile j is committed after the P.V of tile j-1 was issued
+                // by the same thread, so that P.V has completed: O is stable and the
+                // P columns are free)
+                if (warp_has) {
                     const float mm = (m_used == -INFINITY) ? INFINITY : m_used;
-                    if (full)
-                        tile_exp_full(s_addr, p.scale_log2, mm, p.lse != nullptr, se, sr);
-                    else
-                        tile_exp(s_addr, vm, p.scale_log2, mm, se, sr);
+                    float se = 0.0f, sr = 0.0f;
+                    half_exp(s_half, vm, full, p.scale_log2, mm, p.lse != nullptr, se, sr);
                     l_r += sr;
                     l_e += se;
+                } else {
+                    // no key of this half is visible to any row of the warp: P = 0
+                    uint32_t zero[16];
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) zero[i] = 0u;
+                    tmem_st16(s_half, zero);
+                    tmem_st16(s_half + 32, zero);
                 }
                 tmem_st_wait();
                 tc_fence_before();
-                mbar_arrive(&ctl->p_ready[mt]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&ctl->p_ready[mt]);
             }
             if (!ok) break;
-            // publish the row statistics of this unit for the epilogue
-            stats[((k & 1) * 2 + mt) * kRows + r] = RowStat{m_used, l_r, l_e};
-            mbar_arrive(&ctl->stats_ready[mt]);
-            J += g.T;
-            L0 += total_loads(p, g);
-        }
-    } else {
-        // ------------------------------------------------------------ epilogue: O / l
-        const int mt = (warp - kEpiWarp0) >> 2;
-        const int quarter = warp & 3;
-        const int r = quarter * 32 + lane;
-        const uint32_t lane_addr = (uint32_t)(quarter * 32) << 16;
-        const int u_tok = r >> 6;
-        const uint32_t o_addr = tmem + lane_addr + 256 + mt * 128;
-        int k = 0;
-        for (int u = blockIdx.x; u < n_units; u += gridDim.x, ++k) {
-            const Unit un = unit_of<PACKED>(p, u);
-            const Geometry g = geometry<PACKED>(p, un);
-            const int t = un.t0 + 2 * mt + u_tok;
-            const bool row_ok = t < u_n<PACKED>(p, un);
-            bool w_ok = mbar_wait(&ctl->stats_ready[mt], k & 1, abort, p.err);
-            const RowStat st = stats[((k & 1) * 2 + mt) * kRows + r];
-            w_ok = w_ok && mbar_wait(&ctl->o_full[mt], k & 1, abort, p.err);
-            if (!__all_sync(0xffffffffu, w_ok)) break;
+            // ---------------------------------------------------------- unit end
+            // the row's sums from both halves, then O / l for this half's 64 dims
+            const int up = k & 1;
+            xc->l[up][mt][h][0][r] = l_r;
+            xc->l[up][mt][h][1][r] = l_e;
+            if (!pair_sync()) break;
+            const float LR = l_r + xc->l[up][mt][h ^ 1][0][r];
+            const float LE = l_e + xc->l[up][mt][h ^ 1][1][r];
+            if (!__all_sync(0xffffffffu, mbar_wait(&ctl->o_full[mt], k & 1, abort, p.err))) break;
             tc_fence_after();
-            __nv_bfloat16* orow = p.out + ((size_t)(u_tok0<PACKED>(p, un) + t) * kH + (r & 63)) * kD;
+            __nv_bfloat16* orow = p.out + ((size_t)(u_tok0<PACKED>(p, un) + t) * kH + (r & 63)) * kD + 64 * h;
             if (g.T > 0) {
-                const float inv = st.lr > 0.0f ? 1.0f / st.lr : 0.0f;
+                const float inv = LR > 0.0f ? 1.0f / LR : 0.0f;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < 2; ++q) {
                     float ov[32];
-                    tmem_ld32(o_addr + q * 32, ov);
+                    tmem_ld32(o_half + q * 32, ov);
                     if (row_ok) {
 #pragma unroll
                         for (int i = 0; i < 32; i += 8) {
@@ -826,16 +862,19 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__
                         }
                     }
                 }
-                if (row_ok && p.lse)
+                if (row_ok && p.lse && h == 0)
                     p.lse[(size_t)(u_tok0<PACKED>(p, un) + t) * kH + (r & 63)] =
-                        st.le > 0.0f ? (st.m + log2f(st.le)) / kLog2e : -INFINITY;
+                        LE > 0.0f ? (m_used + log2f(LE)) / kLog2e : -INFINITY;
             } else if (row_ok) {
                 // no key at all: o = 0, lse = -inf
-                for (int i = 0; i < kD; i += 8) *reinterpret_cast<uint4*>(orow + i) = make_uint4(0, 0, 0, 0);
-                if (p.lse) p.lse[(size_t)(u_tok0<PACKED>(p, un) + t) * kH + (r & 63)] = -INFINITY;
+                for (int i = 0; i < 64; i += 8) *reinterpret_cast<uint4*>(orow + i) = make_uint4(0, 0, 0, 0);
+                if (p.lse && h == 0) p.lse[(size_t)(u_tok0<PACKED>(p, un) + t) * kH + (r & 63)] = -INFINITY;
             }
             tc_fence_before();
-            mbar_arrive(&ctl->o_free[mt]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&ctl->o_free[mt]);
+            J += g.T;
+            L0 += total_loads(p, g);
         }
     }
 
@@ -883,17 +922,16 @@ bool attention_tc_supported(const AttnArgs& a) {
 }
 
 cudaError_t launch_attention_tc(const AttnArgs& a, uint32_t* err, cudaStream_t s) {
-    CUtensorMap tm_q, tm_c, tm_w;
+    CUtensorMap tm_q;
     const uint64_t q_rows = (uint64_t)a.B * a.n_q * kH;
-    const uint64_t c_rows = (uint64_t)a.B * (a.N_cap > 0 ? a.N_cap : 1);
+    const uint64_t c_rows = (uint64_t)a.B * (a.N_cap > 0 ? a.N_cap : 0);
     const uint64_t w_rows = (uint64_t)a.B * a.L_raw;
-    const void* kvc = a.kv_c ? a.kv_c : a.kv_raw;   // any valid address if there are no entries
-    if (!make_map(&tm_q, a.q, q_rows, 128) ||
-        !make_map(&tm_c, kvc, a.N_cap > 0 ? c_rows : w_rows, a.dense ? 128 : 1) ||
-        !make_map(&tm_w, a.kv_raw, w_rows, 128))
-        return cudaErrorInvalidValue;
+    if (!make_map(&tm_q, a.q, q_rows, 128)) return cudaErrorInvalidValue;
     TcParams p;
-    p.kv_c = kvc;
+    p.kv_c = a.kv_c ? a.kv_c : a.kv_raw;   // any valid address when there are no entries
+    p.kv_raw = a.kv_raw;
+    p.rows_c = a.kv_c ? (long)c_rows : 0;
+    p.rows_w = (long)w_rows;
     p.idx = a.idx;
     p.topk = a.dense ? 0 : a.topk;
     p.n_entries = a.n_entries;
@@ -927,7 +965,7 @@ cudaError_t launch_attention_tc(const AttnArgs& a, uint32_t* err, cudaStream_t s
     int dev = 0, sms = 148;
     if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     const int grid = units < sms ? units : sms;     // persistent: one CTA per SM
-    kern<<<(unsigned)grid, kThreads, smem, s>>>(tm_q, tm_c, tm_w, p);
+    kern<<<(unsigned)grid, kThreads, smem, s>>>(tm_q, p);
     count_launch();
     return cudaGetLastError();
 }
