@@ -5,9 +5,14 @@ Headline: CSA prefill queries/s at n = 65536 (batch 1, 64x128 heads MQA, m = 4
 overlapping, fp8 e4m3 indexer 4x64 with per-row scales, top-512, window 512,
 1% 4x-norm outlier keys).  One step = the whole path over one batch:
 compress(kv) -> compress(indexer keys, fp8) -> indexer + top-k -> sparse
-attention.  Also reported: CSA decode tok/s at 128K context (batch 64,
-32768-entry compressed cache, 512-row SWA cache, top-512; one step =
-indexer + top-k -> sparse attention).
+attention.  Also reported, each with its stages' rooflines: the batch-2
+n = 8192 prefill with a bf16 indexer (top-256, window 128), the HCA prefill
+at n = 32768 (m' = 128, dense attention), CSA decode tok/s at 128K context
+(batch 64, 32768-entry compressed cache, 512-row SWA cache, top-512; one
+step = indexer + top-k -> sparse attention) and HCA decode at a 2^20-token
+context.  The e4m3 tensor peak the fp8 indexer is held against is measured
+here (torch._scaled_mm); the HBM and bf16 peaks come from the measured-peaks
+file at the repository root.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 
@@ -37,19 +42,17 @@ sys.path.insert(0, ROOT)
 from long_context_compressed_03_b200 import api, synth  # noqa: E402
 
 PREFILL = "csa_prefill_n64k_fp8idx"
+PREFILL_C2 = "csa_prefill_n8k_bf16"
+HCA_PREFILL = "hca_prefill_n32k"
 DECODE = "csa_decode_b64_ctx128k"
 HCA_DECODE = "hca_decode_b16_ctx1m"
 METRIC = "CSA prefill queries/s at n=64K & decode tok/s at 128K ctx; % HBM/TC roofline"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # DRAM bytes per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
-# keyed by kernel family; valid only while the kernel source hashes the same.
-NCU_TRAFFIC = {
-    # the ncu capture of the prefill attention at n=16384: 307.4 MB read + 220.4 MB
-    # written, scaled by 4 (units = queries) to one n=65536 launch
-    "sparse_attn": {"bytes": (307.403008e6 + 220.389120e6) * 4, "file": "attention_tc.cu",
-                    "src": "ee13d0b93b5e"},
-}
+# keyed by kernel family and workload; valid only while the kernel source
+# hashes the same (a changed kernel reports null traffic).
+NCU_TRAFFIC = {}
 
 
 # ---------------------------------------------------------------------- helpers
@@ -62,10 +65,105 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def measure_fp8_peak(dev, sustain_s=1.5):
+    """Dense e4m3 tensor-core throughput on this GPU: torch._scaled_mm
+    (cuBLASLt) of 8192^3 e4m3 x e4m3 -> bf16 with unit per-tensor scales,
+    2*N^3 flops.  Burst = best of 10 single launches (CUDA events); sustained =
+    back-to-back launches for ``sustain_s`` seconds (the power cap settles
+    within that)."""
+    N = 8192
+    g = torch.Generator(device=dev).manual_seed(7)
+    a = torch.randn(N, N, device=dev, generator=g).to(torch.float8_e4m3fn)
+    b = torch.randn(N, N, device=dev, generator=g).to(torch.float8_e4m3fn).t()   # column-major
+    one = torch.ones((), device=dev, dtype=torch.float32)
+    mm = lambda: torch._scaled_mm(a, b, scale_a=one, scale_b=one, out_dtype=torch.bfloat16)
+    for _ in range(3):
+        mm()
+    torch.cuda.synchronize()
+    best = float("inf")
+    for _ in range(10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        mm()
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    flops = 2.0 * N ** 3
+    # sustained: batches of 20 launches until sustain_s has passed; the last half counts
+    times = []
+    t_end = time.perf_counter() + sustain_s
+    while time.perf_counter() < t_end:
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(20):
+            mm()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1) / 20)
+    tail = times[len(times) // 2:] or times
+    del a, b
+    return {"burst": flops / (best / 1e3) / 1e12,
+            "sustained": flops / (float(np.median(tail)) / 1e3) / 1e12,
+            "how": "measured by bench: torch._scaled_mm e4m3 8192^3 -> bf16, best of 10 "
+                   f"(burst) / median of back-to-back launches over {sustain_s} s (sustained)"}
+
+
+class Peaks:
+    """Roofline denominators: HBM copy GB/s and dense tensor TFLOP/s per
+    operand type, burst (kernel timed alone or in a short region at full
+    clock) and sustained (under the power cap)."""
+
+    def __init__(self, peaks, src, fp8=None):
+        self.hbm = peaks["hbm_gbs"]
+        self.src = src
+        self.tf = {("bf16", "burst"): peaks["bf16_tflops"],
+                   ("bf16", "sustained"): peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])}
+        # fp16 runs at the bf16 rate on the tensor cores (same nominal dense peak)
+        self.tf[("f16", "burst")] = self.tf[("bf16", "burst")]
+        self.tf[("f16", "sustained")] = self.tf[("bf16", "sustained")]
+        if fp8:
+            self.tf[("e4m3", "burst")] = fp8["burst"]
+            self.tf[("e4m3", "sustained")] = fp8["sustained"]
+            self.fp8_src = fp8["how"]
+        else:   # the nominal dense ratio e4m3 : bf16 = 4.5 : 2.25
+            self.tf[("e4m3", "burst")] = 2 * self.tf[("bf16", "burst")]
+            self.tf[("e4m3", "sustained")] = 2 * self.tf[("bf16", "sustained")]
+            self.fp8_src = f"2 x {src} bf16 (nominal dense ratio 4.5 : 2.25 PFLOP/s)"
+
+    def source(self, bound, dtype, regime):
+        if bound == "hbm":
+            return f"{self.src} HBM copy"
+        if dtype == "e4m3":
+            return f"{regime} e4m3: {self.fp8_src}"
+        what = "bf16 (fp16 runs at the bf16 rate)" if dtype == "f16" else "bf16"
+        return f"{self.src} {regime} {what}"
+
+
+def regime_of(clocks, timed_ms):
+    """Burst or sustained peak for kernels timed inside a region: sustained
+    when the sampled clocks show the power cap or a median SM clock more than
+    7% under its maximum, or when the region is seconds long."""
+    sm, smax = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    capped = "sw_power_cap" in clocks.get("reasons", [])
+    low = bool(sm and smax and sm < 0.93 * smax)
+    if capped or low or timed_ms > 2000.0:
+        why = ("sw_power_cap active" if capped else
+               f"median SM clock {sm:.0f} of {smax:.0f} MHz" if low else
+               f"timed region {timed_ms / 1e3:.1f} s")
+        return "sustained", why
+    return "burst", (f"median SM clock {sm:.0f} of {smax:.0f} MHz, no power cap, "
+                     f"timed region {timed_ms:.0f} ms" if sm else "no clock samples")
+
+
 def src_hash(name: str) -> str:
     p = os.path.join(ROOT, "long_context_compressed_03_b200", "csrc", name)
     with open(p, "rb") as f:
         return hashlib.sha1(f.read()).hexdigest()[:12]
+
+
+def ncu_traffic(key):
+    tr = NCU_TRAFFIC.get(key)
+    return tr["bytes"] if tr and tr["src"] == src_hash(tr["file"]) else None
 
 
 def visible(t, m, ne):
@@ -73,18 +171,21 @@ def visible(t, m, ne):
 
 
 def prefill_work(w):
-    """Algorithmic flops / bytes per stage for one prefill step (see DESIGN)."""
+    """Algorithmic flops / bytes per stage for one CSA prefill step: every
+    input read once, every output written once (the per-unit figures of the
+    design notes times the units of one launch)."""
     B, n, H, D, m, k, W = w.B, w.n, w.H, w.D, w.m, w.topk, w.window
     HI, dI = w.H_I, w.d_I
     N_c = n // m
     t = np.arange(n, dtype=np.int64)
     V = visible(t, m, N_c)
     e = 2  # bf16
+    key_bytes = dI + 4 if w.indexer == "e4m3" else dI * e     # fp8 row + scale, or bf16 row
     comp_kv_bytes = B * n * D * e + B * N_c * D * e + D * D * e
-    comp_kI_bytes = B * n * dI * e + B * N_c * (dI * 1 + 4) + dI * dI * e
+    comp_kI_bytes = B * n * dI * e + B * N_c * key_bytes + dI * dI * e
     sel = V > k
     idx_flops = 2.0 * B * HI * dI * float(V[sel].sum())
-    idx_bytes = B * n * HI * dI * e + B * N_c * (dI + 4) + B * n * k * 4
+    idx_bytes = B * n * HI * dI * e + B * N_c * key_bytes + B * n * k * 4
     keys = np.minimum(k, V) + np.minimum(W, t + 1)
     attn_flops = 4.0 * B * H * D * float(keys.sum())
     attn_bytes = 2 * B * n * H * D * e + B * N_c * D * e + B * n * D * e + B * n * k * 4
@@ -109,20 +210,62 @@ def varlen_work(w, lens):
     return tot
 
 
-def roofline_of(work, ms, peaks, timed_alone):
-    """Where one kernel sits against the roofline its algorithmic intensity
-    picks (ridge = measured bf16 TFLOP/s over measured HBM GB/s): achieved
-    flops or bytes per second over that peak.  Kernels timed alone use the
-    burst bf16 figure, kernels inside a long step the sustained one."""
-    tf = peaks["bf16_tflops"] if timed_alone else peaks.get("bf16_tflops_sustained",
-                                                              peaks["bf16_tflops"])
-    ridge = tf * 1e12 / (peaks["hbm_gbs"] * 1e9)
-    if work["flops"] > ridge * max(work["bytes"], 1.0):
+def hca_prefill_work(w):
+    """HCA prefill: compress (m' non-overlapping) then dense attention over
+    every visible entry plus the window."""
+    B, n, H, D, m, W = w.B, w.n, w.H, w.D, w.m, w.window
+    N_c = n // m
+    t = np.arange(n, dtype=np.int64)
+    keys = visible(t, m, N_c) + np.minimum(W, t + 1)
+    e = 2
+    return {
+        "compress_kv": dict(bytes=B * n * D * e + B * N_c * D * e + D * D * e,
+                            flops=2.0 * B * N_c * D * D),
+        "hca_dense_attn": dict(bytes=2 * B * n * H * D * e + B * N_c * D * e + B * n * D * e,
+                               flops=4.0 * B * H * D * float(keys.sum())),
+    }
+
+
+# Which roofline bounds each stage, and the operand type of its contraction.
+STAGE_BOUND = {
+    "compress_kv": ("hbm", None), "compress_kI": ("hbm", None),
+    "indexer_topk": ("tensor", None),      # e4m3 or bf16, by the workload's indexer type
+    "sparse_attn": ("tensor", "f16"), "hca_dense_attn": ("tensor", "f16"),
+}
+
+
+def roofline_of(work, ms, peaks, regime, bound=None, dtype="bf16"):
+    """One kernel against its roofline: achieved flops (tensor-bound) or
+    bytes (HBM-bound) per second over the peak for its operand type and
+    regime.  bound=None picks by intensity against the ridge point."""
+    tf = peaks.tf[(dtype, regime)]
+    if bound is None:
+        ridge = tf * 1e12 / (peaks.hbm * 1e9)
+        bound = "tensor" if work["flops"] > ridge * max(work["bytes"], 1.0) else "hbm"
+    if bound == "tensor":
         a = work["flops"] / (ms / 1e3) / 1e12
-        return {"bound": "tensor", "achieved": a, "peak": tf, "unit": "TFLOP/s", "frac": a / tf}
-    a = work["bytes"] / (ms / 1e3) / 1e9
-    return {"bound": "hbm", "achieved": a, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": a / peaks["hbm_gbs"]}
+        r = {"bound": "tensor", "achieved": a, "peak": tf, "unit": "TFLOP/s", "frac": a / tf}
+    else:
+        a = work["bytes"] / (ms / 1e3) / 1e9
+        r = {"bound": "hbm", "achieved": a, "peak": peaks.hbm, "unit": "GB/s",
+             "frac": a / peaks.hbm}
+    r["peak_source"] = peaks.source(r["bound"], dtype, regime)
+    return r
+
+
+def stage_rooflines(work, kern_ms, peaks, regime, indexer_dtype="bf16"):
+    out = {}
+    total = sum(kern_ms.values())
+    for nm, ms in kern_ms.items():
+        bound, dt = STAGE_BOUND[nm]
+        if nm == "indexer_topk":
+            dt = indexer_dtype
+        wk = work[nm]
+        out[nm] = {"ms": ms, "share": ms / max(1e-9, total),
+                   "TFLOP/s": wk["flops"] / (ms / 1e3) / 1e12,
+                   "GB/s": wk["bytes"] / (ms / 1e3) / 1e9,
+                   "roofline": roofline_of(wk, ms, peaks, regime, bound, dt or "bf16")}
+    return out
 
 
 def decode_work(w, inp):
@@ -205,24 +348,23 @@ class ClockSampler:
 
 # ---------------------------------------------------------------------- our arm
 class PrefillPath:
-    """Device buffers + the four ABI calls of one prefill step."""
+    """Device buffers + the four ABI calls of one CSA prefill step."""
 
     def __init__(self, w, inp, dev):
         self.w = w
         self.d = {k: v.to(dev) for k, v in inp.items()}
         B, n = w.B, w.n
         N_c = n // w.m
+        self.fp8 = w.indexer == "e4m3"
         self.kv_c = torch.empty(B, N_c, w.D, dtype=torch.bfloat16, device=dev)
-        self.kI_c = torch.empty(B, N_c, w.d_I, dtype=torch.uint8, device=dev)
-        self.kI_s = torch.empty(B, N_c, dtype=torch.float32, device=dev)
+        self.kI_c = torch.empty(B, N_c, w.d_I, dtype=torch.uint8 if self.fp8 else torch.bfloat16,
+                                device=dev)
+        self.kI_s = torch.empty(B, N_c, dtype=torch.float32, device=dev) if self.fp8 else None
         self.idx = torch.empty(B, n, w.topk, dtype=torch.int32, device=dev)
         self.out = torch.empty_like(self.d["q"])
         self.names = ["compress_kv", "compress_kI", "indexer_topk", "sparse_attn"]
-        self.ev = None
-
-    def step(self, record=False):
-        d, w = self.d, self.w
-        calls = [
+        d = self.d
+        self.calls = [
             lambda: api.csa_compress(d["kv"], d["W_c"], w.m, True, self.kv_c),
             lambda: api.csa_compress(d["kI_raw"], d["W_Ic"], w.m, True, self.kI_c, self.kI_s),
             lambda: api.csa_indexer_topk(d["qI"], self.kI_c, w.m, w.topk, self.idx,
@@ -230,21 +372,40 @@ class PrefillPath:
             lambda: api.csa_sparse_attn(d["q"], self.kv_c, self.idx, d["kv"], w.window,
                                         self.out),
         ]
+
+    def step(self, record=False):
         if not record:
-            for c in calls:
+            for c in self.calls:
                 c()
             return None
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)]
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(self.calls) + 1)]
         evs[0].record()
-        for i, c in enumerate(calls):
+        for i, c in enumerate(self.calls):
             c()
             evs[i + 1].record()
         return evs
 
 
-def run_prefill(w, dev, steps, warmup, dist_ctx, rank):
-    inp = synth.csa_prefill_inputs(w, seed=rank)
-    path = PrefillPath(w, inp, dev)
+class HcaPrefillPath(PrefillPath):
+    """The HCA prefill step: compress (m' non-overlapping) -> hca_dense_attn."""
+
+    def __init__(self, w, inp, dev):
+        self.w = w
+        self.d = d = {k: v.to(dev) for k, v in inp.items()}
+        self.kv_c = torch.empty(w.B, w.n // w.m, w.D, dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty_like(d["q"])
+        self.names = ["compress_kv", "hca_dense_attn"]
+        self.calls = [
+            lambda: api.csa_compress(d["kv"], d["W_c"], w.m, False, self.kv_c),
+            lambda: api.hca_dense_attn(d["q"], self.kv_c, w.m, d["kv"], w.window, self.out),
+        ]
+
+
+def run_path(path, steps, warmup, dist_ctx):
+    """Times K steps of a path bracketed by a barrier and synchronize.  The
+    step time is the whole region's; a stage's time is its median over the
+    steps (events between stages measure the kernel once the queue is ahead
+    of the GPU, which holds after the first timed step)."""
     for _ in range(warmup):
         path.step()
     torch.cuda.synchronize()
@@ -263,13 +424,9 @@ def run_prefill(w, dev, steps, warmup, dist_ctx, rank):
         dist_ctx.barrier()
     launches = api.csa_kernel_launches() - launches0
     total_ms = start.elapsed_time(end)
-    kern_ms = {nm: 0.0 for nm in path.names}
-    for evs in per_step:
-        for i, nm in enumerate(path.names):
-            kern_ms[nm] += evs[i].elapsed_time(evs[i + 1])
-    kern_ms = {k: v / steps for k, v in kern_ms.items()}
-    return dict(total_ms=total_ms, kern_ms=kern_ms, launches=launches, clocks=clocks.summary(),
-                path=path, inp=inp)
+    kern_ms = {nm: float(np.median([evs[i].elapsed_time(evs[i + 1]) for evs in per_step]))
+               for i, nm in enumerate(path.names)}
+    return dict(total_ms=total_ms, kern_ms=kern_ms, launches=launches, clocks=clocks.summary())
 
 
 def run_variants(w, path, dev, steps, rank, peaks):
@@ -304,6 +461,8 @@ def run_variants(w, path, dev, steps, rank, peaks):
         "compress_kI_hadamard": prefill_work(w)["compress_kI"],
         "indexer_topk_gated_hadamard": prefill_work(w)["indexer_topk"],
     }
+    bounds = {"compress_gated_kv": (None, "bf16"), "compress_kI_hadamard": ("hbm", "bf16"),
+              "indexer_topk_gated_hadamard": ("tensor", "e4m3")}
     out = {}
     for name, fn in calls.items():
         for _ in range(2):
@@ -317,10 +476,10 @@ def run_variants(w, path, dev, steps, rank, peaks):
             b_.record()
             ts.append((a_, b_))
         torch.cuda.synchronize()
-        ms = float(np.mean([a_.elapsed_time(b_) for a_, b_ in ts]))
+        ms = float(np.median([a_.elapsed_time(b_) for a_, b_ in ts]))
         out[name] = {"ms": ms, "TFLOP/s": work[name]["flops"] / (ms / 1e3) / 1e12,
                      "GB/s": work[name]["bytes"] / (ms / 1e3) / 1e9,
-                     "roofline": roofline_of(work[name], ms, peaks, timed_alone=True)}
+                     "roofline": roofline_of(work[name], ms, peaks, "burst", *bounds[name])}
     del flush
     return out
 
@@ -362,7 +521,7 @@ def run_prefill_varlen(w, path, dev, steps, warmup, S=8):
     recs = [step() for _ in range(steps)]
     torch.cuda.synchronize()
     ms = float(np.mean([r[0].elapsed_time(r[4]) for r in recs]))
-    stages = {nm: float(np.mean([r[i].elapsed_time(r[i + 1]) for r in recs]))
+    stages = {nm: float(np.median([r[i].elapsed_time(r[i + 1]) for r in recs]))
               for i, nm in enumerate(names)}
     return dict(lens=lens, T=T, ms=ms, stages=stages)
 
@@ -488,8 +647,9 @@ def run_decode(dev, steps, warmup, rank):
     t_att = [r[2].elapsed_time(r[3]) for r in recs]
     tot = [a + b for a, b in zip(t_idx, t_att)]
     return dict(w=w, inp=inp, ms=float(np.mean(tot)), ms_median=float(np.median(tot)),
-                kern_ms={"indexer_topk": float(np.mean(t_idx)), "sparse_attn": float(np.mean(t_att))},
-                append_ms=float(np.mean(t_app)))
+                kern_ms={"indexer_topk": float(np.median(t_idx)),
+                         "sparse_attn": float(np.median(t_att))},
+                append_ms=float(np.median(t_app)))
 
 
 def run_decode_paged(dev, steps, warmup, rank, page_size=64):
@@ -540,7 +700,8 @@ def run_decode_paged(dev, steps, warmup, rank, page_size=64):
     t_att = [r[1].elapsed_time(r[2]) for r in recs]
     tot = [a + b for a, b in zip(t_idx, t_att)]
     return dict(w=w, ms=float(np.mean(tot)), page_size=page_size, work=decode_work(w, inp),
-                kern_ms={"indexer_topk": float(np.mean(t_idx)), "sparse_attn": float(np.mean(t_att))})
+                kern_ms={"indexer_topk": float(np.median(t_idx)),
+                         "sparse_attn": float(np.median(t_att))})
 
 
 def run_hca_decode(dev, steps, warmup, rank):
@@ -577,39 +738,69 @@ def run_hca_decode(dev, steps, warmup, rank):
 
 # ---------------------------------------------------------------------- oracle arm
 def oracle_prefill_sample(w, inp, n_sample, seed=5):
-    """The fp64 oracle on a bounded sample of the prefill workload: both
-    compressors over the whole sequence, then indexer + top-k and attention
-    for n_sample sampled queries.  Returns (seconds per query, detail)."""
+    """The fp64 oracle on a bounded sample of a CSA prefill workload: both
+    compressors over every token, then indexer + top-k and attention for
+    n_sample sampled queries of the first sequence (fp8 indexers quantise
+    keys and queries as the kernels do; bf16 ones score the bf16-stored
+    keys).  Returns (seconds per query, detail)."""
     import oracle
     f64 = lambda t: t.detach().to("cpu", torch.float64).numpy()
-    n = w.n
+    B, n = w.B, w.n
     t0 = time.perf_counter()
     kv_c = oracle.compress(f64(inp["kv"]), f64(inp["W_c"]), w.m, True)
     kI_c = oracle.compress(f64(inp["kI_raw"]), f64(inp["W_Ic"]), w.m, True)
     t_comp = time.perf_counter() - t0
-    codes, scales = oracle.quantize_rows_e4m3(kI_c.astype(np.float32))
     rows = synth.query_sample(n, w.m, w.window, n_sample, seed=seed).numpy()[:n_sample]
     rb = np.zeros(rows.size, np.int32)
     rt = rows.astype(np.int32)
-    qrows = oracle.quantized_query_rows(inp["qI"][0, rows].float().numpy())
+    if w.indexer == "e4m3":
+        keys, scales = oracle.quantize_rows_e4m3(kI_c.astype(np.float32))
+        qrows = oracle.quantized_query_rows(inp["qI"][0, rows].float().numpy())
+    else:
+        keys = torch.from_numpy(kI_c).to(torch.bfloat16).double().numpy()
+        scales = None
+        qrows = f64(inp["qI"][0, rows])
     t1 = time.perf_counter()
-    idx, _, _ = oracle.indexer_topk_rows(qrows, rb, rt, codes, w.m, w.topk,
-                                         np.array([n // w.m], np.int32), scales)
+    idx, _, _ = oracle.indexer_topk_rows(qrows, rb, rt, keys, w.m, w.topk,
+                                         np.full(B, n // w.m, np.int32), scales)
     oracle.sparse_attn_rows(f64(inp["q"][0, rows]), rb, rt, kv_c, idx, f64(inp["kv"]), w.window)
     t_rows = time.perf_counter() - t1
-    per_query = t_comp / n + t_rows / rows.size
-    return per_query, dict(compress_s=t_comp, rows=int(rows.size), rows_s=t_rows)
+    per_query = t_comp / (B * n) + t_rows / rows.size
+    return per_query, dict(compress_s=t_comp, rows=int(rows.size), rows_s=t_rows,
+                           wall_s=time.perf_counter() - t0)
 
 
-def cpu_baseline(w, inp, n_sample):
+def oracle_hca_prefill_sample(w, inp, n_sample, seed=6):
+    """The fp64 oracle on a bounded sample of the HCA prefill: compress every
+    token, dense attention for n_sample sampled queries."""
     import oracle
-    per_q, det = oracle_prefill_sample(w, inp, n_sample)
+    f64 = lambda t: t.detach().to("cpu", torch.float64).numpy()
+    n = w.n
+    t0 = time.perf_counter()
+    kv_c = oracle.compress(f64(inp["kv"]), f64(inp["W_c"]), w.m, False)
+    t_comp = time.perf_counter() - t0
+    rows = synth.query_sample(n, w.m, w.window, n_sample, seed=seed).numpy()[:n_sample]
+    rb = np.zeros(rows.size, np.int32)
+    t1 = time.perf_counter()
+    oracle.hca_attn_rows(f64(inp["q"][0, rows]), rb, rows.astype(np.int32), kv_c, w.m,
+                         f64(inp["kv"]), w.window)
+    t_rows = time.perf_counter() - t1
+    return t_comp / (w.B * n) + t_rows / rows.size, dict(compress_s=t_comp, rows=int(rows.size),
+                                                         rows_s=t_rows)
+
+
+def cpu_baseline(w, inp, n_sample, hca=False):
+    import oracle
+    fn = oracle_hca_prefill_sample if hca else oracle_prefill_sample
+    per_q, det = fn(w, inp, n_sample)
+    what = "the compressor" if hca else "both compressors"
+    rest = "dense attention" if hca else "indexer/top-k and attention"
     return {"value": 1.0 / per_q, "unit": "queries/s", "cores": oracle.num_threads(),
             "kind": "oracle",
-            "sample": (f"fp64 oracle: both compressors over all {w.n} tokens "
-                       f"({det['compress_s']:.2f} s) + indexer/top-k and attention for "
-                       f"{det['rows']} of {w.n} queries ({det['rows_s']:.2f} s); "
-                       f"queries/s = 1 / (compress_s/n + rows_s/rows)")}
+            "sample": (f"fp64 oracle: {what} over all {w.B * w.n} tokens "
+                       f"({det['compress_s']:.2f} s) + {rest} for {det['rows']} of "
+                       f"{w.B * w.n} queries ({det['rows_s']:.2f} s); "
+                       f"queries/s = 1 / (compress_s/tokens + rows_s/rows)")}
 
 
 # ---------------------------------------------------------------------- distributed
@@ -675,6 +866,10 @@ def main():
                     help="run only the decode steps (profiler captures of the decode kernels)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the c2 (n=8192, bf16 indexer) and HCA prefill (n=32768) lines")
+    ap.add_argument("--no-fp8-peak", action="store_true",
+                    help="skip the e4m3 peak measurement (the nominal ratio to bf16 is used)")
     args = ap.parse_args()
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -695,23 +890,26 @@ def main():
         import oracle
         inp = synth.csa_prefill_inputs(w, seed=0)
         sample = max(16, args.cpu_sample // 4)
-        times = []
         for _ in range(args.warmup):
             oracle_prefill_sample(w, inp, 16)
+        per_qs, walls = [], []
         for i in range(args.steps):
             per_q, det = oracle_prefill_sample(w, inp, sample, seed=10 + i)
-            times.append(per_q)
-        per_q = float(np.mean(times))
-        v = 1.0 / per_q
+            per_qs.append(per_q)
+            walls.append(det["wall_s"])
+        v = 1.0 / float(np.mean(per_qs))
         line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "queries/s",
                 "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": per_q * w.n * 1e3, "higher_is_better": True, "scaling": "weak",
-                "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1))",
-                "config": config,
+                "ms_per_step": float(np.mean(walls)) * 1e3, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic (seeded N(0,1))", "config": config,
                 "cpu_baseline": {"value": v, "unit": "queries/s", "cores": oracle.num_threads(),
                                  "kind": "oracle",
-                                 "sample": f"{sample} sampled queries per step + full compress, "
-                                           f"extrapolated to n={w.n}"},
+                                 "sample": f"one step = both compressors over all {w.n} tokens + "
+                                           f"indexer/top-k and attention for {sample} sampled "
+                                           "queries (ms_per_step is that step's measured wall "
+                                           "time); value = queries/s over the whole workload, "
+                                           "1 / (compress_s/n + rows_s/rows)"},
                 "e2e": {"value": v, "unit": "queries/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}}
         print(json.dumps(line))
@@ -722,8 +920,9 @@ def main():
     dev = torch.device("cuda", dist_ctx.local)
     torch.cuda.set_device(dev)
     api.load()
-    peaks, peak_src = load_peaks()
+    raw_peaks, peak_src = load_peaks()
     if args.decode_only:
+        peaks = Peaks(raw_peaks, peak_src)
         dec = run_decode(dev, args.steps, args.warmup, rank)
         hd = run_hca_decode(dev, args.steps, args.warmup, rank)
         dval, dms = dist_ctx.job_rate(dec["w"].B, dec["ms"])
@@ -739,40 +938,72 @@ def main():
         dist_ctx.close()
         return 0
 
-    pre = run_prefill(w, dev, args.steps, args.warmup, dist_ctx, rank)
-    value, ms_step = dist_ctx.job_rate(w.B * w.n, pre["total_ms"] / args.steps)
+    fp8 = None
+    if not args.no_fp8_peak:
+        try:
+            fp8 = measure_fp8_peak(dev)
+        except Exception as e:  # no fp8 GEMM in this torch build
+            print(f"warning: fp8 peak not measured ({e})", file=sys.stderr)
+    peaks = Peaks(raw_peaks, peak_src, fp8)
+    torch.cuda.empty_cache()
 
+    inp = synth.csa_prefill_inputs(w, seed=rank)
+    path = PrefillPath(w, inp, dev)
+    pre = run_path(path, args.steps, args.warmup, dist_ctx)
+    value, ms_step = dist_ctx.job_rate(w.B * w.n, pre["total_ms"] / args.steps)
+    regime, regime_why = regime_of(pre["clocks"], pre["total_ms"])
     work = prefill_work(w)
+    stages = stage_rooflines(work, pre["kern_ms"], peaks, regime, "e4m3")
     dom = max(pre["kern_ms"], key=pre["kern_ms"].get)
-    dom_work = work[dom]
-    tensor_kernels = {"sparse_attn", "indexer_topk"}
-    if dom in tensor_kernels:
-        achieved = dom_work["flops"] / (pre["kern_ms"][dom] / 1e3) / 1e12
-        peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
-        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak}
-    else:
-        achieved = dom_work["bytes"] / (pre["kern_ms"][dom] / 1e3) / 1e9
-        peak = peaks["hbm_gbs"]
-        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                "frac": achieved / peak}
-    tr = NCU_TRAFFIC.get(dom)
-    roof["traffic"] = tr["bytes"] if tr and tr["src"] == src_hash(tr["file"]) else None
+    roof = {k: v for k, v in stages[dom]["roofline"].items()}
+    roof["traffic"] = ncu_traffic((dom, PREFILL))
     roof["kernel"] = dom
-    roof["peak_source"] = f"{peak_src} ({'sustained bf16' if roof['unit'] == 'TFLOP/s' else 'hbm copy'})"
-    stages = {}
-    for nm, ms in pre["kern_ms"].items():
-        wk = work[nm]
-        stages[nm] = {"ms": ms, "share": ms / max(1e-9, sum(pre["kern_ms"].values())),
-                      "TFLOP/s": wk["flops"] / (ms / 1e3) / 1e12,
-                      "GB/s": wk["bytes"] / (ms / 1e3) / 1e9}
+    roof["regime"] = f"{regime}: {regime_why}"
 
     line = {"metric": METRIC, "value": value, "unit": "queries/s", "n_gpus": dist_ctx.world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic (seeded N(0,1), 1% 4x outlier keys)", "config": config,
             "roofline": roof, "stages": stages, "gpu_launches": pre["launches"],
-            "clocks": pre["clocks"]}
+            "clocks": pre["clocks"],
+            "peaks": {"hbm_gbs": peaks.hbm, "bf16_tflops": peaks.tf[("bf16", "burst")],
+                      "bf16_tflops_sustained": peaks.tf[("bf16", "sustained")],
+                      "e4m3_tflops": peaks.tf[("e4m3", "burst")],
+                      "e4m3_tflops_sustained": peaks.tf[("e4m3", "sustained")],
+                      "e4m3_source": peaks.fp8_src, "source": peak_src}}
+    if rank == 0 and dist_ctx.world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, inp, args.cpu_sample)
+
+    if not args.no_configs:
+        # the other two prefill configurations, each timed like the headline
+        for name, mk, path_cls, hca, n_cpu in (
+                (PREFILL_C2, synth.csa_prefill_inputs, PrefillPath, False, 1024),
+                (HCA_PREFILL, synth.hca_prefill_inputs, HcaPrefillPath, True, 256)):
+            wc = synth.WORKLOADS[name]
+            inp_c = mk(wc, seed=rank)
+            pc = path_cls(wc, inp_c, dev)
+            rc = run_path(pc, args.steps, args.warmup, dist_ctx)
+            cval, cms = dist_ctx.job_rate(wc.B * wc.n, rc["total_ms"] / args.steps)
+            creg, creg_why = regime_of(rc["clocks"], rc["total_ms"])
+            cwork = hca_prefill_work(wc) if hca else prefill_work(wc)
+            cst = stage_rooflines(cwork, rc["kern_ms"], peaks, creg, wc.indexer)
+            cdom = max(rc["kern_ms"], key=rc["kern_ms"].get)
+            croof = dict(cst[cdom]["roofline"], kernel=cdom, regime=f"{creg}: {creg_why}",
+                         traffic=ncu_traffic((cdom, name)))
+            entry = {"workload": name, "value": cval, "unit": "queries/s", "ms_per_step": cms,
+                     "B": wc.B, "n": wc.n, "m": wc.m, "overlap": wc.overlap,
+                     "l2": "inputs larger than L2 (q alone is 256 MiB or more)",
+                     "roofline": croof, "stages": cst, "gpu_launches": rc["launches"],
+                     "clocks": rc["clocks"]}
+            if not hca:
+                entry.update(topk=wc.topk, window=wc.window, indexer=f"{wc.indexer} {wc.H_I}x{wc.d_I}")
+            else:
+                entry.update(window=wc.window, attention="dense over every visible entry + window")
+            if rank == 0 and dist_ctx.world == 1 and not args.no_cpu_baseline:
+                entry["cpu_baseline"] = cpu_baseline(wc, inp_c, n_cpu, hca=hca)
+            line["hca_prefill" if hca else "c2_prefill"] = entry
+            del pc, inp_c
+            torch.cuda.empty_cache()
 
     if not args.no_variants:
         line["variants"] = {
@@ -780,23 +1011,22 @@ def main():
             "note": "NEXT rows, each timed alone: gated-softmax compressor (kv, d 128, m 4 "
                     "overlapping), Hadamard-rotated fp8 indexer keys, gated indexer + top-k "
                     "against rotated keys",
-            **run_variants(w, pre["path"], dev, max(3, args.steps), rank, peaks)}
+            **run_variants(w, path, dev, max(3, args.steps), rank, peaks)}
     if not args.no_variants:
-        pv = run_prefill_varlen(w, pre["path"], dev, max(3, args.steps), args.warmup)
+        pv = run_prefill_varlen(w, path, dev, max(3, args.steps), args.warmup)
         vval, vms = dist_ctx.job_rate(pv["T"], pv["ms"])
         line["prefill_varlen"] = {
             "workload": "csa_prefill_packed8_n64k_fp8idx", "value": vval, "unit": "queries/s",
             "ms_per_step": vms, "lengths": pv["lens"], "stages_ms": pv["stages"],
-            "roofline": {nm: roofline_of(wk, pv["stages"][nm], peaks, timed_alone=False)
-                         for nm, wk in varlen_work(w, pv["lens"]).items()},
+            "stages": stage_rooflines(varlen_work(w, pv["lens"]), pv["stages"], peaks, regime,
+                                      "e4m3"),
             "note": "the c3 tokens re-cut into 8 packed sequences (csa_*_varlen entry points); "
                     "less causal work than one 64K sequence, so not comparable to the headline"}
     if not args.no_decode:
         dec = run_decode(dev, args.steps, args.warmup, rank)
         dval, dms = dist_ctx.job_rate(dec["w"].B, dec["ms"])
         dw = decode_work(dec["w"], dec["inp"])
-        dstages = {nm: {"ms": ms, "GB/s": dw[nm]["bytes"] / (ms / 1e3) / 1e9,
-                        "frac_hbm": dw[nm]["bytes"] / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+        dstages = {nm: {"ms": ms, "roofline": roofline_of(dw[nm], ms, peaks, "burst", "hbm")}
                    for nm, ms in dec["kern_ms"].items()}
         line["decode"] = {"workload": DECODE, "value": dval,
                           "unit": "tok/s", "ms_per_step": dms, "ms_median": dec["ms_median"],
@@ -809,7 +1039,8 @@ def main():
         line["decode_paged"] = {"workload": DECODE, "value": pval, "unit": "tok/s",
                                 "ms_per_step": pms, "page_size": dp["page_size"],
                                 "stages_ms": dp["kern_ms"],
-                                "roofline": {nm: roofline_of(dp["work"][nm], ms_, peaks, True)
+                                "roofline": {nm: roofline_of(dp["work"][nm], ms_, peaks, "burst",
+                                                             "hbm")
                                              for nm, ms_ in dp["kern_ms"].items()},
                                 "l2": "flushed (512 MiB write) between steps",
                                 "note": "the decode step over caches scattered into a shuffled "
@@ -819,19 +1050,17 @@ def main():
         line["hca_decode"] = {"workload": HCA_DECODE, "value": hval,
                               "unit": "tok/s", "ms_per_step": hms, "ms_median": hd["ms_median"],
                               "l2": "flushed (512 MiB write) between steps",
-                              "GB/s": hd["bytes"] / (hms / 1e3) / 1e9,
-                              "frac_hbm": hd["bytes"] / (hms / 1e3) / 1e9 / peaks["hbm_gbs"],
+                              "roofline": roofline_of(dict(bytes=hd["bytes"], flops=hd["flops"]),
+                                                      hms, peaks, "burst", "hbm"),
                               "TFLOP/s": hd["flops"] / (hms / 1e3) / 1e12}
     if not args.no_e2e:
-        e2e = run_e2e(w, pre["inp"], dev, max(3, args.steps // 2))
+        e2e = run_e2e(w, inp, dev, max(3, args.steps // 2))
         eval_, ems = dist_ctx.job_rate(w.B * w.n, e2e["ms"])
         line["e2e"] = {"value": eval_, "unit": "queries/s",
                        "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                        "ms_per_step": ems, "serial_ms_per_step": e2e["serial_ms"],
                        "mode": "pipelined: step i+1's h2d and step i-1's d2h overlap step i's "
                                "kernels (3 streams, double-buffered device tensors)"}
-    if rank == 0 and dist_ctx.world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(w, pre["inp"], args.cpu_sample)
     if rank == 0:
         print(json.dumps(line))
     dist_ctx.close()
