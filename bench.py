@@ -854,7 +854,7 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--cpu-sample", type=int, default=4096,
+    ap.add_argument("--cpu-sample", type=int, default=16384,
                     help="queries the oracle baseline scores (bounded CPU sample)")
     ap.add_argument("--n", type=int, default=0,
                     help="override the prefill length (smaller cases for profiler captures; "
@@ -889,7 +889,7 @@ def main():
             return 0
         import oracle
         inp = synth.csa_prefill_inputs(w, seed=0)
-        sample = max(16, args.cpu_sample // 4)
+        sample = max(16, args.cpu_sample // 16)
         for _ in range(args.warmup):
             oracle_prefill_sample(w, inp, 16)
         per_qs, walls = [], []
@@ -977,8 +977,8 @@ def main():
     if not args.no_configs:
         # the other two prefill configurations, each timed like the headline
         for name, mk, path_cls, hca, n_cpu in (
-                (PREFILL_C2, synth.csa_prefill_inputs, PrefillPath, False, 1024),
-                (HCA_PREFILL, synth.hca_prefill_inputs, HcaPrefillPath, True, 256)):
+                (PREFILL_C2, synth.csa_prefill_inputs, PrefillPath, False, 8192),
+                (HCA_PREFILL, synth.hca_prefill_inputs, HcaPrefillPath, True, 32768)):
             wc = synth.WORKLOADS[name]
             inp_c = mk(wc, seed=rank)
             pc = path_cls(wc, inp_c, dev)

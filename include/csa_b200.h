@@ -373,6 +373,41 @@ csa_status_t hca_dense_attn_varlen(const void* q, int dt, int S, const int* cu_s
                                    int D, const void* kv_c, int m, const void* kv_raw, int window,
                                    float softmax_scale, void* out, float* lse_out, void* stream);
 
+/*
+ * Query spans at an offset (context-parallel shards).  "DeepSeek V4 CSA + CP
+ * 迁移到 HP：困难点深度分析" lays a long sequence over ranks (the pipeline that
+ * opens the page): a rank holds spans of consecutive positions, all-gathers
+ * the compressed entries and runs stage 2 and 3 for its own queries, whose
+ * positions start past 0.  These calls are the unpacked calls with q_pos and
+ * raw_pos0 / raw_len given as uniform host offsets:
+ *   query q of every element sits at position q_pos0 + q (q_pos0 >= 0);
+ *   raw row j of every element holds position raw_pos0 + j (raw_pos0 >= 0),
+ *   all L_raw rows present (raw_len = L_raw).
+ * Every other argument, the arithmetic, the error behaviour and the results
+ * are those of csa_indexer_topk / csa_sparse_attn / hca_dense_attn with
+ * q_pos[b][q] = q_pos0 + q, raw_pos0[b] = raw_pos0 and raw_len[b] = L_raw.
+ * Unlike a per-element position array, a uniform offset keeps the prefill
+ * shape, so these calls take the tensor-core kernels (64 heads x 128, d_I 64)
+ * where the unpacked prefill call would.
+ */
+csa_status_t csa_indexer_topk_at(const void* qI, int qI_dt, const float* qI_scale,
+                                 const float* qI_weight, const void* kI, int kI_dt,
+                                 const float* kI_scale, int B, int n_q, int H_I, int d_I,
+                                 int N_cap, const int* n_entries, int q_pos0, int m, int topk,
+                                 int* idx_out, void* stream);
+
+csa_status_t csa_sparse_attn_at(const void* q, int dt, int B, int n_q, int H, int D,
+                                const void* kv_c, int N_cap, const int* idx, int topk,
+                                const void* kv_raw, int L_raw, int raw_pos0, int window,
+                                int q_pos0, float softmax_scale, void* out, float* lse_out,
+                                void* stream);
+
+csa_status_t hca_dense_attn_at(const void* q, int dt, int B, int n_q, int H, int D,
+                               const void* kv_c, int N_cap, const int* n_entries, int m,
+                               const void* kv_raw, int L_raw, int raw_pos0, int window,
+                               int q_pos0, float softmax_scale, void* out, float* lse_out,
+                               void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -53,6 +53,9 @@ SIGNATURES = {
                                   P]),
     "hca_dense_attn_paged": (I, [P, I, I, I, I, I, P, P, I, I, I, P, I, P, I, P, P, I, P, F, P, P,
                                  P]),
+    "csa_indexer_topk_at": (I, [P, I, P, P, P, I, P, I, I, I, I, I, P, I, I, I, P, P]),
+    "csa_sparse_attn_at": (I, [P, I, I, I, I, I, P, I, P, I, P, I, I, I, I, F, P, P, P]),
+    "hca_dense_attn_at": (I, [P, I, I, I, I, I, P, I, P, I, P, I, I, I, I, F, P, P, P]),
 }
 
 
@@ -321,6 +324,47 @@ def hca_dense_attn_varlen(q: torch.Tensor, cu_seqlens, kv_c: torch.Tensor, m: in
     _check(load().hca_dense_attn_varlen(_ptr(q), _dt(q), S, cup, H, D, _ptr(kv_c), m, _ptr(kv_raw),
                                         window, float(softmax_scale), _ptr(out), _ptr(lse_out),
                                         _stream(stream)))
+
+
+# ---------------------------------------------------------------- spans at an offset
+def csa_indexer_topk_at(qI: torch.Tensor, kI: torch.Tensor, m: int, topk: int,
+                        idx_out: torch.Tensor, q_pos0: int, kI_scale: torch.Tensor | None = None,
+                        n_entries: torch.Tensor | None = None, qI_scale: torch.Tensor | None = None,
+                        kI_rotated: bool = False, qI_weight: torch.Tensor | None = None,
+                        stream=None) -> None:
+    """csa_indexer_topk with query q of every element at position q_pos0 + q."""
+    B, n_q, H_I, d_I = qI.shape
+    _check(load().csa_indexer_topk_at(_ptr(qI), _dt(qI), _ptr(qI_scale), _ptr(qI_weight),
+                                      _ptr(kI), _dt_rot(kI, kI_rotated), _ptr(kI_scale), B, n_q,
+                                      H_I, d_I, kI.shape[1], _i32(n_entries, "n_entries"),
+                                      int(q_pos0), m, topk, _i32(idx_out, "idx_out"),
+                                      _stream(stream)))
+
+
+def csa_sparse_attn_at(q: torch.Tensor, kv_c: torch.Tensor, idx: torch.Tensor | None,
+                       kv_raw: torch.Tensor, window: int, out: torch.Tensor, q_pos0: int,
+                       raw_pos0: int, lse_out: torch.Tensor | None = None,
+                       softmax_scale: float = 0.0, stream=None) -> None:
+    """csa_sparse_attn with query q at position q_pos0 + q and raw row j at raw_pos0 + j."""
+    B, n_q, H, D = q.shape
+    topk = 0 if idx is None else idx.shape[-1]
+    _check(load().csa_sparse_attn_at(_ptr(q), _dt(q), B, n_q, H, D, _ptr(kv_c), kv_c.shape[1],
+                                     _i32(idx, "idx"), topk, _ptr(kv_raw), kv_raw.shape[1],
+                                     int(raw_pos0), window, int(q_pos0), float(softmax_scale),
+                                     _ptr(out), _ptr(lse_out), _stream(stream)))
+
+
+def hca_dense_attn_at(q: torch.Tensor, kv_c: torch.Tensor, m: int, kv_raw: torch.Tensor,
+                      window: int, out: torch.Tensor, q_pos0: int, raw_pos0: int,
+                      lse_out: torch.Tensor | None = None, n_entries: torch.Tensor | None = None,
+                      softmax_scale: float = 0.0, stream=None) -> None:
+    """hca_dense_attn with query q at position q_pos0 + q and raw row j at raw_pos0 + j."""
+    B, n_q, H, D = q.shape
+    _check(load().hca_dense_attn_at(_ptr(q), _dt(q), B, n_q, H, D, _ptr(kv_c), kv_c.shape[1],
+                                    _i32(n_entries, "n_entries"), m, _ptr(kv_raw),
+                                    kv_raw.shape[1], int(raw_pos0), window, int(q_pos0),
+                                    float(softmax_scale), _ptr(out), _ptr(lse_out),
+                                    _stream(stream)))
 
 
 # ---------------------------------------------------------------- paged caches

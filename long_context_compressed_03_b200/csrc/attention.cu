@@ -41,7 +41,7 @@ __global__ void __launch_bounds__(kThreads) attn_generic_kernel(AttnArgs a) {
 
     const int row = blockIdx.x;
     const int b = row / a.n_q;
-    const int t = a.q_pos ? a.q_pos[row] : row - b * a.n_q;
+    const int t = a.q_pos ? a.q_pos[row] : a.pos0 + (row - b * a.n_q);
     const RowKeys rk = row_keys(a, b, t);
     const int total = rk.n_comp + rk.n_win;
 

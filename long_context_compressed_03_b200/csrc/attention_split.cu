@@ -120,7 +120,7 @@ __global__ void __launch_bounds__(H * 2, min_blocks<H>()) attn_split_kernel(Attn
     const int rank = (int)cluster.block_rank();
     const int row = blockIdx.y;
     const int b = row / a.n_q;
-    const int t = a.q_pos ? a.q_pos[row] : row - b * a.n_q;
+    const int t = a.q_pos ? a.q_pos[row] : a.pos0 + (row - b * a.n_q);
     const RowKeys rk = row_keys(a, b, t);
     const int T = rk.n_comp + rk.n_win;
     const int ch = ((T + C - 1) / C + kBN - 1) / kBN * kBN;

@@ -113,6 +113,8 @@ struct TcParams {
     int m;
     int dense;
     int B, n, N_cap, L_raw, window;
+    int qpos0;                 // query q of every element sits at position qpos0 + q
+    int rawpos0;               // raw row j of every element holds position rawpos0 + j
     float scale_log2;          // softmax scale * log2(e)
     __nv_bfloat16* out;
     float* lse;
@@ -157,7 +159,7 @@ struct Geometry {
     int T;         // tiles per M tile
     int bn_c_last; // N of the last compressed tile
     int bn_w_last;
-    int p_lo;      // first window position
+    int p_lo;      // first window position (absolute)
     int Lw;
     int Vmax;      // dense: entries needed by the CTA's last token
 };
@@ -231,11 +233,14 @@ template <bool PACKED> __device__ __forceinline__ int u_raw0(const TcParams& p, 
     return PACKED ? u.raw0 : u.b * p.L_raw;
 }
 
+// A unit's tokens t0 .. sit at positions qpos0 + t0 .. (packed sequences:
+// qpos0 = rawpos0 = 0); its window reads the raw rows present, positions
+// [rawpos0, rawpos0 + L_raw).
 template <bool PACKED>
 __device__ __forceinline__ Geometry geometry(const TcParams& p, const Unit& un) {
     Geometry g;
-    const int t0 = un.t0;
-    const int t_last = min(t0 + kTokens - 1, u_n<PACKED>(p, un) - 1);
+    const int t0 = un.t0 + p.qpos0;                                  // positions
+    const int t_last = min(un.t0 + kTokens - 1, u_n<PACKED>(p, un) - 1) + p.qpos0;
     if (p.dense) {
         g.Vmax = min((t_last + 1) / p.m, u_ne_dense<PACKED>(p, un));
         g.cc = 0;
@@ -249,8 +254,8 @@ __device__ __forceinline__ Geometry geometry(const TcParams& p, const Unit& un) 
         g.bn_c_last = p.topk ? round16(p.topk - (cc - 1) * kBN) : 0;
     }
     if (p.window > 0) {
-        g.p_lo = max(0, t0 - p.window + 1);
-        const int p_hi = min(t_last, u_L_raw<PACKED>(p, un) - 1);
+        g.p_lo = max(max(0, p.rawpos0), t0 - p.window + 1);
+        const int p_hi = min(t_last, p.rawpos0 + u_L_raw<PACKED>(p, un) - 1);
         g.Lw = max(0, p_hi - g.p_lo + 1);
     } else {
         g.p_lo = 0;
@@ -597,9 +602,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcParams p) {
                     });
                 } else {
                     load_tile_h(dst, lt, [&](int row) -> const uint8_t* {
-                        const int pos = g.p_lo + chunk * kBN + row;
-                        const long gr = raw0 + pos;
-                        return (pos < un_L && gr < p.rows_w) ? kvr + (size_t)gr * (kD * 2) : nullptr;
+                        const int jr = g.p_lo - p.rawpos0 + chunk * kBN + row;   // raw row
+                        const long gr = raw0 + jr;
+                        return (jr < un_L && gr < p.rows_w) ? kvr + (size_t)gr * (kD * 2) : nullptr;
                     });
                 }
                 // the tile (and, for a gathered one, the mask) is written:
@@ -742,11 +747,12 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcParams p) {
             const Unit un = unit_of<PACKED>(p, u);
             const int t0 = un.t0;
             const Geometry g = geometry<PACKED>(p, un);
-            const int t = t0 + 2 * mt + u_tok;               // position in the sequence
+            const int t = t0 + 2 * mt + u_tok;               // the row's token
             const bool row_ok = t < u_n<PACKED>(p, un);
+            const int tp = t + p.qpos0;                      // and its position
             int Vt = 0;
-            if (p.dense && row_ok) Vt = min((t + 1) / p.m, u_ne_dense<PACKED>(p, un));
-            const int w_lo = t - p.window + 1;               // window [w_lo, t]
+            if (p.dense && row_ok) Vt = min((tp + 1) / p.m, u_ne_dense<PACKED>(p, un));
+            const int w_lo = tp - p.window + 1;              // window [w_lo, tp]
             // m_used: running max (base 2, shared by the row's two threads);
             // l_r / l_e: this half's sums of the rounded / exact weights
             float m_used = -INFINITY, l_r = 0.0f, l_e = 0.0f;
@@ -774,7 +780,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcParams p) {
                     } else {
                         const int p0 = g.p_lo + tr.chunk * kBN;
                         c_lo = max(0, w_lo - p0);
-                        c_hi = min(tr.bn, t - p0 + 1) - 1;
+                        c_hi = min(tr.bn, tp - p0 + 1) - 1;
                     }
                 }
                 uint32_t vm4[4];
@@ -916,6 +922,8 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint32_t box_rows)
 }  // namespace
 
 bool attention_tc_supported(const AttnArgs& a) {
+    // positions come as the uniform offsets pos0 / raw_base (per-element
+    // arrays go to the row kernels)
     return a.dt == DT_BF16 && a.H == kH && a.D == kD && a.q_pos == nullptr &&
            a.raw_pos0 == nullptr && a.raw_len == nullptr && a.L_raw >= a.n_q && a.n_q > 0 &&
            a.topk <= 1024;   // the CTA's index rows are staged in shared memory
@@ -942,6 +950,8 @@ cudaError_t launch_attention_tc(const AttnArgs& a, uint32_t* err, cudaStream_t s
     p.N_cap = a.N_cap;
     p.L_raw = a.L_raw;
     p.window = a.window;
+    p.qpos0 = a.vl ? 0 : a.pos0;
+    p.rawpos0 = a.vl ? 0 : a.raw_base;
     p.scale_log2 = a.scale * kLog2e;
     p.out = static_cast<__nv_bfloat16*>(a.out);
     p.lse = a.lse_out;

@@ -25,7 +25,7 @@ __device__ __forceinline__ RowKeys row_keys(const AttnArgs& a, int b, int t) {
     } else {
         k.n_comp = a.topk;
     }
-    const int p0 = a.raw_pos0 ? a.raw_pos0[b] : 0;
+    const int p0 = a.raw_pos0 ? a.raw_pos0[b] : a.raw_base;
     const int len = clampi(a.raw_len ? a.raw_len[b] : a.L_raw, 0, a.L_raw);
     // positions [max(0, t-W+1), t] ∩ [max(p0, 0), p0 + len - 1], as raw rows
     long lo = max((long)t - a.window + 1, 0L);

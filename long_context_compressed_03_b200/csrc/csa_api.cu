@@ -240,8 +240,10 @@ static csa_status_t indexer_impl(const void* qI, int qI_dt, const float* qI_scal
                                  const float* qI_weight, const void* kI, int kI_dt,
                                  const float* kI_scale, int B, int n_q, int H_I, int d_I, int N_cap,
                                  const int* n_entries, const int* q_pos, int m, int topk,
-                                 int* idx_out, const csa::PageMap& pm, void* stream) {
+                                 int* idx_out, const csa::PageMap& pm, void* stream,
+                                 int q_pos0 = 0) {
     REQUIRE(B >= 0 && n_q >= 0 && N_cap >= 0, "csa_indexer_topk: negative size");
+    REQUIRE(q_pos0 >= 0, "csa_indexer_topk_at: q_pos0 must be >= 0");
     REQUIRE(H_I >= 1 && d_I >= 1, "csa_indexer_topk: H_I and d_I must be positive");
     REQUIRE(m >= 1, "csa_indexer_topk: m must be >= 1");
     REQUIRE(topk >= 1 && topk <= 2048, "csa_indexer_topk: topk must be in [1, 2048]");
@@ -268,6 +270,7 @@ static csa_status_t indexer_impl(const void* qI, int qI_dt, const float* qI_scal
     REQUIRE_ALIGNED4(q_pos, "q_pos");
     csa::IndexerArgs a{qI, qI_dt, qI_scale, kI, kI_dt, kI_scale, B, n_q, H_I, d_I, N_cap,
                        n_entries, q_pos, m, topk, idx_out, hadamard_norm(d_I), qI_weight, pm};
+    a.pos0 = q_pos0;
     const char* why = nullptr;
     return from_cuda(LAUNCH(csa::launch_indexer_topk(a, static_cast<cudaStream_t>(stream), &why)),
                      "csa_indexer_topk", why);
@@ -422,6 +425,46 @@ csa_status_t hca_dense_attn_paged(const void* q, int dt, int B, int n_q, int H, 
     csa::AttnArgs a{q, dt, B, n_q, H, D, kv_c_pages, N_cap, nullptr, 0, n_entries, m, 1, kv_raw,
                     L_raw, raw_pos0, raw_len, window, q_pos, softmax_scale, out, lse_out, pm};
     return attention_common("hca_dense_attn_paged", a, stream);
+}
+
+// ------------------------------------------------------------ spans at an offset
+csa_status_t csa_indexer_topk_at(const void* qI, int qI_dt, const float* qI_scale,
+                                 const float* qI_weight, const void* kI, int kI_dt,
+                                 const float* kI_scale, int B, int n_q, int H_I, int d_I,
+                                 int N_cap, const int* n_entries, int q_pos0, int m, int topk,
+                                 int* idx_out, void* stream) {
+    return indexer_impl(qI, qI_dt, qI_scale, qI_weight, kI, kI_dt, kI_scale, B, n_q, H_I, d_I,
+                        N_cap, n_entries, nullptr, m, topk, idx_out, csa::PageMap{}, stream,
+                        q_pos0);
+}
+
+csa_status_t csa_sparse_attn_at(const void* q, int dt, int B, int n_q, int H, int D,
+                                const void* kv_c, int N_cap, const int* idx, int topk,
+                                const void* kv_raw, int L_raw, int raw_pos0, int window,
+                                int q_pos0, float softmax_scale, void* out, float* lse_out,
+                                void* stream) {
+    REQUIRE(topk >= 0 && topk <= 2048, "csa_sparse_attn_at: topk must be in [0, 2048]");
+    REQUIRE(idx || topk == 0 || (long)B * n_q == 0, "csa_sparse_attn_at: null idx");
+    REQUIRE(q_pos0 >= 0 && raw_pos0 >= 0, "csa_sparse_attn_at: q_pos0 and raw_pos0 must be >= 0");
+    csa::AttnArgs a{q, dt, B, n_q, H, D, kv_c, N_cap, idx, topk, nullptr, 1, 0, kv_raw, L_raw,
+                    nullptr, nullptr, window, nullptr, softmax_scale, out, lse_out};
+    a.pos0 = q_pos0;
+    a.raw_base = raw_pos0;
+    return attention_common("csa_sparse_attn_at", a, stream);
+}
+
+csa_status_t hca_dense_attn_at(const void* q, int dt, int B, int n_q, int H, int D,
+                               const void* kv_c, int N_cap, const int* n_entries, int m,
+                               const void* kv_raw, int L_raw, int raw_pos0, int window,
+                               int q_pos0, float softmax_scale, void* out, float* lse_out,
+                               void* stream) {
+    REQUIRE(m >= 1, "hca_dense_attn_at: m must be >= 1");
+    REQUIRE(q_pos0 >= 0 && raw_pos0 >= 0, "hca_dense_attn_at: q_pos0 and raw_pos0 must be >= 0");
+    csa::AttnArgs a{q, dt, B, n_q, H, D, kv_c, N_cap, nullptr, 0, n_entries, m, 1, kv_raw, L_raw,
+                    nullptr, nullptr, window, nullptr, softmax_scale, out, lse_out};
+    a.pos0 = q_pos0;
+    a.raw_base = raw_pos0;
+    return attention_common("hca_dense_attn_at", a, stream);
 }
 
 // ------------------------------------------------------------------ test hooks

@@ -151,7 +151,7 @@ __global__ void __launch_bounds__(kThreads, min_blocks<NU>()) indexer_split_kern
     const int b = row / a.n_q;
     const int H = a.H_I, topk = a.topk;
     int* out = a.idx_out + (size_t)row * topk;
-    const int t = a.q_pos ? a.q_pos[row] : row - b * a.n_q;
+    const int t = a.q_pos ? a.q_pos[row] : a.pos0 + (row - b * a.n_q);
     const int ne = clampi(a.n_entries ? a.n_entries[b] : a.N_cap, 0, a.N_cap);
     const int V = t < 0 ? 0 : min((t + 1) / a.m, ne);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;

@@ -1056,7 +1056,7 @@ cudaError_t launch_indexer_tc(const IndexerArgs& a, uint32_t* err, cudaStream_t 
     p.topk = a.topk;
     p.n_entries = a.n_entries;
     p.idx_out = a.idx_out;
-    p.pos0 = 0;
+    p.pos0 = a.vl ? 0 : a.pos0;
     p.err = err;
     p.qw = a.qI_weight;
     const int tiles = (a.n_q + kRows - 1) / kRows;

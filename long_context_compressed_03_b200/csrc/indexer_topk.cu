@@ -75,7 +75,7 @@ __global__ void __launch_bounds__(kThreads) indexer_topk_kernel(IndexerArgs a) {
     const int b = row / a.n_q;
     const int H = a.H_I, d = a.d_I, topk = a.topk;
     int* out = a.idx_out + (size_t)row * topk;
-    const int t = a.q_pos ? a.q_pos[row] : row - b * a.n_q;
+    const int t = a.q_pos ? a.q_pos[row] : a.pos0 + (row - b * a.n_q);
     const int ne = clampi(a.n_entries ? a.n_entries[b] : a.N_cap, 0, a.N_cap);
     const int V = t < 0 ? 0 : min((t + 1) / a.m, ne);
 

@@ -88,6 +88,7 @@ struct IndexerArgs {
     PageMap pages;             // kI (and kI_scale) layout
     const VarlenMap* vl = nullptr;   // packed (tensor-core kernel only): B = S, n_q = longest,
                                      // N_cap = total entries
+    int pos0 = 0;              // q_pos == NULL: query q of every element sits at pos0 + q
 };
 
 struct AttnArgs {
@@ -106,6 +107,8 @@ struct AttnArgs {
     PageMap pages;             // kv_c layout
     const VarlenMap* vl = nullptr;   // packed (tensor-core kernel only): B = 1, n_q = L_raw = T
                                      // tokens, N_cap = total entries
+    int pos0 = 0;              // q_pos == NULL: query q of every element sits at pos0 + q
+    int raw_base = 0;          // raw_pos0 == NULL: raw row j of every element holds position raw_base + j
 };
 
 // Device address of this library's error word on the current device (set by
