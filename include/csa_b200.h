@@ -100,6 +100,21 @@ csa_status_t csa_check_device_error(void* stream, int clear);
 csa_status_t csa_debug_inject_launch_error(int cuda_error);
 
 /*
+ * Test hook for the timeout path (it never faults, traps or hangs a GPU).
+ * `ns`: the time limit, in ns, of each bounded wait of the tensor-core
+ * kernels' work in launches made after this call (0: back to the default
+ * 1 s; < 0: CSA_ERR_INVALID_ARG).  `stall_next` != 0: the next tensor-core
+ * launch (prefill indexer or attention) makes one thread of every CTA wait on
+ * a barrier that nothing completes, so that wait runs out after `ns`.  When a
+ * wait runs out the kernel records CSA_ERR_TIMEOUT in the device error word,
+ * every CTA stops issuing work, waits (with the default limit) for the copies
+ * and MMAs it already issued, releases its tensor memory and exits; outputs
+ * of that launch are unspecified, later launches see the word set and do
+ * nothing until csa_check_device_error clears it.  Process-wide.
+ */
+csa_status_t csa_debug_set_wait_limit(long long ns, int stall_next);
+
+/*
  * csa_compress -- stage 1: overlapping (or plain) mean-pool compression
  * followed by a projection, optionally quantised to fp8.
  * Follows "百万上下文从「奢侈品」变「日用品」…" §3.2 (C[i] = W . mean of the

@@ -36,6 +36,7 @@ SIGNATURES = {
     "csa_kernel_launches": (ctypes.c_ulonglong, []),
     "csa_check_device_error": (I, [P, I]),
     "csa_debug_inject_launch_error": (I, [I]),
+    "csa_debug_set_wait_limit": (I, [ctypes.c_longlong, I]),
     "csa_compress": (I, [P, I, I, I, I, P, I, I, I, P, I, P, P]),
     "csa_compress_gated": (I, [P, I, I, I, I, P, P, P, I, I, I, P, I, P, P]),
     "csa_compress_append": (I, [P, I, I, I, P, I, I, I, P, P, P, I, P, I, P, P]),

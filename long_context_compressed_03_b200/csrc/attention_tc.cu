@@ -85,11 +85,15 @@ struct __align__(8) Ctrl {
     uint64_t s_full[2];
     uint64_t p_ready[2];
     uint64_t fin;
+    uint64_t stall_bar;             // test hook: a barrier nothing completes
     uint64_t xbar[2][4];            // [M tile][quarter]: the two half-row warps meet
     uint32_t mask[kStages][4];      // gathered tiles: valid rows of the stage
     uint32_t tmem_base;
     int abort;
-    int load_go;               // loaders: continue with the next load
+    int load_go[2];            // loaders: continue with the next load (alternating slots:
+                               // decision d+1 is written only after every loader passed
+                               // the barrier of decision d, so d is never overwritten
+                               // before it is read)
 };
 
 // Exchange between the two half-row threads of a row (double-buffered by
@@ -119,6 +123,8 @@ struct TcParams {
     __nv_bfloat16* out;
     float* lse;
     uint32_t* err;
+    uint64_t wait_ns;          // time limit of each wait of the work
+    int stall;                 // test hook: one thread waits on stall_bar first
     VarlenMap vl;              // packed sequences (vl.S > 0)
 };
 
@@ -492,6 +498,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcParams p) {
             mbar_init(&ctl->o_free[i], 8);
         }
         mbar_init(&ctl->fin, 1);
+        mbar_init(&ctl->stall_bar, 1);
         // a CTA started after another one timed out does no work
         ctl->abort = (*reinterpret_cast<volatile uint32_t*>(p.err) != 0u) ? 1 : 0;
         fence_barrier_init();
@@ -511,6 +518,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcParams p) {
         const uint8_t* kvc = static_cast<const uint8_t*>(p.kv_c);
         const uint8_t* kvr = static_cast<const uint8_t*>(p.kv_raw);
         int Lg = 0;                                          // loads issued by this CTA
+        int dn = 0;                                          // go / stop decisions taken
         int k = 0;                                           // units done
         bool go = true;
         for (int u = blockIdx.x; u < n_units && go; u += gridDim.x, ++k) {
@@ -539,9 +547,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcParams p) {
                 if (L == q_at) {
                     // the unit's Q (bf16, by TMA) has landed: convert it in place.
                     // One thread waits and decides for all loaders.
-                    if (lt == 0) ctl->load_go = mbar_wait(&ctl->bar_q, k & 1, abort, p.err) ? 1 : 0;
+                    if (lt == 0) ctl->load_go[dn & 1] = mbar_wait(&ctl->bar_q, k & 1, abort, p.err, p.wait_ns) ? 1 : 0;
                     named_sync(1, kLoadThreads);
-                    if (!ctl->load_go) { go = false; break; }
+                    if (!ctl->load_go[dn++ & 1]) { go = false; break; }
 #pragma unroll 1
                     for (int i0 = lt; i0 < 2 * kTileBytes / 16; i0 += 8 * kLoadThreads) {
                         uint4 v[8];
@@ -573,11 +581,11 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcParams p) {
                 // one thread acquires the free slot and decides for all loaders;
                 // the named barrier orders the others after it
                 if (lt == 0) {
-                    const bool okw = use == 0 || mbar_wait(&ctl->freeb[slot], (use - 1) & 1, abort, p.err);
-                    ctl->load_go = (okw && !*abort) ? 1 : 0;
+                    const bool okw = use == 0 || mbar_wait(&ctl->freeb[slot], (use - 1) & 1, abort, p.err, p.wait_ns);
+                    ctl->load_go[dn & 1] = (okw && !*abort) ? 1 : 0;
                 }
                 named_sync(1, kLoadThreads);
-                if (!ctl->load_go) { go = false; break; }
+                if (!ctl->load_go[dn++ & 1]) { go = false; break; }
                 if (kind == 0) {
                     const int* ir = sIdx + token * p.topk + chunk * kBN;
                     const int tpos = t0 + token;
@@ -635,19 +643,21 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcParams p) {
             int J[2] = {0, 0};                // tiles before this unit, per M tile
             int k = 0;                        // units done
             bool ok = true;
+            // test hook: a wait that runs out (nothing completes stall_bar)
+            if (p.stall) mbar_wait(&ctl->stall_bar, 0, abort, p.err, p.wait_ns);
             // nothing is loaded by a CTA that starts aborted
             if (blockIdx.x < n_units && !*abort) load_q(blockIdx.x);
             for (int u = blockIdx.x; u < n_units && ok; u += gridDim.x, ++k) {
                 const Unit un = unit_of<PACKED>(p, u);
                 const Geometry g = geometry<PACKED>(p, un);
-                ok = q_issued > q_done && mbar_wait(&ctl->q_conv, k & 1, abort, p.err);
+                ok = q_issued > q_done && mbar_wait(&ctl->q_conv, k & 1, abort, p.err, p.wait_ns);
                 if (ok) ++q_done;
                 tc_fence_after();
                 auto issue_qk = [&](int mt, int j) -> bool {
                     const TileRef r = tile_ref(p, g, mt, j);
                     const int ld = L0 + r.load;
                     const int slot = ld % kStages;
-                    if (!mbar_wait(&ctl->full[slot], (ld / kStages) & 1, abort, p.err)) return false;
+                    if (!mbar_wait(&ctl->full[slot], (ld / kStages) & 1, abort, p.err, p.wait_ns)) return false;
                     tc_fence_after();
                     // descriptors of the k-step 0 operands; a k step adds its byte
                     // offset / 16 to the start-address field (no carry: smem < 256 KB)
@@ -667,7 +677,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcParams p) {
                 auto next_q = [&]() -> bool {
                     mma_commit(&ctl->q_free);
                     if (un_next >= n_units) return true;
-                    if (!mbar_wait(&ctl->q_free, k & 1, abort, p.err) || *abort) return false;
+                    if (!mbar_wait(&ctl->q_free, k & 1, abort, p.err, p.wait_ns) || *abort) return false;
                     load_q(un_next);
                     return true;
                 };
@@ -677,9 +687,9 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcParams p) {
                 bool o_ready[2] = {k == 0, k == 0};
                 for (int j = 0; ok && j < g.T; ++j) {
                     for (int mt = 0; mt < 2 && ok; ++mt) {
-                        if (!mbar_wait(&ctl->p_ready[mt], (J[mt] + j) & 1, abort, p.err)) { ok = false; break; }
+                        if (!mbar_wait(&ctl->p_ready[mt], (J[mt] + j) & 1, abort, p.err, p.wait_ns)) { ok = false; break; }
                         if (!o_ready[mt]) {
-                            if (!mbar_wait(&ctl->o_free[mt], (k - 1) & 1, abort, p.err)) { ok = false; break; }
+                            if (!mbar_wait(&ctl->o_free[mt], (k - 1) & 1, abort, p.err, p.wait_ns)) { ok = false; break; }
                             o_ready[mt] = true;
                         }
                         tc_fence_after();
@@ -702,7 +712,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcParams p) {
                 // this unit's O is complete (or untouched when it has no tiles)
                 if (ok) {
                     for (int mt = 0; mt < 2; ++mt) {
-                        if (!o_ready[mt] && !mbar_wait(&ctl->o_free[mt], (k - 1) & 1, abort, p.err)) { ok = false; break; }
+                        if (!o_ready[mt] && !mbar_wait(&ctl->o_free[mt], (k - 1) & 1, abort, p.err, p.wait_ns)) { ok = false; break; }
                         mma_commit(&ctl->o_full[mt]);
                     }
                 }
@@ -735,7 +745,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcParams p) {
         auto pair_sync = [&]() -> bool {
             __syncwarp();
             if (lane == 0) mbar_arrive(pair_bar);
-            const bool okx = __all_sync(0xffffffffu, mbar_wait(pair_bar, xcount & 1, abort, p.err));
+            const bool okx = __all_sync(0xffffffffu, mbar_wait(pair_bar, xcount & 1, abort, p.err, p.wait_ns));
             ++xcount;
             return okx;
         };
@@ -759,7 +769,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcParams p) {
             for (int j = 0; j < g.T && ok; ++j) {
                 const TileRef tr = tile_ref(p, g, mt, j);
                 // every wait is warp-collective: the TMEM accesses below are .sync.aligned
-                if (!__all_sync(0xffffffffu, mbar_wait(&ctl->s_full[mt], (J + j) & 1, abort, p.err))) { ok = false; break; }
+                if (!__all_sync(0xffffffffu, mbar_wait(&ctl->s_full[mt], (J + j) & 1, abort, p.err, p.wait_ns))) { ok = false; break; }
                 tc_fence_after();
                 // which columns are keys of this row?
                 int c_lo = 0, c_hi = -1;                     // contiguous range
@@ -770,7 +780,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcParams p) {
                             const int lg = L0 + tr.load;     // the loaders' index of this tile
                             const int slot = lg % kStages;
                             // the loaders wrote the mask before arriving on this stage
-                            if (!__all_sync(0xffffffffu, mbar_wait(&ctl->full[slot], (lg / kStages) & 1, abort, p.err))) { ok = false; break; }
+                            if (!__all_sync(0xffffffffu, mbar_wait(&ctl->full[slot], (lg / kStages) & 1, abort, p.err, p.wait_ns))) { ok = false; break; }
 #pragma unroll
                             for (int q = 0; q < 4; ++q) mw[q] = ctl->mask[slot][q];
                             c_hi = tr.bn - 1;
@@ -843,7 +853,7 @@ attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, TcParams p) {
             if (!pair_sync()) break;
             const float LR = l_r + xc->l[up][mt][h ^ 1][0][r];
             const float LE = l_e + xc->l[up][mt][h ^ 1][1][r];
-            if (!__all_sync(0xffffffffu, mbar_wait(&ctl->o_full[mt], k & 1, abort, p.err))) break;
+            if (!__all_sync(0xffffffffu, mbar_wait(&ctl->o_full[mt], k & 1, abort, p.err, p.wait_ns))) break;
             tc_fence_after();
             __nv_bfloat16* orow = p.out + ((size_t)(u_tok0<PACKED>(p, un) + t) * kH + (r & 63)) * kD + 64 * h;
             if (g.T > 0) {
@@ -956,6 +966,8 @@ cudaError_t launch_attention_tc(const AttnArgs& a, uint32_t* err, cudaStream_t s
     p.out = static_cast<__nv_bfloat16*>(a.out);
     p.lse = a.lse_out;
     p.err = err;
+    p.wait_ns = wait_limit_ns();
+    p.stall = take_stall();
     int units = a.B * ((a.n_q + kTokens - 1) / kTokens);
     if (a.vl) {                                     // packed: units per sequence
         p.vl = *a.vl;

@@ -37,6 +37,14 @@ uint32_t* device_error_word() {
     }
     return w;
 }
+
+// The wait limit the tensor-core kernels' work is launched with (ns).
+static std::atomic<uint64_t> g_wait_limit_ns{1000000000ull};
+static std::atomic<int> g_stall_next{0};
+uint64_t wait_limit_ns() { return g_wait_limit_ns.load(std::memory_order_relaxed); }
+void set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns, std::memory_order_relaxed); }
+int take_stall() { return g_stall_next.exchange(0); }
+void set_stall(int on) { g_stall_next.store(on ? 1 : 0); }
 }  // namespace csa
 
 namespace {
@@ -475,6 +483,13 @@ csa_status_t csa_debug_inject_launch_error(int cuda_error) {
     REQUIRE(cuda_error != (int)cudaErrorNotSupported,
             "csa_debug_inject_launch_error: cudaErrorNotSupported (801) is not a launch failure");
     g_inject_error.store(cuda_error);
+    return ok();
+}
+
+csa_status_t csa_debug_set_wait_limit(long long ns, int stall_next) {
+    REQUIRE(ns >= 0, "csa_debug_set_wait_limit: the limit must be >= 0 (0: the default 1 s)");
+    csa::set_wait_limit_ns(ns == 0 ? 1000000000ull : (uint64_t)ns);
+    csa::set_stall(stall_next);
     return ok();
 }
 

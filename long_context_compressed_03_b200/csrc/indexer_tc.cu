@@ -104,6 +104,8 @@ struct IdxParams {
     const int* n_entries;
     int* idx_out;
     uint32_t* err;
+    uint64_t wait_ns;          // time limit of each wait of the work
+    int stall;                 // test hook: one thread waits on stall_bar first
     VarlenMap vl;              // packed sequences (vl.S > 0): grid.y = sequence
 };
 
@@ -113,6 +115,7 @@ struct __align__(8) Ctrl {
     uint64_t acc_full[kBufs];
     uint64_t acc_free[kBufs];
     uint64_t fin;
+    uint64_t stall_bar;          // test hook: a barrier nothing completes
     uint32_t tmem_base;
     int abort;
     int kind;                  // the pass about to run
@@ -430,7 +433,7 @@ template <bool FP8, bool GATED, int MODE>
 __device__ __forceinline__ bool group_pass(Ctrl* ctl, uint32_t tbase, float* ksb2, int grp, int nchunks,
                                            bool active, const RowCtx& rc, int (&cons)[kBufs], float& ksv,
                                            const float* ksc, int Vmax, volatile int* abort, uint32_t* err,
-                                           bool first_waited) {
+                                           uint64_t wait_ns, bool first_waited) {
     constexpr int kParts = kSlice / kPart;
     static_assert(kParts % 2 == 0, "parts alternate between two register sets");
     const int lane = threadIdx.x & 31;
@@ -444,7 +447,7 @@ __device__ __forceinline__ bool group_pass(Ctrl* ctl, uint32_t tbase, float* ksb
     int i = 0, buf = 0;
     const uint32_t col0 = tbase + grp * kSlice;
     if (!first_waited) {
-        if (!__all_sync(0xffffffffu, mbar_wait(&ctl->acc_full[0], cons[0] & 1, abort, err))) return false;
+        if (!__all_sync(0xffffffffu, mbar_wait(&ctl->acc_full[0], cons[0] & 1, abort, err, wait_ns))) return false;
         tc_fence_after();
         if (FP8) {
             __syncwarp();
@@ -469,7 +472,7 @@ __device__ __forceinline__ bool group_pass(Ctrl* ctl, uint32_t tbase, float* ksb
                 tmem_wait_ld_x4(B, taddr + (q + 2) * kPart, A);        // part q+1 ready, q+2 in flight
             } else {
                 if (more) {
-                    more = __all_sync(0xffffffffu, mbar_wait(&ctl->acc_full[bufn], cons[bufn] & 1, abort, err));
+                    more = __all_sync(0xffffffffu, mbar_wait(&ctl->acc_full[bufn], cons[bufn] & 1, abort, err, wait_ns));
                     if (more) tc_fence_after();
                 }
                 if (more)
@@ -562,6 +565,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
             mbar_init(&ctl->acc_free[g], kEpiWarps);   // one arrival per epilogue warp
         }
         mbar_init(&ctl->fin, 1);
+        mbar_init(&ctl->stall_bar, 1);
         ctl->abort = (*reinterpret_cast<volatile uint32_t*>(p.err) != 0u) ? 1 : 0;
         ctl->kind = kWindow;
         fence_barrier_init();
@@ -693,10 +697,12 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
         if (warp == 0) {
             // ------------------------------------------------------------ TMA producer
             if (lane == 0) {
+                // test hook: a wait that runs out (nothing completes stall_bar)
+                if (p.stall && pass == 0) mbar_wait(&ctl->stall_bar, 0, abort, p.err, p.wait_ns);
                 for (int i = 0; i < nchunks; ++i, ++L) {
                     const int slot = L % C::kStages, u = L / C::kStages;
                     if (*abort) break;     // nothing is issued once the CTA aborts
-                    if (u > 0 && !mbar_wait(&ctl->freeb[slot], (u - 1) & 1, abort, p.err)) break;
+                    if (u > 0 && !mbar_wait(&ctl->freeb[slot], (u - 1) & 1, abort, p.err, p.wait_ns)) break;
                     mbar_arrive_expect_tx(&ctl->full[slot], C::kBTile);
                     tma_load_2d(sB + slot * C::kBTile, &tm_k, 0, (int)ent0 + chunk_at(i) * kN, &ctl->full[slot]);
                 }
@@ -710,8 +716,8 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
                 for (int i = 0; i < nchunks; ++i, ++L) {
                     const int slot = L % C::kStages;
                     const int g = i % kBufs;
-                    if (!mbar_wait(&ctl->full[slot], (L / C::kStages) & 1, abort, p.err)) break;
-                    if (use_buf[g] > 0 && !mbar_wait(&ctl->acc_free[g], (use_buf[g] - 1) & 1, abort, p.err)) break;
+                    if (!mbar_wait(&ctl->full[slot], (L / C::kStages) & 1, abort, p.err, p.wait_ns)) break;
+                    if (use_buf[g] > 0 && !mbar_wait(&ctl->acc_free[g], (use_buf[g] - 1) & 1, abort, p.err, p.wait_ns)) break;
                     tc_fence_after();
                     const uint32_t bsa = smem_u32(sB + slot * C::kBTile);
                     for (int h = 0; h < kHeads; ++h) {
@@ -780,7 +786,7 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
                 // epilogue warp joins the barrier once, with or without a chunk.
                 uint32_t mx = 0;
                 if (nchunks > 0) {
-                    ok = __all_sync(0xffffffffu, mbar_wait(&ctl->acc_full[0], cons[0] & 1, abort, p.err));
+                    ok = __all_sync(0xffffffffu, mbar_wait(&ctl->acc_full[0], cons[0] & 1, abort, p.err, p.wait_ns));
                     if (ok) {
                         tc_fence_after();
                         if (FP8) {
@@ -805,19 +811,19 @@ indexer_tc_kernel(const __grid_constant__ CUtensorMap tm_k, IdxParams p) {
                 switch (wmode) {
                     case kWindow:
                         group_pass<FP8, GATED, kWindow>(ctl, tbase, ksb2, grp, nchunks, active, rc, cons, ksv,
-                                                        ksc, Vmax, abort, p.err, first_waited);
+                                                        ksc, Vmax, abort, p.err, p.wait_ns, first_waited);
                         break;
                     case kDigit:
                         group_pass<FP8, GATED, kDigit>(ctl, tbase, ksb2, grp, nchunks, active, rc, cons, ksv,
-                                                       ksc, Vmax, abort, p.err, first_waited);
+                                                       ksc, Vmax, abort, p.err, p.wait_ns, first_waited);
                         break;
                     case kEmit32:
                         group_pass<FP8, GATED, kEmit32>(ctl, tbase, ksb2, grp, nchunks, active, rc, cons, ksv,
-                                                        ksc, Vmax, abort, p.err, first_waited);
+                                                        ksc, Vmax, abort, p.err, p.wait_ns, first_waited);
                         break;
                     default:
                         group_pass<FP8, GATED, kEmit64>(ctl, tbase, ksb2, grp, nchunks, active, rc, cons, ksv,
-                                                        ksc, Vmax, abort, p.err, first_waited);
+                                                        ksc, Vmax, abort, p.err, p.wait_ns, first_waited);
                         break;
                 }
             }
@@ -1058,6 +1064,8 @@ cudaError_t launch_indexer_tc(const IndexerArgs& a, uint32_t* err, cudaStream_t 
     p.idx_out = a.idx_out;
     p.pos0 = a.vl ? 0 : a.pos0;
     p.err = err;
+    p.wait_ns = wait_limit_ns();
+    p.stall = take_stall();
     p.qw = a.qI_weight;
     const int tiles = (a.n_q + kRows - 1) / kRows;
     dim3 grid((unsigned)(a.B * tiles));

@@ -115,6 +115,15 @@ struct AttnArgs {
 // kernels whose bounded waits expired; read back by csa_check_device_error).
 uint32_t* device_error_word();
 
+// Time limit (ns) of each bounded wait of the tensor-core kernels' work,
+// 1 s unless a test set a shorter one (csa_debug_set_wait_limit).
+uint64_t wait_limit_ns();
+void set_wait_limit_ns(uint64_t ns);
+// One-shot test hook: the next tensor-core launch makes one thread of every
+// CTA wait on a barrier that nothing completes, so that wait runs out.
+int take_stall();
+void set_stall(int on);
+
 // tcgen05 prefill attention (64 heads x 128, bf16, positions 0..n-1).
 bool attention_tc_supported(const AttnArgs& a);
 cudaError_t launch_attention_tc(const AttnArgs& a, uint32_t* err, cudaStream_t s);

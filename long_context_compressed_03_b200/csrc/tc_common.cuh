@@ -54,10 +54,12 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // Waits for the phase with the given parity to complete.  Spins on try_wait
 // (which may suspend the thread in hardware for a while when the phase is
 // pending) and every 64 tries looks at the clock and the abort flag.  Gives up
-// after kWaitLimitNs or once *abort is set; on its own timeout it records
+// after limit_ns or once *abort is set; on its own timeout it records
 // ERR_TIMEOUT in *err and sets *abort.  Returns false when it gave up.
+// Waits of the work take the launch's limit; the drains before a CTA exits
+// (copies and MMAs it issued must land) always take kWaitLimitNs.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint32_t* err) {
+                                          uint32_t* err, uint64_t limit_ns = kWaitLimitNs) {
     uint64_t t0 = 0;
     while (true) {
         for (int i = 0; i < 64; ++i)
@@ -66,7 +68,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
         const uint64_t now = globaltimer();
         if (t0 == 0) {
             t0 = now;
-        } else if (now - t0 > kWaitLimitNs) {
+        } else if (now - t0 > limit_ns) {
             atomicCAS(err, ERR_NONE, ERR_TIMEOUT);
             *abort = 1;
             return false;

@@ -323,3 +323,9 @@ def test_injected_launch_error_maps_to_cuda_status(lib):
         return
     # consumed: the next call launches normally
     assert lib.csa_compress(x, 0, 1, 8, 16, W, 16, 4, 1, out, 0, None, None) == api.CSA_OK
+
+
+def test_wait_limit_hook_validates_and_resets(lib):
+    assert lib.csa_debug_set_wait_limit(-1, 0) == api.CSA_ERR_INVALID_ARG
+    assert lib.csa_debug_set_wait_limit(2_000_000, 0) == api.CSA_OK
+    assert lib.csa_debug_set_wait_limit(0, 0) == api.CSA_OK          # back to the default
