@@ -848,6 +848,43 @@ class DistCtx:
             self.dist.destroy_process_group()
 
 
+CONFIGS = {
+    # name: (input builder, path, HCA, oracle sample rows)
+    PREFILL_C2: (synth.csa_prefill_inputs, PrefillPath, False, 8192),
+    HCA_PREFILL: (synth.hca_prefill_inputs, HcaPrefillPath, True, 32768),
+}
+
+
+def run_config(name, dev, args, dist_ctx, rank, peaks):
+    """One of the other prefill configurations, timed like the headline
+    step, with its stages' rooflines and (rank 0, one GPU) the oracle's
+    baseline on a sample of the same workload."""
+    mk, path_cls, hca, n_cpu = CONFIGS[name]
+    wc = synth.WORKLOADS[name]
+    inp_c = mk(wc, seed=rank)
+    pc = path_cls(wc, inp_c, dev)
+    rc = run_path(pc, args.steps, args.warmup, dist_ctx)
+    cval, cms = dist_ctx.job_rate(wc.B * wc.n, rc["total_ms"] / args.steps)
+    creg, creg_why = regime_of(rc["clocks"], rc["total_ms"])
+    cwork = hca_prefill_work(wc) if hca else prefill_work(wc)
+    cst = stage_rooflines(cwork, rc["kern_ms"], peaks, creg, wc.indexer)
+    cdom = max(rc["kern_ms"], key=rc["kern_ms"].get)
+    croof = dict(cst[cdom]["roofline"], kernel=cdom, regime=f"{creg}: {creg_why}",
+                 traffic=ncu_traffic((cdom, name)))
+    entry = {"workload": name, "value": cval, "unit": "queries/s", "ms_per_step": cms,
+             "B": wc.B, "n": wc.n, "m": wc.m, "overlap": wc.overlap,
+             "l2": "inputs larger than L2 (q alone is 256 MiB or more)",
+             "roofline": croof, "stages": cst, "gpu_launches": rc["launches"],
+             "clocks": rc["clocks"]}
+    if not hca:
+        entry.update(topk=wc.topk, window=wc.window, indexer=f"{wc.indexer} {wc.H_I}x{wc.d_I}")
+    else:
+        entry.update(window=wc.window, attention="dense over every visible entry + window")
+    if rank == 0 and dist_ctx.world == 1 and not args.no_cpu_baseline:
+        entry["cpu_baseline"] = cpu_baseline(wc, inp_c, n_cpu, hca=hca)
+    return entry
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -868,6 +905,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the c2 (n=8192, bf16 indexer) and HCA prefill (n=32768) lines")
+    ap.add_argument("--only", choices=["c2", "hca"], default=None,
+                    help="run only the n=8192 (c2) or the HCA n=32768 prefill (profiler "
+                         "captures; the line is then not the headline)")
     ap.add_argument("--no-fp8-peak", action="store_true",
                     help="skip the e4m3 peak measurement (the nominal ratio to bf16 is used)")
     args = ap.parse_args()
@@ -938,6 +978,21 @@ def main():
         dist_ctx.close()
         return 0
 
+    if args.only:
+        peaks = Peaks(raw_peaks, peak_src)
+        name = PREFILL_C2 if args.only == "c2" else HCA_PREFILL
+        entry = run_config(name, dev, args, dist_ctx, rank, peaks)
+        line = {"metric": f"{name} prefill queries/s (profiling case, not the headline)",
+                "value": entry["value"], "unit": "queries/s", "n_gpus": dist_ctx.world,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": entry["ms_per_step"],
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+                "dtype": "bf16", "data": "synthetic", "config": {"workload": name},
+                "detail": entry}
+        if rank == 0:
+            print(json.dumps(line))
+        dist_ctx.close()
+        return 0
+
     fp8 = None
     if not args.no_fp8_peak:
         try:
@@ -976,33 +1031,9 @@ def main():
 
     if not args.no_configs:
         # the other two prefill configurations, each timed like the headline
-        for name, mk, path_cls, hca, n_cpu in (
-                (PREFILL_C2, synth.csa_prefill_inputs, PrefillPath, False, 8192),
-                (HCA_PREFILL, synth.hca_prefill_inputs, HcaPrefillPath, True, 32768)):
-            wc = synth.WORKLOADS[name]
-            inp_c = mk(wc, seed=rank)
-            pc = path_cls(wc, inp_c, dev)
-            rc = run_path(pc, args.steps, args.warmup, dist_ctx)
-            cval, cms = dist_ctx.job_rate(wc.B * wc.n, rc["total_ms"] / args.steps)
-            creg, creg_why = regime_of(rc["clocks"], rc["total_ms"])
-            cwork = hca_prefill_work(wc) if hca else prefill_work(wc)
-            cst = stage_rooflines(cwork, rc["kern_ms"], peaks, creg, wc.indexer)
-            cdom = max(rc["kern_ms"], key=rc["kern_ms"].get)
-            croof = dict(cst[cdom]["roofline"], kernel=cdom, regime=f"{creg}: {creg_why}",
-                         traffic=ncu_traffic((cdom, name)))
-            entry = {"workload": name, "value": cval, "unit": "queries/s", "ms_per_step": cms,
-                     "B": wc.B, "n": wc.n, "m": wc.m, "overlap": wc.overlap,
-                     "l2": "inputs larger than L2 (q alone is 256 MiB or more)",
-                     "roofline": croof, "stages": cst, "gpu_launches": rc["launches"],
-                     "clocks": rc["clocks"]}
-            if not hca:
-                entry.update(topk=wc.topk, window=wc.window, indexer=f"{wc.indexer} {wc.H_I}x{wc.d_I}")
-            else:
-                entry.update(window=wc.window, attention="dense over every visible entry + window")
-            if rank == 0 and dist_ctx.world == 1 and not args.no_cpu_baseline:
-                entry["cpu_baseline"] = cpu_baseline(wc, inp_c, n_cpu, hca=hca)
-            line["hca_prefill" if hca else "c2_prefill"] = entry
-            del pc, inp_c
+        for name in (PREFILL_C2, HCA_PREFILL):
+            key = "hca_prefill" if name == HCA_PREFILL else "c2_prefill"
+            line[key] = run_config(name, dev, args, dist_ctx, rank, peaks)
             torch.cuda.empty_cache()
 
     if not args.no_variants:
