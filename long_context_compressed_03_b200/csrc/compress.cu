@@ -173,6 +173,238 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(CompressKArgs a) {
     store_entry_rows<OUT, kThreads>(outs, ne, d_out, a.out, a.out_row_scale, ent0 + i0, a.hnorm);
 }
 
+// ---------------------------------------------------------------- tensor-core path
+// bf16 x and W: the projection runs on the tensor cores (mma.sync m16n8k16,
+// bf16 operands, fp32 accumulate).  The pooled fp32 value is split into
+// three bf16 parts, v = h1 + h2 + h3 exactly (8 + 8 + 8 significant bits;
+// each residual is exact in fp32), and W is bf16 already, so the three
+// products per term are exact and only the accumulation rounds -- fp32
+// accuracy, as the FFMA path above.  A CTA owns E entries (E = 32 for small
+// m; fewer for long blocks, so a CTA reads at most 64 KB of x); its x rows
+// are summed with 16-byte loads, R rows per work item, all in flight.
+constexpr int kME = 32;                  // entry rows of the MMA tile (two m16 tiles)
+
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+// D(16x8, f32) += A(16x16, bf16, row) * B(16x8, bf16, col)
+__device__ __forceinline__ void mma_bf16(float (&c)[4], const uint32_t (&a)[4], uint32_t b0,
+                                         uint32_t b1) {
+    asm volatile("mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, "
+                 "{%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                 : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Two fp32 values split into three bf16 pairs (lo element in the low half):
+// v = h1 + h2 + h3 exactly for normal values.
+__device__ __forceinline__ void split3(float v0, float v1, uint32_t& p1, uint32_t& p2, uint32_t& p3) {
+    const __nv_bfloat16 a1 = __float2bfloat16_rn(v0), b1 = __float2bfloat16_rn(v1);
+    const float r0 = v0 - __bfloat162float(a1), s0 = v1 - __bfloat162float(b1);
+    const __nv_bfloat16 a2 = __float2bfloat16_rn(r0), b2 = __float2bfloat16_rn(s0);
+    const __nv_bfloat16 a3 = __float2bfloat16_rn(r0 - __bfloat162float(a2));
+    const __nv_bfloat16 b3 = __float2bfloat16_rn(s0 - __bfloat162float(b2));
+    p1 = (uint32_t)__bfloat16_as_ushort(a1) | ((uint32_t)__bfloat16_as_ushort(b1) << 16);
+    p2 = (uint32_t)__bfloat16_as_ushort(a2) | ((uint32_t)__bfloat16_as_ushort(b2) << 16);
+    p3 = (uint32_t)__bfloat16_as_ushort(a3) | ((uint32_t)__bfloat16_as_ushort(b3) << 16);
+}
+
+// Shared memory of the tensor-core path: W (bf16, rows padded by 8), the
+// partial block sums, the pooled rows (fp32, rows padded by 4); the output
+// rows reuse the last two.
+struct MmaSmem {
+    int ws, ps;                      // row strides of W (bf16) and pooled (fp32), elements
+    size_t w_bytes, sum_bytes, pool_bytes, bytes;
+};
+__host__ __device__ inline MmaSmem mma_smem(int d_in, int d_out, int G, int nb) {
+    MmaSmem s;
+    s.ws = d_out + 8;
+    s.ps = d_in + 4;
+    s.w_bytes = (size_t)d_in * s.ws * 2;
+    s.sum_bytes = (size_t)G * nb * d_in * 4;
+    s.pool_bytes = (size_t)kME * s.ps * 4;
+    size_t tail = s.sum_bytes + s.pool_bytes;
+    const size_t outs = (size_t)kME * d_out * 4;
+    if (outs > tail) tail = outs;
+    s.bytes = s.w_bytes + tail;
+    return s;
+}
+
+template <int R, int OUT>
+__global__ void __launch_bounds__(kThreads) compress_mma_kernel(CompressKArgs a, int E) {
+    extern __shared__ __align__(16) uint8_t smem8[];
+    const int d_in = a.d_in, d_out = a.d_out, m = a.m;
+    const int G = m / R;                               // row groups of a block
+    const int b = blockIdx.y;
+    size_t tok0 = (size_t)b * a.n, ent0 = (size_t)b * a.N_c;
+    int N_c = a.N_c;
+    if (a.map.S) {
+        tok0 = (size_t)a.map.tok[b];
+        ent0 = (size_t)a.map.ent[b];
+        N_c = (a.map.tok[b + 1] - a.map.tok[b]) / m;
+    }
+    const int i0 = blockIdx.x * E;
+    if (i0 >= N_c) return;                             // a shorter packed sequence
+    const int ne = min(E, N_c - i0);
+    const int jb0 = a.overlap ? -1 : 0;                // block i0 - 1 when overlapping
+    const int nb = ne - jb0;                           // blocks summed
+    const MmaSmem L = mma_smem(d_in, d_out, G, nb);
+    __nv_bfloat16* sW = reinterpret_cast<__nv_bfloat16*>(smem8);
+    float* psum = reinterpret_cast<float*>(smem8 + L.w_bytes);            // [G][nb][d_in]
+    float* pool = reinterpret_cast<float*>(smem8 + L.w_bytes + L.sum_bytes);  // [kME][ps]
+    float* outs = reinterpret_cast<float*>(smem8 + L.w_bytes);            // [kME][d_out], later
+    const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(a.x) + tok0 * d_in;
+    const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(a.W);
+    const int tid = threadIdx.x;
+
+    // ---- W, with 16-byte loads (L2-resident across CTAs)
+    {
+        const int c8s = d_out / 8;
+        for (int q = tid; q < d_in * c8s; q += kThreads) {
+            const int k = q / c8s, c8 = q - k * c8s;
+            *reinterpret_cast<uint4*>(sW + k * L.ws + c8 * 8) =
+                __ldg(reinterpret_cast<const uint4*>(W + (size_t)k * d_out) + c8);
+        }
+    }
+    // ---- partial block sums: work item (group g, block jb, 16-byte piece f), R rows
+    {
+        const int pieces = d_in / 8;
+        const int items = G * nb * pieces;
+        constexpr int kPer = 16 / R;                   // items per thread with loads in flight together
+        for (int w0 = tid; w0 < items; w0 += kThreads * kPer) {
+            uint4 v[kPer][R];
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) {
+                const int w = w0 + q * kThreads;
+                const int f = w % pieces, rest = w / pieces;
+                const int jb = rest % nb, g = rest / nb;
+                const int blk = i0 + jb0 + jb;
+                const bool live = w < items && blk >= 0;
+                const uint4* src = reinterpret_cast<const uint4*>(x + ((size_t)(live ? blk : 0) * m + g * R) * d_in) + f;
+#pragma unroll
+                for (int r = 0; r < R; ++r)
+                    v[q][r] = live ? __ldg(src + (size_t)r * pieces) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int q = 0; q < kPer; ++q) {
+                const int w = w0 + q * kThreads;
+                if (w >= items) continue;
+                float acc[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+#pragma unroll
+                for (int r = 0; r < R; ++r) Vec<__nv_bfloat16>::add(acc, v[q][r]);
+                const int f = w % pieces, rest = w / pieces;
+                float* dst = psum + (size_t)rest * d_in + f * 8;      // rest = g * nb + jb
+                *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+            }
+        }
+    }
+    __syncthreads();
+    // ---- pooled rows: (previous block + own block) / count; rows >= ne are 0
+    for (int q = tid; q < kME * d_in; q += kThreads) {
+        const int e = q / d_in, c = q - e * d_in;
+        float v = 0.0f;
+        if (e < ne) {
+            float cur = 0.0f, prev = 0.0f;
+            for (int g = 0; g < G; ++g) {
+                cur += psum[((size_t)g * nb + e - jb0) * d_in + c];
+                if (a.overlap) prev += psum[((size_t)g * nb + e - jb0 - 1) * d_in + c];
+            }
+            const int i = i0 + e;
+            const int lo = a.overlap ? max(0, m * (i - 1)) : m * i;
+            v = (a.overlap ? prev + cur : cur) / (float)(m * (i + 1) - lo);
+        }
+        pool[e * L.ps + c] = v;
+    }
+    __syncthreads();
+    // ---- projection: warp w takes m16 tile (w % mtiles) and a range of n8 tiles
+    const int warp = tid >> 5, lane = tid & 31;
+    const int mtiles = ne > 16 ? 2 : 1;
+    const int wpm = 8 / mtiles;                        // warps per m16 tile
+    const int ncols = d_out / wpm;                     // a multiple of 8 (d_out % 64 == 0)
+    const int mt = warp % mtiles, n0 = (warp / mtiles) * ncols;
+    const int ntiles = ncols / 8;                      // 1 .. 8
+    float acc[8][4];
+#pragma unroll
+    for (int t = 0; t < 8; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.0f;
+    const int g8 = lane >> 2, c2 = 2 * (lane & 3);
+    const float* prow0 = pool + (mt * 16 + g8) * L.ps;
+    const float* prow1 = prow0 + 8 * L.ps;
+    const uint32_t sw_base = (uint32_t)__cvta_generic_to_shared(sW);
+    for (int ks = 0; ks < d_in / 16; ++ks) {
+        const int k0 = ks * 16 + c2;
+        const float2 v00 = *reinterpret_cast<const float2*>(prow0 + k0);
+        const float2 v10 = *reinterpret_cast<const float2*>(prow1 + k0);
+        const float2 v01 = *reinterpret_cast<const float2*>(prow0 + k0 + 8);
+        const float2 v11 = *reinterpret_cast<const float2*>(prow1 + k0 + 8);
+        uint32_t A[3][4];
+        split3(v00.x, v00.y, A[0][0], A[1][0], A[2][0]);
+        split3(v10.x, v10.y, A[0][1], A[1][1], A[2][1]);
+        split3(v01.x, v01.y, A[0][2], A[1][2], A[2][2]);
+        split3(v11.x, v11.y, A[0][3], A[1][3], A[2][3]);
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+            if (2 * np >= ntiles) break;
+            uint32_t b0, b1, b2, b3;
+            const uint32_t addr = sw_base + (uint32_t)(((ks * 16 + (lane & 15)) * L.ws + n0 + np * 16 +
+                                                        (lane >> 4) * 8) * 2);
+            ldsm_x4_t(addr, b0, b1, b2, b3);
+#pragma unroll
+            for (int sp = 0; sp < 3; ++sp) {
+                mma_bf16(acc[2 * np], A[sp], b0, b1);
+                if (2 * np + 1 < ntiles) mma_bf16(acc[2 * np + 1], A[sp], b2, b3);
+            }
+        }
+    }
+    __syncthreads();                                   // pooled rows and sums are no longer read
+#pragma unroll
+    for (int t = 0; t < 8; ++t) {
+        if (t >= ntiles) break;
+        const int col = n0 + t * 8 + c2;
+        const int r0 = mt * 16 + g8, r1 = r0 + 8;
+        if (r0 < ne) *reinterpret_cast<float2*>(outs + r0 * d_out + col) = make_float2(acc[t][0], acc[t][1]);
+        if (r1 < ne) *reinterpret_cast<float2*>(outs + r1 * d_out + col) = make_float2(acc[t][2], acc[t][3]);
+    }
+    __syncthreads();
+    store_entry_rows<OUT, kThreads>(outs, ne, d_out, a.out, a.out_row_scale, ent0 + i0, a.hnorm);
+}
+
+template <int R, int OUT>
+cudaError_t launch_mma_r(const CompressKArgs& a, cudaStream_t s) {
+    // entries per CTA: at most 64 KB of x (and 32, the MMA tile)
+    int E = (int)(65536 / ((size_t)a.m * a.d_in * 2));
+    E = E < 1 ? 1 : (E > kME ? kME : E);
+    const int G = a.m / R;
+    const MmaSmem L = mma_smem(a.d_in, a.d_out, G, E + (a.overlap ? 1 : 0));
+    auto kern = compress_mma_kernel<R, OUT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.bytes);
+    if (e != cudaSuccess) return e;
+    dim3 grid((a.N_c + E - 1) / E, a.B);
+    kern<<<grid, kThreads, L.bytes, s>>>(a, E);
+    count_launch();
+    return cudaGetLastError();
+}
+
+template <int OUT>
+cudaError_t launch_mma(const CompressKArgs& a, cudaStream_t s) {
+    const int m = a.m;
+    if (m % 16 == 0) return launch_mma_r<16, OUT>(a, s);
+    if (m % 8 == 0) return launch_mma_r<8, OUT>(a, s);
+    if (m % 4 == 0) return launch_mma_r<4, OUT>(a, s);
+    if (m % 2 == 0) return launch_mma_r<2, OUT>(a, s);
+    return launch_mma_r<1, OUT>(a, s);
+}
+
+// The tensor-core path serves bf16 x / W with d_in a multiple of 16 and d_out
+// a multiple of 64, both at most 256 (shared memory: W, sums, pooled rows).
+bool mma_path(const CompressArgs& a) {
+    return a.x_dt == DT_BF16 && a.d_in % 16 == 0 && a.d_out % 64 == 0 && a.d_in <= 256 &&
+           a.d_out <= 256;
+}
+
 template <typename Tin, int OUT>
 cudaError_t launch_t(const CompressArgs& args, cudaStream_t s) {
     CompressKArgs a;
@@ -198,6 +430,13 @@ cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s, const char** 
         if (a.out_dt == DT_BF16) return launch_t<float, DT_BF16>(a, s);
         if (a.out_dt == DT_E4M3) return launch_t<float, DT_E4M3>(a, s);
         if (a.out_dt == DT_E4M3H) return launch_t<float, DT_E4M3H>(a, s);
+    } else if (a.x_dt == DT_BF16 && mma_path(a)) {
+        CompressKArgs k;
+        static_cast<CompressArgs&>(k) = a;
+        if (a.vl) k.map = *a.vl;
+        if (a.out_dt == DT_BF16) return launch_mma<DT_BF16>(k, s);
+        if (a.out_dt == DT_E4M3) return launch_mma<DT_E4M3>(k, s);
+        if (a.out_dt == DT_E4M3H) return launch_mma<DT_E4M3H>(k, s);
     } else if (a.x_dt == DT_BF16) {
         if (a.out_dt == DT_BF16) return launch_t<__nv_bfloat16, DT_BF16>(a, s);
         if (a.out_dt == DT_E4M3) return launch_t<__nv_bfloat16, DT_E4M3>(a, s);

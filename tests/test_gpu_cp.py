@@ -57,13 +57,12 @@ def test_one_rank_zigzag_matches_the_single_call(fp8):
             _same(res[key], ref[key])
     # and against the oracle on sampled rows of the second span
     rows = np.arange(N // 2, N, 97)
-    kI = res["kI_c"].cpu().numpy()[None]
+    kI = res["kI_c"].cpu().numpy()[None] if fp8 else np64(res["kI_c"])[None]
     sc = res["kI_scale"].cpu().numpy()[None] if fp8 else None
     qrows = inp["qI"][rows].float().cpu().numpy()
     qrows = oracle.quantized_query_rows(qrows) if fp8 else qrows.astype(np.float64)
     scores = oracle.indexer_scores_rows(qrows, np.zeros(rows.size, np.int32),
-                                        rows.astype(np.int32), kI if fp8 else np64(res["kI_c"])[None],
-                                        M, np.array([N // M], np.int32), sc)
+                                        rows.astype(np.int32), kI, M, np.array([N // M], np.int32), sc)
     idx = res["idx"].cpu().numpy()[rows]
     check_topk(idx, scores, K, label=f"CP span indexer (fp8={fp8})")
     ro, _ = oracle.sparse_attn_rows(np64(inp["q"])[rows], np.zeros(rows.size, np.int32),
