@@ -258,13 +258,24 @@ __global__ void __launch_bounds__(kThreads) compress_mma_kernel(CompressKArgs a,
     const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(a.W);
     const int tid = threadIdx.x;
 
-    // ---- W, with 16-byte loads (L2-resident across CTAs)
+    // ---- W, with 16-byte loads (L2-resident across CTAs), eight in flight per thread
     {
-        const int c8s = d_out / 8;
-        for (int q = tid; q < d_in * c8s; q += kThreads) {
-            const int k = q / c8s, c8 = q - k * c8s;
-            *reinterpret_cast<uint4*>(sW + k * L.ws + c8 * 8) =
-                __ldg(reinterpret_cast<const uint4*>(W + (size_t)k * d_out) + c8);
+        const int c8s = d_out / 8, nw = d_in * c8s;
+        for (int q0 = tid; q0 < nw; q0 += 8 * kThreads) {
+            uint4 wv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int q = q0 + i * kThreads;
+                wv[i] = q < nw ? __ldg(reinterpret_cast<const uint4*>(W) + q) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int q = q0 + i * kThreads;
+                if (q < nw) {
+                    const int k = q / c8s, c8 = q - k * c8s;
+                    *reinterpret_cast<uint4*>(sW + k * L.ws + c8 * 8) = wv[i];
+                }
+            }
         }
     }
     // ---- partial block sums: work item (group g, block jb, 16-byte piece f), R rows
