@@ -22,6 +22,7 @@
 #include "common.cuh"
 #include "entry_epilogue.cuh"
 #include "kernels.h"
+#include "tc_common.cuh"
 
 namespace csa {
 namespace {
@@ -383,6 +384,308 @@ __global__ void __launch_bounds__(kThreads) compress_mma_kernel(CompressKArgs a,
     store_entry_rows<OUT, kThreads>(outs, ne, d_out, a.out, a.out_row_scale, ent0 + i0, a.hnorm);
 }
 
+// ---------------------------------------------------------------- streaming path
+// The same arithmetic as compress_mma_kernel, persistent: one CTA per SM
+// walks the tiles t = blockIdx.x, + gridDim.x, ... of every batch element.
+// W is staged once per CTA.  A tile's rows of x are one contiguous range of
+// global memory, so one thread brings them into shared memory with a single
+// bulk copy (TMA, no multicast) on an mbarrier; the next tile's copy is in
+// flight while a tile is summed, projected and stored (two slab buffers).
+// The pooled rows are split into their three bf16 planes once, in shared
+// memory, and read by ldmatrix.
+struct StreamArgs {
+    CompressKArgs a;
+    int E;                  // entries per tile
+    int tiles_per_seq;
+    int tiles;              // B * tiles_per_seq
+    uint32_t* err;
+    uint64_t wait_ns;
+};
+
+struct StreamSmem {
+    int ws, as;
+    size_t w_bytes, slab_bytes, sum_bytes, plane_bytes, bar_off, bytes;
+};
+__host__ __device__ inline StreamSmem stream_smem(int d_in, int d_out, int m, int G, int E) {
+    StreamSmem s;
+    s.ws = d_out + 8;
+    s.as = d_in + 8;
+    s.w_bytes = (size_t)d_in * s.ws * 2;
+    s.slab_bytes = (size_t)(E + 1) * m * d_in * 2;
+    s.sum_bytes = (size_t)G * (E + 1) * d_in * 4;
+    s.plane_bytes = (size_t)3 * kME * s.as * 2;
+    size_t tail = s.sum_bytes + s.plane_bytes;
+    const size_t outs = (size_t)kME * d_out * 4;
+    if (outs > tail) tail = outs;
+    s.bar_off = s.w_bytes + 2 * s.slab_bytes + tail;
+    s.bytes = s.bar_off + 32 + kME * 4;      // barriers, abort flag, 1 / count per entry
+    return s;
+}
+
+__device__ __forceinline__ void bulk_copy(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+        ::"r"(tc::smem_u32(dst)), "l"(src), "r"(bytes), "r"(tc::smem_u32(bar))
+        : "memory");
+}
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+    asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3) : "r"(addr));
+}
+
+template <int R, int OUT>
+__global__ void __launch_bounds__(kThreads, 1) compress_stream_kernel(StreamArgs sa) {
+    extern __shared__ __align__(128) uint8_t smem8[];
+    const CompressKArgs& a = sa.a;
+    const int d_in = a.d_in, d_out = a.d_out, m = a.m, E = sa.E;
+    const int G = m / R;
+    const int jb0 = a.overlap ? -1 : 0;
+    const StreamSmem L = stream_smem(d_in, d_out, m, G, E);
+    __nv_bfloat16* sW = reinterpret_cast<__nv_bfloat16*>(smem8);
+    uint8_t* slab0 = smem8 + L.w_bytes;                                     // [2][(E+1) m][d_in] bf16
+    float* psum = reinterpret_cast<float*>(smem8 + L.w_bytes + 2 * L.slab_bytes);   // [G][E+1][d_in]
+    __nv_bfloat16* planes = reinterpret_cast<__nv_bfloat16*>(
+        smem8 + L.w_bytes + 2 * L.slab_bytes + L.sum_bytes);                // [3][kME][as]
+    float* outs = psum;                                                     // [kME][d_out], later
+    uint64_t* bar = reinterpret_cast<uint64_t*>(smem8 + L.bar_off);         // [2]
+    volatile int* abort = reinterpret_cast<volatile int*>(smem8 + L.bar_off + 16);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const __nv_bfloat16* xg = static_cast<const __nv_bfloat16*>(a.x);
+    const size_t row_bytes = (size_t)d_in * 2;
+
+    // a tile's rows: blocks i0 + jb0 .. i0 + ne - 1 of element b (block -1 absent)
+    auto tile_of = [&](int t, int& b, int& i0, int& ne) {
+        b = t / sa.tiles_per_seq;
+        i0 = (t - b * sa.tiles_per_seq) * E;
+        ne = min(E, a.N_c - i0);
+    };
+    auto issue = [&](int t, int buf) {           // one thread
+        int b, i0, ne;
+        tile_of(t, b, i0, ne);
+        const int blk0 = max(i0 + jb0, 0);
+        const int nblk = i0 + ne - blk0;
+        const uint32_t bytes = (uint32_t)((size_t)nblk * m * row_bytes);
+        uint8_t* dst = slab0 + (size_t)buf * L.slab_bytes + (size_t)(blk0 - (i0 + jb0)) * m * row_bytes;
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(xg + ((size_t)b * a.n + (size_t)blk0 * m) * d_in);
+        tc::mbar_arrive_expect_tx(&bar[buf], bytes);
+        bulk_copy(dst, src, bytes, &bar[buf]);
+    };
+
+    if (tid == 0) {
+        tc::mbar_init(&bar[0], 1);
+        tc::mbar_init(&bar[1], 1);
+        *abort = (*reinterpret_cast<volatile uint32_t*>(sa.err) != 0u) ? 1 : 0;
+        tc::fence_barrier_init();
+    }
+    __syncthreads();
+    int issued = 0;                                   // copies issued (thread 0)
+    if (tid == 0 && blockIdx.x < sa.tiles && !*abort) { issue(blockIdx.x, 0); issued = 1; }
+    // ---- W once, eight 16-byte loads in flight per thread
+    {
+        const int c8s = d_out / 8, nw = d_in * c8s;
+        const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(a.W);
+        for (int q0 = tid; q0 < nw; q0 += 8 * kThreads) {
+            uint4 wv[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int q = q0 + i * kThreads;
+                wv[i] = q < nw ? __ldg(reinterpret_cast<const uint4*>(W) + q) : make_uint4(0u, 0u, 0u, 0u);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int q = q0 + i * kThreads;
+                if (q < nw) {
+                    const int k = q / c8s, c8 = q - k * c8s;
+                    *reinterpret_cast<uint4*>(sW + k * L.ws + c8 * 8) = wv[i];
+                }
+            }
+        }
+    }
+    // per-thread coordinates of the sums and the pooled rows (one division each)
+    const int pieces = d_in / 8;
+    const int sum_f = tid % pieces, sum_q0 = tid / pieces, sum_step = kThreads / pieces;
+    const int dh = d_in / 2;
+    const int pool_c = 2 * (tid % dh), pool_e0 = tid / dh, pool_estep = kThreads / dh;
+    float* inv_cnt = reinterpret_cast<float*>(smem8 + L.bar_off + 32);   // [kME]
+    int k = 0;
+    for (int t = blockIdx.x; t < sa.tiles; t += gridDim.x, ++k) {
+        const int buf = k & 1;
+        // the next tile's rows into the other buffer (its last reader finished
+        // at the end of the previous tile)
+        if (tid == 0 && t + (int)gridDim.x < sa.tiles && !*abort) { issue(t + gridDim.x, buf ^ 1); ++issued; }
+        // this tile's rows have landed (every thread waits: bounded)
+        const bool okw = tc::mbar_wait(&bar[buf], (k >> 1) & 1, abort, sa.err, sa.wait_ns);
+        if (__syncthreads_or(!okw)) break;
+        int b, i0, ne;
+        tile_of(t, b, i0, ne);
+        const int nb = ne - jb0;
+        const __nv_bfloat16* slab = reinterpret_cast<const __nv_bfloat16*>(slab0 + (size_t)buf * L.slab_bytes);
+        // ---- partial block sums from shared memory: item (g, jb, 16-byte piece f), R rows;
+        //      a thread keeps its piece and steps (g, jb) without divisions
+        {
+            const int items = G * nb;
+            int q = sum_q0, jb = sum_q0, g = 0;
+            while (jb >= nb) { jb -= nb; ++g; }
+            for (; q < items; q += sum_step) {
+                float acc[8];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = 0.0f;
+                if (i0 + jb0 + jb >= 0) {
+                    const uint4* src = reinterpret_cast<const uint4*>(slab + ((size_t)jb * m + g * R) * d_in) + sum_f;
+#pragma unroll
+                    for (int r = 0; r < R; ++r) Vec<__nv_bfloat16>::add(acc, src[(size_t)r * pieces]);
+                }
+                float* dst = psum + (size_t)(g * nb + jb) * d_in + sum_f * 8;
+                *reinterpret_cast<float4*>(dst) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+                *reinterpret_cast<float4*>(dst + 4) = make_float4(acc[4], acc[5], acc[6], acc[7]);
+                jb += sum_step;
+                while (jb >= nb) { jb -= nb; ++g; }
+            }
+        }
+        // the tile's 1 / count per entry (exact for the power-of-two counts of
+        // m = 2^j; otherwise one more rounding, inside the same error bound)
+        if (tid < kME) {
+            const int i = i0 + tid;
+            const int lo = a.overlap ? max(0, m * (i - 1)) : m * i;
+            inv_cnt[tid] = 1.0f / (float)(m * (i + 1) - lo);
+        }
+        __syncthreads();
+        // ---- pooled rows split into three bf16 planes (rows >= ne are 0); a
+        //      thread keeps its column pair and steps the entry
+        for (int e = pool_e0; e < kME; e += pool_estep) {
+            float v0 = 0.0f, v1 = 0.0f;
+            if (e < ne) {
+                float c0 = 0.0f, c1 = 0.0f, p0 = 0.0f, p1 = 0.0f;
+                for (int g = 0; g < G; ++g) {
+                    const float2 cur = *reinterpret_cast<const float2*>(psum + ((size_t)g * nb + e - jb0) * d_in + pool_c);
+                    c0 += cur.x;
+                    c1 += cur.y;
+                    if (a.overlap) {
+                        const float2 pr = *reinterpret_cast<const float2*>(psum + ((size_t)g * nb + e - jb0 - 1) * d_in + pool_c);
+                        p0 += pr.x;
+                        p1 += pr.y;
+                    }
+                }
+                const float ic = inv_cnt[e];
+                v0 = (a.overlap ? p0 + c0 : c0) * ic;
+                v1 = (a.overlap ? p1 + c1 : c1) * ic;
+            }
+            uint32_t h1, h2, h3;
+            split3(v0, v1, h1, h2, h3);
+            const size_t o = (size_t)e * L.as + pool_c;
+            *reinterpret_cast<uint32_t*>(planes + o) = h1;
+            *reinterpret_cast<uint32_t*>(planes + (size_t)kME * L.as + o) = h2;
+            *reinterpret_cast<uint32_t*>(planes + 2 * (size_t)kME * L.as + o) = h3;
+        }
+        __syncthreads();
+        // ---- projection: warp w takes m16 tile (w % mtiles) and a range of n8 tiles
+        const int mtiles = ne > 16 ? 2 : 1;
+        const int wpm = 8 / mtiles;
+        const int ncols = d_out / wpm;
+        const int mt = warp % mtiles, n0 = (warp / mtiles) * ncols;
+        const int ntiles = ncols / 8;
+        float acc[8][4];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.0f;
+        const uint32_t sw_base = tc::smem_u32(sW);
+        const uint32_t pl_base = tc::smem_u32(planes);
+        for (int ks = 0; ks < d_in / 16; ++ks) {
+            uint32_t A[3][4];
+#pragma unroll
+            for (int sp = 0; sp < 3; ++sp) {
+                const uint32_t addr = pl_base + (uint32_t)((((size_t)sp * kME + mt * 16 + (lane & 15)) * L.as +
+                                                           ks * 16 + (lane >> 4) * 8) * 2);
+                ldsm_x4(addr, A[sp][0], A[sp][1], A[sp][2], A[sp][3]);
+            }
+#pragma unroll
+            for (int np = 0; np < 4; ++np) {
+                if (2 * np >= ntiles) break;
+                uint32_t b0, b1, b2, b3;
+                const uint32_t addr = sw_base + (uint32_t)(((ks * 16 + (lane & 15)) * L.ws + n0 + np * 16 +
+                                                            (lane >> 4) * 8) * 2);
+                ldsm_x4_t(addr, b0, b1, b2, b3);
+#pragma unroll
+                for (int sp = 0; sp < 3; ++sp) {
+                    mma_bf16(acc[2 * np], A[sp], b0, b1);
+                    if (2 * np + 1 < ntiles) mma_bf16(acc[2 * np + 1], A[sp], b2, b3);
+                }
+            }
+        }
+        __syncthreads();                               // sums and planes are no longer read
+        {
+            const int g8 = lane >> 2, c2 = 2 * (lane & 3);
+#pragma unroll
+            for (int tt = 0; tt < 8; ++tt) {
+                if (tt >= ntiles) break;
+                const int col = n0 + tt * 8 + c2;
+                const int r0 = mt * 16 + g8, r1 = r0 + 8;
+                if (r0 < ne) *reinterpret_cast<float2*>(outs + r0 * d_out + col) = make_float2(acc[tt][0], acc[tt][1]);
+                if (r1 < ne) *reinterpret_cast<float2*>(outs + r1 * d_out + col) = make_float2(acc[tt][2], acc[tt][3]);
+            }
+        }
+        __syncthreads();
+        store_entry_rows<OUT, kThreads>(outs, ne, d_out, a.out, a.out_row_scale,
+                                        (size_t)b * a.N_c + i0, a.hnorm);
+        __syncthreads();                               // outs (and this slab) free for the next tile
+    }
+    // copies still in flight (an abort) land before the CTA's shared memory is given up
+    if (tid == 0) {
+        volatile int never = 0;
+        for (int j = max(0, issued - 2); j < issued; ++j)
+            tc::mbar_wait(&bar[j & 1], (j >> 1) & 1, &never, sa.err);
+    }
+    __syncthreads();
+}
+
+template <int R, int OUT>
+cudaError_t launch_stream_r(const CompressKArgs& a, cudaStream_t s) {
+    int E = (int)(65536 / ((size_t)a.m * a.d_in * 2));
+    E = E < 1 ? 1 : (E > kME ? kME : E);
+    const int G = a.m / R;
+    const StreamSmem L = stream_smem(a.d_in, a.d_out, a.m, G, E);
+    uint32_t* err = device_error_word();
+    if (!err) return cudaErrorUnknown;
+    StreamArgs sa;
+    sa.a = a;
+    sa.E = E;
+    sa.tiles_per_seq = (a.N_c + E - 1) / E;
+    sa.tiles = a.B * sa.tiles_per_seq;
+    sa.err = err;
+    sa.wait_ns = wait_limit_ns();
+    auto kern = compress_stream_kernel<R, OUT>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)L.bytes);
+    if (e != cudaSuccess) return e;
+    int dev = 0, sms = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int grid = sa.tiles < sms ? sa.tiles : sms;
+    kern<<<grid, kThreads, L.bytes, s>>>(sa);
+    count_launch();
+    return cudaGetLastError();
+}
+
+template <int OUT>
+cudaError_t launch_stream(const CompressKArgs& a, cudaStream_t s) {
+    const int m = a.m;
+    if (m % 16 == 0) return launch_stream_r<16, OUT>(a, s);
+    if (m % 8 == 0) return launch_stream_r<8, OUT>(a, s);
+    if (m % 4 == 0) return launch_stream_r<4, OUT>(a, s);
+    if (m % 2 == 0) return launch_stream_r<2, OUT>(a, s);
+    return launch_stream_r<1, OUT>(a, s);
+}
+
+// The streaming path: unpacked calls whose tiles fit the shared memory (two
+// row slabs, W, sums and planes) and whose rows are 16-byte multiples.
+bool stream_path(const CompressArgs& a) {
+    if (a.vl || a.B <= 0 || a.N_c <= 0) return false;
+    int E = (int)(65536 / ((size_t)a.m * a.d_in * 2));
+    E = E < 1 ? 1 : (E > kME ? kME : E);
+    int R = 16;
+    while (a.m % R) R >>= 1;
+    const StreamSmem L = stream_smem(a.d_in, a.d_out, a.m, a.m / R, E);
+    return L.bytes <= 227 * 1024;
+}
+
 template <int R, int OUT>
 cudaError_t launch_mma_r(const CompressKArgs& a, cudaStream_t s) {
     // entries per CTA: at most 64 KB of x (and 32, the MMA tile)
@@ -445,6 +748,11 @@ cudaError_t launch_compress(const CompressArgs& a, cudaStream_t s, const char** 
         CompressKArgs k;
         static_cast<CompressArgs&>(k) = a;
         if (a.vl) k.map = *a.vl;
+        if (stream_path(a)) {
+            if (a.out_dt == DT_BF16) return launch_stream<DT_BF16>(k, s);
+            if (a.out_dt == DT_E4M3) return launch_stream<DT_E4M3>(k, s);
+            if (a.out_dt == DT_E4M3H) return launch_stream<DT_E4M3H>(k, s);
+        }
         if (a.out_dt == DT_BF16) return launch_mma<DT_BF16>(k, s);
         if (a.out_dt == DT_E4M3) return launch_mma<DT_E4M3>(k, s);
         if (a.out_dt == DT_E4M3H) return launch_mma<DT_E4M3H>(k, s);

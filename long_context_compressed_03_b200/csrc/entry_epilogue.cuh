@@ -33,8 +33,33 @@ __device__ __forceinline__ void store_entry_rows(float* rows, int ne, int d_out,
         }
     } else {
         using Tout = typename std::conditional<OUT == DT_F32, float, __nv_bfloat16>::type;
-        Tout* out = static_cast<Tout*>(out_v);
-        for (int p = tid; p < ne * d_out; p += kThreads) store_out<Tout>(out + row0 * d_out + p, rows[p]);
+        Tout* out = static_cast<Tout*>(out_v) + row0 * d_out;
+        constexpr int kV = 16 / (int)sizeof(Tout);          // values per 16-byte store
+        if (d_out % kV == 0 && (reinterpret_cast<uintptr_t>(out) & 15u) == 0 &&
+            (reinterpret_cast<uintptr_t>(rows) & 15u) == 0) {
+            // the rows are contiguous in the output: 16-byte stores, same rounding
+            const int nv = ne * d_out / kV;
+            for (int p = tid; p < nv; p += kThreads) {
+                const float4* r = reinterpret_cast<const float4*>(rows + p * kV);
+                uint4 v;
+                if constexpr (OUT == DT_F32) {
+                    const float4 f = r[0];
+                    v = make_uint4(__float_as_uint(f.x), __float_as_uint(f.y), __float_as_uint(f.z),
+                                   __float_as_uint(f.w));
+                } else {
+                    const float4 f0 = r[0], f1 = r[1];
+                    const __nv_bfloat162 h0 = __floats2bfloat162_rn(f0.x, f0.y);
+                    const __nv_bfloat162 h1 = __floats2bfloat162_rn(f0.z, f0.w);
+                    const __nv_bfloat162 h2 = __floats2bfloat162_rn(f1.x, f1.y);
+                    const __nv_bfloat162 h3 = __floats2bfloat162_rn(f1.z, f1.w);
+                    v = make_uint4(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1),
+                                   *reinterpret_cast<const uint32_t*>(&h2), *reinterpret_cast<const uint32_t*>(&h3));
+                }
+                *reinterpret_cast<uint4*>(out + (size_t)p * kV) = v;
+            }
+        } else {
+            for (int p = tid; p < ne * d_out; p += kThreads) store_out<Tout>(out + p, rows[p]);
+        }
     }
 }
 
