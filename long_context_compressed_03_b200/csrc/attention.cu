@@ -181,6 +181,11 @@ cudaError_t launch_attention(const AttnArgs& a, cudaStream_t s, const char** why
         if (!err) return cudaErrorUnknown;
         return launch_attention_tc(a, err, s);
     }
+    if (attention_dec_tc_supported(a)) {
+        uint32_t* err = device_error_word();
+        if (!err) return cudaErrorUnknown;
+        return launch_attention_dec_tc(a, err, s);
+    }
     if (attention_split_supported(a)) return launch_attention_split(a, s);
     if (a.dt == DT_F32) return launch_dims<float>(a, s, why);
     if (a.dt == DT_BF16) return launch_dims<__nv_bfloat16>(a, s, why);

@@ -128,6 +128,12 @@ void set_stall(int on);
 bool attention_tc_supported(const AttnArgs& a);
 cudaError_t launch_attention_tc(const AttnArgs& a, uint32_t* err, cudaStream_t s);
 
+// tcgen05 attention for few query rows (decode): bf16, 64 heads x 128, the
+// score tile transposed (128 keys x 64 heads), one row's key tiles dealt over
+// a thread-block cluster sized so that every cluster is resident at once.
+bool attention_dec_tc_supported(const AttnArgs& a);
+cudaError_t launch_attention_dec_tc(const AttnArgs& a, uint32_t* err, cudaStream_t s);
+
 // tcgen05 indexer + fused exact top-k for prefill (d_I = 64, H_I <= 4).
 bool indexer_tc_supported(const IndexerArgs& a);
 cudaError_t launch_indexer_tc(const IndexerArgs& a, uint32_t* err, cudaStream_t s);
