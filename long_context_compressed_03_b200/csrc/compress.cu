@@ -436,7 +436,7 @@ __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r
 
 template <int R, int OUT>
 __global__ void __launch_bounds__(kThreads, 1) compress_stream_kernel(StreamArgs sa) {
-    extern __shared__ __align__(128) uint8_t smem8[];
+    extern __shared__ __align__(16) uint8_t smem8[];
     const CompressKArgs& a = sa.a;
     const int d_in = a.d_in, d_out = a.d_out, m = a.m, E = sa.E;
     const int G = m / R;
