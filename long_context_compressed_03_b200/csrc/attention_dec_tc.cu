@@ -299,6 +299,11 @@ __global__ void __launch_bounds__(kThreads, 1) attn_dec_tc_kernel(const __grid_c
         }
         asm volatile("cp.async.commit_group;" ::: "memory");          // Q: the oldest group
     }
+    // The indices may come from the kernel launched just before this one (the
+    // indexer lets this grid start early, see launch_attention_dec_tc): wait
+    // for it before the first read of idx.  Everything above reads only the
+    // caller's inputs, never a preceding kernel's output.
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     // ---- row codes: >= 0 physical row of a compressed entry, <= -2 raw row -(code + 2), -1 none
     for (int i = tid; i < ntile * kBN; i += kThreads) {
         const int kk = kk0_of(i / kBN) + (i % kBN);
@@ -742,13 +747,19 @@ cudaError_t launch_attention_dec_tc(const AttnArgs& a, uint32_t* err, cudaStream
     cfg.blockDim = dim3(kThreads, 1, 1);
     cfg.dynamicSmemBytes = L.bytes;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    // Programmatic stream serialisation: when the kernel before this one
+    // (the decode indexer) signals early, this grid launches and runs its
+    // prologue -- TMEM, barriers, Q and the first window tiles -- while that
+    // kernel finishes; griddepcontrol.wait orders the read of idx after it.
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = (unsigned)C;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = 2;
     e = lse ? cudaLaunchKernelEx(&cfg, attn_dec_tc_kernel<true>, tm_c, tm_w, a, max_chunk, err, wait_limit_ns())
             : cudaLaunchKernelEx(&cfg, attn_dec_tc_kernel<false>, tm_c, tm_w, a, max_chunk, err, wait_limit_ns());
     count_launch();

@@ -429,6 +429,11 @@ __global__ void __launch_bounds__(kThreads, min_blocks<NU>()) indexer_split_kern
         run_eq += __popc(be);
     }
     cluster.sync();     // keep this CTA's shared memory alive until every peer has read it
+    // This CTA's indices are written: a kernel launched after this one with
+    // programmatic serialisation (the decode attention) may begin its
+    // prologue; it still waits for this grid's completion before reading idx.
+    // Signalled last, so every CTA of this grid already holds its SM.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
 int num_sms() {
