@@ -94,6 +94,7 @@ struct __align__(8) Ctrl {
     uint64_t pv_done;            // one phase per P.V
     uint64_t o_done;             // the last P.V completed (one phase)
     uint64_t fin;
+    uint64_t stall_bar;          // test hook: a barrier nothing completes
     uint32_t tmem_base;
     int abort;
 };
@@ -199,7 +200,7 @@ template <bool LSE>
 __global__ void __launch_bounds__(kThreads, 1) attn_dec_tc_kernel(const __grid_constant__ CUtensorMap tm_c,
                                                                  const __grid_constant__ CUtensorMap tm_w,
                                                                  AttnArgs a, int max_chunk, uint32_t* err,
-                                                                 uint64_t wait_ns) {
+                                                                 uint64_t wait_ns, int stall) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const DecSmem L = dec_smem(max_chunk);
@@ -270,6 +271,7 @@ __global__ void __launch_bounds__(kThreads, 1) attn_dec_tc_kernel(const __grid_c
         mbar_init(&ctl->pv_done, 1);
         mbar_init(&ctl->o_done, 1);
         mbar_init(&ctl->fin, 1);
+        mbar_init(&ctl->stall_bar, 1);
         ctl->abort = (*reinterpret_cast<volatile uint32_t*>(err) != 0u) ? 1 : 0;
         fence_barrier_init();
     }
@@ -283,7 +285,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_dec_tc_kernel(const __grid_c
     }
     __syncthreads();
     // the first contiguous tiles and Q need no row codes: start them now
-    if (tid == 0) {
+    // (nothing is started when an earlier launch left the error word set)
+    if (tid == 0 && !*abort) {
         prefetch_tmap(&tm_c);
         prefetch_tmap(&tm_w);
         for (int j = 0; j < lead; ++j)
@@ -327,14 +330,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_dec_tc_kernel(const __grid_c
     if (warp < kLoadWarps) {
         // ------------------------------------------------------------ loaders
         const int lt = tid;
+        int last = -1;                                   // the last tile handed to issue_tile
         // tile j: TMA tiles were started by thread 0 (prologue) or start here,
         // and every loader arrives at once (the barrier then completes on the
         // TMA bytes; before tile 0 this loader's part of Q must have landed);
         // gathered rows by 16-byte copies, whose loaders arrive once they
         // landed.  One commit group per tile, after the group of Q.
         auto issue_tile = [&](int j, bool tma_started) {
+            last = j;
             if (tile_kind(j)) {
-                if (lt == 0 && !tma_started) issue_tma(j);
+                if (lt == 0 && !tma_started && !*abort) issue_tma(j);
                 if (j == 0) {
                     asm volatile("cp.async.wait_group 0;" ::: "memory");   // only Q is pending
                     fence_proxy_async_smem();
@@ -375,6 +380,16 @@ __global__ void __launch_bounds__(kThreads, 1) attn_dec_tc_kernel(const __grid_c
             }
         }
         cp_async_wait_all();
+        // TMA tiles still landing (an abort) land before the CTA's shared
+        // memory is given up.  The last kStages tiles handed out are the
+        // latest phase of each stage's barrier (so its parity is unambiguous);
+        // a TMA tile's loaders arrived when it was handed out, so its phase
+        // completes once its bytes land (at once if it was not started).
+        if (lt == 0) {
+            volatile int never = 0;
+            for (int j = max(0, last - (kStages - 1)); j <= last; ++j)
+                if (tile_kind(j)) mbar_wait(&ctl->full[j % kStages], (j / kStages) & 1, &never, err);
+        }
     } else if (warp < kMmaWarp) {
         // ------------------------------------------------------------ softmax
         const int sw = warp - kLoadWarps;
@@ -503,6 +518,8 @@ __global__ void __launch_bounds__(kThreads, 1) attn_dec_tc_kernel(const __grid_c
             const uint32_t id_pv = idesc_bf16(kH, kD, true, true);
             const uint64_t qdesc = sw128_desc(smem_u32(sQ), 16, 1024);
             bool ok = true;
+            // test hook: a wait that runs out (nothing completes stall_bar)
+            if (stall) ok = mbar_wait(&ctl->stall_bar, 0, abort, err, wait_ns);
             auto pv = [&](int jj) -> bool {
                 if (!mbar_wait(&ctl->p_ready[jj & 1], (jj >> 1) & 1, abort, err, wait_ns)) return false;
                 tc_fence_after();
@@ -760,8 +777,10 @@ cudaError_t launch_attention_dec_tc(const AttnArgs& a, uint32_t* err, cudaStream
     attr[1].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 2;
-    e = lse ? cudaLaunchKernelEx(&cfg, attn_dec_tc_kernel<true>, tm_c, tm_w, a, max_chunk, err, wait_limit_ns())
-            : cudaLaunchKernelEx(&cfg, attn_dec_tc_kernel<false>, tm_c, tm_w, a, max_chunk, err, wait_limit_ns());
+    const uint64_t wait_ns = wait_limit_ns();
+    const int stall = take_stall();
+    e = lse ? cudaLaunchKernelEx(&cfg, attn_dec_tc_kernel<true>, tm_c, tm_w, a, max_chunk, err, wait_ns, stall)
+            : cudaLaunchKernelEx(&cfg, attn_dec_tc_kernel<false>, tm_c, tm_w, a, max_chunk, err, wait_ns, stall);
     count_launch();
     return e != cudaSuccess ? e : cudaGetLastError();
 }

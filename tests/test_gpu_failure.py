@@ -67,3 +67,23 @@ def test_indexer_wait_timeout_is_reported_and_the_next_call_runs_clean():
     qI = torch.randn(1, n, 4, 64, generator=g).to(torch.bfloat16).to(DEV)
     kI = torch.randn(1, n // 4, 64, generator=g).to(torch.bfloat16).to(DEV)
     _expect_timeout_then_clean(lambda: api.indexer_topk(qI, kI, 4, 64))
+
+
+def test_decode_attention_wait_timeout_is_reported_and_the_next_call_runs_clean():
+    # decode rows (positions given): the tcgen05 decode kernel with its TMA
+    # window tiles and gathered entry tiles in flight when the wait runs out
+    g = torch.Generator().manual_seed(13)
+    B, N_cap, k, W = 4, 4000, 512, 256
+    q = torch.randn(B, 1, 64, 128, generator=g).to(torch.bfloat16).to(DEV)
+    kv_c = torch.randn(B, N_cap, 128, generator=g).to(torch.bfloat16).to(DEV)
+    swa = torch.randn(B, W, 128, generator=g).to(torch.bfloat16).to(DEV)
+    ctx = torch.tensor([16000, 9000, 12345, 700], dtype=torch.int32)
+    idx = torch.full((B, k), -1, dtype=torch.int32)
+    for b in range(B):
+        sel = torch.randperm(min(int(ctx[b]) // 4, N_cap), generator=g)[:k]
+        idx[b, :sel.numel()] = sel.to(torch.int32)
+    kw = dict(raw_pos0=(ctx - W).to(DEV), raw_len=torch.full((B,), W, dtype=torch.int32).to(DEV),
+              q_pos=(ctx - 1).reshape(B, 1).to(DEV))
+    idx = idx.reshape(B, 1, k).to(DEV)
+    _expect_timeout_then_clean(lambda: api.sparse_attn(q, kv_c, idx, swa, W, **kw))
+
