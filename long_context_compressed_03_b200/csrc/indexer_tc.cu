@@ -303,9 +303,11 @@ struct RowCtx {
     uint64_t c2[kHeads];       // (c_h, c_h): half the head's query scale (times its gate weight)
 };
 
-// Shared-memory atomics on 32-bit shared addresses.
-__device__ __forceinline__ void red_add_shared(uint32_t addr) {
-    asm volatile("red.shared.add.u32 [%0], 1;" ::"r"(addr) : "memory");
+// Shared-memory atomics on 32-bit shared addresses.  The counting passes
+// take the predicated form: one instruction per score, no branch.
+__device__ __forceinline__ void red_add_shared_if(uint32_t addr, bool pred) {
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.u32 p, %1, 0;\n\t@p red.shared.add.u32 [%0], 1;\n\t}"
+                 ::"r"(addr), "r"((uint32_t)pred) : "memory");
 }
 __device__ __forceinline__ int atom_add_shared(uint32_t addr, int v) {
     int old;
@@ -342,11 +344,11 @@ __device__ __forceinline__ void take(float sc, int s, const RowCtx& rc, uint32_t
         mx = max(mx, u);
     } else if constexpr (MODE == kWindow) {
         const int jj = max(rc.T1 - (int)(u >> kWinShift), 0);
-        if (jj <= kWinBins) red_add_shared(rc.hrow + (uint32_t)jj * (kRows * 4));
+        red_add_shared_if(rc.hrow + (uint32_t)jj * (kRows * 4), jj <= kWinBins);
     } else if constexpr (MODE == kDigit) {
         const uint64_t key = ((uint64_t)u << 16) | (uint64_t)(65535 - s);
-        if ((key >> rc.sh) == rc.prefix)
-            red_add_shared(rc.hrow + (uint32_t)((key >> (rc.sh - rc.w)) & rc.wmask) * (kRows * 4));
+        red_add_shared_if(rc.hrow + (uint32_t)((key >> (rc.sh - rc.w)) & rc.wmask) * (kRows * 4),
+                          (key >> rc.sh) == rc.prefix);
     } else if constexpr (MODE == kEmit32) {
         // mx collects the slice's certain keys (bit s mod kSlice)
         const uint32_t kp = u >> rc.sh32;
@@ -385,10 +387,42 @@ __device__ __forceinline__ void part_work(const float (&a)[kHeads][kPart], const
             if (FP8) k4 = *reinterpret_cast<const float4*>(ksb + e);
             const uint64_t v0 = fold2<FP8>(a, e, rc.c2, k4.x, k4.y);
             const uint64_t v1 = fold2<FP8>(a, e + 2, rc.c2, k4.z, k4.w);
-            take<MODE, GATED>(f2_lo(v0), s0 + e, rc, mx);
-            take<MODE, GATED>(f2_hi(v0), s0 + e + 1, rc, mx);
-            take<MODE, GATED>(f2_lo(v1), s0 + e + 2, rc, mx);
-            take<MODE, GATED>(f2_hi(v1), s0 + e + 3, rc, mx);
+            if constexpr (MODE == kEmit32 || MODE == kEmit64) {
+                // the four keys' certain bits into mx, the rare boundary keys
+                // after them: one branch per four scores
+                const float sc[4] = {f2_lo(v0), f2_hi(v0), f2_lo(v1), f2_hi(v1)};
+                uint32_t eq = 0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t u = GATED ? score_key(sc[i]) : __float_as_uint(sc[i]);
+                    const int si = s0 + e + i;
+                    bool gt, same;
+                    if constexpr (MODE == kEmit32) {
+                        const uint32_t kp = u >> rc.sh32;
+                        gt = kp > rc.p32;
+                        same = kp == rc.p32;
+                    } else {
+                        const uint64_t kp = (((uint64_t)u << 16) | (uint64_t)(65535 - si)) >> rc.sh;
+                        gt = kp > rc.prefix;
+                        same = kp == rc.prefix;
+                    }
+                    mx |= (gt ? 1u : 0u) << (si & (kSlice - 1));
+                    eq |= (same ? 1u : 0u) << i;
+                }
+                if (eq) {
+#pragma unroll
+                    for (int i = 0; i < 4; ++i)
+                        if ((eq >> i) & 1u) {
+                            const uint32_t u = GATED ? score_key(sc[i]) : __float_as_uint(sc[i]);
+                            list_one(((uint64_t)u << 16) | (uint64_t)(65535 - (s0 + e + i)), rc);
+                        }
+                }
+            } else {
+                take<MODE, GATED>(f2_lo(v0), s0 + e, rc, mx);
+                take<MODE, GATED>(f2_hi(v0), s0 + e + 1, rc, mx);
+                take<MODE, GATED>(f2_lo(v1), s0 + e + 2, rc, mx);
+                take<MODE, GATED>(f2_hi(v1), s0 + e + 3, rc, mx);
+            }
         }
     } else {
 #pragma unroll
