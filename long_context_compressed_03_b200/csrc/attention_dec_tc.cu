@@ -31,16 +31,17 @@
 //   * each softmax thread adds its key's weights into per-head registers (the
 //     bf16-rounded ones the product used, l_r, and the exact ones, l_e, for
 //     the log-sum-exp); one transposing warp reduction at the end sums them;
-//   * publishes (offset m, l_r, l_e, unnormalised O) in its shared memory;
-//     after a cluster barrier CTA c merges its range of heads from all shares
-//     and writes o and the log-sum-exp.
+//   * pushes (offset m, l_r, l_e, unnormalised O) of every head over DSMEM
+//     to the CTA of the cluster that finalises it; after a cluster barrier
+//     CTA c merges its range of heads from its inbox and writes o and the
+//     log-sum-exp.
 // The offset m of a head is a whole number: set from the head's first keys
 // and raised by whole steps only when a weight would exceed 2^15, so every
 // rescale (of O in TMEM and of the sums) is an exact power of two.  O is
 // normalised by l_r, the sum of the bf16-rounded weights the products used.
-// Roles (13 warps): warps 0-3 load; warps 4-11 run the softmax (warp w reads
-// TMEM lanes 32 (w % 4) .. +31, i.e. keys, and heads 32 ((w - 4) / 4) .. +31);
-// warp 12 allocates TMEM and one lane issues every MMA.
+// Roles (21 warps): warps 0-3 load; warps 4-19 run the softmax (warp w reads
+// TMEM lanes 32 (w % 4) .. +31, i.e. keys, and heads 16 ((w - 4) / 4) .. +15);
+// warp 20 allocates TMEM and one lane issues every MMA.
 #include <cooperative_groups.h>
 #include <cudaTypedefs.h>
 #include <limits.h>
