@@ -210,3 +210,35 @@ def test_decode_attention_is_deterministic():
     a = api.hca_attn(T(q), T(kv_c), 4, T(swa), W, **kw)
     b = api.hca_attn(T(q), T(kv_c), 4, T(swa), W, **kw)
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("B", [3, 160])
+def test_decode_csa_rows_of_mixed_shape_both_decode_kernels(B):
+    # 64 heads x 128: up to one row per SM takes the tcgen05 decode kernel
+    # (transposed score tiles, TMA window tiles, clusters sized by occupancy);
+    # more rows than SMs take the mma.sync cluster kernel.  Rows mix a full
+    # selection, a short context (index padding, a window shorter than W and
+    # a compressed part that does not fill a tile) and the first token.
+    H, D, N_cap, W, k = 64, 128, 3000, 256, 320
+    q, kv_c, swa = _decode_attn_inputs(90 + B, B, H, D, N_cap, W)
+    rng = np.random.default_rng(B)
+    ctx = rng.integers(W + 1, 4 * N_cap, size=B).astype(np.int64)
+    ctx[1] = 150                                      # 37 entries, window of 150
+    ctx[2] = 1                                        # nothing compressed, one raw row
+    q_pos = (ctx - 1).reshape(B, 1).astype(np.int32)
+    raw_pos0 = (ctx - W).astype(np.int32)
+    raw_len = np.minimum(ctx, W).astype(np.int32)
+    ne = np.minimum(ctx // 4, N_cap)
+    idx = np.full((B, 1, k), -1, np.int32)
+    for b in range(B):
+        v = int(ne[b])
+        if v:
+            idx[b, 0, :min(k, v)] = rng.choice(v, size=min(k, v), replace=False)
+    out, lse = api.sparse_attn(T(q), T(kv_c), T(idx), T(swa), W, with_lse=True,
+                               raw_pos0=T(raw_pos0), raw_len=T(raw_len), q_pos=T(q_pos))
+    rows = np.unique(np.concatenate([[0, 1, 2], rng.choice(B, size=min(B, 12), replace=False)]))
+    ro, rl = oracle.sparse_attn(np64(q)[rows], np64(kv_c)[rows], idx[rows], np64(swa)[rows], W,
+                                q_pos=q_pos[rows], raw_pos0=raw_pos0[rows], raw_len=raw_len[rows])
+    check_out(np64(out)[rows].reshape(ro.shape), ro, torch.bfloat16,
+              label=f"decode attention, {B} rows of mixed shape")
+    np.testing.assert_allclose(lse.cpu().numpy()[rows].reshape(rl.shape), rl, atol=1e-3)
