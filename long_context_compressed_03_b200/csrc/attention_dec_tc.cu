@@ -48,6 +48,7 @@
 #include <math.h>
 
 #include <algorithm>
+#include <mutex>
 
 #include "attn_rows.cuh"
 #include "common.cuh"
@@ -688,7 +689,8 @@ cudaError_t prepare(int C, size_t smem) {
 }
 
 // Clusters of C CTAs (one CTA per SM) that can be resident at once; 0 when
-// the query fails.  Cached per (device, C, shared-memory size).
+// the query fails.  Cached per (device, C, shared-memory size), under a lock
+// (host threads may launch concurrently).
 int active_clusters(int C, size_t smem) {
     struct Entry {
         int dev, C;
@@ -697,8 +699,10 @@ int active_clusters(int C, size_t smem) {
     };
     static Entry cache[64];
     static int used = 0;
+    static std::mutex mu;
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    std::lock_guard<std::mutex> lock(mu);
     for (int i = 0; i < used; ++i)
         if (cache[i].dev == dev && cache[i].C == C && cache[i].smem == smem) return cache[i].n;
     int n = 0;
